@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE FFN layer on B200.
+
+Default workload (decode_t1): one V4-Flash MoE layer (hidden 4096, 256
+routed IQ2_XXS/Q2_K experts of intermediate 2048, top-6, one Q8_0 shared
+expert) on one token per call, 1000 timed calls rotating over 8 layer
+weight sets (8 x 1.84 GB, far beyond the 126 MB L2) after warm-up calls.
+A step is one layer call.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_t1|decode_t32|prefill_t4096]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on
+its own GPU with no exchange (replicas; the layer has no data-path
+collective), timed between barriers, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and % HBM roofline (decode) / % bf16 TC roofline (prefill)"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="decode_t1", choices=["decode_t1", "decode_t32", "prefill_t4096"])
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(world, value: float) -> float:
+    import torch
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- workloads
+
+def decode_bytes(s: synth.LayerShape, n_distinct: float) -> dict:
+    """Algorithmic bytes: packed weights each selected expert / the shared
+    expert contributes once per call, plus the router."""
+    gate_up_routed = 2 * s.gate_bytes_per_expert
+    shared_gate_up = 2 * s.shared_inter * s.row_bytes(synth.KIND_Q80, s.hidden)
+    router = s.n_experts * s.hidden * 2
+    return {"layer": n_distinct * s.expert_bytes + s.shared_bytes + router,
+            "experts": n_distinct * s.expert_bytes + s.shared_bytes,
+            "k2_gateup": n_distinct * gate_up_routed + shared_gate_up}
+
+
+def run_ours(args, world, rank):
+    import torch
+
+    import bit_moe_expert_sqrtsoftplus_b200 as moe
+
+    s = synth.workload(args.workload)
+    T = s.tokens
+    nsets = s.weight_sets
+    layers, weights = [], []
+    scratch = None
+    for i in range(nsets):
+        W = synth.device_layer(0, i, s)
+        cfg = moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
+                              routed_scaling=s.routed_scaling)
+        L = moe.Layer(cfg, W, max_tokens=T, scratch=scratch)
+        scratch = L.scratch
+        layers.append(L)
+        weights.append(W)
+    npool = 16
+    xs = [torch.from_numpy(synth.activations(7 + rank, T, s.hidden, stream=j)).cuda() for j in range(npool)]
+    ys = [torch.empty_like(xs[0]) for _ in range(npool)]
+    torch.cuda.synchronize()
+
+    def step(i):
+        layers[i % nsets].forward(xs[i % npool], None, ys[i % npool])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    layers[0].poll()
+
+    # distinct experts per call (for the byte count): from the routing of the pool
+    nd = []
+    for j in range(min(npool, 8)):
+        idx, _ = layers[j % nsets].route(xs[j])
+        nd.append(len(np.unique(idx.cpu().numpy())))
+    n_distinct = float(np.mean(nd))
+
+    stream = torch.cuda.current_stream()
+    clock = ClockSampler(torch.cuda.current_device())
+    with clock:
+        # pass 1: the timed region
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        e1.record(stream)
+        barrier(world)
+        ms = e0.elapsed_time(e1)
+        # pass 2: the dominant kernel, timed live around each launch
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            L = layers[(args.warmup + i) % nsets]
+            moe.moe_set_timing_events(L.handle, *evs[i])
+            step(args.warmup + i)
+        torch.cuda.synchronize()
+        for L in layers:
+            moe.moe_set_timing_events(L.handle)
+        k2_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        # pass 3: end to end with host buffers (pinned), copies inside the timed region
+        hx = [xs[j].cpu().pin_memory() for j in range(npool)]
+        hy = [torch.empty_like(hx[0]).pin_memory() for _ in range(npool)]
+        dx = torch.empty_like(xs[0])
+        dy = torch.empty_like(xs[0])
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.steps):
+            j = i % npool
+            dx.copy_(hx[j], non_blocking=True)
+            layers[i % nsets].forward(dx, None, dy)
+            hy[j].copy_(dy, non_blocking=True)
+        f1.record(stream)
+        barrier(world)
+        e2e_ms = f0.elapsed_time(f1)
+    for L in layers:
+        L.poll()
+
+    ms = max_over_ranks(world, ms)
+    e2e_ms = max_over_ranks(world, e2e_ms)
+    k2_ms = max_over_ranks(world, k2_ms)
+    ms_step = ms / args.steps
+    value = world * args.steps * T / (ms / 1e3)
+    e2e_value = world * args.steps * T / (e2e_ms / 1e3)
+    peaks = load_peaks()
+    b = decode_bytes(s, n_distinct)
+    achieved = b["k2_gateup"] / (k2_ms / 1e3) / 1e9
+    layer_gbs = b["experts"] / (ms_step / 1e3) / 1e9
+    clocks = clock.summary()
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "us_per_layer": ms_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 tensor-core products, fp32 scaling",
+        "data": "synthetic (seeded generator; V4-Flash shapes, random weights)",
+        "config": {"workload": f"{args.workload}: V4-Flash MoE layer, T={T} tokens/call, hidden {s.hidden}, "
+                               f"{s.n_experts} experts top-{s.top_k}, inter {s.inter}, shared {s.shared_inter}",
+                   "tokens_per_call": T, "weight_sets_rotated": nsets,
+                   "l2": f"{nsets} rotating weight sets of {s.n_experts * s.expert_bytes / 1e9:.2f} GB "
+                         "(inputs far larger than the 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "k2_gateup (routed IQ2_XXS gate/up + shared Q8_0 gate/up)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_launch": b["k2_gateup"], "ms_per_launch": k2_ms},
+        "layer_hbm": {"bytes_per_call": b["experts"], "router_bytes": s.n_experts * s.hidden * 2,
+                      "achieved_gbs": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"],
+                      "distinct_experts_per_call": n_distinct},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 4,
+                "d2h_bytes_per_step": T * s.hidden * 4},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    return out
+
+
+def oracle_rate(s: synth.LayerShape, budget_s: float, max_steps: int, seed: int = 0):
+    """Tokens/s of the fp64 oracle on full layer calls of the workload
+    (weight set 0, inputs resident), as many calls as fit in the budget."""
+    import oracle
+    W = synth.host_layer(seed, 0, s)
+    Wr, b = W["router_w"], W["bias"]
+    T = s.tokens
+    n = 0
+    t0 = time.perf_counter()
+    elapsed = 0.0
+    while n < max_steps and (n == 0 or elapsed < budget_s):
+        x = synth.activations(7, T, s.hidden, stream=100 + n).astype(np.float64)
+        a = time.perf_counter()
+        idx, w, _ = oracle.route(x, Wr, b, s.top_k, s.routed_scaling)
+        oracle.layer(W, s, x, idx, w)
+        elapsed += time.perf_counter() - a
+        n += 1
+    del t0
+    return n * T / elapsed, n, elapsed
+
+
+def run_reference(args, world, rank):
+    s = synth.workload(args.workload)
+    if rank != 0:
+        return None
+    budget = 90.0
+    value, n, elapsed = oracle_rate(s, budget, max(1, args.steps))
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": n,
+            "steps_requested": args.steps, "warmup": 0, "ms_per_step": 1e3 * elapsed / n, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{args.workload} (same shapes), one weight set resident on the host",
+                       "tokens_per_call": s.tokens},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} full layer calls (T={s.tokens}) of the fp64 C oracle, single thread, "
+                                       f"{elapsed:.1f} s; calls capped by a {budget:.0f} s budget"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    out = run_ours(args, world, rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = synth.workload(args.workload)
+        value, n, elapsed = oracle_rate(s, args.cpu_seconds, 1000)
+        out["cpu_baseline"] = {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{n} full layer calls (T={s.tokens}) of the fp64 C oracle on weight set 0, "
+                                         f"single thread, {elapsed:.1f} s"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,308 @@
+// api.cu -- the extern "C" boundary declared in include/moe.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <string>
+
+#include "../../include/moe.h"
+#include "layer.cuh"
+#include "prefill.cuh"
+
+struct moe_handle {
+  moe_config cfg;
+  moe_weights w;
+  moe::LayerDims d;
+  moe::LayerWeights wt;
+  int *err;          // device error word inside persist
+  float *row_norms;  // [E] 2-norms of the router rows (fp32), inside persist
+  int num_sms;
+  int device;
+  cudaEvent_t ev_begin, ev_end;  // optional timing of the dominant kernel
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+moe_status fail(moe_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kPersistHeader = 256;
+
+size_t persist_bytes_for(const moe_config &c) {
+  return kPersistHeader + sizeof(float) * (size_t)(c.n_experts > 0 ? c.n_experts : 0) + 256;
+}
+
+moe_status check_config(const moe_config *c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+  if (c->hidden <= 0 || c->hidden % 256)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "hidden=%d must be a positive multiple of 256", c->hidden);
+  if (c->inter <= 0 || c->inter % 256)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "inter=%d must be a positive multiple of 256", c->inter);
+  if (c->shared_inter <= 0 || c->shared_inter % 256)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "shared_inter=%d must be a positive multiple of 256", c->shared_inter);
+  if (c->top_k < 1 || c->top_k > moe::kMaxK)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "top_k=%d must be in 1..%d", c->top_k, moe::kMaxK);
+  if (c->n_experts < c->top_k || c->n_experts > moe::kMaxE)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_experts=%d must be in top_k..%d", c->n_experts, moe::kMaxE);
+  if (c->mode != MOE_ROUTE_ROUTER && c->mode != MOE_ROUTE_HASH)
+    return fail(MOE_ERR_INVALID_ARG, "mode=%d is not a moe_route_mode", c->mode);
+  if (c->mode == MOE_ROUTE_HASH && c->vocab <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "hash mode needs vocab > 0 (got %d)", c->vocab);
+  if (!isfinite(c->routed_scaling)) return fail(MOE_ERR_INVALID_ARG, "routed_scaling is not finite");
+  if ((c->flags & MOE_FLAG_PRENORM_RESIDUAL) && !(c->rms_eps >= 0.f && isfinite(c->rms_eps)))
+    return fail(MOE_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
+  if (c->flags & ~MOE_FLAG_PRENORM_RESIDUAL) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
+  return MOE_OK;
+}
+
+moe::LayerDims dims_of(const moe_config &c) {
+  moe::LayerDims d;
+  d.H = c.hidden;
+  d.I = c.inter;
+  d.Is = c.shared_inter;
+  d.E = c.n_experts;
+  d.k = c.top_k;
+  d.mode = c.mode;
+  d.flags = c.flags;
+  d.vocab = c.vocab;
+  d.scaling = c.routed_scaling;
+  d.eps = c.rms_eps;
+  return d;
+}
+
+size_t scratch_bytes_for(const moe::LayerDims &d, int max_tokens) {
+  size_t dec = moe::decode_scratch_bytes(d, max_tokens < moe::kDecodeMaxT ? max_tokens : moe::kDecodeMaxT);
+  size_t pre = max_tokens > moe::kDecodeMaxT ? moe::prefill_scratch_bytes(d, max_tokens) : 0;
+  return dec > pre ? dec : pre;
+}
+
+moe_status check_call(moe_handle *h, const float *x, const int32_t *token_ids, int T, void *scratch,
+                      size_t scratch_bytes) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  if (T == 0) return MOE_OK;
+  if (!x) return fail(MOE_ERR_INVALID_ARG, "x is NULL");
+  if (!aligned16(x)) return fail(MOE_ERR_MISALIGNED, "x is not 16-byte aligned");
+  if (h->d.mode == MOE_ROUTE_HASH && !token_ids) return fail(MOE_ERR_INVALID_ARG, "hash mode needs token_ids");
+  if (!scratch) return fail(MOE_ERR_INVALID_ARG, "scratch is NULL");
+  if (!aligned16(scratch)) return fail(MOE_ERR_MISALIGNED, "scratch is not 16-byte aligned");
+  const size_t need = scratch_bytes_for(h->d, T);
+  if (scratch_bytes < need)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for T=%d", scratch_bytes, need, T);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_last_error.c_str(); }
+
+moe_status moe_workspace_size(const moe_config *cfg, int max_tokens, size_t *persist_bytes, size_t *scratch_bytes) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "max_tokens=%d is negative", max_tokens);
+  if (persist_bytes) *persist_bytes = persist_bytes_for(*cfg);
+  if (scratch_bytes) *scratch_bytes = max_tokens > 0 ? scratch_bytes_for(dims_of(*cfg), max_tokens) : 0;
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, size_t persist_bytes,
+                    moe_stream_t stream, moe_handle **out) {
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
+  const void *need[] = {w->gate_iq2xxs, w->up_iq2xxs, w->down_q2k, w->sh_gate_q80, w->sh_up_q80, w->sh_down_q80,
+                        w->iq2_grid};
+  const char *names[] = {"gate_iq2xxs", "up_iq2xxs", "down_q2k", "sh_gate_q80", "sh_up_q80", "sh_down_q80",
+                         "iq2_grid"};
+  for (int i = 0; i < 7; ++i) {
+    if (!need[i]) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(need[i])) return fail(MOE_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+  }
+  if (cfg->mode == MOE_ROUTE_ROUTER) {
+    if (!w->router_w_f16 || !w->router_bias) return fail(MOE_ERR_INVALID_ARG, "router mode needs router_w_f16 and router_bias");
+    if (!aligned16(w->router_w_f16) || !aligned16(w->router_bias))
+      return fail(MOE_ERR_MISALIGNED, "router weights are not 16-byte aligned");
+  } else {
+    if (!w->tid2eid) return fail(MOE_ERR_INVALID_ARG, "hash mode needs tid2eid");
+    if (!aligned16(w->tid2eid)) return fail(MOE_ERR_MISALIGNED, "tid2eid is not 16-byte aligned");
+  }
+  if (!persist) return fail(MOE_ERR_INVALID_ARG, "persist is NULL");
+  if (!aligned16(persist)) return fail(MOE_ERR_MISALIGNED, "persist is not 16-byte aligned");
+  if (persist_bytes < persist_bytes_for(*cfg))
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "persist has %zu bytes, %zu needed", persist_bytes,
+                persist_bytes_for(*cfg));
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+
+  moe_handle *h = new (std::nothrow) moe_handle;
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "out of host memory");
+  h->cfg = *cfg;
+  h->w = *w;
+  h->d = dims_of(*cfg);
+  h->wt.Wr = static_cast<const uint16_t *>(w->router_w_f16);
+  h->wt.bias = w->router_bias;
+  h->wt.tid2eid = w->tid2eid;
+  h->wt.gate = static_cast<const uint8_t *>(w->gate_iq2xxs);
+  h->wt.up = static_cast<const uint8_t *>(w->up_iq2xxs);
+  h->wt.down = static_cast<const uint8_t *>(w->down_q2k);
+  h->wt.sh_gate = static_cast<const uint8_t *>(w->sh_gate_q80);
+  h->wt.sh_up = static_cast<const uint8_t *>(w->sh_up_q80);
+  h->wt.sh_down = static_cast<const uint8_t *>(w->sh_down_q80);
+  h->wt.grid = w->iq2_grid;
+  h->err = static_cast<int *>(persist);
+  h->row_norms = reinterpret_cast<float *>(static_cast<uint8_t *>(persist) + kPersistHeader);
+  h->num_sms = sms;
+  h->device = dev;
+  h->ev_begin = nullptr;
+  h->ev_end = nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = cudaMemsetAsync(persist, 0, kPersistHeader, s);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e, "cudaMemsetAsync(persist)");
+  }
+  e = moe::prefill_init(h->d, h->wt, h->row_norms, h->err, s);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e, "init kernels");
+  }
+  *out = h;
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+static moe::DecodeArgs decode_args(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
+                                   void *scratch) {
+  moe::DecodeArgs a;
+  a.d = h->d;
+  a.wt = h->wt;
+  a.T = T;
+  a.x = x;
+  a.token_ids = token_ids;
+  a.y = y;
+  moe::decode_carve(a.s, h->d, T, scratch);
+  a.err = h->err;
+  a.ev_begin = h->ev_begin;
+  a.ev_end = h->ev_end;
+  return a;
+}
+
+moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, int T, int32_t *idx, float *w,
+                     int32_t *expert_offsets, int32_t *perm, void *scratch, size_t scratch_bytes,
+                     moe_stream_t stream) {
+  moe_status st = check_call(h, x, token_ids, T, scratch, scratch_bytes);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!idx || !w) return fail(MOE_ERR_INVALID_ARG, "idx and w must not be NULL");
+  if ((expert_offsets == nullptr) != (perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "expert_offsets and perm must both be set or both be NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (T <= moe::kDecodeMaxT) {
+    moe::DecodeArgs a = decode_args(h, x, token_ids, T, nullptr, scratch);
+    e = moe::decode_route(a, idx, w, s);
+  } else {
+    moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, nullptr, scratch, h->row_norms, h->err);
+    e = moe::prefill_route(p, idx, w, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "moe_route launch");
+  if (perm) {
+    e = moe::permute(idx, T, h->d.k, h->d.E, expert_offsets, perm, s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_route permutation");
+  }
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y, void *scratch,
+                           size_t scratch_bytes, moe_stream_t stream) {
+  moe_status st = check_call(h, x, token_ids, T, scratch, scratch_bytes);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y) return fail(MOE_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y)) return fail(MOE_ERR_MISALIGNED, "y is not 16-byte aligned");
+  if (y == x && !(h->d.flags & MOE_FLAG_PRENORM_RESIDUAL))
+    return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (T <= moe::kDecodeMaxT) {
+    moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
+    e = moe::decode_forward(a, s, h->num_sms);
+  } else {
+    moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, y, scratch, h->row_norms, h->err);
+    e = moe::prefill_forward(p, s, h->num_sms);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward launch");
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_poll_device_error(moe_handle *h, moe_stream_t stream) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int code = 0;
+  e = cudaMemcpy(&code, h->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (code != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(h->err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    switch (code) {
+      case MOE_ERR_TIMEOUT:
+        return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out");
+      case MOE_ERR_UNSUPPORTED_SHAPE:
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "an IQ2_XXS codebook entry exceeds 127");
+      case MOE_ERR_INVALID_ARG:
+        return fail(MOE_ERR_INVALID_ARG, "a token id was outside [0, vocab)");
+      default:
+        return fail(MOE_ERR_DEVICE_FAULT, "device error code %d", code);
+    }
+  }
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if ((ev_begin == nullptr) != (ev_end == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "ev_begin and ev_end must both be set or both be NULL");
+  h->ev_begin = static_cast<cudaEvent_t>(ev_begin);
+  h->ev_end = static_cast<cudaEvent_t>(ev_end);
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+void moe_destroy(moe_handle *h) { delete h; }
+
+}  // extern "C"

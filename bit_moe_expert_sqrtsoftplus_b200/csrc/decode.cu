@@ -1,0 +1,1172 @@
+// decode.cu -- the layer for small token counts (T <= 8): three kernels.
+//
+//   k1_prep_router  x -> int8 limbs (optionally RMSNorm first) and fp64
+//                   router logits z = W_r x.
+//   k2_gateup       top-k routing (recomputed per CTA from z), then every
+//                   (expert, 16-row tile) of gate/up and every (16-row tile,
+//                   K quarter) of the shared expert as a warp-sized unit:
+//                   packed rows are staged into shared memory with cp.async,
+//                   decoded in registers into int8 A fragments and multiplied
+//                   with mma.sync m16n8k32 against the int8 limbs of x; the
+//                   SwiGLU is applied in the epilogue.  The warp that
+//                   finishes the last tile of a vector quantises it into
+//                   limbs for the down projection.
+//   k3_down         every (16-row output tile, expert or shared K quarter)
+//                   unit: Q2_K / Q8_0 rows against the limbs of h, weighted
+//                   by the routing weight; the last unit of a tile sums the
+//                   parts in a fixed order (deterministic) into y.
+//
+// Activations enter the tensor cores as three int8 limbs with one scale per
+// vector: x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254, s3 = s2/254, which keeps
+// x to 6e-8 of max|x|; the weight side is exact in int8 (IQ2_XXS grid values
+// with signs, Q2_K code*scale <= 45, Q8_0 values), so the products are exact
+// integers and only the fp32 block scaling rounds.
+#include <float.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "layer.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads2 = 256;  // 8 warps in k2 / k3
+constexpr int kWarps2 = kThreads2 / kWarp;
+constexpr int kStageBytes = 16 * 544;  // one 16-row chunk of at most 544 bytes per row
+constexpr int kGpmBytes = 256 * 128;   // +/- codebook, 8 replicas
+constexpr int kSelBytes = 128 * 128;   // byte-permute selectors per sign mask, 16 replicas
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ k1
+
+template <int MAXT>
+__global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
+  const LayerDims &d = a.d;
+  const int T = a.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ double red[4][2 * MAXT + MAXT];
+  __shared__ float redf[4];
+
+  if (blockIdx.x == 0) {
+    const int V = T * d.k + T;
+    for (int i = tid; i < V; i += blockDim.x) {
+      a.s.hmax[i] = 0u;
+      a.s.Xmax[i] = 0u;
+      a.s.vcount[i] = 0;
+    }
+    for (int i = tid; i < d.Is / 16; i += blockDim.x) a.s.shcount[i] = 0;
+    for (int i = tid; i < d.H / 16; i += blockDim.x) a.s.ycount[i] = 0;
+    if (tid < 4) a.s.work[tid] = 0;
+  }
+
+  if ((int)blockIdx.x < T) {
+    // ---- activation limbs for token t
+    const int t = blockIdx.x;
+    const float *xt = a.x + (size_t)t * d.H;
+    double ss = 0.0;
+    float amax = 0.f;
+    for (int j = tid; j < d.H; j += blockDim.x) {
+      float v = xt[j];
+      ss += (double)v * (double)v;
+      amax = fmaxf(amax, fabsf(v));
+    }
+    ss = warp_sum_d(ss);
+    amax = warp_max(amax);
+    if (lane == 0) {
+      red[warp][0] = ss;
+      redf[warp] = amax;
+    }
+    __syncthreads();
+    ss = red[0][0] + red[1][0] + red[2][0] + red[3][0];
+    amax = fmaxf(fmaxf(redf[0], redf[1]), fmaxf(redf[2], redf[3]));
+    float inv = 1.f;
+    if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) {
+      double invd = 1.0 / sqrt(ss / (double)d.H + (double)d.eps);
+      inv = (float)invd;
+      amax = amax * inv;  // max of the normalised vector (positive scaling)
+    }
+    const float s1 = amax > 0.f ? amax / 127.f : 1.f;
+    const float s2 = s1 / 254.f, s3 = s2 / 254.f;
+    const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
+    int8_t *q = a.s.xq + (size_t)t * 3 * d.H;
+    for (int j = tid; j < d.H; j += blockDim.x) {
+      float v = xt[j] * inv;
+      float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
+      float e1 = fmaf(-q1, s1, v);
+      float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+      float e2 = fmaf(-q2, s2, e1);
+      float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+      q[j] = (int8_t)q1;
+      q[d.H + j] = (int8_t)q2;
+      q[2 * d.H + j] = (int8_t)q3;
+    }
+    if (tid == 0) {
+      float *s = a.s.xs + 4 * t;
+      s[0] = s1;
+      s[1] = s2;
+      s[2] = s3;
+      s[3] = 0.f;
+    }
+    return;
+  }
+
+  if (d.mode != MOE_ROUTE_ROUTER) return;
+  // ---- router logits for experts e0, e0 + 1 in fp64
+  const int e0 = 2 * ((int)blockIdx.x - T);
+  if (e0 >= d.E) return;
+  const bool two = e0 + 1 < d.E;
+  double acc[2][MAXT];
+  double ssq[MAXT];
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t) acc[0][t] = acc[1][t] = ssq[t] = 0.0;
+  const int jq = d.H / 4;
+  const int jb = warp * jq, je = jb + jq;
+  const uint16_t *w0 = a.wt.Wr + (size_t)e0 * d.H;
+  const uint16_t *w1 = a.wt.Wr + (size_t)(two ? e0 + 1 : e0) * d.H;
+  for (int j = jb + lane * 8; j < je; j += 256) {
+    uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
+    uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
+    double wa[8], wb[8];
+    const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
+    const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      wa[i] = (double)half_bits_to_float(p0[i]);
+      wb[i] = (double)half_bits_to_float(p1[i]);
+    }
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t) {
+      if (t < T) {
+        const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H + j);
+        float4 u0 = xp[0], u1 = xp[1];
+        double xv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc[0][t] = fma(wa[i], xv[i], acc[0][t]);
+          acc[1][t] = fma(wb[i], xv[i], acc[1][t]);
+          ssq[t] = fma(xv[i], xv[i], ssq[t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t) {
+    if (t < T) {
+      double v0 = warp_sum_d(acc[0][t]);
+      double v1 = warp_sum_d(acc[1][t]);
+      double v2 = warp_sum_d(ssq[t]);
+      if (lane == 0) {
+        red[warp][t] = v0;
+        red[warp][MAXT + t] = v1;
+        red[warp][2 * MAXT + t] = v2;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < T) {
+    const int t = tid;
+    double z0 = red[0][t] + red[1][t] + red[2][t] + red[3][t];
+    double z1 = red[0][MAXT + t] + red[1][MAXT + t] + red[2][MAXT + t] + red[3][MAXT + t];
+    if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) {
+      double s = red[0][2 * MAXT + t] + red[1][2 * MAXT + t] + red[2][2 * MAXT + t] + red[3][2 * MAXT + t];
+      double inv = 1.0 / sqrt(s / (double)d.H + (double)d.eps);
+      z0 *= inv;
+      z1 *= inv;
+    }
+    a.s.z[(size_t)t * d.E + e0] = z0;
+    if (two) a.s.z[(size_t)t * d.E + e0 + 1] = z1;
+  }
+}
+
+// ------------------------------------------------------------------ routing
+
+// sqrt(softplus(z)) in fp64, softplus computed as max(z,0) + log1p(exp(-|z|)).
+__device__ __forceinline__ double sqrtsoftplus(double z) {
+  return sqrt(fmax(z, 0.0) + log1p(exp(-fabs(z))));
+}
+
+// One warp: top-k of token t by s + bias (ties to the lower id), ids in
+// ascending order, weights scaling * s / sum(s).
+__device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, float *w_out) {
+  const LayerDims &d = a.d;
+  const int lane = threadIdx.x & 31;
+  const int k = d.k;
+  int sel[kMaxK];
+  if (d.mode == MOE_ROUTE_HASH) {
+    int tid = a.token_ids[t];
+    if (tid < 0 || tid >= d.vocab) {
+      if (lane == 0) set_error(a.err, kErrTokenId);
+      tid = 0;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxK; ++i) sel[i] = i < k ? a.wt.tid2eid[(size_t)tid * k + i] : INT_MAX;
+  } else {
+    const double *zt = a.s.z + (size_t)t * d.E;
+    double key[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = e < d.E ? sqrtsoftplus(zt[e]) + (double)a.wt.bias[e] : -DBL_MAX;
+    }
+    unsigned taken = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      if (r < k) {
+        double bk = -INFINITY;
+        int be = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = lane + 32 * i;
+          if (e < d.E && !((taken >> i) & 1u) && key[i] > bk) {
+            bk = key[i];
+            be = e;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+          int oe = __shfl_xor_sync(0xffffffffu, be, o);
+          if (ok > bk || (ok == bk && oe < be)) {
+            bk = ok;
+            be = oe;
+          }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        sel[r] = be;
+      } else {
+        sel[r] = INT_MAX;
+      }
+    }
+  }
+  // ascending ids
+#pragma unroll
+  for (int i = 1; i < kMaxK; ++i) {
+#pragma unroll
+    for (int j = kMaxK - 1; j >= i; --j) {
+      if (sel[j - 1] > sel[j]) {
+        int tmp = sel[j - 1];
+        sel[j - 1] = sel[j];
+        sel[j] = tmp;
+      }
+    }
+  }
+  if (lane == 0) {
+    if (d.mode == MOE_ROUTE_HASH) {
+      for (int i = 0; i < k; ++i) {
+        idx_out[i] = sel[i];
+        w_out[i] = d.scaling / (float)k;
+      }
+    } else {
+      const double *zt = a.s.z + (size_t)t * d.E;
+      double sv[kMaxK];
+      double tot = 0.0;
+      for (int i = 0; i < k; ++i) {
+        sv[i] = sqrtsoftplus(zt[sel[i]]);
+        tot += sv[i];
+      }
+      for (int i = 0; i < k; ++i) {
+        idx_out[i] = sel[i];
+        w_out[i] = (float)((double)d.scaling * sv[i] / tot);
+      }
+    }
+  }
+}
+
+// Job table: the distinct selected experts in ascending order, each with its
+// (token, slot) pairs in ascending token order.
+struct Jobs {
+  int n;
+  int e[kDecodeMaxT * kMaxK];
+  int first[kDecodeMaxT * kMaxK];
+  int cnt[kDecodeMaxT * kMaxK];
+  int pair[kDecodeMaxT * kMaxK];  // sorted t*k + slot
+};
+
+__device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
+  const int np = T * k;
+  const int tid = threadIdx.x;
+  __shared__ int rank_e[kDecodeMaxT * kMaxK];
+  if (tid < np) {
+    const int ei = idx_s[tid], ti = tid / k;
+    int rank = 0;
+    for (int j = 0; j < np; ++j) {
+      const int ej = idx_s[j], tj = j / k;
+      rank += (ej < ei) || (ej == ei && tj < ti);
+    }
+    J.pair[rank] = tid;
+    rank_e[rank] = ei;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int n = 0;
+    for (int r = 0; r < np; ++r) {
+      if (r == 0 || rank_e[r] != rank_e[r - 1]) {
+        J.e[n] = rank_e[r];
+        J.first[n] = r;
+        J.cnt[n] = 0;
+        ++n;
+      }
+      J.cnt[n - 1]++;
+    }
+    J.n = n;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ staging
+
+// Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS).
+__device__ __forceinline__ void stage_chunk(uint8_t *st, int RS, const uint8_t *g, size_t gstride, int bpr,
+                                            bool a16) {
+  const int lane = threadIdx.x & 31;
+  if (a16) {
+    const int n16 = bpr >> 4;
+    const int total = 16 * n16;
+    for (int i = lane; i < total; i += 32) {
+      const int row = i / n16, o = i - row * n16;
+      cp_async16(st + row * RS + o * 16, g + row * gstride + o * 16);
+    }
+  } else {
+    const int n2 = bpr >> 1;
+    const int total = 16 * n2;
+    for (int i = lane; i < total; i += 32) {
+      const int row = i / n2, o = i - row * n2;
+      *reinterpret_cast<uint16_t *>(st + row * RS + 2 * o) =
+          *reinterpret_cast<const uint16_t *>(g + row * gstride + 2 * o);
+    }
+  }
+  cp_async_commit();
+}
+
+struct Chunk {
+  const uint8_t *g;  // row 0 of the tile at the chunk's first block
+  size_t gstride;    // global row stride (bytes)
+  int bpr;           // bytes per row in the chunk
+  int nb;            // blocks in the chunk
+  int k0;            // first element (K index) of the chunk
+  bool a16;
+};
+
+__device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
+
+// ------------------------------------------------------------------ decoders
+
+// IQ2_XXS group -> int8 A fragment halves for sub-vector c of one row.
+__device__ __forceinline__ void iq2_group(const uint8_t *grp, int c, const uint8_t *gpm_l, const uint8_t *sel_l,
+                                          uint32_t &lo, uint32_t &hi, int &f) {
+  const uint32_t ix = grp[c];
+  const uint32_t S = lds_u16(grp + 4) | (lds_u16(grp + 6) << 16);
+  const uint32_t m7 = (S >> (7 * c)) & 127u;
+  f = 2 * (int)(S >> 28) + 1;
+  const uint4 gv = *reinterpret_cast<const uint4 *>(gpm_l + ix * 128u);
+  const uint2 sv = *reinterpret_cast<const uint2 *>(sel_l + m7 * 128u);
+  lo = __byte_perm(gv.x, gv.y, sv.x);
+  hi = __byte_perm(gv.z, gv.w, sv.y);
+}
+
+template <int MAXP>
+__device__ __forceinline__ void iq2_chunk(const uint8_t *st, int RS, const Chunk &ch, const uint8_t *gpm_l,
+                                          const uint8_t *sel_l, const int8_t *const (&bcol)[MAXP], int npairs,
+                                          float (&F)[MAXP][4]) {
+  const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const uint8_t *row0 = st + r * RS;
+  const uint8_t *row1 = st + (r + 8) * RS;
+  for (int b = 0; b < ch.nb; ++b) {
+    const float d0 = half_bits_to_float(lds_u16(row0 + 66 * b)) * 0.125f;
+    const float d1 = half_bits_to_float(lds_u16(row1 + 66 * b)) * 0.125f;
+    int acc[MAXP][4];
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      uint32_t A[4];
+      int f0, f1;
+      iq2_group(row0 + 66 * b + 2 + 8 * g, c, gpm_l, sel_l, A[0], A[2], f0);
+      iq2_group(row1 + 66 * b + 2 + 8 * g, c, gpm_l, sel_l, A[1], A[3], f1);
+      const int kel = ch.k0 + 256 * b + 32 * g + 8 * c;
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < npairs) {
+          uint32_t b0 = 0, b1 = 0;
+          if (bcol[p]) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
+            b0 = v.x;
+            b1 = v.y;
+          }
+          const int zero[4] = {0, 0, 0, 0};
+          int cg[4];
+          mma_s8(cg, A, b0, b1, zero);
+          acc[p][0] += cg[0] * f0;
+          acc[p][1] += cg[1] * f0;
+          acc[p][2] += cg[2] * f1;
+          acc[p][3] += cg[3] * f1;
+        }
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) {
+      F[p][0] = fmaf(d0, (float)acc[p][0], F[p][0]);
+      F[p][1] = fmaf(d0, (float)acc[p][1], F[p][1]);
+      F[p][2] = fmaf(d1, (float)acc[p][2], F[p][2]);
+      F[p][3] = fmaf(d1, (float)acc[p][3], F[p][3]);
+    }
+  }
+}
+
+// Q8_0: 34-byte blocks, the 8 int8 values of sub-range c (bytes 2+8c..9+8c).
+__device__ __forceinline__ void q80_vals(const uint8_t *blk, int b, int c, uint32_t &lo, uint32_t &hi) {
+  const uint8_t *p = blk + 2 + 8 * c;
+  if (b & 1) {  // 34*b + 2 + 8c is a multiple of 4
+    lo = lds_u32(p);
+    hi = lds_u32(p + 4);
+  } else {  // two bytes past a multiple of 4
+    const uint32_t u0 = lds_u32(p - 2), u1 = lds_u32(p + 2), u2 = lds_u32(p + 6);
+    lo = __byte_perm(u0, u1, 0x5432);
+    hi = __byte_perm(u1, u2, 0x5432);
+  }
+}
+
+template <int MAXP>
+__device__ __forceinline__ void q80_chunk(const uint8_t *st, int RS, const Chunk &ch,
+                                          const int8_t *const (&bcol)[MAXP], int npairs, float (&F)[MAXP][4]) {
+  const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const uint8_t *row0 = st + r * RS;
+  const uint8_t *row1 = st + (r + 8) * RS;
+  for (int b = 0; b < ch.nb; ++b) {
+    const uint8_t *p0 = row0 + 34 * b;
+    const uint8_t *p1 = row1 + 34 * b;
+    const float d0 = half_bits_to_float(lds_u16(p0));
+    const float d1 = half_bits_to_float(lds_u16(p1));
+    uint32_t A[4];
+    q80_vals(p0, b, c, A[0], A[2]);
+    q80_vals(p1, b, c, A[1], A[3]);
+    const int kel = ch.k0 + 32 * b + 8 * c;
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) {
+      if (p < npairs) {
+        uint32_t b0 = 0, b1 = 0;
+        if (bcol[p]) {
+          const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
+          b0 = v.x;
+          b1 = v.y;
+        }
+        const int zero[4] = {0, 0, 0, 0};
+        int cg[4];
+        mma_s8(cg, A, b0, b1, zero);
+        F[p][0] = fmaf(d0, (float)cg[0], F[p][0]);
+        F[p][1] = fmaf(d0, (float)cg[1], F[p][1]);
+        F[p][2] = fmaf(d1, (float)cg[2], F[p][2]);
+        F[p][3] = fmaf(d1, (float)cg[3], F[p][3]);
+      }
+    }
+  }
+}
+
+// Q2_K: value = d*sc*q - dmin*m.  Main term: A = q*sc (exact int8) against
+// the limbs of h.  Min term: A = m (per 16-element sub-block) against the
+// limbs of the 16-element sums of h.
+template <int MAXP>
+__device__ __forceinline__ void q2k_chunk(const uint8_t *st, int RS, const Chunk &ch,
+                                          const int8_t *const (&bcol)[MAXP], const int8_t *const (&xcol)[MAXP],
+                                          int npairs, float (&F)[MAXP][4], float (&G)[MAXP][4]) {
+  const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const uint8_t *row0 = st + r * RS;
+  const uint8_t *row1 = st + (r + 8) * RS;
+  for (int b = 0; b < ch.nb; ++b) {
+    const uint8_t *p0 = row0 + 84 * b;
+    const uint8_t *p1 = row1 + 84 * b;
+    const uint32_t dd0 = lds_u32(p0 + 80), dd1 = lds_u32(p1 + 80);
+    const float d0 = half_bits_to_float((uint16_t)(dd0 & 0xFFFFu)), m0 = half_bits_to_float((uint16_t)(dd0 >> 16));
+    const float d1 = half_bits_to_float((uint16_t)(dd1 & 0xFFFFu)), m1 = half_bits_to_float((uint16_t)(dd1 >> 16));
+    int Cm[MAXP][4];
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) Cm[p][0] = Cm[p][1] = Cm[p][2] = Cm[p][3] = 0;
+    const int kb = (ch.k0 >> 8) + b;  // global block index along K
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t q00 = lds_u32(p0 + 16 + 32 * hf + 8 * c), q01 = lds_u32(p0 + 20 + 32 * hf + 8 * c);
+      const uint32_t q10 = lds_u32(p1 + 16 + 32 * hf + 8 * c), q11 = lds_u32(p1 + 20 + 32 * hf + 8 * c);
+      const uint32_t s00 = lds_u32(p0 + 8 * hf), s01 = lds_u32(p0 + 8 * hf + 4);
+      const uint32_t s10 = lds_u32(p1 + 8 * hf), s11 = lds_u32(p1 + 8 * hf + 4);
+#pragma unroll
+      for (int sh = 0; sh < 4; ++sh) {
+        const int bsh = 8 * (2 * (sh & 1) + (c >> 1));
+        const uint32_t sc0 = ((sh < 2 ? s00 : s01) >> bsh) & 15u;
+        const uint32_t sc1 = ((sh < 2 ? s10 : s11) >> bsh) & 15u;
+        uint32_t A[4];
+        A[0] = ((q00 >> (2 * sh)) & 0x03030303u) * sc0;
+        A[2] = ((q01 >> (2 * sh)) & 0x03030303u) * sc0;
+        A[1] = ((q10 >> (2 * sh)) & 0x03030303u) * sc1;
+        A[3] = ((q11 >> (2 * sh)) & 0x03030303u) * sc1;
+        const int kel = ch.k0 + 256 * b + 128 * hf + 32 * sh + 8 * c;
+#pragma unroll
+        for (int p = 0; p < MAXP; ++p) {
+          if (p < npairs) {
+            uint32_t b0 = 0, b1 = 0;
+            if (bcol[p]) {
+              const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
+              b0 = v.x;
+              b1 = v.y;
+            }
+            mma_s8(Cm[p], A, b0, b1, Cm[p]);
+          }
+        }
+      }
+    }
+    // min term over the 16 sub-blocks: thread c covers sub-blocks 4c..4c+3
+    uint32_t Am[4];
+    Am[0] = (lds_u32(p0 + 4 * c) >> 4) & 0x0F0F0F0Fu;
+    Am[1] = (lds_u32(p1 + 4 * c) >> 4) & 0x0F0F0F0Fu;
+    Am[2] = 0u;
+    Am[3] = 0u;
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) {
+      if (p < npairs) {
+        uint32_t b0 = 0;
+        if (xcol[p]) b0 = *reinterpret_cast<const uint32_t *>(xcol[p] + kb * 16 + 4 * c);
+        const int zero[4] = {0, 0, 0, 0};
+        int cn[4];
+        mma_s8(cn, Am, b0, 0u, zero);
+        F[p][0] = fmaf(d0, (float)Cm[p][0], F[p][0]);
+        F[p][1] = fmaf(d0, (float)Cm[p][1], F[p][1]);
+        F[p][2] = fmaf(d1, (float)Cm[p][2], F[p][2]);
+        F[p][3] = fmaf(d1, (float)Cm[p][3], F[p][3]);
+        G[p][0] = fmaf(m0, (float)cn[0], G[p][0]);
+        G[p][1] = fmaf(m0, (float)cn[1], G[p][1]);
+        G[p][2] = fmaf(m1, (float)cn[2], G[p][2]);
+        G[p][3] = fmaf(m1, (float)cn[3], G[p][3]);
+      }
+    }
+  }
+}
+
+// Sum of the limb columns: thread (r, c) holds columns 2c, 2c+1 = limbs
+// 2(c&1), 2(c&1)+1 of token slot c>>1 of the pair.  Returns the row-r and
+// row-(r+8) values of that token (identical in lanes c and c^1).
+__device__ __forceinline__ void combine_limbs(const float (&F)[4], const float *scale, float &v0, float &v1) {
+  const int c = threadIdx.x & 3;
+  const int l0 = 2 * (c & 1);
+  const float s0 = scale ? scale[l0] : 0.f;
+  const float s1 = (scale && l0 + 1 < 3) ? scale[l0 + 1] : 0.f;
+  v0 = s0 * F[0] + s1 * F[1];
+  v1 = s0 * F[2] + s1 * F[3];
+  v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+  v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+}
+
+// Three-limb int8 quantisation of n floats with scale max/127.
+__device__ void quantise_vector(const float *src, int n, float vmax, int8_t *dst, int dstride, float *scales) {
+  const int lane = threadIdx.x & 31;
+  const float s1 = vmax > 0.f ? vmax / 127.f : 1.f;
+  const float s2 = s1 / 254.f, s3 = s2 / 254.f;
+  const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
+  for (int j = lane; j < n; j += 32) {
+    const float v = __ldcg(src + j);
+    const float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
+    const float e1 = fmaf(-q1, s1, v);
+    const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+    const float e2 = fmaf(-q2, s2, e1);
+    const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+    dst[j] = (int8_t)q1;
+    dst[dstride + j] = (int8_t)q2;
+    dst[2 * dstride + j] = (int8_t)q3;
+  }
+  if (lane == 0) {
+    scales[0] = s1;
+    scales[1] = s2;
+    scales[2] = s3;
+    scales[3] = 0.f;
+  }
+}
+
+// Shared-memory tables of k2: +/- codebook and byte-permute selectors.
+__device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, int *err) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 256 * 8; i += blockDim.x) {
+    const int ix = i >> 3, rep = i & 7;
+    uint8_t g[8];
+    bool bad = false;
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+      g[l] = grid[8 * ix + l];
+      bad |= g[l] > 127;
+    }
+    if (bad) set_error(err, kErrGrid);
+    uint8_t *e = gpm + ix * 128 + rep * 16;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      e[l] = g[l];
+      e[4 + l] = (uint8_t)(-(int)g[l]);
+      e[8 + l] = g[4 + l];
+      e[12 + l] = (uint8_t)(-(int)g[4 + l]);
+    }
+  }
+  for (int i = tid; i < 128 * 16; i += blockDim.x) {
+    const int m7 = i >> 4, rep = i & 15;
+    const uint32_t m8 = (uint32_t)m7 | ((uint32_t)(__popc(m7) & 1) << 7);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      lo |= (uint32_t)(l + 4 * ((m8 >> l) & 1u)) << (4 * l);
+      hi |= (uint32_t)(l + 4 * ((m8 >> (l + 4)) & 1u)) << (4 * l);
+    }
+    uint32_t *e = reinterpret_cast<uint32_t *>(selt + m7 * 128 + rep * 8);
+    e[0] = lo;
+    e[1] = hi;
+  }
+}
+
+// ------------------------------------------------------------------ k2
+
+struct K2Shared {
+  int32_t idx[kDecodeMaxT * kMaxK];
+  float w[kDecodeMaxT * kMaxK];
+  Jobs J;
+  float hsm[kWarps2][kDecodeMaxT][16];
+};
+
+// Writes the 16 x ntok SwiGLU outputs held in hs (token slot, row) for the
+// vectors vec[slot], updates max|h|, the 16-row sum and the tile counters;
+// the warp that completes a vector quantises it.
+__device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int ntok, const int *vec, int r0,
+                              int n, int ntiles) {
+  const int lane = threadIdx.x & 31;
+  const DecodeScratch &s = a.s;
+  for (int base = 0; base < ntok; base += 2) {
+    const int slot = base + (lane >> 4), row = lane & 15;
+    const bool ok = slot < ntok;
+    const float h = ok ? hs[slot][row] : 0.f;
+    float m = fabsf(h), sum = h;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    if (ok) {
+      const int v = vec[slot];
+      s.hbuf[(size_t)v * s.Imax + r0 + row] = h;
+      if (row == 0) {
+        s.Xbuf[(size_t)v * (s.Imax / 16) + r0 / 16] = sum;
+        atomicMax(s.hmax + v, __float_as_uint(m));
+        atomicMax(s.Xmax + v, __float_as_uint(fabsf(sum)));
+      }
+    }
+  }
+  __threadfence();
+  __syncwarp();
+  for (int slot = 0; slot < ntok; ++slot) {
+    const int v = vec[slot];
+    int last = 0;
+    if (lane == 0) last = atomicAdd(s.vcount + v, 1) == ntiles - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence();
+      const float hm = __uint_as_float(__ldcg(s.hmax + v));
+      const float xm = __uint_as_float(__ldcg(s.Xmax + v));
+      quantise_vector(s.hbuf + (size_t)v * s.Imax, n, hm, s.hq + (size_t)v * 3 * s.Imax, s.Imax, s.hsc + 4 * v);
+      quantise_vector(s.Xbuf + (size_t)v * (s.Imax / 16), n / 16, xm, s.Xq + (size_t)v * 3 * (s.Imax / 16),
+                      s.Imax / 16, s.Xsc + 4 * v);
+    }
+  }
+}
+
+// Runs a list of chunks through the warp's two-stage ring; `compute(i, st)`
+// consumes chunk i from stage st.
+template <typename ChunkAt, typename Compute>
+__device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int n, ChunkAt chunk_at,
+                                           Compute compute) {
+  {
+    const Chunk c0 = chunk_at(0);
+    stage_chunk(stage0, stage_rs(c0.bpr), c0.g, c0.gstride, c0.bpr, c0.a16);
+  }
+  for (int i = 0; i < n; ++i) {
+    uint8_t *cur = (i & 1) ? stage1 : stage0;
+    uint8_t *nxt = (i & 1) ? stage0 : stage1;
+    if (i + 1 < n) {
+      const Chunk cn = chunk_at(i + 1);
+      stage_chunk(nxt, stage_rs(cn.bpr), cn.g, cn.gstride, cn.bpr, cn.a16);
+    } else {
+      cp_async_commit();
+    }
+    cp_async_wait<1>();
+    __syncwarp();
+    compute(i, cur);
+    __syncwarp();
+  }
+}
+
+template <int MAXP>
+__global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const LayerDims &d = a.d;
+  const DecodeScratch &s = a.s;
+  const int T = a.T;
+  uint8_t *gpm = smem;
+  uint8_t *selt = gpm + kGpmBytes;
+  uint8_t *stages = selt + kSelBytes;
+  K2Shared &S = *reinterpret_cast<K2Shared *>(stages + 2 * kWarps2 * kStageBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  build_tables(a.wt.grid, gpm, selt, a.err);
+  for (int t = warp; t < T; t += kWarps2) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int i = tid; i < T * d.k; i += blockDim.x) {
+      s.idx[i] = S.idx[i];
+      s.w[i] = S.w[i];
+    }
+  }
+  build_jobs(S.idx, T, d.k, S.J);
+
+  const uint8_t *gpm_l = gpm + (lane & 7) * 16;
+  const uint8_t *sel_l = selt + (lane & 15) * 8;
+  uint8_t *st0 = stages + warp * 2 * kStageBytes;
+  uint8_t *st1 = st0 + kStageBytes;
+  const int r = lane >> 2, c = lane & 3;
+
+  const int tilesI = d.I / 16, tilesS = d.Is / 16;
+  const int n_sh = tilesS * 4;
+  const int n_units = n_sh + S.J.n * tilesI;
+  // IQ2 chunking along H
+  const int nbH = d.H / 256;
+  const int cbI = nbH < 8 ? nbH : 8;
+  const int nckI = nbH / cbI;
+  const size_t rbI = (size_t)nbH * 66;
+  // Q8_0 shared: a quarter of H in chunks of up to 16 blocks
+  const int nbQ = d.H / 128;  // blocks per quarter
+  const int cbQ = nbQ < 16 ? nbQ : 16;
+  const int nckQ = nbQ / cbQ;
+  const size_t rbQ = (size_t)(d.H / 32) * 34;
+
+  while (true) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(s.work + 0, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= n_units) break;
+
+    if (u < n_sh) {
+      // ---- shared expert: 16-row tile, one K quarter, gate and up
+      const int tile = u >> 2, q = u & 3;
+      const int r0 = tile * 16;
+      const int npairs = (T + 1) >> 1;
+      const int8_t *bcol[MAXP];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        const int ts = 2 * p + (r >> 2), limb = r & 3;
+        bcol[p] = (ts < T && limb < 3) ? s.xq + ((size_t)ts * 3 + limb) * d.H : nullptr;
+      }
+      float F[2][MAXP][4];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
+      auto chunk_at = [&](int i) {
+        const int m = i / nckQ, ck = i % nckQ;
+        const uint8_t *base = (m == 0 ? a.wt.sh_gate : a.wt.sh_up) + (size_t)r0 * rbQ +
+                              (size_t)(q * nbQ + ck * cbQ) * 34;
+        Chunk ch;
+        ch.g = base;
+        ch.gstride = rbQ;
+        ch.bpr = cbQ * 34;
+        ch.nb = cbQ;
+        ch.k0 = (q * nbQ + ck * cbQ) * 32;
+        ch.a16 = ((rbQ & 15) == 0) && (((size_t)(q * nbQ + ck * cbQ) * 34) & 15) == 0 && ((cbQ * 34) & 15) == 0;
+        return ch;
+      };
+      run_chunks(st0, st1, 2 * nckQ, chunk_at, [&](int i, uint8_t *st) {
+        const Chunk ch = chunk_at(i);
+        if (i / nckQ == 0)
+          q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F[0]);
+        else
+          q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F[1]);
+      });
+      // partial sums of this quarter -> global, last quarter finishes the tile
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < npairs) {
+          const int ts = 2 * p + (c >> 1);
+          const float *sc = ts < T ? s.xs + 4 * ts : nullptr;
+          float g0, g1, u0, u1;
+          combine_limbs(F[0][p], sc, g0, g1);
+          combine_limbs(F[1][p], sc, u0, u1);
+          if ((c & 1) == 0 && ts < T) {
+            float *pg = s.shpart + ((size_t)(0 * 4 + q) * T + ts) * d.Is + r0;
+            float *pu = s.shpart + ((size_t)(1 * 4 + q) * T + ts) * d.Is + r0;
+            pg[r] = g0;
+            pg[r + 8] = g1;
+            pu[r] = u0;
+            pu[r + 8] = u1;
+          }
+        }
+      }
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(s.shcount + tile, 1) == 3;
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();
+        for (int i = lane; i < 16 * T; i += 32) {
+          const int ts = i >> 4, row = i & 15;
+          float ga = 0.f, ub = 0.f;
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            ga += __ldcg(s.shpart + ((size_t)(0 * 4 + qq) * T + ts) * d.Is + r0 + row);
+            ub += __ldcg(s.shpart + ((size_t)(1 * 4 + qq) * T + ts) * d.Is + r0 + row);
+          }
+          S.hsm[warp][ts][row] = silu(ga) * ub;
+        }
+        __syncwarp();
+        int vec[kDecodeMaxT];
+#pragma unroll
+        for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = T * d.k + t;
+        finish_h_tile(a, S.hsm[warp], T, vec, r0, d.Is, tilesS);
+      }
+    } else {
+      // ---- routed expert: 16-row tile of gate and up, full K
+      const int uu = u - n_sh;
+      const int j = uu / tilesI, tile = uu % tilesI;
+      const int r0 = tile * 16;
+      const int e = S.J.e[j], ntok = S.J.cnt[j];
+      const int *pairs = S.J.pair + S.J.first[j];
+      const int npairs = (ntok + 1) >> 1;
+      const int8_t *bcol[MAXP];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        const int ts = 2 * p + (r >> 2), limb = r & 3;
+        bcol[p] = (ts < ntok && limb < 3) ? s.xq + ((size_t)(pairs[ts] / d.k) * 3 + limb) * d.H : nullptr;
+      }
+      float F[2][MAXP][4];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
+      auto chunk_at = [&](int i) {
+        const int m = i / nckI, ck = i % nckI;
+        const uint8_t *base = (m == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + (size_t)ck * cbI * 66;
+        Chunk ch;
+        ch.g = base;
+        ch.gstride = rbI;
+        ch.bpr = cbI * 66;
+        ch.nb = cbI;
+        ch.k0 = ck * cbI * 256;
+        ch.a16 = ((rbI & 15) == 0) && (((size_t)ck * cbI * 66) & 15) == 0 && ((cbI * 66) & 15) == 0;
+        return ch;
+      };
+      run_chunks(st0, st1, 2 * nckI, chunk_at, [&](int i, uint8_t *st) {
+        const Chunk ch = chunk_at(i);
+        if (i / nckI == 0)
+          iq2_chunk<MAXP>(st, stage_rs(ch.bpr), ch, gpm_l, sel_l, bcol, npairs, F[0]);
+        else
+          iq2_chunk<MAXP>(st, stage_rs(ch.bpr), ch, gpm_l, sel_l, bcol, npairs, F[1]);
+      });
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < npairs) {
+          const int ts = 2 * p + (c >> 1);
+          const float *sc = ts < ntok ? s.xs + 4 * (pairs[ts] / d.k) : nullptr;
+          float g0, g1, u0, u1;
+          combine_limbs(F[0][p], sc, g0, g1);
+          combine_limbs(F[1][p], sc, u0, u1);
+          if ((c & 1) == 0 && ts < ntok) {
+            S.hsm[warp][ts][r] = silu(g0) * u0;
+            S.hsm[warp][ts][r + 8] = silu(g1) * u1;
+          }
+        }
+      }
+      __syncwarp();
+      int vec[kDecodeMaxT];
+#pragma unroll
+      for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < ntok ? pairs[t] : 0;
+      finish_h_tile(a, S.hsm[warp], ntok, vec, r0, d.I, tilesI);
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ k3
+
+struct K3Shared {
+  int32_t idx[kDecodeMaxT * kMaxK];
+  float w[kDecodeMaxT * kMaxK];
+  Jobs J;
+  float ysm[kWarps2][kDecodeMaxT][16];
+};
+
+template <int MAXP>
+__global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const LayerDims &d = a.d;
+  const DecodeScratch &s = a.s;
+  const int T = a.T;
+  uint8_t *stages = smem;
+  K3Shared &S = *reinterpret_cast<K3Shared *>(stages + 2 * kWarps2 * kStageBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < T * d.k; i += blockDim.x) {
+    S.idx[i] = s.idx[i];
+    S.w[i] = s.w[i];
+  }
+  __syncthreads();
+  build_jobs(S.idx, T, d.k, S.J);
+
+  uint8_t *st0 = stages + warp * 2 * kStageBytes;
+  uint8_t *st1 = st0 + kStageBytes;
+  const int r = lane >> 2, c = lane & 3;
+  const int tilesH = d.H / 16;
+  const int nparts = S.J.n + 4;
+  const int n_units = tilesH * nparts;
+  const int Im16 = s.Imax / 16;
+  // Q2_K chunking along I: up to 4 blocks (336 bytes) per chunk
+  const int nbI = d.I / 256;
+  const int cbD = nbI < 4 ? nbI : 4;
+  const int nckD = nbI / cbD;
+  const size_t rbD = (size_t)nbI * 84;
+  // Q8_0 shared down: a quarter of Is in chunks of up to 16 blocks
+  const int nbQ = d.Is / 128;
+  const int cbQ = nbQ < 16 ? nbQ : 16;
+  const int nckQ = nbQ / cbQ;
+  const size_t rbQ = (size_t)(d.Is / 32) * 34;
+
+  while (true) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(s.work + 1, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= n_units) break;
+    const int ot = u / nparts, part = u % nparts;
+    const int r0 = ot * 16;
+    float(*ys)[16] = S.ysm[warp];
+    for (int i = lane; i < kDecodeMaxT * 16; i += 32) ys[i >> 4][i & 15] = 0.f;
+    __syncwarp();
+
+    if (part < S.J.n) {
+      const int j = part;
+      const int e = S.J.e[j], ntok = S.J.cnt[j];
+      const int *pairs = S.J.pair + S.J.first[j];
+      const int npairs = (ntok + 1) >> 1;
+      const int8_t *bcol[MAXP];
+      const int8_t *xcol[MAXP];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        const int ts = 2 * p + (r >> 2), limb = r & 3;
+        const bool ok = ts < ntok && limb < 3;
+        const int v = ok ? pairs[ts] : 0;
+        bcol[p] = ok ? s.hq + ((size_t)v * 3 + limb) * s.Imax : nullptr;
+        xcol[p] = ok ? s.Xq + ((size_t)v * 3 + limb) * Im16 : nullptr;
+      }
+      float F[MAXP][4], G[MAXP][4];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
+      auto chunk_at = [&](int i) {
+        Chunk ch;
+        ch.g = a.wt.down + ((size_t)e * d.H + r0) * rbD + (size_t)i * cbD * 84;
+        ch.gstride = rbD;
+        ch.bpr = cbD * 84;
+        ch.nb = cbD;
+        ch.k0 = i * cbD * 256;
+        ch.a16 = ((rbD & 15) == 0) && (((size_t)i * cbD * 84) & 15) == 0 && ((cbD * 84) & 15) == 0;
+        return ch;
+      };
+      run_chunks(st0, st1, nckD, chunk_at, [&](int i, uint8_t *st) {
+        const Chunk ch = chunk_at(i);
+        q2k_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, xcol, npairs, F, G);
+      });
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < npairs) {
+          const int ts = 2 * p + (c >> 1);
+          const bool ok = ts < ntok;
+          const int v = ok ? pairs[ts] : 0;
+          const int l0 = 2 * (c & 1);
+          float v0 = 0.f, v1 = 0.f;
+          if (ok) {
+            const float *hs = s.hsc + 4 * v;
+            const float *xs = s.Xsc + 4 * v;
+            v0 = hs[l0] * F[p][0] - xs[l0] * G[p][0];
+            v1 = hs[l0] * F[p][2] - xs[l0] * G[p][2];
+            if (l0 + 1 < 3) {
+              v0 += hs[l0 + 1] * F[p][1] - xs[l0 + 1] * G[p][1];
+              v1 += hs[l0 + 1] * F[p][3] - xs[l0 + 1] * G[p][3];
+            }
+          }
+          v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+          v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+          if ((c & 1) == 0 && ok) {
+            const int t = v / d.k;
+            const float wt = S.w[v];
+            ys[t][r] = wt * v0;
+            ys[t][r + 8] = wt * v1;
+          }
+        }
+      }
+    } else {
+      const int q = part - S.J.n;
+      const int npairs = (T + 1) >> 1;
+      const int8_t *bcol[MAXP];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        const int ts = 2 * p + (r >> 2), limb = r & 3;
+        bcol[p] = (ts < T && limb < 3) ? s.hq + ((size_t)(T * d.k + ts) * 3 + limb) * s.Imax : nullptr;
+      }
+      float F[MAXP][4];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
+      auto chunk_at = [&](int i) {
+        Chunk ch;
+        const size_t off = (size_t)(q * nbQ + i * cbQ) * 34;
+        ch.g = a.wt.sh_down + (size_t)r0 * rbQ + off;
+        ch.gstride = rbQ;
+        ch.bpr = cbQ * 34;
+        ch.nb = cbQ;
+        ch.k0 = (q * nbQ + i * cbQ) * 32;
+        ch.a16 = ((rbQ & 15) == 0) && (off & 15) == 0 && ((cbQ * 34) & 15) == 0;
+        return ch;
+      };
+      run_chunks(st0, st1, nckQ, chunk_at, [&](int i, uint8_t *st) {
+        const Chunk ch = chunk_at(i);
+        q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F);
+      });
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) {
+        if (p < npairs) {
+          const int ts = 2 * p + (c >> 1);
+          const float *sc = ts < T ? s.hsc + 4 * (T * d.k + ts) : nullptr;
+          float v0, v1;
+          combine_limbs(F[p], sc, v0, v1);
+          if ((c & 1) == 0 && ts < T) {
+            ys[ts][r] = v0;
+            ys[ts][r + 8] = v1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // part -> global, the last part of the tile writes y
+    float *dst = s.ypart + ((size_t)ot * s.P + part) * T * 16;
+    for (int i = lane; i < 16 * T; i += 32) dst[i] = ys[i >> 4][i & 15];
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(s.ycount + ot, 1) == nparts - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence();
+      for (int i = lane; i < 16 * T; i += 32) {
+        const int t = i >> 4, row = i & 15;
+        float acc = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[(size_t)t * d.H + r0 + row] : 0.f;
+        for (int pp = 0; pp < nparts; ++pp) acc += __ldcg(s.ypart + ((size_t)ot * s.P + pp) * T * 16 + i);
+        a.y[(size_t)t * d.H + r0 + row] = acc;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ route only
+
+__global__ void k_route_only(DecodeArgs a, int32_t *idx, float *w) {
+  const int warp = threadIdx.x >> 5;
+  for (int t = blockIdx.x * (blockDim.x / 32) + warp; t < a.T; t += gridDim.x * (blockDim.x / 32))
+    warp_route_token(a, t, idx + (size_t)t * a.d.k, w + (size_t)t * a.d.k);
+}
+
+size_t k2_smem_bytes() {
+  return kGpmBytes + kSelBytes + 2 * kWarps2 * kStageBytes + sizeof(K2Shared);
+}
+size_t k3_smem_bytes() { return 2 * kWarps2 * kStageBytes + sizeof(K3Shared); }
+
+template <int MAXP>
+cudaError_t launch_k23(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(k2_gateup<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)k2_smem_bytes());
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k3_down<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k3_smem_bytes());
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
+  k2_gateup<MAXP><<<num_sms, kThreads2, k2_smem_bytes(), stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.ev_end) cudaEventRecord(a.ev_end, stream);
+  k3_down<MAXP><<<num_sms, kThreads2, k3_smem_bytes(), stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
+  const int nr = a.d.mode == MOE_ROUTE_ROUTER ? (a.d.E + 1) / 2 : 0;
+  const int grid = a.T + nr;
+  if (a.T <= 1)
+    k1_prep_router<1><<<grid, 128, 0, stream>>>(a);
+  else if (a.T <= 2)
+    k1_prep_router<2><<<grid, 128, 0, stream>>>(a);
+  else if (a.T <= 4)
+    k1_prep_router<4><<<grid, 128, 0, stream>>>(a);
+  else
+    k1_prep_router<8><<<grid, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_scratch_bytes(const LayerDims &d, int T) {
+  DecodeScratch s;
+  decode_carve(s, d, T, nullptr);
+  return reinterpret_cast<size_t>(s.work) + 4 * sizeof(int) + 256;
+}
+
+void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
+  const int V = T * d.k + T;
+  const int Imax = d.I > d.Is ? d.I : d.Is;
+  const int P = (T * d.k < d.E ? T * d.k : d.E) + 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    off = align_up(off, 256);
+    uint8_t *p = static_cast<uint8_t *>(base) + off;
+    off += bytes;
+    return p;
+  };
+  s.Imax = Imax;
+  s.P = P;
+  s.z = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
+  s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * T * d.k));
+  s.w = reinterpret_cast<float *>(take(sizeof(float) * T * d.k));
+  s.xq = reinterpret_cast<int8_t *>(take((size_t)T * 3 * d.H));
+  s.xs = reinterpret_cast<float *>(take(sizeof(float) * 4 * T));
+  s.hbuf = reinterpret_cast<float *>(take(sizeof(float) * (size_t)V * Imax));
+  s.hq = reinterpret_cast<int8_t *>(take((size_t)V * 3 * Imax));
+  s.hsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V));
+  s.Xbuf = reinterpret_cast<float *>(take(sizeof(float) * (size_t)V * (Imax / 16)));
+  s.Xq = reinterpret_cast<int8_t *>(take((size_t)V * 3 * (Imax / 16)));
+  s.Xsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V));
+  s.hmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
+  s.Xmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
+  s.vcount = reinterpret_cast<int *>(take(sizeof(int) * V));
+  s.shpart = reinterpret_cast<float *>(take(sizeof(float) * 2 * 4 * (size_t)T * d.Is));
+  s.shcount = reinterpret_cast<int *>(take(sizeof(int) * (d.Is / 16)));
+  s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * P * T * 16));
+  s.ycount = reinterpret_cast<int *>(take(sizeof(int) * (d.H / 16)));
+  s.work = reinterpret_cast<int *>(take(sizeof(int) * 4));
+}
+
+cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
+  cudaError_t e = launch_k1(a, stream);
+  if (e != cudaSuccess) return e;
+  if (a.T <= 2) return launch_k23<1>(a, stream, num_sms);
+  if (a.T <= 4) return launch_k23<2>(a, stream, num_sms);
+  return launch_k23<4>(a, stream, num_sms);
+}
+
+cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {
+  cudaError_t e = launch_k1(a, stream);
+  if (e != cudaSuccess) return e;
+  k_route_only<<<(a.T + 7) / 8, 256, 0, stream>>>(a, idx, w);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,70 @@
+// layer.cuh -- argument block and scratch layout shared by the layer's host
+// code and kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kDecodeMaxT = 8;  // token counts handled by the GEMV (mma.sync) path
+constexpr int kMaxK = 8;
+constexpr int kMaxE = 256;
+
+struct LayerDims {
+  int H, I, Is, E, k, mode, flags, vocab;
+  float scaling, eps;
+};
+
+struct LayerWeights {
+  const uint16_t *Wr;
+  const float *bias;
+  const int32_t *tid2eid;
+  const uint8_t *gate, *up, *down, *sh_gate, *sh_up, *sh_down, *grid;
+};
+
+// Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
+// t*k + slot, shared vector T*k + t.
+struct DecodeScratch {
+  double *z;        // [T][E] router logits (fp64)
+  int32_t *idx;     // [T][k]
+  float *w;         // [T][k]
+  int8_t *xq;       // [T][3][H] int8 limbs of the expert input
+  float *xs;        // [T][4] limb scales
+  float *hbuf;      // [V][Imax] SwiGLU outputs
+  int8_t *hq;       // [V][3][Imax]
+  float *hsc;       // [V][4]
+  float *Xbuf;      // [V][Imax/16] sums of 16 consecutive h
+  int8_t *Xq;       // [V][3][Imax/16]
+  float *Xsc;       // [V][4]
+  unsigned *hmax;   // [V] max |h| (float bits)
+  unsigned *Xmax;   // [V]
+  int *vcount;      // [V] finished 16-row tiles per vector
+  float *shpart;    // [2][4][T][Is] shared gate/up partial sums per K quarter
+  int *shcount;     // [Is/16]
+  float *ypart;     // [H/16][P][T][16] per-part output tiles
+  int *ycount;      // [H/16]
+  int *work;        // [4] unit counters
+  int Imax;
+  int P;            // max parts per output tile = min(T*k, E) + 4
+};
+
+struct DecodeArgs {
+  LayerDims d;
+  LayerWeights wt;
+  int T;
+  const float *x;
+  const int32_t *token_ids;
+  float *y;
+  DecodeScratch s;
+  int *err;
+  cudaEvent_t ev_begin, ev_end;  // recorded around k2 when set
+};
+
+size_t decode_scratch_bytes(const LayerDims &d, int T);
+void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base);
+cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms);
+cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,482 @@
+// prefill.cu -- routing and token permutation for larger token counts.
+//
+// Router: z = W_r x for all tokens as a tiled fp32 GEMM on the CUDA cores,
+// each 32-element K chunk summed with fp32 FMAs and the chunk sums added in
+// fp64.  A chunk of n FMAs has error at most gamma_n * sum|w x| (Higham,
+// "Accuracy and Stability of Numerical Algorithms", Thm 3.1 with
+// gamma_n = n u / (1 - n u), u = 2^-24), and sum|w x| <= |w_e|_2 |x_t|_2
+// (Cauchy-Schwarz), so each logit comes with a rigorous interval.  The
+// sqrtsoftplus score is increasing in z, so the selection is certified when
+// every selected key's lower end beats every other key's upper end; tokens
+// that fail the test are recomputed in fp64 (exactly the oracle's reduction
+// up to fp64 rounding order).
+#include <float.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "prefill.cuh"
+
+namespace moe {
+
+namespace {
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+__device__ __forceinline__ double sqrtsoftplus(double z) { return sqrt(fmax(z, 0.0) + log1p(exp(-fabs(z)))); }
+
+// ---------------------------------------------------------------- init
+
+// 2-norm of every router row, rounded up to fp32.
+__global__ void k_row_norms(const uint16_t *Wr, int E, int H, float *out) {
+  const int e = blockIdx.x;
+  double ss = 0.0;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) {
+    double v = (double)half_bits_to_float(Wr[(size_t)e * H + j]);
+    ss += v * v;
+  }
+  ss = warp_sum_d(ss);
+  __shared__ double red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    out[e] = __double2float_ru(sqrt(t) * (1.0 + 1e-15));
+  }
+}
+
+// ---------------------------------------------------------------- router
+
+// Per token: inverse RMS (1 without the pre-norm flag) and the 2-norm of the
+// router input, both in fp64.
+__global__ void k_token_norms(const float *x, int T, int H, int flags, float eps, double *inv, double *nrm) {
+  const int t = blockIdx.x;
+  double ss = 0.0;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) {
+    double v = x[(size_t)t * H + j];
+    ss += v * v;
+  }
+  ss = warp_sum_d(ss);
+  __shared__ double red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    double iv = (flags & MOE_FLAG_PRENORM_RESIDUAL) ? 1.0 / sqrt(tot / (double)H + (double)eps) : 1.0;
+    inv[t] = iv;
+    nrm[t] = sqrt(tot) * iv;
+  }
+}
+
+// z[t][e] for a 64-token x 64-expert tile; 256 threads, each 4 x 4 outputs.
+constexpr int RT = 64, RE = 64, RK = 32;
+__global__ void __launch_bounds__(256) k_router_f32(const float *x, const double *inv, const uint16_t *Wr, int T,
+                                                    int E, int H, double *z) {
+  __shared__ __align__(16) float xs[RK][RT + 4];
+  __shared__ __align__(16) float ws[RK][RE + 4];
+  const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int k0 = 0; k0 < H; k0 += RK) {
+    // stage x (scaled by the token's inverse RMS) and W as fp32, K-major
+    for (int i = tid; i < RT * RK; i += 256) {
+      const int tt = i / RK, kk = i % RK;
+      const int t = t0 + tt;
+      float v = 0.f;
+      if (t < T) v = x[(size_t)t * H + k0 + kk] * (float)inv[t];
+      xs[kk][tt] = v;
+    }
+    for (int i = tid; i < RE * RK; i += 256) {
+      const int ee = i / RK, kk = i % RK;
+      const int e = e0 + ee;
+      ws[kk][ee] = e < E ? half_bits_to_float(Wr[(size_t)e * H + k0 + kk]) : 0.f;
+    }
+    __syncthreads();
+    float part[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+#pragma unroll 8
+    for (int kk = 0; kk < RK; ++kk) {
+      const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
+      const float4 wv = *reinterpret_cast<const float4 *>(&ws[kk][tx * 4]);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) z[(size_t)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+// Error bound of one logit.  The staged fp32 input fl(x * fl(inv)) is within
+// 2u of x*inv per element; a 32-term FMA chunk adds at most gamma_33; the
+// fp64 chunk additions and the oracle's own fp64 reduction are covered by
+// the 1e-12 term; everything is proportional to sum|w x| <= |w|_2 |x|_2.
+__device__ __forceinline__ double logit_bound(float wn, double xn) {
+  const double u = 5.9604644775390625e-8;  // 2^-24
+  const double g = 33.0 * u / (1.0 - 33.0 * u);
+  return (g + 2.0 * u + 1e-12) * (double)wn * xn * (1.0 + 1e-6) + 1e-300;
+}
+
+// One warp per token: top-k from the fp32-GEMM logits; certified tokens get
+// idx/w, the others are queued for the fp64 router.
+__global__ void k_topk_cert(const double *z, const float *bias, const float *wn, const double *xn, int T, int E,
+                            int k, float scaling, int32_t *idx, float *w, int32_t *fix) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const double *zt = z + (size_t)t * E;
+  double key[8], lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const double b = (double)bias[e];
+      const double dz = logit_bound(wn[e], xn[t]);
+      key[i] = sqrtsoftplus(zt[e]) + b;
+      lo[i] = sqrtsoftplus(zt[e] - dz) + b - 1e-12;
+      hi[i] = sqrtsoftplus(zt[e] + dz) + b + 1e-12;
+    } else {
+      key[i] = lo[i] = hi[i] = -DBL_MAX;
+    }
+  }
+  unsigned taken = 0;
+  int sel[kMaxK];
+#pragma unroll
+  for (int r = 0; r < kMaxK; ++r) {
+    sel[r] = INT_MAX;
+    if (r < k) {
+      double bk = -INFINITY;
+      int be = INT_MAX;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u) && key[i] > bk) {
+          bk = key[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ok > bk || (ok == bk && oe < be)) {
+          bk = ok;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      sel[r] = be;
+    }
+  }
+  // certificate: min lower end of the selected vs max upper end of the rest
+  double sel_lo = DBL_MAX, rest_hi = -DBL_MAX;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    if (e >= E) continue;
+    if ((taken >> i) & 1u)
+      sel_lo = fmin(sel_lo, lo[i]);
+    else
+      rest_hi = fmax(rest_hi, hi[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sel_lo = fmin(sel_lo, __shfl_xor_sync(0xffffffffu, sel_lo, o));
+    rest_hi = fmax(rest_hi, __shfl_xor_sync(0xffffffffu, rest_hi, o));
+  }
+  const bool certified = (k == E) || sel_lo > rest_hi;
+  if (lane != 0) return;
+  if (!certified) {
+    const int slot = atomicAdd(fix, 1);
+    fix[1 + slot] = t;
+    return;
+  }
+  // ascending ids
+  for (int i = 1; i < k; ++i)
+    for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
+      const int tmp = sel[j - 1];
+      sel[j - 1] = sel[j];
+      sel[j] = tmp;
+    }
+  double sv[kMaxK], tot = 0.0;
+  for (int i = 0; i < k; ++i) {
+    sv[i] = sqrtsoftplus(zt[sel[i]]);
+    tot += sv[i];
+  }
+  for (int i = 0; i < k; ++i) {
+    idx[(size_t)t * k + i] = sel[i];
+    w[(size_t)t * k + i] = (float)((double)scaling * sv[i] / tot);
+  }
+}
+
+// fp64 router for the queued tokens: one block (8 warps) per token.
+__global__ void __launch_bounds__(256) k_router_fix(const float *x, const double *inv, const uint16_t *Wr,
+                                                    const float *bias, int T, int E, int H, int k, float scaling,
+                                                    const int32_t *fix, double *z, int32_t *idx, float *w) {
+  const int nfix = fix[0];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ double zs[kMaxE];
+  for (int f = blockIdx.x; f < nfix; f += gridDim.x) {
+    const int t = fix[1 + f];
+    const float *xt = x + (size_t)t * H;
+    const double iv = inv[t];
+    for (int e = warp; e < E; e += 8) {
+      double acc = 0.0;
+      for (int j = lane; j < H; j += 32)
+        acc = fma((double)half_bits_to_float(Wr[(size_t)e * H + j]), (double)xt[j] * iv, acc);
+      acc = warp_sum_d(acc);
+      if (lane == 0) zs[e] = acc;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      double key[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = e < E ? sqrtsoftplus(zs[e]) + (double)bias[e] : -DBL_MAX;
+      }
+      unsigned taken = 0;
+      int sel[kMaxK];
+#pragma unroll
+      for (int r = 0; r < kMaxK; ++r) {
+        sel[r] = INT_MAX;
+        if (r < k) {
+          double bk = -INFINITY;
+          int be = INT_MAX;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && key[i] > bk) {
+              bk = key[i];
+              be = e;
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (ok > bk || (ok == bk && oe < be)) {
+              bk = ok;
+              be = oe;
+            }
+          }
+          if ((be & 31) == lane) taken |= 1u << (be >> 5);
+          sel[r] = be;
+        }
+      }
+      if (lane == 0) {
+        for (int i = 1; i < k; ++i)
+          for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
+            const int tmp = sel[j - 1];
+            sel[j - 1] = sel[j];
+            sel[j] = tmp;
+          }
+        double sv[kMaxK], tot = 0.0;
+        for (int i = 0; i < k; ++i) {
+          sv[i] = sqrtsoftplus(zs[sel[i]]);
+          tot += sv[i];
+        }
+        for (int i = 0; i < k; ++i) {
+          idx[(size_t)t * k + i] = sel[i];
+          w[(size_t)t * k + i] = (float)((double)scaling * sv[i] / tot);
+        }
+        for (int e = 0; e < E; ++e) z[(size_t)t * E + e] = zs[e];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Hash routing: ids from the table (ascending), weights scaling / k.
+__global__ void k_hash_route(const int32_t *token_ids, const int32_t *tid2eid, int vocab, int T, int k,
+                             float scaling, int32_t *idx, float *w, int *err) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  int tid = token_ids[t];
+  if (tid < 0 || tid >= vocab) {
+    set_error(err, kErrTokenId);
+    tid = 0;
+  }
+  int sel[kMaxK];
+  for (int i = 0; i < k; ++i) sel[i] = tid2eid[(size_t)tid * k + i];
+  for (int i = 1; i < k; ++i)
+    for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
+      const int tmp = sel[j - 1];
+      sel[j - 1] = sel[j];
+      sel[j] = tmp;
+    }
+  for (int i = 0; i < k; ++i) {
+    idx[(size_t)t * k + i] = sel[i];
+    w[(size_t)t * k + i] = scaling / (float)k;
+  }
+}
+
+// ---------------------------------------------------------------- permutation
+
+// counts[e] = number of pairs routed to e (one block per expert).
+__global__ void k_perm_count(const int32_t *idx, int n, int32_t *counts) {
+  const int e = blockIdx.x;
+  int c = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) c += idx[i] == e;
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  __shared__ int red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    counts[e] = t;
+  }
+}
+
+__global__ void k_perm_scan(const int32_t *counts, int E, int32_t *offsets) {
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      const int c = counts[e];  // counts may alias offsets: read before writing
+      offsets[e] = run;
+      run += c;
+    }
+    offsets[E] = run;
+  }
+}
+
+// perm[offsets[e] + rank] = pair id, ranks in ascending pair order (stable).
+__global__ void k_perm_scatter(const int32_t *idx, int n, const int32_t *offsets, int32_t *perm) {
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __shared__ int wcount[32];
+  int base = offsets[e];
+  for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const bool hit = i < n && idx[i] == e;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) wcount[warp] = __popc(m);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int q = 0; q < nw; ++q) {
+      if (q < warp) before += wcount[q];
+      total += wcount[q];
+    }
+    if (hit) perm[base + before + __popc(m & ((1u << lane) - 1u))] = i;
+    base += total;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t prefill_scratch_bytes(const LayerDims &d, int T) {
+  PrefillArgs p = prefill_args(d, LayerWeights{}, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return reinterpret_cast<size_t>(p.s.big) + 256;
+}
+
+PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, const float *x,
+                         const int32_t *token_ids, float *y, void *scratch, const float *row_norms, int *err) {
+  PrefillArgs p;
+  p.d = d;
+  p.wt = wt;
+  p.T = T;
+  p.x = x;
+  p.token_ids = token_ids;
+  p.y = y;
+  p.row_norms = row_norms;
+  p.err = err;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    off = align_up(off, 256);
+    uint8_t *q = static_cast<uint8_t *>(scratch) + off;
+    off += bytes;
+    return q;
+  };
+  p.s.z = reinterpret_cast<float *>(take(sizeof(double) * (size_t)T * d.E));
+  p.s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)T * d.k));
+  p.s.w = reinterpret_cast<float *>(take(sizeof(float) * (size_t)T * d.k));
+  p.s.counts = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * d.E));
+  p.s.offsets = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (d.E + 1)));
+  p.s.perm = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)T * d.k));
+  p.s.fix = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)(T + 1)));
+  // token norms (2 x fp64 per token)
+  take(2 * sizeof(double) * (size_t)T);
+  p.s.big = static_cast<uint8_t *>(scratch) + align_up(off, 256);
+  p.s.big_bytes = 0;
+  return p;
+}
+
+cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_norms, int *err, cudaStream_t s) {
+  (void)err;
+  if (d.mode != MOE_ROUTE_ROUTER) return cudaSuccess;
+  k_row_norms<<<d.E, 256, 0, s>>>(wt.Wr, d.E, d.H, row_norms);
+  return cudaGetLastError();
+}
+
+static double *token_norm_ptr(const PrefillArgs &p) {
+  uint8_t *fixp = reinterpret_cast<uint8_t *>(p.s.fix);
+  return reinterpret_cast<double *>(fixp + align_up(sizeof(int32_t) * (size_t)(p.T + 1), 256));
+}
+
+cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStream_t s) {
+  const LayerDims &d = p.d;
+  const int T = p.T;
+  if (d.mode == MOE_ROUTE_HASH) {
+    k_hash_route<<<(T + 255) / 256, 256, 0, s>>>(p.token_ids, p.wt.tid2eid, d.vocab, T, d.k, d.scaling, idx, w,
+                                                 p.err);
+    return cudaGetLastError();
+  }
+  double *inv = token_norm_ptr(p);
+  double *xn = inv + T;
+  double *z = reinterpret_cast<double *>(p.s.z);
+  cudaError_t e = cudaMemsetAsync(p.s.fix, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  k_token_norms<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, inv, xn);
+  dim3 g((T + RT - 1) / RT, (d.E + RE - 1) / RE);
+  k_router_f32<<<g, 256, 0, s>>>(p.x, inv, p.wt.Wr, T, d.E, d.H, z);
+  k_topk_cert<<<(T + 7) / 8, 256, 0, s>>>(z, p.wt.bias, p.row_norms, xn, T, d.E, d.k, d.scaling, idx, w, p.s.fix);
+  int nfix_blocks = T < 148 ? T : 148;
+  k_router_fix<<<nfix_blocks, 256, 0, s>>>(p.x, inv, p.wt.Wr, p.wt.bias, T, d.E, d.H, d.k, d.scaling, p.s.fix, z,
+                                          idx, w);
+  return cudaGetLastError();
+}
+
+cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
+  (void)p;
+  (void)s;
+  (void)num_sms;
+  return cudaErrorNotSupported;
+}
+
+cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, cudaStream_t s) {
+  // the counts are written into offsets[0..E) and scanned in place
+  const int n = T * k;
+  k_perm_count<<<E, 256, 0, s>>>(idx, n, offsets);
+  k_perm_scan<<<1, 32, 0, s>>>(offsets, E, offsets);
+  k_perm_scatter<<<E, 256, 0, s>>>(idx, n, offsets, perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

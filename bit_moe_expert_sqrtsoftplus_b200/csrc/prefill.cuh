@@ -1,0 +1,46 @@
+// prefill.cuh -- the layer for larger token counts (T > 8): certified router,
+// token permutation and grouped tensor-core GEMMs.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "layer.cuh"
+
+namespace moe {
+
+struct PrefillScratch {
+  float *z;          // [T][E] fp32 router logits
+  int32_t *idx;      // [T][k]
+  float *w;          // [T][k]
+  int32_t *counts;   // [E]
+  int32_t *offsets;  // [E+1]
+  int32_t *perm;     // [T*k]
+  int32_t *fix;      // [1 + T] tokens that need the fp64 router
+  void *big;         // remaining scratch for the expert GEMMs
+  size_t big_bytes;
+};
+
+struct PrefillArgs {
+  LayerDims d;
+  LayerWeights wt;
+  int T;
+  const float *x;
+  const int32_t *token_ids;
+  float *y;
+  PrefillScratch s;
+  const float *row_norms;  // [E] 2-norms of the router rows
+  int *err;
+};
+
+size_t prefill_scratch_bytes(const LayerDims &d, int T);
+PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, const float *x,
+                         const int32_t *token_ids, float *y, void *scratch, const float *row_norms, int *err);
+cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_norms, int *err, cudaStream_t s);
+cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStream_t s);
+cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms);
+// Stable grouping of the T*k (token, slot) pairs by expert.
+cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, cudaStream_t s);
+
+}  // namespace moe

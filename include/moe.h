@@ -1,0 +1,160 @@
+/*
+ * moe.h -- C ABI of one DwarfStar-quantised DeepSeek-V4-Flash MoE FFN layer
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * The layer (source: "DeepSeek-V4-Flash one-token computation flow, Dwarf
+ * Star q2", qiita.com/sukimaengineer/items/cd76fec76d49a098abed, section
+ * "MoE FFN 部の中身: router → top-6 → expert → 加重和"):
+ *
+ *   z = W_r x                      (F16 router, 4096 -> 256)
+ *   s = sqrt(softplus(z))          (sqrtsoftplus scoring)
+ *   top-k experts by s + bias      (bias for selection only; ties -> lower id)
+ *   g_i = s_i / sum_sel s          (norm_topk_prob), w_i = routed_scaling * g_i
+ *   y = shared(x) + sum_i w_i E_i(x),  E(x) = W_down (SiLU(W_gate x) * (W_up x))
+ *
+ * Hash-routed layers (the first three) skip the router: the expert ids come
+ * from a token-id table and every selected expert gets routed_scaling / k.
+ *
+ * Weight formats ("2bit 量子化はなぜ「冗談ではない」のか", ds4.c を読み解く #2,
+ * qiita.com/yoshiyakato/items/4678be0e7860ddb444ec, sections 3 and 4; and the
+ * bit-allocation table of the first page):
+ *   routed gate/up  IQ2_XXS  256 elements in 66 bytes
+ *   routed down     Q2_K     256 elements in 84 bytes
+ *   shared expert   Q8_0     32 elements in 34 bytes
+ *   router          F16      [n_experts][hidden]
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates no device memory: persistent state lives in the
+ *     caller's `persist` buffer, per-call temporaries in `scratch`.
+ *   - Every call is asynchronous on the given stream and never synchronises
+ *     the host, except moe_poll_device_error.
+ *   - Argument and shape errors are returned synchronously as a negative
+ *     moe_status and described by moe_last_error() (thread-local).  No C++
+ *     exception crosses this boundary.  Device-side problems (a bounded wait
+ *     that ran out) are recorded in a device error word read back by
+ *     moe_poll_device_error.
+ *   - Layouts are row-major; packed weight matrices are [out_row][in_block],
+ *     routed ones stacked as [expert][out_row][in_block].
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,       /* null pointer, negative count, bad enum */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2, /* dimensions this build does not handle */
+  MOE_ERR_MISALIGNED = -3,        /* a pointer is not 16-byte aligned */
+  MOE_ERR_WORKSPACE_TOO_SMALL = -4,
+  MOE_ERR_CUDA = -5,              /* a CUDA runtime call failed */
+  MOE_ERR_TIMEOUT = -6,           /* a bounded device wait ran out */
+  MOE_ERR_DEVICE_FAULT = -7       /* the device reported another error */
+} moe_status;
+
+typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
+
+/* flags */
+#define MOE_FLAG_PRENORM_RESIDUAL 1 /* forward computes x + MoE(RMSNorm(x)) */
+
+typedef struct {
+  int hidden;           /* H: multiple of 256 (4096 for V4-Flash) */
+  int inter;            /* I: routed expert intermediate, multiple of 256 (2048) */
+  int n_experts;        /* E: routed experts, k <= E <= 256 */
+  int top_k;            /* k: 1..8 (6) */
+  int shared_inter;     /* Is: shared expert intermediate, multiple of 256 (2048) */
+  int vocab;            /* rows of tid2eid (hash mode; 129280 for V4-Flash) */
+  float routed_scaling; /* 1.5 */
+  float rms_eps;        /* RMSNorm epsilon when MOE_FLAG_PRENORM_RESIDUAL is set (1e-6) */
+  int mode;             /* moe_route_mode */
+  int flags;            /* MOE_FLAG_* */
+} moe_config;
+
+typedef struct {
+  const void *router_w_f16;   /* [E][H] IEEE f16; NULL in hash mode */
+  const float *router_bias;   /* [E] fp32 selection bias; NULL in hash mode */
+  const int32_t *tid2eid;     /* [vocab][k] expert ids; NULL in router mode */
+  const void *gate_iq2xxs;    /* [E][I][H/256] 66-byte blocks */
+  const void *up_iq2xxs;      /* [E][I][H/256] 66-byte blocks */
+  const void *down_q2k;       /* [E][H][I/256] 84-byte blocks */
+  const void *sh_gate_q80;    /* [Is][H/32] 34-byte blocks */
+  const void *sh_up_q80;      /* [Is][H/32] 34-byte blocks */
+  const void *sh_down_q80;    /* [H][Is/32] 34-byte blocks */
+  const uint8_t *iq2_grid;    /* [256][8] codebook; every entry must be <= 127 */
+} moe_weights;
+
+typedef struct moe_handle moe_handle;
+
+/*
+ * Sizes of the two caller-owned buffers for calls with up to `max_tokens`
+ * tokens.  `persist` must outlive the handle; `scratch` is needed only for
+ * the duration of each call (stream order).  Either output may be NULL.
+ */
+moe_status moe_workspace_size(const moe_config *cfg, int max_tokens, size_t *persist_bytes,
+                              size_t *scratch_bytes);
+
+/*
+ * Validates the configuration and the weight pointers (non-null as the mode
+ * requires, 16-byte aligned), records them in a host-side handle and
+ * enqueues the initialisation of `persist` on `stream` (it checks the
+ * codebook range into the device error word).  The weight buffers are read,
+ * never written, and must stay valid while the handle is used.
+ */
+moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, size_t persist_bytes,
+                    moe_stream_t stream, moe_handle **out);
+
+/*
+ * Routing only.  x: [T][H] fp32 (device).  token_ids: [T] int32 (hash mode;
+ * ignored in router mode, may be NULL there).  Writes idx [T][k] int32 with
+ * each row's expert ids in ascending order and w [T][k] fp32 routing weights
+ * in the same order (each row sums to routed_scaling).  When both
+ * expert_offsets ([E+1]) and perm ([T*k]) are non-NULL it also writes the
+ * grouping of the T*k (token, slot) pairs by expert: offsets[e] is the
+ * number of pairs on experts below e, and perm lists t*k + slot for each
+ * expert in ascending token order.  With MOE_FLAG_PRENORM_RESIDUAL the
+ * router sees RMSNorm(x).
+ */
+moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, int T, int32_t *idx, float *w,
+                     int32_t *expert_offsets, int32_t *perm, void *scratch, size_t scratch_bytes,
+                     moe_stream_t stream);
+
+/*
+ * The whole layer.  x: [T][H] fp32 input; y: [T][H] fp32 output
+ * (overwritten; may alias x only with MOE_FLAG_PRENORM_RESIDUAL, where
+ * y = x + MoE(RMSNorm(x))).  T = 0 is a no-op.
+ */
+moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
+                           void *scratch, size_t scratch_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device error word:
+ * MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED_SHAPE (codebook entry > 127)
+ * or MOE_ERR_DEVICE_FAULT. */
+moe_status moe_poll_device_error(moe_handle *h, moe_stream_t stream);
+
+/* Human-readable description of the last error on this thread ("" if none). */
+const char *moe_last_error(void);
+
+/*
+ * Optional instrumentation.  While set, every moe_ffn_forward on this handle
+ * records `ev_begin` on its stream right before the layer's dominant kernel
+ * (the routed gate/up kernel) and `ev_end` right after it.  Both are
+ * cudaEvent_t handles created and owned by the caller; pass NULL for both to
+ * stop recording.  Recording changes no work the layer does.
+ */
+moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end);
+
+/* Frees the host-side handle (the caller frees `persist`). NULL is a no-op. */
+void moe_destroy(moe_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -131,7 +131,8 @@ def silu(u: float) -> float:
 
 
 def router_logits(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
-    xx, px = _c(x, np.float32)
+    """z = W_r x in fp64 (fp32 inputs convert exactly)."""
+    xx, px = _c(x, np.float64)
     T, H = xx.shape
     E = Wr.shape[0]
     w, pw = _c(np.asarray(Wr).view(np.uint16) if np.asarray(Wr).dtype == np.float16 else Wr, np.uint16)

@@ -166,14 +166,14 @@ double oracle_sqrtsoftplus(double z) {
   return sqrt(softplus);
 }
 
-void oracle_router_logits(const float *x, int T, int H, const uint16_t *Wr, int E, double *z) {
+void oracle_router_logits(const double *x, int T, int H, const uint16_t *Wr, int E, double *z) {
   double *wrow = (double *)malloc(sizeof(double) * (size_t)H);
   for (int e = 0; e < E; ++e) {
     for (int c = 0; c < H; ++c) wrow[c] = oracle_f16(Wr[(size_t)e * H + c]);
     for (int t = 0; t < T; ++t) {
       double acc = 0.0;
-      const float *xt = x + (size_t)t * H;
-      for (int c = 0; c < H; ++c) acc += wrow[c] * (double)xt[c];
+      const double *xt = x + (size_t)t * H;
+      for (int c = 0; c < H; ++c) acc += wrow[c] * xt[c];
       z[(size_t)t * E + e] = acc;
     }
   }

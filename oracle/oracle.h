@@ -55,7 +55,7 @@ void oracle_matvec(int kind, const uint8_t *W, int rows, int cols, const uint8_t
 
 /* Router. */
 double oracle_sqrtsoftplus(double z);
-void oracle_router_logits(const float *x, int T, int H, const uint16_t *Wr, int E, double *z);
+void oracle_router_logits(const double *x, int T, int H, const uint16_t *Wr, int E, double *z);
 void oracle_select(const double *z, const float *bias, int T, int E, int k, double scaling, int32_t *idx,
                    double *w, double *margin);
 void oracle_hash_select(const int32_t *token_ids, int T, const int32_t *tid2eid, int vocab, int k,

@@ -1,0 +1,54 @@
+"""Shared helpers for the GPU parity tests: build device layers from the
+seeded generator, run the oracle on the same inputs, compare."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+
+GEMV_REL_L2 = 1e-4        # decode (mma.sync int8 limbs) path
+MMA_REL_L2 = 3e-3         # bf16 tensor-core path
+MAX_ABS_FRAC = 2e-2       # max |err| <= 2e-2 * max |y|
+
+
+def config_for(s: synth.LayerShape, mode=None, flags=0):
+    import bit_moe_expert_sqrtsoftplus_b200 as moe
+    if mode is None:
+        mode = moe.MOE_ROUTE_ROUTER
+    return moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
+                           routed_scaling=s.routed_scaling, rms_eps=1e-6, mode=mode, flags=flags)
+
+
+def device_layer(s: synth.LayerShape, seed: int, layer: int, router=True):
+    return synth.device_layer(seed, layer, s, router=router)
+
+
+def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, token_ids=None, router=True,
+                 prenorm=False):
+    """fp64 oracle: returns (idx, w, y, margin)."""
+    xin = x.astype(np.float64)
+    if prenorm:
+        xin = oracle.rmsnorm(xin, 1e-6)
+    if router:
+        Wr = synth.router_weight(seed, layer, s.n_experts, s.hidden)
+        b = synth.bias(seed, layer, s.n_experts, s.skew)
+        z = oracle.router_logits(xin, Wr)
+        idx, w, margin = oracle.select(z, b, s.top_k, s.routed_scaling)
+    else:
+        tab = synth.tid2eid(seed, layer, s.vocab, s.n_experts, s.top_k)
+        idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling)
+        margin = np.full(x.shape[0], np.inf)
+    W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router)
+    y = oracle.layer(W, s, xin, idx, w)
+    if prenorm:
+        y = y + x.astype(np.float64)
+    return idx, w, y, margin
+
+
+def errors(y: np.ndarray, ref: np.ndarray):
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rel_l2 = float(np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300))
+    max_abs = float(np.abs(y - ref).max() / max(np.abs(ref).max(), 1e-300))
+    return rel_l2, max_abs

@@ -1,0 +1,118 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every function
+declared in include/moe.h, and rejects bad arguments before touching the
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from bit_moe_expert_sqrtsoftplus_b200 import build
+    build.build()
+    import bit_moe_expert_sqrtsoftplus_b200 as m
+    return m
+
+
+def test_exports_every_declared_function(moe):
+    declared = _declared()
+    assert {"moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
+            "moe_last_error", "moe_destroy"} <= set(declared)
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def _cfg(moe, **over):
+    base = dict(hidden=4096, inter=2048, n_experts=256, top_k=6, shared_inter=2048, vocab=129280)
+    base.update(over)
+    return moe.make_config(**base)
+
+
+def test_workspace_size_and_shape_checks(moe):
+    p, s = moe.moe_workspace_size(_cfg(moe), 1)
+    assert p >= 4 and s > 0
+    p2, s32 = moe.moe_workspace_size(_cfg(moe), 4096)
+    assert s32 > s
+    for bad, status in ((dict(hidden=4000), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(inter=100), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(shared_inter=96), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(top_k=0), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(top_k=9), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(n_experts=300), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(n_experts=4, top_k=6), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                        (dict(mode=7), moe.MOE_ERR_INVALID_ARG),
+                        (dict(mode=1, vocab=0), moe.MOE_ERR_INVALID_ARG),
+                        (dict(flags=8), moe.MOE_ERR_INVALID_ARG)):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_workspace_size(_cfg(moe, **bad), 1)
+        assert ei.value.status == status, bad
+        assert moe.moe_last_error()
+
+
+def _fake_weights(moe, base=0x10000000, step=0x1000000, misalign=None, null=None):
+    names = [f for f, _ in moe.moe_weights._fields_]
+    vals = {}
+    for i, n in enumerate(names):
+        vals[n] = base + i * step
+    if misalign:
+        vals[misalign] += 8
+    if null:
+        vals[null] = None
+    return moe.moe_weights(**vals)
+
+
+class _FakeTensor:
+    def __init__(self, ptr, n):
+        self.ptr, self.n = ptr, n
+
+    def data_ptr(self):
+        return self.ptr
+
+    def numel(self):
+        return self.n
+
+    def element_size(self):
+        return 1
+
+
+def _init(moe, cfg, w, persist_ptr=0x7000000, persist_bytes=1 << 20):
+    h = ctypes.c_void_p(None)
+    st = moe.lib().moe_init(ctypes.byref(cfg), ctypes.byref(w), persist_ptr, persist_bytes, None, ctypes.byref(h))
+    return st, h.value
+
+
+def test_init_validates_before_touching_the_device(moe):
+    cfg = _cfg(moe)
+    assert _init(moe, cfg, _fake_weights(moe, null="gate_iq2xxs"))[0] == moe.MOE_ERR_INVALID_ARG
+    assert "gate_iq2xxs" in moe.moe_last_error()
+    assert _init(moe, cfg, _fake_weights(moe, misalign="down_q2k"))[0] == moe.MOE_ERR_MISALIGNED
+    assert _init(moe, cfg, _fake_weights(moe, null="router_w_f16"))[0] == moe.MOE_ERR_INVALID_ARG
+    hcfg = _cfg(moe, mode=moe.MOE_ROUTE_HASH)
+    assert _init(moe, hcfg, _fake_weights(moe, null="tid2eid"))[0] == moe.MOE_ERR_INVALID_ARG
+    assert _init(moe, cfg, _fake_weights(moe), persist_ptr=0)[0] == moe.MOE_ERR_INVALID_ARG
+    assert _init(moe, cfg, _fake_weights(moe), persist_ptr=0x7000004)[0] == moe.MOE_ERR_MISALIGNED
+    assert _init(moe, cfg, _fake_weights(moe), persist_bytes=8)[0] == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_calls_reject_null_handle(moe):
+    L = moe.lib()
+    assert L.moe_ffn_forward(None, None, None, 1, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(None, None, None, 1, None, None, None, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_poll_device_error(None, None) == moe.MOE_ERR_INVALID_ARG
+    L.moe_destroy(None)

@@ -70,3 +70,18 @@ def test_gaussian_inputs_are_seeded():
     assert a.dtype == np.float32 and abs(float(a.std()) - 1) < 0.1
     w = synth.router_weight(3, 5, 16, 256)
     assert w.dtype == np.float16 and abs(float(w.astype(np.float64).std()) - 0.02) < 0.002
+
+
+@pytest.mark.gpu
+def test_device_fill_is_byte_identical_to_host_fill():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    for kind, tensor, rows, cols in ((synth.KIND_IQ2XXS, synth.T_GATE, 64, 4096),
+                                     (synth.KIND_Q2K, synth.T_DOWN, 64, 2048),
+                                     (synth.KIND_Q80, synth.T_SH_UP, 64, 4096)):
+        host = synth.routed(3, 5, tensor, kind, 7, 2, rows, cols)
+        dev = torch.empty(host.shape, dtype=torch.uint8, device="cuda")
+        synth.device_routed(dev, 3, 5, tensor, kind, 7, 2, rows, cols)
+        torch.cuda.synchronize()
+        assert np.array_equal(dev.cpu().numpy(), host)
