@@ -43,6 +43,7 @@ def parse():
     p.add_argument("--workload", default="decode_t1", choices=["decode_t1", "decode_t32", "prefill_t4096"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
     return p.parse_args()
 
 
@@ -168,7 +169,7 @@ def run_ours(args, world, rank):
 
     s = synth.workload(args.workload)
     T = s.tokens
-    nsets = s.weight_sets
+    nsets = args.weight_sets if args.weight_sets > 0 else s.weight_sets
     layers, weights = [], []
     scratch = None
     for i in range(nsets):
@@ -216,6 +217,10 @@ def run_ours(args, world, rank):
                for _ in range(args.steps)]
         for i in range(args.steps):
             L = layers[(args.warmup + i) % nsets]
+            # torch only reports elapsed time for events it recorded itself; the
+            # library re-records the same events around the kernel afterwards
+            evs[i][0].record(stream)
+            evs[i][1].record(stream)
             moe.moe_set_timing_events(L.handle, *evs[i])
             step(args.warmup + i)
         torch.cuda.synchronize()
