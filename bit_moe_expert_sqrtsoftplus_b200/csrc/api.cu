@@ -259,6 +259,8 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
     e = moe::decode_forward(a, s, h->num_sms);
   } else {
     moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, y, scratch, h->row_norms, h->err);
+    p.ev_begin = h->ev_begin;
+    p.ev_end = h->ev_end;
     e = moe::prefill_forward(p, s, h->num_sms);
   }
   if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward launch");

@@ -1,0 +1,543 @@
+// gemm.cu -- persistent, warp-specialised grouped GEMM on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// One CTA per SM, 13 warps:
+//   warps 0-3   epilogue: tcgen05.ld of the 128-lane accumulator, SwiGLU /
+//               scatter-add / store
+//   warps 4-11  producers: dequantise the 128 x 64 weight tile(s) of a K step
+//               into 16-bit values written straight into the 128-byte-swizzled
+//               K-major operand layout, and gather the N x 64 activation tile
+//               with cp.async
+//   warp 12     allocates tensor memory and issues tcgen05.mma (one thread)
+// Shared memory holds a ring of stages (A tile(s) + B tile); mbarriers carry
+// full/empty hand-offs between producers and the MMA thread and
+// full/empty hand-offs of the accumulator between the MMA thread and the
+// epilogue.  Every wait is bounded: on expiry the CTA records
+// MOE_ERR_TIMEOUT in the device error word, every role leaves its loop, the
+// MMA thread drains its outstanding tensor-core work and tensor memory is
+// freed before the kernel returns.
+//
+// Tiles: M = 128 weight rows, N = up to 256 columns (tokens) of one group, K
+// stepped 64 at a time (four K=16 MMAs per step).  A gate/up pair shares the
+// B tile and uses two accumulators (columns 0-255 and 256-511).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kEpiWarps = 4;
+constexpr int kProdWarps = 8;
+constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 12
+constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 416
+constexpr int kProd = kProdWarps * 32;             // 256 producer threads
+constexpr int BM = 128, BK = 64, BN = 256;
+constexpr int kATile = BM * BK * 2;  // 16 KB
+constexpr int kBTile = BN * BK * 2;  // 32 KB
+constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
+
+struct alignas(8) GemmCtl {
+  uint64_t full[4], empty[4], acc_full, acc_empty, drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_groups;
+  int total_tiles;
+  int tile_prefix[257];  // tiles before group g
+  int col_off[257];      // first column of group g
+};
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false when this CTA is aborting (timeout here or elsewhere).
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, GemmCtl &ctl, int *err) {
+  if (mbar_try(b, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try(b, parity)) {
+    if (*((volatile int *)&ctl.abort)) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *((volatile int *)&ctl.abort) = 1;
+      set_error(err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+// K-major operand tile, 128-byte rows, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;               // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024u >> 4) << 32;     // stride byte offset
+  d |= (uint64_t)1u << 46;               // descriptor version
+  d |= (uint64_t)2u << 61;               // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, K-major A and B, M = 128.
+__device__ __forceinline__ uint32_t instr_desc(int n, int bf16) {
+  return (1u << 4) | ((uint32_t)bf16 << 7) | ((uint32_t)bf16 << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void mma_commit(uint64_t *b) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(b))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ldg16(const uint8_t *p) { return *reinterpret_cast<const uint16_t *>(p); }
+__device__ __forceinline__ uint32_t ldg32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+__device__ __forceinline__ void sts128(uint8_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+
+// 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint8_t *swz(uint8_t *tile, int row, int chunk) {
+  return tile + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 bits2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// ---------------------------------------------------------------- tile map
+
+struct Tile {
+  int g, m0, n0, nt, col0;
+};
+
+__device__ __forceinline__ Tile tile_at(const GemmCtl &ctl, int t, int m_tiles) {
+  int lo = 0, hi = ctl.n_groups - 1;
+  while (lo < hi) {  // last group with prefix <= t
+    const int mid = (lo + hi + 1) >> 1;
+    if (ctl.tile_prefix[mid] <= t)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  Tile r;
+  r.g = lo;
+  const int local = t - ctl.tile_prefix[lo];
+  const int n = ctl.col_off[lo + 1] - ctl.col_off[lo];
+  const int ntl = (n + BN - 1) / BN;
+  const int mt = local / ntl, nti = local - mt * ntl;
+  r.m0 = mt * BM;
+  r.n0 = nti * BN;
+  r.nt = min(BN, n - r.n0);
+  r.col0 = ctl.col_off[lo] + r.n0;
+  return r;
+}
+
+// ---------------------------------------------------------------- producers
+
+// IQ2_XXS: 32 elements (one group) of row `rowp` -> f16 into chunks 4*item..4*item+3.
+__device__ __forceinline__ void deq_iq2(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item,
+                                        const uint8_t *gridh, const uint8_t *signm) {
+  const int blk = kel >> 8, gib = (kel >> 5) & 7;
+  const uint8_t *bp = rowp + (size_t)blk * 66;
+  const uint8_t *gp = bp + 2 + 8 * gib;
+  const uint32_t d16 = ldg16(bp);
+  const uint32_t idx4 = ldg16(gp) | (ldg16(gp + 2) << 16);
+  const uint32_t S = ldg16(gp + 4) | (ldg16(gp + 6) << 16);
+  const __half2 f2 = __half2half2(__int2half_rn(2 * (int)(S >> 28) + 1));
+  const __half2 d2 = __half2half2(__hmul(__ushort_as_half((unsigned short)d16), __float2half(0.125f)));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t ix = (idx4 >> (8 * j)) & 255u;
+    const uint32_t m7 = (S >> (7 * j)) & 127u;
+    const uint4 g = *reinterpret_cast<const uint4 *>(gridh + ix * 16u);
+    const uint4 sm = *reinterpret_cast<const uint4 *>(signm + m7 * 16u);
+    const uint32_t o0 = h2bits(__hmul2(__hmul2(bits2h(g.x ^ sm.x), f2), d2));
+    const uint32_t o1 = h2bits(__hmul2(__hmul2(bits2h(g.y ^ sm.y), f2), d2));
+    const uint32_t o2 = h2bits(__hmul2(__hmul2(bits2h(g.z ^ sm.z), f2), d2));
+    const uint32_t o3 = h2bits(__hmul2(__hmul2(bits2h(g.w ^ sm.w), f2), d2));
+    sts128(swz(tile, row, 4 * item + j), o0, o1, o2, o3);
+  }
+}
+
+__device__ __forceinline__ uint32_t bf16pair(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Q2_K: 32 elements of row `rowp` at K offset kel (64-aligned k step, half `item`).
+__device__ __forceinline__ void deq_q2k(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item) {
+  const int blk = kel >> 8, qq = (kel >> 6) & 3;
+  const uint8_t *bp = rowp + (size_t)blk * 84;
+  const int hf = qq >> 1, sh = 2 * (qq & 1) + item;
+  const uint32_t dd = ldg32(bp + 80);
+  const float d = __half2float(__ushort_as_half((unsigned short)(dd & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half((unsigned short)(dd >> 16)));
+  const int j0 = 8 * hf + 2 * sh;
+  const uint32_t scw = ldg16(bp + j0);  // scale bytes of sub-blocks j0, j0 + 1
+#pragma unroll
+  for (int sub = 0; sub < 2; ++sub) {
+    const uint32_t sb = (scw >> (8 * sub)) & 0xFFu;
+    const float dsc = d * (float)(sb & 15u);
+    const float mn = -dmin * (float)(sb >> 4);
+    const uint32_t V0 = bf16pair(mn, fmaf(dsc, 1.f, mn));
+    const uint32_t V1 = bf16pair(fmaf(dsc, 2.f, mn), fmaf(dsc, 3.f, mn));
+    uint32_t o[8];
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const uint32_t w = ldg32(bp + 16 + 32 * hf + 16 * sub + 4 * wi);
+      const uint32_t q = (w >> (2 * sh)) & 0x03030303u;
+      const uint32_t t = q * 0x22u + 0x10101010u;
+      o[2 * wi] = __byte_perm(V0, V1, t & 0xFFFFu);
+      o[2 * wi + 1] = __byte_perm(V0, V1, t >> 16);
+    }
+    sts128(swz(tile, row, 4 * item + 2 * sub), o[0], o[1], o[2], o[3]);
+    sts128(swz(tile, row, 4 * item + 2 * sub + 1), o[4], o[5], o[6], o[7]);
+  }
+}
+
+// Q8_0: one 32-element block (index kel/32) of row `rowp`.
+__device__ __forceinline__ void deq_q80(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item, int bf16) {
+  const uint8_t *bp = rowp + (size_t)(kel >> 5) * 34;
+  const uint32_t d16 = ldg16(bp);
+  const uint8_t *qp = bp + 2;
+  uint32_t w[8];
+  if ((reinterpret_cast<uintptr_t>(qp) & 3u) == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = ldg32(qp + 4 * i);
+  } else {
+    const uint8_t *base = qp - 2;  // 4-byte aligned; the last word is read as 16 bits to stay in the block
+    uint32_t u[9];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = ldg32(base + 4 * i);
+    u[8] = ldg16(base + 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = __byte_perm(u[i], u[i + 1], 0x5432);
+  }
+  uint32_t o[16];
+  const __half dh = __ushort_as_half((unsigned short)d16);
+  const __half2 bias = __half2half2(__float2half(1152.f));
+  if (!bf16) {
+    const __half2 d2 = __half2half2(dh);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t x = w[i] ^ 0x80808080u;
+      const __half2 lo = __hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x5140)), bias);
+      const __half2 hi = __hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x7362)), bias);
+      o[2 * i] = h2bits(__hmul2(lo, d2));
+      o[2 * i + 1] = h2bits(__hmul2(hi, d2));
+    }
+  } else {
+    const float d = __half2float(dh);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t x = w[i] ^ 0x80808080u;
+      const float2 lo = __half22float2(__hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x5140)), bias));
+      const float2 hi = __half22float2(__hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x7362)), bias));
+      o[2 * i] = bf16pair(lo.x * d, lo.y * d);
+      o[2 * i + 1] = bf16pair(hi.x * d, hi.y * d);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sts128(swz(tile, row, 4 * item + c), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+}
+
+// ---------------------------------------------------------------- kernel
+
+template <bool PAIRED>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
+  constexpr int NA = PAIRED ? 2 : 1;
+  constexpr int S = PAIRED ? 3 : 4;
+  constexpr int STAGE = NA * kATile + kBTile;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *stages = smem;
+  uint8_t *gridh = stages + S * STAGE;  // 256 x 16 B: codebook as f16
+  uint8_t *signm = gridh + 4096;        // 128 x 16 B: f16 sign masks per 7-bit mask
+  GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + 2048);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m_tiles = a.M / BM;
+  const int ksteps = a.K / BK;
+
+  // ---- set-up
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ctl.full[s], kProd);
+      mbar_init(&ctl.empty[s], 1);
+    }
+    mbar_init(&ctl.acc_full, 1);
+    mbar_init(&ctl.acc_empty, kEpiWarps * 32);
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (tid == 32) {  // group table
+    const int G = a.offsets ? a.n_groups : 1;
+    int pre = 0;
+    for (int g = 0; g < G; ++g) {
+      const int c0 = a.offsets ? a.offsets[g] : 0;
+      const int c1 = a.offsets ? a.offsets[g + 1] : a.cols;
+      ctl.col_off[g] = c0;
+      ctl.tile_prefix[g] = pre;
+      pre += m_tiles * ((c1 - c0 + BN - 1) / BN);
+    }
+    ctl.col_off[G] = a.offsets ? a.offsets[G] : a.cols;
+    ctl.tile_prefix[G] = pre;
+    ctl.n_groups = G;
+    ctl.total_tiles = pre;
+  }
+  if (a.fmt == kFmtIQ2) {
+    for (int i = tid; i < 256 * 8; i += blockDim.x) {  // codebook -> f16
+      const int ix = i >> 3, l = i & 7;
+      reinterpret_cast<__half *>(gridh)[ix * 8 + l] = __int2half_rn(a.grid[ix * 8 + l]);
+    }
+    for (int m7 = tid; m7 < 128; m7 += blockDim.x) {
+      const uint32_t m8 = (uint32_t)m7 | ((uint32_t)(__popc(m7) & 1) << 7);
+      uint32_t *e = reinterpret_cast<uint32_t *>(signm + m7 * 16);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        e[p] = (((m8 >> (2 * p)) & 1u) << 15) | (((m8 >> (2 * p + 1)) & 1u) << 31);
+    }
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&ctl.tmem_base)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+  const int total = ctl.total_tiles;
+
+  if (warp >= kEpiWarps && warp < kMmaWarp) {
+    // =================================================== producers
+    const int p = tid - kEpiWarps * 32;
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const Tile tl = tile_at(ctl, t, m_tiles);
+      // B rows this thread copies: rows (p >> 3) + 32 i, chunk p & 7
+      const int ch = p & 7;
+      const uint16_t *brow[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = (p >> 3) + 32 * i;
+        brow[i] = nullptr;
+        if (r < tl.nt) {
+          const int c = tl.col0 + r;
+          const int br = a.b_perm ? a.b_perm[c] / a.b_div : c;
+          brow[i] = a.b_base + (size_t)br * a.b_ld + ch * 8;
+        }
+      }
+      // A items: row p/2, 32-element half p%2 of the 64-element K step
+      const uint8_t *arow0, *arow1 = nullptr;
+      const int row = p >> 1, item = p & 1;
+      arow0 = a.A0 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
+      if (PAIRED) arow1 = a.A1 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
+      bool ok = true;
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(&ctl.empty[st], ph ^ 1u, ctl, a.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t *A0s = stages + st * STAGE;
+        uint8_t *Bs = A0s + NA * kATile;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 32 * i, ch), brow[i] + ks * BK);
+        }
+        cp_async_commit();
+        const int kel = ks * BK + 32 * item;
+        if (a.fmt == kFmtIQ2) {
+          deq_iq2(arow0, kel, A0s, row, item, gridh, signm);
+          if (PAIRED) deq_iq2(arow1, kel, A0s + kATile, row, item, gridh, signm);
+        } else if (a.fmt == kFmtQ2K) {
+          deq_q2k(arow0, ks * BK, A0s, row, item);
+        } else {
+          deq_q80(arow0, kel, A0s, row, item, a.bf16);
+          if (PAIRED) deq_q80(arow1, kel, A0s + kATile, row, item, a.bf16);
+        }
+        cp_async_wait<0>();
+        fence_proxy_async();
+        mbar_arrive(&ctl.full[st]);
+      }
+      if (!ok) break;
+    }
+    cp_async_wait<0>();
+  } else if (warp == kMmaWarp) {
+    // =================================================== MMA issue
+    uint32_t it = 0, tc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
+      const Tile tl = tile_at(ctl, t, m_tiles);
+      const int nmma = (tl.nt + 15) & ~15;
+      const uint32_t idesc = instr_desc(nmma, a.bf16);
+      if (!mbar_wait(&ctl.acc_empty, (tc & 1u) ^ 1u, ctl, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(&ctl.full[st], ph, ctl, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(stages + st * STAGE);
+          const uint32_t b0 = a0 + NA * kATile;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            mma_f16(tmem, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+            if (PAIRED) mma_f16(tmem + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+          }
+          mma_commit(&ctl.empty[st]);
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) mma_commit(&ctl.acc_full);
+      __syncwarp();
+    }
+    // drain: every MMA this thread issued has finished before tensor memory is freed
+    if (lane == 0) {
+      mma_commit(&ctl.drain);
+      const long long t0 = clock64();
+      while (!mbar_try(&ctl.drain, 0u)) {
+        if (clock64() - t0 > kWaitCycles) {
+          set_error(a.err, kErrTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // =================================================== epilogue
+    const int row = tid;  // TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const Tile tl = tile_at(ctl, t, m_tiles);
+      if (!mbar_wait(&ctl.acc_full, tc & 1u, ctl, a.err)) break;
+      tc_fence_after();
+      const int m = tl.m0 + row;
+      for (int c0 = 0; c0 < tl.nt; c0 += 16) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(lane_base + c0, r0);
+        if (PAIRED) tmem_ld16(lane_base + BN + c0, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + j;
+          if (n >= tl.nt) break;
+          const int c = tl.col0 + n;
+          const float dv = __uint_as_float(r0[j]);
+          if (a.epi == kEpiSwiGLU) {
+            const float u = __uint_as_float(PAIRED ? r1[j] : 0u);
+            const float h = silu(dv) * u;
+            uint16_t hb;
+            if (a.h_bf16) {
+              __nv_bfloat16 v = __float2bfloat16_rn(h);
+              hb = *reinterpret_cast<uint16_t *>(&v);
+            } else {
+              __half v = __float2half_rn(h);
+              hb = *reinterpret_cast<uint16_t *>(&v);
+            }
+            a.h_out[(size_t)c * a.h_ld + m] = hb;
+          } else if (a.epi == kEpiScatterAdd) {
+            const int pr = a.perm[c];
+            atomicAdd(a.y + (size_t)(pr / a.k) * a.y_ld + m, a.w[pr] * dv);
+          } else {
+            float v = dv;
+            if (a.res) v += a.res[(size_t)c * a.y_ld + m];
+            a.y[(size_t)c * a.y_ld + m] = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl.acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512));
+  }
+}
+
+}  // namespace
+
+size_t grouped_gemm_smem(int paired) {
+  const int na = paired ? 2 : 1;
+  const int s = paired ? 3 : 4;
+  return 1024 + (size_t)s * (na * kATile + kBTile) + 4096 + 2048 + sizeof(GemmCtl);
+}
+
+cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
+  static bool configured[2] = {false, false};
+  const bool paired = a.A1 != nullptr;
+  const size_t smem = grouped_gemm_smem(paired);
+  if (paired) {
+    if (!configured[1]) {
+      cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      configured[1] = true;
+    }
+    k_grouped_gemm<true><<<num_sms, kGemmThreads, smem, s>>>(a);
+  } else {
+    if (!configured[0]) {
+      cudaError_t e =
+          cudaFuncSetAttribute(k_grouped_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      configured[0] = true;
+    }
+    k_grouped_gemm<false><<<num_sms, kGemmThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

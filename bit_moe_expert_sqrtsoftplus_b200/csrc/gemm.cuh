@@ -1,0 +1,53 @@
+// gemm.cuh -- grouped tensor-core GEMM of the large-T path.
+//
+// D[m][n] = sum_k A[m][k] * B[n][k] for column groups (one per expert, or one
+// for the shared expert), A = packed weight rows dequantised on the fly, B =
+// 16-bit activation rows gathered per column.  Epilogues: SwiGLU of a paired
+// gate/up product into 16-bit h rows; routing-weighted scatter-add into y;
+// plain store into y.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+enum GemmFmt { kFmtIQ2 = 0, kFmtQ2K = 1, kFmtQ80 = 2 };
+enum GemmEpi { kEpiSwiGLU = 0, kEpiScatterAdd = 1, kEpiStore = 2 };
+
+struct GemmArgs {
+  int fmt;    // GemmFmt of the A operand
+  int bf16;   // operand type: 0 = f16, 1 = bf16
+  int epi;    // GemmEpi
+  int M, K;   // weight rows / reduction length (multiples of 128 / 256)
+  int n_groups;
+  const int32_t *offsets;  // [n_groups+1] column ranges; nullptr: one group of `cols` columns
+  int cols;
+  const uint8_t *A0, *A1;  // packed weights of group 0 (A1: the up matrix of a gate/up pair)
+  size_t a_group_stride;   // bytes between consecutive groups' matrices
+  size_t a_row_bytes;
+  const uint8_t *grid;     // IQ2_XXS codebook [256][8]
+  // B: row of column c (global column index, offsets[g] + n) is
+  //    b_base + b_ld * (b_perm ? b_perm[c] / b_div : c)
+  const uint16_t *b_base;
+  int b_ld;
+  const int32_t *b_perm;
+  int b_div;
+  // epilogues
+  uint16_t *h_out;   // SwiGLU: h_out[c * h_ld + m] (16-bit, same type as `h_bf16`)
+  int h_ld;
+  int h_bf16;
+  float *y;          // ScatterAdd: y[(perm[c]/k) * y_ld + m] += w[perm[c]] * D
+  int y_ld;          // Store: y[c * y_ld + m] = D (+ res[c * y_ld + m])
+  const float *res;
+  const float *w;
+  const int32_t *perm;
+  int k;
+  int *err;
+};
+
+cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms);
+size_t grouped_gemm_smem(int paired);
+
+}  // namespace moe

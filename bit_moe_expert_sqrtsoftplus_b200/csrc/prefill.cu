@@ -13,7 +13,10 @@
 #include <float.h>
 #include <math.h>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
+#include "gemm.cuh"
 #include "prefill.cuh"
 
 namespace moe {
@@ -391,9 +394,11 @@ __global__ void k_perm_scatter(const int32_t *idx, int n, const int32_t *offsets
 
 }  // namespace
 
+size_t prefill_big_bytes(const LayerDims &d, int T);
+
 size_t prefill_scratch_bytes(const LayerDims &d, int T) {
   PrefillArgs p = prefill_args(d, LayerWeights{}, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
-  return reinterpret_cast<size_t>(p.s.big) + 256;
+  return reinterpret_cast<size_t>(p.s.big) + prefill_big_bytes(d, T) + 256;
 }
 
 PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, const float *x,
@@ -406,6 +411,8 @@ PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, cons
   p.token_ids = token_ids;
   p.y = y;
   p.row_norms = row_norms;
+  p.ev_begin = nullptr;
+  p.ev_end = nullptr;
   p.err = err;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -463,11 +470,162 @@ cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStre
   return cudaGetLastError();
 }
 
+namespace {
+
+// x (optionally RMS-normalised) -> f16 [T][H], the B operand of the gate/up GEMMs.
+__global__ void k_prep_x16(const float *x, int T, int H, int flags, float eps, __half *out) {
+  const int t = blockIdx.x;
+  const float *xt = x + (size_t)t * H;
+  float inv = 1.f;
+  if (flags & MOE_FLAG_PRENORM_RESIDUAL) {
+    double ss = 0.0;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) ss += (double)xt[j] * (double)xt[j];
+    ss = warp_sum_d(ss);
+    __shared__ double red[32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    double tot = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    inv = (float)(1.0 / sqrt(tot / (double)H + (double)eps));
+  }
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4 *>(xt + j);
+    __half2 a = __floats2half2_rn(v.x * inv, v.y * inv);
+    __half2 b = __floats2half2_rn(v.z * inv, v.w * inv);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t *>(&a);
+    o.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(out + (size_t)t * H + j) = o;
+  }
+}
+
+struct BigScratch {
+  __half *x16;      // [T][H]
+  uint16_t *hperm;  // [T*k][I] bf16, rows in permuted order
+  uint16_t *hs;     // [T][Is] bf16
+  size_t bytes;
+};
+
+BigScratch carve_big(const LayerDims &d, int T, void *base) {
+  BigScratch b;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    off = align_up(off, 256);
+    uint8_t *q = static_cast<uint8_t *>(base) + off;
+    off += n;
+    return q;
+  };
+  b.x16 = reinterpret_cast<__half *>(take(2 * (size_t)T * d.H));
+  b.hperm = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.k * d.I));
+  b.hs = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.Is));
+  b.bytes = off;
+  return b;
+}
+
+}  // namespace
+
+size_t prefill_big_bytes(const LayerDims &d, int T) { return carve_big(d, T, nullptr).bytes; }
+
 cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
-  (void)p;
-  (void)s;
-  (void)num_sms;
-  return cudaErrorNotSupported;
+  const LayerDims &d = p.d;
+  const int T = p.T;
+  cudaError_t e = prefill_route(p, p.s.idx, p.s.w, s);
+  if (e != cudaSuccess) return e;
+  e = permute(p.s.idx, T, d.k, d.E, p.s.offsets, p.s.perm, s);
+  if (e != cudaSuccess) return e;
+  BigScratch b = carve_big(d, T, p.s.big);
+  k_prep_x16<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, b.x16);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  const size_t rbIQ = (size_t)(d.H / 256) * 66;
+  const size_t rbQ2 = (size_t)(d.I / 256) * 84;
+  const size_t rbQ8h = (size_t)(d.H / 32) * 34;
+  const size_t rbQ8s = (size_t)(d.Is / 32) * 34;
+
+  // routed gate/up: IQ2_XXS x f16 activations, SwiGLU -> h (bf16) in permuted order
+  GemmArgs g{};
+  g.fmt = kFmtIQ2;
+  g.bf16 = 0;
+  g.epi = kEpiSwiGLU;
+  g.M = d.I;
+  g.K = d.H;
+  g.n_groups = d.E;
+  g.offsets = p.s.offsets;
+  g.A0 = p.wt.gate;
+  g.A1 = p.wt.up;
+  g.a_group_stride = (size_t)d.I * rbIQ;
+  g.a_row_bytes = rbIQ;
+  g.grid = p.wt.grid;
+  g.b_base = reinterpret_cast<const uint16_t *>(b.x16);
+  g.b_ld = d.H;
+  g.b_perm = p.s.perm;
+  g.b_div = d.k;
+  g.h_out = b.hperm;
+  g.h_ld = d.I;
+  g.h_bf16 = 1;
+  g.err = p.err;
+  if (p.ev_begin) cudaEventRecord(p.ev_begin, s);
+  if ((e = grouped_gemm(g, s, num_sms)) != cudaSuccess) return e;
+  if (p.ev_end) cudaEventRecord(p.ev_end, s);
+
+  // shared gate/up: Q8_0 x f16 activations over all tokens, SwiGLU -> hs (bf16)
+  GemmArgs sg = g;
+  sg.fmt = kFmtQ80;
+  sg.M = d.Is;
+  sg.n_groups = 1;
+  sg.offsets = nullptr;
+  sg.cols = T;
+  sg.A0 = p.wt.sh_gate;
+  sg.A1 = p.wt.sh_up;
+  sg.a_group_stride = 0;
+  sg.a_row_bytes = rbQ8h;
+  sg.b_perm = nullptr;
+  sg.b_div = 1;
+  sg.h_out = b.hs;
+  sg.h_ld = d.Is;
+  if ((e = grouped_gemm(sg, s, num_sms)) != cudaSuccess) return e;
+
+  // shared down: Q8_0 x bf16 hs -> y (plus the residual input when pre-norm)
+  GemmArgs sd{};
+  sd.fmt = kFmtQ80;
+  sd.bf16 = 1;
+  sd.epi = kEpiStore;
+  sd.M = d.H;
+  sd.K = d.Is;
+  sd.n_groups = 1;
+  sd.offsets = nullptr;
+  sd.cols = T;
+  sd.A0 = p.wt.sh_down;
+  sd.A1 = nullptr;
+  sd.a_row_bytes = rbQ8s;
+  sd.b_base = b.hs;
+  sd.b_ld = d.Is;
+  sd.b_div = 1;
+  sd.y = p.y;
+  sd.y_ld = d.H;
+  sd.res = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr;
+  sd.err = p.err;
+  if ((e = grouped_gemm(sd, s, num_sms)) != cudaSuccess) return e;
+
+  // routed down: Q2_K x bf16 h, y[token] += w * (W_down h)
+  GemmArgs rd = sd;
+  rd.fmt = kFmtQ2K;
+  rd.epi = kEpiScatterAdd;
+  rd.M = d.H;
+  rd.K = d.I;
+  rd.n_groups = d.E;
+  rd.offsets = p.s.offsets;
+  rd.A0 = p.wt.down;
+  rd.a_group_stride = (size_t)d.H * rbQ2;
+  rd.a_row_bytes = rbQ2;
+  rd.b_base = b.hperm;
+  rd.b_ld = d.I;
+  rd.b_perm = nullptr;
+  rd.res = nullptr;
+  rd.w = p.s.w;
+  rd.perm = p.s.perm;
+  rd.k = d.k;
+  return grouped_gemm(rd, s, num_sms);
 }
 
 cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, cudaStream_t s) {

@@ -32,6 +32,7 @@ struct PrefillArgs {
   PrefillScratch s;
   const float *row_norms;  // [E] 2-norms of the router rows
   int *err;
+  cudaEvent_t ev_begin, ev_end;  // recorded around the routed gate/up GEMM when set
 };
 
 size_t prefill_scratch_bytes(const LayerDims &d, int T);

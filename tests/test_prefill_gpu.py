@@ -1,0 +1,89 @@
+"""Parity of the large-T path (certified router, permutation, tcgen05 grouped
+GEMMs with f16/bf16 operands) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import harness
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from bit_moe_expert_sqrtsoftplus_b200 import build
+    build.build()
+    import bit_moe_expert_sqrtsoftplus_b200 as m
+    return m
+
+
+def _forward(moe, s, seed, layer, T, mode=0, flags=0):
+    router = mode == moe.MOE_ROUTE_ROUTER
+    W = harness.device_layer(s, seed, layer, router=router)
+    L = moe.Layer(harness.config_for(s, mode, flags), W, max_tokens=T)
+    x_np = synth.activations(seed, T, s.hidden, stream=layer)
+    tok_np = synth.token_ids(seed, T, s.vocab, stream=layer)
+    x = torch.from_numpy(x_np).cuda()
+    tok = torch.from_numpy(tok_np).cuda()
+    y = L.forward(x, tok)
+    torch.cuda.synchronize()
+    L.poll()
+    return x_np, tok_np, y.cpu().numpy(), L
+
+
+def _oracle_rows(s, seed, layer, x_np, tok_np, rows, router=True, prenorm=False):
+    sub = synth.LayerShape(s.hidden, s.inter, s.shared_inter, s.n_experts, s.top_k, len(rows), vocab=s.vocab,
+                           skew=s.skew)
+    _, _, yref, _ = harness.oracle_layer(sub, seed, layer, x_np[rows], tok_np[rows], router=router,
+                                         prenorm=prenorm)
+    return yref
+
+
+@pytest.mark.parametrize("T", [9, 64, 300])
+def test_tiny_shapes_large_T(moe, T):
+    s = synth.workload("tiny", tokens=T)
+    x, tok, y, _ = _forward(moe, s, 0, 0, T)
+    yref = _oracle_rows(s, 0, 0, x, tok, np.arange(T))
+    rel, mx = harness.errors(y, yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def test_tiny_hash_prenorm_large_T(moe):
+    s = synth.workload("tiny", tokens=100)
+    x, tok, y, _ = _forward(moe, s, 2, 1, 100, mode=moe.MOE_ROUTE_HASH, flags=moe.MOE_FLAG_PRENORM_RESIDUAL)
+    yref = _oracle_rows(s, 2, 1, x, tok, np.arange(100), router=False, prenorm=True)
+    rel, mx = harness.errors(y, yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def test_decode32_full_shape(moe):
+    s = synth.workload("decode_t32")
+    x, tok, y, _ = _forward(moe, s, 1, 2, 32)
+    rows = np.arange(0, 32, 4)
+    yref = _oracle_rows(s, 1, 2, x, tok, rows)
+    rel, mx = harness.errors(y[rows], yref)
+    print(f"decode_t32 rel_l2={rel:.3e} max_abs_frac={mx:.3e}")
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def test_prefill_4096_sampled_tokens(moe):
+    s = synth.workload("prefill_t4096")
+    x, tok, y, L = _forward(moe, s, 0, 0, 4096)
+    # sample: spread tokens plus tokens of the most and least loaded experts
+    idx, _ = L.route(torch.from_numpy(x).cuda())
+    idx = idx.cpu().numpy()
+    counts = np.bincount(idx.ravel(), minlength=s.n_experts)
+    busiest, quietest = int(counts.argmax()), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    rows = sorted(set([0, 1, 777, 2048, 4095] + list(np.nonzero((idx == busiest).any(1))[0][:3]) +
+                      list(np.nonzero((idx == quietest).any(1))[0][:2])))
+    yref = _oracle_rows(s, 0, 0, x, tok, np.array(rows))
+    rel, mx = harness.errors(y[rows], yref)
+    print(f"prefill_t4096 rows={rows} rel_l2={rel:.3e} max_abs_frac={mx:.3e} "
+          f"tokens/expert min {counts.min()} max {counts.max()}")
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+    assert np.all(np.isfinite(y))
