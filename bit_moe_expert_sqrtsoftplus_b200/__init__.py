@@ -30,7 +30,7 @@ MOE_ROUTE_HASH = 1
 MOE_FLAG_PRENORM_RESIDUAL = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
-            "moe_last_error", "moe_set_timing_events", "moe_destroy")
+            "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_destroy")
 
 
 class moe_config(ctypes.Structure):
@@ -69,6 +69,8 @@ def lib():
                                ctypes.POINTER(vp)]
         L.moe_route.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.moe_ffn_forward.argtypes = [vp, vp, vp, i32, vp, vp, sz, vp]
+        L.moe_ffn_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp]
+        L.moe_ffn_forward_noalloc.restype = i32
         L.moe_poll_device_error.argtypes = [vp, vp]
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_set_timing_events.argtypes = [vp, vp, vp]
@@ -133,6 +135,11 @@ def moe_route(handle, x, token_ids, T, idx, w, expert_offsets=None, perm=None, s
 def moe_ffn_forward(handle, x, token_ids, T, y, scratch, stream=None):
     _check(lib().moe_ffn_forward(handle, _ptr(x), _ptr(token_ids), T, _ptr(y), _ptr(scratch),
                                  0 if scratch is None else scratch.numel() * scratch.element_size(), _stream(stream)))
+
+
+def moe_ffn_forward_noalloc(handle, x, token_ids, T, y, stream=None):
+    """Forward without a scratch buffer (small T only; see include/moe.h)."""
+    _check(lib().moe_ffn_forward_noalloc(handle, _ptr(x), _ptr(token_ids), T, _ptr(y), _stream(stream)))
 
 
 def moe_poll_device_error(handle, stream=None):

@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -264,6 +265,74 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
     e = moe::prefill_forward(p, s, h->num_sms);
   }
   if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward launch");
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation forward
+//
+// Scratch for moe_ffn_forward_noalloc: one buffer per device that loads this
+// library, held until the process exits.  Host code must not take the
+// array's address directly (its name stands for a host-side shadow); the
+// device address comes from cudaGetSymbolAddress, looked up once per device
+// with that device current and cached below.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 128;
+void *g_static_scratch_addr[kMaxDevices] = {};
+std::mutex g_static_scratch_mutex;
+
+moe_status static_scratch_for(int dev, void **out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_addr[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
+                                   moe_stream_t stream) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  if (T == 0) return MOE_OK;
+  if (T > moe::kDecodeMaxT)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_forward_noalloc handles at most %d tokens per call (got %d)",
+                moe::kDecodeMaxT, T);
+  const size_t need = moe::decode_scratch_bytes(h->d, T);
+  if (need > kStaticScratchBytes)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL,
+                "this layer needs %zu bytes of scratch for T=%d; the built-in buffer holds %zu bytes", need, T,
+                kStaticScratchBytes);
+  if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x and y must not be NULL");
+  if (!aligned16(x) || !aligned16(y)) return fail(MOE_ERR_MISALIGNED, "x and y must be 16-byte aligned");
+  if (h->d.mode == MOE_ROUTE_HASH && !token_ids) return fail(MOE_ERR_INVALID_ARG, "hash mode needs token_ids");
+  if (y == x && !(h->d.flags & MOE_FLAG_PRENORM_RESIDUAL))
+    return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != h->device)
+    return fail(MOE_ERR_INVALID_ARG, "the current device (%d) is not the handle's device (%d)", dev, h->device);
+  void *scratch = nullptr;
+  moe_status st = static_scratch_for(dev, &scratch);
+  if (st != MOE_OK) return st;
+  moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
+  e = moe::decode_forward(a, reinterpret_cast<cudaStream_t>(stream), h->num_sms);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward_noalloc launch");
   g_last_error.clear();
   return MOE_OK;
 }

@@ -134,6 +134,38 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
 moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
                            void *scratch, size_t scratch_bytes, moe_stream_t stream);
 
+/*
+ * moe_ffn_forward for callers that cannot allocate device memory.  (This
+ * entry point has no counterpart in the source pages; it only changes where
+ * the per-call temporaries live.)
+ *
+ * Some callers of this layer are not allowed to call cudaMalloc or any other
+ * allocator: for example a plugin inside a serving engine or framework that
+ * owns every device allocation through its own memory pool, or a program that
+ * must keep a fixed device-memory plan once it has started.  Such a caller
+ * can still hand over its inputs and outputs, but has no scratch buffer to
+ * give.  This variant runs the same small-T kernels as moe_ffn_forward with
+ * their scratch in a buffer built into the library: a 16 MiB array in device
+ * global memory that every GPU loading the library holds until the process
+ * exits.  Nothing is allocated by the call (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *
+ * Limits: 1 <= T <= 8 tokens, and the layer's small-T scratch for T must fit
+ * in 16 MiB (the V4-Flash shapes need about 8 MiB at T = 8); larger requests
+ * return MOE_ERR_UNSUPPORTED_SHAPE or MOE_ERR_WORKSPACE_TOO_SMALL with a
+ * message.  T = 0 is a no-op.  The current device must be the handle's
+ * device.  The first call on a device looks up the buffer's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  Every call on a device shares the one
+ * buffer and leaves its contents behind; the kernels clear the counters they
+ * need at the start of each call.  Calls whose executions overlap on the GPU
+ * (different streams, or different handles on the same device) race on the
+ * buffer: order them on one stream or synchronise between them.
+ * Arguments and errors are as for moe_ffn_forward.
+ */
+moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
+                                   moe_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device error word:
  * MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED_SHAPE (codebook entry > 127)
  * or MOE_ERR_DEVICE_FAULT. */
