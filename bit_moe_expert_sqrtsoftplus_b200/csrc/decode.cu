@@ -1,20 +1,24 @@
 // decode.cu -- the layer for small token counts (T <= 8): three kernels.
 //
-//   k1_prep_router  x -> int8 limbs (optionally RMSNorm first) and fp64
-//                   router logits z = W_r x.
-//   k2_gateup       top-k routing (recomputed per CTA from z), then every
-//                   (expert, 16-row tile) of gate/up and every (16-row tile,
-//                   K quarter) of the shared expert as a warp-sized unit:
-//                   packed rows are staged into shared memory with cp.async,
-//                   decoded in registers into int8 A fragments and multiplied
-//                   with mma.sync m16n8k32 against the int8 limbs of x; the
-//                   SwiGLU is applied in the epilogue.  The warp that
-//                   finishes the last tile of a vector quantises it into
-//                   limbs for the down projection.
+//   k1_prep_router  x -> int8 limbs (optionally RMSNorm first); fp64 router
+//                   logits, scores s = sqrtsoftplus(z) and selection keys
+//                   s + bias, one block per pair of experts.
+//   k2_gateup       top-k routing from the keys (comparisons only, per CTA),
+//                   then every (expert, 16-row tile) of gate/up and every
+//                   (16-row tile, K quarter) of the shared expert as a
+//                   warp-sized unit: packed rows are staged into shared memory
+//                   with cp.async, decoded in registers into int8 A fragments
+//                   and multiplied with mma.sync m16n8k32 against the int8
+//                   limbs of x; the SwiGLU is applied in the epilogue.  The
+//                   warp that finishes the last tile of a vector quantises it
+//                   into limbs for the down projection.
 //   k3_down         every (16-row output tile, expert or shared K quarter)
 //                   unit: Q2_K / Q8_0 rows against the limbs of h, weighted
 //                   by the routing weight; the last unit of a tile sums the
 //                   parts in a fixed order (deterministic) into y.
+// k2 and k3 are launched as programmatic dependents: their set-up (tables,
+// shared memory) overlaps the previous kernel, and griddepcontrol.wait
+// guards every read of the previous kernel's results.
 //
 // Activations enter the tensor cores as three int8 limbs with one scale per
 // vector: x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254, s3 = s2/254, which keeps
@@ -31,23 +35,34 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads2 = 256;  // 8 warps in k2 / k3
-constexpr int kWarps2 = kThreads2 / kWarp;
-constexpr int kStageBytes = 16 * 544;  // one 16-row chunk of at most 544 bytes per row
+constexpr int kWarps2 = 16;  // warps per CTA in k2 / k3
+constexpr int kThreads2 = kWarps2 * kWarp;
+constexpr int kStage2 = 16 * 272;      // k2 chunk: 16 rows of <= 272 bytes
+constexpr int kStage3 = 16 * 336;      // k3 chunk: 16 rows of <= 336 bytes
 constexpr int kGpmBytes = 256 * 128;   // +/- codebook, 8 replicas
 constexpr int kSelBytes = 128 * 128;   // byte-permute selectors per sign mask, 16 replicas
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// sqrt(softplus(z)) in fp64, softplus computed as max(z,0) + log1p(exp(-|z|)).
+__device__ __forceinline__ double sqrtsoftplus(double z) { return sqrt(fmax(z, 0.0) + log1p(exp(-fabs(z)))); }
+
 // ------------------------------------------------------------------ k1
 
+constexpr int kRouterThreads = 256;
+
 template <int MAXT>
-__global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
+__global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
+  pdl_launch_dependents();
   const LayerDims &d = a.d;
   const int T = a.T;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ double red[4][2 * MAXT + MAXT];
-  __shared__ float redf[4];
+  constexpr int NW = kRouterThreads / 32;
+  __shared__ double red[NW][3 * MAXT];
+  __shared__ float redf[NW];
 
   if (blockIdx.x == 0) {
     const int V = T * d.k + T;
@@ -68,7 +83,7 @@ __global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
     double ss = 0.0;
     float amax = 0.f;
     for (int j = tid; j < d.H; j += blockDim.x) {
-      float v = xt[j];
+      const float v = xt[j];
       ss += (double)v * (double)v;
       amax = fmaxf(amax, fabsf(v));
     }
@@ -79,25 +94,28 @@ __global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
       redf[warp] = amax;
     }
     __syncthreads();
-    ss = red[0][0] + red[1][0] + red[2][0] + red[3][0];
-    amax = fmaxf(fmaxf(redf[0], redf[1]), fmaxf(redf[2], redf[3]));
+    ss = 0.0;
+    amax = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      ss += red[w][0];
+      amax = fmaxf(amax, redf[w]);
+    }
     float inv = 1.f;
     if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) {
-      double invd = 1.0 / sqrt(ss / (double)d.H + (double)d.eps);
-      inv = (float)invd;
-      amax = amax * inv;  // max of the normalised vector (positive scaling)
+      inv = (float)(1.0 / sqrt(ss / (double)d.H + (double)d.eps));
+      amax = amax * inv;
     }
     const float s1 = amax > 0.f ? amax / 127.f : 1.f;
     const float s2 = s1 / 254.f, s3 = s2 / 254.f;
     const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
     int8_t *q = a.s.xq + (size_t)t * 3 * d.H;
     for (int j = tid; j < d.H; j += blockDim.x) {
-      float v = xt[j] * inv;
-      float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
-      float e1 = fmaf(-q1, s1, v);
-      float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
-      float e2 = fmaf(-q2, s2, e1);
-      float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+      const float v = xt[j] * inv;
+      const float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
+      const float e1 = fmaf(-q1, s1, v);
+      const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+      const float e2 = fmaf(-q2, s2, e1);
+      const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
       q[j] = (int8_t)q1;
       q[d.H + j] = (int8_t)q2;
       q[2 * d.H + j] = (int8_t)q3;
@@ -113,40 +131,41 @@ __global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
   }
 
   if (d.mode != MOE_ROUTE_ROUTER) return;
-  // ---- router logits for experts e0, e0 + 1 in fp64
+  // ---- router logits, scores and keys for experts e0, e0 + 1 (fp64)
   const int e0 = 2 * ((int)blockIdx.x - T);
   if (e0 >= d.E) return;
   const bool two = e0 + 1 < d.E;
-  double acc[2][MAXT];
-  double ssq[MAXT];
+  double acc0[MAXT], acc1[MAXT], ssq[MAXT];
 #pragma unroll
-  for (int t = 0; t < MAXT; ++t) acc[0][t] = acc[1][t] = ssq[t] = 0.0;
-  const int jq = d.H / 4;
-  const int jb = warp * jq, je = jb + jq;
+  for (int t = 0; t < MAXT; ++t) acc0[t] = acc1[t] = ssq[t] = 0.0;
   const uint16_t *w0 = a.wt.Wr + (size_t)e0 * d.H;
   const uint16_t *w1 = a.wt.Wr + (size_t)(two ? e0 + 1 : e0) * d.H;
-  for (int j = jb + lane * 8; j < je; j += 256) {
-    uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
-    uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
-    double wa[8], wb[8];
-    const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
-    const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      wa[i] = (double)half_bits_to_float(p0[i]);
-      wb[i] = (double)half_bits_to_float(p1[i]);
-    }
+  // every thread covers 8 consecutive elements per pass; all loads of a pass are independent
+  for (int j = tid * 8; j < d.H; j += kRouterThreads * 8) {
+    const uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
+    const uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
+    float4 xv[MAXT][2];
 #pragma unroll
     for (int t = 0; t < MAXT; ++t) {
       if (t < T) {
         const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H + j);
-        float4 u0 = xp[0], u1 = xp[1];
-        double xv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        xv[t][0] = xp[0];
+        xv[t][1] = xp[1];
+      }
+    }
+    const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
+    const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t) {
+      if (t < T) {
+        const float xe[8] = {xv[t][0].x, xv[t][0].y, xv[t][0].z, xv[t][0].w,
+                             xv[t][1].x, xv[t][1].y, xv[t][1].z, xv[t][1].w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          acc[0][t] = fma(wa[i], xv[i], acc[0][t]);
-          acc[1][t] = fma(wb[i], xv[i], acc[1][t]);
-          ssq[t] = fma(xv[i], xv[i], ssq[t]);
+          const double xd = (double)xe[i];
+          acc0[t] = fma((double)half_bits_to_float(p0[i]), xd, acc0[t]);
+          acc1[t] = fma((double)half_bits_to_float(p1[i]), xd, acc1[t]);
+          ssq[t] = fma(xd, xd, ssq[t]);
         }
       }
     }
@@ -154,9 +173,9 @@ __global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
 #pragma unroll
   for (int t = 0; t < MAXT; ++t) {
     if (t < T) {
-      double v0 = warp_sum_d(acc[0][t]);
-      double v1 = warp_sum_d(acc[1][t]);
-      double v2 = warp_sum_d(ssq[t]);
+      const double v0 = warp_sum_d(acc0[t]);
+      const double v1 = warp_sum_d(acc1[t]);
+      const double v2 = warp_sum_d(ssq[t]);
       if (lane == 0) {
         red[warp][t] = v0;
         red[warp][MAXT + t] = v1;
@@ -165,30 +184,27 @@ __global__ void __launch_bounds__(128) k1_prep_router(DecodeArgs a) {
     }
   }
   __syncthreads();
-  if (tid < T) {
-    const int t = tid;
-    double z0 = red[0][t] + red[1][t] + red[2][t] + red[3][t];
-    double z1 = red[0][MAXT + t] + red[1][MAXT + t] + red[2][MAXT + t] + red[3][MAXT + t];
-    if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) {
-      double s = red[0][2 * MAXT + t] + red[1][2 * MAXT + t] + red[2][2 * MAXT + t] + red[3][2 * MAXT + t];
-      double inv = 1.0 / sqrt(s / (double)d.H + (double)d.eps);
-      z0 *= inv;
-      z1 *= inv;
+  if (tid < 2 * T) {
+    const int t = tid >> 1, which = tid & 1;
+    if (which == 1 && !two) return;
+    double z = 0.0, s2 = 0.0;
+    for (int w = 0; w < NW; ++w) {
+      z += red[w][which * MAXT + t];
+      s2 += red[w][2 * MAXT + t];
     }
-    a.s.z[(size_t)t * d.E + e0] = z0;
-    if (two) a.s.z[(size_t)t * d.E + e0 + 1] = z1;
+    if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) z *= 1.0 / sqrt(s2 / (double)d.H + (double)d.eps);
+    const int e = e0 + which;
+    const double sc = sqrtsoftplus(z);
+    a.s.sc[(size_t)t * d.E + e] = sc;
+    a.s.z[(size_t)t * d.E + e] = sc + (double)a.wt.bias[e];
   }
 }
 
 // ------------------------------------------------------------------ routing
 
-// sqrt(softplus(z)) in fp64, softplus computed as max(z,0) + log1p(exp(-|z|)).
-__device__ __forceinline__ double sqrtsoftplus(double z) {
-  return sqrt(fmax(z, 0.0) + log1p(exp(-fabs(z))));
-}
-
-// One warp: top-k of token t by s + bias (ties to the lower id), ids in
-// ascending order, weights scaling * s / sum(s).
+// One warp: top-k of token t by key (ties to the lower id), ids in ascending
+// order, weights scaling * s / sum(s).  Keys come from k1 (router mode) or the
+// token-id table (hash mode).
 __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, float *w_out) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31;
@@ -203,16 +219,17 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
 #pragma unroll
     for (int i = 0; i < kMaxK; ++i) sel[i] = i < k ? a.wt.tid2eid[(size_t)tid * k + i] : INT_MAX;
   } else {
-    const double *zt = a.s.z + (size_t)t * d.E;
+    const double *kt = a.s.z + (size_t)t * d.E;
     double key[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
-      key[i] = e < d.E ? sqrtsoftplus(zt[e]) + (double)a.wt.bias[e] : -DBL_MAX;
+      key[i] = e < d.E ? kt[e] : -DBL_MAX;
     }
     unsigned taken = 0;
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r) {
+      sel[r] = INT_MAX;
       if (r < k) {
         double bk = -INFINITY;
         int be = INT_MAX;
@@ -226,8 +243,8 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-          double ok = __shfl_xor_sync(0xffffffffu, bk, o);
-          int oe = __shfl_xor_sync(0xffffffffu, be, o);
+          const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
           if (ok > bk || (ok == bk && oe < be)) {
             bk = ok;
             be = oe;
@@ -235,35 +252,26 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
         sel[r] = be;
-      } else {
-        sel[r] = INT_MAX;
-      }
-    }
-  }
-  // ascending ids
-#pragma unroll
-  for (int i = 1; i < kMaxK; ++i) {
-#pragma unroll
-    for (int j = kMaxK - 1; j >= i; --j) {
-      if (sel[j - 1] > sel[j]) {
-        int tmp = sel[j - 1];
-        sel[j - 1] = sel[j];
-        sel[j] = tmp;
       }
     }
   }
   if (lane == 0) {
+    for (int i = 1; i < k; ++i)
+      for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
+        const int tmp = sel[j - 1];
+        sel[j - 1] = sel[j];
+        sel[j] = tmp;
+      }
     if (d.mode == MOE_ROUTE_HASH) {
       for (int i = 0; i < k; ++i) {
         idx_out[i] = sel[i];
         w_out[i] = d.scaling / (float)k;
       }
     } else {
-      const double *zt = a.s.z + (size_t)t * d.E;
-      double sv[kMaxK];
-      double tot = 0.0;
+      const double *st = a.s.sc + (size_t)t * d.E;
+      double sv[kMaxK], tot = 0.0;
       for (int i = 0; i < k; ++i) {
-        sv[i] = sqrtsoftplus(zt[sel[i]]);
+        sv[i] = st[sel[i]];
         tot += sv[i];
       }
       for (int i = 0; i < k; ++i) {
@@ -282,12 +290,12 @@ struct Jobs {
   int first[kDecodeMaxT * kMaxK];
   int cnt[kDecodeMaxT * kMaxK];
   int pair[kDecodeMaxT * kMaxK];  // sorted t*k + slot
+  int rank_e[kDecodeMaxT * kMaxK];
 };
 
 __device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
   const int np = T * k;
   const int tid = threadIdx.x;
-  __shared__ int rank_e[kDecodeMaxT * kMaxK];
   if (tid < np) {
     const int ei = idx_s[tid], ti = tid / k;
     int rank = 0;
@@ -296,14 +304,14 @@ __device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
       rank += (ej < ei) || (ej == ei && tj < ti);
     }
     J.pair[rank] = tid;
-    rank_e[rank] = ei;
+    J.rank_e[rank] = ei;
   }
   __syncthreads();
   if (tid == 0) {
     int n = 0;
     for (int r = 0; r < np; ++r) {
-      if (r == 0 || rank_e[r] != rank_e[r - 1]) {
-        J.e[n] = rank_e[r];
+      if (r == 0 || J.rank_e[r] != J.rank_e[r - 1]) {
+        J.e[n] = J.rank_e[r];
         J.first[n] = r;
         J.cnt[n] = 0;
         ++n;
@@ -317,27 +325,11 @@ __device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
 
 // ------------------------------------------------------------------ staging
 
-// Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS).
-__device__ __forceinline__ void stage_chunk(uint8_t *st, int RS, const uint8_t *g, size_t gstride, int bpr,
-                                            bool a16) {
-  const int lane = threadIdx.x & 31;
-  if (a16) {
-    const int n16 = bpr >> 4;
-    const int total = 16 * n16;
-    for (int i = lane; i < total; i += 32) {
-      const int row = i / n16, o = i - row * n16;
-      cp_async16(st + row * RS + o * 16, g + row * gstride + o * 16);
-    }
-  } else {
-    const int n2 = bpr >> 1;
-    const int total = 16 * n2;
-    for (int i = lane; i < total; i += 32) {
-      const int row = i / n2, o = i - row * n2;
-      *reinterpret_cast<uint16_t *>(st + row * RS + 2 * o) =
-          *reinterpret_cast<const uint16_t *>(g + row * gstride + 2 * o);
-    }
-  }
-  cp_async_commit();
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 struct Chunk {
@@ -346,58 +338,124 @@ struct Chunk {
   int bpr;           // bytes per row in the chunk
   int nb;            // blocks in the chunk
   int k0;            // first element (K index) of the chunk
-  bool a16;
+  int piece;         // copy granularity: 16, 8, 4 (cp.async) or 2 (plain loads)
 };
 
+__host__ __device__ __forceinline__ int piece_for(size_t gstride, size_t off, int bpr) {
+  const size_t m = gstride | off | (size_t)bpr;
+  return (m & 15) == 0 ? 16 : (m & 7) == 0 ? 8 : (m & 3) == 0 ? 4 : 2;
+}
+
 __device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
+
+// Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS).
+__device__ __forceinline__ void stage_chunk(uint8_t *st, const Chunk &c) {
+  const int lane = threadIdx.x & 31;
+  const int RS = stage_rs(c.bpr);
+  const int n = c.bpr / c.piece;
+  for (int row = 0; row < 16; ++row) {
+    const uint8_t *g = c.g + row * c.gstride;
+    uint8_t *s = st + row * RS;
+    for (int o = lane; o < n; o += 32) {
+      const int off = o * c.piece;
+      if (c.piece == 16)
+        cp_async16(s + off, g + off);
+      else if (c.piece == 8)
+        cp_async8(s + off, g + off);
+      else if (c.piece == 4)
+        cp_async4(s + off, g + off);
+      else
+        *reinterpret_cast<uint16_t *>(s + off) = *reinterpret_cast<const uint16_t *>(g + off);
+    }
+  }
+  cp_async_commit();
+}
+
+// Runs a list of chunks through the warp's two-stage ring; `compute(i, st)`
+// consumes chunk i from stage st.
+template <typename ChunkAt, typename Compute>
+__device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int n, ChunkAt chunk_at,
+                                           Compute compute) {
+  stage_chunk(stage0, chunk_at(0));
+  for (int i = 0; i < n; ++i) {
+    uint8_t *cur = (i & 1) ? stage1 : stage0;
+    uint8_t *nxt = (i & 1) ? stage0 : stage1;
+    if (i + 1 < n)
+      stage_chunk(nxt, chunk_at(i + 1));
+    else
+      cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    compute(i, cur);
+    __syncwarp();
+  }
+}
 
 // ------------------------------------------------------------------ decoders
 
 // IQ2_XXS group -> int8 A fragment halves for sub-vector c of one row.
-__device__ __forceinline__ void iq2_group(const uint8_t *grp, int c, const uint8_t *gpm_l, const uint8_t *sel_l,
-                                          uint32_t &lo, uint32_t &hi, int &f) {
+__device__ __forceinline__ void iq2_group(const uint8_t *grp, uint32_t S, int c, const uint8_t *gpm_l,
+                                          const uint8_t *sel_l, uint32_t &lo, uint32_t &hi) {
   const uint32_t ix = grp[c];
-  const uint32_t S = lds_u16(grp + 4) | (lds_u16(grp + 6) << 16);
   const uint32_t m7 = (S >> (7 * c)) & 127u;
-  f = 2 * (int)(S >> 28) + 1;
   const uint4 gv = *reinterpret_cast<const uint4 *>(gpm_l + ix * 128u);
   const uint2 sv = *reinterpret_cast<const uint2 *>(sel_l + m7 * 128u);
   lo = __byte_perm(gv.x, gv.y, sv.x);
   hi = __byte_perm(gv.z, gv.w, sv.y);
 }
 
+// The 32-bit word at grp+4 (S: sign masks and scale); grp is 2-byte aligned.
+__device__ __forceinline__ uint32_t iq2_sword(const uint8_t *grp) {
+  const uint8_t *p = grp + 4;
+  if ((reinterpret_cast<uintptr_t>(p) & 3u) == 0) return lds_u32(p);
+  return lds_u16(p) | (lds_u16(p + 2) << 16);
+}
+
+// B fragment (8 int8 of one limb column) from shared or global memory.
+__device__ __forceinline__ void load_b(const int8_t *col, int kel, uint32_t &b0, uint32_t &b1) {
+  if (col) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(col + kel);
+    b0 = v.x;
+    b1 = v.y;
+  } else {
+    b0 = b1 = 0u;
+  }
+}
+
 template <int MAXP>
-__device__ __forceinline__ void iq2_chunk(const uint8_t *st, int RS, const Chunk &ch, const uint8_t *gpm_l,
+__device__ __forceinline__ void iq2_chunk(const uint8_t *st, const Chunk &ch, const uint8_t *gpm_l,
                                           const uint8_t *sel_l, const int8_t *const (&bcol)[MAXP], int npairs,
                                           float (&F)[MAXP][4]) {
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const int RS = stage_rs(ch.bpr);
   const uint8_t *row0 = st + r * RS;
   const uint8_t *row1 = st + (r + 8) * RS;
   for (int b = 0; b < ch.nb; ++b) {
-    const float d0 = half_bits_to_float(lds_u16(row0 + 66 * b)) * 0.125f;
-    const float d1 = half_bits_to_float(lds_u16(row1 + 66 * b)) * 0.125f;
+    const uint8_t *b0p = row0 + 66 * b;
+    const uint8_t *b1p = row1 + 66 * b;
+    const float d0 = half_bits_to_float(lds_u16(b0p)) * 0.125f;
+    const float d1 = half_bits_to_float(lds_u16(b1p)) * 0.125f;
     int acc[MAXP][4];
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
+      const uint8_t *g0 = b0p + 2 + 8 * g;
+      const uint8_t *g1 = b1p + 2 + 8 * g;
+      const uint32_t S0 = iq2_sword(g0), S1 = iq2_sword(g1);
       uint32_t A[4];
-      int f0, f1;
-      iq2_group(row0 + 66 * b + 2 + 8 * g, c, gpm_l, sel_l, A[0], A[2], f0);
-      iq2_group(row1 + 66 * b + 2 + 8 * g, c, gpm_l, sel_l, A[1], A[3], f1);
+      iq2_group(g0, S0, c, gpm_l, sel_l, A[0], A[2]);
+      iq2_group(g1, S1, c, gpm_l, sel_l, A[1], A[3]);
+      const int f0 = 2 * (int)(S0 >> 28) + 1, f1 = 2 * (int)(S1 >> 28) + 1;
       const int kel = ch.k0 + 256 * b + 32 * g + 8 * c;
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         if (p < npairs) {
-          uint32_t b0 = 0, b1 = 0;
-          if (bcol[p]) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
-            b0 = v.x;
-            b1 = v.y;
-          }
+          uint32_t bb0, bb1;
+          load_b(bcol[p], kel, bb0, bb1);
           const int zero[4] = {0, 0, 0, 0};
           int cg[4];
-          mma_s8(cg, A, b0, b1, zero);
+          mma_s8(cg, A, bb0, bb1, zero);
           acc[p][0] += cg[0] * f0;
           acc[p][1] += cg[1] * f0;
           acc[p][2] += cg[2] * f1;
@@ -416,9 +474,9 @@ __device__ __forceinline__ void iq2_chunk(const uint8_t *st, int RS, const Chunk
 }
 
 // Q8_0: 34-byte blocks, the 8 int8 values of sub-range c (bytes 2+8c..9+8c).
-__device__ __forceinline__ void q80_vals(const uint8_t *blk, int b, int c, uint32_t &lo, uint32_t &hi) {
+__device__ __forceinline__ void q80_vals(const uint8_t *blk, int c, uint32_t &lo, uint32_t &hi) {
   const uint8_t *p = blk + 2 + 8 * c;
-  if (b & 1) {  // 34*b + 2 + 8c is a multiple of 4
+  if ((reinterpret_cast<uintptr_t>(p) & 3u) == 0) {
     lo = lds_u32(p);
     hi = lds_u32(p + 4);
   } else {  // two bytes past a multiple of 4
@@ -429,9 +487,10 @@ __device__ __forceinline__ void q80_vals(const uint8_t *blk, int b, int c, uint3
 }
 
 template <int MAXP>
-__device__ __forceinline__ void q80_chunk(const uint8_t *st, int RS, const Chunk &ch,
-                                          const int8_t *const (&bcol)[MAXP], int npairs, float (&F)[MAXP][4]) {
+__device__ __forceinline__ void q80_chunk(const uint8_t *st, const Chunk &ch, const int8_t *const (&bcol)[MAXP],
+                                          int npairs, float (&F)[MAXP][4]) {
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const int RS = stage_rs(ch.bpr);
   const uint8_t *row0 = st + r * RS;
   const uint8_t *row1 = st + (r + 8) * RS;
   for (int b = 0; b < ch.nb; ++b) {
@@ -440,21 +499,17 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int RS, const Chunk
     const float d0 = half_bits_to_float(lds_u16(p0));
     const float d1 = half_bits_to_float(lds_u16(p1));
     uint32_t A[4];
-    q80_vals(p0, b, c, A[0], A[2]);
-    q80_vals(p1, b, c, A[1], A[3]);
+    q80_vals(p0, c, A[0], A[2]);
+    q80_vals(p1, c, A[1], A[3]);
     const int kel = ch.k0 + 32 * b + 8 * c;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        uint32_t b0 = 0, b1 = 0;
-        if (bcol[p]) {
-          const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
-          b0 = v.x;
-          b1 = v.y;
-        }
+        uint32_t bb0, bb1;
+        load_b(bcol[p], kel, bb0, bb1);
         const int zero[4] = {0, 0, 0, 0};
         int cg[4];
-        mma_s8(cg, A, b0, b1, zero);
+        mma_s8(cg, A, bb0, bb1, zero);
         F[p][0] = fmaf(d0, (float)cg[0], F[p][0]);
         F[p][1] = fmaf(d0, (float)cg[1], F[p][1]);
         F[p][2] = fmaf(d1, (float)cg[2], F[p][2]);
@@ -468,10 +523,11 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int RS, const Chunk
 // the limbs of h.  Min term: A = m (per 16-element sub-block) against the
 // limbs of the 16-element sums of h.
 template <int MAXP>
-__device__ __forceinline__ void q2k_chunk(const uint8_t *st, int RS, const Chunk &ch,
-                                          const int8_t *const (&bcol)[MAXP], const int8_t *const (&xcol)[MAXP],
-                                          int npairs, float (&F)[MAXP][4], float (&G)[MAXP][4]) {
+__device__ __forceinline__ void q2k_chunk(const uint8_t *st, const Chunk &ch, const int8_t *const (&bcol)[MAXP],
+                                          const int8_t *const (&xcol)[MAXP], int npairs, float (&F)[MAXP][4],
+                                          float (&G)[MAXP][4]) {
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const int RS = stage_rs(ch.bpr);
   const uint8_t *row0 = st + r * RS;
   const uint8_t *row1 = st + (r + 8) * RS;
   for (int b = 0; b < ch.nb; ++b) {
@@ -504,13 +560,9 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int RS, const Chunk
 #pragma unroll
         for (int p = 0; p < MAXP; ++p) {
           if (p < npairs) {
-            uint32_t b0 = 0, b1 = 0;
-            if (bcol[p]) {
-              const uint2 v = *reinterpret_cast<const uint2 *>(bcol[p] + kel);
-              b0 = v.x;
-              b1 = v.y;
-            }
-            mma_s8(Cm[p], A, b0, b1, Cm[p]);
+            uint32_t bb0, bb1;
+            load_b(bcol[p], kel, bb0, bb1);
+            mma_s8(Cm[p], A, bb0, bb1, Cm[p]);
           }
         }
       }
@@ -524,11 +576,11 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int RS, const Chunk
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        uint32_t b0 = 0;
-        if (xcol[p]) b0 = *reinterpret_cast<const uint32_t *>(xcol[p] + kb * 16 + 4 * c);
+        uint32_t bx = 0;
+        if (xcol[p]) bx = *reinterpret_cast<const uint32_t *>(xcol[p] + kb * 16 + 4 * c);
         const int zero[4] = {0, 0, 0, 0};
         int cn[4];
-        mma_s8(cn, Am, b0, 0u, zero);
+        mma_s8(cn, Am, bx, 0u, zero);
         F[p][0] = fmaf(d0, (float)Cm[p][0], F[p][0]);
         F[p][1] = fmaf(d0, (float)Cm[p][1], F[p][1]);
         F[p][2] = fmaf(d1, (float)Cm[p][2], F[p][2]);
@@ -584,27 +636,16 @@ __device__ void quantise_vector(const float *src, int n, float vmax, int8_t *dst
 // Shared-memory tables of k2: +/- codebook and byte-permute selectors.
 __device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, int *err) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < 256 * 8; i += blockDim.x) {
-    const int ix = i >> 3, rep = i & 7;
-    uint8_t g[8];
-    bool bad = false;
+  for (int ix = tid; ix < 256; ix += blockDim.x) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(grid + 8 * ix);
+    if ((raw.x | raw.y) & 0x80808080u) set_error(err, kErrGrid);
+    // negate each byte: (0x80 - b) ^ 0x80 computed per byte without carries
+    const uint32_t n0 = __vsub4(0u, raw.x), n1 = __vsub4(0u, raw.y);
+    const uint4 e = make_uint4(raw.x, n0, raw.y, n1);
 #pragma unroll
-    for (int l = 0; l < 8; ++l) {
-      g[l] = grid[8 * ix + l];
-      bad |= g[l] > 127;
-    }
-    if (bad) set_error(err, kErrGrid);
-    uint8_t *e = gpm + ix * 128 + rep * 16;
-#pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      e[l] = g[l];
-      e[4 + l] = (uint8_t)(-(int)g[l]);
-      e[8 + l] = g[4 + l];
-      e[12 + l] = (uint8_t)(-(int)g[4 + l]);
-    }
+    for (int rep = 0; rep < 8; ++rep) *reinterpret_cast<uint4 *>(gpm + ix * 128 + rep * 16) = e;
   }
-  for (int i = tid; i < 128 * 16; i += blockDim.x) {
-    const int m7 = i >> 4, rep = i & 15;
+  for (int m7 = tid; m7 < 128; m7 += blockDim.x) {
     const uint32_t m8 = (uint32_t)m7 | ((uint32_t)(__popc(m7) & 1) << 7);
     uint32_t lo = 0, hi = 0;
 #pragma unroll
@@ -612,9 +653,9 @@ __device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, i
       lo |= (uint32_t)(l + 4 * ((m8 >> l) & 1u)) << (4 * l);
       hi |= (uint32_t)(l + 4 * ((m8 >> (l + 4)) & 1u)) << (4 * l);
     }
-    uint32_t *e = reinterpret_cast<uint32_t *>(selt + m7 * 128 + rep * 8);
-    e[0] = lo;
-    e[1] = hi;
+    const uint2 e = make_uint2(lo, hi);
+#pragma unroll
+    for (int rep = 0; rep < 16; ++rep) *reinterpret_cast<uint2 *>(selt + m7 * 128 + rep * 8) = e;
   }
 }
 
@@ -630,8 +671,8 @@ struct K2Shared {
 // Writes the 16 x ntok SwiGLU outputs held in hs (token slot, row) for the
 // vectors vec[slot], updates max|h|, the 16-row sum and the tile counters;
 // the warp that completes a vector quantises it.
-__device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int ntok, const int *vec, int r0,
-                              int n, int ntiles) {
+__device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int ntok, const int *vec, int r0, int n,
+                              int ntiles) {
   const int lane = threadIdx.x & 31;
   const DecodeScratch &s = a.s;
   for (int base = 0; base < ntok; base += 2) {
@@ -672,32 +713,9 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
   }
 }
 
-// Runs a list of chunks through the warp's two-stage ring; `compute(i, st)`
-// consumes chunk i from stage st.
-template <typename ChunkAt, typename Compute>
-__device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int n, ChunkAt chunk_at,
-                                           Compute compute) {
-  {
-    const Chunk c0 = chunk_at(0);
-    stage_chunk(stage0, stage_rs(c0.bpr), c0.g, c0.gstride, c0.bpr, c0.a16);
-  }
-  for (int i = 0; i < n; ++i) {
-    uint8_t *cur = (i & 1) ? stage1 : stage0;
-    uint8_t *nxt = (i & 1) ? stage0 : stage1;
-    if (i + 1 < n) {
-      const Chunk cn = chunk_at(i + 1);
-      stage_chunk(nxt, stage_rs(cn.bpr), cn.g, cn.gstride, cn.bpr, cn.a16);
-    } else {
-      cp_async_commit();
-    }
-    cp_async_wait<1>();
-    __syncwarp();
-    compute(i, cur);
-    __syncwarp();
-  }
-}
-
-template <int MAXP>
+// XSMEM: the x limbs of all tokens are staged in shared memory (rows of
+// H + 32 bytes, which spreads the B-fragment loads over all banks).
+template <int MAXP, bool XSMEM>
 __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const LayerDims &d = a.d;
@@ -706,10 +724,22 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
   uint8_t *gpm = smem;
   uint8_t *selt = gpm + kGpmBytes;
   uint8_t *stages = selt + kSelBytes;
-  K2Shared &S = *reinterpret_cast<K2Shared *>(stages + 2 * kWarps2 * kStageBytes);
+  K2Shared &S = *reinterpret_cast<K2Shared *>(stages + 2 * kWarps2 * kStage2);
+  int8_t *xsm = reinterpret_cast<int8_t *>(reinterpret_cast<uint8_t *>(&S) + align_up(sizeof(K2Shared), 128));
+  const int XS = d.H + 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   build_tables(a.wt.grid, gpm, selt, a.err);
+  pdl_launch_dependents();
+  pdl_wait();  // k1's limbs and keys are visible from here on
+  if (XSMEM) {
+    const int n16 = d.H / 16;
+    for (int i = tid; i < T * 3 * n16; i += blockDim.x) {
+      const int rowi = i / n16, o = i - rowi * n16;
+      *reinterpret_cast<uint4 *>(xsm + (size_t)rowi * XS + 16 * o) =
+          *reinterpret_cast<const uint4 *>(s.xq + (size_t)rowi * d.H + 16 * o);
+    }
+  }
   for (int t = warp; t < T; t += kWarps2) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
   __syncthreads();
   if (blockIdx.x == 0) {
@@ -722,21 +752,24 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
   const uint8_t *sel_l = selt + (lane & 15) * 8;
-  uint8_t *st0 = stages + warp * 2 * kStageBytes;
-  uint8_t *st1 = st0 + kStageBytes;
+  uint8_t *st0 = stages + warp * 2 * kStage2;
+  uint8_t *st1 = st0 + kStage2;
   const int r = lane >> 2, c = lane & 3;
+  auto xcol = [&](int t, int limb) -> const int8_t * {
+    return XSMEM ? xsm + (size_t)(t * 3 + limb) * XS : s.xq + ((size_t)t * 3 + limb) * d.H;
+  };
 
   const int tilesI = d.I / 16, tilesS = d.Is / 16;
   const int n_sh = tilesS * 4;
   const int n_units = n_sh + S.J.n * tilesI;
-  // IQ2 chunking along H
+  // IQ2 along H: chunks of up to 4 blocks (264 bytes per row)
   const int nbH = d.H / 256;
-  const int cbI = nbH < 8 ? nbH : 8;
+  const int cbI = nbH < 4 ? nbH : 4;
   const int nckI = nbH / cbI;
   const size_t rbI = (size_t)nbH * 66;
-  // Q8_0 shared: a quarter of H in chunks of up to 16 blocks
-  const int nbQ = d.H / 128;  // blocks per quarter
-  const int cbQ = nbQ < 16 ? nbQ : 16;
+  // Q8_0 shared: a quarter of H in chunks of up to 8 blocks (272 bytes per row)
+  const int nbQ = d.H / 128;
+  const int cbQ = nbQ < 8 ? nbQ : 8;
   const int nckQ = nbQ / cbQ;
   const size_t rbQ = (size_t)(d.H / 32) * 34;
 
@@ -755,7 +788,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p] = (ts < T && limb < 3) ? s.xq + ((size_t)ts * 3 + limb) * d.H : nullptr;
+        bcol[p] = (ts < T && limb < 3) ? xcol(ts, limb) : nullptr;
       }
       float F[2][MAXP][4];
 #pragma unroll
@@ -764,25 +797,23 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
         for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
       auto chunk_at = [&](int i) {
         const int m = i / nckQ, ck = i % nckQ;
-        const uint8_t *base = (m == 0 ? a.wt.sh_gate : a.wt.sh_up) + (size_t)r0 * rbQ +
-                              (size_t)(q * nbQ + ck * cbQ) * 34;
+        const size_t off = (size_t)(q * nbQ + ck * cbQ) * 34;
         Chunk ch;
-        ch.g = base;
+        ch.g = (m == 0 ? a.wt.sh_gate : a.wt.sh_up) + (size_t)r0 * rbQ + off;
         ch.gstride = rbQ;
         ch.bpr = cbQ * 34;
         ch.nb = cbQ;
         ch.k0 = (q * nbQ + ck * cbQ) * 32;
-        ch.a16 = ((rbQ & 15) == 0) && (((size_t)(q * nbQ + ck * cbQ) * 34) & 15) == 0 && ((cbQ * 34) & 15) == 0;
+        ch.piece = piece_for(rbQ, off, ch.bpr);
         return ch;
       };
       run_chunks(st0, st1, 2 * nckQ, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
         if (i / nckQ == 0)
-          q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F[0]);
+          q80_chunk<MAXP>(st, ch, bcol, npairs, F[0]);
         else
-          q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F[1]);
+          q80_chunk<MAXP>(st, ch, bcol, npairs, F[1]);
       });
-      // partial sums of this quarter -> global, last quarter finishes the tile
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         if (p < npairs) {
@@ -836,7 +867,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p] = (ts < ntok && limb < 3) ? s.xq + ((size_t)(pairs[ts] / d.k) * 3 + limb) * d.H : nullptr;
+        bcol[p] = (ts < ntok && limb < 3) ? xcol(pairs[ts] / d.k, limb) : nullptr;
       }
       float F[2][MAXP][4];
 #pragma unroll
@@ -845,22 +876,22 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
         for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
       auto chunk_at = [&](int i) {
         const int m = i / nckI, ck = i % nckI;
-        const uint8_t *base = (m == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + (size_t)ck * cbI * 66;
+        const size_t off = (size_t)ck * cbI * 66;
         Chunk ch;
-        ch.g = base;
+        ch.g = (m == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + off;
         ch.gstride = rbI;
         ch.bpr = cbI * 66;
         ch.nb = cbI;
         ch.k0 = ck * cbI * 256;
-        ch.a16 = ((rbI & 15) == 0) && (((size_t)ck * cbI * 66) & 15) == 0 && ((cbI * 66) & 15) == 0;
+        ch.piece = piece_for(rbI, off, ch.bpr);
         return ch;
       };
       run_chunks(st0, st1, 2 * nckI, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
         if (i / nckI == 0)
-          iq2_chunk<MAXP>(st, stage_rs(ch.bpr), ch, gpm_l, sel_l, bcol, npairs, F[0]);
+          iq2_chunk<MAXP>(st, ch, gpm_l, sel_l, bcol, npairs, F[0]);
         else
-          iq2_chunk<MAXP>(st, stage_rs(ch.bpr), ch, gpm_l, sel_l, bcol, npairs, F[1]);
+          iq2_chunk<MAXP>(st, ch, gpm_l, sel_l, bcol, npairs, F[1]);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -902,8 +933,9 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const DecodeScratch &s = a.s;
   const int T = a.T;
   uint8_t *stages = smem;
-  K3Shared &S = *reinterpret_cast<K3Shared *>(stages + 2 * kWarps2 * kStageBytes);
+  K3Shared &S = *reinterpret_cast<K3Shared *>(stages + 2 * kWarps2 * kStage3);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();  // k2's routing and h limbs are visible from here on
   for (int i = tid; i < T * d.k; i += blockDim.x) {
     S.idx[i] = s.idx[i];
     S.w[i] = s.w[i];
@@ -911,21 +943,21 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   __syncthreads();
   build_jobs(S.idx, T, d.k, S.J);
 
-  uint8_t *st0 = stages + warp * 2 * kStageBytes;
-  uint8_t *st1 = st0 + kStageBytes;
+  uint8_t *st0 = stages + warp * 2 * kStage3;
+  uint8_t *st1 = st0 + kStage3;
   const int r = lane >> 2, c = lane & 3;
   const int tilesH = d.H / 16;
   const int nparts = S.J.n + 4;
   const int n_units = tilesH * nparts;
   const int Im16 = s.Imax / 16;
-  // Q2_K chunking along I: up to 4 blocks (336 bytes) per chunk
+  // Q2_K along I: chunks of up to 4 blocks (336 bytes per row)
   const int nbI = d.I / 256;
   const int cbD = nbI < 4 ? nbI : 4;
   const int nckD = nbI / cbD;
   const size_t rbD = (size_t)nbI * 84;
-  // Q8_0 shared down: a quarter of Is in chunks of up to 16 blocks
+  // Q8_0 shared down: a quarter of Is in chunks of up to 8 blocks
   const int nbQ = d.Is / 128;
-  const int cbQ = nbQ < 16 ? nbQ : 16;
+  const int cbQ = nbQ < 8 ? nbQ : 8;
   const int nckQ = nbQ / cbQ;
   const size_t rbQ = (size_t)(d.Is / 32) * 34;
 
@@ -961,18 +993,19 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
       auto chunk_at = [&](int i) {
+        const size_t off = (size_t)i * cbD * 84;
         Chunk ch;
-        ch.g = a.wt.down + ((size_t)e * d.H + r0) * rbD + (size_t)i * cbD * 84;
+        ch.g = a.wt.down + ((size_t)e * d.H + r0) * rbD + off;
         ch.gstride = rbD;
         ch.bpr = cbD * 84;
         ch.nb = cbD;
         ch.k0 = i * cbD * 256;
-        ch.a16 = ((rbD & 15) == 0) && (((size_t)i * cbD * 84) & 15) == 0 && ((cbD * 84) & 15) == 0;
+        ch.piece = piece_for(rbD, off, ch.bpr);
         return ch;
       };
       run_chunks(st0, st1, nckD, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        q2k_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, xcol, npairs, F, G);
+        q2k_chunk<MAXP>(st, ch, bcol, xcol, npairs, F, G);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -1022,12 +1055,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
         ch.bpr = cbQ * 34;
         ch.nb = cbQ;
         ch.k0 = (q * nbQ + i * cbQ) * 32;
-        ch.a16 = ((rbQ & 15) == 0) && (off & 15) == 0 && ((cbQ * 34) & 15) == 0;
+        ch.piece = piece_for(rbQ, off, ch.bpr);
         return ch;
       };
       run_chunks(st0, st1, nckQ, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        q80_chunk<MAXP>(st, stage_rs(ch.bpr), ch, bcol, npairs, F);
+        q80_chunk<MAXP>(st, ch, bcol, npairs, F);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -1073,42 +1106,59 @@ __global__ void k_route_only(DecodeArgs a, int32_t *idx, float *w) {
     warp_route_token(a, t, idx + (size_t)t * a.d.k, w + (size_t)t * a.d.k);
 }
 
-size_t k2_smem_bytes() {
-  return kGpmBytes + kSelBytes + 2 * kWarps2 * kStageBytes + sizeof(K2Shared);
+size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
+  size_t b = kGpmBytes + kSelBytes + 2 * kWarps2 * kStage2 + align_up(sizeof(K2Shared), 128);
+  if (xsmem) b += (size_t)T * 3 * (d.H + 32);
+  return b;
 }
-size_t k3_smem_bytes() { return 2 * kWarps2 * kStageBytes + sizeof(K3Shared); }
+size_t k3_smem_bytes() { return 2 * kWarps2 * kStage3 + sizeof(K3Shared); }
 
-template <int MAXP>
+constexpr size_t kSmemLimit = 227 * 1024;
+
+template <typename K>
+cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+template <int MAXP, bool XSMEM>
 cudaError_t launch_k23(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k2_gateup<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)k2_smem_bytes());
+    cudaError_t e = cudaFuncSetAttribute(k2_gateup<MAXP, XSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemLimit);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k3_down<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k3_smem_bytes());
     if (e != cudaSuccess) return e;
     configured = true;
   }
   if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
-  k2_gateup<MAXP><<<num_sms, kThreads2, k2_smem_bytes(), stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(k2_gateup<MAXP, XSMEM>, num_sms, kThreads2, k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
   if (e != cudaSuccess) return e;
   if (a.ev_end) cudaEventRecord(a.ev_end, stream);
-  k3_down<MAXP><<<num_sms, kThreads2, k3_smem_bytes(), stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k3_down<MAXP>, num_sms, kThreads2, k3_smem_bytes(), stream, a);
 }
 
 cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
   const int nr = a.d.mode == MOE_ROUTE_ROUTER ? (a.d.E + 1) / 2 : 0;
   const int grid = a.T + nr;
   if (a.T <= 1)
-    k1_prep_router<1><<<grid, 128, 0, stream>>>(a);
+    k1_prep_router<1><<<grid, kRouterThreads, 0, stream>>>(a);
   else if (a.T <= 2)
-    k1_prep_router<2><<<grid, 128, 0, stream>>>(a);
+    k1_prep_router<2><<<grid, kRouterThreads, 0, stream>>>(a);
   else if (a.T <= 4)
-    k1_prep_router<4><<<grid, 128, 0, stream>>>(a);
+    k1_prep_router<4><<<grid, kRouterThreads, 0, stream>>>(a);
   else
-    k1_prep_router<8><<<grid, 128, 0, stream>>>(a);
+    k1_prep_router<8><<<grid, kRouterThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -1134,6 +1184,7 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.Imax = Imax;
   s.P = P;
   s.z = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
+  s.sc = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * T * d.k));
   s.w = reinterpret_cast<float *>(take(sizeof(float) * T * d.k));
   s.xq = reinterpret_cast<int8_t *>(take((size_t)T * 3 * d.H));
@@ -1157,9 +1208,12 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
-  if (a.T <= 2) return launch_k23<1>(a, stream, num_sms);
-  if (a.T <= 4) return launch_k23<2>(a, stream, num_sms);
-  return launch_k23<4>(a, stream, num_sms);
+  if (a.T <= 2) {
+    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k23<1, true>(a, stream, num_sms);
+    return launch_k23<1, false>(a, stream, num_sms);
+  }
+  if (a.T <= 4) return launch_k23<2, false>(a, stream, num_sms);
+  return launch_k23<4, false>(a, stream, num_sms);
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {

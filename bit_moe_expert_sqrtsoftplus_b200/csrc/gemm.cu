@@ -171,22 +171,51 @@ __device__ __forceinline__ Tile tile_at(const GemmCtl &ctl, int t, int m_tiles) 
 }
 
 // ---------------------------------------------------------------- producers
+//
+// A producer thread owns one (row, 32-element half) item of the 128 x 64 K
+// step (for a gate/up pair, the same item of both matrices).  fetch() reads
+// the packed bytes of an item into registers (issued two K steps ahead of
+// their use); decode() turns them into 16-bit values in the swizzled tile.
 
-// IQ2_XXS: 32 elements (one group) of row `rowp` -> f16 into chunks 4*item..4*item+3.
-__device__ __forceinline__ void deq_iq2(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item,
-                                        const uint8_t *gridh, const uint8_t *signm) {
+template <int FMT>
+struct Raw;
+template <>
+struct Raw<kFmtIQ2> {
+  uint32_t d16, idx4, S;
+};
+template <>
+struct Raw<kFmtQ2K> {
+  uint32_t dd, scw, q[8];
+};
+template <>
+struct Raw<kFmtQ80> {
+  uint32_t d16, q[8];
+};
+
+// IQ2_XXS: group (kel/32) of the row.
+__device__ __forceinline__ void fetch(Raw<kFmtIQ2> &r, const uint8_t *rowp, int ks, int item) {
+  const int kel = ks * BK + 32 * item;
   const int blk = kel >> 8, gib = (kel >> 5) & 7;
   const uint8_t *bp = rowp + (size_t)blk * 66;
   const uint8_t *gp = bp + 2 + 8 * gib;
-  const uint32_t d16 = ldg16(bp);
-  const uint32_t idx4 = ldg16(gp) | (ldg16(gp + 2) << 16);
-  const uint32_t S = ldg16(gp + 4) | (ldg16(gp + 6) << 16);
-  const __half2 f2 = __half2half2(__int2half_rn(2 * (int)(S >> 28) + 1));
-  const __half2 d2 = __half2half2(__hmul(__ushort_as_half((unsigned short)d16), __float2half(0.125f)));
+  r.d16 = ldg16(bp);
+  if ((reinterpret_cast<uintptr_t>(gp) & 3u) == 0) {
+    r.idx4 = ldg32(gp);
+    r.S = ldg32(gp + 4);
+  } else {
+    r.idx4 = ldg16(gp) | (ldg16(gp + 2) << 16);
+    r.S = ldg16(gp + 4) | (ldg16(gp + 6) << 16);
+  }
+}
+
+__device__ __forceinline__ void decode(const Raw<kFmtIQ2> &r, uint8_t *tile, int row, int item, int,
+                                       const uint8_t *gridh, const uint8_t *signm) {
+  const __half2 f2 = __half2half2(__int2half_rn(2 * (int)(r.S >> 28) + 1));
+  const __half2 d2 = __half2half2(__hmul(__ushort_as_half((unsigned short)r.d16), __float2half(0.125f)));
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t ix = (idx4 >> (8 * j)) & 255u;
-    const uint32_t m7 = (S >> (7 * j)) & 127u;
+    const uint32_t ix = (r.idx4 >> (8 * j)) & 255u;
+    const uint32_t m7 = (r.S >> (7 * j)) & 127u;
     const uint4 g = *reinterpret_cast<const uint4 *>(gridh + ix * 16u);
     const uint4 sm = *reinterpret_cast<const uint4 *>(signm + m7 * 16u);
     const uint32_t o0 = h2bits(__hmul2(__hmul2(bits2h(g.x ^ sm.x), f2), d2));
@@ -202,19 +231,25 @@ __device__ __forceinline__ uint32_t bf16pair(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Q2_K: 32 elements of row `rowp` at K offset kel (64-aligned k step, half `item`).
-__device__ __forceinline__ void deq_q2k(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item) {
-  const int blk = kel >> 8, qq = (kel >> 6) & 3;
+// Q2_K: the K step covers 64 elements of block ks/4; item = which of its two shifts.
+__device__ __forceinline__ void fetch(Raw<kFmtQ2K> &r, const uint8_t *rowp, int ks, int item) {
+  const int blk = ks >> 2, qq = ks & 3;
   const uint8_t *bp = rowp + (size_t)blk * 84;
   const int hf = qq >> 1, sh = 2 * (qq & 1) + item;
-  const uint32_t dd = ldg32(bp + 80);
-  const float d = __half2float(__ushort_as_half((unsigned short)(dd & 0xFFFFu)));
-  const float dmin = __half2float(__ushort_as_half((unsigned short)(dd >> 16)));
-  const int j0 = 8 * hf + 2 * sh;
-  const uint32_t scw = ldg16(bp + j0);  // scale bytes of sub-blocks j0, j0 + 1
+  r.dd = ldg32(bp + 80);
+  r.scw = ldg16(bp + 8 * hf + 2 * sh);  // scale bytes of sub-blocks 8hf+2sh, +1
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.q[i] = ldg32(bp + 16 + 32 * hf + 4 * i);
+}
+
+__device__ __forceinline__ void decode(const Raw<kFmtQ2K> &r, uint8_t *tile, int row, int item, int ks,
+                                       const uint8_t *, const uint8_t *) {
+  const int sh = 2 * (ks & 1) + item;
+  const float d = __half2float(__ushort_as_half((unsigned short)(r.dd & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half((unsigned short)(r.dd >> 16)));
 #pragma unroll
   for (int sub = 0; sub < 2; ++sub) {
-    const uint32_t sb = (scw >> (8 * sub)) & 0xFFu;
+    const uint32_t sb = (r.scw >> (8 * sub)) & 0xFFu;
     const float dsc = d * (float)(sb & 15u);
     const float mn = -dmin * (float)(sb >> 4);
     const uint32_t V0 = bf16pair(mn, fmaf(dsc, 1.f, mn));
@@ -222,8 +257,7 @@ __device__ __forceinline__ void deq_q2k(const uint8_t *rowp, int kel, uint8_t *t
     uint32_t o[8];
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
-      const uint32_t w = ldg32(bp + 16 + 32 * hf + 16 * sub + 4 * wi);
-      const uint32_t q = (w >> (2 * sh)) & 0x03030303u;
+      const uint32_t q = (r.q[4 * sub + wi] >> (2 * sh)) & 0x03030303u;
       const uint32_t t = q * 0x22u + 0x10101010u;
       o[2 * wi] = __byte_perm(V0, V1, t & 0xFFFFu);
       o[2 * wi + 1] = __byte_perm(V0, V1, t >> 16);
@@ -233,15 +267,15 @@ __device__ __forceinline__ void deq_q2k(const uint8_t *rowp, int kel, uint8_t *t
   }
 }
 
-// Q8_0: one 32-element block (index kel/32) of row `rowp`.
-__device__ __forceinline__ void deq_q80(const uint8_t *rowp, int kel, uint8_t *tile, int row, int item, int bf16) {
+// Q8_0: 32-element block (kel/32) of the row.
+__device__ __forceinline__ void fetch(Raw<kFmtQ80> &r, const uint8_t *rowp, int ks, int item) {
+  const int kel = ks * BK + 32 * item;
   const uint8_t *bp = rowp + (size_t)(kel >> 5) * 34;
-  const uint32_t d16 = ldg16(bp);
+  r.d16 = ldg16(bp);
   const uint8_t *qp = bp + 2;
-  uint32_t w[8];
   if ((reinterpret_cast<uintptr_t>(qp) & 3u) == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = ldg32(qp + 4 * i);
+    for (int i = 0; i < 8; ++i) r.q[i] = ldg32(qp + 4 * i);
   } else {
     const uint8_t *base = qp - 2;  // 4-byte aligned; the last word is read as 16 bits to stay in the block
     uint32_t u[9];
@@ -249,16 +283,20 @@ __device__ __forceinline__ void deq_q80(const uint8_t *rowp, int kel, uint8_t *t
     for (int i = 0; i < 8; ++i) u[i] = ldg32(base + 4 * i);
     u[8] = ldg16(base + 32);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = __byte_perm(u[i], u[i + 1], 0x5432);
+    for (int i = 0; i < 8; ++i) r.q[i] = __byte_perm(u[i], u[i + 1], 0x5432);
   }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void decode_q80(const Raw<kFmtQ80> &r, uint8_t *tile, int row, int item) {
   uint32_t o[16];
-  const __half dh = __ushort_as_half((unsigned short)d16);
+  const __half dh = __ushort_as_half((unsigned short)r.d16);
   const __half2 bias = __half2half2(__float2half(1152.f));
-  if (!bf16) {
+  if (!BF16) {
     const __half2 d2 = __half2half2(dh);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t x = w[i] ^ 0x80808080u;
+      const uint32_t x = r.q[i] ^ 0x80808080u;
       const __half2 lo = __hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x5140)), bias);
       const __half2 hi = __hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x7362)), bias);
       o[2 * i] = h2bits(__hmul2(lo, d2));
@@ -268,7 +306,7 @@ __device__ __forceinline__ void deq_q80(const uint8_t *rowp, int kel, uint8_t *t
     const float d = __half2float(dh);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t x = w[i] ^ 0x80808080u;
+      const uint32_t x = r.q[i] ^ 0x80808080u;
       const float2 lo = __half22float2(__hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x5140)), bias));
       const float2 hi = __half22float2(__hsub2(bits2h(__byte_perm(x, 0x64646464u, 0x7362)), bias));
       o[2 * i] = bf16pair(lo.x * d, lo.y * d);
@@ -279,9 +317,17 @@ __device__ __forceinline__ void deq_q80(const uint8_t *rowp, int kel, uint8_t *t
   for (int c = 0; c < 4; ++c) sts128(swz(tile, row, 4 * item + c), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
 }
 
+__device__ __forceinline__ void decode(const Raw<kFmtQ80> &r, uint8_t *tile, int row, int item, int bf16,
+                                       const uint8_t *, const uint8_t *) {
+  if (bf16)
+    decode_q80<true>(r, tile, row, item);
+  else
+    decode_q80<false>(r, tile, row, item);
+}
+
 // ---------------------------------------------------------------- kernel
 
-template <bool PAIRED>
+template <int FMT, bool PAIRED>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   constexpr int NA = PAIRED ? 2 : 1;
   constexpr int S = PAIRED ? 3 : 4;
@@ -324,7 +370,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     ctl.n_groups = G;
     ctl.total_tiles = pre;
   }
-  if (a.fmt == kFmtIQ2) {
+  if (FMT == kFmtIQ2) {
     for (int i = tid; i < 256 * 8; i += blockDim.x) {  // codebook -> f16
       const int ix = i >> 3, l = i & 7;
       reinterpret_cast<__half *>(gridh)[ix * 8 + l] = __int2half_rn(a.grid[ix * 8 + l]);
@@ -368,38 +414,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
         }
       }
       // A items: row p/2, 32-element half p%2 of the 64-element K step
-      const uint8_t *arow0, *arow1 = nullptr;
       const int row = p >> 1, item = p & 1;
-      arow0 = a.A0 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
-      if (PAIRED) arow1 = a.A1 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
-      bool ok = true;
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1u;
-        if (!mbar_wait(&ctl.empty[st], ph ^ 1u, ctl, a.err)) {
-          ok = false;
-          break;
-        }
-        uint8_t *A0s = stages + st * STAGE;
-        uint8_t *Bs = A0s + NA * kATile;
+      const uint8_t *arow[2];
+      arow[0] = a.A0 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
+      arow[1] = PAIRED ? a.A1 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row) : arow[0];
+      const int dsel = FMT == kFmtQ80 ? a.bf16 : 0;
+      Raw<FMT> r0[PAIRED ? 2 : 1], r1[PAIRED ? 2 : 1], r2[PAIRED ? 2 : 1];
+#pragma unroll
+      for (int m = 0; m < (PAIRED ? 2 : 1); ++m) {
+        fetch(r0[m], arow[m], 0, item);
+        if (ksteps > 1) fetch(r1[m], arow[m], 1, item);
+      }
+      auto issue_b = [&](int ks, int st) {
+        uint8_t *Bs = stages + st * STAGE + NA * kATile;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 32 * i, ch), brow[i] + ks * BK);
         }
         cp_async_commit();
-        const int kel = ks * BK + 32 * item;
-        if (a.fmt == kFmtIQ2) {
-          deq_iq2(arow0, kel, A0s, row, item, gridh, signm);
-          if (PAIRED) deq_iq2(arow1, kel, A0s + kATile, row, item, gridh, signm);
-        } else if (a.fmt == kFmtQ2K) {
-          deq_q2k(arow0, ks * BK, A0s, row, item);
+      };
+      bool ok = mbar_wait(&ctl.empty[it % S], ((it / S) & 1u) ^ 1u, ctl, a.err);
+      if (ok) issue_b(0, it % S);
+      for (int ks = 0; ok && ks < ksteps; ++ks, ++it) {
+        const int st = it % S;
+        if (ks + 1 < ksteps) {
+          const uint32_t nt = it + 1;
+          if (!mbar_wait(&ctl.empty[nt % S], ((nt / S) & 1u) ^ 1u, ctl, a.err)) {
+            ok = false;
+            break;
+          }
+          issue_b(ks + 1, nt % S);
         } else {
-          deq_q80(arow0, kel, A0s, row, item, a.bf16);
-          if (PAIRED) deq_q80(arow1, kel, A0s + kATile, row, item, a.bf16);
+          cp_async_commit();
         }
-        cp_async_wait<0>();
+        if (ks + 2 < ksteps) {
+#pragma unroll
+          for (int m = 0; m < (PAIRED ? 2 : 1); ++m) fetch(r2[m], arow[m], ks + 2, item);
+        }
+        uint8_t *A0s = stages + st * STAGE;
+#pragma unroll
+        for (int m = 0; m < (PAIRED ? 2 : 1); ++m)
+          decode(r0[m], A0s + m * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh, signm);
+        cp_async_wait<1>();  // this step's B tile has landed
         fence_proxy_async();
         mbar_arrive(&ctl.full[st]);
+#pragma unroll
+        for (int m = 0; m < (PAIRED ? 2 : 1); ++m) {
+          r0[m] = r1[m];
+          r1[m] = r2[m];
+        }
       }
       if (!ok) break;
     }
@@ -517,27 +580,27 @@ size_t grouped_gemm_smem(int paired) {
   return 1024 + (size_t)s * (na * kATile + kBTile) + 4096 + 2048 + sizeof(GemmCtl);
 }
 
-cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
-  static bool configured[2] = {false, false};
-  const bool paired = a.A1 != nullptr;
-  const size_t smem = grouped_gemm_smem(paired);
-  if (paired) {
-    if (!configured[1]) {
-      cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      configured[1] = true;
-    }
-    k_grouped_gemm<true><<<num_sms, kGemmThreads, smem, s>>>(a);
-  } else {
-    if (!configured[0]) {
-      cudaError_t e =
-          cudaFuncSetAttribute(k_grouped_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      configured[0] = true;
-    }
-    k_grouped_gemm<false><<<num_sms, kGemmThreads, smem, s>>>(a);
+template <int FMT, bool PAIRED>
+static cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
+  static bool configured = false;
+  const size_t smem = grouped_gemm_smem(PAIRED);
+  if (!configured) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_grouped_gemm<FMT, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
   }
+  k_grouped_gemm<FMT, PAIRED><<<num_sms, kGemmThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
+  const bool paired = a.A1 != nullptr;
+  if (a.fmt == kFmtIQ2 && paired) return launch_gemm<kFmtIQ2, true>(a, s, num_sms);
+  if (a.fmt == kFmtQ80 && paired) return launch_gemm<kFmtQ80, true>(a, s, num_sms);
+  if (a.fmt == kFmtQ80 && !paired) return launch_gemm<kFmtQ80, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ2K && !paired) return launch_gemm<kFmtQ2K, false>(a, s, num_sms);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

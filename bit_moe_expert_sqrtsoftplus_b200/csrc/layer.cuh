@@ -27,7 +27,8 @@ struct LayerWeights {
 // Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
 // t*k + slot, shared vector T*k + t.
 struct DecodeScratch {
-  double *z;        // [T][E] router logits (fp64)
+  double *z;        // [T][E] selection keys sqrtsoftplus(z) + bias (fp64)
+  double *sc;       // [T][E] scores sqrtsoftplus(z) (fp64)
   int32_t *idx;     // [T][k]
   float *w;         // [T][k]
   int8_t *xq;       // [T][3][H] int8 limbs of the expert input

@@ -29,7 +29,7 @@ def build() -> None:
     if os.path.exists(_SO) and os.path.getmtime(_SO) >= max(os.path.getmtime(s) for s in srcs):
         return
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-                           "-o", _SO, srcs[0], "-lm"])
+                           "-o", _SO, srcs[0], "-lm", "-pthread"])
 
 
 def lib():
@@ -60,6 +60,8 @@ def lib():
         L.oracle_swiglu_expert.argtypes = [i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.oracle_layer.argtypes = [vp, vp, i32, vp, vp, vp]
         L.oracle_layer.restype = i32
+        L.oracle_layer_mt.argtypes = [vp, vp, i32, vp, vp, vp, i32]
+        L.oracle_layer_mt.restype = i32
         L.oracle_permutation.argtypes = [vp, i32, i32, i32, vp, vp]
         L.oracle_rmsnorm.argtypes = [vp, i32, d, vp]
         _lib = L
@@ -208,7 +210,7 @@ def swiglu_expert(gate, up, down, hidden, inter, x, grid=None, gate_kind=KIND_IQ
     return out
 
 
-def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray) -> np.ndarray:
+def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray, threads: int = 1) -> np.ndarray:
     """y [T][H] fp64 for the given routing.  ``weights`` as returned by
     ``synth.host_layer`` (routed tensors as full arrays or dicts by id)."""
     keep = []
@@ -231,7 +233,10 @@ def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray) -
     ii, pi = _c(idx, np.int32)
     ww, pw = _c(w, np.float64)
     y = np.zeros((T, shape.hidden), dtype=np.float64)
-    rc = lib().oracle_layer(ctypes.byref(lw), px, T, pi, pw, y.ctypes.data)
+    if threads > 1:
+        rc = lib().oracle_layer_mt(ctypes.byref(lw), px, T, pi, pw, y.ctypes.data, int(threads))
+    else:
+        rc = lib().oracle_layer(ctypes.byref(lw), px, T, pi, pw, y.ctypes.data)
     if rc != 0:
         raise ValueError("oracle_layer: a selected expert has no weights")
     return y

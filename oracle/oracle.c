@@ -13,6 +13,7 @@
 #include "oracle.h"
 
 #include <math.h>
+#include <pthread.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -327,6 +328,53 @@ int oracle_layer(const oracle_layer_w *W, const double *x, int T, const int32_t 
   free(slot);
   free(wrow);
   return 0;
+}
+
+/* The same layer with the tokens split over threads; every token's arithmetic
+ * is exactly that of oracle_layer (tokens are independent). */
+typedef struct {
+  const oracle_layer_w *W;
+  const double *x;
+  int T;
+  const int32_t *idx;
+  const double *w;
+  double *y;
+  int rc;
+} layer_job;
+
+static void *layer_job_run(void *arg) {
+  layer_job *j = (layer_job *)arg;
+  j->rc = oracle_layer(j->W, j->x, j->T, j->idx, j->w, j->y);
+  return NULL;
+}
+
+int oracle_layer_mt(const oracle_layer_w *W, const double *x, int T, const int32_t *idx, const double *w, double *y,
+                    int nthreads) {
+  if (nthreads <= 1 || T <= 1) return oracle_layer(W, x, T, idx, w, y);
+  if (nthreads > T) nthreads = T;
+  if (nthreads > 64) nthreads = 64;
+  pthread_t th[64];
+  layer_job jobs[64];
+  const int H = W->hidden, k = W->top_k;
+  int t0 = 0;
+  for (int i = 0; i < nthreads; ++i) {
+    const int n = T / nthreads + (i < T % nthreads);
+    jobs[i].W = W;
+    jobs[i].x = x + (size_t)t0 * H;
+    jobs[i].T = n;
+    jobs[i].idx = idx + (size_t)t0 * k;
+    jobs[i].w = w + (size_t)t0 * k;
+    jobs[i].y = y + (size_t)t0 * H;
+    jobs[i].rc = 0;
+    pthread_create(&th[i], NULL, layer_job_run, &jobs[i]);
+    t0 += n;
+  }
+  int rc = 0;
+  for (int i = 0; i < nthreads; ++i) {
+    pthread_join(th[i], NULL);
+    if (jobs[i].rc) rc = jobs[i].rc;
+  }
+  return rc;
 }
 
 /* ---------------------------------------------------------- permutation */

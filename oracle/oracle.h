@@ -83,6 +83,10 @@ typedef struct {
 int oracle_layer(const oracle_layer_w *Wt, const double *x, int T, const int32_t *idx, const double *w,
                  double *y);
 
+/* oracle_layer with the tokens split over `nthreads` threads (same results). */
+int oracle_layer_mt(const oracle_layer_w *Wt, const double *x, int T, const int32_t *idx, const double *w,
+                    double *y, int nthreads);
+
 /* Stable counting sort of the T*k (token, slot) pairs by expert. */
 void oracle_permutation(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm);
 

@@ -25,7 +25,7 @@ def device_layer(s: synth.LayerShape, seed: int, layer: int, router=True):
 
 
 def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, token_ids=None, router=True,
-                 prenorm=False):
+                 prenorm=False, threads: int = 1):
     """fp64 oracle: returns (idx, w, y, margin)."""
     xin = x.astype(np.float64)
     if prenorm:
@@ -40,7 +40,7 @@ def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, toke
         idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling)
         margin = np.full(x.shape[0], np.inf)
     W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router)
-    y = oracle.layer(W, s, xin, idx, w)
+    y = oracle.layer(W, s, xin, idx, w, threads=threads)
     if prenorm:
         y = y + x.astype(np.float64)
     return idx, w, y, margin
