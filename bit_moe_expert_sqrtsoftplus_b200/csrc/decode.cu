@@ -28,6 +28,8 @@
 #include <float.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "layer.cuh"
 
@@ -349,23 +351,32 @@ __host__ __device__ __forceinline__ int piece_for(size_t gstride, size_t off, in
 __device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
 
 // Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS).
+// Rows are walked in order; each lane issues the pieces lane, lane + 32, ...
+// of a row (a chunk row is at most 34 pieces).
 __device__ __forceinline__ void stage_chunk(uint8_t *st, const Chunk &c) {
   const int lane = threadIdx.x & 31;
   const int RS = stage_rs(c.bpr);
   const int n = c.bpr / c.piece;
-  for (int row = 0; row < 16; ++row) {
-    const uint8_t *g = c.g + row * c.gstride;
-    uint8_t *s = st + row * RS;
-    for (int o = lane; o < n; o += 32) {
-      const int off = o * c.piece;
-      if (c.piece == 16)
-        cp_async16(s + off, g + off);
-      else if (c.piece == 8)
-        cp_async8(s + off, g + off);
-      else if (c.piece == 4)
-        cp_async4(s + off, g + off);
-      else
-        *reinterpret_cast<uint16_t *>(s + off) = *reinterpret_cast<const uint16_t *>(g + off);
+  const uint8_t *g = c.g;
+  uint8_t *s = st;
+  if (c.piece == 8) {
+#pragma unroll 4
+    for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
+      for (int o = lane; o < n; o += 32) cp_async8(s + 8 * o, g + 8 * o);
+    }
+  } else if (c.piece == 16) {
+#pragma unroll 4
+    for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
+      for (int o = lane; o < n; o += 32) cp_async16(s + 16 * o, g + 16 * o);
+    }
+  } else if (c.piece == 4) {
+    for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
+      for (int o = lane; o < n; o += 32) cp_async4(s + 4 * o, g + 4 * o);
+    }
+  } else {
+    for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
+      for (int o = lane; o < n; o += 32)
+        *reinterpret_cast<uint16_t *>(s + 2 * o) = *reinterpret_cast<const uint16_t *>(g + 2 * o);
     }
   }
   cp_async_commit();
@@ -393,69 +404,77 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
 
 // ------------------------------------------------------------------ decoders
 
-// IQ2_XXS group -> int8 A fragment halves for sub-vector c of one row.
-__device__ __forceinline__ void iq2_group(const uint8_t *grp, uint32_t S, int c, const uint8_t *gpm_l,
-                                          const uint8_t *sel_l, uint32_t &lo, uint32_t &hi) {
-  const uint32_t ix = grp[c];
-  const uint32_t m7 = (S >> (7 * c)) & 127u;
-  const uint4 gv = *reinterpret_cast<const uint4 *>(gpm_l + ix * 128u);
-  const uint2 sv = *reinterpret_cast<const uint2 *>(sel_l + m7 * 128u);
+// B operand column (the int8 limbs of one vector) in shared or global memory;
+// `ok` is false for the padding columns, which read as zero.
+struct BColS {
+  const int8_t *p;  // shared memory
+  bool ok;
+};
+struct BColG {
+  const int8_t *p;  // global memory
+  bool ok;
+};
+__device__ __forceinline__ uint2 ldb(const BColS &b, int kel) {
+  uint2 v = make_uint2(0u, 0u);
+  if (b.ok) v = *reinterpret_cast<const uint2 *>(b.p + kel);
+  return v;
+}
+__device__ __forceinline__ uint2 ldb(const BColG &b, int kel) {
+  uint2 v = make_uint2(0u, 0u);
+  if (b.ok) v = __ldg(reinterpret_cast<const uint2 *>(b.p + kel));
+  return v;
+}
+
+// IQ2_XXS group of one staged row -> the A fragment halves of sub-vector c,
+// and the group's scale factor 2s+1.  `o` is the group's byte offset in the row
+// (a compile-time constant once the loops are unrolled, so is its alignment).
+__device__ __forceinline__ void iq2_group(const uint8_t *rowc, const uint8_t *row, int o, int sh7,
+                                          const uint8_t *gpm_l, const uint8_t *sel_l, uint32_t &lo, uint32_t &hi,
+                                          int &f) {
+  const uint32_t ix = rowc[o];  // rowc = row + c
+  uint32_t S;
+  if (((o + 4) & 3) == 0)
+    S = lds_u32(row + o + 4);
+  else
+    S = lds_u16(row + o + 4) | (lds_u16(row + o + 6) << 16);
+  const uint32_t m7 = (S >> sh7) & 127u;
+  const uint4 gv = *reinterpret_cast<const uint4 *>(gpm_l + (ix << 7));
+  const uint2 sv = *reinterpret_cast<const uint2 *>(sel_l + (m7 << 7));
   lo = __byte_perm(gv.x, gv.y, sv.x);
   hi = __byte_perm(gv.z, gv.w, sv.y);
+  f = (int)((S >> 27) | 1u);  // 2s + 1
 }
 
-// The 32-bit word at grp+4 (S: sign masks and scale); grp is 2-byte aligned.
-__device__ __forceinline__ uint32_t iq2_sword(const uint8_t *grp) {
-  const uint8_t *p = grp + 4;
-  if ((reinterpret_cast<uintptr_t>(p) & 3u) == 0) return lds_u32(p);
-  return lds_u16(p) | (lds_u16(p + 2) << 16);
-}
-
-// B fragment (8 int8 of one limb column) from shared or global memory.
-__device__ __forceinline__ void load_b(const int8_t *col, int kel, uint32_t &b0, uint32_t &b1) {
-  if (col) {
-    const uint2 v = *reinterpret_cast<const uint2 *>(col + kel);
-    b0 = v.x;
-    b1 = v.y;
-  } else {
-    b0 = b1 = 0u;
-  }
-}
-
-template <int MAXP>
-__device__ __forceinline__ void iq2_chunk(const uint8_t *st, const Chunk &ch, const uint8_t *gpm_l,
-                                          const uint8_t *sel_l, const int8_t *const (&bcol)[MAXP], int npairs,
-                                          float (&F)[MAXP][4]) {
+template <int NB, int MAXP, typename BCol>
+__device__ __forceinline__ void iq2_chunk(const uint8_t *st, int k0, const uint8_t *gpm_l, const uint8_t *sel_l,
+                                          const BCol (&bcol)[MAXP], int npairs, float (&F)[MAXP][4]) {
+  constexpr int RS = (NB * 66 + 15) / 16 * 16;
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-  const int RS = stage_rs(ch.bpr);
+  const int sh7 = 7 * c;
   const uint8_t *row0 = st + r * RS;
-  const uint8_t *row1 = st + (r + 8) * RS;
-  for (int b = 0; b < ch.nb; ++b) {
-    const uint8_t *b0p = row0 + 66 * b;
-    const uint8_t *b1p = row1 + 66 * b;
-    const float d0 = half_bits_to_float(lds_u16(b0p)) * 0.125f;
-    const float d1 = half_bits_to_float(lds_u16(b1p)) * 0.125f;
+  const uint8_t *row1 = row0 + 8 * RS;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const float d0 = half_bits_to_float(lds_u16(row0 + 66 * b)) * 0.125f;
+    const float d1 = half_bits_to_float(lds_u16(row1 + 66 * b)) * 0.125f;
     int acc[MAXP][4];
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-      const uint8_t *g0 = b0p + 2 + 8 * g;
-      const uint8_t *g1 = b1p + 2 + 8 * g;
-      const uint32_t S0 = iq2_sword(g0), S1 = iq2_sword(g1);
+      const int o = 66 * b + 2 + 8 * g;
       uint32_t A[4];
-      iq2_group(g0, S0, c, gpm_l, sel_l, A[0], A[2]);
-      iq2_group(g1, S1, c, gpm_l, sel_l, A[1], A[3]);
-      const int f0 = 2 * (int)(S0 >> 28) + 1, f1 = 2 * (int)(S1 >> 28) + 1;
-      const int kel = ch.k0 + 256 * b + 32 * g + 8 * c;
+      int f0, f1;
+      iq2_group(row0 + c, row0, o, sh7, gpm_l, sel_l, A[0], A[2], f0);
+      iq2_group(row1 + c, row1, o, sh7, gpm_l, sel_l, A[1], A[3], f1);
+      const int kel = k0 + 256 * b + 32 * g;  // the column base includes 8c
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         if (p < npairs) {
-          uint32_t bb0, bb1;
-          load_b(bcol[p], kel, bb0, bb1);
+          const uint2 bb = ldb(bcol[p], kel);
           const int zero[4] = {0, 0, 0, 0};
           int cg[4];
-          mma_s8(cg, A, bb0, bb1, zero);
+          mma_s8(cg, A, bb.x, bb.y, zero);
           acc[p][0] += cg[0] * f0;
           acc[p][1] += cg[1] * f0;
           acc[p][2] += cg[2] * f1;
@@ -473,10 +492,10 @@ __device__ __forceinline__ void iq2_chunk(const uint8_t *st, const Chunk &ch, co
   }
 }
 
-// Q8_0: 34-byte blocks, the 8 int8 values of sub-range c (bytes 2+8c..9+8c).
-__device__ __forceinline__ void q80_vals(const uint8_t *blk, int c, uint32_t &lo, uint32_t &hi) {
-  const uint8_t *p = blk + 2 + 8 * c;
-  if ((reinterpret_cast<uintptr_t>(p) & 3u) == 0) {
+// Q8_0: 34-byte block at row offset `o`; the 8 int8 values of sub-range c.
+__device__ __forceinline__ void q80_vals(const uint8_t *row, int o, int c, uint32_t &lo, uint32_t &hi) {
+  const uint8_t *p = row + o + 2 + 8 * c;
+  if (((o + 2) & 3) == 0) {
     lo = lds_u32(p);
     hi = lds_u32(p + 4);
   } else {  // two bytes past a multiple of 4
@@ -486,30 +505,29 @@ __device__ __forceinline__ void q80_vals(const uint8_t *blk, int c, uint32_t &lo
   }
 }
 
-template <int MAXP>
-__device__ __forceinline__ void q80_chunk(const uint8_t *st, const Chunk &ch, const int8_t *const (&bcol)[MAXP],
-                                          int npairs, float (&F)[MAXP][4]) {
+template <int NB, int MAXP, typename BCol>
+__device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol (&bcol)[MAXP], int npairs,
+                                          float (&F)[MAXP][4]) {
+  constexpr int RS = (NB * 34 + 15) / 16 * 16;
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-  const int RS = stage_rs(ch.bpr);
   const uint8_t *row0 = st + r * RS;
-  const uint8_t *row1 = st + (r + 8) * RS;
-  for (int b = 0; b < ch.nb; ++b) {
-    const uint8_t *p0 = row0 + 34 * b;
-    const uint8_t *p1 = row1 + 34 * b;
-    const float d0 = half_bits_to_float(lds_u16(p0));
-    const float d1 = half_bits_to_float(lds_u16(p1));
+  const uint8_t *row1 = row0 + 8 * RS;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const int o = 34 * b;
+    const float d0 = half_bits_to_float(lds_u16(row0 + o));
+    const float d1 = half_bits_to_float(lds_u16(row1 + o));
     uint32_t A[4];
-    q80_vals(p0, c, A[0], A[2]);
-    q80_vals(p1, c, A[1], A[3]);
-    const int kel = ch.k0 + 32 * b + 8 * c;
+    q80_vals(row0, o, c, A[0], A[2]);
+    q80_vals(row1, o, c, A[1], A[3]);
+    const int kel = k0 + 32 * b;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        uint32_t bb0, bb1;
-        load_b(bcol[p], kel, bb0, bb1);
+        const uint2 bb = ldb(bcol[p], kel);
         const int zero[4] = {0, 0, 0, 0};
         int cg[4];
-        mma_s8(cg, A, bb0, bb1, zero);
+        mma_s8(cg, A, bb.x, bb.y, zero);
         F[p][0] = fmaf(d0, (float)cg[0], F[p][0]);
         F[p][1] = fmaf(d0, (float)cg[1], F[p][1]);
         F[p][2] = fmaf(d1, (float)cg[2], F[p][2]);
@@ -522,15 +540,17 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, const Chunk &ch, co
 // Q2_K: value = d*sc*q - dmin*m.  Main term: A = q*sc (exact int8) against
 // the limbs of h.  Min term: A = m (per 16-element sub-block) against the
 // limbs of the 16-element sums of h.
-template <int MAXP>
-__device__ __forceinline__ void q2k_chunk(const uint8_t *st, const Chunk &ch, const int8_t *const (&bcol)[MAXP],
-                                          const int8_t *const (&xcol)[MAXP], int npairs, float (&F)[MAXP][4],
+template <int NB, int MAXP, typename BCol>
+__device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol (&bcol)[MAXP],
+                                          const BCol (&xcol)[MAXP], int npairs, float (&F)[MAXP][4],
                                           float (&G)[MAXP][4]) {
+  constexpr int RS = (NB * 84 + 15) / 16 * 16;
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-  const int RS = stage_rs(ch.bpr);
+  const int cs = 8 * (c >> 1);  // byte of the scale word holding this lane's sub-block, within a pair
   const uint8_t *row0 = st + r * RS;
-  const uint8_t *row1 = st + (r + 8) * RS;
-  for (int b = 0; b < ch.nb; ++b) {
+  const uint8_t *row1 = row0 + 8 * RS;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
     const uint8_t *p0 = row0 + 84 * b;
     const uint8_t *p1 = row1 + 84 * b;
     const uint32_t dd0 = lds_u32(p0 + 80), dd1 = lds_u32(p1 + 80);
@@ -539,30 +559,29 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, const Chunk &ch, co
     int Cm[MAXP][4];
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) Cm[p][0] = Cm[p][1] = Cm[p][2] = Cm[p][3] = 0;
-    const int kb = (ch.k0 >> 8) + b;  // global block index along K
+    const int kb = (k0 >> 8) + b;  // global block index along K
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const uint32_t q00 = lds_u32(p0 + 16 + 32 * hf + 8 * c), q01 = lds_u32(p0 + 20 + 32 * hf + 8 * c);
-      const uint32_t q10 = lds_u32(p1 + 16 + 32 * hf + 8 * c), q11 = lds_u32(p1 + 20 + 32 * hf + 8 * c);
-      const uint32_t s00 = lds_u32(p0 + 8 * hf), s01 = lds_u32(p0 + 8 * hf + 4);
-      const uint32_t s10 = lds_u32(p1 + 8 * hf), s11 = lds_u32(p1 + 8 * hf + 4);
+      const uint2 q0 = *reinterpret_cast<const uint2 *>(p0 + 16 + 32 * hf + 8 * c);
+      const uint2 q1 = *reinterpret_cast<const uint2 *>(p1 + 16 + 32 * hf + 8 * c);
+      const uint2 s0 = *reinterpret_cast<const uint2 *>(p0 + 8 * hf);
+      const uint2 s1 = *reinterpret_cast<const uint2 *>(p1 + 8 * hf);
 #pragma unroll
       for (int sh = 0; sh < 4; ++sh) {
-        const int bsh = 8 * (2 * (sh & 1) + (c >> 1));
-        const uint32_t sc0 = ((sh < 2 ? s00 : s01) >> bsh) & 15u;
-        const uint32_t sc1 = ((sh < 2 ? s10 : s11) >> bsh) & 15u;
+        const int bsh = 16 * (sh & 1) + cs;
+        const uint32_t sc0 = ((sh < 2 ? s0.x : s0.y) >> bsh) & 15u;
+        const uint32_t sc1 = ((sh < 2 ? s1.x : s1.y) >> bsh) & 15u;
         uint32_t A[4];
-        A[0] = ((q00 >> (2 * sh)) & 0x03030303u) * sc0;
-        A[2] = ((q01 >> (2 * sh)) & 0x03030303u) * sc0;
-        A[1] = ((q10 >> (2 * sh)) & 0x03030303u) * sc1;
-        A[3] = ((q11 >> (2 * sh)) & 0x03030303u) * sc1;
-        const int kel = ch.k0 + 256 * b + 128 * hf + 32 * sh + 8 * c;
+        A[0] = ((q0.x >> (2 * sh)) & 0x03030303u) * sc0;
+        A[2] = ((q0.y >> (2 * sh)) & 0x03030303u) * sc0;
+        A[1] = ((q1.x >> (2 * sh)) & 0x03030303u) * sc1;
+        A[3] = ((q1.y >> (2 * sh)) & 0x03030303u) * sc1;
+        const int kel = k0 + 256 * b + 128 * hf + 32 * sh;  // the column base includes 8c
 #pragma unroll
         for (int p = 0; p < MAXP; ++p) {
           if (p < npairs) {
-            uint32_t bb0, bb1;
-            load_b(bcol[p], kel, bb0, bb1);
-            mma_s8(Cm[p], A, bb0, bb1, Cm[p]);
+            const uint2 bb = ldb(bcol[p], kel);
+            mma_s8(Cm[p], A, bb.x, bb.y, Cm[p]);
           }
         }
       }
@@ -577,7 +596,7 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, const Chunk &ch, co
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
         uint32_t bx = 0;
-        if (xcol[p]) bx = *reinterpret_cast<const uint32_t *>(xcol[p] + kb * 16 + 4 * c);
+        if (xcol[p].ok) bx = *reinterpret_cast<const uint32_t *>(xcol[p].p + kb * 16);  // base includes 4c
         const int zero[4] = {0, 0, 0, 0};
         int cn[4];
         mma_s8(cn, Am, bx, 0u, zero);
@@ -755,8 +774,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
   uint8_t *st0 = stages + warp * 2 * kStage2;
   uint8_t *st1 = st0 + kStage2;
   const int r = lane >> 2, c = lane & 3;
+  using BCol = typename std::conditional<XSMEM, BColS, BColG>::type;
+  // column of limb `limb` of token t, offset by this lane's 8-element sub-range
   auto xcol = [&](int t, int limb) -> const int8_t * {
-    return XSMEM ? xsm + (size_t)(t * 3 + limb) * XS : s.xq + ((size_t)t * 3 + limb) * d.H;
+    return (XSMEM ? xsm + (size_t)(t * 3 + limb) * XS : s.xq + ((size_t)t * 3 + limb) * d.H) + 8 * c;
   };
 
   const int tilesI = d.I / 16, tilesS = d.Is / 16;
@@ -764,12 +785,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
   const int n_units = n_sh + S.J.n * tilesI;
   // IQ2 along H: chunks of up to 4 blocks (264 bytes per row)
   const int nbH = d.H / 256;
-  const int cbI = nbH < 4 ? nbH : 4;
+  const int cbI = (nbH % 4 == 0) ? 4 : 1;
   const int nckI = nbH / cbI;
   const size_t rbI = (size_t)nbH * 66;
   // Q8_0 shared: a quarter of H in chunks of up to 8 blocks (272 bytes per row)
   const int nbQ = d.H / 128;
-  const int cbQ = nbQ < 8 ? nbQ : 8;
+  const int cbQ = (nbQ % 8 == 0) ? 8 : 2;
   const int nckQ = nbQ / cbQ;
   const size_t rbQ = (size_t)(d.H / 32) * 34;
 
@@ -784,11 +805,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
       const int tile = u >> 2, q = u & 3;
       const int r0 = tile * 16;
       const int npairs = (T + 1) >> 1;
-      const int8_t *bcol[MAXP];
+      BCol bcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p] = (ts < T && limb < 3) ? xcol(ts, limb) : nullptr;
+        bcol[p].ok = ts < T && limb < 3;
+        bcol[p].p = bcol[p].ok ? xcol(ts, limb) : nullptr;
       }
       float F[2][MAXP][4];
 #pragma unroll
@@ -809,10 +831,18 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
       };
       run_chunks(st0, st1, 2 * nckQ, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        if (i / nckQ == 0)
-          q80_chunk<MAXP>(st, ch, bcol, npairs, F[0]);
-        else
-          q80_chunk<MAXP>(st, ch, bcol, npairs, F[1]);
+        const bool up = i >= nckQ;
+        if (ch.nb == 8) {
+          if (up)
+            q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F[1]);
+          else
+            q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F[0]);
+        } else {
+          if (up)
+            q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F[1]);
+          else
+            q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F[0]);
+        }
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -863,11 +893,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
       const int e = S.J.e[j], ntok = S.J.cnt[j];
       const int *pairs = S.J.pair + S.J.first[j];
       const int npairs = (ntok + 1) >> 1;
-      const int8_t *bcol[MAXP];
+      BCol bcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p] = (ts < ntok && limb < 3) ? xcol(pairs[ts] / d.k, limb) : nullptr;
+        bcol[p].ok = ts < ntok && limb < 3;
+        bcol[p].p = bcol[p].ok ? xcol(pairs[ts] / d.k, limb) : nullptr;
       }
       float F[2][MAXP][4];
 #pragma unroll
@@ -888,10 +919,18 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
       };
       run_chunks(st0, st1, 2 * nckI, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        if (i / nckI == 0)
-          iq2_chunk<MAXP>(st, ch, gpm_l, sel_l, bcol, npairs, F[0]);
-        else
-          iq2_chunk<MAXP>(st, ch, gpm_l, sel_l, bcol, npairs, F[1]);
+        const bool up = i >= nckI;
+        if (ch.nb == 4) {
+          if (up)
+            iq2_chunk<4, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[1]);
+          else
+            iq2_chunk<4, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[0]);
+        } else {
+          if (up)
+            iq2_chunk<1, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[1]);
+          else
+            iq2_chunk<1, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[0]);
+        }
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -952,12 +991,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const int Im16 = s.Imax / 16;
   // Q2_K along I: chunks of up to 4 blocks (336 bytes per row)
   const int nbI = d.I / 256;
-  const int cbD = nbI < 4 ? nbI : 4;
+  const int cbD = (nbI % 4 == 0) ? 4 : 1;
   const int nckD = nbI / cbD;
   const size_t rbD = (size_t)nbI * 84;
   // Q8_0 shared down: a quarter of Is in chunks of up to 8 blocks
   const int nbQ = d.Is / 128;
-  const int cbQ = nbQ < 8 ? nbQ : 8;
+  const int cbQ = (nbQ % 8 == 0) ? 8 : 2;
   const int nckQ = nbQ / cbQ;
   const size_t rbQ = (size_t)(d.Is / 32) * 34;
 
@@ -977,15 +1016,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
       const int e = S.J.e[j], ntok = S.J.cnt[j];
       const int *pairs = S.J.pair + S.J.first[j];
       const int npairs = (ntok + 1) >> 1;
-      const int8_t *bcol[MAXP];
-      const int8_t *xcol[MAXP];
+      BColG bcol[MAXP], xcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
         const bool ok = ts < ntok && limb < 3;
         const int v = ok ? pairs[ts] : 0;
-        bcol[p] = ok ? s.hq + ((size_t)v * 3 + limb) * s.Imax : nullptr;
-        xcol[p] = ok ? s.Xq + ((size_t)v * 3 + limb) * Im16 : nullptr;
+        bcol[p].ok = xcol[p].ok = ok;
+        bcol[p].p = ok ? s.hq + ((size_t)v * 3 + limb) * s.Imax + 8 * c : nullptr;
+        xcol[p].p = ok ? s.Xq + ((size_t)v * 3 + limb) * Im16 + 4 * c : nullptr;
       }
       float F[MAXP][4], G[MAXP][4];
 #pragma unroll
@@ -1005,7 +1044,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
       };
       run_chunks(st0, st1, nckD, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        q2k_chunk<MAXP>(st, ch, bcol, xcol, npairs, F, G);
+        if (ch.nb == 4)
+          q2k_chunk<4, MAXP>(st, ch.k0, bcol, xcol, npairs, F, G);
+        else
+          q2k_chunk<1, MAXP>(st, ch.k0, bcol, xcol, npairs, F, G);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -1038,11 +1080,12 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
     } else {
       const int q = part - S.J.n;
       const int npairs = (T + 1) >> 1;
-      const int8_t *bcol[MAXP];
+      BColG bcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p] = (ts < T && limb < 3) ? s.hq + ((size_t)(T * d.k + ts) * 3 + limb) * s.Imax : nullptr;
+        bcol[p].ok = ts < T && limb < 3;
+        bcol[p].p = bcol[p].ok ? s.hq + ((size_t)(T * d.k + ts) * 3 + limb) * s.Imax + 8 * c : nullptr;
       }
       float F[MAXP][4];
 #pragma unroll
@@ -1060,7 +1103,10 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
       };
       run_chunks(st0, st1, nckQ, chunk_at, [&](int i, uint8_t *st) {
         const Chunk ch = chunk_at(i);
-        q80_chunk<MAXP>(st, ch, bcol, npairs, F);
+        if (ch.nb == 8)
+          q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F);
+        else
+          q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
