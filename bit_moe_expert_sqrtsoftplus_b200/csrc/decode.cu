@@ -37,8 +37,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kWarps2 = 16;  // warps per CTA in k2 / k3
+constexpr int kWarps2 = 16;  // warps per CTA in k2 / k3 (at most)
 constexpr int kThreads2 = kWarps2 * kWarp;
+// k2 threads: 12 warps for four token pairs, whose accumulators need more
+// than the 128 registers a thread has at 16 warps
+__host__ __device__ constexpr int k2_threads(int maxp) { return maxp >= 4 ? 12 * kWarp : kThreads2; }
 constexpr int kStage2 = 16 * 272;      // k2 chunk: 16 rows of <= 272 bytes
 constexpr int kStage3 = 16 * 336;      // k3 chunk: 16 rows of <= 336 bytes
 constexpr int kGpmBytes = 256 * 128;   // +/- codebook, 8 replicas
@@ -73,7 +76,7 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
       a.s.Xmax[i] = 0u;
       a.s.vcount[i] = 0;
     }
-    for (int i = tid; i < d.Is / 16; i += blockDim.x) a.s.shcount[i] = 0;
+    for (int i = tid; i < (1 + a.s.Jmax) * a.s.TM; i += blockDim.x) a.s.hcount[i] = 0;
     for (int i = tid; i < d.H / 16; i += blockDim.x) a.s.ycount[i] = 0;
     if (tid < 4) a.s.work[tid] = 0;
   }
@@ -350,22 +353,50 @@ __host__ __device__ __forceinline__ int piece_for(size_t gstride, size_t off, in
 
 __device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
 
-// Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS).
-// Rows are walked in order; each lane issues the pieces lane, lane + 32, ...
-// of a row (a chunk row is at most 34 pieces).
-__device__ __forceinline__ void stage_chunk(uint8_t *st, const Chunk &c) {
+// Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS) and
+// returns where the chunk's data starts in each staged row.
+//
+// Fast path, when all rows start at the same 8-byte phase of a 16-byte line
+// (row stride a multiple of 16): each row is copied from the 16-byte boundary
+// at or below its start, in 16-byte pieces plus an 8-byte tail, two rows per
+// pass of the warp; the data then starts `shift` (0 or 8) bytes into the
+// staged row.  The bytes before the chunk belong to the same row.
+// Otherwise rows are walked in order and each lane issues the pieces lane,
+// lane + 32, ... of a row in the chunk's own granularity (data at offset 0).
+__device__ __forceinline__ int stage_chunk(uint8_t *st, const Chunk &c) {
   const int lane = threadIdx.x & 31;
   const int RS = stage_rs(c.bpr);
+  const int shift = (int)(reinterpret_cast<uintptr_t>(c.g) & 15);
+  if ((c.gstride & 15) == 0 && (shift & 7) == 0 && shift + c.bpr <= RS && ((shift + c.bpr) & 7) == 0) {
+    const int n16 = (shift + c.bpr) >> 4;
+    const bool tail = ((shift + c.bpr) & 15) != 0;
+    const uint8_t *g0 = c.g - shift;
+    const int half = lane >> 4, l16 = lane & 15;
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+      const int row = 2 * i + half;
+      const uint8_t *gr = g0 + (size_t)row * c.gstride;
+      uint8_t *sr = st + row * RS;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int pc = l16 + 16 * m;
+        if (pc < n16)
+          cp_async16(sr + 16 * pc, gr + 16 * pc);
+        else if (tail && pc == n16)
+          cp_async8(sr + 16 * pc, gr + 16 * pc);
+      }
+    }
+    cp_async_commit();
+    return shift;
+  }
   const int n = c.bpr / c.piece;
   const uint8_t *g = c.g;
   uint8_t *s = st;
   if (c.piece == 8) {
-#pragma unroll 4
     for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
       for (int o = lane; o < n; o += 32) cp_async8(s + 8 * o, g + 8 * o);
     }
   } else if (c.piece == 16) {
-#pragma unroll 4
     for (int row = 0; row < 16; ++row, g += c.gstride, s += RS) {
       for (int o = lane; o < n; o += 32) cp_async16(s + 16 * o, g + 16 * o);
     }
@@ -380,25 +411,28 @@ __device__ __forceinline__ void stage_chunk(uint8_t *st, const Chunk &c) {
     }
   }
   cp_async_commit();
+  return 0;
 }
 
-// Runs a list of chunks through the warp's two-stage ring; `compute(i, st)`
-// consumes chunk i from stage st.
+// Runs a list of chunks through the warp's two-stage ring; `compute(i, data)`
+// consumes chunk i, whose staged rows start at `data` (row stride RS).
 template <typename ChunkAt, typename Compute>
 __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int n, ChunkAt chunk_at,
                                            Compute compute) {
-  stage_chunk(stage0, chunk_at(0));
+  int sh_cur = stage_chunk(stage0, chunk_at(0));
   for (int i = 0; i < n; ++i) {
     uint8_t *cur = (i & 1) ? stage1 : stage0;
     uint8_t *nxt = (i & 1) ? stage0 : stage1;
+    int sh_next = 0;
     if (i + 1 < n)
-      stage_chunk(nxt, chunk_at(i + 1));
+      sh_next = stage_chunk(nxt, chunk_at(i + 1));
     else
       cp_async_commit();
     cp_async_wait<1>();
     __syncwarp();
-    compute(i, cur);
+    compute(i, cur + sh_cur);
     __syncwarp();
+    sh_cur = sh_next;
   }
 }
 
@@ -537,6 +571,13 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol 
   }
 }
 
+// 8 bytes at a 4-byte aligned shared address: one 8-byte load when `al8`
+// (a compile-time constant at every call site), else two 4-byte loads.
+__device__ __forceinline__ uint2 lds_u64_al4(const uint8_t *p, bool al8) {
+  if (al8) return *reinterpret_cast<const uint2 *>(p);
+  return make_uint2(lds_u32(p), lds_u32(p + 4));
+}
+
 // Q2_K: value = d*sc*q - dmin*m.  Main term: A = q*sc (exact int8) against
 // the limbs of h.  Min term: A = m (per 16-element sub-block) against the
 // limbs of the 16-element sums of h.
@@ -562,10 +603,12 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
     const int kb = (k0 >> 8) + b;  // global block index along K
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const uint2 q0 = *reinterpret_cast<const uint2 *>(p0 + 16 + 32 * hf + 8 * c);
-      const uint2 q1 = *reinterpret_cast<const uint2 *>(p1 + 16 + 32 * hf + 8 * c);
-      const uint2 s0 = *reinterpret_cast<const uint2 *>(p0 + 8 * hf);
-      const uint2 s1 = *reinterpret_cast<const uint2 *>(p1 + 8 * hf);
+      // a block at an odd position of the staged row starts 4 (not 8) bytes aligned
+      const bool al8 = ((84 * b) & 7) == 0;
+      const uint2 q0 = lds_u64_al4(p0 + 16 + 32 * hf + 8 * c, al8);
+      const uint2 q1 = lds_u64_al4(p1 + 16 + 32 * hf + 8 * c, al8);
+      const uint2 s0 = lds_u64_al4(p0 + 8 * hf, al8);
+      const uint2 s1 = lds_u64_al4(p1 + 8 * hf, al8);
 #pragma unroll
       for (int sh = 0; sh < 4; ++sh) {
         const int bsh = 16 * (sh & 1) + cs;
@@ -627,22 +670,45 @@ __device__ __forceinline__ void combine_limbs(const float (&F)[4], const float *
   v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
 }
 
-// Three-limb int8 quantisation of n floats with scale max/127.
+// Three-limb int8 quantisation of n floats with scale max/127 (n a multiple
+// of 4; src 16-byte and dst 4-byte aligned).  Every lane takes 4 consecutive
+// elements per step and a batch of steps is loaded before any is used, so
+// the warp waits for memory once per batch rather than once per element.
 __device__ void quantise_vector(const float *src, int n, float vmax, int8_t *dst, int dstride, float *scales) {
   const int lane = threadIdx.x & 31;
   const float s1 = vmax > 0.f ? vmax / 127.f : 1.f;
   const float s2 = s1 / 254.f, s3 = s2 / 254.f;
   const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
-  for (int j = lane; j < n; j += 32) {
-    const float v = __ldcg(src + j);
-    const float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
-    const float e1 = fmaf(-q1, s1, v);
-    const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
-    const float e2 = fmaf(-q2, s2, e1);
-    const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
-    dst[j] = (int8_t)q1;
-    dst[dstride + j] = (int8_t)q2;
-    dst[2 * dstride + j] = (int8_t)q3;
+  constexpr int kBatch = 8;
+  for (int base = 0; base < n; base += 4 * 32 * kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int j = base + 4 * (lane + 32 * i);
+      v[i] = j < n ? __ldcg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int j = base + 4 * (lane + 32 * i);
+      if (j < n) {
+        const float e[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        uint32_t w1 = 0u, w2 = 0u, w3 = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float q1 = fminf(fmaxf(rintf(e[q] * r1), -127.f), 127.f);
+          const float e1 = fmaf(-q1, s1, e[q]);
+          const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+          const float e2 = fmaf(-q2, s2, e1);
+          const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+          w1 |= ((uint32_t)(int)q1 & 255u) << (8 * q);
+          w2 |= ((uint32_t)(int)q2 & 255u) << (8 * q);
+          w3 |= ((uint32_t)(int)q3 & 255u) << (8 * q);
+        }
+        *reinterpret_cast<uint32_t *>(dst + j) = w1;
+        *reinterpret_cast<uint32_t *>(dst + dstride + j) = w2;
+        *reinterpret_cast<uint32_t *>(dst + 2 * dstride + j) = w3;
+      }
+    }
   }
   if (lane == 0) {
     scales[0] = s1;
@@ -735,7 +801,7 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
 // XSMEM: the x limbs of all tokens are staged in shared memory (rows of
 // H + 32 bytes, which spreads the B-fragment loads over all banks).
 template <int MAXP, bool XSMEM>
-__global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
+__global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const LayerDims &d = a.d;
   const DecodeScratch &s = a.s;
@@ -759,7 +825,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
           *reinterpret_cast<const uint4 *>(s.xq + (size_t)rowi * d.H + 16 * o);
     }
   }
-  for (int t = warp; t < T; t += kWarps2) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
+  for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
   __syncthreads();
   if (blockIdx.x == 0) {
     for (int i = tid; i < T * d.k; i += blockDim.x) {
@@ -781,18 +847,15 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
   };
 
   const int tilesI = d.I / 16, tilesS = d.Is / 16;
-  const int n_sh = tilesS * 4;
-  const int n_units = n_sh + S.J.n * tilesI;
-  // IQ2 along H: chunks of up to 4 blocks (264 bytes per row)
-  const int nbH = d.H / 256;
-  const int cbI = (nbH % 4 == 0) ? 4 : 1;
-  const int nckI = nbH / cbI;
-  const size_t rbI = (size_t)nbH * 66;
-  // Q8_0 shared: a quarter of H in chunks of up to 8 blocks (272 bytes per row)
-  const int nbQ = d.H / 128;
-  const int cbQ = (nbQ % 8 == 0) ? 8 : 2;
-  const int nckQ = nbQ / cbQ;
+  const int PH = s.PH;
+  const int kpart = d.H / PH;  // K elements per unit
+  const int cbI = kpart / 256;  // IQ2_XXS blocks per unit: one chunk per matrix
+  const int nq8 = kpart / 256;  // Q8_0 chunks of 8 blocks per unit and matrix
+  const size_t rbI = (size_t)(d.H / 256) * 66;
   const size_t rbQ = (size_t)(d.H / 32) * 34;
+  const int V = T * d.k + T;
+  const int n_sh = tilesS * PH;
+  const int n_units = n_sh + S.J.n * tilesI * PH;
 
   while (true) {
     int u = 0;
@@ -800,157 +863,128 @@ __global__ void __launch_bounds__(kThreads2, 1) k2_gateup(DecodeArgs a) {
     u = __shfl_sync(0xffffffffu, u, 0);
     if (u >= n_units) break;
 
-    if (u < n_sh) {
-      // ---- shared expert: 16-row tile, one K quarter, gate and up
-      const int tile = u >> 2, q = u & 3;
-      const int r0 = tile * 16;
-      const int npairs = (T + 1) >> 1;
-      BCol bcol[MAXP];
+    // ---- unit: (vector set, 16-row tile, K part) of gate and up
+    const bool shared = u < n_sh;
+    int j = 0, tile, part, ntok, e = 0;
+    const int *pairs = nullptr;
+    if (shared) {
+      tile = u / PH;
+      part = u % PH;
+      ntok = T;
+    } else {
+      const int uu = u - n_sh;
+      j = uu / (tilesI * PH);
+      const int rem = uu % (tilesI * PH);
+      tile = rem / PH;
+      part = rem % PH;
+      e = S.J.e[j];
+      ntok = S.J.cnt[j];
+      pairs = S.J.pair + S.J.first[j];
+    }
+    const int r0 = tile * 16;
+    // token slot ts -> row of x / vector of h
+    auto xrow = [&](int ts) { return shared ? ts : pairs[ts] / d.k; };
+    auto hvec = [&](int ts) { return shared ? T * d.k + ts : pairs[ts]; };
+    const int npairs = (ntok + 1) >> 1;
+    BCol bcol[MAXP];
+#pragma unroll
+    for (int p = 0; p < MAXP; ++p) {
+      const int ts = 2 * p + (r >> 2), limb = r & 3;
+      bcol[p].ok = ts < ntok && limb < 3;
+      bcol[p].p = bcol[p].ok ? xcol(xrow(ts), limb) : nullptr;
+    }
+    // F accumulates gate, then up; each matrix's sums of this K part are
+    // combined over limbs and stored as partials (m = 0 gate, 1 up)
+    float F[MAXP][4] = {};
+    auto store_part = [&](int m) {
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
-        const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p].ok = ts < T && limb < 3;
-        bcol[p].p = bcol[p].ok ? xcol(ts, limb) : nullptr;
+        if (p < npairs) {
+          const int ts = 2 * p + (c >> 1);
+          float v0, v1;
+          combine_limbs(F[p], ts < ntok ? s.xs + 4 * xrow(ts) : nullptr, v0, v1);
+          if ((c & 1) == 0 && ts < ntok) {
+            float *pp = s.gpart + ((size_t)(m * PH + part) * V + hvec(ts)) * s.Imax + r0;
+            pp[r] = v0;
+            pp[r + 8] = v1;
+          }
+        }
+        F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
       }
-      float F[2][MAXP][4];
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
+    };
+    auto end_gate = [&]() { store_part(0); };
+    if (shared) {
       auto chunk_at = [&](int i) {
-        const int m = i / nckQ, ck = i % nckQ;
-        const size_t off = (size_t)(q * nbQ + ck * cbQ) * 34;
+        const int m = i / nq8, ck = i % nq8;
+        const size_t off = (size_t)(part * kpart / 32 + ck * 8) * 34;
         Chunk ch;
         ch.g = (m == 0 ? a.wt.sh_gate : a.wt.sh_up) + (size_t)r0 * rbQ + off;
         ch.gstride = rbQ;
-        ch.bpr = cbQ * 34;
-        ch.nb = cbQ;
-        ch.k0 = (q * nbQ + ck * cbQ) * 32;
+        ch.bpr = 8 * 34;
+        ch.nb = 8;
+        ch.k0 = part * kpart + ck * 256;
         ch.piece = piece_for(rbQ, off, ch.bpr);
         return ch;
       };
-      run_chunks(st0, st1, 2 * nckQ, chunk_at, [&](int i, uint8_t *st) {
-        const Chunk ch = chunk_at(i);
-        const bool up = i >= nckQ;
-        if (ch.nb == 8) {
-          if (up)
-            q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F[1]);
-          else
-            q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F[0]);
-        } else {
-          if (up)
-            q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F[1]);
-          else
-            q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F[0]);
-        }
+      run_chunks(st0, st1, 2 * nq8, chunk_at, [&](int i, uint8_t *st) {
+        q80_chunk<8, MAXP>(st, part * kpart + (i % nq8) * 256, bcol, npairs, F);
+        if (i == nq8 - 1) end_gate();
       });
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
-          const int ts = 2 * p + (c >> 1);
-          const float *sc = ts < T ? s.xs + 4 * ts : nullptr;
-          float g0, g1, u0, u1;
-          combine_limbs(F[0][p], sc, g0, g1);
-          combine_limbs(F[1][p], sc, u0, u1);
-          if ((c & 1) == 0 && ts < T) {
-            float *pg = s.shpart + ((size_t)(0 * 4 + q) * T + ts) * d.Is + r0;
-            float *pu = s.shpart + ((size_t)(1 * 4 + q) * T + ts) * d.Is + r0;
-            pg[r] = g0;
-            pg[r + 8] = g1;
-            pu[r] = u0;
-            pu[r + 8] = u1;
-          }
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = atomicAdd(s.shcount + tile, 1) == 3;
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        for (int i = lane; i < 16 * T; i += 32) {
-          const int ts = i >> 4, row = i & 15;
-          float ga = 0.f, ub = 0.f;
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            ga += __ldcg(s.shpart + ((size_t)(0 * 4 + qq) * T + ts) * d.Is + r0 + row);
-            ub += __ldcg(s.shpart + ((size_t)(1 * 4 + qq) * T + ts) * d.Is + r0 + row);
-          }
-          S.hsm[warp][ts][row] = silu(ga) * ub;
-        }
-        __syncwarp();
-        int vec[kDecodeMaxT];
-#pragma unroll
-        for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = T * d.k + t;
-        finish_h_tile(a, S.hsm[warp], T, vec, r0, d.Is, tilesS);
-      }
     } else {
-      // ---- routed expert: 16-row tile of gate and up, full K
-      const int uu = u - n_sh;
-      const int j = uu / tilesI, tile = uu % tilesI;
-      const int r0 = tile * 16;
-      const int e = S.J.e[j], ntok = S.J.cnt[j];
-      const int *pairs = S.J.pair + S.J.first[j];
-      const int npairs = (ntok + 1) >> 1;
-      BCol bcol[MAXP];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p].ok = ts < ntok && limb < 3;
-        bcol[p].p = bcol[p].ok ? xcol(pairs[ts] / d.k, limb) : nullptr;
-      }
-      float F[2][MAXP][4];
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int p = 0; p < MAXP; ++p) F[m][p][0] = F[m][p][1] = F[m][p][2] = F[m][p][3] = 0.f;
       auto chunk_at = [&](int i) {
-        const int m = i / nckI, ck = i % nckI;
-        const size_t off = (size_t)ck * cbI * 66;
+        const size_t off = (size_t)part * cbI * 66;
         Chunk ch;
-        ch.g = (m == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + off;
+        ch.g = (i == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + off;
         ch.gstride = rbI;
         ch.bpr = cbI * 66;
         ch.nb = cbI;
-        ch.k0 = ck * cbI * 256;
+        ch.k0 = part * kpart;
         ch.piece = piece_for(rbI, off, ch.bpr);
         return ch;
       };
-      run_chunks(st0, st1, 2 * nckI, chunk_at, [&](int i, uint8_t *st) {
-        const Chunk ch = chunk_at(i);
-        const bool up = i >= nckI;
-        if (ch.nb == 4) {
-          if (up)
-            iq2_chunk<4, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[1]);
-          else
-            iq2_chunk<4, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[0]);
-        } else {
-          if (up)
-            iq2_chunk<1, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[1]);
-          else
-            iq2_chunk<1, MAXP>(st, ch.k0, gpm_l, sel_l, bcol, npairs, F[0]);
-        }
+      run_chunks(st0, st1, 2, chunk_at, [&](int i, uint8_t *st) {
+        if (cbI == 4)
+          iq2_chunk<4, MAXP>(st, part * kpart, gpm_l, sel_l, bcol, npairs, F);
+        else
+          iq2_chunk<1, MAXP>(st, part * kpart, gpm_l, sel_l, bcol, npairs, F);
+        if (i == 0) end_gate();
       });
+    }
+    store_part(1);
+    __threadfence();
+    __syncwarp();
+    const int set = shared ? 0 : 1 + j;
+    int last = 0;
+    if (lane == 0) last = atomicAdd(s.hcount + set * s.TM + tile, 1) == PH - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      // every K part of the tile is in: sum them in part order, SwiGLU
+      __threadfence();
+      for (int i = lane; i < 16 * ntok; i += 32) {
+        const int ts = i >> 4, row = i & 15;
+        const int v = hvec(ts);
+        float ga = 0.f, ub = 0.f;
+        for (int p0 = 0; p0 < PH; p0 += 4) {  // loads of a batch are independent; sums keep part order
+          float gb[4], ubb[4];
 #pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
-          const int ts = 2 * p + (c >> 1);
-          const float *sc = ts < ntok ? s.xs + 4 * (pairs[ts] / d.k) : nullptr;
-          float g0, g1, u0, u1;
-          combine_limbs(F[0][p], sc, g0, g1);
-          combine_limbs(F[1][p], sc, u0, u1);
-          if ((c & 1) == 0 && ts < ntok) {
-            S.hsm[warp][ts][r] = silu(g0) * u0;
-            S.hsm[warp][ts][r + 8] = silu(g1) * u1;
+          for (int q = 0; q < 4; ++q) {
+            const bool in = p0 + q < PH;
+            gb[q] = in ? __ldcg(s.gpart + ((size_t)(0 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
+            ubb[q] = in ? __ldcg(s.gpart + ((size_t)(1 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            ga += gb[q];
+            ub += ubb[q];
           }
         }
+        S.hsm[warp][ts][row] = silu(ga) * ub;
       }
       __syncwarp();
       int vec[kDecodeMaxT];
 #pragma unroll
-      for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < ntok ? pairs[t] : 0;
-      finish_h_tile(a, S.hsm[warp], ntok, vec, r0, d.I, tilesI);
+      for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < ntok ? hvec(t) : 0;
+      finish_h_tile(a, S.hsm[warp], ntok, vec, r0, shared ? d.Is : d.I, shared ? tilesS : tilesI);
     }
     __syncwarp();
   }
@@ -962,10 +996,14 @@ struct K3Shared {
   int32_t idx[kDecodeMaxT * kMaxK];
   float w[kDecodeMaxT * kMaxK];
   Jobs J;
-  float ysm[kWarps2][kDecodeMaxT][16];
 };
 
-template <int MAXP>
+// Shared-memory rows of the h limbs (HSMEM): Imax + 32 bytes per limb row of
+// h and Imax/16 + 16 bytes per limb row of the 16-element sums.
+__host__ __device__ inline size_t k3_hrow(int Imax) { return (size_t)Imax + 32; }
+__host__ __device__ inline size_t k3_xrow(int Imax) { return (size_t)Imax / 16 + 16; }
+
+template <int MAXP, bool HSMEM>
 __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const LayerDims &d = a.d;
@@ -973,11 +1011,29 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const int T = a.T;
   uint8_t *stages = smem;
   K3Shared &S = *reinterpret_cast<K3Shared *>(stages + 2 * kWarps2 * kStage3);
+  int8_t *hsm = reinterpret_cast<int8_t *>(reinterpret_cast<uint8_t *>(&S) + align_up(sizeof(K3Shared), 128));
+  const int V = T * d.k + T;
+  const int Im16 = s.Imax / 16;
+  const size_t HR = k3_hrow(s.Imax), XR = k3_xrow(s.Imax);
+  int8_t *xsm = hsm + (size_t)V * 3 * HR;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();  // k2's routing and h limbs are visible from here on
   for (int i = tid; i < T * d.k; i += blockDim.x) {
     S.idx[i] = s.idx[i];
     S.w[i] = s.w[i];
+  }
+  if (HSMEM) {
+    const int n16 = s.Imax / 16;
+    for (int i = tid; i < V * 3 * n16; i += blockDim.x) {
+      const int rowi = i / n16, o = i - rowi * n16;
+      *reinterpret_cast<uint4 *>(hsm + (size_t)rowi * HR + 16 * o) =
+          __ldcg(reinterpret_cast<const uint4 *>(s.hq + (size_t)rowi * s.Imax + 16 * o));
+    }
+    for (int i = tid; i < V * 3 * Im16 / 4; i += blockDim.x) {
+      const int rowi = i / (Im16 / 4), o = i - rowi * (Im16 / 4);
+      *reinterpret_cast<uint32_t *>(xsm + (size_t)rowi * XR + 4 * o) =
+          __ldcg(reinterpret_cast<const unsigned *>(s.Xq + (size_t)rowi * Im16 + 4 * o));
+    }
   }
   __syncthreads();
   build_jobs(S.idx, T, d.k, S.J);
@@ -985,20 +1041,26 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   uint8_t *st0 = stages + warp * 2 * kStage3;
   uint8_t *st1 = st0 + kStage3;
   const int r = lane >> 2, c = lane & 3;
+  using BCol = typename std::conditional<HSMEM, BColS, BColG>::type;
+  // limb `limb` of vector v (h, and its 16-element sums), offset by this lane's sub-range
+  auto hcol = [&](int v, int limb) -> const int8_t * {
+    return (HSMEM ? hsm + ((size_t)v * 3 + limb) * HR : s.hq + ((size_t)v * 3 + limb) * s.Imax) + 8 * c;
+  };
+  auto Xcol = [&](int v, int limb) -> const int8_t * {
+    return (HSMEM ? xsm + ((size_t)v * 3 + limb) * XR : s.Xq + ((size_t)v * 3 + limb) * Im16) + 4 * c;
+  };
   const int tilesH = d.H / 16;
-  const int nparts = S.J.n + 4;
-  const int n_units = tilesH * nparts;
-  const int Im16 = s.Imax / 16;
-  // Q2_K along I: chunks of up to 4 blocks (336 bytes per row)
-  const int nbI = d.I / 256;
-  const int cbD = (nbI % 4 == 0) ? 4 : 1;
-  const int nckD = nbI / cbD;
-  const size_t rbD = (size_t)nbI * 84;
-  // Q8_0 shared down: a quarter of Is in chunks of up to 8 blocks
-  const int nbQ = d.Is / 128;
-  const int cbQ = (nbQ % 8 == 0) ? 8 : 2;
-  const int nckQ = nbQ / cbQ;
+  const int PD = s.PD, PS = s.PS;
+  const int kpd = d.I / PD;      // K elements of a routed unit
+  const int cbD = kpd / 256;     // Q2_K blocks per routed unit: one chunk
+  const int kps = d.Is / PS;     // K elements of a shared unit
+  const int nq8 = kps / 256;     // Q8_0 chunks of 8 blocks per shared unit
+  const size_t rbD = (size_t)(d.I / 256) * 84;
   const size_t rbQ = (size_t)(d.Is / 32) * 34;
+  const int nrp = S.J.n * PD;    // routed parts of an output tile
+  const int nparts = nrp + PS;
+  const int n_units = tilesH * nparts;
+  const int NS = s.NS;
 
   while (true) {
     int u = 0;
@@ -1007,47 +1069,40 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
     if (u >= n_units) break;
     const int ot = u / nparts, part = u % nparts;
     const int r0 = ot * 16;
-    float(*ys)[16] = S.ysm[warp];
-    for (int i = lane; i < kDecodeMaxT * 16; i += 32) ys[i >> 4][i & 15] = 0.f;
-    __syncwarp();
+    float *ytile = s.ypart + (size_t)ot * NS * 16;
 
-    if (part < S.J.n) {
-      const int j = part;
+    if (part < nrp) {
+      // ---- routed: expert j, K part kp of I
+      const int j = part / PD, kp = part % PD;
       const int e = S.J.e[j], ntok = S.J.cnt[j];
       const int *pairs = S.J.pair + S.J.first[j];
       const int npairs = (ntok + 1) >> 1;
-      BColG bcol[MAXP], xcol[MAXP];
+      BCol bcol[MAXP], xcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
         const bool ok = ts < ntok && limb < 3;
-        const int v = ok ? pairs[ts] : 0;
         bcol[p].ok = xcol[p].ok = ok;
-        bcol[p].p = ok ? s.hq + ((size_t)v * 3 + limb) * s.Imax + 8 * c : nullptr;
-        xcol[p].p = ok ? s.Xq + ((size_t)v * 3 + limb) * Im16 + 4 * c : nullptr;
+        bcol[p].p = ok ? hcol(pairs[ts], limb) : nullptr;
+        xcol[p].p = ok ? Xcol(pairs[ts], limb) : nullptr;
       }
-      float F[MAXP][4], G[MAXP][4];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
-      auto chunk_at = [&](int i) {
-        const size_t off = (size_t)i * cbD * 84;
+      float F[MAXP][4] = {}, G[MAXP][4] = {};
+      auto chunk_at = [&](int) {
+        const size_t off = (size_t)kp * cbD * 84;
         Chunk ch;
         ch.g = a.wt.down + ((size_t)e * d.H + r0) * rbD + off;
         ch.gstride = rbD;
         ch.bpr = cbD * 84;
         ch.nb = cbD;
-        ch.k0 = i * cbD * 256;
+        ch.k0 = kp * kpd;
         ch.piece = piece_for(rbD, off, ch.bpr);
         return ch;
       };
-      run_chunks(st0, st1, nckD, chunk_at, [&](int i, uint8_t *st) {
-        const Chunk ch = chunk_at(i);
-        if (ch.nb == 4)
-          q2k_chunk<4, MAXP>(st, ch.k0, bcol, xcol, npairs, F, G);
+      run_chunks(st0, st1, 1, chunk_at, [&](int, uint8_t *st) {
+        if (cbD == 4)
+          q2k_chunk<4, MAXP>(st, kp * kpd, bcol, xcol, npairs, F, G);
         else
-          q2k_chunk<1, MAXP>(st, ch.k0, bcol, xcol, npairs, F, G);
+          q2k_chunk<1, MAXP>(st, kp * kpd, bcol, xcol, npairs, F, G);
       });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
@@ -1070,44 +1125,38 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
           v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
           v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
           if ((c & 1) == 0 && ok) {
-            const int t = v / d.k;
             const float wt = S.w[v];
-            ys[t][r] = wt * v0;
-            ys[t][r + 8] = wt * v1;
+            float *dst = ytile + (size_t)(v * PD + kp) * 16;
+            dst[r] = wt * v0;
+            dst[r + 8] = wt * v1;
           }
         }
       }
     } else {
-      const int q = part - S.J.n;
+      // ---- shared: K part q of Is
+      const int q = part - nrp;
       const int npairs = (T + 1) >> 1;
-      BColG bcol[MAXP];
+      BCol bcol[MAXP];
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         const int ts = 2 * p + (r >> 2), limb = r & 3;
         bcol[p].ok = ts < T && limb < 3;
-        bcol[p].p = bcol[p].ok ? s.hq + ((size_t)(T * d.k + ts) * 3 + limb) * s.Imax + 8 * c : nullptr;
+        bcol[p].p = bcol[p].ok ? hcol(T * d.k + ts, limb) : nullptr;
       }
-      float F[MAXP][4];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
+      float F[MAXP][4] = {};
       auto chunk_at = [&](int i) {
         Chunk ch;
-        const size_t off = (size_t)(q * nbQ + i * cbQ) * 34;
+        const size_t off = (size_t)(q * kps / 32 + i * 8) * 34;
         ch.g = a.wt.sh_down + (size_t)r0 * rbQ + off;
         ch.gstride = rbQ;
-        ch.bpr = cbQ * 34;
-        ch.nb = cbQ;
-        ch.k0 = (q * nbQ + i * cbQ) * 32;
+        ch.bpr = 8 * 34;
+        ch.nb = 8;
+        ch.k0 = q * kps + i * 256;
         ch.piece = piece_for(rbQ, off, ch.bpr);
         return ch;
       };
-      run_chunks(st0, st1, nckQ, chunk_at, [&](int i, uint8_t *st) {
-        const Chunk ch = chunk_at(i);
-        if (ch.nb == 8)
-          q80_chunk<8, MAXP>(st, ch.k0, bcol, npairs, F);
-        else
-          q80_chunk<2, MAXP>(st, ch.k0, bcol, npairs, F);
-      });
+      run_chunks(st0, st1, nq8, chunk_at,
+                 [&](int i, uint8_t *st) { q80_chunk<8, MAXP>(st, q * kps + i * 256, bcol, npairs, F); });
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
         if (p < npairs) {
@@ -1116,27 +1165,38 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
           float v0, v1;
           combine_limbs(F[p], sc, v0, v1);
           if ((c & 1) == 0 && ts < T) {
-            ys[ts][r] = v0;
-            ys[ts][r + 8] = v1;
+            float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + q) * 16;
+            dst[r] = v0;
+            dst[r + 8] = v1;
           }
         }
       }
     }
-    __syncwarp();
-    // part -> global, the last part of the tile writes y
-    float *dst = s.ypart + ((size_t)ot * s.P + part) * T * 16;
-    for (int i = lane; i < 16 * T; i += 32) dst[i] = ys[i >> 4][i & 15];
     __threadfence();
     __syncwarp();
     int last = 0;
     if (lane == 0) last = atomicAdd(s.ycount + ot, 1) == nparts - 1;
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
+      // every part of the tile is in: sum them in a fixed order into y
       __threadfence();
       for (int i = lane; i < 16 * T; i += 32) {
         const int t = i >> 4, row = i & 15;
         float acc = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[(size_t)t * d.H + r0 + row] : 0.f;
-        for (int pp = 0; pp < nparts; ++pp) acc += __ldcg(s.ypart + ((size_t)ot * s.P + pp) * T * 16 + i);
+        // slots in a fixed order: the token's routed parts, then its shared parts;
+        // the loads of a batch are independent
+        const int nr = d.k * PD, ns = nr + PS;
+        for (int s0 = 0; s0 < ns; s0 += 8) {
+          float vb[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int sl = s0 + q;
+            const size_t slot = sl < nr ? (size_t)t * nr + sl : (size_t)T * nr + (size_t)t * PS + (sl - nr);
+            vb[q] = sl < ns ? __ldcg(ytile + slot * 16 + row) : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc += vb[q];
+        }
         a.y[(size_t)t * d.H + r0 + row] = acc;
       }
     }
@@ -1157,7 +1217,11 @@ size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
   if (xsmem) b += (size_t)T * 3 * (d.H + 32);
   return b;
 }
-size_t k3_smem_bytes() { return 2 * kWarps2 * kStage3 + sizeof(K3Shared); }
+size_t k3_smem_bytes(const DecodeScratch &s, int T, int k, bool hsmem) {
+  size_t b = 2 * kWarps2 * kStage3 + align_up(sizeof(K3Shared), 128);
+  if (hsmem) b += (size_t)(T * k + T) * 3 * (k3_hrow(s.Imax) + k3_xrow(s.Imax));
+  return b;
+}
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -1176,22 +1240,23 @@ cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int MAXP, bool XSMEM>
+template <int MAXP, bool XSMEM, bool HSMEM>
 cudaError_t launch_k23(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(k2_gateup<MAXP, XSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemLimit);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k3_down<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k3_smem_bytes());
+    e = cudaFuncSetAttribute(k3_down<MAXP, HSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
-  cudaError_t e = launch_pdl(k2_gateup<MAXP, XSMEM>, num_sms, kThreads2, k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
+  cudaError_t e =
+      launch_pdl(k2_gateup<MAXP, XSMEM>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
   if (e != cudaSuccess) return e;
   if (a.ev_end) cudaEventRecord(a.ev_end, stream);
-  return launch_pdl(k3_down<MAXP>, num_sms, kThreads2, k3_smem_bytes(), stream, a);
+  return launch_pdl(k3_down<MAXP, HSMEM>, num_sms, kThreads2, k3_smem_bytes(a.s, a.T, a.d.k, HSMEM), stream, a);
 }
 
 cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
@@ -1219,7 +1284,6 @@ size_t decode_scratch_bytes(const LayerDims &d, int T) {
 void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   const int V = T * d.k + T;
   const int Imax = d.I > d.Is ? d.I : d.Is;
-  const int P = (T * d.k < d.E ? T * d.k : d.E) + 4;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     off = align_up(off, 256);
@@ -1228,7 +1292,12 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
     return p;
   };
   s.Imax = Imax;
-  s.P = P;
+  s.PH = decode_kparts(d.H);
+  s.PD = decode_kparts(d.I);
+  s.PS = decode_kparts(d.Is);
+  s.Jmax = T * d.k < d.E ? T * d.k : d.E;
+  s.TM = Imax / 16;
+  s.NS = T * d.k * s.PD + T * s.PS;
   s.z = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.sc = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * T * d.k));
@@ -1244,9 +1313,9 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.hmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
   s.Xmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
   s.vcount = reinterpret_cast<int *>(take(sizeof(int) * V));
-  s.shpart = reinterpret_cast<float *>(take(sizeof(float) * 2 * 4 * (size_t)T * d.Is));
-  s.shcount = reinterpret_cast<int *>(take(sizeof(int) * (d.Is / 16)));
-  s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * P * T * 16));
+  s.gpart = reinterpret_cast<float *>(take(sizeof(float) * 2 * (size_t)s.PH * V * Imax));
+  s.hcount = reinterpret_cast<int *>(take(sizeof(int) * (size_t)(1 + s.Jmax) * s.TM));
+  s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * s.NS * 16));
   s.ycount = reinterpret_cast<int *>(take(sizeof(int) * (d.H / 16)));
   s.work = reinterpret_cast<int *>(take(sizeof(int) * 4));
 }
@@ -1255,11 +1324,14 @@ cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms
   cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
   if (a.T <= 2) {
-    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k23<1, true>(a, stream, num_sms);
-    return launch_k23<1, false>(a, stream, num_sms);
+    const bool xs = k2_smem_bytes(a.d, a.T, true) <= kSmemLimit;
+    const bool hs = k3_smem_bytes(a.s, a.T, a.d.k, true) <= kSmemLimit;
+    if (xs && hs) return launch_k23<1, true, true>(a, stream, num_sms);
+    if (xs) return launch_k23<1, true, false>(a, stream, num_sms);
+    return launch_k23<1, false, false>(a, stream, num_sms);
   }
-  if (a.T <= 4) return launch_k23<2, false>(a, stream, num_sms);
-  return launch_k23<4, false>(a, stream, num_sms);
+  if (a.T <= 4) return launch_k23<2, false, false>(a, stream, num_sms);
+  return launch_k23<4, false, false>(a, stream, num_sms);
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {

@@ -1,14 +1,14 @@
 // gemm.cu -- persistent, warp-specialised grouped GEMM on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory).
 //
-// One CTA per SM, 13 warps:
+// One CTA per SM, 21 warps:
 //   warps 0-3   epilogue: tcgen05.ld of the 128-lane accumulator, SwiGLU /
 //               scatter-add / store
-//   warps 4-11  producers: dequantise the 128 x 64 weight tile(s) of a K step
+//   warps 4-19  producers: dequantise the 128 x 64 weight tile(s) of a K step
 //               into 16-bit values written straight into the 128-byte-swizzled
 //               K-major operand layout, and gather the N x 64 activation tile
 //               with cp.async
-//   warp 12     allocates tensor memory and issues tcgen05.mma (one thread)
+//   warp 20     allocates tensor memory and issues tcgen05.mma (one thread)
 // Shared memory holds a ring of stages (A tile(s) + B tile); mbarriers carry
 // full/empty hand-offs between producers and the MMA thread and
 // full/empty hand-offs of the accumulator between the MMA thread and the
@@ -31,10 +31,13 @@ namespace moe {
 namespace {
 
 constexpr int kEpiWarps = 4;
-constexpr int kProdWarps = 8;
-constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 12
-constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 416
-constexpr int kProd = kProdWarps * 32;             // 256 producer threads
+constexpr int kProdWarps = 16;
+constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 20
+constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 672
+constexpr int kProd = kProdWarps * 32;             // 512 producer threads
+constexpr int kGridRep = 4;                        // replicas of the f16 codebook table
+constexpr int kSignRep = 4;                        // replicas of the sign-mask table
+constexpr int kAhead = 3;                          // K steps of packed weights fetched ahead
 constexpr int BM = 128, BK = 64, BN = 256;
 constexpr int kATile = BM * BK * 2;  // 16 KB
 constexpr int kBTile = BN * BK * 2;  // 32 KB
@@ -185,7 +188,7 @@ struct Raw<kFmtIQ2> {
 };
 template <>
 struct Raw<kFmtQ2K> {
-  uint32_t dd, scw, q[8];
+  uint32_t dd, sb, q[4];
 };
 template <>
 struct Raw<kFmtQ80> {
@@ -216,8 +219,8 @@ __device__ __forceinline__ void decode(const Raw<kFmtIQ2> &r, uint8_t *tile, int
   for (int j = 0; j < 4; ++j) {
     const uint32_t ix = (r.idx4 >> (8 * j)) & 255u;
     const uint32_t m7 = (r.S >> (7 * j)) & 127u;
-    const uint4 g = *reinterpret_cast<const uint4 *>(gridh + ix * 16u);
-    const uint4 sm = *reinterpret_cast<const uint4 *>(signm + m7 * 16u);
+    const uint4 g = *reinterpret_cast<const uint4 *>(gridh + ix * (16u * kGridRep));
+    const uint4 sm = *reinterpret_cast<const uint4 *>(signm + m7 * (16u * kSignRep));
     const uint32_t o0 = h2bits(__hmul2(__hmul2(bits2h(g.x ^ sm.x), f2), d2));
     const uint32_t o1 = h2bits(__hmul2(__hmul2(bits2h(g.y ^ sm.y), f2), d2));
     const uint32_t o2 = h2bits(__hmul2(__hmul2(bits2h(g.z ^ sm.z), f2), d2));
@@ -231,40 +234,39 @@ __device__ __forceinline__ uint32_t bf16pair(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Q2_K: the K step covers 64 elements of block ks/4; item = which of its two shifts.
+// Q2_K: the K step covers 64 elements of block ks/4 (two shifts of one half);
+// item (0..3) = shift (item >> 1) and 16-element sub-block (item & 1) of it.
 __device__ __forceinline__ void fetch(Raw<kFmtQ2K> &r, const uint8_t *rowp, int ks, int item) {
   const int blk = ks >> 2, qq = ks & 3;
   const uint8_t *bp = rowp + (size_t)blk * 84;
-  const int hf = qq >> 1, sh = 2 * (qq & 1) + item;
+  const int hf = qq >> 1, sh = 2 * (qq & 1) + (item >> 1), sub = item & 1;
   r.dd = ldg32(bp + 80);
-  r.scw = ldg16(bp + 8 * hf + 2 * sh);  // scale bytes of sub-blocks 8hf+2sh, +1
+  r.sb = bp[8 * hf + 2 * sh + sub];  // scale/min byte of the sub-block
 #pragma unroll
-  for (int i = 0; i < 8; ++i) r.q[i] = ldg32(bp + 16 + 32 * hf + 4 * i);
+  for (int i = 0; i < 4; ++i) r.q[i] = ldg32(bp + 16 + 32 * hf + 16 * sub + 4 * i);
 }
 
 __device__ __forceinline__ void decode(const Raw<kFmtQ2K> &r, uint8_t *tile, int row, int item, int ks,
                                        const uint8_t *, const uint8_t *) {
-  const int sh = 2 * (ks & 1) + item;
+  const int sh = 2 * (ks & 1) + (item >> 1), sub = item & 1;
   const float d = __half2float(__ushort_as_half((unsigned short)(r.dd & 0xFFFFu)));
   const float dmin = __half2float(__ushort_as_half((unsigned short)(r.dd >> 16)));
+  const float dsc = d * (float)(r.sb & 15u);
+  const float mn = -dmin * (float)(r.sb >> 4);
+  const uint32_t V0 = bf16pair(mn, fmaf(dsc, 1.f, mn));
+  const uint32_t V1 = bf16pair(fmaf(dsc, 2.f, mn), fmaf(dsc, 3.f, mn));
+  uint32_t o[8];
 #pragma unroll
-  for (int sub = 0; sub < 2; ++sub) {
-    const uint32_t sb = (r.scw >> (8 * sub)) & 0xFFu;
-    const float dsc = d * (float)(sb & 15u);
-    const float mn = -dmin * (float)(sb >> 4);
-    const uint32_t V0 = bf16pair(mn, fmaf(dsc, 1.f, mn));
-    const uint32_t V1 = bf16pair(fmaf(dsc, 2.f, mn), fmaf(dsc, 3.f, mn));
-    uint32_t o[8];
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-      const uint32_t q = (r.q[4 * sub + wi] >> (2 * sh)) & 0x03030303u;
-      const uint32_t t = q * 0x22u + 0x10101010u;
-      o[2 * wi] = __byte_perm(V0, V1, t & 0xFFFFu);
-      o[2 * wi + 1] = __byte_perm(V0, V1, t >> 16);
-    }
-    sts128(swz(tile, row, 4 * item + 2 * sub), o[0], o[1], o[2], o[3]);
-    sts128(swz(tile, row, 4 * item + 2 * sub + 1), o[4], o[5], o[6], o[7]);
+  for (int wi = 0; wi < 4; ++wi) {
+    const uint32_t q = (r.q[wi] >> (2 * sh)) & 0x03030303u;
+    const uint32_t t = q * 0x22u + 0x10101010u;
+    o[2 * wi] = __byte_perm(V0, V1, t & 0xFFFFu);
+    o[2 * wi + 1] = __byte_perm(V0, V1, t >> 16);
   }
+  // elements 32*(shift in the step) + 16*sub .. +15 of the 64-element step
+  const int chunk = 4 * (item >> 1) + 2 * sub;
+  sts128(swz(tile, row, chunk), o[0], o[1], o[2], o[3]);
+  sts128(swz(tile, row, chunk + 1), o[4], o[5], o[6], o[7]);
 }
 
 // Q8_0: 32-element block (kel/32) of the row.
@@ -335,9 +337,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stages = smem;
-  uint8_t *gridh = stages + S * STAGE;  // 256 x 16 B: codebook as f16
-  uint8_t *signm = gridh + 4096;        // 128 x 16 B: f16 sign masks per 7-bit mask
-  GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + 2048);
+  uint8_t *gridh = stages + S * STAGE;          // 256 x kGridRep x 16 B: codebook as f16
+  uint8_t *signm = gridh + 4096 * kGridRep;     // 128 x kSignRep x 16 B: f16 sign masks
+  GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + 2048 * kSignRep);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_tiles = a.M / BM;
@@ -371,13 +373,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     ctl.total_tiles = pre;
   }
   if (FMT == kFmtIQ2) {
-    for (int i = tid; i < 256 * 8; i += blockDim.x) {  // codebook -> f16
-      const int ix = i >> 3, l = i & 7;
-      reinterpret_cast<__half *>(gridh)[ix * 8 + l] = __int2half_rn(a.grid[ix * 8 + l]);
+    for (int i = tid; i < 256 * 8 * kGridRep; i += blockDim.x) {  // codebook -> f16
+      const int l = i & 7, rep = (i >> 3) % kGridRep, ix = (i >> 3) / kGridRep;
+      reinterpret_cast<__half *>(gridh)[(ix * kGridRep + rep) * 8 + l] = __int2half_rn(a.grid[ix * 8 + l]);
     }
-    for (int m7 = tid; m7 < 128; m7 += blockDim.x) {
+    for (int i = tid; i < 128 * kSignRep; i += blockDim.x) {
+      const int m7 = i / kSignRep, rep = i % kSignRep;
       const uint32_t m8 = (uint32_t)m7 | ((uint32_t)(__popc(m7) & 1) << 7);
-      uint32_t *e = reinterpret_cast<uint32_t *>(signm + m7 * 16);
+      uint32_t *e = reinterpret_cast<uint32_t *>(signm + (m7 * kSignRep + rep) * 16);
 #pragma unroll
       for (int p = 0; p < 4; ++p)
         e[p] = (((m8 >> (2 * p)) & 1u) << 15) | (((m8 >> (2 * p + 1)) & 1u) << 31);
@@ -397,15 +400,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   if (warp >= kEpiWarps && warp < kMmaWarp) {
     // =================================================== producers
     const int p = tid - kEpiWarps * 32;
+    const uint8_t *gridh_l = gridh + 16 * (lane % kGridRep);
+    const uint8_t *signm_l = signm + 16 * (lane % kSignRep);
     uint32_t it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile tl = tile_at(ctl, t, m_tiles);
-      // B rows this thread copies: rows (p >> 3) + 32 i, chunk p & 7
+      // B rows this thread copies: rows (p >> 3) + 64 i, chunk p & 7
       const int ch = p & 7;
-      const uint16_t *brow[8];
+      const uint16_t *brow[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = (p >> 3) + 32 * i;
+      for (int i = 0; i < 4; ++i) {
+        const int r = (p >> 3) + 64 * i;
         brow[i] = nullptr;
         if (r < tl.nt) {
           const int c = tl.col0 + r;
@@ -413,55 +418,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
           brow[i] = a.b_base + (size_t)br * a.b_ld + ch * 8;
         }
       }
-      // A items: row p/2, 32-element half p%2 of the 64-element K step
-      const int row = p >> 1, item = p & 1;
-      const uint8_t *arow[2];
-      arow[0] = a.A0 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
-      arow[1] = PAIRED ? a.A1 + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row) : arow[0];
+      // A item of this thread: paired formats: matrix p/256, row (p/2)%128, 32-element half p%2;
+      // Q2_K: row p/4, item p%4 (16 elements); unpaired Q8_0: row p/2, half p%2 (threads < 256)
+      const int mat = PAIRED ? (p >> 8) : 0;
+      const int row = FMT == kFmtQ2K ? (p >> 2) : ((p >> 1) & 127);
+      const int item = FMT == kFmtQ2K ? (p & 3) : (p & 1);
+      const bool has_a = PAIRED || FMT == kFmtQ2K || p < 256;
+      const uint8_t *arow = (mat ? a.A1 : a.A0) + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
       const int dsel = FMT == kFmtQ80 ? a.bf16 : 0;
-      Raw<FMT> r0[PAIRED ? 2 : 1], r1[PAIRED ? 2 : 1], r2[PAIRED ? 2 : 1];
+      // packed bytes of K steps ks .. ks + kAhead - 1 are in flight in a ring of
+      // registers; slots are compile-time indices of the unrolled loop below, so
+      // no register copy ever waits on a load
+      Raw<FMT> R[kAhead + 1];
+      if (has_a) {
 #pragma unroll
-      for (int m = 0; m < (PAIRED ? 2 : 1); ++m) {
-        fetch(r0[m], arow[m], 0, item);
-        if (ksteps > 1) fetch(r1[m], arow[m], 1, item);
+        for (int j = 0; j < kAhead; ++j)
+          if (j < ksteps) fetch(R[j], arow, j, item);
       }
       auto issue_b = [&](int ks, int st) {
         uint8_t *Bs = stages + st * STAGE + NA * kATile;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 32 * i, ch), brow[i] + ks * BK);
+        for (int i = 0; i < 4; ++i) {
+          if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 64 * i, ch), brow[i] + ks * BK);
         }
         cp_async_commit();
       };
       bool ok = mbar_wait(&ctl.empty[it % S], ((it / S) & 1u) ^ 1u, ctl, a.err);
       if (ok) issue_b(0, it % S);
-      for (int ks = 0; ok && ks < ksteps; ++ks, ++it) {
-        const int st = it % S;
-        if (ks + 1 < ksteps) {
-          const uint32_t nt = it + 1;
-          if (!mbar_wait(&ctl.empty[nt % S], ((nt / S) & 1u) ^ 1u, ctl, a.err)) {
-            ok = false;
-            break;
+      for (int ks0 = 0; ok && ks0 < ksteps; ks0 += kAhead + 1) {
+#pragma unroll
+        for (int j = 0; j <= kAhead; ++j) {
+          const int ks = ks0 + j;
+          if (!ok || ks >= ksteps) break;
+          const int st = it % S;
+          if (ks + 1 < ksteps) {
+            const uint32_t nt = it + 1;
+            if (!mbar_wait(&ctl.empty[nt % S], ((nt / S) & 1u) ^ 1u, ctl, a.err)) {
+              ok = false;
+              break;
+            }
+            issue_b(ks + 1, nt % S);
+          } else {
+            cp_async_commit();
           }
-          issue_b(ks + 1, nt % S);
-        } else {
-          cp_async_commit();
-        }
-        if (ks + 2 < ksteps) {
-#pragma unroll
-          for (int m = 0; m < (PAIRED ? 2 : 1); ++m) fetch(r2[m], arow[m], ks + 2, item);
-        }
-        uint8_t *A0s = stages + st * STAGE;
-#pragma unroll
-        for (int m = 0; m < (PAIRED ? 2 : 1); ++m)
-          decode(r0[m], A0s + m * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh, signm);
-        cp_async_wait<1>();  // this step's B tile has landed
-        fence_proxy_async();
-        mbar_arrive(&ctl.full[st]);
-#pragma unroll
-        for (int m = 0; m < (PAIRED ? 2 : 1); ++m) {
-          r0[m] = r1[m];
-          r1[m] = r2[m];
+          uint8_t *A0s = stages + st * STAGE;
+          if (has_a) decode(R[j], A0s + mat * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh_l, signm_l);
+          cp_async_wait<1>();  // this step's B tile has landed
+          fence_proxy_async();
+          mbar_arrive(&ctl.full[st]);
+          // the next look-ahead fetch goes out after this step is handed over
+          if (has_a && ks + kAhead < ksteps) fetch(R[(j + kAhead) % (kAhead + 1)], arow, ks + kAhead, item);
+          ++it;
         }
       }
       if (!ok) break;
@@ -577,7 +584,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 size_t grouped_gemm_smem(int paired) {
   const int na = paired ? 2 : 1;
   const int s = paired ? 3 : 4;
-  return 1024 + (size_t)s * (na * kATile + kBTile) + 4096 + 2048 + sizeof(GemmCtl);
+  return 1024 + (size_t)s * (na * kATile + kBTile) + 4096 * kGridRep + 2048 * kSignRep + sizeof(GemmCtl);
 }
 
 template <int FMT, bool PAIRED>

@@ -24,6 +24,11 @@ struct LayerWeights {
   const uint8_t *gate, *up, *down, *sh_gate, *sh_up, *sh_down, *grid;
 };
 
+// K parts of the decode path's warp units: every unit covers 16 weight rows
+// and a K range of 1024 elements (256 where the dimension is not a multiple
+// of 1024), so routed and shared units carry the same work.
+__host__ __device__ inline int decode_kparts(int K) { return (K % 1024 == 0) ? K / 1024 : K / 256; }
+
 // Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
 // t*k + slot, shared vector T*k + t.
 struct DecodeScratch {
@@ -42,13 +47,16 @@ struct DecodeScratch {
   unsigned *hmax;   // [V] max |h| (float bits)
   unsigned *Xmax;   // [V]
   int *vcount;      // [V] finished 16-row tiles per vector
-  float *shpart;    // [2][4][T][Is] shared gate/up partial sums per K quarter
-  int *shcount;     // [Is/16]
-  float *ypart;     // [H/16][P][T][16] per-part output tiles
+  float *gpart;     // [2][PH][V][Imax] gate/up partial sums per K part of H
+  int *hcount;      // [1 + Jmax][TM] finished K parts per (vector set, 16-row tile)
+  float *ypart;     // [H/16][NS][16] partial output tiles, NS = T*k*PD + T*PS slots
   int *ycount;      // [H/16]
   int *work;        // [4] unit counters
   int Imax;
-  int P;            // max parts per output tile = min(T*k, E) + 4
+  int PH, PD, PS;   // K parts of H (gate/up), I (routed down), Is (shared down)
+  int Jmax;         // max routed vector sets = min(T*k, E)
+  int TM;           // max(I, Is) / 16
+  int NS;           // output slots per 16-row tile of y
 };
 
 struct DecodeArgs {
