@@ -38,6 +38,20 @@ namespace moe {
 namespace {
 
 constexpr int kWarps2 = 16;  // warps per CTA in k2 / k3 (at most)
+#ifndef MOE_DECODE_CLAIM
+#define MOE_DECODE_CLAIM 1
+#endif
+constexpr int kClaim = MOE_DECODE_CLAIM;  // consecutive units a warp claims at a time
+#ifndef MOE_DECODE_AHEAD
+#define MOE_DECODE_AHEAD 0
+#endif
+// 1: a unit is claimed and its first chunk staged while the previous unit's
+// last chunk is computed; 0: only after it
+constexpr bool kAheadClaim = MOE_DECODE_AHEAD != 0;
+#ifndef MOE_DECODE_GUNROLL
+#define MOE_DECODE_GUNROLL 2
+#endif
+constexpr int kGUnroll = MOE_DECODE_GUNROLL;  // unrolling of the IQ2_XXS group loop
 constexpr int kThreads2 = kWarps2 * kWarp;
 // k2 threads: 12 warps for four token pairs, whose accumulators need more
 // than the 128 registers a thread has at 16 warps
@@ -208,13 +222,17 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
 // ------------------------------------------------------------------ routing
 
 // One warp: top-k of token t by key (ties to the lower id), ids in ascending
-// order, weights scaling * s / sum(s).  Keys come from k1 (router mode) or the
-// token-id table (hash mode).
+// order, weights scaling * s / sum(s) with the sum taken in ascending id
+// order.  Keys come from k1 (router mode) or the token-id table (hash mode).
+// Every lane loads its 8 keys and scores at once; each of the k rounds is a
+// warp arg-max over (key, id) followed by a broadcast of the winner's score;
+// the ids are then ranked in registers, so nothing waits on memory twice.
 __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, float *w_out) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31;
   const int k = d.k;
   int sel[kMaxK];
+  double ssel[kMaxK];
   if (d.mode == MOE_ROUTE_HASH) {
     int tid = a.token_ids[t];
     if (tid < 0 || tid >= d.vocab) {
@@ -222,21 +240,28 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
       tid = 0;
     }
 #pragma unroll
-    for (int i = 0; i < kMaxK; ++i) sel[i] = i < k ? a.wt.tid2eid[(size_t)tid * k + i] : INT_MAX;
+    for (int i = 0; i < kMaxK; ++i) {
+      sel[i] = i < k ? a.wt.tid2eid[(size_t)tid * k + i] : INT_MAX;
+      ssel[i] = 0.0;
+    }
   } else {
     const double *kt = a.s.z + (size_t)t * d.E;
-    double key[8];
+    const double *stt = a.s.sc + (size_t)t * d.E;
+    double key[8], scv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
       key[i] = e < d.E ? kt[e] : -DBL_MAX;
+      scv[i] = e < d.E ? stt[e] : 0.0;
     }
     unsigned taken = 0;
 #pragma unroll
     for (int r = 0; r < kMaxK; ++r) {
       sel[r] = INT_MAX;
+      ssel[r] = 0.0;
       if (r < k) {
-        double bk = -INFINITY;
+        // this lane's best untaken key (slots in id order, so the first wins ties)
+        double bk = -INFINITY, bs = 0.0;
         int be = INT_MAX;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -244,8 +269,10 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
           if (e < d.E && !((taken >> i) & 1u) && key[i] > bk) {
             bk = key[i];
             be = e;
+            bs = scv[i];
           }
         }
+        const double my_s = bs;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
@@ -257,32 +284,41 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
         sel[r] = be;
+        ssel[r] = __shfl_sync(0xffffffffu, my_s, be & 31);
       }
     }
   }
-  if (lane == 0) {
-    for (int i = 1; i < k; ++i)
-      for (int j = i; j > 0 && sel[j - 1] > sel[j]; --j) {
-        const int tmp = sel[j - 1];
-        sel[j - 1] = sel[j];
-        sel[j] = tmp;
+  // rank the ids (stable for repeated ids of the hash table)
+  int rank[kMaxK];
+#pragma unroll
+  for (int i = 0; i < kMaxK; ++i) {
+    rank[i] = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k && i < k) rank[i] += (sel[j] < sel[i]) || (sel[j] == sel[i] && j < i);
+  }
+  int ids[kMaxK];
+  double srt[kMaxK];
+#pragma unroll
+  for (int pos = 0; pos < kMaxK; ++pos) {
+    ids[pos] = INT_MAX;
+    srt[pos] = 0.0;
+#pragma unroll
+    for (int i = 0; i < kMaxK; ++i)
+      if (i < k && rank[i] == pos) {
+        ids[pos] = sel[i];
+        srt[pos] = ssel[i];
       }
-    if (d.mode == MOE_ROUTE_HASH) {
-      for (int i = 0; i < k; ++i) {
-        idx_out[i] = sel[i];
-        w_out[i] = d.scaling / (float)k;
-      }
-    } else {
-      const double *st = a.s.sc + (size_t)t * d.E;
-      double sv[kMaxK], tot = 0.0;
-      for (int i = 0; i < k; ++i) {
-        sv[i] = st[sel[i]];
-        tot += sv[i];
-      }
-      for (int i = 0; i < k; ++i) {
-        idx_out[i] = sel[i];
-        w_out[i] = (float)((double)d.scaling * sv[i] / tot);
-      }
+  }
+  double tot = 0.0;
+#pragma unroll
+  for (int pos = 0; pos < kMaxK; ++pos)
+    if (pos < k) tot += srt[pos];
+#pragma unroll
+  for (int pos = 0; pos < kMaxK; ++pos) {
+    if (pos < k && lane == pos) {
+      idx_out[pos] = ids[pos];
+      w_out[pos] = d.mode == MOE_ROUTE_HASH ? d.scaling / (float)k : (float)((double)d.scaling * srt[pos] / tot);
     }
   }
 }
@@ -297,6 +333,7 @@ struct Jobs {
   int pair[kDecodeMaxT * kMaxK];  // sorted t*k + slot
   int rank_e[kDecodeMaxT * kMaxK];
 };
+static_assert(sizeof(Jobs) == sizeof(int) * kJobsInts, "job table layout");
 
 __device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
   const int np = T * k;
@@ -344,6 +381,7 @@ struct Chunk {
   int nb;            // blocks in the chunk
   int k0;            // first element (K index) of the chunk
   int piece;         // copy granularity: 16, 8, 4 (cp.async) or 2 (plain loads)
+  int align;         // alignment the decoder needs at the start of a staged row (4 or 8)
 };
 
 __host__ __device__ __forceinline__ int piece_for(size_t gstride, size_t off, int bpr) {
@@ -356,20 +394,22 @@ __device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)
 // Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS) and
 // returns where the chunk's data starts in each staged row.
 //
-// Fast path, when all rows start at the same 8-byte phase of a 16-byte line
+// Fast path, when all rows start at the same 4-byte phase of a 16-byte line
 // (row stride a multiple of 16): each row is copied from the 16-byte boundary
-// at or below its start, in 16-byte pieces plus an 8-byte tail, two rows per
-// pass of the warp; the data then starts `shift` (0 or 8) bytes into the
-// staged row.  The bytes before the chunk belong to the same row.
+// at or below its start, in 16-byte pieces plus an 8- and a 4-byte tail, two
+// rows per pass of the warp; the data then starts `shift` (0, 4, 8 or 12)
+// bytes into the staged row.  The bytes before the chunk belong to the same
+// row.
 // Otherwise rows are walked in order and each lane issues the pieces lane,
 // lane + 32, ... of a row in the chunk's own granularity (data at offset 0).
 __device__ __forceinline__ int stage_chunk(uint8_t *st, const Chunk &c) {
   const int lane = threadIdx.x & 31;
   const int RS = stage_rs(c.bpr);
   const int shift = (int)(reinterpret_cast<uintptr_t>(c.g) & 15);
-  if ((c.gstride & 15) == 0 && (shift & 7) == 0 && shift + c.bpr <= RS && ((shift + c.bpr) & 7) == 0) {
-    const int n16 = (shift + c.bpr) >> 4;
-    const bool tail = ((shift + c.bpr) & 15) != 0;
+  if ((c.gstride & 15) == 0 && (shift & (c.align - 1)) == 0 && shift + c.bpr <= RS && ((shift + c.bpr) & 3) == 0) {
+    const int end = shift + c.bpr;
+    const int n16 = end >> 4;
+    const int t8 = end & 8, t4 = end & 4;  // tail: an 8-byte piece, then a 4-byte piece
     const uint8_t *g0 = c.g - shift;
     const int half = lane >> 4, l16 = lane & 15;
 #pragma unroll 1
@@ -380,10 +420,12 @@ __device__ __forceinline__ int stage_chunk(uint8_t *st, const Chunk &c) {
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int pc = l16 + 16 * m;
-        if (pc < n16)
+        if (pc < n16) {
           cp_async16(sr + 16 * pc, gr + 16 * pc);
-        else if (tail && pc == n16)
-          cp_async8(sr + 16 * pc, gr + 16 * pc);
+        } else if (pc == n16) {
+          if (t8) cp_async8(sr + 16 * pc, gr + 16 * pc);
+          if (t4) cp_async4(sr + 16 * pc + t8, gr + 16 * pc + t8);
+        }
       }
     }
     cp_async_commit();
@@ -433,6 +475,73 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
     compute(i, cur + sh_cur);
     __syncwarp();
     sh_cur = sh_next;
+  }
+}
+
+// Dynamic unit scheduling on the warp's two-stage ring.  A warp claims G
+// consecutive units at a time from `counter`; the claim is made when the
+// first chunk of a unit is staged, so its latency overlaps the compute of the
+// previous chunk, and the ring runs on across unit boundaries.
+//   unit_at(u)        -> UnitT with field nch (chunks of the unit)
+//   chunk_of(unit, c) -> Chunk c of the unit
+//   compute(unit, u, c, data, next_u): consume chunk c of unit u, staged at
+//                        `data`; next_u is the unit of the next chunk the warp
+//                        computes (-1 when none), for segment bookkeeping
+template <int G, bool AHEAD, typename UnitT, typename UnitAt, typename ChunkOf, typename Compute>
+__device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *counter, int n_units, UnitAt unit_at,
+                                          ChunkOf chunk_of, Compute compute) {
+  const int lane = threadIdx.x & 31;
+  int s_u = 0, s_left = 0, s_c = 0;
+  UnitT su;
+  auto stage_next = [&](uint8_t *dst, int &uid, int &cidx, int &shift) -> bool {
+    if (s_c == 0) {
+      if (s_left == 0) {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(counter, G);
+        s_u = __shfl_sync(0xffffffffu, u, 0);
+        s_left = G;
+      } else {
+        ++s_u;
+      }
+      --s_left;
+      if (s_u >= n_units) {
+        s_left = 0;
+        cp_async_commit();
+        return false;
+      }
+      su = unit_at(s_u);
+    }
+    uid = s_u;
+    cidx = s_c;
+    shift = stage_chunk(dst, chunk_of(su, s_c));
+    if (++s_c == su.nch) s_c = 0;
+    return true;
+  };
+  int uA = 0, cA = 0, shA = 0;
+  bool haveA = stage_next(st0, uA, cA, shA);
+  UnitT cu;
+  for (int i = 0; haveA; ++i) {
+    uint8_t *cur = (i & 1) ? st1 : st0;
+    uint8_t *nxt = (i & 1) ? st0 : st1;
+    if (cA == 0) cu = unit_at(uA);
+    int uB = 0, cB = 0, shB = 0;
+    bool haveB = false;
+    // the next unit is claimed early only while the warp's last claim lies
+    // more than a grid's worth of warps before the end of the work (near the
+    // end an early claim would only lengthen the tail)
+    const bool defer =
+        s_c == 0 && s_left == 0 && (!AHEAD || s_u + (int)(gridDim.x * (blockDim.x >> 5)) * G >= n_units);
+    if (!defer) haveB = stage_next(nxt, uB, cB, shB);
+    else cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    compute(cu, uA, cA, cur + shA, defer ? -1 : (haveB ? uB : -1));
+    __syncwarp();
+    if (defer) haveB = stage_next(nxt, uB, cB, shB);
+    uA = uB;
+    cA = cB;
+    shA = shB;
+    haveA = haveB;
   }
 }
 
@@ -494,7 +603,7 @@ __device__ __forceinline__ void iq2_chunk(const uint8_t *st, int k0, const uint8
     int acc[MAXP][4];
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0;
-#pragma unroll
+#pragma unroll kGUnroll
     for (int g = 0; g < 8; ++g) {
       const int o = 66 * b + 2 + 8 * g;
       uint32_t A[4];
@@ -744,6 +853,33 @@ __device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, i
   }
 }
 
+// Copies `rows` rows of n16 16-byte words from global (row stride gs bytes)
+// into shared memory (row stride ss bytes) with the whole block; each thread
+// issues a batch of independent loads before storing any.
+__device__ __forceinline__ void copy_rows16(void *dst, size_t ss, const void *src, size_t gs, int rows, int n16) {
+  constexpr int kB = 4;
+  const int n = rows * n16, step = blockDim.x;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kB * step) {
+    uint4 v[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * step;
+      if (i < n) {
+        const int r = i / n16, o = i - r * n16;
+        v[u] = __ldcg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(src) + r * gs + 16 * o));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * step;
+      if (i < n) {
+        const int r = i / n16, o = i - r * n16;
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(dst) + r * ss + 16 * o) = v[u];
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ k2
 
 struct K2Shared {
@@ -819,11 +955,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   pdl_wait();  // k1's limbs and keys are visible from here on
   if (XSMEM) {
     const int n16 = d.H / 16;
-    for (int i = tid; i < T * 3 * n16; i += blockDim.x) {
-      const int rowi = i / n16, o = i - rowi * n16;
-      *reinterpret_cast<uint4 *>(xsm + (size_t)rowi * XS + 16 * o) =
-          *reinterpret_cast<const uint4 *>(s.xq + (size_t)rowi * d.H + 16 * o);
-    }
+    copy_rows16(xsm, XS, s.xq, d.H, T * 3, n16);
   }
   for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
   __syncthreads();
@@ -834,6 +966,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
     }
   }
   build_jobs(S.idx, T, d.k, S.J);
+  if (blockIdx.x == 0)
+    for (int i = tid; i < kJobsInts; i += blockDim.x) s.jobs[i] = reinterpret_cast<const int *>(&S.J)[i];
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
   const uint8_t *sel_l = selt + (lane & 15) * 8;
@@ -849,7 +983,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   const int tilesI = d.I / 16, tilesS = d.Is / 16;
   const int PH = s.PH;
   const int kpart = d.H / PH;  // K elements per unit
-  const int cbI = kpart / 256;  // IQ2_XXS blocks per unit: one chunk per matrix
+  const int cbI = kpart / 256;  // IQ2_XXS blocks per unit (4, 2 or 1): one chunk per matrix
   const int nq8 = kpart / 256;  // Q8_0 chunks of 8 blocks per unit and matrix
   const size_t rbI = (size_t)(d.H / 256) * 66;
   const size_t rbQ = (size_t)(d.H / 32) * 34;
@@ -857,137 +991,156 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   const int n_sh = tilesS * PH;
   const int n_units = n_sh + S.J.n * tilesI * PH;
 
-  while (true) {
-    int u = 0;
-    if (lane == 0) u = atomicAdd(s.work + 0, 1);
-    u = __shfl_sync(0xffffffffu, u, 0);
-    if (u >= n_units) break;
-
-    // ---- unit: (vector set, 16-row tile, K part) of gate and up
-    const bool shared = u < n_sh;
-    int j = 0, tile, part, ntok, e = 0;
-    const int *pairs = nullptr;
-    if (shared) {
-      tile = u / PH;
-      part = u % PH;
-      ntok = T;
+  // ---- units: shared (tile, part), then routed (job, tile, part); the key
+  // u / PH names the (vector set, tile), so a tile's parts are consecutive.
+  // Consecutive parts of one tile that a warp computes in a row form a
+  // segment; the tile's counter is bumped once per segment.
+  struct Unit {
+    bool shared;
+    int j, e, tile, part, ntok, per, nch;  // per: chunks per matrix
+    const int *pairs;
+  };
+  auto unit_at = [&](int u) {
+    Unit x;
+    x.shared = u < n_sh;
+    x.j = 0;
+    x.e = 0;
+    x.pairs = nullptr;
+    if (x.shared) {
+      x.tile = u / PH;
+      x.part = u % PH;
+      x.ntok = T;
+      x.per = nq8;
     } else {
       const int uu = u - n_sh;
-      j = uu / (tilesI * PH);
+      x.j = uu / (tilesI * PH);
       const int rem = uu % (tilesI * PH);
-      tile = rem / PH;
-      part = rem % PH;
-      e = S.J.e[j];
-      ntok = S.J.cnt[j];
-      pairs = S.J.pair + S.J.first[j];
+      x.tile = rem / PH;
+      x.part = rem % PH;
+      x.e = S.J.e[x.j];
+      x.ntok = S.J.cnt[x.j];
+      x.pairs = S.J.pair + S.J.first[x.j];
+      x.per = 1;
     }
-    const int r0 = tile * 16;
-    // token slot ts -> row of x / vector of h
-    auto xrow = [&](int ts) { return shared ? ts : pairs[ts] / d.k; };
-    auto hvec = [&](int ts) { return shared ? T * d.k + ts : pairs[ts]; };
-    const int npairs = (ntok + 1) >> 1;
-    BCol bcol[MAXP];
+    x.nch = 2 * x.per;
+    return x;
+  };
+  // token slot ts of a unit -> row of x / vector of h
+  auto xrow = [&](const Unit &x, int ts) { return x.shared ? ts : x.pairs[ts] / d.k; };
+  auto hvec = [&](const Unit &x, int ts) { return x.shared ? T * d.k + ts : x.pairs[ts]; };
+  auto chunk_of = [&](const Unit &su, int cs) {
+    const bool up = cs >= su.per;
+    const int ck = cs % su.per;
+    Chunk ch;
+    if (su.shared) {
+      const size_t off = (size_t)(su.part * kpart / 32 + ck * 8) * 34;
+      ch.g = (up ? a.wt.sh_up : a.wt.sh_gate) + (size_t)(su.tile * 16) * rbQ + off;
+      ch.gstride = rbQ;
+      ch.bpr = 8 * 34;
+      ch.nb = 8;
+      ch.k0 = su.part * kpart + ck * 256;
+      ch.piece = piece_for(rbQ, off, ch.bpr);
+    } else {
+      const size_t off = (size_t)su.part * cbI * 66;
+      ch.g = (up ? a.wt.up : a.wt.gate) + ((size_t)su.e * d.I + su.tile * 16) * rbI + off;
+      ch.gstride = rbI;
+      ch.bpr = cbI * 66;
+      ch.nb = cbI;
+      ch.k0 = su.part * kpart;
+      ch.piece = piece_for(rbI, off, ch.bpr);
+    }
+    ch.align = 4;
+    return ch;
+  };
+
+  int seg_parts = 0, npairs = 0;
+  BCol bcol[MAXP];
+  // F accumulates gate, then up, of one unit; each matrix's sums are combined
+  // over limbs and stored as the partials of the unit's K part (m = 0 gate, 1 up)
+  float F[MAXP][4] = {};
+  auto store_part = [&](const Unit &cu, int m) {
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
-      const int ts = 2 * p + (r >> 2), limb = r & 3;
-      bcol[p].ok = ts < ntok && limb < 3;
-      bcol[p].p = bcol[p].ok ? xcol(xrow(ts), limb) : nullptr;
-    }
-    // F accumulates gate, then up; each matrix's sums of this K part are
-    // combined over limbs and stored as partials (m = 0 gate, 1 up)
-    float F[MAXP][4] = {};
-    auto store_part = [&](int m) {
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
-          const int ts = 2 * p + (c >> 1);
-          float v0, v1;
-          combine_limbs(F[p], ts < ntok ? s.xs + 4 * xrow(ts) : nullptr, v0, v1);
-          if ((c & 1) == 0 && ts < ntok) {
-            float *pp = s.gpart + ((size_t)(m * PH + part) * V + hvec(ts)) * s.Imax + r0;
-            pp[r] = v0;
-            pp[r + 8] = v1;
-          }
+      if (p < npairs) {
+        const int ts = 2 * p + (c >> 1);
+        float v0, v1;
+        combine_limbs(F[p], ts < cu.ntok ? s.xs + 4 * xrow(cu, ts) : nullptr, v0, v1);
+        if ((c & 1) == 0 && ts < cu.ntok) {
+          float *pp = s.gpart + ((size_t)(m * PH + cu.part) * V + hvec(cu, ts)) * s.Imax + cu.tile * 16;
+          pp[r] = v0;
+          pp[r + 8] = v1;
         }
-        F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
       }
-    };
-    auto end_gate = [&]() { store_part(0); };
-    if (shared) {
-      auto chunk_at = [&](int i) {
-        const int m = i / nq8, ck = i % nq8;
-        const size_t off = (size_t)(part * kpart / 32 + ck * 8) * 34;
-        Chunk ch;
-        ch.g = (m == 0 ? a.wt.sh_gate : a.wt.sh_up) + (size_t)r0 * rbQ + off;
-        ch.gstride = rbQ;
-        ch.bpr = 8 * 34;
-        ch.nb = 8;
-        ch.k0 = part * kpart + ck * 256;
-        ch.piece = piece_for(rbQ, off, ch.bpr);
-        return ch;
-      };
-      run_chunks(st0, st1, 2 * nq8, chunk_at, [&](int i, uint8_t *st) {
-        q80_chunk<8, MAXP>(st, part * kpart + (i % nq8) * 256, bcol, npairs, F);
-        if (i == nq8 - 1) end_gate();
-      });
-    } else {
-      auto chunk_at = [&](int i) {
-        const size_t off = (size_t)part * cbI * 66;
-        Chunk ch;
-        ch.g = (i == 0 ? a.wt.gate : a.wt.up) + ((size_t)e * d.I + r0) * rbI + off;
-        ch.gstride = rbI;
-        ch.bpr = cbI * 66;
-        ch.nb = cbI;
-        ch.k0 = part * kpart;
-        ch.piece = piece_for(rbI, off, ch.bpr);
-        return ch;
-      };
-      run_chunks(st0, st1, 2, chunk_at, [&](int i, uint8_t *st) {
-        if (cbI == 4)
-          iq2_chunk<4, MAXP>(st, part * kpart, gpm_l, sel_l, bcol, npairs, F);
-        else
-          iq2_chunk<1, MAXP>(st, part * kpart, gpm_l, sel_l, bcol, npairs, F);
-        if (i == 0) end_gate();
-      });
+      F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
     }
-    store_part(1);
+  };
+  // count the segment's parts in; the warp that completes the tile sums the
+  // parts in order and applies the SwiGLU
+  auto end_segment = [&](const Unit &cu) {
     __threadfence();
     __syncwarp();
-    const int set = shared ? 0 : 1 + j;
+    const int set = cu.shared ? 0 : 1 + cu.j;
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.hcount + set * s.TM + tile, 1) == PH - 1;
+    if (lane == 0) last = atomicAdd(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
     last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      // every K part of the tile is in: sum them in part order, SwiGLU
-      __threadfence();
-      for (int i = lane; i < 16 * ntok; i += 32) {
-        const int ts = i >> 4, row = i & 15;
-        const int v = hvec(ts);
-        float ga = 0.f, ub = 0.f;
-        for (int p0 = 0; p0 < PH; p0 += 4) {  // loads of a batch are independent; sums keep part order
-          float gb[4], ubb[4];
+    seg_parts = 0;
+    if (!last) return;
+    __threadfence();
+    const int r0 = cu.tile * 16;
+    for (int i = lane; i < 16 * cu.ntok; i += 32) {
+      const int ts = i >> 4, row = i & 15;
+      const int v = hvec(cu, ts);
+      float ga = 0.f, ub = 0.f;
+      for (int p0 = 0; p0 < PH; p0 += 4) {  // loads of a batch are independent; sums keep part order
+        float gb[4], ubb[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const bool in = p0 + q < PH;
-            gb[q] = in ? __ldcg(s.gpart + ((size_t)(0 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
-            ubb[q] = in ? __ldcg(s.gpart + ((size_t)(1 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            ga += gb[q];
-            ub += ubb[q];
-          }
+        for (int q = 0; q < 4; ++q) {
+          const bool in = p0 + q < PH;
+          gb[q] = in ? __ldcg(s.gpart + ((size_t)(0 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
+          ubb[q] = in ? __ldcg(s.gpart + ((size_t)(1 * PH + p0 + q) * V + v) * s.Imax + r0 + row) : 0.f;
         }
-        S.hsm[warp][ts][row] = silu(ga) * ub;
-      }
-      __syncwarp();
-      int vec[kDecodeMaxT];
 #pragma unroll
-      for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < ntok ? hvec(t) : 0;
-      finish_h_tile(a, S.hsm[warp], ntok, vec, r0, shared ? d.Is : d.I, shared ? tilesS : tilesI);
+        for (int q = 0; q < 4; ++q) {
+          ga += gb[q];
+          ub += ubb[q];
+        }
+      }
+      S.hsm[warp][ts][row] = silu(ga) * ub;
     }
     __syncwarp();
-  }
+    int vec[kDecodeMaxT];
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < cu.ntok ? hvec(cu, t) : 0;
+    finish_h_tile(a, S.hsm[warp], cu.ntok, vec, r0, cu.shared ? d.Is : d.I, cu.shared ? tilesS : tilesI);
+  };
+
+  run_units<kClaim, kAheadClaim, Unit>(st0, st1, s.work + 0, n_units, unit_at, chunk_of,
+                     [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
+                       if (cc == 0) {
+                         npairs = (cu.ntok + 1) >> 1;
+#pragma unroll
+                         for (int p = 0; p < MAXP; ++p) {
+                           const int ts = 2 * p + (r >> 2), limb = r & 3;
+                           bcol[p].ok = ts < cu.ntok && limb < 3;
+                           bcol[p].p = bcol[p].ok ? xcol(xrow(cu, ts), limb) : nullptr;
+                         }
+                       }
+                       if (cu.shared) {
+                         q80_chunk<8, MAXP>(st, cu.part * kpart + (cc % nq8) * 256, bcol, npairs, F);
+                       } else if (cbI == 4) {
+                         iq2_chunk<4, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+                       } else if (cbI == 2) {
+                         iq2_chunk<2, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+                       } else {
+                         iq2_chunk<1, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+                       }
+                       if (cc == cu.per - 1) store_part(cu, 0);
+                       if (cc == cu.nch - 1) {
+                         store_part(cu, 1);
+                         ++seg_parts;
+                         if (next_u != u + 1 || (u + 1) / PH != u / PH) end_segment(cu);
+                       }
+                     });
 }
 
 // ------------------------------------------------------------------ k3
@@ -1017,26 +1170,17 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const size_t HR = k3_hrow(s.Imax), XR = k3_xrow(s.Imax);
   int8_t *xsm = hsm + (size_t)V * 3 * HR;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();  // k2's routing and h limbs are visible from here on
+  pdl_wait();  // k2's routing, job table and h limbs are visible from here on
   for (int i = tid; i < T * d.k; i += blockDim.x) {
-    S.idx[i] = s.idx[i];
-    S.w[i] = s.w[i];
+    S.idx[i] = __ldcg(s.idx + i);
+    S.w[i] = __ldcg(s.w + i);
   }
+  for (int i = tid; i < kJobsInts; i += blockDim.x) reinterpret_cast<int *>(&S.J)[i] = __ldcg(s.jobs + i);
   if (HSMEM) {
-    const int n16 = s.Imax / 16;
-    for (int i = tid; i < V * 3 * n16; i += blockDim.x) {
-      const int rowi = i / n16, o = i - rowi * n16;
-      *reinterpret_cast<uint4 *>(hsm + (size_t)rowi * HR + 16 * o) =
-          __ldcg(reinterpret_cast<const uint4 *>(s.hq + (size_t)rowi * s.Imax + 16 * o));
-    }
-    for (int i = tid; i < V * 3 * Im16 / 4; i += blockDim.x) {
-      const int rowi = i / (Im16 / 4), o = i - rowi * (Im16 / 4);
-      *reinterpret_cast<uint32_t *>(xsm + (size_t)rowi * XR + 4 * o) =
-          __ldcg(reinterpret_cast<const unsigned *>(s.Xq + (size_t)rowi * Im16 + 4 * o));
-    }
+    copy_rows16(hsm, HR, s.hq, s.Imax, V * 3, s.Imax / 16);
+    copy_rows16(xsm, XR, s.Xq, Im16, V * 3, Im16 / 16);
   }
   __syncthreads();
-  build_jobs(S.idx, T, d.k, S.J);
 
   uint8_t *st0 = stages + warp * 2 * kStage3;
   uint8_t *st1 = st0 + kStage3;
@@ -1052,7 +1196,7 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const int tilesH = d.H / 16;
   const int PD = s.PD, PS = s.PS;
   const int kpd = d.I / PD;      // K elements of a routed unit
-  const int cbD = kpd / 256;     // Q2_K blocks per routed unit: one chunk
+  const int cbD = kpd / 256;     // Q2_K blocks per routed unit (4, 2 or 1): one chunk
   const int kps = d.Is / PS;     // K elements of a shared unit
   const int nq8 = kps / 256;     // Q8_0 chunks of 8 blocks per shared unit
   const size_t rbD = (size_t)(d.I / 256) * 84;
@@ -1062,146 +1206,174 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   const int n_units = tilesH * nparts;
   const int NS = s.NS;
 
-  while (true) {
-    int u = 0;
-    if (lane == 0) u = atomicAdd(s.work + 1, 1);
-    u = __shfl_sync(0xffffffffu, u, 0);
-    if (u >= n_units) break;
-    const int ot = u / nparts, part = u % nparts;
-    const int r0 = ot * 16;
-    float *ytile = s.ypart + (size_t)ot * NS * 16;
-
-    if (part < nrp) {
-      // ---- routed: expert j, K part kp of I
-      const int j = part / PD, kp = part % PD;
-      const int e = S.J.e[j], ntok = S.J.cnt[j];
-      const int *pairs = S.J.pair + S.J.first[j];
-      const int npairs = (ntok + 1) >> 1;
-      BCol bcol[MAXP], xcol[MAXP];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        const int ts = 2 * p + (r >> 2), limb = r & 3;
-        const bool ok = ts < ntok && limb < 3;
-        bcol[p].ok = xcol[p].ok = ok;
-        bcol[p].p = ok ? hcol(pairs[ts], limb) : nullptr;
-        xcol[p].p = ok ? Xcol(pairs[ts], limb) : nullptr;
-      }
-      float F[MAXP][4] = {}, G[MAXP][4] = {};
-      auto chunk_at = [&](int) {
-        const size_t off = (size_t)kp * cbD * 84;
-        Chunk ch;
-        ch.g = a.wt.down + ((size_t)e * d.H + r0) * rbD + off;
-        ch.gstride = rbD;
-        ch.bpr = cbD * 84;
-        ch.nb = cbD;
-        ch.k0 = kp * kpd;
-        ch.piece = piece_for(rbD, off, ch.bpr);
-        return ch;
-      };
-      run_chunks(st0, st1, 1, chunk_at, [&](int, uint8_t *st) {
-        if (cbD == 4)
-          q2k_chunk<4, MAXP>(st, kp * kpd, bcol, xcol, npairs, F, G);
-        else
-          q2k_chunk<1, MAXP>(st, kp * kpd, bcol, xcol, npairs, F, G);
-      });
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
-          const int ts = 2 * p + (c >> 1);
-          const bool ok = ts < ntok;
-          const int v = ok ? pairs[ts] : 0;
-          const int l0 = 2 * (c & 1);
-          float v0 = 0.f, v1 = 0.f;
-          if (ok) {
-            const float *hs = s.hsc + 4 * v;
-            const float *xs = s.Xsc + 4 * v;
-            v0 = hs[l0] * F[p][0] - xs[l0] * G[p][0];
-            v1 = hs[l0] * F[p][2] - xs[l0] * G[p][2];
-            if (l0 + 1 < 3) {
-              v0 += hs[l0 + 1] * F[p][1] - xs[l0 + 1] * G[p][1];
-              v1 += hs[l0 + 1] * F[p][3] - xs[l0 + 1] * G[p][3];
-            }
-          }
-          v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-          v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-          if ((c & 1) == 0 && ok) {
-            const float wt = S.w[v];
-            float *dst = ytile + (size_t)(v * PD + kp) * 16;
-            dst[r] = wt * v0;
-            dst[r + 8] = wt * v1;
-          }
-        }
-      }
+  // ---- units (output tile ot, part), part fastest: routed parts (job, K
+  // part), then the shared parts; consecutive parts of one output tile that a
+  // warp computes in a row form a segment (see k2)
+  struct Unit {
+    int ot, part, j, kp, q, e, ntok, nch;
+    const int *pairs;
+  };
+  auto unit_at = [&](int u) {
+    Unit x;
+    x.ot = u / nparts;
+    x.part = u % nparts;
+    x.j = x.kp = x.q = x.e = 0;
+    x.pairs = nullptr;
+    if (x.part < nrp) {
+      x.j = x.part / PD;
+      x.kp = x.part % PD;
+      x.e = S.J.e[x.j];
+      x.ntok = S.J.cnt[x.j];
+      x.pairs = S.J.pair + S.J.first[x.j];
+      x.nch = 1;
     } else {
-      // ---- shared: K part q of Is
-      const int q = part - nrp;
-      const int npairs = (T + 1) >> 1;
-      BCol bcol[MAXP];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        const int ts = 2 * p + (r >> 2), limb = r & 3;
-        bcol[p].ok = ts < T && limb < 3;
-        bcol[p].p = bcol[p].ok ? hcol(T * d.k + ts, limb) : nullptr;
-      }
-      float F[MAXP][4] = {};
-      auto chunk_at = [&](int i) {
-        Chunk ch;
-        const size_t off = (size_t)(q * kps / 32 + i * 8) * 34;
-        ch.g = a.wt.sh_down + (size_t)r0 * rbQ + off;
-        ch.gstride = rbQ;
-        ch.bpr = 8 * 34;
-        ch.nb = 8;
-        ch.k0 = q * kps + i * 256;
-        ch.piece = piece_for(rbQ, off, ch.bpr);
-        return ch;
-      };
-      run_chunks(st0, st1, nq8, chunk_at,
-                 [&](int i, uint8_t *st) { q80_chunk<8, MAXP>(st, q * kps + i * 256, bcol, npairs, F); });
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
-          const int ts = 2 * p + (c >> 1);
-          const float *sc = ts < T ? s.hsc + 4 * (T * d.k + ts) : nullptr;
-          float v0, v1;
-          combine_limbs(F[p], sc, v0, v1);
-          if ((c & 1) == 0 && ts < T) {
-            float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + q) * 16;
-            dst[r] = v0;
-            dst[r + 8] = v1;
-          }
-        }
-      }
+      x.q = x.part - nrp;
+      x.ntok = T;
+      x.nch = nq8;
     }
+    return x;
+  };
+  auto chunk_of = [&](const Unit &su, int cs) {
+    Chunk ch;
+    if (su.part < nrp) {
+      const size_t off = (size_t)su.kp * cbD * 84;
+      ch.g = a.wt.down + ((size_t)su.e * d.H + su.ot * 16) * rbD + off;
+      ch.gstride = rbD;
+      ch.bpr = cbD * 84;
+      ch.nb = cbD;
+      ch.k0 = su.kp * kpd;
+      ch.piece = piece_for(rbD, off, ch.bpr);
+      ch.align = 8;
+    } else {
+      const size_t off = (size_t)(su.q * kps / 32 + cs * 8) * 34;
+      ch.g = a.wt.sh_down + (size_t)(su.ot * 16) * rbQ + off;
+      ch.gstride = rbQ;
+      ch.bpr = 8 * 34;
+      ch.nb = 8;
+      ch.k0 = su.q * kps + cs * 256;
+      ch.piece = piece_for(rbQ, off, ch.bpr);
+      ch.align = 4;
+    }
+    return ch;
+  };
+
+  int seg_parts = 0, npairs = 0;
+  BCol bcol[MAXP], xcolv[MAXP];
+  float F[MAXP][4] = {}, G[MAXP][4] = {};
+  auto end_segment = [&](const Unit &cu) {
     __threadfence();
     __syncwarp();
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.ycount + ot, 1) == nparts - 1;
+    if (lane == 0) last = atomicAdd(s.ycount + cu.ot, seg_parts) + seg_parts == nparts;
     last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      // every part of the tile is in: sum them in a fixed order into y
-      __threadfence();
-      for (int i = lane; i < 16 * T; i += 32) {
-        const int t = i >> 4, row = i & 15;
-        float acc = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[(size_t)t * d.H + r0 + row] : 0.f;
-        // slots in a fixed order: the token's routed parts, then its shared parts;
-        // the loads of a batch are independent
-        const int nr = d.k * PD, ns = nr + PS;
-        for (int s0 = 0; s0 < ns; s0 += 8) {
-          float vb[8];
+    seg_parts = 0;
+    if (!last) return;
+    // every part of the tile is in: sum them in a fixed order into y
+    __threadfence();
+    const int r0 = cu.ot * 16;
+    const float *ytile = s.ypart + (size_t)cu.ot * NS * 16;
+    for (int i = lane; i < 16 * T; i += 32) {
+      const int t = i >> 4, row = i & 15;
+      float acc = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[(size_t)t * d.H + r0 + row] : 0.f;
+      // slots in a fixed order: the token's routed parts, then its shared parts;
+      // the loads of a batch are independent
+      const int nr = d.k * PD, ns = nr + PS;
+      for (int s0 = 0; s0 < ns; s0 += 8) {
+        float vb[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int sl = s0 + q;
-            const size_t slot = sl < nr ? (size_t)t * nr + sl : (size_t)T * nr + (size_t)t * PS + (sl - nr);
-            vb[q] = sl < ns ? __ldcg(ytile + slot * 16 + row) : 0.f;
-          }
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc += vb[q];
+        for (int q = 0; q < 8; ++q) {
+          const int sl = s0 + q;
+          const size_t slot = sl < nr ? (size_t)t * nr + sl : (size_t)T * nr + (size_t)t * PS + (sl - nr);
+          vb[q] = sl < ns ? __ldcg(ytile + slot * 16 + row) : 0.f;
         }
-        a.y[(size_t)t * d.H + r0 + row] = acc;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc += vb[q];
       }
+      a.y[(size_t)t * d.H + r0 + row] = acc;
     }
-    __syncwarp();
-  }
+  };
+
+  run_units<kClaim, kAheadClaim, Unit>(
+      st0, st1, s.work + 1, n_units, unit_at, chunk_of,
+      [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
+        if (cc == 0) {
+          npairs = (cu.ntok + 1) >> 1;
+#pragma unroll
+          for (int p = 0; p < MAXP; ++p) {
+            const int ts = 2 * p + (r >> 2), limb = r & 3;
+            const bool ok = ts < cu.ntok && limb < 3;
+            const int v = !ok ? 0 : cu.part < nrp ? cu.pairs[ts] : T * d.k + ts;
+            bcol[p].ok = xcolv[p].ok = ok;
+            bcol[p].p = ok ? hcol(v, limb) : nullptr;
+            xcolv[p].p = ok ? Xcol(v, limb) : nullptr;
+          }
+        }
+        float *ytile = s.ypart + (size_t)cu.ot * NS * 16;
+        if (cu.part < nrp) {
+          // ---- routed: expert j, K part kp of I
+          if (cbD == 4)
+            q2k_chunk<4, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
+          else if (cbD == 2)
+            q2k_chunk<2, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
+          else
+            q2k_chunk<1, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
+#pragma unroll
+          for (int p = 0; p < MAXP; ++p) {
+            if (p < npairs) {
+              const int ts = 2 * p + (c >> 1);
+              const bool ok = ts < cu.ntok;
+              const int v = ok ? cu.pairs[ts] : 0;
+              const int l0 = 2 * (c & 1);
+              float v0 = 0.f, v1 = 0.f;
+              if (ok) {
+                const float *hs = s.hsc + 4 * v;
+                const float *xs = s.Xsc + 4 * v;
+                v0 = hs[l0] * F[p][0] - xs[l0] * G[p][0];
+                v1 = hs[l0] * F[p][2] - xs[l0] * G[p][2];
+                if (l0 + 1 < 3) {
+                  v0 += hs[l0 + 1] * F[p][1] - xs[l0 + 1] * G[p][1];
+                  v1 += hs[l0 + 1] * F[p][3] - xs[l0 + 1] * G[p][3];
+                }
+              }
+              v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+              v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+              if ((c & 1) == 0 && ok) {
+                const float wt = S.w[v];
+                float *dst = ytile + (size_t)(v * PD + cu.kp) * 16;
+                dst[r] = wt * v0;
+                dst[r + 8] = wt * v1;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
+          }
+        } else {
+          // ---- shared: K part q of Is
+          q80_chunk<8, MAXP>(st, cu.q * kps + cc * 256, bcol, npairs, F);
+          if (cc == nq8 - 1) {
+#pragma unroll
+            for (int p = 0; p < MAXP; ++p) {
+              if (p < npairs) {
+                const int ts = 2 * p + (c >> 1);
+                const float *sc = ts < T ? s.hsc + 4 * (T * d.k + ts) : nullptr;
+                float v0, v1;
+                combine_limbs(F[p], sc, v0, v1);
+                if ((c & 1) == 0 && ts < T) {
+                  float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + cu.q) * 16;
+                  dst[r] = v0;
+                  dst[r + 8] = v1;
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) F[p][i] = 0.f;
+            }
+          }
+        }
+        if (cc == cu.nch - 1) {
+          ++seg_parts;
+          if (next_u != u + 1 || (u + 1) / nparts != u / nparts) end_segment(cu);
+        }
+      });
 }
 
 // ------------------------------------------------------------------ route only
@@ -1278,7 +1450,7 @@ cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
 size_t decode_scratch_bytes(const LayerDims &d, int T) {
   DecodeScratch s;
   decode_carve(s, d, T, nullptr);
-  return reinterpret_cast<size_t>(s.work) + 4 * sizeof(int) + 256;
+  return reinterpret_cast<size_t>(s.jobs) + kJobsInts * sizeof(int) + 256;
 }
 
 void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
@@ -1318,6 +1490,7 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * s.NS * 16));
   s.ycount = reinterpret_cast<int *>(take(sizeof(int) * (d.H / 16)));
   s.work = reinterpret_cast<int *>(take(sizeof(int) * 4));
+  s.jobs = reinterpret_cast<int *>(take(sizeof(int) * kJobsInts));
 }
 
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {

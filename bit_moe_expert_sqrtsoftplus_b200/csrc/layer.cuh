@@ -25,9 +25,17 @@ struct LayerWeights {
 };
 
 // K parts of the decode path's warp units: every unit covers 16 weight rows
-// and a K range of 1024 elements (256 where the dimension is not a multiple
-// of 1024), so routed and shared units carry the same work.
-__host__ __device__ inline int decode_kparts(int K) { return (K % 1024 == 0) ? K / 1024 : K / 256; }
+// and a K range of kDecodeKPart elements (256 where the dimension is not a
+// multiple of it), so routed and shared units carry the same work.
+#ifndef MOE_DECODE_KPART
+#define MOE_DECODE_KPART 1024
+#endif
+constexpr int kDecodeKPart = MOE_DECODE_KPART;  // 1024, 512 or 256
+__host__ __device__ inline int decode_kparts(int K) { return (K % kDecodeKPart == 0) ? K / kDecodeKPart : K / 256; }
+
+// Job table of the decode path (distinct experts of a call and their
+// (token, slot) pairs) as ints: n, then e, first, cnt, pair, rank_e.
+constexpr int kJobsInts = 1 + 5 * kDecodeMaxT * kMaxK;
 
 // Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
 // t*k + slot, shared vector T*k + t.
@@ -52,6 +60,7 @@ struct DecodeScratch {
   float *ypart;     // [H/16][NS][16] partial output tiles, NS = T*k*PD + T*PS slots
   int *ycount;      // [H/16]
   int *work;        // [4] unit counters
+  int *jobs;        // [kJobsInts] job table written by k2 for k3
   int Imax;
   int PH, PD, PS;   // K parts of H (gate/up), I (routed down), Is (shared down)
   int Jmax;         // max routed vector sets = min(T*k, E)
