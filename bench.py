@@ -58,6 +58,29 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the workload's dominant kernel from the ncu
+    capture recorded in profiles/traffic.txt, or None when the kernel's
+    sources changed since that capture."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(ROOT, "bit_moe_expert_sqrtsoftplus_b200", "csrc")
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if not parts or parts[0].startswith("#") or parts[0] != workload or len(parts) < 5:
+                continue
+            h = hashlib.sha256()
+            for name in parts[4].split(","):
+                with open(os.path.join(csrc, name), "rb") as g:
+                    h.update(g.read())
+            return int(parts[2]) if h.hexdigest() == parts[3] else None
+    return None
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -275,7 +298,8 @@ def run_ours(args, world, rank):
         roof = {"bound": "tensor", "kernel": "routed gate/up grouped GEMM (tcgen05 kind::f16, IQ2_XXS dequantised "
                                              "to f16 in producer warps)",
                 "achieved": tc_achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": tc_achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": peaks["source"],
+                "frac": tc_achieved / peaks["bf16_tflops"], "traffic": load_traffic(args.workload),
+                "traffic_unit": "bytes per launch (ncu)", "peak_source": peaks["source"],
                 "algorithmic_flops_per_launch": fl["gateup_routed"], "ms_per_launch": k2_ms}
         layer = {"flops_per_call": fl["layer"], "achieved_tflops": fl["layer"] / (ms_step / 1e3) / 1e12,
                  "frac": fl["layer"] / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -303,7 +327,8 @@ def run_ours(args, world, rank):
         "roofline": roof if large else
         {"bound": "hbm", "kernel": "k2_gateup (routed IQ2_XXS gate/up + shared Q8_0 gate/up)",
          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-         "traffic": None, "peak_source": peaks["source"],
+         "traffic": load_traffic(args.workload), "traffic_unit": "bytes per launch (ncu)",
+         "peak_source": peaks["source"],
          "algorithmic_bytes_per_launch": b["k2_gateup"], "ms_per_launch": k2_ms},
         ("layer_tensor" if large else "layer_hbm"): layer if large else
         {"bytes_per_call": b["experts"], "router_bytes": s.n_experts * s.hidden * 2,
