@@ -1,30 +1,31 @@
-// decode.cu -- the layer for small token counts (T <= 8): three kernels.
+// decode.cu -- the layer for small token counts (T <= 8): two kernels.
 //
 //   k1_prep_router  x -> int8 limbs (optionally RMSNorm first); fp64 router
 //                   logits, scores s = sqrtsoftplus(z) and selection keys
 //                   s + bias, one block per pair of experts.
-//   k2_gateup       top-k routing from the keys (comparisons only, per CTA),
-//                   then every (expert, 16-row tile) of gate/up and every
-//                   (16-row tile, K quarter) of the shared expert as a
-//                   warp-sized unit: packed rows are staged into shared memory
+//   k2_experts      top-k routing from the keys (comparisons only, per CTA),
+//                   then all the expert work as warp-sized units on one
+//                   counter: every (16-row tile, 1024-element K part) of the
+//                   shared and the routed gate/up matrices, then every
+//                   (K part, 16-row output tile) of the shared and the routed
+//                   down matrices.  Packed rows are staged into shared memory
 //                   with cp.async, decoded in registers into int8 A fragments
 //                   and multiplied with mma.sync m16n8k32 against the int8
-//                   limbs of x; the SwiGLU is applied in the epilogue.  The
-//                   warp that finishes the last tile of a vector quantises it
-//                   into limbs for the down projection.
-//   k3_down         every (16-row output tile, expert or shared K quarter)
-//                   unit: Q2_K / Q8_0 rows against the limbs of h, weighted
-//                   by the routing weight; the last unit of a tile sums the
-//                   parts in a fixed order (deterministic) into y.
-// k2 and k3 are launched as programmatic dependents: their set-up (tables,
-// shared memory) overlaps the previous kernel, and griddepcontrol.wait
-// guards every read of the previous kernel's results.
+//                   limbs of the activations.  The warp that completes a
+//                   gate/up tile applies the SwiGLU; the warp that completes a
+//                   1024-element slice of h quantises it into limbs and flags
+//                   it, and down units wait for the slices they read.  The
+//                   warp that completes an output tile sums its parts in a
+//                   fixed order (deterministic) into y.
+// k2 is launched as a programmatic dependent of k1: its set-up (tables,
+// shared memory) overlaps k1, and griddepcontrol.wait guards every read of
+// k1's results.
 //
 // Activations enter the tensor cores as three int8 limbs with one scale per
-// vector: x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254, s3 = s2/254, which keeps
-// x to 6e-8 of max|x|; the weight side is exact in int8 (IQ2_XXS grid values
-// with signs, Q2_K code*scale <= 45, Q8_0 values), so the products are exact
-// integers and only the fp32 block scaling rounds.
+// vector (per slice for h): x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254,
+// s3 = s2/254, which keeps x to 6e-8 of max|x|; the weight side is exact in
+// int8 (IQ2_XXS grid values with signs, Q2_K code*scale <= 45, Q8_0 values),
+// so the products are exact integers and only the fp32 block scaling rounds.
 #include <float.h>
 #include <math.h>
 
@@ -52,12 +53,12 @@ constexpr bool kAheadClaim = MOE_DECODE_AHEAD != 0;
 #define MOE_DECODE_GUNROLL 2
 #endif
 constexpr int kGUnroll = MOE_DECODE_GUNROLL;  // unrolling of the IQ2_XXS group loop
+constexpr long long kSliceWaitCycles = 4000000000ll;  // about 2 s: bound of a wait for an h slice
 constexpr int kThreads2 = kWarps2 * kWarp;
 // k2 threads: 12 warps for four token pairs, whose accumulators need more
 // than the 128 registers a thread has at 16 warps
 __host__ __device__ constexpr int k2_threads(int maxp) { return maxp >= 4 ? 12 * kWarp : kThreads2; }
-constexpr int kStage2 = 16 * 272;      // k2 chunk: 16 rows of <= 272 bytes
-constexpr int kStage3 = 16 * 336;      // k3 chunk: 16 rows of <= 336 bytes
+constexpr int kStage2 = 16 * 272;      // chunk: 16 rows of <= 272 bytes
 constexpr int kGpmBytes = 256 * 128;   // +/- codebook, 8 replicas
 constexpr int kSelBytes = 128 * 128;   // byte-permute selectors per sign mask, 16 replicas
 
@@ -85,10 +86,11 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
 
   if (blockIdx.x == 0) {
     const int V = T * d.k + T;
-    for (int i = tid; i < V; i += blockDim.x) {
+    for (int i = tid; i < V * a.s.NSL; i += blockDim.x) {
       a.s.hmax[i] = 0u;
       a.s.Xmax[i] = 0u;
-      a.s.vcount[i] = 0;
+      a.s.scount[i] = 0;
+      a.s.ready[i] = 0;
     }
     for (int i = tid; i < (1 + a.s.Jmax) * a.s.TM; i += blockDim.x) a.s.hcount[i] = 0;
     for (int i = tid; i < d.H / 16; i += blockDim.x) a.s.ycount[i] = 0;
@@ -564,8 +566,11 @@ __device__ __forceinline__ uint2 ldb(const BColS &b, int kel) {
 }
 __device__ __forceinline__ uint2 ldb(const BColG &b, int kel) {
   uint2 v = make_uint2(0u, 0u);
-  if (b.ok) v = __ldg(reinterpret_cast<const uint2 *>(b.p + kel));
+  if (b.ok) v = __ldcg(reinterpret_cast<const uint2 *>(b.p + kel));  // via L2: may be written by this kernel
   return v;
+}
+__device__ __forceinline__ uint32_t ldx(const BColG &b, int off) {
+  return b.ok ? __ldcg(reinterpret_cast<const unsigned *>(b.p + off)) : 0u;
 }
 
 // IQ2_XXS group of one staged row -> the A fragment halves of sub-vector c,
@@ -747,8 +752,7 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        uint32_t bx = 0;
-        if (xcol[p].ok) bx = *reinterpret_cast<const uint32_t *>(xcol[p].p + kb * 16);  // base includes 4c
+        const uint32_t bx = ldx(xcol[p], kb * 16);  // base includes 4c
         const int zero[4] = {0, 0, 0, 0};
         int cn[4];
         mma_s8(cn, Am, bx, 0u, zero);
@@ -890,12 +894,15 @@ struct K2Shared {
 };
 
 // Writes the 16 x ntok SwiGLU outputs held in hs (token slot, row) for the
-// vectors vec[slot], updates max|h|, the 16-row sum and the tile counters;
-// the warp that completes a vector quantises it.
-__device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int ntok, const int *vec, int r0, int n,
-                              int ntiles) {
+// vectors vec[slot] (rows r0.. of h), updates the slice maxima, the 16-row
+// sums and the slice's tile counter; the warp that completes a slice
+// (slice_len / 16 tiles) quantises it into limbs and then sets its ready flag.
+__device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int ntok, const int *vec, int r0,
+                              int slice_len) {
   const int lane = threadIdx.x & 31;
   const DecodeScratch &s = a.s;
+  const int sl = r0 / slice_len;
+  const int Im16 = s.Imax / 16;
   for (int base = 0; base < ntok; base += 2) {
     const int slot = base + (lane >> 4), row = lane & 15;
     const bool ok = slot < ntok;
@@ -910,9 +917,9 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
       const int v = vec[slot];
       s.hbuf[(size_t)v * s.Imax + r0 + row] = h;
       if (row == 0) {
-        s.Xbuf[(size_t)v * (s.Imax / 16) + r0 / 16] = sum;
-        atomicMax(s.hmax + v, __float_as_uint(m));
-        atomicMax(s.Xmax + v, __float_as_uint(fabsf(sum)));
+        s.Xbuf[(size_t)v * Im16 + r0 / 16] = sum;
+        atomicMax(s.hmax + v * s.NSL + sl, __float_as_uint(m));
+        atomicMax(s.Xmax + v * s.NSL + sl, __float_as_uint(fabsf(sum)));
       }
     }
   }
@@ -920,24 +927,59 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
   __syncwarp();
   for (int slot = 0; slot < ntok; ++slot) {
     const int v = vec[slot];
+    const int vs = v * s.NSL + sl;
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.vcount + v, 1) == ntiles - 1;
+    if (lane == 0) last = atomicAdd(s.scount + vs, 1) == slice_len / 16 - 1;
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
       __threadfence();
-      const float hm = __uint_as_float(__ldcg(s.hmax + v));
-      const float xm = __uint_as_float(__ldcg(s.Xmax + v));
-      quantise_vector(s.hbuf + (size_t)v * s.Imax, n, hm, s.hq + (size_t)v * 3 * s.Imax, s.Imax, s.hsc + 4 * v);
-      quantise_vector(s.Xbuf + (size_t)v * (s.Imax / 16), n / 16, xm, s.Xq + (size_t)v * 3 * (s.Imax / 16),
-                      s.Imax / 16, s.Xsc + 4 * v);
+      const float hm = __uint_as_float(__ldcg(s.hmax + vs));
+      const float xm = __uint_as_float(__ldcg(s.Xmax + vs));
+      const int k0 = sl * slice_len;
+      quantise_vector(s.hbuf + (size_t)v * s.Imax + k0, slice_len, hm, s.hq + (size_t)v * 3 * s.Imax + k0, s.Imax,
+                      s.hsc + 4 * vs);
+      quantise_vector(s.Xbuf + (size_t)v * Im16 + k0 / 16, slice_len / 16, xm,
+                      s.Xq + (size_t)v * 3 * Im16 + k0 / 16, Im16, s.Xsc + 4 * vs);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicExch(s.ready + vs, 1);
     }
   }
 }
 
-// XSMEM: the x limbs of all tokens are staged in shared memory (rows of
-// H + 32 bytes, which spreads the B-fragment loads over all banks).
+// Each lane with a flag waits (bounded) until it is set; the warp then reads
+// what the flag's writer published.  A flag that is never set records the
+// timeout error and lets the warp go on.
+__device__ void wait_slice(const int *flag, int *err) {
+  if (flag) {
+    const long long t0 = clock64();
+    while (true) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(flag) : "memory");
+      if (v) break;
+      if (clock64() - t0 > kSliceWaitCycles) {
+        set_error(err, kErrTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  __syncwarp();
+  __threadfence();
+}
+
+// The expert kernel: every unit of the layer's expert work, gate/up and
+// down, on one unit counter.
+//   units [0, n_sh)            shared gate/up (16-row tile of Is, K part of H)
+//   units [n_sh, n2)           routed gate/up (job, tile of I, K part of H)
+//   units [n2, n2 + n3s)       shared down (K part q of Is, 16-row tile of H)
+//   units [n2 + n3s, n_units)  routed down (job, K part of I, 16-row tile of H)
+// A down unit waits for the h slices it reads; every gate/up unit has been
+// claimed by a running warp before the first down unit is claimed, so the
+// waits end.  XSMEM: the x limbs of all tokens are staged in shared memory
+// (rows of H + 32 bytes, which spreads the B-fragment loads over all banks).
 template <int MAXP, bool XSMEM>
-__global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
+__global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const LayerDims &d = a.d;
   const DecodeScratch &s = a.s;
@@ -951,7 +993,6 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   build_tables(a.wt.grid, gpm, selt, a.err);
-  pdl_launch_dependents();
   pdl_wait();  // k1's limbs and keys are visible from here on
   if (XSMEM) {
     const int n16 = d.H / 16;
@@ -966,8 +1007,6 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
     }
   }
   build_jobs(S.idx, T, d.k, S.J);
-  if (blockIdx.x == 0)
-    for (int i = tid; i < kJobsInts; i += blockDim.x) s.jobs[i] = reinterpret_cast<const int *>(&S.J)[i];
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
   const uint8_t *sel_l = selt + (lane & 15) * 8;
@@ -979,85 +1018,137 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
   auto xcol = [&](int t, int limb) -> const int8_t * {
     return (XSMEM ? xsm + (size_t)(t * 3 + limb) * XS : s.xq + ((size_t)t * 3 + limb) * d.H) + 8 * c;
   };
+  // limb `limb` of vector v of h (and of its 16-element sums), offset likewise
+  auto hcol = [&](int v, int limb) -> const int8_t * { return s.hq + ((size_t)v * 3 + limb) * s.Imax + 8 * c; };
+  auto Xcol = [&](int v, int limb) -> const int8_t * {
+    return s.Xq + ((size_t)v * 3 + limb) * (s.Imax / 16) + 4 * c;
+  };
 
+  // ---- gate/up geometry
   const int tilesI = d.I / 16, tilesS = d.Is / 16;
   const int PH = s.PH;
-  const int kpart = d.H / PH;  // K elements per unit
+  const int kpart = d.H / PH;  // K elements of a gate/up unit
   const int cbI = kpart / 256;  // IQ2_XXS blocks per unit (4, 2 or 1): one chunk per matrix
   const int nq8 = kpart / 256;  // Q8_0 chunks of 8 blocks per unit and matrix
   const size_t rbI = (size_t)(d.H / 256) * 66;
   const size_t rbQ = (size_t)(d.H / 32) * 34;
   const int V = T * d.k + T;
+  // ---- down geometry
+  const int tilesH = d.H / 16;
+  const int PD = s.PD, PS = s.PS;
+  const int kpd = d.I / PD;           // K elements of a routed down unit (one slice)
+  const int cbD = kpd / 256;          // Q2_K blocks per routed down unit
+  const int nbD = cbD < 2 ? cbD : 2;  // Q2_K blocks per chunk (rows of <= 168 bytes)
+  const int kps = d.Is / PS;          // K elements of a shared down unit (one slice)
+  const int nqd = kps / 256;          // Q8_0 chunks of 8 blocks per shared down unit
+  const size_t rbD = (size_t)(d.I / 256) * 84;
+  const size_t rbQd = (size_t)(d.Is / 32) * 34;
+  const int nparts = S.J.n * PD + PS;  // parts of an output tile
+  const int NS = s.NS;
+  // ---- unit ranges
   const int n_sh = tilesS * PH;
-  const int n_units = n_sh + S.J.n * tilesI * PH;
+  const int n2 = n_sh + S.J.n * tilesI * PH;
+  const int n3s = PS * tilesH;
+  const int n_units = n2 + n3s + S.J.n * PD * tilesH;
 
-  // ---- units: shared (tile, part), then routed (job, tile, part); the key
-  // u / PH names the (vector set, tile), so a tile's parts are consecutive.
-  // Consecutive parts of one tile that a warp computes in a row form a
-  // segment; the tile's counter is bumped once per segment.
   struct Unit {
-    bool shared;
-    int j, e, tile, part, ntok, per, nch;  // per: chunks per matrix
+    int kind;  // 0 shared gate/up, 1 routed gate/up, 2 shared down, 3 routed down
+    int j, e, tile, part, ntok, per, nch;  // gate/up: 16-row tile, K part of H, chunks per matrix
+    int ot, kp;                            // down: output tile, K part (slice) of I or Is
     const int *pairs;
   };
   auto unit_at = [&](int u) {
     Unit x;
-    x.shared = u < n_sh;
-    x.j = 0;
-    x.e = 0;
+    x.j = x.e = x.tile = x.part = x.ot = x.kp = 0;
+    x.per = 1;
     x.pairs = nullptr;
-    if (x.shared) {
+    x.ntok = T;
+    if (u < n_sh) {
+      x.kind = 0;
       x.tile = u / PH;
       x.part = u % PH;
-      x.ntok = T;
       x.per = nq8;
-    } else {
+      x.nch = 2 * nq8;
+    } else if (u < n2) {
+      x.kind = 1;
       const int uu = u - n_sh;
       x.j = uu / (tilesI * PH);
       const int rem = uu % (tilesI * PH);
       x.tile = rem / PH;
       x.part = rem % PH;
+      x.nch = 2;
+    } else if (u < n2 + n3s) {
+      x.kind = 2;
+      const int w = u - n2;
+      x.kp = w / tilesH;
+      x.ot = w % tilesH;
+      x.nch = nqd;
+    } else {
+      x.kind = 3;
+      const int w = u - n2 - n3s;
+      const int jp = w / tilesH;
+      x.j = jp / PD;
+      x.kp = jp % PD;
+      x.ot = w % tilesH;
+      x.nch = cbD / nbD;
+    }
+    if (x.kind & 1) {
       x.e = S.J.e[x.j];
       x.ntok = S.J.cnt[x.j];
       x.pairs = S.J.pair + S.J.first[x.j];
-      x.per = 1;
     }
-    x.nch = 2 * x.per;
     return x;
   };
   // token slot ts of a unit -> row of x / vector of h
-  auto xrow = [&](const Unit &x, int ts) { return x.shared ? ts : x.pairs[ts] / d.k; };
-  auto hvec = [&](const Unit &x, int ts) { return x.shared ? T * d.k + ts : x.pairs[ts]; };
+  auto xrow = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] / d.k : ts; };
+  auto hvec = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] : T * d.k + ts; };
   auto chunk_of = [&](const Unit &su, int cs) {
-    const bool up = cs >= su.per;
-    const int ck = cs % su.per;
     Chunk ch;
-    if (su.shared) {
+    if (su.kind == 0) {
+      const bool up = cs >= su.per;
+      const int ck = cs % su.per;
       const size_t off = (size_t)(su.part * kpart / 32 + ck * 8) * 34;
       ch.g = (up ? a.wt.sh_up : a.wt.sh_gate) + (size_t)(su.tile * 16) * rbQ + off;
       ch.gstride = rbQ;
       ch.bpr = 8 * 34;
       ch.nb = 8;
       ch.k0 = su.part * kpart + ck * 256;
-      ch.piece = piece_for(rbQ, off, ch.bpr);
-    } else {
+      ch.align = 4;
+    } else if (su.kind == 1) {
       const size_t off = (size_t)su.part * cbI * 66;
-      ch.g = (up ? a.wt.up : a.wt.gate) + ((size_t)su.e * d.I + su.tile * 16) * rbI + off;
+      ch.g = (cs ? a.wt.up : a.wt.gate) + ((size_t)su.e * d.I + su.tile * 16) * rbI + off;
       ch.gstride = rbI;
       ch.bpr = cbI * 66;
       ch.nb = cbI;
       ch.k0 = su.part * kpart;
-      ch.piece = piece_for(rbI, off, ch.bpr);
+      ch.align = 4;
+    } else if (su.kind == 2) {
+      const size_t off = (size_t)(su.kp * kps / 32 + cs * 8) * 34;
+      ch.g = a.wt.sh_down + (size_t)(su.ot * 16) * rbQd + off;
+      ch.gstride = rbQd;
+      ch.bpr = 8 * 34;
+      ch.nb = 8;
+      ch.k0 = su.kp * kps + cs * 256;
+      ch.align = 4;
+    } else {
+      const size_t off = (size_t)(su.kp * cbD + cs * nbD) * 84;
+      ch.g = a.wt.down + ((size_t)su.e * d.H + su.ot * 16) * rbD + off;
+      ch.gstride = rbD;
+      ch.bpr = nbD * 84;
+      ch.nb = nbD;
+      ch.k0 = su.kp * kpd + cs * nbD * 256;
+      ch.align = 8;
     }
-    ch.align = 4;
+    ch.piece = piece_for(ch.gstride, reinterpret_cast<uintptr_t>(ch.g) & 15, ch.bpr);
     return ch;
   };
 
   int seg_parts = 0, npairs = 0;
   BCol bcol[MAXP];
-  // F accumulates gate, then up, of one unit; each matrix's sums are combined
-  // over limbs and stored as the partials of the unit's K part (m = 0 gate, 1 up)
-  float F[MAXP][4] = {};
+  BColG hb[MAXP], xb[MAXP];
+  float F[MAXP][4] = {}, G[MAXP][4] = {};
+  // gate/up: each matrix's sums of a unit are combined over limbs and stored as
+  // the partials of the unit's K part (m = 0 gate, 1 up)
   auto store_part = [&](const Unit &cu, int m) {
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
@@ -1074,12 +1165,12 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
       F[p][0] = F[p][1] = F[p][2] = F[p][3] = 0.f;
     }
   };
-  // count the segment's parts in; the warp that completes the tile sums the
-  // parts in order and applies the SwiGLU
-  auto end_segment = [&](const Unit &cu) {
+  // gate/up: count the segment's parts in; the warp that completes the tile
+  // sums the parts in order, applies the SwiGLU and hands the tile on
+  auto end_gateup = [&](const Unit &cu) {
     __threadfence();
     __syncwarp();
-    const int set = cu.shared ? 0 : 1 + cu.j;
+    const int set = cu.kind == 0 ? 0 : 1 + cu.j;
     int last = 0;
     if (lane == 0) last = atomicAdd(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
     last = __shfl_sync(0xffffffffu, last, 0);
@@ -1111,164 +1202,17 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_gateup(DecodeArgs a) {
     int vec[kDecodeMaxT];
 #pragma unroll
     for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < cu.ntok ? hvec(cu, t) : 0;
-    finish_h_tile(a, S.hsm[warp], cu.ntok, vec, r0, cu.shared ? d.Is : d.I, cu.shared ? tilesS : tilesI);
+    finish_h_tile(a, S.hsm[warp], cu.ntok, vec, r0, cu.kind == 0 ? kps : kpd);
   };
-
-  run_units<kClaim, kAheadClaim, Unit>(st0, st1, s.work + 0, n_units, unit_at, chunk_of,
-                     [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
-                       if (cc == 0) {
-                         npairs = (cu.ntok + 1) >> 1;
-#pragma unroll
-                         for (int p = 0; p < MAXP; ++p) {
-                           const int ts = 2 * p + (r >> 2), limb = r & 3;
-                           bcol[p].ok = ts < cu.ntok && limb < 3;
-                           bcol[p].p = bcol[p].ok ? xcol(xrow(cu, ts), limb) : nullptr;
-                         }
-                       }
-                       if (cu.shared) {
-                         q80_chunk<8, MAXP>(st, cu.part * kpart + (cc % nq8) * 256, bcol, npairs, F);
-                       } else if (cbI == 4) {
-                         iq2_chunk<4, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
-                       } else if (cbI == 2) {
-                         iq2_chunk<2, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
-                       } else {
-                         iq2_chunk<1, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
-                       }
-                       if (cc == cu.per - 1) store_part(cu, 0);
-                       if (cc == cu.nch - 1) {
-                         store_part(cu, 1);
-                         ++seg_parts;
-                         if (next_u != u + 1 || (u + 1) / PH != u / PH) end_segment(cu);
-                       }
-                     });
-}
-
-// ------------------------------------------------------------------ k3
-
-struct K3Shared {
-  int32_t idx[kDecodeMaxT * kMaxK];
-  float w[kDecodeMaxT * kMaxK];
-  Jobs J;
-};
-
-// Shared-memory rows of the h limbs (HSMEM): Imax + 32 bytes per limb row of
-// h and Imax/16 + 16 bytes per limb row of the 16-element sums.
-__host__ __device__ inline size_t k3_hrow(int Imax) { return (size_t)Imax + 32; }
-__host__ __device__ inline size_t k3_xrow(int Imax) { return (size_t)Imax / 16 + 16; }
-
-template <int MAXP, bool HSMEM>
-__global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const LayerDims &d = a.d;
-  const DecodeScratch &s = a.s;
-  const int T = a.T;
-  uint8_t *stages = smem;
-  K3Shared &S = *reinterpret_cast<K3Shared *>(stages + 2 * kWarps2 * kStage3);
-  int8_t *hsm = reinterpret_cast<int8_t *>(reinterpret_cast<uint8_t *>(&S) + align_up(sizeof(K3Shared), 128));
-  const int V = T * d.k + T;
-  const int Im16 = s.Imax / 16;
-  const size_t HR = k3_hrow(s.Imax), XR = k3_xrow(s.Imax);
-  int8_t *xsm = hsm + (size_t)V * 3 * HR;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();  // k2's routing, job table and h limbs are visible from here on
-  for (int i = tid; i < T * d.k; i += blockDim.x) {
-    S.idx[i] = __ldcg(s.idx + i);
-    S.w[i] = __ldcg(s.w + i);
-  }
-  for (int i = tid; i < kJobsInts; i += blockDim.x) reinterpret_cast<int *>(&S.J)[i] = __ldcg(s.jobs + i);
-  if (HSMEM) {
-    copy_rows16(hsm, HR, s.hq, s.Imax, V * 3, s.Imax / 16);
-    copy_rows16(xsm, XR, s.Xq, Im16, V * 3, Im16 / 16);
-  }
-  __syncthreads();
-
-  uint8_t *st0 = stages + warp * 2 * kStage3;
-  uint8_t *st1 = st0 + kStage3;
-  const int r = lane >> 2, c = lane & 3;
-  using BCol = typename std::conditional<HSMEM, BColS, BColG>::type;
-  // limb `limb` of vector v (h, and its 16-element sums), offset by this lane's sub-range
-  auto hcol = [&](int v, int limb) -> const int8_t * {
-    return (HSMEM ? hsm + ((size_t)v * 3 + limb) * HR : s.hq + ((size_t)v * 3 + limb) * s.Imax) + 8 * c;
-  };
-  auto Xcol = [&](int v, int limb) -> const int8_t * {
-    return (HSMEM ? xsm + ((size_t)v * 3 + limb) * XR : s.Xq + ((size_t)v * 3 + limb) * Im16) + 4 * c;
-  };
-  const int tilesH = d.H / 16;
-  const int PD = s.PD, PS = s.PS;
-  const int kpd = d.I / PD;      // K elements of a routed unit
-  const int cbD = kpd / 256;     // Q2_K blocks per routed unit (4, 2 or 1): one chunk
-  const int kps = d.Is / PS;     // K elements of a shared unit
-  const int nq8 = kps / 256;     // Q8_0 chunks of 8 blocks per shared unit
-  const size_t rbD = (size_t)(d.I / 256) * 84;
-  const size_t rbQ = (size_t)(d.Is / 32) * 34;
-  const int nrp = S.J.n * PD;    // routed parts of an output tile
-  const int nparts = nrp + PS;
-  const int n_units = tilesH * nparts;
-  const int NS = s.NS;
-
-  // ---- units (output tile ot, part), part fastest: routed parts (job, K
-  // part), then the shared parts; consecutive parts of one output tile that a
-  // warp computes in a row form a segment (see k2)
-  struct Unit {
-    int ot, part, j, kp, q, e, ntok, nch;
-    const int *pairs;
-  };
-  auto unit_at = [&](int u) {
-    Unit x;
-    x.ot = u / nparts;
-    x.part = u % nparts;
-    x.j = x.kp = x.q = x.e = 0;
-    x.pairs = nullptr;
-    if (x.part < nrp) {
-      x.j = x.part / PD;
-      x.kp = x.part % PD;
-      x.e = S.J.e[x.j];
-      x.ntok = S.J.cnt[x.j];
-      x.pairs = S.J.pair + S.J.first[x.j];
-      x.nch = 1;
-    } else {
-      x.q = x.part - nrp;
-      x.ntok = T;
-      x.nch = nq8;
-    }
-    return x;
-  };
-  auto chunk_of = [&](const Unit &su, int cs) {
-    Chunk ch;
-    if (su.part < nrp) {
-      const size_t off = (size_t)su.kp * cbD * 84;
-      ch.g = a.wt.down + ((size_t)su.e * d.H + su.ot * 16) * rbD + off;
-      ch.gstride = rbD;
-      ch.bpr = cbD * 84;
-      ch.nb = cbD;
-      ch.k0 = su.kp * kpd;
-      ch.piece = piece_for(rbD, off, ch.bpr);
-      ch.align = 8;
-    } else {
-      const size_t off = (size_t)(su.q * kps / 32 + cs * 8) * 34;
-      ch.g = a.wt.sh_down + (size_t)(su.ot * 16) * rbQ + off;
-      ch.gstride = rbQ;
-      ch.bpr = 8 * 34;
-      ch.nb = 8;
-      ch.k0 = su.q * kps + cs * 256;
-      ch.piece = piece_for(rbQ, off, ch.bpr);
-      ch.align = 4;
-    }
-    return ch;
-  };
-
-  int seg_parts = 0, npairs = 0;
-  BCol bcol[MAXP], xcolv[MAXP];
-  float F[MAXP][4] = {}, G[MAXP][4] = {};
-  auto end_segment = [&](const Unit &cu) {
+  // down: the part is in its slot; the warp that completes the output tile
+  // sums its slots in a fixed order into y
+  auto end_down = [&](const Unit &cu) {
     __threadfence();
     __syncwarp();
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.ycount + cu.ot, seg_parts) + seg_parts == nparts;
+    if (lane == 0) last = atomicAdd(s.ycount + cu.ot, 1) == nparts - 1;
     last = __shfl_sync(0xffffffffu, last, 0);
-    seg_parts = 0;
     if (!last) return;
-    // every part of the tile is in: sum them in a fixed order into y
     __threadfence();
     const int r0 = cu.ot * 16;
     const float *ytile = s.ypart + (size_t)cu.ot * NS * 16;
@@ -1294,72 +1238,102 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
   };
 
   run_units<kClaim, kAheadClaim, Unit>(
-      st0, st1, s.work + 1, n_units, unit_at, chunk_of,
+      st0, st1, s.work + 0, n_units, unit_at, chunk_of,
       [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
+        if (cu.kind <= 1) {
+          // ------------------------------------------------ gate/up
+          if (cc == 0) {
+            npairs = (cu.ntok + 1) >> 1;
+#pragma unroll
+            for (int p = 0; p < MAXP; ++p) {
+              const int ts = 2 * p + (r >> 2), limb = r & 3;
+              bcol[p].ok = ts < cu.ntok && limb < 3;
+              bcol[p].p = bcol[p].ok ? xcol(xrow(cu, ts), limb) : nullptr;
+            }
+          }
+          if (cu.kind == 0) {
+            q80_chunk<8, MAXP>(st, cu.part * kpart + (cc % nq8) * 256, bcol, npairs, F);
+          } else if (cbI == 4) {
+            iq2_chunk<4, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+          } else if (cbI == 2) {
+            iq2_chunk<2, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+          } else {
+            iq2_chunk<1, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
+          }
+          if (cc == cu.per - 1) store_part(cu, 0);
+          if (cc == cu.nch - 1) {
+            store_part(cu, 1);
+            ++seg_parts;
+            if (next_u != u + 1 || u + 1 >= n2 || (u + 1) / PH != u / PH) end_gateup(cu);
+          }
+          return;
+        }
+        // -------------------------------------------------- down
         if (cc == 0) {
+          // the h slices this unit reads: one per token slot
+          wait_slice(lane < cu.ntok ? s.ready + hvec(cu, lane) * s.NSL + cu.kp : nullptr, a.err);
           npairs = (cu.ntok + 1) >> 1;
 #pragma unroll
           for (int p = 0; p < MAXP; ++p) {
             const int ts = 2 * p + (r >> 2), limb = r & 3;
             const bool ok = ts < cu.ntok && limb < 3;
-            const int v = !ok ? 0 : cu.part < nrp ? cu.pairs[ts] : T * d.k + ts;
-            bcol[p].ok = xcolv[p].ok = ok;
-            bcol[p].p = ok ? hcol(v, limb) : nullptr;
-            xcolv[p].p = ok ? Xcol(v, limb) : nullptr;
+            const int v = ok ? hvec(cu, ts) : 0;
+            hb[p].ok = xb[p].ok = ok;
+            hb[p].p = ok ? hcol(v, limb) : nullptr;
+            xb[p].p = ok ? Xcol(v, limb) : nullptr;
           }
         }
         float *ytile = s.ypart + (size_t)cu.ot * NS * 16;
-        if (cu.part < nrp) {
-          // ---- routed: expert j, K part kp of I
-          if (cbD == 4)
-            q2k_chunk<4, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
-          else if (cbD == 2)
-            q2k_chunk<2, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
+        if (cu.kind == 3) {
+          if (nbD == 2)
+            q2k_chunk<2, MAXP>(st, cu.kp * kpd + cc * 512, hb, xb, npairs, F, G);
           else
-            q2k_chunk<1, MAXP>(st, cu.kp * kpd, bcol, xcolv, npairs, F, G);
-#pragma unroll
-          for (int p = 0; p < MAXP; ++p) {
-            if (p < npairs) {
-              const int ts = 2 * p + (c >> 1);
-              const bool ok = ts < cu.ntok;
-              const int v = ok ? cu.pairs[ts] : 0;
-              const int l0 = 2 * (c & 1);
-              float v0 = 0.f, v1 = 0.f;
-              if (ok) {
-                const float *hs = s.hsc + 4 * v;
-                const float *xs = s.Xsc + 4 * v;
-                v0 = hs[l0] * F[p][0] - xs[l0] * G[p][0];
-                v1 = hs[l0] * F[p][2] - xs[l0] * G[p][2];
-                if (l0 + 1 < 3) {
-                  v0 += hs[l0 + 1] * F[p][1] - xs[l0 + 1] * G[p][1];
-                  v1 += hs[l0 + 1] * F[p][3] - xs[l0 + 1] * G[p][3];
-                }
-              }
-              v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-              v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-              if ((c & 1) == 0 && ok) {
-                const float wt = S.w[v];
-                float *dst = ytile + (size_t)(v * PD + cu.kp) * 16;
-                dst[r] = wt * v0;
-                dst[r + 8] = wt * v1;
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
-          }
-        } else {
-          // ---- shared: K part q of Is
-          q80_chunk<8, MAXP>(st, cu.q * kps + cc * 256, bcol, npairs, F);
-          if (cc == nq8 - 1) {
+            q2k_chunk<1, MAXP>(st, cu.kp * kpd + cc * 256, hb, xb, npairs, F, G);
+          if (cc == cu.nch - 1) {
 #pragma unroll
             for (int p = 0; p < MAXP; ++p) {
               if (p < npairs) {
                 const int ts = 2 * p + (c >> 1);
-                const float *sc = ts < T ? s.hsc + 4 * (T * d.k + ts) : nullptr;
+                const bool ok = ts < cu.ntok;
+                const int v = ok ? cu.pairs[ts] : 0;
+                const int l0 = 2 * (c & 1);
+                float v0 = 0.f, v1 = 0.f;
+                if (ok) {
+                  const float *hs = s.hsc + 4 * (v * s.NSL + cu.kp);
+                  const float *xs = s.Xsc + 4 * (v * s.NSL + cu.kp);
+                  v0 = hs[l0] * F[p][0] - xs[l0] * G[p][0];
+                  v1 = hs[l0] * F[p][2] - xs[l0] * G[p][2];
+                  if (l0 + 1 < 3) {
+                    v0 += hs[l0 + 1] * F[p][1] - xs[l0 + 1] * G[p][1];
+                    v1 += hs[l0 + 1] * F[p][3] - xs[l0 + 1] * G[p][3];
+                  }
+                }
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                if ((c & 1) == 0 && ok) {
+                  const float wt = S.w[v];
+                  float *dst = ytile + (size_t)(v * PD + cu.kp) * 16;
+                  dst[r] = wt * v0;
+                  dst[r + 8] = wt * v1;
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) F[p][i] = G[p][i] = 0.f;
+            }
+            end_down(cu);
+          }
+        } else {
+          q80_chunk<8, MAXP>(st, cu.kp * kps + cc * 256, hb, npairs, F);
+          if (cc == cu.nch - 1) {
+#pragma unroll
+            for (int p = 0; p < MAXP; ++p) {
+              if (p < npairs) {
+                const int ts = 2 * p + (c >> 1);
+                const float *sc = ts < T ? s.hsc + 4 * ((T * d.k + ts) * s.NSL + cu.kp) : nullptr;
                 float v0, v1;
                 combine_limbs(F[p], sc, v0, v1);
                 if ((c & 1) == 0 && ts < T) {
-                  float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + cu.q) * 16;
+                  float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + cu.kp) * 16;
                   dst[r] = v0;
                   dst[r + 8] = v1;
                 }
@@ -1367,11 +1341,8 @@ __global__ void __launch_bounds__(kThreads2, 1) k3_down(DecodeArgs a) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) F[p][i] = 0.f;
             }
+            end_down(cu);
           }
-        }
-        if (cc == cu.nch - 1) {
-          ++seg_parts;
-          if (next_u != u + 1 || (u + 1) / nparts != u / nparts) end_segment(cu);
         }
       });
 }
@@ -1389,12 +1360,6 @@ size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
   if (xsmem) b += (size_t)T * 3 * (d.H + 32);
   return b;
 }
-size_t k3_smem_bytes(const DecodeScratch &s, int T, int k, bool hsmem) {
-  size_t b = 2 * kWarps2 * kStage3 + align_up(sizeof(K3Shared), 128);
-  if (hsmem) b += (size_t)(T * k + T) * 3 * (k3_hrow(s.Imax) + k3_xrow(s.Imax));
-  return b;
-}
-
 constexpr size_t kSmemLimit = 227 * 1024;
 
 template <typename K>
@@ -1412,23 +1377,21 @@ cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int MAXP, bool XSMEM, bool HSMEM>
-cudaError_t launch_k23(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
+template <int MAXP, bool XSMEM>
+cudaError_t launch_k2(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k2_gateup<MAXP, XSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k2_experts<MAXP, XSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemLimit);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k3_down<MAXP, HSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
   cudaError_t e =
-      launch_pdl(k2_gateup<MAXP, XSMEM>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
+      launch_pdl(k2_experts<MAXP, XSMEM>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
   if (e != cudaSuccess) return e;
   if (a.ev_end) cudaEventRecord(a.ev_end, stream);
-  return launch_pdl(k3_down<MAXP, HSMEM>, num_sms, kThreads2, k3_smem_bytes(a.s, a.T, a.d.k, HSMEM), stream, a);
+  return cudaSuccess;
 }
 
 cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
@@ -1470,6 +1433,7 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.Jmax = T * d.k < d.E ? T * d.k : d.E;
   s.TM = Imax / 16;
   s.NS = T * d.k * s.PD + T * s.PS;
+  s.NSL = s.PD > s.PS ? s.PD : s.PS;
   s.z = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.sc = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * T * d.k));
@@ -1478,13 +1442,14 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.xs = reinterpret_cast<float *>(take(sizeof(float) * 4 * T));
   s.hbuf = reinterpret_cast<float *>(take(sizeof(float) * (size_t)V * Imax));
   s.hq = reinterpret_cast<int8_t *>(take((size_t)V * 3 * Imax));
-  s.hsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V));
+  s.hsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V * s.NSL));
   s.Xbuf = reinterpret_cast<float *>(take(sizeof(float) * (size_t)V * (Imax / 16)));
   s.Xq = reinterpret_cast<int8_t *>(take((size_t)V * 3 * (Imax / 16)));
-  s.Xsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V));
-  s.hmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
-  s.Xmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V));
-  s.vcount = reinterpret_cast<int *>(take(sizeof(int) * V));
+  s.Xsc = reinterpret_cast<float *>(take(sizeof(float) * 4 * V * s.NSL));
+  s.hmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V * s.NSL));
+  s.Xmax = reinterpret_cast<unsigned *>(take(sizeof(unsigned) * V * s.NSL));
+  s.scount = reinterpret_cast<int *>(take(sizeof(int) * V * s.NSL));
+  s.ready = reinterpret_cast<int *>(take(sizeof(int) * V * s.NSL));
   s.gpart = reinterpret_cast<float *>(take(sizeof(float) * 2 * (size_t)s.PH * V * Imax));
   s.hcount = reinterpret_cast<int *>(take(sizeof(int) * (size_t)(1 + s.Jmax) * s.TM));
   s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * s.NS * 16));
@@ -1497,14 +1462,11 @@ cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms
   cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
   if (a.T <= 2) {
-    const bool xs = k2_smem_bytes(a.d, a.T, true) <= kSmemLimit;
-    const bool hs = k3_smem_bytes(a.s, a.T, a.d.k, true) <= kSmemLimit;
-    if (xs && hs) return launch_k23<1, true, true>(a, stream, num_sms);
-    if (xs) return launch_k23<1, true, false>(a, stream, num_sms);
-    return launch_k23<1, false, false>(a, stream, num_sms);
+    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2<1, true>(a, stream, num_sms);
+    return launch_k2<1, false>(a, stream, num_sms);
   }
-  if (a.T <= 4) return launch_k23<2, false, false>(a, stream, num_sms);
-  return launch_k23<4, false, false>(a, stream, num_sms);
+  if (a.T <= 4) return launch_k2<2, false>(a, stream, num_sms);
+  return launch_k2<4, false>(a, stream, num_sms);
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {

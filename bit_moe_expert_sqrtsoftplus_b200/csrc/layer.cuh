@@ -38,7 +38,10 @@ __host__ __device__ inline int decode_kparts(int K) { return (K % kDecodeKPart =
 constexpr int kJobsInts = 1 + 5 * kDecodeMaxT * kMaxK;
 
 // Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
-// t*k + slot, shared vector T*k + t.
+// t*k + slot, shared vector T*k + t.  The SwiGLU output h of a vector is
+// quantised slice by slice: a slice is the K range of one down-projection
+// unit (I/PD elements for a routed vector, Is/PS for a shared one), NSL =
+// max(PD, PS) slices per vector.
 struct DecodeScratch {
   double *z;        // [T][E] selection keys sqrtsoftplus(z) + bias (fp64)
   double *sc;       // [T][E] scores sqrtsoftplus(z) (fp64)
@@ -47,22 +50,24 @@ struct DecodeScratch {
   int8_t *xq;       // [T][3][H] int8 limbs of the expert input
   float *xs;        // [T][4] limb scales
   float *hbuf;      // [V][Imax] SwiGLU outputs
-  int8_t *hq;       // [V][3][Imax]
-  float *hsc;       // [V][4]
+  int8_t *hq;       // [V][3][Imax] int8 limbs of h
+  float *hsc;       // [V][NSL][4] limb scales per slice
   float *Xbuf;      // [V][Imax/16] sums of 16 consecutive h
   int8_t *Xq;       // [V][3][Imax/16]
-  float *Xsc;       // [V][4]
-  unsigned *hmax;   // [V] max |h| (float bits)
-  unsigned *Xmax;   // [V]
-  int *vcount;      // [V] finished 16-row tiles per vector
+  float *Xsc;       // [V][NSL][4]
+  unsigned *hmax;   // [V][NSL] max |h| per slice (float bits)
+  unsigned *Xmax;   // [V][NSL]
+  int *scount;      // [V][NSL] finished 16-row tiles per slice
+  int *ready;       // [V][NSL] 1 once the slice's limbs are written
   float *gpart;     // [2][PH][V][Imax] gate/up partial sums per K part of H
   int *hcount;      // [1 + Jmax][TM] finished K parts per (vector set, 16-row tile)
   float *ypart;     // [H/16][NS][16] partial output tiles, NS = T*k*PD + T*PS slots
   int *ycount;      // [H/16]
   int *work;        // [4] unit counters
-  int *jobs;        // [kJobsInts] job table written by k2 for k3
+  int *jobs;        // [kJobsInts] job table (first block of the expert kernel)
   int Imax;
   int PH, PD, PS;   // K parts of H (gate/up), I (routed down), Is (shared down)
+  int NSL;          // slices per vector = max(PD, PS)
   int Jmax;         // max routed vector sets = min(T*k, E)
   int TM;           // max(I, Is) / 16
   int NS;           // output slots per 16-row tile of y
@@ -77,7 +82,7 @@ struct DecodeArgs {
   float *y;
   DecodeScratch s;
   int *err;
-  cudaEvent_t ev_begin, ev_end;  // recorded around k2 when set
+  cudaEvent_t ev_begin, ev_end;  // recorded around the expert kernel when set
 };
 
 size_t decode_scratch_bytes(const LayerDims &d, int T);
