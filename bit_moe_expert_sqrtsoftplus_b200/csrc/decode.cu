@@ -84,29 +84,51 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
   __shared__ double red[NW][3 * MAXT];
   __shared__ float redf[NW];
 
-  if (blockIdx.x == 0) {
+  {
+    // per-call counters and flags of the expert kernel, spread over the grid
     const int V = T * d.k + T;
-    for (int i = tid; i < V * a.s.NSL; i += blockDim.x) {
-      a.s.hmax[i] = 0u;
-      a.s.Xmax[i] = 0u;
-      a.s.scount[i] = 0;
-      a.s.ready[i] = 0;
+    const int nv = V * a.s.NSL, nh = (1 + a.s.Jmax) * a.s.TM, ny = d.H / 16;
+    for (int i = blockIdx.x * blockDim.x + tid; i < nv + nh + ny + 4; i += gridDim.x * blockDim.x) {
+      if (i < nv) {
+        a.s.hmax[i] = 0u;
+        a.s.Xmax[i] = 0u;
+        a.s.scount[i] = 0;
+        a.s.ready[i] = 0;
+      } else if (i < nv + nh) {
+        a.s.hcount[i - nv] = 0;
+      } else if (i < nv + nh + ny) {
+        a.s.ycount[i - nv - nh] = 0;
+      } else {
+        a.s.work[i - nv - nh - ny] = 0;
+      }
     }
-    for (int i = tid; i < (1 + a.s.Jmax) * a.s.TM; i += blockDim.x) a.s.hcount[i] = 0;
-    for (int i = tid; i < d.H / 16; i += blockDim.x) a.s.ycount[i] = 0;
-    if (tid < 4) a.s.work[tid] = 0;
   }
 
   if ((int)blockIdx.x < T) {
-    // ---- activation limbs for token t
+    // ---- activation limbs for token t; every thread takes float4 words
+    // tid, tid + 256, ... and loads a batch of them before using any
     const int t = blockIdx.x;
-    const float *xt = a.x + (size_t)t * d.H;
+    const float4 *xt = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H);
+    const int n4 = d.H / 4;
+    constexpr int kB = 4;
     double ss = 0.0;
     float amax = 0.f;
-    for (int j = tid; j < d.H; j += blockDim.x) {
-      const float v = xt[j];
-      ss += (double)v * (double)v;
-      amax = fmaxf(amax, fabsf(v));
+    for (int j0 = tid; j0 < n4; j0 += kB * kRouterThreads) {
+      float4 v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int j = j0 + u * kRouterThreads;
+        v[u] = j < n4 ? xt[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          ss += (double)e[q] * (double)e[q];
+          amax = fmaxf(amax, fabsf(e[q]));
+        }
+      }
     }
     ss = warp_sum_d(ss);
     amax = warp_max(amax);
@@ -129,24 +151,44 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
     const float s1 = amax > 0.f ? amax / 127.f : 1.f;
     const float s2 = s1 / 254.f, s3 = s2 / 254.f;
     const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
-    int8_t *q = a.s.xq + (size_t)t * 3 * d.H;
-    for (int j = tid; j < d.H; j += blockDim.x) {
-      const float v = xt[j] * inv;
-      const float q1 = fminf(fmaxf(rintf(v * r1), -127.f), 127.f);
-      const float e1 = fmaf(-q1, s1, v);
-      const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
-      const float e2 = fmaf(-q2, s2, e1);
-      const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
-      q[j] = (int8_t)q1;
-      q[d.H + j] = (int8_t)q2;
-      q[2 * d.H + j] = (int8_t)q3;
+    uint32_t *q = reinterpret_cast<uint32_t *>(a.s.xq + (size_t)t * 3 * d.H);
+    for (int j0 = tid; j0 < n4; j0 += kB * kRouterThreads) {
+      float4 v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int j = j0 + u * kRouterThreads;
+        v[u] = j < n4 ? xt[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int j = j0 + u * kRouterThreads;
+        if (j < n4) {
+          const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t w1 = 0u, w2 = 0u, w3 = 0u;
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const float x = e[k4] * inv;
+            const float q1 = fminf(fmaxf(rintf(x * r1), -127.f), 127.f);
+            const float e1 = fmaf(-q1, s1, x);
+            const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+            const float e2 = fmaf(-q2, s2, e1);
+            const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+            w1 |= ((uint32_t)(int)q1 & 255u) << (8 * k4);
+            w2 |= ((uint32_t)(int)q2 & 255u) << (8 * k4);
+            w3 |= ((uint32_t)(int)q3 & 255u) << (8 * k4);
+          }
+          q[j] = w1;
+          q[n4 + j] = w2;
+          q[2 * n4 + j] = w3;
+        }
+      }
     }
     if (tid == 0) {
-      float *s = a.s.xs + 4 * t;
-      s[0] = s1;
-      s[1] = s2;
-      s[2] = s3;
-      s[3] = 0.f;
+      float *sx = a.s.xs + 4 * t;
+      sx[0] = s1;
+      sx[1] = s2;
+      sx[2] = s3;
+      sx[3] = 0.f;
     }
     return;
   }
@@ -337,34 +379,38 @@ struct Jobs {
 };
 static_assert(sizeof(Jobs) == sizeof(int) * kJobsInts, "job table layout");
 
-__device__ void build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
+// Built by one warp (no block barrier): ranks of the (token, slot) pairs by
+// (expert, token), then the group starts by ballot.
+__device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
+  const int lane = threadIdx.x & 31;
   const int np = T * k;
-  const int tid = threadIdx.x;
-  if (tid < np) {
-    const int ei = idx_s[tid], ti = tid / k;
+  for (int i = lane; i < np; i += 32) {
+    const int ei = idx_s[i], ti = i / k;
     int rank = 0;
     for (int j = 0; j < np; ++j) {
       const int ej = idx_s[j], tj = j / k;
       rank += (ej < ei) || (ej == ei && tj < ti);
     }
-    J.pair[rank] = tid;
+    J.pair[rank] = i;
     J.rank_e[rank] = ei;
   }
-  __syncthreads();
-  if (tid == 0) {
-    int n = 0;
-    for (int r = 0; r < np; ++r) {
-      if (r == 0 || J.rank_e[r] != J.rank_e[r - 1]) {
-        J.e[n] = J.rank_e[r];
-        J.first[n] = r;
-        J.cnt[n] = 0;
-        ++n;
-      }
-      J.cnt[n - 1]++;
+  __syncwarp();
+  int ng = 0;
+  for (int base = 0; base < np; base += 32) {
+    const int rr = base + lane;
+    const bool first = rr < np && (rr == 0 || J.rank_e[rr] != J.rank_e[rr - 1]);
+    const unsigned m = __ballot_sync(0xffffffffu, first);
+    if (first) {
+      const int g = ng + __popc(m & ((1u << lane) - 1u));
+      J.e[g] = J.rank_e[rr];
+      J.first[g] = rr;
     }
-    J.n = n;
+    ng += __popc(m);
   }
-  __syncthreads();
+  __syncwarp();
+  for (int g = lane; g < ng; g += 32) J.cnt[g] = (g + 1 < ng ? J.first[g + 1] : np) - J.first[g];
+  if (lane == 0) J.n = ng;
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------ staging
@@ -481,16 +527,17 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
 }
 
 // Dynamic unit scheduling on the warp's two-stage ring.  A warp claims G
-// consecutive units at a time from `counter`; the claim is made when the
-// first chunk of a unit is staged, so its latency overlaps the compute of the
-// previous chunk, and the ring runs on across unit boundaries.
+// consecutive units at a time from `counter`; the ring runs on across unit
+// boundaries.
+//   valid(u)          -> false once u is past the last unit (may wait until
+//                        the unit count is known)
 //   unit_at(u)        -> UnitT with field nch (chunks of the unit)
 //   chunk_of(unit, c) -> Chunk c of the unit
 //   compute(unit, u, c, data, next_u): consume chunk c of unit u, staged at
 //                        `data`; next_u is the unit of the next chunk the warp
 //                        computes (-1 when none), for segment bookkeeping
-template <int G, bool AHEAD, typename UnitT, typename UnitAt, typename ChunkOf, typename Compute>
-__device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *counter, int n_units, UnitAt unit_at,
+template <int G, bool AHEAD, typename UnitT, typename Valid, typename UnitAt, typename ChunkOf, typename Compute>
+__device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *counter, Valid valid, UnitAt unit_at,
                                           ChunkOf chunk_of, Compute compute) {
   const int lane = threadIdx.x & 31;
   int s_u = 0, s_left = 0, s_c = 0;
@@ -506,7 +553,7 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *count
         ++s_u;
       }
       --s_left;
-      if (s_u >= n_units) {
+      if (!valid(s_u)) {
         s_left = 0;
         cp_async_commit();
         return false;
@@ -528,11 +575,9 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *count
     if (cA == 0) cu = unit_at(uA);
     int uB = 0, cB = 0, shB = 0;
     bool haveB = false;
-    // the next unit is claimed early only while the warp's last claim lies
-    // more than a grid's worth of warps before the end of the work (near the
-    // end an early claim would only lengthen the tail)
-    const bool defer =
-        s_c == 0 && s_left == 0 && (!AHEAD || s_u + (int)(gridDim.x * (blockDim.x >> 5)) * G >= n_units);
+    // with AHEAD the next unit is claimed while this chunk is computed,
+    // otherwise only after it
+    const bool defer = !AHEAD && s_c == 0 && s_left == 0;
     if (!defer) haveB = stage_next(nxt, uB, cB, shB);
     else cp_async_commit();
     cp_async_wait<1>();
@@ -890,6 +935,7 @@ struct K2Shared {
   int32_t idx[kDecodeMaxT * kMaxK];
   float w[kDecodeMaxT * kMaxK];
   Jobs J;
+  int jobs_ready;  // set once the routing warps have published idx, w and J
   float hsm[kWarps2][kDecodeMaxT][16];
 };
 
@@ -992,21 +1038,31 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   const int XS = d.H + 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  if (tid == 0) S.jobs_ready = 0;
   build_tables(a.wt.grid, gpm, selt, a.err);
   pdl_wait();  // k1's limbs and keys are visible from here on
   if (XSMEM) {
     const int n16 = d.H / 16;
     copy_rows16(xsm, XS, s.xq, d.H, T * 3, n16);
   }
-  for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
   __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int i = tid; i < T * d.k; i += blockDim.x) {
-      s.idx[i] = S.idx[i];
-      s.w[i] = S.w[i];
+  // Warps 0..T-1 route one token each and warp 0 builds the job table; the
+  // other warps start on the shared expert's gate/up units, which need no
+  // routing, and wait for the table only when they claim a routed unit.
+  if (warp < T) {
+    warp_route_token(a, warp, S.idx + warp * d.k, S.w + warp * d.k);
+    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * T) : "memory");
+    if (warp == 0) {
+      warp_build_jobs(S.idx, T, d.k, S.J);
+      if (blockIdx.x == 0)
+        for (int i = lane; i < T * d.k; i += 32) {
+          s.idx[i] = S.idx[i];
+          s.w[i] = S.w[i];
+        }
+      __threadfence_block();
+      if (lane == 0) *reinterpret_cast<volatile int *>(&S.jobs_ready) = 1;
     }
   }
-  build_jobs(S.idx, T, d.k, S.J);
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
   const uint8_t *sel_l = selt + (lane & 15) * 8;
@@ -1043,13 +1099,34 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   const int nqd = kps / 256;          // Q8_0 chunks of 8 blocks per shared down unit
   const size_t rbD = (size_t)(d.I / 256) * 84;
   const size_t rbQd = (size_t)(d.Is / 32) * 34;
-  const int nparts = S.J.n * PD + PS;  // parts of an output tile
   const int NS = s.NS;
-  // ---- unit ranges
+  // ---- unit ranges; the ones past the shared gate/up units depend on the
+  // number of jobs and are set once the job table is ready
   const int n_sh = tilesS * PH;
-  const int n2 = n_sh + S.J.n * tilesI * PH;
   const int n3s = PS * tilesH;
-  const int n_units = n2 + n3s + S.J.n * PD * tilesH;
+  int nparts = 0, n2 = 0, n_units = -1;  // parts of an output tile, unit ranges
+  auto valid = [&](int u) {
+    if (u < n_sh) return true;
+    if (n_units < 0) {
+      const long long t0 = clock64();
+      bool ok = true;
+      while (*reinterpret_cast<volatile int *>(&S.jobs_ready) == 0) {
+        if (clock64() - t0 > kSliceWaitCycles) {
+          set_error(a.err, kErrTimeout);
+          ok = false;
+          break;
+        }
+        __nanosleep(32);
+      }
+      __syncwarp();
+      __threadfence_block();
+      if (!ok) return false;
+      nparts = S.J.n * PD + PS;
+      n2 = n_sh + S.J.n * tilesI * PH;
+      n_units = n2 + n3s + S.J.n * PD * tilesH;
+    }
+    return u < n_units;
+  };
 
   struct Unit {
     int kind;  // 0 shared gate/up, 1 routed gate/up, 2 shared down, 3 routed down
@@ -1238,7 +1315,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   };
 
   run_units<kClaim, kAheadClaim, Unit>(
-      st0, st1, s.work + 0, n_units, unit_at, chunk_of,
+      st0, st1, s.work + 0, valid, unit_at, chunk_of,
       [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
         if (cu.kind <= 1) {
           // ------------------------------------------------ gate/up
@@ -1264,7 +1341,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
           if (cc == cu.nch - 1) {
             store_part(cu, 1);
             ++seg_parts;
-            if (next_u != u + 1 || u + 1 >= n2 || (u + 1) / PH != u / PH) end_gateup(cu);
+            if (next_u != u + 1 || (u + 1) / PH != u / PH) end_gateup(cu);
           }
           return;
         }
