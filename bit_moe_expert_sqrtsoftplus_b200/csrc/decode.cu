@@ -614,6 +614,9 @@ __device__ __forceinline__ uint2 ldb(const BColG &b, int kel) {
   if (b.ok) v = __ldcg(reinterpret_cast<const uint2 *>(b.p + kel));  // via L2: may be written by this kernel
   return v;
 }
+__device__ __forceinline__ uint32_t ldx(const BColS &b, int off) {
+  return b.ok ? *reinterpret_cast<const uint32_t *>(b.p + off) : 0u;
+}
 __device__ __forceinline__ uint32_t ldx(const BColG &b, int off) {
   return b.ok ? __ldcg(reinterpret_cast<const unsigned *>(b.p + off)) : 0u;
 }
@@ -705,6 +708,17 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol 
   const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
   const uint8_t *row0 = st + r * RS;
   const uint8_t *row1 = row0 + 8 * RS;
+  // one token pair: the B fragments of the whole chunk are loaded first (from
+  // global memory they are the long-latency loads of this loop); more pairs
+  // load them next to their MMAs (registers)
+  constexpr bool kPre = MAXP == 1;
+  uint2 B[kPre ? NB : 1][MAXP];
+  if (kPre) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) B[kPre ? b : 0][p] = p < npairs ? ldb(bcol[p], k0 + 32 * b) : make_uint2(0u, 0u);
+  }
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     const int o = 34 * b;
@@ -713,11 +727,10 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol 
     uint32_t A[4];
     q80_vals(row0, o, c, A[0], A[2]);
     q80_vals(row1, o, c, A[1], A[3]);
-    const int kel = k0 + 32 * b;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        const uint2 bb = ldb(bcol[p], kel);
+        const uint2 bb = kPre ? B[kPre ? b : 0][p] : ldb(bcol[p], k0 + 32 * b);
         const int zero[4] = {0, 0, 0, 0};
         int cg[4];
         mma_s8(cg, A, bb.x, bb.y, zero);
@@ -760,6 +773,24 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) Cm[p][0] = Cm[p][1] = Cm[p][2] = Cm[p][3] = 0;
     const int kb = (k0 >> 8) + b;  // global block index along K
+    // one token pair: the B fragments of the block's 8 MMAs and its min-term
+    // column are loaded first (from global memory they are the long-latency
+    // loads of this loop); more pairs load them next to their MMAs
+    constexpr bool kPre = MAXP == 1;
+    uint2 B[kPre ? 2 : 1][kPre ? 4 : 1][MAXP];
+    uint32_t BX[MAXP];
+    if (kPre) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int sh = 0; sh < 4; ++sh)
+#pragma unroll
+          for (int p = 0; p < MAXP; ++p)
+            B[kPre ? hf : 0][kPre ? sh : 0][p] =
+                p < npairs ? ldb(bcol[p], k0 + 256 * b + 128 * hf + 32 * sh) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p) BX[p] = p < npairs ? ldx(xcol[p], kb * 16) : 0u;  // base includes 4c
+    }
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       // a block at an odd position of the staged row starts 4 (not 8) bytes aligned
@@ -778,11 +809,10 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
         A[2] = ((q0.y >> (2 * sh)) & 0x03030303u) * sc0;
         A[1] = ((q1.x >> (2 * sh)) & 0x03030303u) * sc1;
         A[3] = ((q1.y >> (2 * sh)) & 0x03030303u) * sc1;
-        const int kel = k0 + 256 * b + 128 * hf + 32 * sh;  // the column base includes 8c
 #pragma unroll
         for (int p = 0; p < MAXP; ++p) {
           if (p < npairs) {
-            const uint2 bb = ldb(bcol[p], kel);
+            const uint2 bb = kPre ? B[kPre ? hf : 0][kPre ? sh : 0][p] : ldb(bcol[p], k0 + 256 * b + 128 * hf + 32 * sh);
             mma_s8(Cm[p], A, bb.x, bb.y, Cm[p]);
           }
         }
@@ -797,7 +827,7 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
       if (p < npairs) {
-        const uint32_t bx = ldx(xcol[p], kb * 16);  // base includes 4c
+        const uint32_t bx = kPre ? BX[p] : ldx(xcol[p], kb * 16);  // base includes 4c
         const int zero[4] = {0, 0, 0, 0};
         int cn[4];
         mma_s8(cn, Am, bx, 0u, zero);
@@ -931,6 +961,18 @@ __device__ __forceinline__ void copy_rows16(void *dst, size_t ss, const void *sr
 
 // ------------------------------------------------------------------ k2
 
+// Counter increment that publishes this warp's earlier writes (release) and,
+// for the warp that sees the final count, makes the other warps' writes
+// visible (acquire).  Call from one lane after __syncwarp().
+__device__ __forceinline__ int atomic_add_acq_rel(int *p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void store_release(int *p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+
 struct K2Shared {
   int32_t idx[kDecodeMaxT * kMaxK];
   float w[kDecodeMaxT * kMaxK];
@@ -969,16 +1011,15 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
       }
     }
   }
-  __threadfence();
   __syncwarp();
   for (int slot = 0; slot < ntok; ++slot) {
     const int v = vec[slot];
     const int vs = v * s.NSL + sl;
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.scount + vs, 1) == slice_len / 16 - 1;
+    if (lane == 0) last = atomic_add_acq_rel(s.scount + vs, 1) == slice_len / 16 - 1;
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
-      __threadfence();
+      __syncwarp();
       const float hm = __uint_as_float(__ldcg(s.hmax + vs));
       const float xm = __uint_as_float(__ldcg(s.Xmax + vs));
       const int k0 = sl * slice_len;
@@ -986,9 +1027,8 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
                       s.hsc + 4 * vs);
       quantise_vector(s.Xbuf + (size_t)v * Im16 + k0 / 16, slice_len / 16, xm,
                       s.Xq + (size_t)v * 3 * Im16 + k0 / 16, Im16, s.Xsc + 4 * vs);
-      __threadfence();
       __syncwarp();
-      if (lane == 0) atomicExch(s.ready + vs, 1);
+      if (lane == 0) store_release(s.ready + vs, 1);
     }
   }
 }
@@ -1007,11 +1047,10 @@ __device__ void wait_slice(const int *flag, int *err) {
         set_error(err, kErrTimeout);
         break;
       }
-      __nanosleep(64);
+      __nanosleep(256);
     }
   }
   __syncwarp();
-  __threadfence();
 }
 
 // The expert kernel: every unit of the layer's expert work, gate/up and
@@ -1116,7 +1155,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
           ok = false;
           break;
         }
-        __nanosleep(32);
+        __nanosleep(256);
       }
       __syncwarp();
       __threadfence_block();
@@ -1142,31 +1181,31 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
     x.ntok = T;
     if (u < n_sh) {
       x.kind = 0;
-      x.tile = u / PH;
-      x.part = u % PH;
+      x.tile = s.fPH.div(u);
+      x.part = u - x.tile * PH;
       x.per = nq8;
       x.nch = 2 * nq8;
     } else if (u < n2) {
       x.kind = 1;
       const int uu = u - n_sh;
-      x.j = uu / (tilesI * PH);
-      const int rem = uu % (tilesI * PH);
-      x.tile = rem / PH;
-      x.part = rem % PH;
+      x.j = s.fTIPH.div(uu);
+      const int rem = uu - x.j * tilesI * PH;
+      x.tile = s.fPH.div(rem);
+      x.part = rem - x.tile * PH;
       x.nch = 2;
     } else if (u < n2 + n3s) {
       x.kind = 2;
       const int w = u - n2;
-      x.kp = w / tilesH;
-      x.ot = w % tilesH;
+      x.kp = s.fTH.div(w);
+      x.ot = w - x.kp * tilesH;
       x.nch = nqd;
     } else {
       x.kind = 3;
       const int w = u - n2 - n3s;
-      const int jp = w / tilesH;
-      x.j = jp / PD;
-      x.kp = jp % PD;
-      x.ot = w % tilesH;
+      const int jp = s.fTH.div(w);
+      x.ot = w - jp * tilesH;
+      x.j = s.fPD.div(jp);
+      x.kp = jp - x.j * PD;
       x.nch = cbD / nbD;
     }
     if (x.kind & 1) {
@@ -1183,7 +1222,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
     Chunk ch;
     if (su.kind == 0) {
       const bool up = cs >= su.per;
-      const int ck = cs % su.per;
+      const int ck = up ? cs - su.per : cs;
       const size_t off = (size_t)(su.part * kpart / 32 + ck * 8) * 34;
       ch.g = (up ? a.wt.sh_up : a.wt.sh_gate) + (size_t)(su.tile * 16) * rbQ + off;
       ch.gstride = rbQ;
@@ -1245,15 +1284,14 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   // gate/up: count the segment's parts in; the warp that completes the tile
   // sums the parts in order, applies the SwiGLU and hands the tile on
   auto end_gateup = [&](const Unit &cu) {
-    __threadfence();
     __syncwarp();
     const int set = cu.kind == 0 ? 0 : 1 + cu.j;
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
+    if (lane == 0) last = atomic_add_acq_rel(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
     last = __shfl_sync(0xffffffffu, last, 0);
     seg_parts = 0;
     if (!last) return;
-    __threadfence();
+    __syncwarp();
     const int r0 = cu.tile * 16;
     for (int i = lane; i < 16 * cu.ntok; i += 32) {
       const int ts = i >> 4, row = i & 15;
@@ -1284,13 +1322,12 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   // down: the part is in its slot; the warp that completes the output tile
   // sums its slots in a fixed order into y
   auto end_down = [&](const Unit &cu) {
-    __threadfence();
     __syncwarp();
     int last = 0;
-    if (lane == 0) last = atomicAdd(s.ycount + cu.ot, 1) == nparts - 1;
+    if (lane == 0) last = atomic_add_acq_rel(s.ycount + cu.ot, 1) == nparts - 1;
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
-    __threadfence();
+    __syncwarp();
     const int r0 = cu.ot * 16;
     const float *ytile = s.ypart + (size_t)cu.ot * NS * 16;
     for (int i = lane; i < 16 * T; i += 32) {
@@ -1329,7 +1366,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
             }
           }
           if (cu.kind == 0) {
-            q80_chunk<8, MAXP>(st, cu.part * kpart + (cc % nq8) * 256, bcol, npairs, F);
+            q80_chunk<8, MAXP>(st, cu.part * kpart + (cc < nq8 ? cc : cc - nq8) * 256, bcol, npairs, F);
           } else if (cbI == 4) {
             iq2_chunk<4, MAXP>(st, cu.part * kpart, gpm_l, sel_l, bcol, npairs, F);
           } else if (cbI == 2) {
@@ -1341,7 +1378,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
           if (cc == cu.nch - 1) {
             store_part(cu, 1);
             ++seg_parts;
-            if (next_u != u + 1 || (u + 1) / PH != u / PH) end_gateup(cu);
+            if (next_u != u + 1 || s.fPH.div(u + 1) != s.fPH.div(u)) end_gateup(cu);
           }
           return;
         }
@@ -1511,6 +1548,10 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.TM = Imax / 16;
   s.NS = T * d.k * s.PD + T * s.PS;
   s.NSL = s.PD > s.PS ? s.PD : s.PS;
+  s.fPH.init(s.PH);
+  s.fTIPH.init((d.I / 16) * s.PH);
+  s.fTH.init(d.H / 16);
+  s.fPD.init(s.PD);
   s.z = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.sc = reinterpret_cast<double *>(take(sizeof(double) * T * d.E));
   s.idx = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * T * d.k));

@@ -37,6 +37,22 @@ __host__ __device__ inline int decode_kparts(int K) { return (K % kDecodeKPart =
 // (token, slot) pairs) as ints: n, then e, first, cnt, pair, rank_e.
 constexpr int kJobsInts = 1 + 5 * kDecodeMaxT * kMaxK;
 
+// Division by a constant d >= 1 as a multiply-high and a shift (round-up
+// method): l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1; for
+// 0 <= n < 2^31, n / d = (umulhi(n, m) + n) >> l.
+struct FastDiv {
+  uint32_t d, m, l;
+  void init(uint32_t div) {
+    d = div;
+    l = 0;
+    while ((1ull << l) < div) ++l;
+    m = (uint32_t)(((1ull << 32) * ((1ull << l) - div)) / div + 1);
+  }
+#ifdef __CUDACC__
+  __device__ __forceinline__ int div(int n) const { return (int)((__umulhi((uint32_t)n, m) + (uint32_t)n) >> l); }
+#endif
+};
+
 // Scratch of the decode (GEMV) path.  V = T*k + T vectors: routed vector
 // t*k + slot, shared vector T*k + t.  The SwiGLU output h of a vector is
 // quantised slice by slice: a slice is the K range of one down-projection
@@ -71,6 +87,7 @@ struct DecodeScratch {
   int Jmax;         // max routed vector sets = min(T*k, E)
   int TM;           // max(I, Is) / 16
   int NS;           // output slots per 16-row tile of y
+  FastDiv fPH, fTIPH, fTH, fPD;  // divisors PH, (I/16)*PH, H/16, PD of the unit numbering
 };
 
 struct DecodeArgs {
