@@ -1,16 +1,18 @@
 // gemm.cu -- persistent, warp-specialised grouped GEMM on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory).
 //
-// One CTA per SM, 21 warps:
-//   warps 0-3   epilogue: tcgen05.ld of the 128-lane accumulator, SwiGLU /
+// One CTA per SM, 25 warps:
+//   warps 0-7   epilogue: tcgen05.ld of the 128-lane accumulator, SwiGLU /
 //               scatter-add / store
-//   warps 4-19  producers: dequantise the 128 x 64 weight tile(s) of a K step
+//   warps 8-23  producers: dequantise the 128 x 64 weight tile(s) of a K step
 //               into 16-bit values written straight into the 128-byte-swizzled
 //               K-major operand layout, and gather the N x 64 activation tile
 //               with cp.async
-//   warp 20     allocates tensor memory and issues tcgen05.mma (one thread)
-// Shared memory holds a ring of stages (A tile(s) + B tile); mbarriers carry
-// full/empty hand-offs between producers and the MMA thread and
+//   warp 24     allocates tensor memory and issues tcgen05.mma (one thread)
+// Shared memory holds a ring of A stages (dequantised weight tiles, written
+// in the step that hands them over) and a ring of B stages (token rows,
+// loaded two K steps ahead); mbarriers carry full/empty hand-offs between
+// producers and the MMA thread and
 // full/empty hand-offs of the accumulator between the MMA thread and the
 // epilogue.  Every wait is bounded: on expiry the CTA records
 // MOE_ERR_TIMEOUT in the device error word, every role leaves its loop, the
@@ -30,10 +32,10 @@ namespace moe {
 
 namespace {
 
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the column groups
 constexpr int kProdWarps = 16;
-constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 20
-constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 672
+constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 24
+constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 800
 constexpr int kProd = kProdWarps * 32;             // 512 producer threads
 constexpr int kGridRep = 4;                        // replicas of the f16 codebook table
 constexpr int kSignRep = 4;                        // replicas of the sign-mask table
@@ -43,8 +45,11 @@ constexpr int kATile = BM * BK * 2;  // 16 KB
 constexpr int kBTile = BN * BK * 2;  // 32 KB
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 
+constexpr int kSB = 4;       // stages of the B (token rows) ring
+constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
+
 struct alignas(8) GemmCtl {
-  uint64_t full[4], empty[4], acc_full, acc_empty, drain;
+  uint64_t full[kSB], emptyA[4], emptyB[kSB], acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort;
   int n_groups;
@@ -331,13 +336,18 @@ __device__ __forceinline__ void decode(const Raw<kFmtQ80> &r, uint8_t *tile, int
 
 template <int FMT, bool PAIRED>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
+  // A (dequantised weights) and B (gathered token rows) have rings of their
+  // own: a B tile is loaded kBAhead steps before its use, an A tile is
+  // written in the step that hands it to the MMA; step `it` uses A stage
+  // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
-  constexpr int S = PAIRED ? 3 : 4;
-  constexpr int STAGE = NA * kATile + kBTile;
+  constexpr int SA = PAIRED ? 2 : 4;
+  constexpr int ASTAGE = NA * kATile;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *stages = smem;
-  uint8_t *gridh = stages + S * STAGE;          // 256 x kGridRep x 16 B: codebook as f16
+  uint8_t *stagesA = smem;
+  uint8_t *stagesB = stagesA + SA * ASTAGE;
+  uint8_t *gridh = stagesB + kSB * kBTile;      // 256 x kGridRep x 16 B: codebook as f16
   uint8_t *signm = gridh + 4096 * kGridRep;     // 128 x kSignRep x 16 B: f16 sign masks
   GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + 2048 * kSignRep);
 
@@ -347,10 +357,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 
   // ---- set-up
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < kSB; ++s) {
       mbar_init(&ctl.full[s], kProd);
-      mbar_init(&ctl.empty[s], 1);
+      mbar_init(&ctl.emptyB[s], 1);
     }
+    for (int s = 0; s < SA; ++s) mbar_init(&ctl.emptyA[s], 1);
     mbar_init(&ctl.acc_full, 1);
     mbar_init(&ctl.acc_empty, kEpiWarps * 32);
     mbar_init(&ctl.drain, 1);
@@ -435,37 +446,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
         for (int j = 0; j < kAhead; ++j)
           if (j < ksteps) fetch(R[j], arow, j, item);
       }
-      auto issue_b = [&](int ks, int st) {
-        uint8_t *Bs = stages + st * STAGE + NA * kATile;
+      // B tile of tile-local step ks into B stage `sb` (one cp.async group)
+      auto issue_b = [&](int ks, int sb) {
+        uint8_t *Bs = stagesB + sb * kBTile;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 64 * i, ch), brow[i] + ks * BK);
         }
         cp_async_commit();
       };
-      bool ok = mbar_wait(&ctl.empty[it % S], ((it / S) & 1u) ^ 1u, ctl, a.err);
-      if (ok) issue_b(0, it % S);
+      // waits until the B stage of global step g is free, then loads it (or
+      // commits an empty group past the tile's last step)
+      auto load_b = [&](int ks, uint32_t g) -> bool {
+        if (ks >= ksteps) {
+          cp_async_commit();
+          return true;
+        }
+        if (!mbar_wait(&ctl.emptyB[g % kSB], ((g / kSB) & 1u) ^ 1u, ctl, a.err)) return false;
+        issue_b(ks, g % kSB);
+        return true;
+      };
+      bool ok = true;
+#pragma unroll
+      for (int q = 0; q < kBAhead; ++q)
+        if (ok) ok = load_b(q, it + q);
       for (int ks0 = 0; ok && ks0 < ksteps; ks0 += kAhead + 1) {
 #pragma unroll
         for (int j = 0; j <= kAhead; ++j) {
           const int ks = ks0 + j;
           if (!ok || ks >= ksteps) break;
-          const int st = it % S;
-          if (ks + 1 < ksteps) {
-            const uint32_t nt = it + 1;
-            if (!mbar_wait(&ctl.empty[nt % S], ((nt / S) & 1u) ^ 1u, ctl, a.err)) {
-              ok = false;
-              break;
-            }
-            issue_b(ks + 1, nt % S);
-          } else {
-            cp_async_commit();
+          if (!load_b(ks + kBAhead, it + kBAhead) ||
+              !mbar_wait(&ctl.emptyA[it % SA], ((it / SA) & 1u) ^ 1u, ctl, a.err)) {
+            ok = false;
+            break;
           }
-          uint8_t *A0s = stages + st * STAGE;
+          uint8_t *A0s = stagesA + (it % SA) * ASTAGE;
           if (has_a) decode(R[j], A0s + mat * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh_l, signm_l);
-          cp_async_wait<1>();  // this step's B tile has landed
+          cp_async_wait<kBAhead>();  // this step's B tile has landed
           fence_proxy_async();
-          mbar_arrive(&ctl.full[st]);
+          mbar_arrive(&ctl.full[it % kSB]);
           // the next look-ahead fetch goes out after this step is handed over
           if (has_a && ks + kAhead < ksteps) fetch(R[(j + kAhead) % (kAhead + 1)], arow, ks + kAhead, item);
           ++it;
@@ -488,23 +507,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       }
       tc_fence_after();
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1u;
-        if (!mbar_wait(&ctl.full[st], ph, ctl, a.err)) {
+        const uint32_t ph = (it / kSB) & 1u;
+        if (!mbar_wait(&ctl.full[it % kSB], ph, ctl, a.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a0 = smem_u32(stages + st * STAGE);
-          const uint32_t b0 = a0 + NA * kATile;
+          const uint32_t a0 = smem_u32(stagesA + (it % SA) * ASTAGE);
+          const uint32_t b0 = smem_u32(stagesB + (it % kSB) * kBTile);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             mma_f16(tmem, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
             if (PAIRED) mma_f16(tmem + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
           }
-          mma_commit(&ctl.empty[st]);
+          mma_commit(&ctl.emptyA[it % SA]);
+          mma_commit(&ctl.emptyB[it % kSB]);
         }
         __syncwarp();
       }
@@ -525,15 +544,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     __syncwarp();
   } else {
     // =================================================== epilogue
-    const int row = tid;  // TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // warp w reads TMEM lanes 32 (w % 4) .. + 31 (the quadrant it may access)
+    // and the 16-column groups g with g % 2 == w / 4
+    const int row = (warp & 3) * 32 + lane;  // TMEM lane = weight row in the tile
+    const int half = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const Tile tl = tile_at(ctl, t, m_tiles);
       if (!mbar_wait(&ctl.acc_full, tc & 1u, ctl, a.err)) break;
       tc_fence_after();
       const int m = tl.m0 + row;
-      for (int c0 = 0; c0 < tl.nt; c0 += 16) {
+      for (int c0 = 16 * half; c0 < tl.nt; c0 += 32) {
         uint32_t r0[16], r1[16];
         tmem_ld16(lane_base + c0, r0);
         if (PAIRED) tmem_ld16(lane_base + BN + c0, r1);
@@ -546,7 +568,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
           const float dv = __uint_as_float(r0[j]);
           if (a.epi == kEpiSwiGLU) {
             const float u = __uint_as_float(PAIRED ? r1[j] : 0u);
-            const float h = silu(dv) * u;
+            // SiLU with the fast exponential and reciprocal (rcp(inf) = 0 for large -dv)
+            const float h = dv * __frcp_rn(1.f + __expf(-dv)) * u;
             uint16_t hb;
             if (a.h_bf16) {
               __nv_bfloat16 v = __float2bfloat16_rn(h);
@@ -583,8 +606,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 
 size_t grouped_gemm_smem(int paired) {
   const int na = paired ? 2 : 1;
-  const int s = paired ? 3 : 4;
-  return 1024 + (size_t)s * (na * kATile + kBTile) + 4096 * kGridRep + 2048 * kSignRep + sizeof(GemmCtl);
+  const int sa = paired ? 2 : 4;
+  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * kBTile + 4096 * kGridRep + 2048 * kSignRep + sizeof(GemmCtl);
 }
 
 template <int FMT, bool PAIRED>
