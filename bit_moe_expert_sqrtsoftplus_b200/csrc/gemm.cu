@@ -49,7 +49,7 @@ constexpr int kSB = 4;       // stages of the B (token rows) ring
 constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
 
 struct alignas(8) GemmCtl {
-  uint64_t full[kSB], emptyA[4], emptyB[kSB], acc_full, acc_empty, drain;
+  uint64_t full[kSB], emptyA[4], emptyB[kSB], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
   int n_groups;
@@ -342,6 +342,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
   constexpr int SA = PAIRED ? 2 : 4;
+  // accumulator buffers in tensor memory: a gate/up pair fills all 512
+  // columns; a single matrix uses 256, so two tiles alternate and the
+  // epilogue of one overlaps the main loop of the next
+  constexpr int NACC = PAIRED ? 1 : 2;
   constexpr int ASTAGE = NA * kATile;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -362,8 +366,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       mbar_init(&ctl.emptyB[s], 1);
     }
     for (int s = 0; s < SA; ++s) mbar_init(&ctl.emptyA[s], 1);
-    mbar_init(&ctl.acc_full, 1);
-    mbar_init(&ctl.acc_empty, kEpiWarps * 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl.acc_full[b], 1);
+      mbar_init(&ctl.acc_empty[b], kEpiWarps * 32);
+    }
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -501,7 +507,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       const Tile tl = tile_at(ctl, t, m_tiles);
       const int nmma = (tl.nt + 15) & ~15;
       const uint32_t idesc = instr_desc(nmma, a.bf16);
-      if (!mbar_wait(&ctl.acc_empty, (tc & 1u) ^ 1u, ctl, a.err)) {
+      const uint32_t buf = tc % NACC;
+      const uint32_t dacc = tmem + buf * BN;  // accumulator columns of this tile
+      if (!mbar_wait(&ctl.acc_empty[buf], ((tc / NACC) & 1u) ^ 1u, ctl, a.err)) {
         ok = false;
         break;
       }
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            mma_f16(tmem, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+            mma_f16(dacc, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
             if (PAIRED) mma_f16(tmem + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
           }
           mma_commit(&ctl.emptyA[it % SA]);
@@ -527,7 +535,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
         }
         __syncwarp();
       }
-      if (ok && lane == 0) mma_commit(&ctl.acc_full);
+      if (ok && lane == 0) mma_commit(&ctl.acc_full[buf]);
       __syncwarp();
     }
     // drain: every MMA this thread issued has finished before tensor memory is freed
@@ -552,12 +560,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const Tile tl = tile_at(ctl, t, m_tiles);
-      if (!mbar_wait(&ctl.acc_full, tc & 1u, ctl, a.err)) break;
+      const uint32_t buf = tc % NACC;
+      if (!mbar_wait(&ctl.acc_full[buf], (tc / NACC) & 1u, ctl, a.err)) break;
       tc_fence_after();
       const int m = tl.m0 + row;
       for (int c0 = 16 * half; c0 < tl.nt; c0 += 32) {
         uint32_t r0[16], r1[16];
-        tmem_ld16(lane_base + c0, r0);
+        tmem_ld16(lane_base + buf * BN + c0, r0);
         if (PAIRED) tmem_ld16(lane_base + BN + c0, r1);
         tmem_wait_ld();
 #pragma unroll
@@ -590,7 +599,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctl.acc_empty);
+      mbar_arrive(&ctl.acc_empty[buf]);
     }
   }
 
