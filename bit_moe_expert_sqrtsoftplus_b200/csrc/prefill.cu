@@ -217,6 +217,7 @@ __global__ void k_topk_cert(const double *z, const float *bias, const float *wn,
   if (!certified) {
     const int slot = atomicAdd(fix, 1);
     fix[1 + slot] = t;
+    fix[1 + T + slot] = 0;  // arrivals of the fix-up blocks of this slot
     return;
   }
   // ascending ids
@@ -237,31 +238,59 @@ __global__ void k_topk_cert(const double *z, const float *bias, const float *wn,
   }
 }
 
-// fp64 router for the queued tokens: one block (8 warps) per token.
+// fp64 router for the queued tokens.  A work item is (queued token, group of
+// kFixGroup experts); blocks stride over the items.  The token's x * inv is
+// staged in shared memory as fp64; each warp takes experts of the group with
+// 8 consecutive weights per 16-byte load per lane and four independent partial
+// sums, and the logits go to z.  The block that completes a token's last group
+// (an acquire/release count per queued token) selects its experts and weights.
+constexpr int kFixGroup = 16;
+
 __global__ void __launch_bounds__(256) k_router_fix(const float *x, const double *inv, const uint16_t *Wr,
                                                     const float *bias, int T, int E, int H, int k, float scaling,
-                                                    const int32_t *fix, double *z, int32_t *idx, float *w) {
+                                                    int32_t *fix, double *z, int32_t *idx, float *w) {
   const int nfix = fix[0];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ double zs[kMaxE];
-  for (int f = blockIdx.x; f < nfix; f += gridDim.x) {
+  const int ngroups = (E + kFixGroup - 1) / kFixGroup;
+  extern __shared__ double xsd[];  // [H]
+  __shared__ int last_s;
+  for (int item = blockIdx.x; item < nfix * ngroups; item += gridDim.x) {
+    const int f = item / ngroups, grp = item % ngroups;
     const int t = fix[1 + f];
     const float *xt = x + (size_t)t * H;
     const double iv = inv[t];
-    for (int e = warp; e < E; e += 8) {
-      double acc = 0.0;
-      for (int j = lane; j < H; j += 32)
-        acc = fma((double)half_bits_to_float(Wr[(size_t)e * H + j]), (double)xt[j] * iv, acc);
-      acc = warp_sum_d(acc);
-      if (lane == 0) zs[e] = acc;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) xsd[j] = (double)xt[j] * iv;
+    __syncthreads();
+    const int e1 = min(E, (grp + 1) * kFixGroup);
+    for (int e = grp * kFixGroup + warp; e < e1; e += 8) {
+      const uint16_t *we = Wr + (size_t)e * H;
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int j0 = 8 * lane; j0 < H; j0 += 256) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(we + j0));
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[q] = fma((double)half_bits_to_float((uint16_t)(ww[q] & 0xFFFFu)), xsd[j0 + 2 * q], acc[q]);
+          acc[q] = fma((double)half_bits_to_float((uint16_t)(ww[q] >> 16)), xsd[j0 + 2 * q + 1], acc[q]);
+        }
+      }
+      const double sum = warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3]));
+      if (lane == 0) z[(size_t)t * E + e] = sum;
     }
     __syncthreads();
-    if (warp == 0) {
+    if (threadIdx.x == 0) {
+      int old;
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;\n" : "=r"(old) : "l"(fix + 1 + T + f) : "memory");
+      last_s = old == ngroups - 1;
+    }
+    __syncthreads();
+    if (last_s && warp == 0) {
+      const double *zt = z + (size_t)t * E;
       double key[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        key[i] = e < E ? sqrtsoftplus(zs[e]) + (double)bias[e] : -DBL_MAX;
+        key[i] = e < E ? sqrtsoftplus(__ldcg(zt + e)) + (double)bias[e] : -DBL_MAX;
       }
       unsigned taken = 0;
       int sel[kMaxK];
@@ -301,14 +330,13 @@ __global__ void __launch_bounds__(256) k_router_fix(const float *x, const double
           }
         double sv[kMaxK], tot = 0.0;
         for (int i = 0; i < k; ++i) {
-          sv[i] = sqrtsoftplus(zs[sel[i]]);
+          sv[i] = sqrtsoftplus(__ldcg(zt + sel[i]));
           tot += sv[i];
         }
         for (int i = 0; i < k; ++i) {
           idx[(size_t)t * k + i] = sel[i];
           w[(size_t)t * k + i] = (float)((double)scaling * sv[i] / tot);
         }
-        for (int e = 0; e < E; ++e) z[(size_t)t * E + e] = zs[e];
       }
     }
     __syncthreads();
@@ -427,7 +455,7 @@ PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, cons
   p.s.counts = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * d.E));
   p.s.offsets = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (d.E + 1)));
   p.s.perm = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)T * d.k));
-  p.s.fix = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)(T + 1)));
+  p.s.fix = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)(2 * T + 1)));
   // token norms (2 x fp64 per token)
   take(2 * sizeof(double) * (size_t)T);
   p.s.big = static_cast<uint8_t *>(scratch) + align_up(off, 256);
@@ -444,7 +472,7 @@ cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_
 
 static double *token_norm_ptr(const PrefillArgs &p) {
   uint8_t *fixp = reinterpret_cast<uint8_t *>(p.s.fix);
-  return reinterpret_cast<double *>(fixp + align_up(sizeof(int32_t) * (size_t)(p.T + 1), 256));
+  return reinterpret_cast<double *>(fixp + align_up(sizeof(int32_t) * (size_t)(2 * p.T + 1), 256));
 }
 
 cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStream_t s) {
@@ -464,9 +492,18 @@ cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStre
   dim3 g((T + RT - 1) / RT, (d.E + RE - 1) / RE);
   k_router_f32<<<g, 256, 0, s>>>(p.x, inv, p.wt.Wr, T, d.E, d.H, z);
   k_topk_cert<<<(T + 7) / 8, 256, 0, s>>>(z, p.wt.bias, p.row_norms, xn, T, d.E, d.k, d.scaling, idx, w, p.s.fix);
-  int nfix_blocks = T < 148 ? T : 148;
-  k_router_fix<<<nfix_blocks, 256, 0, s>>>(p.x, inv, p.wt.Wr, p.wt.bias, T, d.E, d.H, d.k, d.scaling, p.s.fix, z,
-                                          idx, w);
+  // enough blocks for the usual handful of queued tokens; more stride
+  const int nfix_items = T * ((d.E + kFixGroup - 1) / kFixGroup);
+  const int nfix_blocks = nfix_items < 296 ? nfix_items : 296;
+  const size_t fix_smem = sizeof(double) * (size_t)d.H;
+  static bool fix_configured = false;
+  if (!fix_configured && fix_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(k_router_fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fix_smem);
+    if (e != cudaSuccess) return e;
+    fix_configured = true;
+  }
+  k_router_fix<<<nfix_blocks, 256, fix_smem, s>>>(p.x, inv, p.wt.Wr, p.wt.bias, T, d.E, d.H, d.k, d.scaling,
+                                                  p.s.fix, z, idx, w);
   return cudaGetLastError();
 }
 

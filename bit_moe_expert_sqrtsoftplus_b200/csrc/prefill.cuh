@@ -17,7 +17,7 @@ struct PrefillScratch {
   int32_t *counts;   // [E]
   int32_t *offsets;  // [E+1]
   int32_t *perm;     // [T*k]
-  int32_t *fix;      // [1 + T] tokens that need the fp64 router
+  int32_t *fix;      // [1 + 2T] count, tokens that need the fp64 router, per-token block arrivals
   void *big;         // remaining scratch for the expert GEMMs
   size_t big_bytes;
 };
