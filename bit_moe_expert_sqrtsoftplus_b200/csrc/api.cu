@@ -179,6 +179,7 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   h->wt.sh_up = static_cast<const uint8_t *>(w->sh_up_q80);
   h->wt.sh_down = static_cast<const uint8_t *>(w->sh_down_q80);
   h->wt.grid = w->iq2_grid;
+  moe::build_chunk_tensor_maps(h->wt, h->d);
   h->err = static_cast<int *>(persist);
   h->row_norms = reinterpret_cast<float *>(static_cast<uint8_t *>(persist) + kPersistHeader);
   h->num_sms = sms;

@@ -26,6 +26,8 @@
 // s3 = s2/254, which keeps x to 6e-8 of max|x|; the weight side is exact in
 // int8 (IQ2_XXS grid values with signs, Q2_K code*scale <= 45, Q8_0 values),
 // so the products are exact integers and only the fp32 block scaling rounds.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <float.h>
 #include <math.h>
 
@@ -422,6 +424,8 @@ __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+__device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
+
 struct Chunk {
   const uint8_t *g;  // row 0 of the tile at the chunk's first block
   size_t gstride;    // global row stride (bytes)
@@ -430,14 +434,53 @@ struct Chunk {
   int k0;            // first element (K index) of the chunk
   int piece;         // copy granularity: 16, 8, 4 (cp.async) or 2 (plain loads)
   int align;         // alignment the decoder needs at the start of a staged row (4 or 8)
+  int tm;            // TMA: tensor map index
+  int tx, ty;        // TMA: box origin (16-bit elements along the row, first row)
+  int tshift;        // TMA: bytes from the box origin to the chunk's first byte
 };
+
+// TMA chunk load: one lane arms the stage's mbarrier with the box bytes and
+// issues one 2-D tensor copy of 16 rows x the staged row width; returns where
+// the chunk's data starts in each staged row.
+__device__ __forceinline__ int stage_chunk_tma(uint8_t *st, uint64_t *mbar, const TensorMap *tm, const Chunk &c) {
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t bytes = 16u * (uint32_t)stage_rs(c.bpr);
+    const uint32_t mb = smem_u32(mbar);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(mb), "r"(bytes) : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+            "r"(smem_u32(st)),
+        "l"(reinterpret_cast<uint64_t>(tm + c.tm)), "r"(c.tx), "r"(c.ty), "r"(mb)
+        : "memory");
+  }
+  return c.tshift;
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false (and the timeout
+// error recorded) if it does not complete.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parity, int *err) {
+  const uint32_t mb = smem_u32(mbar);
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mb), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > 4000000000ll) {
+      set_error(err, kErrTimeout);
+      return false;
+    }
+  }
+}
 
 __host__ __device__ __forceinline__ int piece_for(size_t gstride, size_t off, int bpr) {
   const size_t m = gstride | off | (size_t)bpr;
   return (m & 15) == 0 ? 16 : (m & 7) == 0 ? 8 : (m & 3) == 0 ? 4 : 2;
 }
 
-__device__ __forceinline__ int stage_rs(int bpr) { return (int)align_up((size_t)bpr, 16); }
 
 // Copies one chunk (16 rows x bpr bytes) into the stage (row stride RS) and
 // returns where the chunk's data starts in each staged row.
@@ -536,13 +579,16 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
 //   compute(unit, u, c, data, next_u): consume chunk c of unit u, staged at
 //                        `data`; next_u is the unit of the next chunk the warp
 //                        computes (-1 when none), for segment bookkeeping
-template <int G, bool AHEAD, typename UnitT, typename Valid, typename UnitAt, typename ChunkOf, typename Compute>
-__device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *counter, Valid valid, UnitAt unit_at,
-                                          ChunkOf chunk_of, Compute compute) {
+template <int G, bool AHEAD, bool TMA, typename UnitT, typename Valid, typename UnitAt, typename ChunkOf,
+          typename Compute>
+__device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, uint64_t *mbar, const TensorMap *tm,
+                                          int *err, int *counter, Valid valid, UnitAt unit_at, ChunkOf chunk_of,
+                                          Compute compute) {
   const int lane = threadIdx.x & 31;
   int s_u = 0, s_left = 0, s_c = 0;
   UnitT su;
-  auto stage_next = [&](uint8_t *dst, int &uid, int &cidx, int &shift) -> bool {
+  // stages the next chunk into slot `slot` (TMA) or commits its cp.async group
+  auto stage_next = [&](uint8_t *dst, int slot, int &uid, int &cidx, int &shift) -> bool {
     if (s_c == 0) {
       if (s_left == 0) {
         int u = 0;
@@ -555,19 +601,19 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *count
       --s_left;
       if (!valid(s_u)) {
         s_left = 0;
-        cp_async_commit();
+        if (!TMA) cp_async_commit();
         return false;
       }
       su = unit_at(s_u);
     }
     uid = s_u;
     cidx = s_c;
-    shift = stage_chunk(dst, chunk_of(su, s_c));
+    shift = TMA ? stage_chunk_tma(dst, mbar + slot, tm, chunk_of(su, s_c)) : stage_chunk(dst, chunk_of(su, s_c));
     if (++s_c == su.nch) s_c = 0;
     return true;
   };
   int uA = 0, cA = 0, shA = 0;
-  bool haveA = stage_next(st0, uA, cA, shA);
+  bool haveA = stage_next(st0, 0, uA, cA, shA);
   UnitT cu;
   for (int i = 0; haveA; ++i) {
     uint8_t *cur = (i & 1) ? st1 : st0;
@@ -578,13 +624,23 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, int *count
     // with AHEAD the next unit is claimed while this chunk is computed,
     // otherwise only after it
     const bool defer = !AHEAD && s_c == 0 && s_left == 0;
-    if (!defer) haveB = stage_next(nxt, uB, cB, shB);
-    else cp_async_commit();
-    cp_async_wait<1>();
+    if (!defer) haveB = stage_next(nxt, (i + 1) & 1, uB, cB, shB);
+    else if (!TMA) cp_async_commit();
+    if (TMA) {
+      // chunk i is the (i / 2)-th use of its slot
+      if (!mbar_wait_bounded(mbar + (i & 1), (uint32_t)(i >> 1) & 1u, err)) {
+        // leave after the other slot's copy (if any) has landed
+        if (haveB) mbar_wait_bounded(mbar + ((i + 1) & 1), (uint32_t)((i + 1) >> 1) & 1u, err);
+        __syncwarp();
+        return;
+      }
+    } else {
+      cp_async_wait<1>();
+    }
     __syncwarp();
     compute(cu, uA, cA, cur + shA, defer ? -1 : (haveB ? uB : -1));
     __syncwarp();
-    if (defer) haveB = stage_next(nxt, uB, cB, shB);
+    if (defer) haveB = stage_next(nxt, (i + 1) & 1, uB, cB, shB);
     uA = uB;
     cA = cB;
     shA = shB;
@@ -979,6 +1035,7 @@ struct K2Shared {
   Jobs J;
   int jobs_ready;  // set once the routing warps have published idx, w and J
   float hsm[kWarps2][kDecodeMaxT][16];
+  uint64_t mbar[kWarps2][2];  // TMA completion of each warp's two stages
 };
 
 // Writes the 16 x ntok SwiGLU outputs held in hs (token slot, row) for the
@@ -1063,8 +1120,8 @@ __device__ void wait_slice(const int *flag, int *err) {
 // claimed by a running warp before the first down unit is claimed, so the
 // waits end.  XSMEM: the x limbs of all tokens are staged in shared memory
 // (rows of H + 32 bytes, which spreads the B-fragment loads over all banks).
-template <int MAXP, bool XSMEM>
-__global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) {
+template <int MAXP, bool XSMEM, bool TMA>
+__global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const LayerDims &d = a.d;
   const DecodeScratch &s = a.s;
@@ -1078,6 +1135,11 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) S.jobs_ready = 0;
+  if (TMA && lane == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&S.mbar[warp][0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&S.mbar[warp][1])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
   build_tables(a.wt.grid, gpm, selt, a.err);
   pdl_wait();  // k1's limbs and keys are visible from here on
   if (XSMEM) {
@@ -1220,42 +1282,55 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
   auto hvec = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] : T * d.k + ts; };
   auto chunk_of = [&](const Unit &su, int cs) {
     Chunk ch;
+    size_t off;  // byte offset of the chunk within its row
+    int row;     // first row of the chunk in its tensor
     if (su.kind == 0) {
       const bool up = cs >= su.per;
       const int ck = up ? cs - su.per : cs;
-      const size_t off = (size_t)(su.part * kpart / 32 + ck * 8) * 34;
-      ch.g = (up ? a.wt.sh_up : a.wt.sh_gate) + (size_t)(su.tile * 16) * rbQ + off;
+      off = (size_t)(su.part * kpart / 32 + ck * 8) * 34;
+      row = su.tile * 16;
+      ch.g = (up ? a.wt.sh_up : a.wt.sh_gate) + (size_t)row * rbQ + off;
       ch.gstride = rbQ;
       ch.bpr = 8 * 34;
       ch.nb = 8;
       ch.k0 = su.part * kpart + ck * 256;
       ch.align = 4;
+      ch.tm = up ? kTmShUp : kTmShGate;
     } else if (su.kind == 1) {
-      const size_t off = (size_t)su.part * cbI * 66;
-      ch.g = (cs ? a.wt.up : a.wt.gate) + ((size_t)su.e * d.I + su.tile * 16) * rbI + off;
+      off = (size_t)su.part * cbI * 66;
+      row = su.e * d.I + su.tile * 16;
+      ch.g = (cs ? a.wt.up : a.wt.gate) + (size_t)row * rbI + off;
       ch.gstride = rbI;
       ch.bpr = cbI * 66;
       ch.nb = cbI;
       ch.k0 = su.part * kpart;
       ch.align = 4;
+      ch.tm = cs ? kTmUp : kTmGate;
     } else if (su.kind == 2) {
-      const size_t off = (size_t)(su.kp * kps / 32 + cs * 8) * 34;
-      ch.g = a.wt.sh_down + (size_t)(su.ot * 16) * rbQd + off;
+      off = (size_t)(su.kp * kps / 32 + cs * 8) * 34;
+      row = su.ot * 16;
+      ch.g = a.wt.sh_down + (size_t)row * rbQd + off;
       ch.gstride = rbQd;
       ch.bpr = 8 * 34;
       ch.nb = 8;
       ch.k0 = su.kp * kps + cs * 256;
       ch.align = 4;
+      ch.tm = kTmShDown;
     } else {
-      const size_t off = (size_t)(su.kp * cbD + cs * nbD) * 84;
-      ch.g = a.wt.down + ((size_t)su.e * d.H + su.ot * 16) * rbD + off;
+      off = (size_t)(su.kp * cbD + cs * nbD) * 84;
+      row = su.e * d.H + su.ot * 16;
+      ch.g = a.wt.down + (size_t)row * rbD + off;
       ch.gstride = rbD;
       ch.bpr = nbD * 84;
       ch.nb = nbD;
       ch.k0 = su.kp * kpd + cs * nbD * 256;
       ch.align = 8;
+      ch.tm = kTmDown;
     }
     ch.piece = piece_for(ch.gstride, reinterpret_cast<uintptr_t>(ch.g) & 15, ch.bpr);
+    ch.tx = (int)((off & ~(size_t)15) / 2);
+    ch.ty = row;
+    ch.tshift = (int)(off & 15);
     return ch;
   };
 
@@ -1351,8 +1426,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(DecodeArgs a) 
     }
   };
 
-  run_units<kClaim, kAheadClaim, Unit>(
-      st0, st1, s.work + 0, valid, unit_at, chunk_of,
+  run_units<kClaim, kAheadClaim, TMA, Unit>(
+      st0, st1, &S.mbar[warp][0], a.wt.tm, a.err, s.work + 0, valid, unit_at, chunk_of,
       [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
         if (cu.kind <= 1) {
           // ------------------------------------------------ gate/up
@@ -1491,21 +1566,26 @@ cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int MAXP, bool XSMEM>
+template <int MAXP, bool XSMEM, bool TMA>
 cudaError_t launch_k2(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k2_experts<MAXP, XSMEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k2_experts<MAXP, XSMEM, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemLimit);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
-  cudaError_t e =
-      launch_pdl(k2_experts<MAXP, XSMEM>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM), stream, a);
+  cudaError_t e = launch_pdl(k2_experts<MAXP, XSMEM, TMA>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM),
+                             stream, a);
   if (e != cudaSuccess) return e;
   if (a.ev_end) cudaEventRecord(a.ev_end, stream);
   return cudaSuccess;
+}
+
+template <int MAXP, bool XSMEM>
+cudaError_t launch_k2_tma(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
+  return a.wt.tma ? launch_k2<MAXP, XSMEM, true>(a, stream, num_sms) : launch_k2<MAXP, XSMEM, false>(a, stream, num_sms);
 }
 
 cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
@@ -1523,6 +1603,42 @@ cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+void build_chunk_tensor_maps(LayerWeights &wt, const LayerDims &d) {
+  wt.tma = 0;
+  const int PH = decode_kparts(d.H), PD = decode_kparts(d.I);
+  const int cbI = d.H / PH / 256;       // IQ2_XXS blocks per gate/up chunk
+  const int cbD = d.I / PD / 256;       // Q2_K blocks per down unit
+  const int nbD = cbD < 2 ? cbD : 2;    // Q2_K blocks per down chunk
+  const size_t rbI = (size_t)(d.H / 256) * 66, rbD = (size_t)(d.I / 256) * 84;
+  const size_t rbQ = (size_t)(d.H / 32) * 34, rbQd = (size_t)(d.Is / 32) * 34;
+  // 16-byte row strides, and chunk starts at 0 or 4/8 (IQ2_XXS) or 0/8 (Q2_K)
+  // bytes past a 16-byte boundary, which the decoders' alignment allows
+  if (rbI % 16 || rbD % 16 || rbQ % 16 || rbQd % 16 || cbI % 2 || nbD != 2) return;
+  PFN_cuTensorMapEncodeTiled encode = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&encode), cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !encode)
+    return;
+  auto make = [&](TensorMap &m, const void *base, size_t row_bytes, size_t rows, int box_bytes) {
+    const cuuint64_t dims[2] = {row_bytes / 2, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(box_bytes / 2), 16};
+    const cuuint32_t es[2] = {1, 1};
+    return encode(reinterpret_cast<CUtensorMap *>(&m), CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base),
+                  dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  const int boxI = (int)align_up((size_t)cbI * 66, 16), boxD = (int)align_up((size_t)nbD * 84, 16), boxQ = 8 * 34;
+  const bool ok = make(wt.tm[kTmGate], wt.gate, rbI, (size_t)d.E * d.I, boxI) &&
+                  make(wt.tm[kTmUp], wt.up, rbI, (size_t)d.E * d.I, boxI) &&
+                  make(wt.tm[kTmDown], wt.down, rbD, (size_t)d.E * d.H, boxD) &&
+                  make(wt.tm[kTmShGate], wt.sh_gate, rbQ, (size_t)d.Is, boxQ) &&
+                  make(wt.tm[kTmShUp], wt.sh_up, rbQ, (size_t)d.Is, boxQ) &&
+                  make(wt.tm[kTmShDown], wt.sh_down, rbQd, (size_t)d.H, boxQ);
+  wt.tma = ok ? 1 : 0;
+}
 
 size_t decode_scratch_bytes(const LayerDims &d, int T) {
   DecodeScratch s;
@@ -1580,11 +1696,11 @@ cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms
   cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
   if (a.T <= 2) {
-    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2<1, true>(a, stream, num_sms);
-    return launch_k2<1, false>(a, stream, num_sms);
+    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2_tma<1, true>(a, stream, num_sms);
+    return launch_k2_tma<1, false>(a, stream, num_sms);
   }
-  if (a.T <= 4) return launch_k2<2, false>(a, stream, num_sms);
-  return launch_k2<4, false>(a, stream, num_sms);
+  if (a.T <= 4) return launch_k2_tma<2, false>(a, stream, num_sms);
+  return launch_k2_tma<4, false>(a, stream, num_sms);
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {

@@ -17,12 +17,32 @@ struct LayerDims {
   float scaling, eps;
 };
 
+// Opaque TMA tensor descriptor (the driver's 128-byte, 64-byte aligned
+// CUtensorMap), built on the host and read by the TMA unit from the kernel's
+// parameter space.
+struct alignas(64) TensorMap {
+  uint64_t v[16];
+};
+
+// Tensor maps of the packed weights for the small-T kernel's chunk loads:
+// each matrix viewed as [rows][row_bytes / 2] 16-bit elements, box = 16 rows x
+// the staged row width.  Order: gate, up, down, shared gate, shared up, shared
+// down.
+enum { kTmGate = 0, kTmUp, kTmDown, kTmShGate, kTmShUp, kTmShDown, kNumTm };
+
 struct LayerWeights {
   const uint16_t *Wr;
   const float *bias;
   const int32_t *tid2eid;
   const uint8_t *gate, *up, *down, *sh_gate, *sh_up, *sh_down, *grid;
+  int tma;  // 1 when tm[] is valid and every chunk start keeps the decoders' alignment
+  TensorMap tm[kNumTm];
 };
+
+// Builds wt.tm[] and sets wt.tma (0 when a shape does not allow TMA chunk
+// loads or the driver entry point is missing); the small-T kernel then
+// stages its chunks with TMA instead of cp.async.
+void build_chunk_tensor_maps(LayerWeights &wt, const struct LayerDims &d);
 
 // K parts of the decode path's warp units: every unit covers 16 weight rows
 // and a K range of kDecodeKPart elements (256 where the dimension is not a
