@@ -570,8 +570,8 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
 }
 
 // Dynamic unit scheduling on the warp's two-stage ring.  A warp claims G
-// consecutive units at a time from `counter`; the ring runs on across unit
-// boundaries.
+// consecutive units at a time (claim() returns the first, warp-uniform); the
+// ring runs on across unit boundaries.
 //   valid(u)          -> false once u is past the last unit (may wait until
 //                        the unit count is known)
 //   unit_at(u)        -> UnitT with field nch (chunks of the unit)
@@ -579,10 +579,10 @@ __device__ __forceinline__ void run_chunks(uint8_t *stage0, uint8_t *stage1, int
 //   compute(unit, u, c, data, next_u): consume chunk c of unit u, staged at
 //                        `data`; next_u is the unit of the next chunk the warp
 //                        computes (-1 when none), for segment bookkeeping
-template <int G, bool AHEAD, bool TMA, typename UnitT, typename Valid, typename UnitAt, typename ChunkOf,
-          typename Compute>
+template <int G, bool AHEAD, bool TMA, typename UnitT, typename Claim, typename Valid, typename UnitAt,
+          typename ChunkOf, typename Compute>
 __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, uint64_t *mbar, const TensorMap *tm,
-                                          int *err, int *counter, Valid valid, UnitAt unit_at, ChunkOf chunk_of,
+                                          int *err, Claim claim, Valid valid, UnitAt unit_at, ChunkOf chunk_of,
                                           Compute compute) {
   const int lane = threadIdx.x & 31;
   int s_u = 0, s_left = 0, s_c = 0;
@@ -591,9 +591,7 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, uint64_t *
   auto stage_next = [&](uint8_t *dst, int slot, int &uid, int &cidx, int &shift) -> bool {
     if (s_c == 0) {
       if (s_left == 0) {
-        int u = 0;
-        if (lane == 0) u = atomicAdd(counter, G);
-        s_u = __shfl_sync(0xffffffffu, u, 0);
+        s_u = claim();
         s_left = G;
       } else {
         ++s_u;
@@ -1036,6 +1034,9 @@ struct K2Shared {
   int jobs_ready;  // set once the routing warps have published idx, w and J
   float hsm[kWarps2][kDecodeMaxT][16];
   uint64_t mbar[kWarps2][2];  // TMA completion of each warp's two stages
+  float xs[kDecodeMaxT * 4];  // limb scales of x (when its limbs are made here)
+  double red[kWarps2];
+  float redf[kWarps2];
 };
 
 // Writes the 16 x ntok SwiGLU outputs held in hs (token slot, row) for the
@@ -1141,16 +1142,80 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   build_tables(a.wt.grid, gpm, selt, a.err);
-  pdl_wait();  // k1's limbs and keys are visible from here on
+  const int nw = (int)(blockDim.x >> 5);
   if (XSMEM) {
-    const int n16 = d.H / 16;
-    copy_rows16(xsm, XS, s.xq, d.H, T * 3, n16);
+    // The x limbs of the T tokens are made here from x itself (as k1 makes
+    // them), so the shared expert's gate/up units can run while k1 is still
+    // computing the router: nothing before the first counter update below
+    // reads k1's results.
+    const int n4 = d.H / 4;
+    for (int t = 0; t < T; ++t) {
+      const float4 *xt = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H);
+      double ss = 0.0;
+      float amax = 0.f;
+      for (int j = tid; j < n4; j += blockDim.x) {
+        const float4 v = xt[j];
+        ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
+      }
+      ss = warp_sum_d(ss);
+      amax = warp_max(amax);
+      if (lane == 0) {
+        S.red[warp] = ss;
+        S.redf[warp] = amax;
+      }
+      __syncthreads();
+      ss = 0.0;
+      amax = 0.f;
+      for (int w = 0; w < nw; ++w) {
+        ss += S.red[w];
+        amax = fmaxf(amax, S.redf[w]);
+      }
+      float inv = 1.f;
+      if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) {
+        inv = (float)(1.0 / sqrt(ss / (double)d.H + (double)d.eps));
+        amax = amax * inv;
+      }
+      const float s1 = amax > 0.f ? amax / 127.f : 1.f;
+      const float s2 = s1 / 254.f, s3 = s2 / 254.f;
+      const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
+      for (int j = tid; j < n4; j += blockDim.x) {
+        const float4 v = xt[j];
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w1 = 0u, w2 = 0u, w3 = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float xv = e[q] * inv;
+          const float q1 = fminf(fmaxf(rintf(xv * r1), -127.f), 127.f);
+          const float e1 = fmaf(-q1, s1, xv);
+          const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+          const float e2 = fmaf(-q2, s2, e1);
+          const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+          w1 |= ((uint32_t)(int)q1 & 255u) << (8 * q);
+          w2 |= ((uint32_t)(int)q2 & 255u) << (8 * q);
+          w3 |= ((uint32_t)(int)q3 & 255u) << (8 * q);
+        }
+        *reinterpret_cast<uint32_t *>(xsm + (size_t)(t * 3 + 0) * XS + 4 * j) = w1;
+        *reinterpret_cast<uint32_t *>(xsm + (size_t)(t * 3 + 1) * XS + 4 * j) = w2;
+        *reinterpret_cast<uint32_t *>(xsm + (size_t)(t * 3 + 2) * XS + 4 * j) = w3;
+      }
+      if (tid == 0) {
+        S.xs[4 * t] = s1;
+        S.xs[4 * t + 1] = s2;
+        S.xs[4 * t + 2] = s3;
+        S.xs[4 * t + 3] = 0.f;
+      }
+      __syncthreads();
+    }
+  } else {
+    pdl_wait();  // k1's limbs and keys are visible from here on
+    __syncthreads();
   }
-  __syncthreads();
   // Warps 0..T-1 route one token each and warp 0 builds the job table; the
   // other warps start on the shared expert's gate/up units, which need no
   // routing, and wait for the table only when they claim a routed unit.
   if (warp < T) {
+    pdl_wait();  // the router's keys
     warp_route_token(a, warp, S.idx + warp * d.k, S.w + warp * d.k);
     asm volatile("bar.sync 1, %0;\n" ::"r"(32 * T) : "memory");
     if (warp == 0) {
@@ -1346,7 +1411,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       if (p < npairs) {
         const int ts = 2 * p + (c >> 1);
         float v0, v1;
-        combine_limbs(F[p], ts < cu.ntok ? s.xs + 4 * xrow(cu, ts) : nullptr, v0, v1);
+        combine_limbs(F[p], ts < cu.ntok ? (XSMEM ? S.xs : s.xs) + 4 * xrow(cu, ts) : nullptr, v0, v1);
         if ((c & 1) == 0 && ts < cu.ntok) {
           float *pp = s.gpart + ((size_t)(m * PH + cu.part) * V + hvec(cu, ts)) * s.Imax + cu.tile * 16;
           pp[r] = v0;
@@ -1359,6 +1424,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   // gate/up: count the segment's parts in; the warp that completes the tile
   // sums the parts in order, applies the SwiGLU and hands the tile on
   auto end_gateup = [&](const Unit &cu) {
+    pdl_wait();  // the counters are reset by k1
     __syncwarp();
     const int set = cu.kind == 0 ? 0 : 1 + cu.j;
     int last = 0;
@@ -1426,8 +1492,24 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     }
   };
 
+  // Claims: with the x limbs made here, every non-routing warp first takes
+  // one shared gate/up unit by its number (no counter: k1 resets the
+  // counters); the remaining units come from the counter after k1 is done.
+  const int gwn = (warp - T) * (int)gridDim.x + (int)blockIdx.x;
+  bool first_static = XSMEM && warp >= T && gwn < n_sh;
+  const int n_static = XSMEM ? min(n_sh, (nw - T) * (int)gridDim.x) : 0;
+  auto claim = [&]() -> int {
+    if (first_static) {
+      first_static = false;
+      return gwn;
+    }
+    pdl_wait();
+    int u = 0;
+    if (lane == 0) u = atomicAdd(s.work + 0, kClaim);
+    return n_static + __shfl_sync(0xffffffffu, u, 0);
+  };
   run_units<kClaim, kAheadClaim, TMA, Unit>(
-      st0, st1, &S.mbar[warp][0], a.wt.tm, a.err, s.work + 0, valid, unit_at, chunk_of,
+      st0, st1, &S.mbar[warp][0], a.wt.tm, a.err, claim, valid, unit_at, chunk_of,
       [&](const Unit &cu, int u, int cc, const uint8_t *st, int next_u) {
         if (cu.kind <= 1) {
           // ------------------------------------------------ gate/up
