@@ -1032,6 +1032,7 @@ struct K2Shared {
   float w[kDecodeMaxT * kMaxK];
   Jobs J;
   int jobs_ready;  // set once the routing warps have published idx, w and J
+  int limbs_ready;  // set once the x limbs made in this block are in xsm
   float hsm[kWarps2][kDecodeMaxT][16];
   uint64_t mbar[kWarps2][2];  // TMA completion of each warp's two stages
   float xs[kDecodeMaxT * 4];  // limb scales of x (when its limbs are made here)
@@ -1135,25 +1136,32 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   const int XS = d.H + 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  if (tid == 0) S.jobs_ready = 0;
+  if (tid == 0) {
+    S.jobs_ready = 0;
+    S.limbs_ready = 0;
+  }
+  __syncthreads();
   if (TMA && lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&S.mbar[warp][0])) : "memory");
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&S.mbar[warp][1])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   build_tables(a.wt.grid, gpm, selt, a.err);
+  __syncthreads();  // tables in place for every warp
   const int nw = (int)(blockDim.x >> 5);
-  if (XSMEM) {
+  if (XSMEM && warp >= T) {
     // The x limbs of the T tokens are made here from x itself (as k1 makes
-    // them), so the shared expert's gate/up units can run while k1 is still
+    // them) by the warps that do not route, on a named barrier of their own,
+    // so the shared expert's gate/up units can run while k1 is still
     // computing the router: nothing before the first counter update below
     // reads k1's results.
+    const int ltid = tid - 32 * T, lthreads = (nw - T) * 32;
     const int n4 = d.H / 4;
     for (int t = 0; t < T; ++t) {
       const float4 *xt = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H);
       double ss = 0.0;
       float amax = 0.f;
-      for (int j = tid; j < n4; j += blockDim.x) {
+      for (int j = ltid; j < n4; j += lthreads) {
         const float4 v = xt[j];
         ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
         amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
@@ -1164,10 +1172,10 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
         S.red[warp] = ss;
         S.redf[warp] = amax;
       }
-      __syncthreads();
+      asm volatile("bar.sync 2, %0;\n" ::"r"(lthreads) : "memory");
       ss = 0.0;
       amax = 0.f;
-      for (int w = 0; w < nw; ++w) {
+      for (int w = T; w < nw; ++w) {
         ss += S.red[w];
         amax = fmaxf(amax, S.redf[w]);
       }
@@ -1179,7 +1187,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       const float s1 = amax > 0.f ? amax / 127.f : 1.f;
       const float s2 = s1 / 254.f, s3 = s2 / 254.f;
       const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
-      for (int j = tid; j < n4; j += blockDim.x) {
+      for (int j = ltid; j < n4; j += lthreads) {
         const float4 v = xt[j];
         const float e[4] = {v.x, v.y, v.z, v.w};
         uint32_t w1 = 0u, w2 = 0u, w3 = 0u;
@@ -1199,15 +1207,19 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
         *reinterpret_cast<uint32_t *>(xsm + (size_t)(t * 3 + 1) * XS + 4 * j) = w2;
         *reinterpret_cast<uint32_t *>(xsm + (size_t)(t * 3 + 2) * XS + 4 * j) = w3;
       }
-      if (tid == 0) {
+      if (ltid == 0) {
         S.xs[4 * t] = s1;
         S.xs[4 * t + 1] = s2;
         S.xs[4 * t + 2] = s3;
         S.xs[4 * t + 3] = 0.f;
       }
-      __syncthreads();
+      asm volatile("bar.sync 2, %0;\n" ::"r"(lthreads) : "memory");
     }
-  } else {
+    if (ltid == 0) {
+      __threadfence_block();
+      *reinterpret_cast<volatile int *>(&S.limbs_ready) = 1;
+    }
+  } else if (!XSMEM) {
     pdl_wait();  // k1's limbs and keys are visible from here on
     __syncthreads();
   }
@@ -1492,6 +1504,19 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     }
   };
 
+  if (XSMEM && warp < T) {
+    // the routing warps compute units only once the limbs are in place
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile int *>(&S.limbs_ready) == 0) {
+      if (clock64() - t0 > kSliceWaitCycles) {
+        set_error(a.err, kErrTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+    __syncwarp();
+    __threadfence_block();
+  }
   // Claims: with the x limbs made here, every non-routing warp first takes
   // one shared gate/up unit by its number (no counter: k1 resets the
   // counters); the remaining units come from the counter after k1 is done.
