@@ -584,7 +584,6 @@ template <int G, bool AHEAD, bool TMA, typename UnitT, typename Claim, typename 
 __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, uint64_t *mbar, const TensorMap *tm,
                                           int *err, Claim claim, Valid valid, UnitAt unit_at, ChunkOf chunk_of,
                                           Compute compute) {
-  const int lane = threadIdx.x & 31;
   int s_u = 0, s_left = 0, s_c = 0;
   UnitT su;
   // stages the next chunk into slot `slot` (TMA) or commits its cp.async group
@@ -667,9 +666,6 @@ __device__ __forceinline__ uint2 ldb(const BColG &b, int kel) {
   uint2 v = make_uint2(0u, 0u);
   if (b.ok) v = __ldcg(reinterpret_cast<const uint2 *>(b.p + kel));  // via L2: may be written by this kernel
   return v;
-}
-__device__ __forceinline__ uint32_t ldx(const BColS &b, int off) {
-  return b.ok ? *reinterpret_cast<const uint32_t *>(b.p + off) : 0u;
 }
 __device__ __forceinline__ uint32_t ldx(const BColG &b, int off) {
   return b.ok ? __ldcg(reinterpret_cast<const unsigned *>(b.p + off)) : 0u;
@@ -986,32 +982,6 @@ __device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, i
   }
 }
 
-// Copies `rows` rows of n16 16-byte words from global (row stride gs bytes)
-// into shared memory (row stride ss bytes) with the whole block; each thread
-// issues a batch of independent loads before storing any.
-__device__ __forceinline__ void copy_rows16(void *dst, size_t ss, const void *src, size_t gs, int rows, int n16) {
-  constexpr int kB = 4;
-  const int n = rows * n16, step = blockDim.x;
-  for (int i0 = threadIdx.x; i0 < n; i0 += kB * step) {
-    uint4 v[kB];
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int i = i0 + u * step;
-      if (i < n) {
-        const int r = i / n16, o = i - r * n16;
-        v[u] = __ldcg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(src) + r * gs + 16 * o));
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int i = i0 + u * step;
-      if (i < n) {
-        const int r = i / n16, o = i - r * n16;
-        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(dst) + r * ss + 16 * o) = v[u];
-      }
-    }
-  }
-}
 
 // ------------------------------------------------------------------ k2
 
