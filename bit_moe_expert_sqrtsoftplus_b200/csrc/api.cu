@@ -282,6 +282,7 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxT = 8;                            // tokens per call of the no-alloc forward
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 128;
@@ -310,9 +311,9 @@ moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t 
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
   if (T == 0) return MOE_OK;
-  if (T > moe::kDecodeMaxT)
+  if (T > kNoAllocMaxT)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_forward_noalloc handles at most %d tokens per call (got %d)",
-                moe::kDecodeMaxT, T);
+                kNoAllocMaxT, T);
   const size_t need = moe::decode_scratch_bytes(h->d, T);
   if (need > kStaticScratchBytes)
     return fail(MOE_ERR_WORKSPACE_TOO_SMALL,

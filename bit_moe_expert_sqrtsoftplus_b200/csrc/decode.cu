@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
   {
     // per-call counters and flags of the expert kernel, spread over the grid
     const int V = T * d.k + T;
-    const int nv = V * a.s.NSL, nh = (1 + a.s.Jmax) * a.s.TM, ny = d.H / 16;
+    const int nv = V * a.s.NSL, nh = (a.s.G + a.s.Jmax) * a.s.TM, ny = d.H / 16;
     for (int i = blockIdx.x * blockDim.x + tid; i < nv + nh + ny + 4; i += gridDim.x * blockDim.x) {
       if (i < nv) {
         a.s.hmax[i] = 0u;
@@ -200,68 +200,74 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
   const int e0 = 2 * ((int)blockIdx.x - T);
   if (e0 >= d.E) return;
   const bool two = e0 + 1 < d.E;
-  double acc0[MAXT], acc1[MAXT], ssq[MAXT];
-#pragma unroll
-  for (int t = 0; t < MAXT; ++t) acc0[t] = acc1[t] = ssq[t] = 0.0;
   const uint16_t *w0 = a.wt.Wr + (size_t)e0 * d.H;
   const uint16_t *w1 = a.wt.Wr + (size_t)(two ? e0 + 1 : e0) * d.H;
-  // every thread covers 8 consecutive elements per pass; all loads of a pass are independent
-  for (int j = tid * 8; j < d.H; j += kRouterThreads * 8) {
-    const uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
-    const uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
-    float4 xv[MAXT][2];
+  // tokens in groups of MAXT (the two weight rows are re-read from L1/L2)
+  for (int t0 = 0; t0 < T; t0 += MAXT) {
+    const int nt = min(MAXT, T - t0);
+    double acc0[MAXT], acc1[MAXT], ssq[MAXT];
 #pragma unroll
-    for (int t = 0; t < MAXT; ++t) {
-      if (t < T) {
-        const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H + j);
-        xv[t][0] = xp[0];
-        xv[t][1] = xp[1];
+    for (int t = 0; t < MAXT; ++t) acc0[t] = acc1[t] = ssq[t] = 0.0;
+    // every thread covers 8 consecutive elements per pass; all loads of a pass are independent
+    for (int j = tid * 8; j < d.H; j += kRouterThreads * 8) {
+      const uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
+      const uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
+      float4 xv[MAXT][2];
+#pragma unroll
+      for (int t = 0; t < MAXT; ++t) {
+        if (t < nt) {
+          const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)(t0 + t) * d.H + j);
+          xv[t][0] = xp[0];
+          xv[t][1] = xp[1];
+        }
       }
-    }
-    const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
-    const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
+      const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
+      const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
 #pragma unroll
-    for (int t = 0; t < MAXT; ++t) {
-      if (t < T) {
-        const float xe[8] = {xv[t][0].x, xv[t][0].y, xv[t][0].z, xv[t][0].w,
-                             xv[t][1].x, xv[t][1].y, xv[t][1].z, xv[t][1].w};
+      for (int t = 0; t < MAXT; ++t) {
+        if (t < nt) {
+          const float xe[8] = {xv[t][0].x, xv[t][0].y, xv[t][0].z, xv[t][0].w,
+                               xv[t][1].x, xv[t][1].y, xv[t][1].z, xv[t][1].w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const double xd = (double)xe[i];
-          acc0[t] = fma((double)half_bits_to_float(p0[i]), xd, acc0[t]);
-          acc1[t] = fma((double)half_bits_to_float(p1[i]), xd, acc1[t]);
-          ssq[t] = fma(xd, xd, ssq[t]);
+          for (int i = 0; i < 8; ++i) {
+            const double xd = (double)xe[i];
+            acc0[t] = fma((double)half_bits_to_float(p0[i]), xd, acc0[t]);
+            acc1[t] = fma((double)half_bits_to_float(p1[i]), xd, acc1[t]);
+            ssq[t] = fma(xd, xd, ssq[t]);
+          }
         }
       }
     }
-  }
 #pragma unroll
-  for (int t = 0; t < MAXT; ++t) {
-    if (t < T) {
-      const double v0 = warp_sum_d(acc0[t]);
-      const double v1 = warp_sum_d(acc1[t]);
-      const double v2 = warp_sum_d(ssq[t]);
-      if (lane == 0) {
-        red[warp][t] = v0;
-        red[warp][MAXT + t] = v1;
-        red[warp][2 * MAXT + t] = v2;
+    for (int t = 0; t < MAXT; ++t) {
+      if (t < nt) {
+        const double v0 = warp_sum_d(acc0[t]);
+        const double v1 = warp_sum_d(acc1[t]);
+        const double v2 = warp_sum_d(ssq[t]);
+        if (lane == 0) {
+          red[warp][t] = v0;
+          red[warp][MAXT + t] = v1;
+          red[warp][2 * MAXT + t] = v2;
+        }
       }
     }
-  }
-  __syncthreads();
-  if (tid < 2 * T) {
-    const int t = tid >> 1, which = tid & 1;
-    if (which == 1 && !two) return;
-    double z = 0.0, s2 = 0.0;
-    for (int w = 0; w < NW; ++w) {
-      z += red[w][which * MAXT + t];
-      s2 += red[w][2 * MAXT + t];
+    __syncthreads();
+    if (tid < 2 * nt) {
+      const int t = tid >> 1, which = tid & 1;
+      if (which == 0 || two) {
+        double z = 0.0, s2 = 0.0;
+        for (int w = 0; w < NW; ++w) {
+          z += red[w][which * MAXT + t];
+          s2 += red[w][2 * MAXT + t];
+        }
+        if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) z *= 1.0 / sqrt(s2 / (double)d.H + (double)d.eps);
+        const int e = e0 + which;
+        const double sc = sqrtsoftplus(z);
+        a.s.sc[(size_t)(t0 + t) * d.E + e] = sc;
+        a.s.z[(size_t)(t0 + t) * d.E + e] = sc + (double)a.wt.bias[e];
+      }
     }
-    if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) z *= 1.0 / sqrt(s2 / (double)d.H + (double)d.eps);
-    const int e = e0 + which;
-    const double sc = sqrtsoftplus(z);
-    a.s.sc[(size_t)t * d.E + e] = sc;
-    a.s.z[(size_t)t * d.E + e] = sc + (double)a.wt.bias[e];
+    __syncthreads();  // red is reused by the next group
   }
 }
 
@@ -370,7 +376,8 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
 }
 
 // Job table: the distinct selected experts in ascending order, each with its
-// (token, slot) pairs in ascending token order.
+// (token, slot) pairs in ascending token order; an expert with more than
+// kUnitMaxTok pairs is split into consecutive jobs of at most kUnitMaxTok.
 struct Jobs {
   int n;
   int e[kDecodeMaxT * kMaxK];
@@ -411,7 +418,43 @@ __device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
   }
   __syncwarp();
   for (int g = lane; g < ng; g += 32) J.cnt[g] = (g + 1 < ng ? J.first[g + 1] : np) - J.first[g];
-  if (lane == 0) J.n = ng;
+  __syncwarp();
+  if (np <= kUnitMaxTok) {  // no expert can hold more pairs than a unit
+    if (lane == 0) J.n = ng;
+    __syncwarp();
+    return;
+  }
+  // split: every lane takes groups lane, lane + 32, ... (at most 8 with
+  // np <= 256); exclusive prefix of the job counts over the groups in order
+  int ge[8], gf[8], gc[8], nj[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int g = lane + 32 * q;
+    ge[q] = g < ng ? J.e[g] : 0;
+    gf[q] = g < ng ? J.first[g] : 0;
+    gc[q] = g < ng ? J.cnt[g] : 0;
+    nj[q] = (gc[q] + kUnitMaxTok - 1) / kUnitMaxTok;
+  }
+  __syncwarp();
+  int base = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    // jobs of the groups before lane + 32q: all of round q's lower lanes plus base
+    int incl = nj[q];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int start = base + incl - nj[q];
+    for (int c = 0; c < nj[q]; ++c) {
+      J.e[start + c] = ge[q];
+      J.first[start + c] = gf[q] + kUnitMaxTok * c;
+      J.cnt[start + c] = min(kUnitMaxTok, gc[q] - kUnitMaxTok * c);
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) J.n = base;
   __syncwarp();
 }
 
@@ -1003,7 +1046,7 @@ struct K2Shared {
   Jobs J;
   int jobs_ready;  // set once the routing warps have published idx, w and J
   int limbs_ready;  // set once the x limbs made in this block are in xsm
-  float hsm[kWarps2][kDecodeMaxT][16];
+  float hsm[kWarps2][kUnitMaxTok][16];
   uint64_t mbar[kWarps2][2];  // TMA completion of each warp's two stages
   float xs[kDecodeMaxT * 4];  // limb scales of x (when its limbs are made here)
   double red[kWarps2];
@@ -1196,10 +1239,11 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   // Warps 0..T-1 route one token each and warp 0 builds the job table; the
   // other warps start on the shared expert's gate/up units, which need no
   // routing, and wait for the table only when they claim a routed unit.
-  if (warp < T) {
+  const int nr = T < nw ? T : nw;  // routing warps
+  if (warp < nr) {
     pdl_wait();  // the router's keys
-    warp_route_token(a, warp, S.idx + warp * d.k, S.w + warp * d.k);
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * T) : "memory");
+    for (int t = warp; t < T; t += nr) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
+    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * nr) : "memory");
     if (warp == 0) {
       warp_build_jobs(S.idx, T, d.k, S.J);
       if (blockIdx.x == 0)
@@ -1250,8 +1294,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   const int NS = s.NS;
   // ---- unit ranges; the ones past the shared gate/up units depend on the
   // number of jobs and are set once the job table is ready
-  const int n_sh = tilesS * PH;
-  const int n3s = PS * tilesH;
+  const int n_sh = s.G * tilesS * PH;
+  const int n3s = s.G * PS * tilesH;
   int nparts = 0, n2 = 0, n_units = -1;  // parts of an output tile, unit ranges
   auto valid = [&](int u) {
     if (u < n_sh) return true;
@@ -1269,7 +1313,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       __syncwarp();
       __threadfence_block();
       if (!ok) return false;
-      nparts = S.J.n * PD + PS;
+      nparts = S.J.n * PD + s.G * PS;
       n2 = n_sh + S.J.n * tilesI * PH;
       n_units = n2 + n3s + S.J.n * PD * tilesH;
     }
@@ -1280,18 +1324,32 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     int kind;  // 0 shared gate/up, 1 routed gate/up, 2 shared down, 3 routed down
     int j, e, tile, part, ntok, per, nch;  // gate/up: 16-row tile, K part of H, chunks per matrix
     int ot, kp;                            // down: output tile, K part (slice) of I or Is
+    int t0;                                // shared: first token of the unit's token group
     const int *pairs;
+  };
+  // the shared expert's tokens in groups of kUnitMaxTok: group g holds tokens
+  // kUnitMaxTok * g ..; its units are numbered like one group's, group-major
+  const int shG = s.G;
+  const int nshg = tilesS * PH, n3sg = PS * tilesH;  // units of one group
+  auto shared_group = [&](int w, int per_group, int &rem) {
+    const int g = shG == 1 ? 0 : w / per_group;
+    rem = w - g * per_group;
+    return g;
   };
   auto unit_at = [&](int u) {
     Unit x;
-    x.j = x.e = x.tile = x.part = x.ot = x.kp = 0;
+    x.j = x.e = x.tile = x.part = x.ot = x.kp = x.t0 = 0;
     x.per = 1;
     x.pairs = nullptr;
     x.ntok = T;
     if (u < n_sh) {
       x.kind = 0;
-      x.tile = s.fPH.div(u);
-      x.part = u - x.tile * PH;
+      int rem;
+      const int g = shared_group(u, nshg, rem);
+      x.t0 = kUnitMaxTok * g;
+      x.ntok = min(kUnitMaxTok, T - x.t0);
+      x.tile = s.fPH.div(rem);
+      x.part = rem - x.tile * PH;
       x.per = nq8;
       x.nch = 2 * nq8;
     } else if (u < n2) {
@@ -1304,7 +1362,10 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       x.nch = 2;
     } else if (u < n2 + n3s) {
       x.kind = 2;
-      const int w = u - n2;
+      int w;
+      const int g = shared_group(u - n2, n3sg, w);
+      x.t0 = kUnitMaxTok * g;
+      x.ntok = min(kUnitMaxTok, T - x.t0);
       x.kp = s.fTH.div(w);
       x.ot = w - x.kp * tilesH;
       x.nch = nqd;
@@ -1325,8 +1386,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     return x;
   };
   // token slot ts of a unit -> row of x / vector of h
-  auto xrow = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] / d.k : ts; };
-  auto hvec = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] : T * d.k + ts; };
+  auto xrow = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] / d.k : x.t0 + ts; };
+  auto hvec = [&](const Unit &x, int ts) { return (x.kind & 1) ? x.pairs[ts] : T * d.k + x.t0 + ts; };
   auto chunk_of = [&](const Unit &su, int cs) {
     Chunk ch;
     size_t off;  // byte offset of the chunk within its row
@@ -1408,7 +1469,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   auto end_gateup = [&](const Unit &cu) {
     pdl_wait();  // the counters are reset by k1
     __syncwarp();
-    const int set = cu.kind == 0 ? 0 : 1 + cu.j;
+    const int set = cu.kind == 0 ? cu.t0 / kUnitMaxTok : s.G + cu.j;
     int last = 0;
     if (lane == 0) last = atomic_add_acq_rel(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
     last = __shfl_sync(0xffffffffu, last, 0);
@@ -1437,9 +1498,9 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       S.hsm[warp][ts][row] = silu(ga) * ub;
     }
     __syncwarp();
-    int vec[kDecodeMaxT];
+    int vec[kUnitMaxTok];
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxT; ++t) vec[t] = t < cu.ntok ? hvec(cu, t) : 0;
+    for (int t = 0; t < kUnitMaxTok; ++t) vec[t] = t < cu.ntok ? hvec(cu, t) : 0;
     finish_h_tile(a, S.hsm[warp], cu.ntok, vec, r0, cu.kind == 0 ? kps : kpd);
   };
   // down: the part is in its slot; the warp that completes the output tile
@@ -1595,11 +1656,11 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
             for (int p = 0; p < MAXP; ++p) {
               if (p < npairs) {
                 const int ts = 2 * p + (c >> 1);
-                const float *sc = ts < T ? s.hsc + 4 * ((T * d.k + ts) * s.NSL + cu.kp) : nullptr;
+                const float *sc = ts < cu.ntok ? s.hsc + 4 * ((T * d.k + cu.t0 + ts) * s.NSL + cu.kp) : nullptr;
                 float v0, v1;
                 combine_limbs(F[p], sc, v0, v1);
-                if ((c & 1) == 0 && ts < T) {
-                  float *dst = ytile + (size_t)(T * d.k * PD + ts * PS + cu.kp) * 16;
+                if ((c & 1) == 0 && ts < cu.ntok) {
+                  float *dst = ytile + (size_t)(T * d.k * PD + (cu.t0 + ts) * PS + cu.kp) * 16;
                   dst[r] = v0;
                   dst[r + 8] = v1;
                 }
@@ -1737,7 +1798,8 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.PH = decode_kparts(d.H);
   s.PD = decode_kparts(d.I);
   s.PS = decode_kparts(d.Is);
-  s.Jmax = T * d.k < d.E ? T * d.k : d.E;
+  s.Jmax = T * d.k;
+  s.G = (T + kUnitMaxTok - 1) / kUnitMaxTok;
   s.TM = Imax / 16;
   s.NS = T * d.k * s.PD + T * s.PS;
   s.NSL = s.PD > s.PS ? s.PD : s.PS;
@@ -1762,7 +1824,7 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.scount = reinterpret_cast<int *>(take(sizeof(int) * V * s.NSL));
   s.ready = reinterpret_cast<int *>(take(sizeof(int) * V * s.NSL));
   s.gpart = reinterpret_cast<float *>(take(sizeof(float) * 2 * (size_t)s.PH * V * Imax));
-  s.hcount = reinterpret_cast<int *>(take(sizeof(int) * (size_t)(1 + s.Jmax) * s.TM));
+  s.hcount = reinterpret_cast<int *>(take(sizeof(int) * (size_t)(s.G + s.Jmax) * s.TM));
   s.ypart = reinterpret_cast<float *>(take(sizeof(float) * (size_t)(d.H / 16) * s.NS * 16));
   s.ycount = reinterpret_cast<int *>(take(sizeof(int) * (d.H / 16)));
   s.work = reinterpret_cast<int *>(take(sizeof(int) * 4));

@@ -8,7 +8,8 @@
 
 namespace moe {
 
-constexpr int kDecodeMaxT = 8;  // token counts handled by the GEMV (mma.sync) path
+constexpr int kDecodeMaxT = 32;  // token counts handled by the GEMV (mma.sync) path
+constexpr int kUnitMaxTok = 8;   // tokens of one warp unit (4 MMA column pairs)
 constexpr int kMaxK = 8;
 constexpr int kMaxE = 256;
 
@@ -96,7 +97,7 @@ struct DecodeScratch {
   int *scount;      // [V][NSL] finished 16-row tiles per slice
   int *ready;       // [V][NSL] 1 once the slice's limbs are written
   float *gpart;     // [2][PH][V][Imax] gate/up partial sums per K part of H
-  int *hcount;      // [1 + Jmax][TM] finished K parts per (vector set, 16-row tile)
+  int *hcount;      // [G + Jmax][TM] finished K parts per (vector set, 16-row tile)
   float *ypart;     // [H/16][NS][16] partial output tiles, NS = T*k*PD + T*PS slots
   int *ycount;      // [H/16]
   int *work;        // [4] unit counters
@@ -104,7 +105,8 @@ struct DecodeScratch {
   int Imax;
   int PH, PD, PS;   // K parts of H (gate/up), I (routed down), Is (shared down)
   int NSL;          // slices per vector = max(PD, PS)
-  int Jmax;         // max routed vector sets = min(T*k, E)
+  int Jmax;         // max routed jobs (an expert's tokens, at most kUnitMaxTok per job) = T*k
+  int G;            // token groups of the shared expert (kUnitMaxTok tokens each)
   int TM;           // max(I, Is) / 16
   int NS;           // output slots per 16-row tile of y
   FastDiv fPH, fTIPH, fTH, fPD;  // divisors PH, (I/16)*PH, H/16, PD of the unit numbering

@@ -1,5 +1,5 @@
 """Parity of the CUDA layer against the fp64 oracle for the small-T path
-(T <= 8: mma.sync int8 GEMV kernels), routing for every T, and the layer's
+(T <= 32: mma.sync int8 GEMV kernels), routing for every T, and the layer's
 error paths.  Everything goes through the C ABI."""
 import numpy as np
 import pytest
@@ -56,6 +56,24 @@ def test_tiny_layer_matches_oracle(moe, T):
     s = synth.workload("tiny", tokens=T)
     got = _run(moe, s, 0, 0, T)
     _check(s, got, 0, 0)
+
+
+@pytest.mark.parametrize("T", [9, 16, 32])
+def test_tiny_layer_medium_token_counts(moe, T):
+    """9..32 tokens: the shared expert's tokens run in groups of 8 units' worth."""
+    s = synth.workload("tiny", tokens=T)
+    got = _run(moe, s, 0, 0, T)
+    _check(s, got, 0, 0)
+
+
+def test_experts_with_more_than_eight_tokens_are_split(moe):
+    """The skewed bias sends (nearly) every token to experts 0 and 8, so their
+    jobs hold more pairs than one unit and are split."""
+    s = synth.workload("tiny", tokens=24, skew=True)
+    got = _run(moe, s, 1, 0, 24)
+    counts = np.bincount(got["idx"].ravel(), minlength=s.n_experts)
+    assert counts.max() > 8, counts
+    _check(s, got, 1, 0)
 
 
 def test_tiny_hash_routed_layer(moe):

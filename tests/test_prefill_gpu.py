@@ -1,5 +1,6 @@
-"""Parity of the large-T path (certified router, permutation, tcgen05 grouped
-GEMMs with f16/bf16 operands) against the fp64 oracle, through the C ABI."""
+"""Parity of the large-T path (T > 32: certified router, permutation, tcgen05
+grouped GEMMs with f16/bf16 operands) against the fp64 oracle, through the C
+ABI; the full-shape 32-token case runs on the small-T path."""
 import numpy as np
 import pytest
 
