@@ -28,6 +28,7 @@ MOE_ERR_DEVICE_FAULT = -7
 MOE_ROUTE_ROUTER = 0
 MOE_ROUTE_HASH = 1
 MOE_FLAG_PRENORM_RESIDUAL = 1
+MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
             "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_destroy")

@@ -13,6 +13,8 @@
 #include "layer.cuh"
 #include "prefill.cuh"
 
+static_assert(MOE_SMALL_T_MAX == moe::kDecodeMaxT, "header and kernels disagree on the small-T limit");
+
 struct moe_handle {
   moe_config cfg;
   moe_weights w;

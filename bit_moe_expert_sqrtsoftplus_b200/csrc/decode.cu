@@ -1,4 +1,4 @@
-// decode.cu -- the layer for small token counts (T <= 8): two kernels.
+// decode.cu -- the layer for small token counts (T <= 32): two kernels.
 //
 //   k1_prep_router  x -> int8 limbs (optionally RMSNorm first); fp64 router
 //                   logits, scores s = sqrtsoftplus(z) and selection keys

@@ -1,4 +1,4 @@
-// prefill.cuh -- the layer for larger token counts (T > 8): certified router,
+// prefill.cuh -- the layer for larger token counts (T > 32): certified router,
 // token permutation and grouped tensor-core GEMMs.
 #pragma once
 

@@ -65,6 +65,8 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 /* flags */
 #define MOE_FLAG_PRENORM_RESIDUAL 1 /* forward computes x + MoE(RMSNorm(x)) */
 
+#define MOE_SMALL_T_MAX 32 /* largest T served by the small-token kernels */
+
 typedef struct {
   int hidden;           /* H: multiple of 256 (4096 for V4-Flash) */
   int inter;            /* I: routed expert intermediate, multiple of 256 (2048) */
@@ -129,7 +131,11 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
 /*
  * The whole layer.  x: [T][H] fp32 input; y: [T][H] fp32 output
  * (overwritten; may alias x only with MOE_FLAG_PRENORM_RESIDUAL, where
- * y = x + MoE(RMSNorm(x))).  T = 0 is a no-op.
+ * y = x + MoE(RMSNorm(x))).  T = 0 is a no-op.  Calls with
+ * T <= MOE_SMALL_T_MAX run the small-token path (two kernel launches: input
+ * preparation and router, then every expert unit); larger T the batched
+ * tensor-core path (twelve launches in router mode: router, certificate,
+ * fix-up, permutation, four grouped GEMMs).
  */
 moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
                            void *scratch, size_t scratch_bytes, moe_stream_t stream);

@@ -38,6 +38,18 @@ def test_exports_every_declared_function(moe):
         assert hasattr(lib, name), name
 
 
+def test_binding_constants_match_the_header(moe):
+    src = ""
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src += open(os.path.join(ROOT, "include", h)).read()
+    values = {n: int(v) for n, v in re.findall(r"#define\s+(MOE_[A-Z0-9_]+)\s+(-?\d+)", src)}
+    values.update({n: int(v) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(-?\d+)", src)})
+    assert {"MOE_OK", "MOE_ERR_TIMEOUT", "MOE_ROUTE_HASH", "MOE_FLAG_PRENORM_RESIDUAL", "MOE_SMALL_T_MAX"} <= set(values)
+    for name, v in values.items():
+        assert getattr(moe, name) == v, name
+
+
 def _cfg(moe, **over):
     base = dict(hidden=4096, inter=2048, n_experts=256, top_k=6, shared_inter=2048, vocab=129280)
     base.update(over)
