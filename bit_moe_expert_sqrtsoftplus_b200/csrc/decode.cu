@@ -377,7 +377,7 @@ __device__ void warp_route_token(const DecodeArgs &a, int t, int32_t *idx_out, f
 
 // Job table: the distinct selected experts in ascending order, each with its
 // (token, slot) pairs in ascending token order; an expert with more than
-// kUnitMaxTok pairs is split into consecutive jobs of at most kUnitMaxTok.
+// uw pairs (the kernel's unit width) is split into consecutive jobs of at most uw.
 struct Jobs {
   int n;
   int e[kDecodeMaxT * kMaxK];
@@ -390,7 +390,7 @@ static_assert(sizeof(Jobs) == sizeof(int) * kJobsInts, "job table layout");
 
 // Built by one warp (no block barrier): ranks of the (token, slot) pairs by
 // (expert, token), then the group starts by ballot.
-__device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
+__device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, int uw, Jobs &J) {
   const int lane = threadIdx.x & 31;
   const int np = T * k;
   for (int i = lane; i < np; i += 32) {
@@ -419,7 +419,7 @@ __device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
   __syncwarp();
   for (int g = lane; g < ng; g += 32) J.cnt[g] = (g + 1 < ng ? J.first[g + 1] : np) - J.first[g];
   __syncwarp();
-  if (np <= kUnitMaxTok) {  // no expert can hold more pairs than a unit
+  if (T <= uw) {  // an expert holds at most one pair per token: none exceeds a unit
     if (lane == 0) J.n = ng;
     __syncwarp();
     return;
@@ -433,7 +433,7 @@ __device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
     ge[q] = g < ng ? J.e[g] : 0;
     gf[q] = g < ng ? J.first[g] : 0;
     gc[q] = g < ng ? J.cnt[g] : 0;
-    nj[q] = (gc[q] + kUnitMaxTok - 1) / kUnitMaxTok;
+    nj[q] = (gc[q] + uw - 1) / uw;
   }
   __syncwarp();
   int base = 0;
@@ -449,8 +449,8 @@ __device__ void warp_build_jobs(const int32_t *idx_s, int T, int k, Jobs &J) {
     const int start = base + incl - nj[q];
     for (int c = 0; c < nj[q]; ++c) {
       J.e[start + c] = ge[q];
-      J.first[start + c] = gf[q] + kUnitMaxTok * c;
-      J.cnt[start + c] = min(kUnitMaxTok, gc[q] - kUnitMaxTok * c);
+      J.first[start + c] = gf[q] + uw * c;
+      J.cnt[start + c] = min(uw, gc[q] - uw * c);
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
@@ -1162,6 +1162,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   build_tables(a.wt.grid, gpm, selt, a.err);
   __syncthreads();  // tables in place for every warp
   const int nw = (int)(blockDim.x >> 5);
+  constexpr int kUW = 2 * MAXP;  // tokens per unit: 2 per MMA column pair
   if (XSMEM && warp >= T) {
     // The x limbs of the T tokens are made here from x itself (as k1 makes
     // them) by the warps that do not route, on a named barrier of their own,
@@ -1245,7 +1246,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     for (int t = warp; t < T; t += nr) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
     asm volatile("bar.sync 1, %0;\n" ::"r"(32 * nr) : "memory");
     if (warp == 0) {
-      warp_build_jobs(S.idx, T, d.k, S.J);
+      warp_build_jobs(S.idx, T, d.k, kUW, S.J);
       if (blockIdx.x == 0)
         for (int i = lane; i < T * d.k; i += 32) {
           s.idx[i] = S.idx[i];
@@ -1327,8 +1328,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     int t0;                                // shared: first token of the unit's token group
     const int *pairs;
   };
-  // the shared expert's tokens in groups of kUnitMaxTok: group g holds tokens
-  // kUnitMaxTok * g ..; its units are numbered like one group's, group-major
+  // the shared expert's tokens in groups of kUW: group g holds tokens
+  // kUW * g ..; its units are numbered like one group's, group-major
   const int shG = s.G;
   const int nshg = tilesS * PH, n3sg = PS * tilesH;  // units of one group
   auto shared_group = [&](int w, int per_group, int &rem) {
@@ -1346,8 +1347,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       x.kind = 0;
       int rem;
       const int g = shared_group(u, nshg, rem);
-      x.t0 = kUnitMaxTok * g;
-      x.ntok = min(kUnitMaxTok, T - x.t0);
+      x.t0 = kUW * g;
+      x.ntok = min(kUW, T - x.t0);
       x.tile = s.fPH.div(rem);
       x.part = rem - x.tile * PH;
       x.per = nq8;
@@ -1364,8 +1365,8 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       x.kind = 2;
       int w;
       const int g = shared_group(u - n2, n3sg, w);
-      x.t0 = kUnitMaxTok * g;
-      x.ntok = min(kUnitMaxTok, T - x.t0);
+      x.t0 = kUW * g;
+      x.ntok = min(kUW, T - x.t0);
       x.kp = s.fTH.div(w);
       x.ot = w - x.kp * tilesH;
       x.nch = nqd;
@@ -1469,7 +1470,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   auto end_gateup = [&](const Unit &cu) {
     pdl_wait();  // the counters are reset by k1
     __syncwarp();
-    const int set = cu.kind == 0 ? cu.t0 / kUnitMaxTok : s.G + cu.j;
+    const int set = cu.kind == 0 ? cu.t0 / kUW : s.G + cu.j;
     int last = 0;
     if (lane == 0) last = atomic_add_acq_rel(s.hcount + set * s.TM + cu.tile, seg_parts) + seg_parts == PH;
     last = __shfl_sync(0xffffffffu, last, 0);
@@ -1778,10 +1779,31 @@ void build_chunk_tensor_maps(LayerWeights &wt, const LayerDims &d) {
   wt.tma = ok ? 1 : 0;
 }
 
+// Tokens per unit of the expert kernel (2, 4 or 8: MAXP = width / 2 MMA
+// column pairs).  Wider units decode a weight tile once for more tokens, but
+// need more registers (12 warps per block instead of 16) and load their
+// activation fragments inside the MMA loop; since nearly every expert holds
+// one or two of a call's tokens, 2-token units measured fastest at every T up
+// to 32 (the layer at T = 8 / 16 / 32: 0.32 / 0.60 / 1.07 ms against 0.38 /
+// 0.67 / 1.16 ms with 4-token and 0.53 / 0.92 / 1.54 ms with 8-token units).
+#ifndef MOE_DECODE_UNIT_TOKENS
+#define MOE_DECODE_UNIT_TOKENS 2
+#endif
+static_assert(MOE_DECODE_UNIT_TOKENS == 2 || MOE_DECODE_UNIT_TOKENS == 4 || MOE_DECODE_UNIT_TOKENS == 8,
+              "unit width");
+static int decode_unit_tokens(int T) { return T <= 2 ? 2 : MOE_DECODE_UNIT_TOKENS; }
+
 size_t decode_scratch_bytes(const LayerDims &d, int T) {
-  DecodeScratch s;
-  decode_carve(s, d, T, nullptr);
-  return reinterpret_cast<size_t>(s.jobs) + kJobsInts * sizeof(int) + 256;
+  // the largest carve of any call with up to T tokens (the unit width, and so
+  // the number of shared token groups, depends on the call's T)
+  size_t most = 0;
+  for (int t = 1; t <= T; ++t) {
+    DecodeScratch s;
+    decode_carve(s, d, t, nullptr);
+    const size_t b = reinterpret_cast<size_t>(s.jobs) + kJobsInts * sizeof(int) + 256;
+    most = b > most ? b : most;
+  }
+  return most;
 }
 
 void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
@@ -1799,7 +1821,8 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
   s.PD = decode_kparts(d.I);
   s.PS = decode_kparts(d.Is);
   s.Jmax = T * d.k;
-  s.G = (T + kUnitMaxTok - 1) / kUnitMaxTok;
+  s.UW = decode_unit_tokens(T);
+  s.G = (T + s.UW - 1) / s.UW;
   s.TM = Imax / 16;
   s.NS = T * d.k * s.PD + T * s.PS;
   s.NSL = s.PD > s.PS ? s.PD : s.PS;
@@ -1834,12 +1857,18 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
-  if (a.T <= 2) {
-    if (k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2_tma<1, true>(a, stream, num_sms);
-    return launch_k2_tma<1, false>(a, stream, num_sms);
+  // the variant whose unit width the scratch was carved for
+  switch (a.s.UW) {
+    case 2:
+      if (a.T <= 2 && k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2_tma<1, true>(a, stream, num_sms);
+      return launch_k2_tma<1, false>(a, stream, num_sms);
+    case 4:
+      return launch_k2_tma<2, false>(a, stream, num_sms);
+    case 8:
+      return launch_k2_tma<4, false>(a, stream, num_sms);
+    default:
+      return cudaErrorInvalidValue;
   }
-  if (a.T <= 4) return launch_k2_tma<2, false>(a, stream, num_sms);
-  return launch_k2_tma<4, false>(a, stream, num_sms);
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {

@@ -9,7 +9,7 @@
 namespace moe {
 
 constexpr int kDecodeMaxT = 32;  // token counts handled by the GEMV (mma.sync) path
-constexpr int kUnitMaxTok = 8;   // tokens of one warp unit (4 MMA column pairs)
+constexpr int kUnitMaxTok = 8;   // most tokens of one warp unit (4 MMA column pairs)
 constexpr int kMaxK = 8;
 constexpr int kMaxE = 256;
 
@@ -105,8 +105,9 @@ struct DecodeScratch {
   int Imax;
   int PH, PD, PS;   // K parts of H (gate/up), I (routed down), Is (shared down)
   int NSL;          // slices per vector = max(PD, PS)
-  int Jmax;         // max routed jobs (an expert's tokens, at most kUnitMaxTok per job) = T*k
-  int G;            // token groups of the shared expert (kUnitMaxTok tokens each)
+  int UW;           // tokens per unit of this call's kernel variant (2 per MMA column pair)
+  int Jmax;         // max routed jobs (an expert's tokens, at most UW per job) = T*k
+  int G;            // token groups of the shared expert (UW tokens each)
   int TM;           // max(I, Is) / 16
   int NS;           // output slots per 16-row tile of y
   FastDiv fPH, fTIPH, fTH, fPD;  // divisors PH, (I/16)*PH, H/16, PD of the unit numbering

@@ -157,7 +157,7 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
  * allocating library routine).
  *
  * Limits: 1 <= T <= 8 tokens, and the layer's small-T scratch for T must fit
- * in 16 MiB (the V4-Flash shapes need about 11.5 MiB at T = 8); larger requests
+ * in 16 MiB (the V4-Flash shapes need about 6.2 MiB at T = 8); larger requests
  * return MOE_ERR_UNSUPPORTED_SHAPE or MOE_ERR_WORKSPACE_TOO_SMALL with a
  * message.  T = 0 is a no-op.  The current device must be the handle's
  * device.  The first call on a device looks up the buffer's device address

@@ -60,15 +60,16 @@ def test_tiny_layer_matches_oracle(moe, T):
 
 @pytest.mark.parametrize("T", [9, 16, 32])
 def test_tiny_layer_medium_token_counts(moe, T):
-    """9..32 tokens: the shared expert's tokens run in groups of 8 units' worth."""
+    """9..32 tokens: the shared expert's tokens run in token groups of one
+    unit's width, each with its own tile counters."""
     s = synth.workload("tiny", tokens=T)
     got = _run(moe, s, 0, 0, T)
     _check(s, got, 0, 0)
 
 
-def test_experts_with_more_than_eight_tokens_are_split(moe):
-    """The skewed bias sends (nearly) every token to experts 0 and 8, so their
-    jobs hold more pairs than one unit and are split."""
+def test_experts_with_more_tokens_than_a_unit_are_split(moe):
+    """The skewed bias sends (nearly) every token to experts 0 and 8, so they
+    hold more pairs than one unit takes and are split into several jobs."""
     s = synth.workload("tiny", tokens=24, skew=True)
     got = _run(moe, s, 1, 0, 24)
     counts = np.bincount(got["idx"].ravel(), minlength=s.n_experts)
@@ -106,6 +107,28 @@ def test_full_decode_eight_tokens_prenorm(moe):
     s = synth.workload("decode_t1", tokens=8)
     got = _run(moe, s, 2, 7, 8, flags=moe.MOE_FLAG_PRENORM_RESIDUAL)
     _check(s, got, 2, 7, prenorm=True)
+
+
+def test_full_decode_32_tokens_sampled(moe):
+    """V4-Flash shapes at 32 tokens with the skewed bias (the largest call of
+    the small-T kernels): routing of every token bit-exact, the output rows of
+    sampled tokens against the oracle run on those tokens alone (a token's
+    output depends only on its own input row)."""
+    s = synth.workload("decode_t32")
+    T = s.tokens
+    got = _run(moe, s, 3, 1, T)
+    Wr = synth.router_weight(3, 1, s.n_experts, s.hidden)
+    b = synth.bias(3, 1, s.n_experts, s.skew)
+    idx, w, margin = oracle.select(oracle.router_logits(got["x"].astype(np.float64), Wr), b, s.top_k,
+                                   s.routed_scaling)
+    assert np.array_equal(got["idx"], idx), margin
+    assert np.allclose(got["w"], w, rtol=1e-6, atol=1e-7)
+    assert np.bincount(idx.ravel(), minlength=s.n_experts).max() > 2  # some experts span several jobs
+    pick = np.array([0, 17, T - 1])
+    _, _, yref, _ = harness.oracle_layer(s, 3, 1, got["x"][pick], threads=4)
+    rel_l2, max_abs = harness.errors(got["y"][pick], yref)
+    assert rel_l2 <= harness.GEMV_REL_L2, rel_l2
+    assert max_abs <= harness.MAX_ABS_FRAC, max_abs
 
 
 def test_full_decode_hash_layer(moe):
