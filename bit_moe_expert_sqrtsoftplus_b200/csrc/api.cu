@@ -98,6 +98,17 @@ size_t scratch_bytes_for(const moe::LayerDims &d, int max_tokens) {
   return dec > pre ? dec : pre;
 }
 
+// The kernels run on the current device with the handle's pointers, which
+// belong to the device that was current at moe_init.
+moe_status check_device(const moe_handle *h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != h->device)
+    return fail(MOE_ERR_INVALID_ARG, "the current device (%d) is not the handle's device (%d)", dev, h->device);
+  return MOE_OK;
+}
+
 moe_status check_call(moe_handle *h, const float *x, const int32_t *token_ids, int T, void *scratch,
                       size_t scratch_bytes) {
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
@@ -111,7 +122,7 @@ moe_status check_call(moe_handle *h, const float *x, const int32_t *token_ids, i
   const size_t need = scratch_bytes_for(h->d, T);
   if (scratch_bytes < need)
     return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for T=%d", scratch_bytes, need, T);
-  return MOE_OK;
+  return check_device(h);
 }
 
 }  // namespace
@@ -326,16 +337,13 @@ moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t 
   if (h->d.mode == MOE_ROUTE_HASH && !token_ids) return fail(MOE_ERR_INVALID_ARG, "hash mode needs token_ids");
   if (y == x && !(h->d.flags & MOE_FLAG_PRENORM_RESIDUAL))
     return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev != h->device)
-    return fail(MOE_ERR_INVALID_ARG, "the current device (%d) is not the handle's device (%d)", dev, h->device);
+  moe_status st = check_device(h);
+  if (st != MOE_OK) return st;
   void *scratch = nullptr;
-  moe_status st = static_scratch_for(dev, &scratch);
+  st = static_scratch_for(h->device, &scratch);
   if (st != MOE_OK) return st;
   moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
-  e = moe::decode_forward(a, reinterpret_cast<cudaStream_t>(stream), h->num_sms);
+  const cudaError_t e = moe::decode_forward(a, reinterpret_cast<cudaStream_t>(stream), h->num_sms);
   if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward_noalloc launch");
   g_last_error.clear();
   return MOE_OK;

@@ -34,6 +34,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "layer.cuh"
 
 namespace moe {
@@ -1688,7 +1689,7 @@ size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
   if (xsmem) b += (size_t)T * 3 * (d.H + 32);
   return b;
 }
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemLimit = kSmemOptInMax;
 
 template <typename K>
 cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a) {
@@ -1707,16 +1708,12 @@ cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t 
 
 template <int MAXP, bool XSMEM, bool TMA>
 cudaError_t launch_k2(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k2_experts<MAXP, XSMEM, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static SmemOptIn opt;
+  cudaError_t e = opt_in_smem(k2_experts<MAXP, XSMEM, TMA>, kSmemLimit, opt);
+  if (e != cudaSuccess) return e;
   if (a.ev_begin) cudaEventRecord(a.ev_begin, stream);
-  cudaError_t e = launch_pdl(k2_experts<MAXP, XSMEM, TMA>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM),
-                             stream, a);
+  e = launch_pdl(k2_experts<MAXP, XSMEM, TMA>, num_sms, k2_threads(MAXP), k2_smem_bytes(a.d, a.T, XSMEM), stream,
+                 a);
   if (e != cudaSuccess) return e;
   if (a.ev_end) cudaEventRecord(a.ev_end, stream);
   return cudaSuccess;

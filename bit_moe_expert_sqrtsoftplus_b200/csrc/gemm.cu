@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -621,14 +622,10 @@ size_t grouped_gemm_smem(int paired) {
 
 template <int FMT, bool PAIRED>
 static cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
-  static bool configured = false;
+  static SmemOptIn opt;
   const size_t smem = grouped_gemm_smem(PAIRED);
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_grouped_gemm<FMT, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = opt_in_smem(k_grouped_gemm<FMT, PAIRED>, smem, opt);
+  if (e != cudaSuccess) return e;
   k_grouped_gemm<FMT, PAIRED><<<num_sms, kGemmThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "launch.cuh"
 #include "prefill.cuh"
 
 namespace moe {
@@ -496,11 +497,9 @@ cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStre
   const int nfix_items = T * ((d.E + kFixGroup - 1) / kFixGroup);
   const int nfix_blocks = nfix_items < 296 ? nfix_items : 296;
   const size_t fix_smem = sizeof(double) * (size_t)d.H;
-  static bool fix_configured = false;
-  if (!fix_configured && fix_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(k_router_fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fix_smem);
-    if (e != cudaSuccess) return e;
-    fix_configured = true;
+  if (fix_smem > 48 * 1024) {  // the x row in fp64 for H > 6144; opt in to the most any H may need
+    static SmemOptIn opt;
+    if ((e = opt_in_smem(k_router_fix, kSmemOptInMax, opt)) != cudaSuccess) return e;
   }
   k_router_fix<<<nfix_blocks, 256, fix_smem, s>>>(p.x, inv, p.wt.Wr, p.wt.bias, T, d.E, d.H, d.k, d.scaling,
                                                   p.s.fix, z, idx, w);

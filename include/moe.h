@@ -29,6 +29,9 @@
  *     caller's `persist` buffer, per-call temporaries in `scratch`.
  *   - Every call is asynchronous on the given stream and never synchronises
  *     the host, except moe_poll_device_error.
+ *   - A handle belongs to the device that is current at moe_init; moe_route
+ *     and the forward calls return MOE_ERR_INVALID_ARG when another device
+ *     is current.
  *   - Argument and shape errors are returned synchronously as a negative
  *     moe_status and described by moe_last_error() (thread-local).  No C++
  *     exception crosses this boundary.  Device-side problems (a bounded wait
