@@ -77,6 +77,18 @@ def test_workspace_size_and_shape_checks(moe):
         assert moe.moe_last_error()
 
 
+def test_scratch_size_never_shrinks_with_more_tokens(moe):
+    """A scratch buffer sized for max_tokens serves every call with fewer
+    tokens, so the size must not decrease as max_tokens grows (the small-T
+    layout changes with the unit width, the large-T one starts above 32)."""
+    for shape in (dict(), dict(hidden=256, inter=256, n_experts=16, top_k=2, shared_inter=256)):
+        prev = 0
+        for T in list(range(1, 70)) + [128, 4096]:
+            _, s = moe.moe_workspace_size(_cfg(moe, **shape), T)
+            assert s >= prev, (shape, T, s, prev)
+            prev = s
+
+
 def _fake_weights(moe, base=0x10000000, step=0x1000000, misalign=None, null=None):
     names = [f for f, _ in moe.moe_weights._fields_]
     vals = {}
