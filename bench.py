@@ -160,21 +160,32 @@ def dist_setup(args):
 
 
 def barrier(world):
+    """All ranks meet, then this rank's device work drains (on CPU-only
+    process groups, as in the gloo tests, only the meeting)."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(world, value: float) -> float:
+    """The largest of every rank's value (device timings: the slowest rank)."""
     import torch
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, steps: int, tokens_per_step: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` steps of `tokens_per_step`
+    tokens (weak scaling), timed as the slowest rank's `ms_max`."""
+    return world * steps * tokens_per_step / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------- workloads
@@ -288,8 +299,8 @@ def run_ours(args, world, rank):
     e2e_ms = max_over_ranks(world, e2e_ms)
     k2_ms = max_over_ranks(world, k2_ms)
     ms_step = ms / args.steps
-    value = world * args.steps * T / (ms / 1e3)
-    e2e_value = world * args.steps * T / (e2e_ms / 1e3)
+    value = job_throughput(world, args.steps, T, ms)
+    e2e_value = job_throughput(world, args.steps, T, e2e_ms)
     peaks = load_peaks()
     b = decode_bytes(s, n_distinct)
     achieved = b["k2_experts"] / (k2_ms / 1e3) / 1e9
@@ -418,7 +429,7 @@ def run_stack(args, world, rank):
     ms_step = ms / args.steps
     gbs = nd_bytes / (ms_step / 1e3) / 1e9
     return {
-        "metric": METRIC, "value": world * args.steps * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": job_throughput(world, args.steps, T, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "us_per_layer": ms_step * 1e3 / s.layers, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "s8xs8->s32 tensor-core products, fp32 scaling",
@@ -431,7 +442,7 @@ def run_stack(args, world, rank):
         "roofline": {"bound": "hbm", "kernel": "whole stack step (43 x k1/k2)", "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": peaks["source"], "algorithmic_bytes_per_step": nd_bytes},
-        "e2e": {"value": world * args.steps * T / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * s.hidden * 4, "d2h_bytes_per_step": T * s.hidden * 4},
         "gpu_launches": 2 * s.layers * args.steps,
         "clocks": clock.summary(),
