@@ -8,15 +8,17 @@
 //                   counter: every (16-row tile, 1024-element K part) of the
 //                   shared and the routed gate/up matrices, then every
 //                   (K part, 16-row output tile) of the shared and the routed
-//                   down matrices.  Packed rows are staged into shared memory
-//                   with cp.async, decoded in registers into int8 A fragments
-//                   and multiplied with mma.sync m16n8k32 against the int8
-//                   limbs of the activations.  The warp that completes a
-//                   gate/up tile applies the SwiGLU; the warp that completes a
-//                   1024-element slice of h quantises it into limbs and flags
-//                   it, and down units wait for the slices they read.  The
-//                   warp that completes an output tile sums its parts in a
-//                   fixed order (deterministic) into y.
+//                   down matrices, for the tokens of one job (2 per unit by
+//                   default: one MMA column pair).  Packed rows are staged
+//                   into shared memory by TMA tensor copies (cp.async where
+//                   the row stride rules TMA out), decoded in registers into
+//                   int8 A fragments and multiplied with mma.sync m16n8k32
+//                   against the int8 limbs of the activations.  The warp that
+//                   completes a gate/up tile applies the SwiGLU; the warp that
+//                   completes a 1024-element slice of h quantises it into
+//                   limbs and flags it, and down units wait for the slices
+//                   they read.  The warp that completes an output tile sums
+//                   its parts in a fixed order (deterministic) into y.
 // k2 is launched as a programmatic dependent of k1: its set-up (tables,
 // shared memory) overlaps k1, and griddepcontrol.wait guards every read of
 // k1's results.
