@@ -64,6 +64,11 @@ def lib():
         L.oracle_layer_mt.restype = i32
         L.oracle_permutation.argtypes = [vp, i32, i32, i32, vp, vp]
         L.oracle_rmsnorm.argtypes = [vp, i32, d, vp]
+        L.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_f16.restype = ctypes.c_uint16
+        for name in ("oracle_quantize_q80", "oracle_quantize_q2k"):
+            getattr(L, name).argtypes = [vp, i32, vp]
+            getattr(L, name).restype = i32
         _lib = L
     return _lib
 
@@ -256,4 +261,28 @@ def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     out = np.empty_like(xx)
     for t in range(xx.shape[0]):
         lib().oracle_rmsnorm(xx[t].ctypes.data, xx.shape[1], float(eps), out[t].ctypes.data)
+    return out
+
+
+# -------------------------------------------------------------------- encoders
+
+def f32_to_f16(f: float) -> int:
+    """Bits of the nearest binary16 (ties to even) of the binary32 value f."""
+    return int(lib().oracle_f32_to_f16(float(np.float32(f))))
+
+
+def quantize(kind: int, x: np.ndarray) -> np.ndarray:
+    """Encode fp32 values (a multiple of the block size) into Q8_0 or Q2_K
+    blocks: uint8 [n_blocks][block_bytes].  Raises on non-finite input."""
+    if kind not in (KIND_Q80, KIND_Q2K):
+        raise ValueError("only the Q8_0 and Q2_K encoders exist")
+    xx, px = _c(np.asarray(x, dtype=np.float32).ravel(), np.float32)
+    n = xx.size
+    if n % _BE[kind]:
+        raise ValueError(f"{n} values is not a multiple of {_BE[kind]}")
+    out = np.zeros((n // _BE[kind], _BB[kind]), dtype=np.uint8)
+    fn = lib().oracle_quantize_q80 if kind == KIND_Q80 else lib().oracle_quantize_q2k
+    rc = fn(px, n, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("non-finite input" if rc == -1 else f"encoder error {rc}")
     return out

@@ -404,3 +404,125 @@ void oracle_rmsnorm(const double *x, int H, double eps, double *out) {
   double inv = 1.0 / sqrt(ss / (double)H + eps);
   for (int c = 0; c < H; ++c) out[c] = x[c] * inv;
 }
+
+/* ------------------------------------------------------------- encoders */
+/*
+ * The encoder side of the two scalar block formats.  [QUANT] section 3: the
+ * Q2_K writer estimates a scale and a min for every 16-element sub-block,
+ * rounds each value to a 2-bit code 0..3 and packs four codes per byte with
+ * the printed expression (code of element e at byte 32*(e/128) + e%32, shift
+ * 2*((e%128)/32)); d at byte 80 and dmin at 82 are the f16 bases of the
+ * sub-block scale and min nibbles.  [FLOW] "Dwarf Star の量子化の工夫": Q8_0
+ * keeps one symmetric scale per 32 elements.
+ *
+ * Readings (the pages give neither the estimator nor a precision): plain
+ * min/max estimation; every decision in IEEE binary32 with round-to-nearest-
+ * even, in the order written below (the arithmetic a device encoder uses, so
+ * both take each integer decision in the same precision); the f16 bases are
+ * the nearest binary16 values; a block holding a non-finite value is an
+ * error.  The decoded value is the one the decoders above compute:
+ * Q8_0 d*q, Q2_K d*sc*q - dmin*m.
+ */
+
+/* Nearest IEEE binary16 (ties to even) of a binary32 value, from the format's
+ * definition: 10 fraction bits, exponent bias 15, subnormal quantum 2^-24,
+ * values at or above 65520 (the midpoint past 65504) go to infinity. */
+uint16_t oracle_f32_to_f16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  const float a = fabsf(f);
+  if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+  if (a >= 65520.0f) return (uint16_t)(sign | 0x7c00u);
+  if (a == 0.0f) return sign;
+  int e;
+  frexp((double)a, &e); /* a = m 2^e, m in [0.5, 1): the binade's exponent is e - 1 */
+  int ex = e - 1;
+  if (ex < -14) ex = -14;                     /* subnormal binade: quantum 2^-24 */
+  const double quantum = ldexp(1.0, ex - 10); /* spacing of binary16 values there */
+  const double r = nearbyint((double)a / quantum); /* exact quotient; ties to even */
+  uint32_t bits;
+  if (ex == -14 && r < 1024.0) {
+    bits = (uint32_t)r; /* subnormal */
+  } else {
+    double m = r;
+    if (m >= 2048.0) { /* rounded up into the next binade */
+      m = 1024.0;
+      ex += 1;
+    }
+    bits = ((uint32_t)(ex + 15) << 10) | ((uint32_t)m - 1024u);
+  }
+  return (uint16_t)(sign | bits);
+}
+
+static void put16(uint8_t *p, uint16_t v) {
+  p[0] = (uint8_t)(v & 0xff);
+  p[1] = (uint8_t)(v >> 8);
+}
+
+static float clampf(float v, float lo, float hi) { return v < lo ? lo : v > hi ? hi : v; }
+
+int oracle_quantize_q80(const float *x, int n, uint8_t *out) {
+  if (n < 0 || n % 32) return -2;
+  for (int b = 0; b < n / 32; ++b) {
+    const float *v = x + (size_t)b * 32;
+    uint8_t *blk = out + (size_t)b * 34;
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+      if (!isfinite(v[i])) return -1;
+      if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+    }
+    const float d = amax / 127.0f;
+    const uint16_t dh = oracle_f32_to_f16(d);
+    const float dq = (float)oracle_f16(dh);
+    put16(blk, dh);
+    for (int i = 0; i < 32; ++i) {
+      float q = 0.0f;
+      if (dq > 0.0f) q = clampf(rintf(v[i] / dq), -127.0f, 127.0f);
+      blk[2 + i] = (uint8_t)(int8_t)q;
+    }
+  }
+  return 0;
+}
+
+int oracle_quantize_q2k(const float *x, int n, uint8_t *out) {
+  if (n < 0 || n % 256) return -2;
+  for (int b = 0; b < n / 256; ++b) {
+    const float *v = x + (size_t)b * 256;
+    uint8_t *blk = out + (size_t)b * 84;
+    memset(blk, 0, 84);
+    float scale[16], mn[16], maxs = 0.0f, maxm = 0.0f;
+    for (int j = 0; j < 16; ++j) {
+      /* the sub-block's range, widened to include 0 below: the min term
+       * -dmin*m is never positive */
+      float lo = 0.0f, hi = -INFINITY;
+      for (int i = 0; i < 16; ++i) {
+        const float t = v[16 * j + i];
+        if (!isfinite(t)) return -1;
+        if (t < lo) lo = t;
+        if (t > hi) hi = t;
+      }
+      scale[j] = (hi - lo) / 3.0f; /* four codes span the range */
+      mn[j] = 0.0f - lo;
+      if (scale[j] > maxs) maxs = scale[j];
+      if (mn[j] > maxm) maxm = mn[j];
+    }
+    const uint16_t dh = oracle_f32_to_f16(maxs / 15.0f), mh = oracle_f32_to_f16(maxm / 15.0f);
+    const float dq = (float)oracle_f16(dh), mq = (float)oracle_f16(mh);
+    put16(blk + 80, dh);
+    put16(blk + 82, mh);
+    for (int j = 0; j < 16; ++j) {
+      const float sc = dq > 0.0f ? clampf(rintf(scale[j] / dq), 0.0f, 15.0f) : 0.0f;
+      const float m = mq > 0.0f ? clampf(rintf(mn[j] / mq), 0.0f, 15.0f) : 0.0f;
+      blk[j] = (uint8_t)((int)sc | ((int)m << 4));
+      const float step = dq * sc, off = mq * m;
+      for (int i = 0; i < 16; ++i) {
+        const int e = 16 * j + i;
+        float q = 0.0f;
+        if (step > 0.0f) q = clampf(rintf((v[e] + off) / step), 0.0f, 3.0f);
+        blk[16 + 32 * (e / 128) + e % 32] |= (uint8_t)((int)q << (2 * ((e % 128) / 32)));
+      }
+    }
+  }
+  return 0;
+}
