@@ -8,7 +8,10 @@ weight sets (8 x 1.84 GB, far beyond the 126 MB L2) after warm-up calls.
 A step is one layer call.  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8]
+                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|quantize_q2k|quantize_q80]
+
+quantize_q2k / quantize_q80 time the offline encoder (moe_quantize) on
+8 x 2048 x 4096 fp32 values per step, in values/s against the HBM roofline.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on
 its own GPU with no exchange (replicas; the layer has no data-path
@@ -45,7 +48,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_t1",
-                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8"])
+                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "quantize_q2k",
+                            "quantize_q80"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
@@ -535,10 +539,116 @@ class OracleSampler:
         return self.T / self.F
 
 
+# ------------------------------------------------------- offline encoders
+
+QUANT_ROWS, QUANT_COLS, QUANT_MATS = 2048, 4096, 8  # eight gate-projection-sized matrices per step
+QUANT_METRIC = "encoded values/s (offline Q2_K / Q8_0 encoder) and % HBM roofline"
+
+
+def quant_format(workload: str):
+    """(binary format id, values per block, bytes per block) of an encoder workload."""
+    return (1, 256, 84) if workload == "quantize_q2k" else (0, 32, 34)
+
+
+def run_quant(args, world, rank):
+    """moe_quantize over 8 x 2048 x 4096 fp32 values (268 MB, beyond the
+    126 MB L2) per step; HBM roofline on 4 bytes read plus the block bytes
+    written per value."""
+    import torch
+
+    import bit_moe_expert_sqrtsoftplus_b200 as moe
+
+    fmt, per, nbytes = quant_format(args.workload)
+    n = QUANT_ROWS * QUANT_COLS * QUANT_MATS
+    gen = torch.Generator(device="cuda").manual_seed(7 + rank)
+    x = torch.randn(n, device="cuda", generator=gen) * 0.02
+    out = torch.empty(n // per * nbytes, dtype=torch.uint8, device="cuda")
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(args.warmup):
+        moe.moe_quantize(fmt, x, out, bad)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    clock = ClockSampler(torch.cuda.current_device())
+    with clock:
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            moe.moe_quantize(fmt, x, out, bad)
+        e1.record(stream)
+        barrier(world)
+        ms = e0.elapsed_time(e1)
+        # end to end: pinned host values -> device -> encoder -> pinned host blocks
+        hx = x.cpu().pin_memory()
+        hy = torch.empty_like(out, device="cpu").pin_memory()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            x.copy_(hx, non_blocking=True)
+            moe.moe_quantize(fmt, x, out, bad)
+            hy.copy_(out, non_blocking=True)
+        f1.record(stream)
+        barrier(world)
+        e2e_ms = f0.elapsed_time(f1)
+    if int(bad.item()) != 0:
+        raise RuntimeError("the encoder counted non-finite blocks in finite input")
+    ms = max_over_ranks(world, ms)
+    e2e_ms = max_over_ranks(world, e2e_ms)
+    peaks = load_peaks()
+    ms_launch = ms / args.steps
+    bytes_launch = n * 4 + n // per * nbytes
+    gbs = bytes_launch / (ms_launch / 1e3) / 1e9
+    return {
+        "metric": QUANT_METRIC, "value": job_throughput(world, args.steps, n, ms), "unit": "values/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_launch,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> binary32 decisions",
+        "data": "synthetic (N(0, 0.02^2) fp32 values from torch's generator)",
+        "config": {"workload": f"{args.workload}: {QUANT_MATS} x {QUANT_ROWS} x {QUANT_COLS} fp32 values per step "
+                               f"-> {'Q2_K' if per == 256 else 'Q8_0'} blocks",
+                   "l2": f"{n * 4 / 1e6:.0f} MB of input per step, beyond the 126 MB L2",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": f"k_quantize_{'q2k' if per == 256 else 'q80'}", "achieved": gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": load_traffic(args.workload), "traffic_unit": "bytes per launch (ncu)",
+                     "peak_source": peaks["source"], "algorithmic_bytes_per_launch": bytes_launch,
+                     "ms_per_launch": ms_launch},
+        "e2e": {"value": job_throughput(world, args.steps, n, e2e_ms), "unit": "values/s",
+                "h2d_bytes_per_step": n * 4, "d2h_bytes_per_step": n // per * nbytes},
+        "gpu_launches": args.steps,
+        "clocks": clock.summary(),
+    }
+
+
+def oracle_quant_rate(workload: str, steps: int, warmup: int, values_per_step: int = 1 << 20):
+    """Values/s of the oracle's encoder on steps of 2^20 values."""
+    import oracle
+    fmt, per, _ = quant_format(workload)
+    kind = oracle.KIND_Q2K if per == 256 else oracle.KIND_Q80
+    x = (np.random.default_rng(7).standard_normal(values_per_step) * 0.02).astype(np.float32)
+    for _ in range(warmup):
+        oracle.quantize(kind, x)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.quantize(kind, x)
+    elapsed = time.perf_counter() - t0
+    return steps * values_per_step / elapsed, elapsed
+
+
 def run_reference(args, world, rank):
-    s = synth.workload(args.workload)
     if rank != 0:
         return None
+    if args.workload.startswith("quantize_"):
+        value, elapsed = oracle_quant_rate(args.workload, args.steps, args.warmup)
+        sample = (f"{args.steps} steps of 2^20 values through the C oracle's encoder, single thread, "
+                  f"{elapsed:.2f} s after {args.warmup} warm-up steps")
+        return {"metric": QUANT_METRIC, "value": value, "unit": "values/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> binary32 decisions", "data": "synthetic",
+                "impl": "reference", "config": {"workload": f"{args.workload} (2^20 values per step)"},
+                "cpu_baseline": {"value": value, "unit": "values/s", "cores": 1, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": "values/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    s = synth.workload(args.workload)
     smp = OracleSampler(s)
     for _ in range(args.warmup):
         smp.step()
@@ -564,6 +674,20 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def cpu_baseline(args) -> dict:
+    """The oracle on a bounded sample of the workload, on one host core."""
+    if args.workload.startswith("quantize_"):
+        steps = max(1, int(args.cpu_seconds / 0.005))  # about 5 ms per 2^20 values
+        value, elapsed = oracle_quant_rate(args.workload, steps, 3)
+        return {"value": value, "unit": "values/s", "cores": 1, "kind": "oracle",
+                "sample": f"{steps} x 2^20 values through the C oracle's encoder, single thread, {elapsed:.1f} s"}
+    s = synth.workload(args.workload)
+    value, n, elapsed = oracle_rate(s, args.cpu_seconds, 1000)
+    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} full layer calls (T={s.tokens}) of the fp64 C oracle on weight set 0, "
+                      f"single thread, {elapsed:.1f} s"}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -574,13 +698,14 @@ def main():
             print(json.dumps(out), flush=True)
         return
     world, rank, local = dist_setup(args)
-    out = run_stack(args, world, rank) if args.workload == "stack43_t8" else run_ours(args, world, rank)
+    if args.workload.startswith("quantize_"):
+        out = run_quant(args, world, rank)
+    elif args.workload == "stack43_t8":
+        out = run_stack(args, world, rank)
+    else:
+        out = run_ours(args, world, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s = synth.workload(args.workload)
-        value, n, elapsed = oracle_rate(s, args.cpu_seconds, 1000)
-        out["cpu_baseline"] = {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                               "sample": f"{n} full layer calls (T={s.tokens}) of the fp64 C oracle on weight set 0, "
-                                         f"single thread, {elapsed:.1f} s"}
+        out["cpu_baseline"] = cpu_baseline(args)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -29,9 +29,11 @@ MOE_ROUTE_ROUTER = 0
 MOE_ROUTE_HASH = 1
 MOE_FLAG_PRENORM_RESIDUAL = 1
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
+MOE_QUANT_Q8_0 = 0
+MOE_QUANT_Q2_K = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
-            "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_destroy")
+            "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_quantize", "moe_destroy")
 
 
 class moe_config(ctypes.Structure):
@@ -76,6 +78,8 @@ def lib():
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_set_timing_events.argtypes = [vp, vp, vp]
         L.moe_set_timing_events.restype = i32
+        L.moe_quantize.argtypes = [i32, vp, ctypes.c_int64, vp, vp, vp]
+        L.moe_quantize.restype = i32
         L.moe_destroy.argtypes = [vp]
         L.moe_destroy.restype = None
         for name in ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error"):
@@ -151,6 +155,27 @@ def moe_set_timing_events(handle, ev_begin=None, ev_end=None):
     """ev_begin / ev_end: torch.cuda.Event objects (or None to stop)."""
     _check(lib().moe_set_timing_events(handle, None if ev_begin is None else ev_begin.cuda_event,
                                        None if ev_end is None else ev_end.cuda_event))
+
+
+def moe_quantize(fmt, x, out, nonfinite=None, stream=None):
+    """Encode the fp32 CUDA tensor x (numel a multiple of the block size) into
+    the uint8 CUDA tensor out (numel/32 * 34 or numel/256 * 84 bytes)."""
+    per, nbytes = (32, 34) if fmt == MOE_QUANT_Q8_0 else (256, 84)
+    if out.numel() * out.element_size() < x.numel() // per * nbytes:
+        raise MoeError(MOE_ERR_WORKSPACE_TOO_SMALL, "out is too small for the encoded blocks")
+    _check(lib().moe_quantize(fmt, _ptr(x), x.numel(), _ptr(out), _ptr(nonfinite), _stream(stream)))
+
+
+def quantize(fmt, x, stream=None):
+    """Encoded blocks of x as a uint8 CUDA tensor [n_blocks][block_bytes] and a
+    device int32 count of blocks that held a non-finite value."""
+    import torch
+    per, nbytes = (32, 34) if fmt == MOE_QUANT_Q8_0 else (256, 84)
+    x = x.contiguous()
+    out = torch.empty((x.numel() // per, nbytes), dtype=torch.uint8, device=x.device)
+    bad = torch.zeros(1, dtype=torch.int32, device=x.device)
+    moe_quantize(fmt, x, out, bad, stream)
+    return out, bad
 
 
 def moe_destroy(handle):

@@ -12,6 +12,7 @@
 #include "../../include/moe.h"
 #include "layer.cuh"
 #include "prefill.cuh"
+#include "quant.cuh"
 
 static_assert(MOE_SMALL_T_MAX == moe::kDecodeMaxT, "header and kernels disagree on the small-T limit");
 
@@ -382,6 +383,31 @@ moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end) {
     return fail(MOE_ERR_INVALID_ARG, "ev_begin and ev_end must both be set or both be NULL");
   h->ev_begin = static_cast<cudaEvent_t>(ev_begin);
   h->ev_end = static_cast<cudaEvent_t>(ev_end);
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_quantize(int format, const float *x, int64_t n, void *out, int32_t *nonfinite_blocks,
+                        moe_stream_t stream) {
+  if (format != MOE_QUANT_Q8_0 && format != MOE_QUANT_Q2_K)
+    return fail(MOE_ERR_INVALID_ARG, "format=%d is not a MOE_QUANT_* format", format);
+  if (n < 0) return fail(MOE_ERR_INVALID_ARG, "n=%lld is negative", (long long)n);
+  const int per = format == MOE_QUANT_Q8_0 ? 32 : 256;
+  if (n % per)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n=%lld is not a multiple of the block size %d", (long long)n, per);
+  if (n == 0) {
+    g_last_error.clear();
+    return MOE_OK;
+  }
+  if (!x || !out) return fail(MOE_ERR_INVALID_ARG, "x and out must not be NULL");
+  if (!aligned16(x) || !aligned16(out)) return fail(MOE_ERR_MISALIGNED, "x and out must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  e = moe::quantize_blocks(format, x, n / per, out, nonfinite_blocks, reinterpret_cast<cudaStream_t>(stream), sms);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_quantize launch");
   g_last_error.clear();
   return MOE_OK;
 }

@@ -70,6 +70,10 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 
 #define MOE_SMALL_T_MAX 32 /* largest T served by the small-token kernels */
 
+/* block formats of moe_quantize */
+#define MOE_QUANT_Q8_0 0 /* 32 values in 34 bytes */
+#define MOE_QUANT_Q2_K 1 /* 256 values in 84 bytes */
+
 typedef struct {
   int hidden;           /* H: multiple of 256 (4096 for V4-Flash) */
   int inter;            /* I: routed expert intermediate, multiple of 256 (2048) */
@@ -191,6 +195,24 @@ const char *moe_last_error(void);
  * stop recording.  Recording changes no work the layer does.
  */
 moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end);
+
+/*
+ * Offline encoder: n fp32 values -> blocks of `format` (MOE_QUANT_Q8_0: n a
+ * multiple of 32, n/32 blocks of 34 bytes; MOE_QUANT_Q2_K: n a multiple of
+ * 256, n/256 blocks of 84 bytes), the writer side of the formats the layer
+ * reads ("2bit 量子化はなぜ「冗談ではない」のか", section 3: per 16-element
+ * sub-block a scale and a min, codes 0..3, the page's packing; "DeepSeek-V4-
+ * Flash one-token computation flow", section "Dwarf Star の量子化の工夫": Q8_0
+ * has one symmetric scale per 32 values).  The estimator is plain min/max with
+ * every decision in IEEE binary32, round to nearest even; the steps are listed
+ * in csrc/quant.cu.  x and out are device pointers, 16-byte aligned; a matrix
+ * of rows whose length is a multiple of the block size is encoded row after
+ * row by passing it whole.  nonfinite_blocks (device int32, may be NULL) is
+ * incremented once per block that holds a NaN or an infinity; such blocks are
+ * written as zeros.  Asynchronous on `stream`; n = 0 is a no-op.
+ */
+moe_status moe_quantize(int format, const float *x, int64_t n, void *out, int32_t *nonfinite_blocks,
+                        moe_stream_t stream);
 
 /* Frees the host-side handle (the caller frees `persist`). NULL is a no-op. */
 void moe_destroy(moe_handle *h);

@@ -89,6 +89,24 @@ def test_scratch_size_never_shrinks_with_more_tokens(moe):
             prev = s
 
 
+def test_quantize_argument_checks(moe):
+    """moe_quantize rejects bad arguments before it touches a device."""
+    L = moe.lib()
+    ok = 0x20000000
+    cases = [((7, ok, 256, ok), moe.MOE_ERR_INVALID_ARG),
+             ((moe.MOE_QUANT_Q2_K, ok, -256, ok), moe.MOE_ERR_INVALID_ARG),
+             ((moe.MOE_QUANT_Q2_K, ok, 300, ok), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+             ((moe.MOE_QUANT_Q8_0, ok, 48, ok), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+             ((moe.MOE_QUANT_Q8_0, None, 64, ok), moe.MOE_ERR_INVALID_ARG),
+             ((moe.MOE_QUANT_Q2_K, ok, 256, None), moe.MOE_ERR_INVALID_ARG),
+             ((moe.MOE_QUANT_Q2_K, ok + 4, 256, ok), moe.MOE_ERR_MISALIGNED),
+             ((moe.MOE_QUANT_Q8_0, ok, 32, ok + 2), moe.MOE_ERR_MISALIGNED)]
+    for (fmt, x, n, out), status in cases:
+        assert L.moe_quantize(fmt, x, n, out, None, None) == status, (fmt, x, n, out)
+        assert moe.moe_last_error()
+    assert L.moe_quantize(moe.MOE_QUANT_Q2_K, None, 0, None, None, None) == moe.MOE_OK  # n = 0: no-op
+
+
 def _fake_weights(moe, base=0x10000000, step=0x1000000, misalign=None, null=None):
     names = [f for f, _ in moe.moe_weights._fields_]
     vals = {}
