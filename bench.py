@@ -53,6 +53,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
+    p.add_argument("--sweep", action="store_true",
+                   help="time one layer call at T = 1, 2, 4, ..., 256 (skewed bias; one JSON line per T)")
     return p.parse_args()
 
 
@@ -674,6 +676,53 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 128, 256)
+
+
+def run_sweep(args, world, rank):
+    """Latency and bandwidth of one layer call against the union of the
+    experts its tokens select: V4-Flash shapes with the skewed bias, one
+    weight set, T = 1 ... 256 (the small-token path up to 32, the batched path
+    above).  Bytes per call = distinct experts x 7,077,888 + the shared expert
+    + the router, the least a call must read."""
+    import torch
+
+    import bit_moe_expert_sqrtsoftplus_b200 as moe
+
+    base = synth.workload("decode_t32")
+    W = synth.device_layer(0, 0, base)
+    cfg = moe.make_config(base.hidden, base.inter, base.n_experts, base.top_k, base.shared_inter,
+                          vocab=base.vocab, routed_scaling=base.routed_scaling)
+    peaks = load_peaks()
+    lines = []
+    for T in SWEEP_T:
+        L = moe.Layer(cfg, W, max_tokens=T)
+        xs = [torch.from_numpy(synth.activations(7 + rank, T, base.hidden, stream=600 + j)).cuda() for j in range(8)]
+        ys = [torch.empty_like(x) for x in xs]
+        nd = float(np.mean([len(np.unique(L.route(x)[0].cpu().numpy())) for x in xs]))
+        for i in range(max(args.warmup, 3)):
+            L.forward(xs[i % 8], None, ys[i % 8])
+        steps = max(5, min(args.steps, 200))
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            L.forward(xs[i % 8], None, ys[i % 8])
+        e1.record()
+        barrier(world)
+        L.poll()
+        ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
+        nbytes = nd * base.expert_bytes + base.shared_bytes + base.n_experts * base.hidden * 2
+        gbs = nbytes / (ms / 1e3) / 1e9
+        lines.append({"sweep_T": T, "path": "small-token" if T <= moe.MOE_SMALL_T_MAX else "batched",
+                      "ms_per_call": ms, "tokens_per_s": job_throughput(world, 1, T, ms),
+                      "distinct_experts": nd, "bytes_per_call": nbytes, "achieved_gbs": gbs,
+                      "hbm_frac": gbs / peaks["hbm_gbs"], "floor_ms": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                      "n_gpus": world, "steps": steps})
+        del L
+    return lines
+
+
 def cpu_baseline(args) -> dict:
     """The oracle on a bounded sample of the workload, on one host core."""
     if args.workload.startswith("quantize_"):
@@ -698,6 +747,14 @@ def main():
             print(json.dumps(out), flush=True)
         return
     world, rank, local = dist_setup(args)
+    if args.sweep:
+        for line in run_sweep(args, world, rank):
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if args.workload.startswith("quantize_"):
         out = run_quant(args, world, rank)
     elif args.workload == "stack43_t8":
