@@ -19,9 +19,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "_oracle.so")
 _lib = None
 
-KIND_IQ2XXS, KIND_Q2K, KIND_Q80 = 0, 1, 2
-_BB = {0: 66, 1: 84, 2: 34}
-_BE = {0: 256, 1: 256, 2: 32}
+KIND_IQ2XXS, KIND_Q2K, KIND_Q80, KIND_Q4K = 0, 1, 2, 3
+_BB = {0: 66, 1: 84, 2: 34, 3: 144}
+_BE = {0: 256, 1: 256, 2: 32, 3: 256}
 
 
 def build() -> None:
@@ -43,12 +43,13 @@ def lib():
         for name in ("oracle_iq2xxs_elem",):
             getattr(L, name).argtypes = [vp, vp, i32]
             getattr(L, name).restype = d
-        for name in ("oracle_q2k_elem", "oracle_q80_elem"):
+        for name in ("oracle_q2k_elem", "oracle_q80_elem", "oracle_q4k_elem"):
             getattr(L, name).argtypes = [vp, i32]
             getattr(L, name).restype = d
         L.oracle_row_iq2xxs.argtypes = [vp, i32, vp, vp]
         L.oracle_row_q2k.argtypes = [vp, i32, vp]
         L.oracle_row_q80.argtypes = [vp, i32, vp]
+        L.oracle_row_q4k.argtypes = [vp, i32, vp]
         L.oracle_matvec.argtypes = [i32, vp, i32, i32, vp, vp, vp]
         L.oracle_sqrtsoftplus.argtypes = [d]
         L.oracle_sqrtsoftplus.restype = d
@@ -100,6 +101,11 @@ def q80_elem(block: np.ndarray, e: int) -> float:
     return lib().oracle_q80_elem(pb, int(e))
 
 
+def q4k_elem(block: np.ndarray, e: int) -> float:
+    b, pb = _c(block, np.uint8)
+    return lib().oracle_q4k_elem(pb, int(e))
+
+
 def decode_row(kind: int, row: np.ndarray, cols: int, grid: np.ndarray | None = None) -> np.ndarray:
     r, pr = _c(row, np.uint8)
     out = np.empty(cols, dtype=np.float64)
@@ -108,6 +114,8 @@ def decode_row(kind: int, row: np.ndarray, cols: int, grid: np.ndarray | None = 
         lib().oracle_row_iq2xxs(pr, cols, pg, out.ctypes.data)
     elif kind == KIND_Q2K:
         lib().oracle_row_q2k(pr, cols, out.ctypes.data)
+    elif kind == KIND_Q4K:
+        lib().oracle_row_q4k(pr, cols, out.ctypes.data)
     else:
         lib().oracle_row_q80(pr, cols, out.ctypes.data)
     return out
@@ -181,7 +189,8 @@ class _LayerW(ctypes.Structure):
                 ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("gate", ctypes.POINTER(ctypes.c_void_p)), ("up", ctypes.POINTER(ctypes.c_void_p)),
                 ("down", ctypes.POINTER(ctypes.c_void_p)), ("sh_gate", ctypes.c_void_p),
-                ("sh_up", ctypes.c_void_p), ("sh_down", ctypes.c_void_p), ("grid", ctypes.c_void_p)]
+                ("sh_up", ctypes.c_void_p), ("sh_down", ctypes.c_void_p), ("grid", ctypes.c_void_p),
+                ("gate_kind", ctypes.c_int), ("down_kind", ctypes.c_int)]
 
 
 def _expert_ptrs(src, E, keep):
@@ -217,7 +226,9 @@ def swiglu_expert(gate, up, down, hidden, inter, x, grid=None, gate_kind=KIND_IQ
 
 def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray, threads: int = 1) -> np.ndarray:
     """y [T][H] fp64 for the given routing.  ``weights`` as returned by
-    ``synth.host_layer`` (routed tensors as full arrays or dicts by id)."""
+    ``synth.host_layer`` (routed tensors as full arrays or dicts by id;
+    optional "gate_kind" / "down_kind" name the routed formats, IQ2_XXS and
+    Q2_K when absent)."""
     keep = []
     E = shape.n_experts
     lw = _LayerW()
@@ -229,6 +240,9 @@ def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray, t
     lw.gate = ctypes.cast(garr, ctypes.POINTER(ctypes.c_void_p))
     lw.up = ctypes.cast(uarr, ctypes.POINTER(ctypes.c_void_p))
     lw.down = ctypes.cast(darr, ctypes.POINTER(ctypes.c_void_p))
+    # routed formats: the q2 build by default, Q4_K for the q2-q4 layers
+    lw.gate_kind = int(weights.get("gate_kind", KIND_IQ2XXS))
+    lw.down_kind = int(weights.get("down_kind", KIND_Q2K))
     for name in ("sh_gate", "sh_up", "sh_down", "grid"):
         a = np.ascontiguousarray(weights[name], dtype=np.uint8)
         keep.append(a)

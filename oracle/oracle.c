@@ -122,6 +122,50 @@ void oracle_row_q80(const uint8_t *row, int cols, double *out) {
   for (int c = 0; c < cols; ++c) out[c] = oracle_q80_elem(row + (size_t)(c / 32) * 34, c % 32);
 }
 
+/* ----------------------------------------------------------------- Q4_K */
+/*
+ * [QUANT] section 3 type table: q4_K holds 256 values in 144 bytes; [FLOW]
+ * format paragraph: like Q2_K it is affine with a scale and a min per
+ * sub-block (w = d*q + m roughly); [FLOW] bit-width table after "パラメータは
+ * どこにあるか: 層別の内訳": about 4.5 bpw.  144 = 2 + 2 + 12 + 128 fits two f16
+ * bases, eight 6-bit scales and eight 6-bit mins (8 sub-blocks of 32) and 256
+ * 4-bit codes.
+ *
+ * Reading (the pages print no layout; this is the public GGUF Q4_K block, so
+ * that real files decode unchanged; parity unpinned against real files):
+ * bytes 0-1 d, bytes 2-3 dmin, bytes 4-15 the scales and mins, bytes 16-143
+ * the codes.  Sub-block j < 4: scale = low 6 bits of scale byte j, min = low
+ * 6 bits of scale byte j+4.  Sub-block j >= 4: scale = low nibble of scale
+ * byte j+4 with the top two bits of scale byte j-4 above it, min = high
+ * nibble of scale byte j+4 with the top two bits of scale byte j above it.
+ * Element e lies in sub-block e/32; its code is in code byte 32*(e/64) + e%32,
+ * low nibble for e%64 < 32 and high nibble otherwise (the two-codes-per-byte
+ * form of the printed Q2_K packing).  Value = d * scale * q - dmin * min, the
+ * same sign convention as Q2_K.
+ */
+static void q4k_scale_min(const uint8_t *sm, int j, int *scale, int *min) {
+  if (j < 4) {
+    *scale = sm[j] & 63;
+    *min = sm[j + 4] & 63;
+  } else {
+    *scale = (sm[j + 4] & 15) | ((sm[j - 4] >> 6) << 4);
+    *min = (sm[j + 4] >> 4) | ((sm[j] >> 6) << 4);
+  }
+}
+
+double oracle_q4k_elem(const uint8_t *blk, int e) {
+  double d = oracle_f16(le16(blk));
+  double dmin = oracle_f16(le16(blk + 2));
+  int scale, min;
+  q4k_scale_min(blk + 4, e / 32, &scale, &min);
+  int q = (blk[16 + 32 * (e / 64) + e % 32] >> (4 * ((e % 64) / 32))) & 15;
+  return d * (double)scale * (double)q - dmin * (double)min;
+}
+
+void oracle_row_q4k(const uint8_t *row, int cols, double *out) {
+  for (int c = 0; c < cols; ++c) out[c] = oracle_q4k_elem(row + (size_t)(c / 256) * 144, c % 256);
+}
+
 /* ------------------------------------------------------------- mat-vec */
 
 static void decode_row(int kind, const uint8_t *row, int cols, const uint8_t *grid, double *out) {
@@ -129,12 +173,17 @@ static void decode_row(int kind, const uint8_t *row, int cols, const uint8_t *gr
     oracle_row_iq2xxs(row, cols, grid, out);
   else if (kind == 1)
     oracle_row_q2k(row, cols, out);
+  else if (kind == 3)
+    oracle_row_q4k(row, cols, out);
   else
     oracle_row_q80(row, cols, out);
 }
 
 static size_t row_bytes(int kind, int cols) {
-  return kind == 0 ? (size_t)cols / 256 * 66 : kind == 1 ? (size_t)cols / 256 * 84 : (size_t)cols / 32 * 34;
+  return kind == 0   ? (size_t)cols / 256 * 66
+         : kind == 1 ? (size_t)cols / 256 * 84
+         : kind == 3 ? (size_t)cols / 256 * 144
+                     : (size_t)cols / 32 * 34;
 }
 
 void oracle_matvec(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, const double *x,
@@ -294,16 +343,16 @@ int oracle_layer(const oracle_layer_w *W, const double *x, int T, const int32_t 
     }
     double *a = (double *)calloc((size_t)n * I, sizeof(double));
     double *b = (double *)calloc((size_t)n * I, sizeof(double));
-    size_t rg = row_bytes(0, H), rd = row_bytes(1, I);
+    size_t rg = row_bytes(W->gate_kind, H), rd = row_bytes(W->down_kind, I);
     for (int r = 0; r < I; ++r) {
-      oracle_row_iq2xxs(W->gate[e] + rg * (size_t)r, H, W->grid, wrow);
+      decode_row(W->gate_kind, W->gate[e] + rg * (size_t)r, H, W->grid, wrow);
       for (int m = 0; m < n; ++m) {
         const double *xt = x + (size_t)tok[m] * H;
         double acc = 0.0;
         for (int c = 0; c < H; ++c) acc += wrow[c] * xt[c];
         a[(size_t)m * I + r] = acc;
       }
-      oracle_row_iq2xxs(W->up[e] + rg * (size_t)r, H, W->grid, wrow);
+      decode_row(W->gate_kind, W->up[e] + rg * (size_t)r, H, W->grid, wrow);
       for (int m = 0; m < n; ++m) {
         const double *xt = x + (size_t)tok[m] * H;
         double acc = 0.0;
@@ -313,7 +362,7 @@ int oracle_layer(const oracle_layer_w *W, const double *x, int T, const int32_t 
     }
     for (size_t q = 0; q < (size_t)n * I; ++q) a[q] = oracle_silu(a[q]) * b[q];
     for (int r = 0; r < H; ++r) {
-      oracle_row_q2k(W->down[e] + rd * (size_t)r, I, wrow);
+      decode_row(W->down_kind, W->down[e] + rd * (size_t)r, I, W->grid, wrow);
       for (int m = 0; m < n; ++m) {
         const double *h = a + (size_t)m * I;
         double acc = 0.0;

@@ -41,13 +41,16 @@ extern "C" {
 /* IEEE binary16 (little-endian bits) to double, subnormals included. */
 double oracle_f16(uint16_t bits);
 
-/* Decode one element / one full row of `cols` elements. */
+/* Decode one element / one full row of `cols` elements.  Formats (kind):
+ * 0 IQ2_XXS, 1 Q2_K, 2 Q8_0, 3 Q4_K. */
 double oracle_iq2xxs_elem(const uint8_t *block66, const uint8_t *grid, int e);
 double oracle_q2k_elem(const uint8_t *block84, int e);
 double oracle_q80_elem(const uint8_t *block34, int e);
+double oracle_q4k_elem(const uint8_t *block144, int e);
 void oracle_row_iq2xxs(const uint8_t *row, int cols, const uint8_t *grid, double *out);
 void oracle_row_q2k(const uint8_t *row, int cols, double *out);
 void oracle_row_q80(const uint8_t *row, int cols, double *out);
+void oracle_row_q4k(const uint8_t *row, int cols, double *out);
 
 /* y[r] = sum_c W[r][c] x[c] with W decoded row by row (fused route). */
 void oracle_matvec(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, const double *x,
@@ -71,13 +74,15 @@ void oracle_swiglu_expert(int gate_kind, int down_kind, const uint8_t *gate, con
  * pointers (NULL for experts no token selects). */
 typedef struct {
   int hidden, inter, shared_inter, n_experts, top_k;
-  const uint8_t *const *gate; /* [n_experts] -> IQ2_XXS [inter][hidden/256][66] */
-  const uint8_t *const *up;   /* [n_experts] -> IQ2_XXS [inter][hidden/256][66] */
-  const uint8_t *const *down; /* [n_experts] -> Q2_K [hidden][inter/256][84] */
+  const uint8_t *const *gate; /* [n_experts] -> [inter][hidden/256] blocks of gate_kind */
+  const uint8_t *const *up;   /* [n_experts] -> [inter][hidden/256] blocks of gate_kind */
+  const uint8_t *const *down; /* [n_experts] -> [hidden][inter/256] blocks of down_kind */
   const uint8_t *sh_gate;     /* Q8_0 [shared_inter][hidden/32][34] */
   const uint8_t *sh_up;       /* Q8_0 [shared_inter][hidden/32][34] */
   const uint8_t *sh_down;     /* Q8_0 [hidden][shared_inter/32][34] */
   const uint8_t *grid;        /* [256][8] */
+  int gate_kind;              /* routed gate/up format: 0 IQ2_XXS (q2 build), 3 Q4_K (q2-q4 layers) */
+  int down_kind;              /* routed down format: 1 Q2_K (q2 build), 3 Q4_K */
 } oracle_layer_w;
 
 int oracle_layer(const oracle_layer_w *Wt, const double *x, int T, const int32_t *idx, const double *w,
