@@ -35,10 +35,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _HOST_SO = os.path.join(_HERE, "_synth_host.so")
 _DEV_SO = os.path.join(_HERE, "_synth_dev.so")
 
-KIND_IQ2XXS, KIND_Q2K, KIND_Q80 = 0, 1, 2
+KIND_IQ2XXS, KIND_Q2K, KIND_Q80, KIND_Q4K = 0, 1, 2, 3
 T_BIAS, T_GATE, T_UP, T_DOWN, T_SH_GATE, T_SH_UP, T_SH_DOWN, T_GRID, T_TID2EID = 2, 3, 4, 5, 6, 7, 8, 9, 10
-BLOCK_BYTES = {KIND_IQ2XXS: 66, KIND_Q2K: 84, KIND_Q80: 34}
-BLOCK_ELEMS = {KIND_IQ2XXS: 256, KIND_Q2K: 256, KIND_Q80: 32}
+BLOCK_BYTES = {KIND_IQ2XXS: 66, KIND_Q2K: 84, KIND_Q80: 34, KIND_Q4K: 144}
+BLOCK_ELEMS = {KIND_IQ2XXS: 256, KIND_Q2K: 256, KIND_Q80: 32, KIND_Q4K: 256}
 
 
 @dataclass(frozen=True)

@@ -24,6 +24,9 @@
  *   Q2_K     scales/mins bytes and 2-bit codes are raw random bytes (so every
  *            nibble and code is uniform); d, dmin = f16(0.001 + 0.009 u).
  *   Q8_0     d = f16(0.0005); int8 values U[-127,127].
+ *   Q4_K     the 12 scale/min bytes and the 4-bit codes are raw random bytes
+ *            (every 6-bit scale, 6-bit min and code uniform); d, dmin =
+ *            f16(0.0001 + 0.0009 u), so d * 63 * 15 stays below 1.
  *   codebook 256 x 8 bytes, each drawn from {8, 25, 43}.
  *   bias     U(-0.1, 0.1) in fp32, +0.5 on experts with e % 8 == 0 when the
  *            skewed variant is asked for.
@@ -54,7 +57,7 @@ enum {
   SYNTH_T_TID2EID = 10,
 };
 
-enum { SYNTH_IQ2XXS_BYTES = 66, SYNTH_Q2K_BYTES = 84, SYNTH_Q80_BYTES = 34 };
+enum { SYNTH_IQ2XXS_BYTES = 66, SYNTH_Q2K_BYTES = 84, SYNTH_Q80_BYTES = 34, SYNTH_Q4K_BYTES = 144 };
 
 SYNTH_FN uint64_t synth_mix64(uint64_t z) {
   z += 0x9E3779B97F4A7C15ull;
@@ -157,6 +160,17 @@ SYNTH_FN void synth_q80_block(uint64_t key, uint64_t block, uint8_t *out) {
     out[2 + 2 * w] = (uint8_t)(int8_t)a;
     out[3 + 2 * w] = (uint8_t)(int8_t)b;
   }
+}
+
+/* One Q4_K block (256 elements, 144 bytes): f16 d, f16 dmin, then 140 raw
+ * bytes (12 of scales and mins, 128 of codes). */
+SYNTH_FN void synth_q4k_block(uint64_t key, uint64_t block, uint8_t *out) {
+  for (int w = 0; w < 17; ++w) synth_put64(out + 4 + 8 * w, synth_word(key, block, w)); /* bytes 4..139 */
+  uint64_t wt = synth_word(key, block, 17);
+  for (int i = 0; i < 4; ++i) out[140 + i] = (uint8_t)(wt >> (8 * i));
+  uint64_t wd = synth_word(key, block, 18);
+  synth_put16(out, synth_f16_bits(synth_affine24((uint32_t)(wd >> 40), 0.0001f, 0.0009f)));
+  synth_put16(out + 2, synth_f16_bits(synth_affine24((uint32_t)(wd >> 8) & 0xFFFFFFu, 0.0001f, 0.0009f)));
 }
 
 /* Codebook entry (row r, lane l) drawn from {8, 25, 43}. */

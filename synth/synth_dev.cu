@@ -8,7 +8,10 @@ namespace {
 
 template <int KIND>
 __global__ void fill_kernel(uint64_t key, uint64_t first, uint64_t n, uint8_t *__restrict__ out) {
-  constexpr int BYTES = KIND == 0 ? SYNTH_IQ2XXS_BYTES : (KIND == 1 ? SYNTH_Q2K_BYTES : SYNTH_Q80_BYTES);
+  constexpr int BYTES = KIND == 0   ? SYNTH_IQ2XXS_BYTES
+                        : KIND == 1 ? SYNTH_Q2K_BYTES
+                        : KIND == 3 ? SYNTH_Q4K_BYTES
+                                    : SYNTH_Q80_BYTES;
   uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   for (uint64_t b = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n; b += stride) {
     uint8_t tmp[BYTES];
@@ -16,6 +19,8 @@ __global__ void fill_kernel(uint64_t key, uint64_t first, uint64_t n, uint8_t *_
       synth_iq2xxs_block(key, first + b, tmp);
     else if (KIND == 1)
       synth_q2k_block(key, first + b, tmp);
+    else if (KIND == 3)
+      synth_q4k_block(key, first + b, tmp);
     else
       synth_q80_block(key, first + b, tmp);
     uint8_t *dst = out + b * BYTES;
@@ -31,7 +36,7 @@ __global__ void fill_kernel(uint64_t key, uint64_t first, uint64_t n, uint8_t *_
 
 extern "C" int synth_dev_fill_routed(uint64_t seed, uint32_t layer, uint32_t tensor, int kind, int e0, int ne,
                                      int rows, int cols, void *out, void *stream) {
-  if (kind < 0 || kind > 2 || ne < 0 || rows <= 0 || cols <= 0 || out == nullptr) return -1;
+  if (kind < 0 || kind > 3 || ne < 0 || rows <= 0 || cols <= 0 || out == nullptr) return -1;
   if ((reinterpret_cast<uintptr_t>(out) & 1u) != 0) return -1;
   uint64_t bpr = (uint64_t)cols / (kind == 2 ? 32u : 256u);
   uint64_t per_expert = (uint64_t)rows * bpr;
@@ -48,6 +53,8 @@ extern "C" int synth_dev_fill_routed(uint64_t seed, uint32_t layer, uint32_t ten
     fill_kernel<0><<<blocks, threads, 0, s>>>(key, first, n, o);
   else if (kind == 1)
     fill_kernel<1><<<blocks, threads, 0, s>>>(key, first, n, o);
+  else if (kind == 3)
+    fill_kernel<3><<<blocks, threads, 0, s>>>(key, first, n, o);
   else
     fill_kernel<2><<<blocks, threads, 0, s>>>(key, first, n, o);
   return cudaGetLastError() == cudaSuccess ? 0 : -2;

@@ -2,7 +2,7 @@
  * synth_host.c -- host fills built on synth.h (shared library for ctypes).
  *
  * Each fill writes the canonical layout the layer's boundary takes:
- *   routed IQ2_XXS / Q2_K tensors: [expert][row][block], experts
+ *   routed IQ2_XXS / Q2_K / Q4_K tensors: [expert][row][block], experts
  *   [expert_begin, expert_begin + n_experts) of the tensor;
  *   shared Q8_0 tensors: [row][block].
  * Threads split the work by expert or row only; every byte is a pure
@@ -17,7 +17,7 @@ typedef struct {
   uint64_t key;
   uint64_t first_block;
   uint64_t n_blocks;
-  int kind; /* 0 iq2xxs, 1 q2k, 2 q80 */
+  int kind; /* 0 iq2xxs, 1 q2k, 2 q80, 3 q4k */
   uint8_t *out;
 } fill_job;
 
@@ -29,6 +29,8 @@ static void *fill_run(void *arg) {
       synth_iq2xxs_block(j->key, gb, j->out + b * SYNTH_IQ2XXS_BYTES);
     else if (j->kind == 1)
       synth_q2k_block(j->key, gb, j->out + b * SYNTH_Q2K_BYTES);
+    else if (j->kind == 3)
+      synth_q4k_block(j->key, gb, j->out + b * SYNTH_Q4K_BYTES);
     else
       synth_q80_block(j->key, gb, j->out + b * SYNTH_Q80_BYTES);
   }
@@ -36,7 +38,7 @@ static void *fill_run(void *arg) {
 }
 
 static void fill_blocks(uint64_t key, uint64_t first, uint64_t n, int kind, uint8_t *out, int threads) {
-  const uint64_t bytes[3] = {SYNTH_IQ2XXS_BYTES, SYNTH_Q2K_BYTES, SYNTH_Q80_BYTES};
+  const uint64_t bytes[4] = {SYNTH_IQ2XXS_BYTES, SYNTH_Q2K_BYTES, SYNTH_Q80_BYTES, SYNTH_Q4K_BYTES};
   if (threads < 1) threads = 1;
   if (threads > 64) threads = 64;
   if (n < 4096) threads = 1;

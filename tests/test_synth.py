@@ -51,6 +51,23 @@ def test_block_field_distributions():
     assert np.all(S8[:, 0:2].copy().view(np.float16) == np.float16(0.0005))
 
 
+def test_q4k_block_fields():
+    """Q4_K blocks: f16 d and dmin in [0.0001, 0.001], raw scale/min and code
+    bytes (every byte value occurs), deterministic and thread-invariant."""
+    W = synth.routed(2, 40, synth.T_DOWN, synth.KIND_Q4K, 0, 1, 512, 2048)[0].reshape(-1, 144)
+    for off in (0, 2):
+        v = W[:, off:off + 2].copy().view(np.float16).astype(np.float64).ravel()
+        assert v.min() >= 0.0001 - 1e-7 and v.max() <= 0.001 + 1e-6
+    for lo, hi in ((4, 16), (16, 144)):
+        assert np.unique(W[:, lo:hi]).size == 256
+    lib = synth._hostlib()
+    a = synth.routed(2, 40, synth.T_GATE, synth.KIND_Q4K, 3, 2, 64, 512)
+    b = np.empty_like(a)
+    lib.synth_fill_routed(2, 40, synth.T_GATE, synth.KIND_Q4K, 3, 2, 64, 512, b.ctypes.data, 1)
+    assert np.array_equal(a, b)
+    assert np.array_equal(synth.routed(2, 40, synth.T_GATE, synth.KIND_Q4K, 0, 5, 64, 512)[3:5], a)
+
+
 def test_grid_bias_and_hash_table():
     g = synth.grid(0)
     assert g.shape == (256, 8) and set(np.unique(g).tolist()) == {8, 25, 43}
