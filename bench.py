@@ -337,7 +337,10 @@ def run_ours(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8xs8->s32 tensor-core products, fp32 scaling",
+        # small-token path: int8 weights x int8 activation limbs, exact int32
+        # products, fp32 scaling; batched path: tcgen05 f16 (gate/up) and
+        # bf16 (down) operands with fp32 accumulation
+        "dtype": "f16/bf16" if large else "s8",
         "data": "synthetic (seeded generator; V4-Flash shapes, random weights)",
         "config": {"workload": f"{args.workload}: V4-Flash MoE layer, T={T} tokens/call, hidden {s.hidden}, "
                                f"{s.n_experts} experts top-{s.top_k}, inter {s.inter}, shared {s.shared_inter}",
@@ -438,7 +441,7 @@ def run_stack(args, world, rank):
         "metric": METRIC, "value": job_throughput(world, args.steps, T, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "us_per_layer": ms_step * 1e3 / s.layers, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8xs8->s32 tensor-core products, fp32 scaling",
+        "vs_baseline": None, "dtype": "s8",
         "data": "synthetic (seeded generator; V4-Flash shapes, random weights)",
         "config": {"workload": f"{args.workload}: {s.layers} chained V4-Flash MoE layers (0-{s.hash_layers - 1} hash-"
                                f"routed), T={T}, x <- x + MoE(RMSNorm(x))",
@@ -604,7 +607,7 @@ def run_quant(args, world, rank):
     return {
         "metric": QUANT_METRIC, "value": job_throughput(world, args.steps, n, ms), "unit": "values/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_launch,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> binary32 decisions",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (N(0, 0.02^2) fp32 values from torch's generator)",
         "config": {"workload": f"{args.workload}: {QUANT_MATS} x {QUANT_ROWS} x {QUANT_COLS} fp32 values per step "
                                f"-> {'Q2_K' if per == 256 else 'Q8_0'} blocks",
@@ -646,7 +649,7 @@ def run_reference(args, world, rank):
                   f"{elapsed:.2f} s after {args.warmup} warm-up steps")
         return {"metric": QUANT_METRIC, "value": value, "unit": "values/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / max(args.steps, 1), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> binary32 decisions", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "impl": "reference", "config": {"workload": f"{args.workload} (2^20 values per step)"},
                 "cpu_baseline": {"value": value, "unit": "values/s", "cores": 1, "kind": "oracle", "sample": sample},
                 "e2e": {"value": value, "unit": "values/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
