@@ -324,7 +324,8 @@ def run_ours(args, world, rank):
                 "achieved": tc_achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tc_achieved / peaks["bf16_tflops"], "traffic": load_traffic(args.workload),
                 "traffic_unit": "bytes per launch (ncu)", "peak_source": peaks["source"],
-                "algorithmic_flops_per_launch": fl["gateup_routed"], "ms_per_launch": k2_ms, "median_ms_per_launch": k2_median}
+                "algorithmic_flops_per_launch": fl["gateup_routed"], "ms_per_launch": k2_ms,
+                "median_ms_per_launch": k2_median}
         layer = {"flops_per_call": fl["layer"], "achieved_tflops": fl["layer"] / (ms_step / 1e3) / 1e12,
                  "frac": fl["layer"] / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"],
                  "frac_of_nominal_2250": fl["layer"] / (ms_step / 1e3) / 1e12 / 2250.0}
