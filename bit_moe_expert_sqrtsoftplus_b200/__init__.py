@@ -31,6 +31,8 @@ MOE_FLAG_PRENORM_RESIDUAL = 1
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
 MOE_QUANT_Q8_0 = 0
 MOE_QUANT_Q2_K = 1
+MOE_ROUTED_Q2 = 0
+MOE_ROUTED_Q4K = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
             "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_quantize", "moe_destroy")
@@ -40,7 +42,7 @@ class moe_config(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("shared_inter", ctypes.c_int), ("vocab", ctypes.c_int),
                 ("routed_scaling", ctypes.c_float), ("rms_eps", ctypes.c_float), ("mode", ctypes.c_int),
-                ("flags", ctypes.c_int)]
+                ("flags", ctypes.c_int), ("routed_format", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):
@@ -108,8 +110,9 @@ def _stream(stream):
 
 
 def make_config(hidden, inter, n_experts, top_k, shared_inter, vocab=0, routed_scaling=1.5, rms_eps=1e-6,
-                mode=MOE_ROUTE_ROUTER, flags=0) -> moe_config:
-    return moe_config(hidden, inter, n_experts, top_k, shared_inter, vocab, routed_scaling, rms_eps, mode, flags)
+                mode=MOE_ROUTE_ROUTER, flags=0, routed_format=MOE_ROUTED_Q2) -> moe_config:
+    return moe_config(hidden, inter, n_experts, top_k, shared_inter, vocab, routed_scaling, rms_eps, mode, flags,
+                      routed_format)
 
 
 def moe_workspace_size(cfg: moe_config, max_tokens: int):
@@ -121,7 +124,7 @@ def moe_workspace_size(cfg: moe_config, max_tokens: int):
 def make_weights(w: dict) -> moe_weights:
     return moe_weights(_ptr(w.get("router_w")), _ptr(w.get("bias")), _ptr(w.get("tid2eid")), _ptr(w["gate"]),
                        _ptr(w["up"]), _ptr(w["down"]), _ptr(w["sh_gate"]), _ptr(w["sh_up"]), _ptr(w["sh_down"]),
-                       _ptr(w["grid"]))
+                       _ptr(w.get("grid")))
 
 
 def moe_init(cfg: moe_config, weights: moe_weights, persist, stream=None) -> int:

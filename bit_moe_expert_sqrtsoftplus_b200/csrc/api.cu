@@ -12,6 +12,7 @@
 #include "../../include/moe.h"
 #include "layer.cuh"
 #include "prefill.cuh"
+#include "q4k.cuh"
 #include "quant.cuh"
 
 static_assert(MOE_SMALL_T_MAX == moe::kDecodeMaxT, "header and kernels disagree on the small-T limit");
@@ -75,6 +76,8 @@ moe_status check_config(const moe_config *c) {
   if ((c->flags & MOE_FLAG_PRENORM_RESIDUAL) && !(c->rms_eps >= 0.f && isfinite(c->rms_eps)))
     return fail(MOE_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
   if (c->flags & ~MOE_FLAG_PRENORM_RESIDUAL) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
+  if (c->routed_format != MOE_ROUTED_Q2 && c->routed_format != MOE_ROUTED_Q4K)
+    return fail(MOE_ERR_INVALID_ARG, "routed_format=%d is not a MOE_ROUTED_* format", c->routed_format);
   return MOE_OK;
 }
 
@@ -93,10 +96,29 @@ moe::LayerDims dims_of(const moe_config &c) {
   return d;
 }
 
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
 size_t scratch_bytes_for(const moe::LayerDims &d, int max_tokens) {
   size_t dec = moe::decode_scratch_bytes(d, max_tokens < moe::kDecodeMaxT ? max_tokens : moe::kDecodeMaxT);
   size_t pre = max_tokens > moe::kDecodeMaxT ? moe::prefill_scratch_bytes(d, max_tokens) : 0;
   return dec > pre ? dec : pre;
+}
+
+// Q4_K forward (T <= kDecodeMaxT): the routing scratch, then idx and w, then
+// the expert kernels' buffers.
+size_t q4k_scratch_bytes(const moe::LayerDims &d, int T) {
+  return align256(moe::decode_scratch_bytes(d, T)) + 2 * align256(sizeof(int32_t) * (size_t)T * d.k) +
+         moe::q4k_expert_bytes(d, T);
+}
+
+size_t scratch_bytes_for(const moe_config &c, int max_tokens) {
+  const moe::LayerDims d = dims_of(c);
+  size_t s = scratch_bytes_for(d, max_tokens);
+  if (c.routed_format == MOE_ROUTED_Q4K) {
+    const size_t q = q4k_scratch_bytes(d, max_tokens < moe::kDecodeMaxT ? max_tokens : moe::kDecodeMaxT);
+    s = q > s ? q : s;
+  }
+  return s;
 }
 
 // The kernels run on the current device with the handle's pointers, which
@@ -120,7 +142,7 @@ moe_status check_call(moe_handle *h, const float *x, const int32_t *token_ids, i
   if (h->d.mode == MOE_ROUTE_HASH && !token_ids) return fail(MOE_ERR_INVALID_ARG, "hash mode needs token_ids");
   if (!scratch) return fail(MOE_ERR_INVALID_ARG, "scratch is NULL");
   if (!aligned16(scratch)) return fail(MOE_ERR_MISALIGNED, "scratch is not 16-byte aligned");
-  const size_t need = scratch_bytes_for(h->d, T);
+  const size_t need = scratch_bytes_for(h->cfg, T);
   if (scratch_bytes < need)
     return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for T=%d", scratch_bytes, need, T);
   return check_device(h);
@@ -137,7 +159,7 @@ moe_status moe_workspace_size(const moe_config *cfg, int max_tokens, size_t *per
   if (st != MOE_OK) return st;
   if (max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "max_tokens=%d is negative", max_tokens);
   if (persist_bytes) *persist_bytes = persist_bytes_for(*cfg);
-  if (scratch_bytes) *scratch_bytes = max_tokens > 0 ? scratch_bytes_for(dims_of(*cfg), max_tokens) : 0;
+  if (scratch_bytes) *scratch_bytes = max_tokens > 0 ? scratch_bytes_for(*cfg, max_tokens) : 0;
   g_last_error.clear();
   return MOE_OK;
 }
@@ -153,7 +175,8 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
                         w->iq2_grid};
   const char *names[] = {"gate_iq2xxs", "up_iq2xxs", "down_q2k", "sh_gate_q80", "sh_up_q80", "sh_down_q80",
                          "iq2_grid"};
-  for (int i = 0; i < 7; ++i) {
+  const int n_need = cfg->routed_format == MOE_ROUTED_Q4K ? 6 : 7;  // Q4_K layers read no codebook
+  for (int i = 0; i < n_need; ++i) {
     if (!need[i]) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", names[i]);
     if (!aligned16(need[i])) return fail(MOE_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
   }
@@ -193,7 +216,8 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   h->wt.sh_up = static_cast<const uint8_t *>(w->sh_up_q80);
   h->wt.sh_down = static_cast<const uint8_t *>(w->sh_down_q80);
   h->wt.grid = w->iq2_grid;
-  moe::build_chunk_tensor_maps(h->wt, h->d);
+  h->wt.tma = 0;
+  if (cfg->routed_format == MOE_ROUTED_Q2) moe::build_chunk_tensor_maps(h->wt, h->d);
   h->err = static_cast<int *>(persist);
   h->row_norms = reinterpret_cast<float *>(static_cast<uint8_t *>(persist) + kPersistHeader);
   h->num_sms = sms;
@@ -230,6 +254,43 @@ static moe::DecodeArgs decode_args(moe_handle *h, const float *x, const int32_t 
   a.ev_begin = h->ev_begin;
   a.ev_end = h->ev_end;
   return a;
+}
+
+// Routing as the small-token path does it, then the Q4_K expert kernels.
+static cudaError_t q4k_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y, void *scratch,
+                               cudaStream_t s) {
+  uint8_t *base = static_cast<uint8_t *>(scratch);
+  size_t off = align256(moe::decode_scratch_bytes(h->d, T));
+  int32_t *idx = reinterpret_cast<int32_t *>(base + off);
+  off += align256(sizeof(int32_t) * (size_t)T * h->d.k);
+  float *w = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * (size_t)T * h->d.k);
+  moe::DecodeArgs a = decode_args(h, x, token_ids, T, nullptr, scratch);
+  a.ev_begin = a.ev_end = nullptr;
+  cudaError_t e = moe::decode_route(a, idx, w, s);
+  if (e != cudaSuccess) return e;
+  moe::Q4kArgs q;
+  q.d = h->d;
+  q.gate = h->wt.gate;
+  q.up = h->wt.up;
+  q.down = h->wt.down;
+  q.sh_gate = h->wt.sh_gate;
+  q.sh_up = h->wt.sh_up;
+  q.sh_down = h->wt.sh_down;
+  q.T = T;
+  q.x = x;
+  q.y = y;
+  q.idx = idx;
+  q.w = w;
+  q.xn = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * (size_t)T * h->d.H);
+  q.h = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * (size_t)T * h->d.k * h->d.I);
+  q.hs = reinterpret_cast<float *>(base + off);
+  if (h->ev_begin) cudaEventRecord(h->ev_begin, s);
+  e = moe::q4k_experts(q, s);
+  if (h->ev_end) cudaEventRecord(h->ev_end, s);
+  return e;
 }
 
 moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, int T, int32_t *idx, float *w,
@@ -270,7 +331,12 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
     return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (T <= moe::kDecodeMaxT) {
+  if (h->cfg.routed_format == MOE_ROUTED_Q4K) {
+    if (T > moe::kDecodeMaxT)
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "Q4_K layers run at most %d tokens per call (got %d)", moe::kDecodeMaxT,
+                  T);
+    e = q4k_forward(h, x, token_ids, T, y, scratch, s);
+  } else if (T <= moe::kDecodeMaxT) {
     moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
     e = moe::decode_forward(a, s, h->num_sms);
   } else {
@@ -325,6 +391,8 @@ moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t 
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
   if (T == 0) return MOE_OK;
+  if (h->cfg.routed_format != MOE_ROUTED_Q2)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_forward_noalloc runs the q2 routed formats only");
   if (T > kNoAllocMaxT)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_forward_noalloc handles at most %d tokens per call (got %d)",
                 kNoAllocMaxT, T);

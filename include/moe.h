@@ -70,6 +70,10 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 
 #define MOE_SMALL_T_MAX 32 /* largest T served by the small-token kernels */
 
+/* formats of the routed experts (moe_config.routed_format) */
+#define MOE_ROUTED_Q2 0  /* the q2 build: gate/up IQ2_XXS, down Q2_K */
+#define MOE_ROUTED_Q4K 1 /* the q2-q4 build's upgraded layers: gate, up and down Q4_K (144 bytes per 256) */
+
 /* block formats of moe_quantize */
 #define MOE_QUANT_Q8_0 0 /* 32 values in 34 bytes */
 #define MOE_QUANT_Q2_K 1 /* 256 values in 84 bytes */
@@ -85,19 +89,21 @@ typedef struct {
   float rms_eps;        /* RMSNorm epsilon when MOE_FLAG_PRENORM_RESIDUAL is set (1e-6) */
   int mode;             /* moe_route_mode */
   int flags;            /* MOE_FLAG_* */
+  int routed_format;    /* MOE_ROUTED_*; MOE_ROUTED_Q4K layers run moe_ffn_forward for T <= MOE_SMALL_T_MAX
+                           only (moe_route takes any T) and not moe_ffn_forward_noalloc */
 } moe_config;
 
 typedef struct {
   const void *router_w_f16;   /* [E][H] IEEE f16; NULL in hash mode */
   const float *router_bias;   /* [E] fp32 selection bias; NULL in hash mode */
   const int32_t *tid2eid;     /* [vocab][k] expert ids; NULL in router mode */
-  const void *gate_iq2xxs;    /* [E][I][H/256] 66-byte blocks */
-  const void *up_iq2xxs;      /* [E][I][H/256] 66-byte blocks */
-  const void *down_q2k;       /* [E][H][I/256] 84-byte blocks */
+  const void *gate_iq2xxs;    /* [E][I][H/256] 66-byte blocks (144-byte Q4_K blocks with MOE_ROUTED_Q4K) */
+  const void *up_iq2xxs;      /* [E][I][H/256] 66-byte blocks (Q4_K likewise) */
+  const void *down_q2k;       /* [E][H][I/256] 84-byte blocks (Q4_K likewise) */
   const void *sh_gate_q80;    /* [Is][H/32] 34-byte blocks */
   const void *sh_up_q80;      /* [Is][H/32] 34-byte blocks */
   const void *sh_down_q80;    /* [H][Is/32] 34-byte blocks */
-  const uint8_t *iq2_grid;    /* [256][8] codebook; every entry must be <= 127 */
+  const uint8_t *iq2_grid;    /* [256][8] codebook; every entry must be <= 127 (may be NULL with MOE_ROUTED_Q4K) */
 } moe_weights;
 
 typedef struct moe_handle moe_handle;

@@ -202,9 +202,11 @@ def shared(seed: int, layer: int, tensor: int, rows: int, cols: int) -> np.ndarr
     return routed(seed, layer, tensor, KIND_Q80, 0, 1, rows, cols)[0]
 
 
-def host_layer(seed: int, layer: int, s: LayerShape, experts=None, router: bool = True) -> dict:
+def host_layer(seed: int, layer: int, s: LayerShape, experts=None, router: bool = True, q4k: bool = False) -> dict:
     """All inputs of one layer on the host.  ``experts`` limits the routed
-    tensors to the listed expert ids (returned as dicts id -> array)."""
+    tensors to the listed expert ids (returned as dicts id -> array).  With
+    ``q4k`` the routed gate, up and down tensors are Q4_K (the q2-q4 build's
+    upgraded layers) and the dict names their formats."""
     ids = range(s.n_experts) if experts is None else sorted(set(int(e) for e in experts))
     out = {
         "grid": grid(seed, layer),
@@ -217,14 +219,16 @@ def host_layer(seed: int, layer: int, s: LayerShape, experts=None, router: bool 
         out["bias"] = bias(seed, layer, s.n_experts, s.skew)
     else:
         out["tid2eid"] = tid2eid(seed, layer, s.vocab, s.n_experts, s.top_k)
+    kg, kd = (KIND_Q4K, KIND_Q4K) if q4k else (KIND_IQ2XXS, KIND_Q2K)
+    out["gate_kind"], out["down_kind"] = kg, kd
     if experts is None:
-        out["gate"] = routed(seed, layer, T_GATE, KIND_IQ2XXS, 0, s.n_experts, s.inter, s.hidden)
-        out["up"] = routed(seed, layer, T_UP, KIND_IQ2XXS, 0, s.n_experts, s.inter, s.hidden)
-        out["down"] = routed(seed, layer, T_DOWN, KIND_Q2K, 0, s.n_experts, s.hidden, s.inter)
+        out["gate"] = routed(seed, layer, T_GATE, kg, 0, s.n_experts, s.inter, s.hidden)
+        out["up"] = routed(seed, layer, T_UP, kg, 0, s.n_experts, s.inter, s.hidden)
+        out["down"] = routed(seed, layer, T_DOWN, kd, 0, s.n_experts, s.hidden, s.inter)
     else:
-        out["gate"] = {e: routed(seed, layer, T_GATE, KIND_IQ2XXS, e, 1, s.inter, s.hidden)[0] for e in ids}
-        out["up"] = {e: routed(seed, layer, T_UP, KIND_IQ2XXS, e, 1, s.inter, s.hidden)[0] for e in ids}
-        out["down"] = {e: routed(seed, layer, T_DOWN, KIND_Q2K, e, 1, s.hidden, s.inter)[0] for e in ids}
+        out["gate"] = {e: routed(seed, layer, T_GATE, kg, e, 1, s.inter, s.hidden)[0] for e in ids}
+        out["up"] = {e: routed(seed, layer, T_UP, kg, e, 1, s.inter, s.hidden)[0] for e in ids}
+        out["down"] = {e: routed(seed, layer, T_DOWN, kd, e, 1, s.hidden, s.inter)[0] for e in ids}
     return out
 
 
@@ -239,20 +243,22 @@ def device_routed(out_tensor, seed: int, layer: int, tensor: int, kind: int, e0:
         raise RuntimeError(f"synth_dev_fill_routed failed ({rc})")
 
 
-def device_layer(seed: int, layer: int, s: LayerShape, router: bool = True, device="cuda") -> dict:
-    """All inputs of one layer as CUDA tensors (packed weights generated on the GPU)."""
+def device_layer(seed: int, layer: int, s: LayerShape, router: bool = True, device="cuda", q4k: bool = False) -> dict:
+    """All inputs of one layer as CUDA tensors (packed weights generated on
+    the GPU); ``q4k`` as in :func:`host_layer`."""
     import torch
 
     stream = torch.cuda.current_stream().cuda_stream
-    rb_g = s.row_bytes(KIND_IQ2XXS, s.hidden)
-    rb_d = s.row_bytes(KIND_Q2K, s.inter)
-    out = {}
+    kg, kd = (KIND_Q4K, KIND_Q4K) if q4k else (KIND_IQ2XXS, KIND_Q2K)
+    rb_g = s.row_bytes(kg, s.hidden)
+    rb_d = s.row_bytes(kd, s.inter)
+    out = {"gate_kind": kg, "down_kind": kd}
     out["gate"] = torch.empty((s.n_experts, s.inter, rb_g), dtype=torch.uint8, device=device)
     out["up"] = torch.empty((s.n_experts, s.inter, rb_g), dtype=torch.uint8, device=device)
     out["down"] = torch.empty((s.n_experts, s.hidden, rb_d), dtype=torch.uint8, device=device)
-    device_routed(out["gate"], seed, layer, T_GATE, KIND_IQ2XXS, 0, s.n_experts, s.inter, s.hidden, stream)
-    device_routed(out["up"], seed, layer, T_UP, KIND_IQ2XXS, 0, s.n_experts, s.inter, s.hidden, stream)
-    device_routed(out["down"], seed, layer, T_DOWN, KIND_Q2K, 0, s.n_experts, s.hidden, s.inter, stream)
+    device_routed(out["gate"], seed, layer, T_GATE, kg, 0, s.n_experts, s.inter, s.hidden, stream)
+    device_routed(out["up"], seed, layer, T_UP, kg, 0, s.n_experts, s.inter, s.hidden, stream)
+    device_routed(out["down"], seed, layer, T_DOWN, kd, 0, s.n_experts, s.hidden, s.inter, stream)
     for name, t, rows, cols in (("sh_gate", T_SH_GATE, s.shared_inter, s.hidden),
                                 ("sh_up", T_SH_UP, s.shared_inter, s.hidden),
                                 ("sh_down", T_SH_DOWN, s.hidden, s.shared_inter)):

@@ -12,20 +12,21 @@ MMA_REL_L2 = 3e-3         # bf16 tensor-core path
 MAX_ABS_FRAC = 2e-2       # max |err| <= 2e-2 * max |y|
 
 
-def config_for(s: synth.LayerShape, mode=None, flags=0):
+def config_for(s: synth.LayerShape, mode=None, flags=0, q4k=False):
     import bit_moe_expert_sqrtsoftplus_b200 as moe
     if mode is None:
         mode = moe.MOE_ROUTE_ROUTER
     return moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
-                           routed_scaling=s.routed_scaling, rms_eps=1e-6, mode=mode, flags=flags)
+                           routed_scaling=s.routed_scaling, rms_eps=1e-6, mode=mode, flags=flags,
+                           routed_format=moe.MOE_ROUTED_Q4K if q4k else moe.MOE_ROUTED_Q2)
 
 
-def device_layer(s: synth.LayerShape, seed: int, layer: int, router=True):
-    return synth.device_layer(seed, layer, s, router=router)
+def device_layer(s: synth.LayerShape, seed: int, layer: int, router=True, q4k=False):
+    return synth.device_layer(seed, layer, s, router=router, q4k=q4k)
 
 
 def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, token_ids=None, router=True,
-                 prenorm=False, threads: int = 1):
+                 prenorm=False, threads: int = 1, q4k=False):
     """fp64 oracle: returns (idx, w, y, margin)."""
     xin = x.astype(np.float64)
     if prenorm:
@@ -39,7 +40,7 @@ def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, toke
         tab = synth.tid2eid(seed, layer, s.vocab, s.n_experts, s.top_k)
         idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling)
         margin = np.full(x.shape[0], np.inf)
-    W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router)
+    W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router, q4k=q4k)
     y = oracle.layer(W, s, xin, idx, w, threads=threads)
     if prenorm:
         y = y + x.astype(np.float64)

@@ -70,7 +70,8 @@ def test_workspace_size_and_shape_checks(moe):
                         (dict(n_experts=4, top_k=6), moe.MOE_ERR_UNSUPPORTED_SHAPE),
                         (dict(mode=7), moe.MOE_ERR_INVALID_ARG),
                         (dict(mode=1, vocab=0), moe.MOE_ERR_INVALID_ARG),
-                        (dict(flags=8), moe.MOE_ERR_INVALID_ARG)):
+                        (dict(flags=8), moe.MOE_ERR_INVALID_ARG),
+                        (dict(routed_format=5), moe.MOE_ERR_INVALID_ARG)):
         with pytest.raises(moe.MoeError) as ei:
             moe.moe_workspace_size(_cfg(moe, **bad), 1)
         assert ei.value.status == status, bad
@@ -81,12 +82,21 @@ def test_scratch_size_never_shrinks_with_more_tokens(moe):
     """A scratch buffer sized for max_tokens serves every call with fewer
     tokens, so the size must not decrease as max_tokens grows (the small-T
     layout changes with the unit width, the large-T one starts above 32)."""
-    for shape in (dict(), dict(hidden=256, inter=256, n_experts=16, top_k=2, shared_inter=256)):
+    for shape in (dict(), dict(hidden=256, inter=256, n_experts=16, top_k=2, shared_inter=256),
+                  dict(routed_format=moe.MOE_ROUTED_Q4K)):
         prev = 0
         for T in list(range(1, 70)) + [128, 4096]:
             _, s = moe.moe_workspace_size(_cfg(moe, **shape), T)
             assert s >= prev, (shape, T, s, prev)
             prev = s
+
+
+def test_q4k_layers_take_more_scratch_up_to_32_tokens(moe):
+    """The Q4_K forward keeps its expert buffers beside the routing scratch."""
+    for T in (1, 8, 32):
+        _, q2 = moe.moe_workspace_size(_cfg(moe), T)
+        _, q4 = moe.moe_workspace_size(_cfg(moe, routed_format=moe.MOE_ROUTED_Q4K), T)
+        assert q4 >= q2 + 4 * T * (4096 + 6 * 2048 + 2048)
 
 
 def test_quantize_argument_checks(moe):

@@ -21,3 +21,78 @@ def test_q4k_device_fill_is_byte_identical_to_host_fill():
         synth.device_routed(dev, 3, 40, tensor, synth.KIND_Q4K, e0, ne, rows, cols)
         torch.cuda.synchronize()
         assert np.array_equal(dev.cpu().numpy(), host)
+
+
+# ------------------------------------------------------------ the Q4_K layer
+
+from tests import harness  # noqa: E402
+
+import oracle  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from bit_moe_expert_sqrtsoftplus_b200 import build
+    build.build()
+    import bit_moe_expert_sqrtsoftplus_b200 as m
+    return m
+
+
+def _run_q4k(moe, s, seed, layer, T, mode=0, flags=0):
+    router = mode == moe.MOE_ROUTE_ROUTER
+    W = harness.device_layer(s, seed, layer, router=router, q4k=True)
+    L = moe.Layer(harness.config_for(s, mode, flags, q4k=True), W, max_tokens=T)
+    x_np = synth.activations(seed, T, s.hidden, stream=layer)
+    tok_np = synth.token_ids(seed, T, s.vocab, stream=layer)
+    x = torch.from_numpy(x_np).cuda()
+    tok = torch.from_numpy(tok_np).cuda()
+    y = L.forward(x, tok)
+    idx, w = L.route(x, tok)
+    torch.cuda.synchronize()
+    L.poll()
+    return dict(x=x_np, tok=tok_np, y=y.cpu().numpy(), idx=idx.cpu().numpy(), w=w.cpu().numpy())
+
+
+def _check_q4k(s, got, seed, layer, router=True, prenorm=False):
+    idx, w, yref, margin = harness.oracle_layer(s, seed, layer, got["x"], got["tok"], router=router, prenorm=prenorm,
+                                                q4k=True)
+    assert np.array_equal(got["idx"], idx), margin
+    assert np.allclose(got["w"], w, rtol=1e-6, atol=1e-7)
+    rel_l2, max_abs = harness.errors(got["y"], yref)
+    assert rel_l2 <= harness.GEMV_REL_L2, rel_l2
+    assert max_abs <= harness.MAX_ABS_FRAC, max_abs
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 32])
+def test_tiny_q4k_layer_matches_oracle(moe, T):
+    s = synth.workload("tiny", tokens=T)
+    _check_q4k(s, _run_q4k(moe, s, 0, 0, T), 0, 0)
+
+
+def test_tiny_q4k_hash_layer_with_prenorm_residual(moe):
+    s = synth.workload("tiny", tokens=5)
+    got = _run_q4k(moe, s, 2, 1, 5, mode=moe.MOE_ROUTE_HASH, flags=moe.MOE_FLAG_PRENORM_RESIDUAL)
+    _check_q4k(s, got, 2, 1, router=False, prenorm=True)
+
+
+def test_full_q4k_layer_one_and_eight_tokens(moe):
+    """V4-Flash shapes (3.6 GB of Q4_K routed experts)."""
+    for T, seed in ((1, 0), (8, 5)):
+        s = synth.workload("decode_t1", tokens=T)
+        _check_q4k(s, _run_q4k(moe, s, seed, 39, T), seed, 39)
+
+
+def test_q4k_layer_limits(moe):
+    s = synth.workload("tiny", tokens=40)
+    W = harness.device_layer(s, 0, 0, q4k=True)
+    L = moe.Layer(harness.config_for(s, q4k=True), W, max_tokens=40)
+    x = torch.from_numpy(synth.activations(0, 40, s.hidden)).cuda()
+    with pytest.raises(moe.MoeError) as ei:
+        L.forward(x)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    idx, _ = L.route(x)  # routing takes any T
+    torch.cuda.synchronize()
+    assert idx.shape == (40, s.top_k)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ffn_forward_noalloc(L.handle, x[:2], None, 2, torch.empty_like(x[:2]))
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
