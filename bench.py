@@ -8,7 +8,11 @@ weight sets (8 x 1.84 GB, far beyond the 126 MB L2) after warm-up calls.
 A step is one layer call.  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|quantize_q2k|quantize_q80]
+                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|decode_t1_q4k|
+                                quantize_q2k|quantize_q80]
+
+decode_t1_q4k is decode_t1 with Q4_K routed experts (the q2-q4 build's
+upgraded layers; 8 rotating weight sets of 3.6 GB).
 
 quantize_q2k / quantize_q80 time the offline encoder (moe_quantize) on
 8 x 2048 x 4096 fp32 values per step, in values/s against the HBM roofline.
@@ -48,8 +52,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_t1",
-                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "quantize_q2k",
-                            "quantize_q80"])
+                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "decode_t1_q4k",
+                            "quantize_q2k", "quantize_q80"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
@@ -228,9 +232,10 @@ def run_ours(args, world, rank):
     layers, weights = [], []
     scratch = None
     for i in range(nsets):
-        W = synth.device_layer(0, i, s)
+        W = synth.device_layer(0, i, s, q4k=s.q4k)
         cfg = moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
-                              routed_scaling=s.routed_scaling)
+                              routed_scaling=s.routed_scaling,
+                              routed_format=moe.MOE_ROUTED_Q4K if s.q4k else moe.MOE_ROUTED_Q2)
         L = moe.Layer(cfg, W, max_tokens=T, scratch=scratch)
         scratch = L.scratch
         layers.append(L)
@@ -353,7 +358,8 @@ def run_ours(args, world, rank):
                          "(inputs far larger than the 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof if large else
-        {"bound": "hbm", "kernel": "k2_experts (routed IQ2_XXS gate/up and Q2_K down, shared Q8_0 expert)",
+        {"bound": "hbm", "kernel": ("Q4_K expert kernels (input, gate/up with SwiGLU, down with the combine)" if s.q4k
+                                    else "k2_experts (routed IQ2_XXS gate/up and Q2_K down, shared Q8_0 expert)"),
          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
          "traffic": load_traffic(args.workload), "traffic_unit": "bytes per launch (ncu)",
          "peak_source": peaks["source"],
@@ -363,7 +369,9 @@ def run_ours(args, world, rank):
          "achieved_gbs": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"], "distinct_experts_per_call": n_distinct},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 4,
                 "d2h_bytes_per_step": T * s.hidden * 4},
-        "gpu_launches": (12 if large else 2) * args.steps,
+        # batched: router (4), permutation (3), input, 4 GEMMs; small-token: k1 and
+        # k2, or for Q4_K layers k1, the routing kernel and the 3 expert kernels
+        "gpu_launches": (12 if large else 5 if s.q4k else 2) * args.steps,
         "clocks": clocks,
     }
     return out
@@ -466,7 +474,7 @@ def oracle_rate(s: synth.LayerShape, budget_s: float, max_steps: int, seed: int 
     """Tokens/s of the fp64 oracle on full layer calls of the workload
     (weight set 0, inputs resident), as many calls as fit in the budget."""
     import oracle
-    W = synth.host_layer(seed, 0, s)
+    W = synth.host_layer(seed, 0, s, q4k=s.q4k)
     Wr, b = W["router_w"], W["bias"]
     T = min(s.tokens, 4)  # large batches: a 4-token slice per oracle call
     n = 0
@@ -505,9 +513,9 @@ class OracleSampler:
         self.Wr = synth.router_weight(seed, 0, s.n_experts, s.hidden)
         b = synth.bias(seed, 0, s.n_experts, s.skew)
         self.idx, self.w, _ = oracle.route(self.x, self.Wr, b, s.top_k, s.routed_scaling)
-        self.W = synth.host_layer(seed, 0, s, experts=np.unique(self.idx))
+        self.W = synth.host_layer(seed, 0, s, experts=np.unique(self.idx), q4k=s.q4k)
         g = self.W["grid"]
-        K2, KQ, K8 = synth.KIND_IQ2XXS, synth.KIND_Q2K, synth.KIND_Q80
+        K2, K8 = self.W["gate_kind"], synth.KIND_Q80
         self.h, self.hs = {}, []
         for t in range(self.T):
             xt = self.x[t]
@@ -524,7 +532,7 @@ class OracleSampler:
 
     def step(self):
         o, s, g = self.o, self.s, self.W["grid"]
-        K2, KQ, K8 = synth.KIND_IQ2XXS, synth.KIND_Q2K, synth.KIND_Q80
+        K2, KQ, K8 = self.W["gate_kind"], self.W["down_kind"], synth.KIND_Q80
         c, F = self.c % self.F, self.F
         nE, nI, nH, nS = s.n_experts // F, s.inter // F, s.hidden // F, s.shared_inter // F
         rE, rI, rH, rS = (slice(c * n, (c + 1) * n) for n in (nE, nI, nH, nS))

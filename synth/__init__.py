@@ -20,6 +20,7 @@ decode_t1          4096   2048  2048  256  6   1      8 rotating weight sets
 decode_t32         4096   2048  2048  256  6   32     bias +0.5 on e % 8 == 0
 prefill_t4096      4096   2048  2048  256  6   4096   bias +0.5 on e % 8 == 0
 stack43_t8         4096   2048  2048  256  6   8      43 layers, 0-2 hashed
+decode_t1_q4k      4096   2048  2048  256  6   1      Q4_K routed experts
 =================  =====  ====  ====  ===  ==  =====  ======================
 """
 from __future__ import annotations
@@ -55,17 +56,26 @@ class LayerShape:
     layers: int = 1
     hash_layers: int = 0
     weight_sets: int = 1
+    q4k: bool = False  # routed experts in Q4_K (the q2-q4 build's upgraded layers)
 
     def row_bytes(self, kind: int, cols: int) -> int:
         return cols // BLOCK_ELEMS[kind] * BLOCK_BYTES[kind]
 
     @property
+    def gate_kind(self) -> int:
+        return KIND_Q4K if self.q4k else KIND_IQ2XXS
+
+    @property
+    def down_kind(self) -> int:
+        return KIND_Q4K if self.q4k else KIND_Q2K
+
+    @property
     def gate_bytes_per_expert(self) -> int:
-        return self.inter * self.row_bytes(KIND_IQ2XXS, self.hidden)
+        return self.inter * self.row_bytes(self.gate_kind, self.hidden)
 
     @property
     def down_bytes_per_expert(self) -> int:
-        return self.hidden * self.row_bytes(KIND_Q2K, self.inter)
+        return self.hidden * self.row_bytes(self.down_kind, self.inter)
 
     @property
     def expert_bytes(self) -> int:
@@ -83,6 +93,7 @@ WORKLOADS = {
     "decode_t32": LayerShape(4096, 2048, 2048, 256, 6, 32, skew=True),
     "prefill_t4096": LayerShape(4096, 2048, 2048, 256, 6, 4096, skew=True),
     "stack43_t8": LayerShape(4096, 2048, 2048, 256, 6, 8, layers=43, hash_layers=3),
+    "decode_t1_q4k": LayerShape(4096, 2048, 2048, 256, 6, 1, weight_sets=8, q4k=True),
 }
 
 
