@@ -8,11 +8,12 @@ weight sets (8 x 1.84 GB, far beyond the 126 MB L2) after warm-up calls.
 A step is one layer call.  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|decode_t1_q4k|
-                                quantize_q2k|quantize_q80]
+                    [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|stack43_t8_q2q4|
+                                decode_t1_q4k|quantize_q2k|quantize_q80]
 
 decode_t1_q4k is decode_t1 with Q4_K routed experts (the q2-q4 build's
-upgraded layers; 8 rotating weight sets of 3.6 GB).
+upgraded layers; 8 rotating weight sets of 3.6 GB); stack43_t8_q2q4 is the
+43-layer stack with layers 37-42 in Q4_K.
 
 quantize_q2k / quantize_q80 time the offline encoder (moe_quantize) on
 8 x 2048 x 4096 fp32 values per step, in values/s against the HBM roofline.
@@ -52,8 +53,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_t1",
-                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "decode_t1_q4k",
-                            "quantize_q2k", "quantize_q80"])
+                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "stack43_t8_q2q4",
+                            "decode_t1_q4k", "quantize_q2k", "quantize_q80"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
@@ -379,7 +380,8 @@ def run_ours(args, world, rank):
 
 def run_stack(args, world, rank):
     """43 chained layers at T=8 (layers 0-2 hash-routed), x <- x + MoE(RMSNorm(x));
-    a step is one pass through the whole stack."""
+    a step is one pass through the whole stack.  stack43_t8_q2q4 keeps the
+    routed experts of its last six layers in Q4_K."""
     import torch
 
     import bit_moe_expert_sqrtsoftplus_b200 as moe
@@ -389,11 +391,13 @@ def run_stack(args, world, rank):
     layers, scratch = [], None
     for l in range(s.layers):
         router = l >= s.hash_layers
-        W = synth.device_layer(0, l, s, router=router)
+        sl = s.layer_shape(l)
+        W = synth.device_layer(0, l, sl, router=router, q4k=sl.q4k)
         cfg = moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
                               routed_scaling=s.routed_scaling, rms_eps=1e-6,
                               mode=moe.MOE_ROUTE_ROUTER if router else moe.MOE_ROUTE_HASH,
-                              flags=moe.MOE_FLAG_PRENORM_RESIDUAL)
+                              flags=moe.MOE_FLAG_PRENORM_RESIDUAL,
+                              routed_format=moe.MOE_ROUTED_Q4K if sl.q4k else moe.MOE_ROUTED_Q2)
         L = moe.Layer(cfg, W, max_tokens=T, scratch=scratch)
         scratch = L.scratch
         layers.append(L)
@@ -415,7 +419,8 @@ def run_stack(args, world, rank):
     for l, L in enumerate(layers):
         idx, _ = L.route(x, tok)
         nd = len(np.unique(idx.cpu().numpy()))
-        nd_bytes += nd * s.expert_bytes + s.shared_bytes + (s.n_experts * s.hidden * 2 if l >= s.hash_layers else 0)
+        nd_bytes += (nd * s.layer_shape(l).expert_bytes + s.shared_bytes +
+                     (s.n_experts * s.hidden * 2 if l >= s.hash_layers else 0))
         L.forward(x, tok, y=x)
     stream = torch.cuda.current_stream()
     clock = ClockSampler(torch.cuda.current_device())
@@ -460,12 +465,14 @@ def run_stack(args, world, rank):
                    "l2": f"{s.layers} distinct layer weight sets ({s.layers * s.n_experts * s.expert_bytes / 1e9:.1f} "
                          "GB, far larger than the 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "whole stack step (43 x k1/k2)", "achieved": gbs,
+        "roofline": {"bound": "hbm", "kernel": (f"whole stack step ({s.layers - s.q4k_layers} x k1/k2"
+                                              + (f", {s.q4k_layers} Q4_K layers x 5 launches)" if s.q4k_layers
+                                                 else ")")), "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": peaks["source"], "algorithmic_bytes_per_step": nd_bytes},
         "e2e": {"value": job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * s.hidden * 4, "d2h_bytes_per_step": T * s.hidden * 4},
-        "gpu_launches": 2 * s.layers * args.steps,
+        "gpu_launches": (2 * (s.layers - s.q4k_layers) + 5 * s.q4k_layers) * args.steps,
         "clocks": clock.summary(),
     }
 
@@ -772,7 +779,7 @@ def main():
         return
     if args.workload.startswith("quantize_"):
         out = run_quant(args, world, rank)
-    elif args.workload == "stack43_t8":
+    elif args.workload.startswith("stack"):
         out = run_stack(args, world, rank)
     else:
         out = run_ours(args, world, rank)

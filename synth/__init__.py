@@ -21,6 +21,7 @@ decode_t32         4096   2048  2048  256  6   32     bias +0.5 on e % 8 == 0
 prefill_t4096      4096   2048  2048  256  6   4096   bias +0.5 on e % 8 == 0
 stack43_t8         4096   2048  2048  256  6   8      43 layers, 0-2 hashed
 decode_t1_q4k      4096   2048  2048  256  6   1      Q4_K routed experts
+stack43_t8_q2q4    4096   2048  2048  256  6   8      stack43_t8, layers 37-42 Q4_K
 =================  =====  ====  ====  ===  ==  =====  ======================
 """
 from __future__ import annotations
@@ -57,6 +58,12 @@ class LayerShape:
     hash_layers: int = 0
     weight_sets: int = 1
     q4k: bool = False  # routed experts in Q4_K (the q2-q4 build's upgraded layers)
+    q4k_layers: int = 0  # in a stack: the last q4k_layers layers have Q4_K routed experts
+
+    def layer_shape(self, layer: int) -> "LayerShape":
+        """The shape of one layer of a stack (its routed format included)."""
+        q4k = self.q4k or layer >= self.layers - self.q4k_layers
+        return replace(self, q4k=q4k, q4k_layers=0)
 
     def row_bytes(self, kind: int, cols: int) -> int:
         return cols // BLOCK_ELEMS[kind] * BLOCK_BYTES[kind]
@@ -94,6 +101,7 @@ WORKLOADS = {
     "prefill_t4096": LayerShape(4096, 2048, 2048, 256, 6, 4096, skew=True),
     "stack43_t8": LayerShape(4096, 2048, 2048, 256, 6, 8, layers=43, hash_layers=3),
     "decode_t1_q4k": LayerShape(4096, 2048, 2048, 256, 6, 1, weight_sets=8, q4k=True),
+    "stack43_t8_q2q4": LayerShape(4096, 2048, 2048, 256, 6, 8, layers=43, hash_layers=3, q4k_layers=6),
 }
 
 

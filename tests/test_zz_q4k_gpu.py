@@ -96,3 +96,31 @@ def test_q4k_layer_limits(moe):
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_ffn_forward_noalloc(L.handle, x[:2], None, 2, torch.empty_like(x[:2]))
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_q2q4_stack_tail_teacher_forced(moe):
+    """Layers 35-42 of the q2-q4 stack (37-42 with Q4_K routed experts) at
+    T = 8 with the pre-norm residual, each checked against the oracle on the
+    GPU's own input to that layer."""
+    import os
+    s = synth.workload("stack43_t8_q2q4")
+    seed, T = 0, s.tokens
+    threads = max(1, min(32, os.cpu_count() or 1))
+    x0 = synth.activations(seed, T, s.hidden, stream=4343)
+    x = torch.from_numpy(x0).cuda()
+    tok = synth.token_ids(seed, T, s.vocab, stream=4343)
+    tokd = torch.from_numpy(tok).cuda()
+    for l in range(35, s.layers):
+        sl = s.layer_shape(l)
+        W = synth.device_layer(seed, l, sl, q4k=sl.q4k)
+        L = moe.Layer(harness.config_for(sl, None, moe.MOE_FLAG_PRENORM_RESIDUAL, q4k=sl.q4k), W, max_tokens=T)
+        xin = x.cpu().numpy()
+        idx, _ = L.route(x, tokd)
+        x = L.forward(x, tokd, y=x)
+        torch.cuda.synchronize()
+        L.poll()
+        ridx, _, yref, margin = harness.oracle_layer(sl, seed, l, xin, tok, prenorm=True, threads=threads, q4k=sl.q4k)
+        assert np.array_equal(idx.cpu().numpy(), ridx), (l, margin)
+        rel, mx = harness.errors(x.cpu().numpy(), yref)
+        assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (l, rel, mx)
+        del L, W
