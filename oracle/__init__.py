@@ -67,7 +67,7 @@ def lib():
         L.oracle_rmsnorm.argtypes = [vp, i32, d, vp]
         L.oracle_f32_to_f16.argtypes = [ctypes.c_float]
         L.oracle_f32_to_f16.restype = ctypes.c_uint16
-        for name in ("oracle_quantize_q80", "oracle_quantize_q2k"):
+        for name in ("oracle_quantize_q80", "oracle_quantize_q2k", "oracle_quantize_q4k"):
             getattr(L, name).argtypes = [vp, i32, vp]
             getattr(L, name).restype = i32
         _lib = L
@@ -286,16 +286,17 @@ def f32_to_f16(f: float) -> int:
 
 
 def quantize(kind: int, x: np.ndarray) -> np.ndarray:
-    """Encode fp32 values (a multiple of the block size) into Q8_0 or Q2_K
-    blocks: uint8 [n_blocks][block_bytes].  Raises on non-finite input."""
-    if kind not in (KIND_Q80, KIND_Q2K):
-        raise ValueError("only the Q8_0 and Q2_K encoders exist")
+    """Encode fp32 values (a multiple of the block size) into Q8_0, Q2_K or
+    Q4_K blocks: uint8 [n_blocks][block_bytes].  Raises on non-finite input."""
+    if kind not in (KIND_Q80, KIND_Q2K, KIND_Q4K):
+        raise ValueError("only the Q8_0, Q2_K and Q4_K encoders exist")
     xx, px = _c(np.asarray(x, dtype=np.float32).ravel(), np.float32)
     n = xx.size
     if n % _BE[kind]:
         raise ValueError(f"{n} values is not a multiple of {_BE[kind]}")
     out = np.zeros((n // _BE[kind], _BB[kind]), dtype=np.uint8)
-    fn = lib().oracle_quantize_q80 if kind == KIND_Q80 else lib().oracle_quantize_q2k
+    fn = {KIND_Q80: lib().oracle_quantize_q80, KIND_Q2K: lib().oracle_quantize_q2k,
+          KIND_Q4K: lib().oracle_quantize_q4k}[kind]
     rc = fn(px, n, out.ctypes.data)
     if rc != 0:
         raise ValueError("non-finite input" if rc == -1 else f"encoder error {rc}")

@@ -575,3 +575,60 @@ int oracle_quantize_q2k(const float *x, int n, uint8_t *out) {
   }
   return 0;
 }
+
+/*
+ * Q4_K encoder: the same estimator one level up (reading, as for Q2_K): for
+ * every 32-value sub-block j, lo = min(0, min x), hi = max x, scale = (hi -
+ * lo) / 15 (sixteen codes span the range), min = 0 - lo; d = f16(max scale /
+ * 63) and dmin = f16(max min / 63); sc = clamp(rint(scale / d), 0, 63), m =
+ * clamp(rint(min / dmin), 0, 63); q = clamp(rint((x + dmin*m) / (d*sc)), 0, 15);
+ * packed in the Q4_K layout read above.  Decisions in binary32, ties to even.
+ */
+int oracle_quantize_q4k(const float *x, int n, uint8_t *out) {
+  if (n < 0 || n % 256) return -2;
+  for (int b = 0; b < n / 256; ++b) {
+    const float *v = x + (size_t)b * 256;
+    uint8_t *blk = out + (size_t)b * 144;
+    memset(blk, 0, 144);
+    float scale[8], mn[8], maxs = 0.0f, maxm = 0.0f;
+    for (int j = 0; j < 8; ++j) {
+      float lo = 0.0f, hi = -INFINITY;
+      for (int i = 0; i < 32; ++i) {
+        const float t = v[32 * j + i];
+        if (!isfinite(t)) return -1;
+        if (t < lo) lo = t;
+        if (t > hi) hi = t;
+      }
+      scale[j] = (hi - lo) / 15.0f;
+      mn[j] = 0.0f - lo;
+      if (scale[j] > maxs) maxs = scale[j];
+      if (mn[j] > maxm) maxm = mn[j];
+    }
+    const uint16_t dh = oracle_f32_to_f16(maxs / 63.0f), mh = oracle_f32_to_f16(maxm / 63.0f);
+    const float dq = (float)oracle_f16(dh), mq = (float)oracle_f16(mh);
+    put16(blk, dh);
+    put16(blk + 2, mh);
+    uint8_t *sm = blk + 4;
+    for (int j = 0; j < 8; ++j) {
+      const float sc = dq > 0.0f ? clampf(rintf(scale[j] / dq), 0.0f, 63.0f) : 0.0f;
+      const float m = mq > 0.0f ? clampf(rintf(mn[j] / mq), 0.0f, 63.0f) : 0.0f;
+      const int isc = (int)sc, im = (int)m;
+      if (j < 4) {
+        sm[j] |= (uint8_t)isc;
+        sm[j + 4] |= (uint8_t)im;
+      } else {
+        sm[j + 4] |= (uint8_t)((isc & 15) | ((im & 15) << 4));
+        sm[j - 4] |= (uint8_t)((isc >> 4) << 6);
+        sm[j] |= (uint8_t)((im >> 4) << 6);
+      }
+      const float step = dq * sc, off = mq * m;
+      for (int i = 0; i < 32; ++i) {
+        const int e = 32 * j + i;
+        float q = 0.0f;
+        if (step > 0.0f) q = clampf(rintf((v[e] + off) / step), 0.0f, 15.0f);
+        blk[16 + 32 * (e / 64) + e % 32] |= (uint8_t)((int)q << (4 * ((e % 64) / 32)));
+      }
+    }
+  }
+  return 0;
+}

@@ -99,11 +99,12 @@ void oracle_permutation(const int32_t *idx, int T, int k, int E, int32_t *offset
 void oracle_rmsnorm(const double *x, int H, double eps, double *out);
 
 /* Encoders (binary32 decisions, see oracle.c).  n is a multiple of the block
- * size (32 / 256); out receives n/32 34-byte / n/256 84-byte blocks.  Return
- * 0, -1 for a non-finite input, -2 for a bad n. */
+ * size (32 / 256 / 256); out receives n/32 34-byte, n/256 84-byte or n/256
+ * 144-byte blocks.  Return 0, -1 for a non-finite input, -2 for a bad n. */
 uint16_t oracle_f32_to_f16(float f);
 int oracle_quantize_q80(const float *x, int n, uint8_t *out);
 int oracle_quantize_q2k(const float *x, int n, uint8_t *out);
+int oracle_quantize_q4k(const float *x, int n, uint8_t *out);
 
 #ifdef __cplusplus
 }

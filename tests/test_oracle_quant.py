@@ -1,4 +1,4 @@
-"""Pins of the oracle's block encoders (Q8_0, Q2_K) and its binary32 ->
+"""Pins of the oracle's block encoders (Q8_0, Q2_K, Q4_K) and its binary32 ->
 binary16 rounding, each against something other than the encoder's own
 formula: every binary16 code, numpy's conversion, blocks built so that the
 encoder must return them byte for byte, brute-force nearest codes through the
@@ -207,3 +207,90 @@ def test_q2k_closed_forms():
     x[300] = np.nan
     with pytest.raises(ValueError):
         oracle.quantize(KQ, x)
+
+
+# --------------------------------------------------------------------- Q4_K
+
+K4 = oracle.KIND_Q4K
+
+
+def _q4k_block(dh: int, mh: int, sc, mn, codes) -> np.ndarray:
+    from tests.test_oracle_q4k import _pack
+    return _pack(dh, mh, sc, mn, codes)
+
+
+def test_q4k_exact_blocks_come_back_byte_for_byte():
+    """Sub-blocks with a non-zero scale hold codes 0 and 15, scale 63 and (when
+    there are mins) min 63 occur, and d, dmin have 3 significant bits within
+    a few binades of each other: every step the encoder takes is exact, so it
+    must return the block it was given."""
+    rng = np.random.default_rng(13)
+    for trial in range(300):
+        dh = _short_f16(rng, -8, -4)
+        with_min = trial % 3 != 0
+        mh = _short_f16(rng, -8, -4) if with_min else 0
+        sc = rng.integers(0, 64, 8)
+        m = rng.integers(0, 64, 8) if with_min else np.zeros(8, np.int64)
+        sc[rng.integers(0, 8)] = 63
+        if with_min:
+            m[rng.integers(0, 8)] = 63
+        codes = rng.integers(0, 16, 256)
+        for j in range(8):
+            if sc[j] == 0:
+                codes[32 * j:32 * j + 32] = 0
+            else:
+                p0, p15 = rng.choice(32, 2, replace=False)
+                codes[32 * j + p0], codes[32 * j + p15] = 0, 15
+        blk = _q4k_block(dh, mh, sc, m, codes)
+        x64 = oracle.decode_row(K4, blk, 256)
+        x = x64.astype(np.float32)
+        assert np.array_equal(x.astype(np.float64), x64)  # exact in fp32
+        got = oracle.quantize(K4, x)[0]
+        assert np.array_equal(got, blk), (trial, np.nonzero(got != blk)[0][:8])
+
+
+def _with_q4k_code(blk: np.ndarray, e: int, q: int) -> np.ndarray:
+    b = blk.copy()
+    byte, shift = 16 + 32 * (e // 64) + e % 32, 4 * ((e % 64) // 32)
+    b[byte] = (int(b[byte]) & ~(15 << shift) & 0xFF) | (q << shift)
+    return b
+
+
+def test_q4k_codes_are_the_nearest_of_the_sixteen():
+    rng = np.random.default_rng(14)
+    for scale, shift in ((1.0, 0.0), (0.05, 0.03), (10.0, -4.0)):
+        x = (rng.standard_normal(256) * scale + shift).astype(np.float32)
+        blk = oracle.quantize(K4, x)[0]
+        for e in range(0, 256, 5):
+            vals = np.array([oracle.q4k_elem(_with_q4k_code(blk, e, q), e) for q in range(16)])
+            dist = np.abs(vals - float(x[e]))
+            assert dist[oracle.q4k_elem(blk, e) == vals].min() <= dist.min() * (1 + 1e-5) + 1e-12, e
+
+
+def test_q4k_widest_sub_block_takes_the_top_values_and_error_level():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal(256 * 64).astype(np.float32)
+    blocks = oracle.quantize(K4, x)
+    for blk in blocks[:50]:
+        sc = [oracle.q4k_elem(_with_q4k_code(blk, 32 * j, 1), 32 * j) - oracle.q4k_elem(_with_q4k_code(blk, 32 * j, 0),
+                                                                                      32 * j) for j in range(8)]
+        d = oracle.f16(int(blk[0]) | int(blk[1]) << 8)
+        assert round(max(sc) / d) == 63  # the widest range/15 is d*63
+    y = np.concatenate([oracle.decode_row(K4, b, 256) for b in blocks])
+    rel = np.sqrt(np.mean((x - y) ** 2)) / np.std(x)
+    assert 0.05 < rel < 0.11, rel  # 16 levels over ~4.1 sigma: step/sqrt(12) ~ 0.079
+
+
+def test_q4k_closed_forms():
+    assert not oracle.quantize(K4, np.zeros(256, np.float32)).any()
+    # constants whose base c/945 (codes 15 at scale 63) is a normal binary16,
+    # so the only rounding is d's 11 significant bits
+    for c in (0.75, 0.1, 123.0):
+        y = oracle.decode_row(K4, oracle.quantize(K4, np.full(256, c, np.float32))[0], 256)
+        assert np.allclose(y, c, rtol=2.0 ** -10)
+        y = oracle.decode_row(K4, oracle.quantize(K4, np.full(256, -c, np.float32))[0], 256)
+        assert np.allclose(y, -c, rtol=2.0 ** -10)
+    x = np.zeros(512, np.float32)
+    x[300] = np.inf
+    with pytest.raises(ValueError):
+        oracle.quantize(K4, x)
