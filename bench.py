@@ -9,7 +9,7 @@ A step is one layer call.  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload decode_t1|decode_t32|prefill_t4096|stack43_t8|stack43_t8_q2q4|
-                                decode_t1_q4k|quantize_q2k|quantize_q80]
+                                decode_t1_q4k|quantize_q2k|quantize_q80|quantize_q4k]
 
 decode_t1_q4k is decode_t1 with Q4_K routed experts (the q2-q4 build's
 upgraded layers; 8 rotating weight sets of 3.6 GB); stack43_t8_q2q4 is the
@@ -54,7 +54,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_t1",
                    choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "stack43_t8_q2q4",
-                            "decode_t1_q4k", "quantize_q2k", "quantize_q80"])
+                            "decode_t1_q4k", "quantize_q2k", "quantize_q80", "quantize_q4k"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
@@ -571,7 +571,7 @@ QUANT_METRIC = "encoded values/s (offline Q2_K / Q8_0 encoder) and % HBM rooflin
 
 def quant_format(workload: str):
     """(binary format id, values per block, bytes per block) of an encoder workload."""
-    return (1, 256, 84) if workload == "quantize_q2k" else (0, 32, 34)
+    return {"quantize_q2k": (1, 256, 84), "quantize_q4k": (2, 256, 144)}.get(workload, (0, 32, 34))
 
 
 def run_quant(args, world, rank):
@@ -629,10 +629,10 @@ def run_quant(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (N(0, 0.02^2) fp32 values from torch's generator)",
         "config": {"workload": f"{args.workload}: {QUANT_MATS} x {QUANT_ROWS} x {QUANT_COLS} fp32 values per step "
-                               f"-> {'Q2_K' if per == 256 else 'Q8_0'} blocks",
+                               f"-> {args.workload[len('quantize_'):].upper().replace('Q80', 'Q8_0')} blocks",
                    "l2": f"{n * 4 / 1e6:.0f} MB of input per step, beyond the 126 MB L2",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": f"k_quantize_{'q2k' if per == 256 else 'q80'}", "achieved": gbs,
+        "roofline": {"bound": "hbm", "kernel": f"k_{args.workload}", "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "traffic": load_traffic(args.workload), "traffic_unit": "bytes per launch (ncu)",
                      "peak_source": peaks["source"], "algorithmic_bytes_per_launch": bytes_launch,
@@ -648,7 +648,7 @@ def oracle_quant_rate(workload: str, steps: int, warmup: int, values_per_step: i
     """Values/s of the oracle's encoder on steps of 2^20 values."""
     import oracle
     fmt, per, _ = quant_format(workload)
-    kind = oracle.KIND_Q2K if per == 256 else oracle.KIND_Q80
+    kind = {0: oracle.KIND_Q80, 1: oracle.KIND_Q2K, 2: oracle.KIND_Q4K}[fmt]
     x = (np.random.default_rng(7).standard_normal(values_per_step) * 0.02).astype(np.float32)
     for _ in range(warmup):
         oracle.quantize(kind, x)

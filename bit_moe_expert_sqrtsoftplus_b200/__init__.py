@@ -31,6 +31,8 @@ MOE_FLAG_PRENORM_RESIDUAL = 1
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
 MOE_QUANT_Q8_0 = 0
 MOE_QUANT_Q2_K = 1
+MOE_QUANT_Q4_K = 2
+_QUANT_BLOCK = {MOE_QUANT_Q8_0: (32, 34), MOE_QUANT_Q2_K: (256, 84), MOE_QUANT_Q4_K: (256, 144)}
 MOE_ROUTED_Q2 = 0
 MOE_ROUTED_Q4K = 1
 
@@ -162,8 +164,9 @@ def moe_set_timing_events(handle, ev_begin=None, ev_end=None):
 
 def moe_quantize(fmt, x, out, nonfinite=None, stream=None):
     """Encode the fp32 CUDA tensor x (numel a multiple of the block size) into
-    the uint8 CUDA tensor out (numel/32 * 34 or numel/256 * 84 bytes)."""
-    per, nbytes = (32, 34) if fmt == MOE_QUANT_Q8_0 else (256, 84)
+    the uint8 CUDA tensor out (numel/32 * 34, numel/256 * 84 or numel/256 *
+    144 bytes)."""
+    per, nbytes = _QUANT_BLOCK.get(fmt, (32, 34))
     if out.numel() * out.element_size() < x.numel() // per * nbytes:
         raise MoeError(MOE_ERR_WORKSPACE_TOO_SMALL, "out is too small for the encoded blocks")
     _check(lib().moe_quantize(fmt, _ptr(x), x.numel(), _ptr(out), _ptr(nonfinite), _stream(stream)))
@@ -173,7 +176,7 @@ def quantize(fmt, x, stream=None):
     """Encoded blocks of x as a uint8 CUDA tensor [n_blocks][block_bytes] and a
     device int32 count of blocks that held a non-finite value."""
     import torch
-    per, nbytes = (32, 34) if fmt == MOE_QUANT_Q8_0 else (256, 84)
+    per, nbytes = _QUANT_BLOCK.get(fmt, (32, 34))
     x = x.contiguous()
     out = torch.empty((x.numel() // per, nbytes), dtype=torch.uint8, device=x.device)
     bad = torch.zeros(1, dtype=torch.int32, device=x.device)

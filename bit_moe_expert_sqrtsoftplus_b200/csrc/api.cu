@@ -457,7 +457,7 @@ moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end) {
 
 moe_status moe_quantize(int format, const float *x, int64_t n, void *out, int32_t *nonfinite_blocks,
                         moe_stream_t stream) {
-  if (format != MOE_QUANT_Q8_0 && format != MOE_QUANT_Q2_K)
+  if (format != MOE_QUANT_Q8_0 && format != MOE_QUANT_Q2_K && format != MOE_QUANT_Q4_K)
     return fail(MOE_ERR_INVALID_ARG, "format=%d is not a MOE_QUANT_* format", format);
   if (n < 0) return fail(MOE_ERR_INVALID_ARG, "n=%lld is negative", (long long)n);
   const int per = format == MOE_QUANT_Q8_0 ? 32 : 256;

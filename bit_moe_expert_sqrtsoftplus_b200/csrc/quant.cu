@@ -1,4 +1,4 @@
-// quant.cu -- offline encoders: fp32 values -> Q8_0 / Q2_K blocks (sm_100a).
+// quant.cu -- offline encoders: fp32 values -> Q8_0 / Q2_K / Q4_K blocks (sm_100a).
 //
 // The Q2_K writer's steps ("2bit 量子化はなぜ「冗談ではない」のか", section 3
 // "Q2_K: 256 要素を 84 バイトにする K-quant"): a scale and a min for every
@@ -16,8 +16,11 @@
 //         min = 0 - lo;  d = f16(max scale / 15), dmin = f16(max min / 15);
 //         sc = clamp(rint(scale / d), 0, 15), m = clamp(rint(min / dmin), 0, 15);
 //         q = clamp(rint((x + dmin*m) / (d*sc)), 0, 3)
+//   Q4_K  the same as Q2_K one level up: 32-value sub-blocks, scale =
+//         (hi - lo) / 15, bases max / 63, 6-bit scales and mins, codes 0..15,
+//         in the Q4_K layout (see k_quantize_q4k)
 // where a zero base gives zero nibbles and a zero step zero codes.  The
-// decoded value is d*q (Q8_0) and d*sc*q - dmin*m (Q2_K).
+// decoded value is d*q (Q8_0) and d*sc*q - dmin*m (Q2_K, Q4_K).
 //
 // One warp encodes one block per loop trip.  Q2_K: lane l holds elements
 // 32i + l (i = 0..7), so element 32i + l lies in sub-block 2i + l/16 (a
@@ -135,6 +138,88 @@ __global__ void __launch_bounds__(kQuantWarps * kWarp) k_quantize_q2k(const floa
   }
 }
 
+// Q4_K (the same estimator one level up, 32-value sub-blocks, sixteen codes,
+// 6-bit scales and mins under f16 bases of max/63, the Q4_K layout: d, dmin,
+// 12 bytes of scales and mins, 128 bytes of codes).  Lane l holds values
+// 8l .. 8l+7: sub-block l/4 (four lanes reduce its range), code bytes
+// 32*(l/8) + 8*(l%4) .. +7, nibble (l%8)/4, so lanes l and l+4 fill the same
+// eight bytes and one shuffle joins them.
+__global__ void __launch_bounds__(kQuantWarps * kWarp) k_quantize_q4k(const float *__restrict__ x, int64_t nblocks,
+                                                                     uint8_t *__restrict__ out, int32_t *nonfinite) {
+  __shared__ __align__(16) uint8_t stage[kQuantWarps][144];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint8_t *st = stage[w];
+  for (int64_t b = (int64_t)blockIdx.x * kQuantWarps + w; b < nblocks; b += (int64_t)gridDim.x * kQuantWarps) {
+    const float4 *xb = reinterpret_cast<const float4 *>(x + b * 256 + 8 * lane);
+    const float4 a0 = xb[0], a1 = xb[1];
+    const float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    bool bad = false;
+    float lo = 0.0f, hi = v[0];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      bad |= !isfinite(v[k]);
+      lo = fminf(lo, v[k]);
+      hi = fmaxf(hi, v[k]);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    const float scale = __fdiv_rn(__fsub_rn(hi, lo), 15.0f), mn = __fsub_rn(0.0f, lo);
+    float maxs = scale, maxm = mn;
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      maxs = fmaxf(maxs, __shfl_xor_sync(0xffffffffu, maxs, o));
+      maxm = fmaxf(maxm, __shfl_xor_sync(0xffffffffu, maxm, o));
+    }
+    maxs = fmaxf(maxs, 0.0f);
+    const uint16_t dh = bad ? 0 : f16_rn_bits(__fdiv_rn(maxs, 63.0f));
+    const uint16_t mh = bad ? 0 : f16_rn_bits(__fdiv_rn(maxm, 63.0f));
+    const float dq = f16_value(dh), mq = f16_value(mh);
+    const float sc = dq > 0.0f ? clamp_rint(__fdiv_rn(scale, dq), 0.0f, 63.0f) : 0.0f;
+    const float m = mq > 0.0f ? clamp_rint(__fdiv_rn(mn, mq), 0.0f, 63.0f) : 0.0f;
+    const float step = __fmul_rn(dq, sc), off = __fmul_rn(mq, m);
+    uint32_t codes = 0;  // eight 4-bit codes, value 8l+k in bits 4k..4k+3
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float q = 0.0f;
+      if (step > 0.0f) q = clamp_rint(__fdiv_rn(__fadd_rn(v[k], off), step), 0.0f, 15.0f);
+      codes |= (uint32_t)(int)q << (4 * k);
+    }
+    const uint32_t upper = __shfl_down_sync(0xffffffffu, codes, 4);  // lane l+4: the high nibbles
+    if ((lane & 7) < 4) {
+      uint8_t *dst = st + 16 + 32 * (lane >> 3) + 8 * (lane & 3);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dst[k] = (uint8_t)(((codes >> (4 * k)) & 15u) | (((upper >> (4 * k)) & 15u) << 4));
+    }
+    // the eight (scale, min) pairs, from lanes 0, 4, ..., 28
+    int scj[8], mj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      scj[j] = __shfl_sync(0xffffffffu, (int)sc, 4 * j);
+      mj[j] = __shfl_sync(0xffffffffu, (int)m, 4 * j);
+    }
+    if (lane == 0) {
+      st[0] = (uint8_t)(dh & 0xff);
+      st[1] = (uint8_t)(dh >> 8);
+      st[2] = (uint8_t)(mh & 0xff);
+      st[3] = (uint8_t)(mh >> 8);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        st[4 + j] = (uint8_t)(scj[j] | ((scj[j + 4] >> 4) << 6));
+        st[8 + j] = (uint8_t)(mj[j] | ((mj[j + 4] >> 4) << 6));
+        st[12 + j] = (uint8_t)((scj[j + 4] & 15) | ((mj[j + 4] & 15) << 4));
+      }
+      if (bad && nonfinite) atomicAdd(nonfinite, 1);
+    }
+    __syncwarp();
+    if (lane < 9) reinterpret_cast<uint4 *>(out + b * 144)[lane] = reinterpret_cast<const uint4 *>(st)[lane];
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 cudaError_t quantize_blocks(int format, const float *x, int64_t nblocks, void *out, int32_t *nonfinite,
@@ -146,8 +231,10 @@ cudaError_t quantize_blocks(int format, const float *x, int64_t nblocks, void *o
   uint8_t *o = static_cast<uint8_t *>(out);
   if (format == kQuantQ80)
     k_quantize_q80<<<grid, kQuantWarps * kWarp, 0, stream>>>(x, nblocks, o, nonfinite);
-  else
+  else if (format == kQuantQ2K)
     k_quantize_q2k<<<grid, kQuantWarps * kWarp, 0, stream>>>(x, nblocks, o, nonfinite);
+  else
+    k_quantize_q4k<<<grid, kQuantWarps * kWarp, 0, stream>>>(x, nblocks, o, nonfinite);
   return cudaGetLastError();
 }
 

@@ -77,6 +77,7 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 /* block formats of moe_quantize */
 #define MOE_QUANT_Q8_0 0 /* 32 values in 34 bytes */
 #define MOE_QUANT_Q2_K 1 /* 256 values in 84 bytes */
+#define MOE_QUANT_Q4_K 2 /* 256 values in 144 bytes (the Q4_K layout of MOE_ROUTED_Q4K) */
 
 typedef struct {
   int hidden;           /* H: multiple of 256 (4096 for V4-Flash) */
@@ -204,8 +205,9 @@ moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end);
 
 /*
  * Offline encoder: n fp32 values -> blocks of `format` (MOE_QUANT_Q8_0: n a
- * multiple of 32, n/32 blocks of 34 bytes; MOE_QUANT_Q2_K: n a multiple of
- * 256, n/256 blocks of 84 bytes), the writer side of the formats the layer
+ * multiple of 32, n/32 blocks of 34 bytes; MOE_QUANT_Q2_K / MOE_QUANT_Q4_K: n
+ * a multiple of 256, n/256 blocks of 84 / 144 bytes), the writer side of the
+ * formats the layer
  * reads ("2bit 量子化はなぜ「冗談ではない」のか", section 3: per 16-element
  * sub-block a scale and a min, codes 0..3, the page's packing; "DeepSeek-V4-
  * Flash one-token computation flow", section "Dwarf Star の量子化の工夫": Q8_0

@@ -107,6 +107,7 @@ def test_quantize_argument_checks(moe):
              ((moe.MOE_QUANT_Q2_K, ok, -256, ok), moe.MOE_ERR_INVALID_ARG),
              ((moe.MOE_QUANT_Q2_K, ok, 300, ok), moe.MOE_ERR_UNSUPPORTED_SHAPE),
              ((moe.MOE_QUANT_Q8_0, ok, 48, ok), moe.MOE_ERR_UNSUPPORTED_SHAPE),
+             ((moe.MOE_QUANT_Q4_K, ok, 512 + 32, ok), moe.MOE_ERR_UNSUPPORTED_SHAPE),
              ((moe.MOE_QUANT_Q8_0, None, 64, ok), moe.MOE_ERR_INVALID_ARG),
              ((moe.MOE_QUANT_Q2_K, ok, 256, None), moe.MOE_ERR_INVALID_ARG),
              ((moe.MOE_QUANT_Q2_K, ok + 4, 256, ok), moe.MOE_ERR_MISALIGNED),
