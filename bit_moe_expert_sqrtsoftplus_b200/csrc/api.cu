@@ -331,10 +331,7 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
     return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (h->cfg.routed_format == MOE_ROUTED_Q4K) {
-    if (T > moe::kDecodeMaxT)
-      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "Q4_K layers run at most %d tokens per call (got %d)", moe::kDecodeMaxT,
-                  T);
+  if (h->cfg.routed_format == MOE_ROUTED_Q4K && T <= moe::kDecodeMaxT) {
     e = q4k_forward(h, x, token_ids, T, y, scratch, s);
   } else if (T <= moe::kDecodeMaxT) {
     moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
@@ -343,6 +340,7 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
     moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, y, scratch, h->row_norms, h->err);
     p.ev_begin = h->ev_begin;
     p.ev_end = h->ev_end;
+    p.q4k = h->cfg.routed_format == MOE_ROUTED_Q4K;
     e = moe::prefill_forward(p, s, h->num_sms);
   }
   if (e != cudaSuccess) return cuda_fail(e, "moe_ffn_forward launch");

@@ -200,6 +200,10 @@ template <>
 struct Raw<kFmtQ80> {
   uint32_t d16, q[8];
 };
+template <>
+struct Raw<kFmtQ4K> {
+  uint32_t dd, scm, q[8];  // d | dmin << 16; scale | min << 8 of the sub-block; 32 code bytes
+};
 
 // IQ2_XXS: group (kel/32) of the row.
 __device__ __forceinline__ void fetch(Raw<kFmtIQ2> &r, const uint8_t *rowp, int ks, int item) {
@@ -293,6 +297,47 @@ __device__ __forceinline__ void fetch(Raw<kFmtQ80> &r, const uint8_t *rowp, int 
 #pragma unroll
     for (int i = 0; i < 8; ++i) r.q[i] = __byte_perm(u[i], u[i + 1], 0x5432);
   }
+}
+
+// Q4_K (144-byte blocks: f16 d, f16 dmin, 12 bytes of 6-bit scales and mins,
+// 128 code bytes; value e of a block has code byte 32*(e/64) + e%32, nibble
+// (e%64)/32): the K step covers the 64-value chunk ks%4 of block ks/4, and
+// item (0, 1) is its sub-block 2*(ks%4) + item, whose 32 codes are the low or
+// the high nibbles of the chunk's 32 code bytes.
+__device__ __forceinline__ void fetch(Raw<kFmtQ4K> &r, const uint8_t *rowp, int ks, int item) {
+  const uint8_t *bp = rowp + (size_t)(ks >> 2) * 144;
+  const int c = ks & 3, j = 2 * c + item;
+  r.dd = ldg32(bp);
+  const uint8_t *sm = bp + 4;
+  int sc, mn;
+  if (j < 4) {
+    sc = sm[j] & 63;
+    mn = sm[j + 4] & 63;
+  } else {
+    sc = (sm[j + 4] & 15) | ((sm[j - 4] >> 6) << 4);
+    mn = (sm[j + 4] >> 4) | ((sm[j] >> 6) << 4);
+  }
+  r.scm = (uint32_t)sc | ((uint32_t)mn << 8);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.q[i] = ldg32(bp + 16 + 32 * c + 4 * i);
+}
+
+__device__ __forceinline__ void decode(const Raw<kFmtQ4K> &r, uint8_t *tile, int row, int item, int bf16,
+                                       const uint8_t *, const uint8_t *) {
+  const float d = __half2float(__ushort_as_half((unsigned short)(r.dd & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half((unsigned short)(r.dd >> 16)));
+  const float dsc = d * (float)(r.scm & 255u), mn = -dmin * (float)(r.scm >> 8);
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t x = (r.q[i] >> (4 * item)) & 0x0F0F0F0Fu;
+    const float v0 = fmaf(dsc, (float)(x & 255u), mn), v1 = fmaf(dsc, (float)((x >> 8) & 255u), mn);
+    const float v2 = fmaf(dsc, (float)((x >> 16) & 255u), mn), v3 = fmaf(dsc, (float)(x >> 24), mn);
+    o[2 * i] = bf16 ? bf16pair(v0, v1) : h2bits(__floats2half2_rn(v0, v1));
+    o[2 * i + 1] = bf16 ? bf16pair(v2, v3) : h2bits(__floats2half2_rn(v2, v3));
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sts128(swz(tile, row, 4 * item + c), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
 }
 
 template <bool BF16>
@@ -437,13 +482,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
         }
       }
       // A item of this thread: paired formats: matrix p/256, row (p/2)%128, 32-element half p%2;
-      // Q2_K: row p/4, item p%4 (16 elements); unpaired Q8_0: row p/2, half p%2 (threads < 256)
+      // Q2_K: row p/4, item p%4 (16 elements); unpaired Q8_0 / Q4_K: row p/2, half p%2 (threads < 256)
       const int mat = PAIRED ? (p >> 8) : 0;
       const int row = FMT == kFmtQ2K ? (p >> 2) : ((p >> 1) & 127);
       const int item = FMT == kFmtQ2K ? (p & 3) : (p & 1);
       const bool has_a = PAIRED || FMT == kFmtQ2K || p < 256;
       const uint8_t *arow = (mat ? a.A1 : a.A0) + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
-      const int dsel = FMT == kFmtQ80 ? a.bf16 : 0;
+      const int dsel = (FMT == kFmtQ80 || FMT == kFmtQ4K) ? a.bf16 : 0;
       // packed bytes of K steps ks .. ks + kAhead - 1 are in flight in a ring of
       // registers; slots are compile-time indices of the unrolled loop below, so
       // no register copy ever waits on a load
@@ -636,6 +681,8 @@ cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   if (a.fmt == kFmtQ80 && paired) return launch_gemm<kFmtQ80, true>(a, s, num_sms);
   if (a.fmt == kFmtQ80 && !paired) return launch_gemm<kFmtQ80, false>(a, s, num_sms);
   if (a.fmt == kFmtQ2K && !paired) return launch_gemm<kFmtQ2K, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ4K && paired) return launch_gemm<kFmtQ4K, true>(a, s, num_sms);
+  if (a.fmt == kFmtQ4K && !paired) return launch_gemm<kFmtQ4K, false>(a, s, num_sms);
   return cudaErrorInvalidValue;
 }
 

@@ -13,7 +13,7 @@
 
 namespace moe {
 
-enum GemmFmt { kFmtIQ2 = 0, kFmtQ2K = 1, kFmtQ80 = 2 };
+enum GemmFmt { kFmtIQ2 = 0, kFmtQ2K = 1, kFmtQ80 = 2, kFmtQ4K = 3 };
 enum GemmEpi { kEpiSwiGLU = 0, kEpiScatterAdd = 1, kEpiStore = 2 };
 
 struct GemmArgs {

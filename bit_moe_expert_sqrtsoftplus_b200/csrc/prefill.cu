@@ -443,6 +443,7 @@ PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, cons
   p.ev_begin = nullptr;
   p.ev_end = nullptr;
   p.err = err;
+  p.q4k = 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     off = align_up(off, 256);
@@ -573,14 +574,15 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   k_prep_x16<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, b.x16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  const size_t rbIQ = (size_t)(d.H / 256) * 66;
-  const size_t rbQ2 = (size_t)(d.I / 256) * 84;
+  // routed rows: IQ2_XXS gate/up and Q2_K down, or Q4_K for all three
+  const size_t rbIQ = (size_t)(d.H / 256) * (p.q4k ? 144 : 66);
+  const size_t rbQ2 = (size_t)(d.I / 256) * (p.q4k ? 144 : 84);
   const size_t rbQ8h = (size_t)(d.H / 32) * 34;
   const size_t rbQ8s = (size_t)(d.Is / 32) * 34;
 
   // routed gate/up: IQ2_XXS x f16 activations, SwiGLU -> h (bf16) in permuted order
   GemmArgs g{};
-  g.fmt = kFmtIQ2;
+  g.fmt = p.q4k ? kFmtQ4K : kFmtIQ2;
   g.bf16 = 0;
   g.epi = kEpiSwiGLU;
   g.M = d.I;
@@ -645,7 +647,7 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
 
   // routed down: Q2_K x bf16 h, y[token] += w * (W_down h)
   GemmArgs rd = sd;
-  rd.fmt = kFmtQ2K;
+  rd.fmt = p.q4k ? kFmtQ4K : kFmtQ2K;
   rd.epi = kEpiScatterAdd;
   rd.M = d.H;
   rd.K = d.I;

@@ -33,6 +33,7 @@ struct PrefillArgs {
   const float *row_norms;  // [E] 2-norms of the router rows
   int *err;
   cudaEvent_t ev_begin, ev_end;  // recorded around the routed gate/up GEMM when set
+  int q4k;                       // routed gate/up/down in Q4_K (else IQ2_XXS gate/up, Q2_K down)
 };
 
 size_t prefill_scratch_bytes(const LayerDims &d, int T);

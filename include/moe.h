@@ -90,8 +90,7 @@ typedef struct {
   float rms_eps;        /* RMSNorm epsilon when MOE_FLAG_PRENORM_RESIDUAL is set (1e-6) */
   int mode;             /* moe_route_mode */
   int flags;            /* MOE_FLAG_* */
-  int routed_format;    /* MOE_ROUTED_*; MOE_ROUTED_Q4K layers run moe_ffn_forward for T <= MOE_SMALL_T_MAX
-                           only (moe_route takes any T) and not moe_ffn_forward_noalloc */
+  int routed_format;    /* MOE_ROUTED_*; MOE_ROUTED_Q4K layers do not run moe_ffn_forward_noalloc */
 } moe_config;
 
 typedef struct {

@@ -82,20 +82,51 @@ def test_full_q4k_layer_one_and_eight_tokens(moe):
         _check_q4k(s, _run_q4k(moe, s, seed, 39, T), seed, 39)
 
 
-def test_q4k_layer_limits(moe):
-    s = synth.workload("tiny", tokens=40)
+def test_q4k_layer_has_no_noalloc_forward(moe):
+    s = synth.workload("tiny", tokens=2)
     W = harness.device_layer(s, 0, 0, q4k=True)
-    L = moe.Layer(harness.config_for(s, q4k=True), W, max_tokens=40)
-    x = torch.from_numpy(synth.activations(0, 40, s.hidden)).cuda()
+    L = moe.Layer(harness.config_for(s, q4k=True), W, max_tokens=2)
+    x = torch.from_numpy(synth.activations(0, 2, s.hidden)).cuda()
     with pytest.raises(moe.MoeError) as ei:
-        L.forward(x)
+        moe.moe_ffn_forward_noalloc(L.handle, x, None, 2, torch.empty_like(x))
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    idx, _ = L.route(x)  # routing takes any T
-    torch.cuda.synchronize()
-    assert idx.shape == (40, s.top_k)
-    with pytest.raises(moe.MoeError) as ei:
-        moe.moe_ffn_forward_noalloc(L.handle, x[:2], None, 2, torch.empty_like(x[:2]))
-    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+# ------------------------------------------- the batched path with Q4_K (T > 32)
+
+def _oracle_rows_q4k(s, seed, layer, x_np, tok_np, rows, router=True, prenorm=False):
+    sub = synth.LayerShape(s.hidden, s.inter, s.shared_inter, s.n_experts, s.top_k, len(rows), vocab=s.vocab,
+                           skew=s.skew)
+    _, _, yref, _ = harness.oracle_layer(sub, seed, layer, x_np[rows], tok_np[rows], router=router, prenorm=prenorm,
+                                         q4k=True)
+    return yref
+
+
+@pytest.mark.parametrize("T", [33, 64, 300])
+def test_tiny_q4k_large_T(moe, T):
+    s = synth.workload("tiny", tokens=T)
+    got = _run_q4k(moe, s, 0, 0, T)
+    yref = _oracle_rows_q4k(s, 0, 0, got["x"], got["tok"], np.arange(T))
+    rel, mx = harness.errors(got["y"], yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def test_tiny_q4k_hash_prenorm_large_T(moe):
+    s = synth.workload("tiny", tokens=100)
+    got = _run_q4k(moe, s, 2, 1, 100, mode=moe.MOE_ROUTE_HASH, flags=moe.MOE_FLAG_PRENORM_RESIDUAL)
+    yref = _oracle_rows_q4k(s, 2, 1, got["x"], got["tok"], np.arange(100), router=False, prenorm=True)
+    rel, mx = harness.errors(got["y"], yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def test_full_q4k_512_tokens_sampled(moe):
+    """V4-Flash shapes, 512 tokens with the skewed bias: sampled output rows."""
+    s = synth.workload("prefill_t4096", tokens=512)
+    got = _run_q4k(moe, s, 3, 38, 512)
+    rows = np.arange(0, 512, 37)
+    yref = _oracle_rows_q4k(s, 3, 38, got["x"], got["tok"], rows)
+    rel, mx = harness.errors(got["y"][rows], yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
 
 
 def test_q2q4_stack_tail_teacher_forced(moe):
