@@ -47,7 +47,8 @@ __device__ float dot_q4k(const uint8_t *row, const float *v, int K, int lane) {
   const int code_off = 16 + 32 * (lane >> 3) + 8 * (lane & 3);
   const int shift = 4 * ((lane & 7) >> 2);
   float part = 0.0f;
-  for (int b = 0; b < K / 256; ++b) {
+#pragma unroll 4
+  for (int b = 0; b < K / 256; ++b) {  // unrolled so several blocks' loads are in flight
     const uint8_t *blk = row + (size_t)b * 144;
     const uint4 hd = *reinterpret_cast<const uint4 *>(blk);  // d, dmin, scale bytes 0..11
     const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
@@ -84,6 +85,7 @@ __device__ float dot_q4k(const uint8_t *row, const float *v, int K, int lane) {
 // every block.
 __device__ float dot_q80(const uint8_t *row, const float *v, int K, int lane) {
   float part = 0.0f;
+#pragma unroll 8
   for (int b = 0; b < K / 32; ++b) {
     const uint8_t *blk = row + (size_t)b * 34;
     part = fmaf(f16_at(blk) * (float)(int8_t)blk[2 + lane], v[32 * b + lane], part);
