@@ -202,7 +202,7 @@ struct Raw<kFmtQ80> {
 };
 template <>
 struct Raw<kFmtQ4K> {
-  uint32_t dd, scm, q[8];  // d | dmin << 16; scale | min << 8 of the sub-block; 32 code bytes
+  uint32_t sm, q[8];  // half2 (d * scale, -dmin * min) of the sub-block; its 32 code bytes
 };
 
 // IQ2_XXS: group (kel/32) of the row.
@@ -303,11 +303,13 @@ __device__ __forceinline__ void fetch(Raw<kFmtQ80> &r, const uint8_t *rowp, int 
 // 128 code bytes; value e of a block has code byte 32*(e/64) + e%32, nibble
 // (e%64)/32): the K step covers the 64-value chunk ks%4 of block ks/4, and
 // item (0, 1) is its sub-block 2*(ks%4) + item, whose 32 codes are the low or
-// the high nibbles of the chunk's 32 code bytes.
+// the high nibbles of the chunk's 32 code bytes.  The sub-block's step
+// d * scale and offset -dmin * min travel as one f16 pair (their rounding,
+// at most 2^-12 of each, is below that of the f16 / bf16 tile values).
 __device__ __forceinline__ void fetch(Raw<kFmtQ4K> &r, const uint8_t *rowp, int ks, int item) {
   const uint8_t *bp = rowp + (size_t)(ks >> 2) * 144;
   const int c = ks & 3, j = 2 * c + item;
-  r.dd = ldg32(bp);
+  const uint32_t dd = ldg32(bp);
   const uint8_t *sm = bp + 4;
   int sc, mn;
   if (j < 4) {
@@ -317,27 +319,32 @@ __device__ __forceinline__ void fetch(Raw<kFmtQ4K> &r, const uint8_t *rowp, int 
     sc = (sm[j + 4] & 15) | ((sm[j - 4] >> 6) << 4);
     mn = (sm[j + 4] >> 4) | ((sm[j] >> 6) << 4);
   }
-  r.scm = (uint32_t)sc | ((uint32_t)mn << 8);
+  const float d = __half2float(__ushort_as_half((unsigned short)(dd & 0xFFFFu)));
+  const float dmin = __half2float(__ushort_as_half((unsigned short)(dd >> 16)));
+  r.sm = h2bits(__floats2half2_rn(d * (float)sc, -dmin * (float)mn));
 #pragma unroll
   for (int i = 0; i < 8; ++i) r.q[i] = ldg32(bp + 16 + 32 * c + 4 * i);
 }
 
 __device__ __forceinline__ void decode(const Raw<kFmtQ4K> &r, uint8_t *tile, int row, int item, int bf16,
                                        const uint8_t *, const uint8_t *) {
-  const float d = __half2float(__ushort_as_half((unsigned short)(r.dd & 0xFFFFu)));
-  const float dmin = __half2float(__ushort_as_half((unsigned short)(r.dd >> 16)));
-  const float dsc = d * (float)(r.scm & 255u), mn = -dmin * (float)(r.scm >> 8);
-  uint32_t o[16];
+  const float2 f = __half22float2(bits2h(r.sm));
+  const float dsc = f.x, mn = f.y;
+  // 16-byte chunk c of the item: values 8c .. 8c+7 (code words 2c, 2c+1),
+  // stored as soon as they are made
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t x = (r.q[i] >> (4 * item)) & 0x0F0F0F0Fu;
-    const float v0 = fmaf(dsc, (float)(x & 255u), mn), v1 = fmaf(dsc, (float)((x >> 8) & 255u), mn);
-    const float v2 = fmaf(dsc, (float)((x >> 16) & 255u), mn), v3 = fmaf(dsc, (float)(x >> 24), mn);
-    o[2 * i] = bf16 ? bf16pair(v0, v1) : h2bits(__floats2half2_rn(v0, v1));
-    o[2 * i + 1] = bf16 ? bf16pair(v2, v3) : h2bits(__floats2half2_rn(v2, v3));
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t x = (r.q[2 * c + h] >> (4 * item)) & 0x0F0F0F0Fu;
+      const float v0 = fmaf(dsc, (float)(x & 255u), mn), v1 = fmaf(dsc, (float)((x >> 8) & 255u), mn);
+      const float v2 = fmaf(dsc, (float)((x >> 16) & 255u), mn), v3 = fmaf(dsc, (float)(x >> 24), mn);
+      o[2 * h] = bf16 ? bf16pair(v0, v1) : h2bits(__floats2half2_rn(v0, v1));
+      o[2 * h + 1] = bf16 ? bf16pair(v2, v3) : h2bits(__floats2half2_rn(v2, v3));
+    }
+    sts128(swz(tile, row, 4 * item + c), o[0], o[1], o[2], o[3]);
   }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) sts128(swz(tile, row, 4 * item + c), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
 }
 
 template <bool BF16>
