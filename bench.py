@@ -647,7 +647,7 @@ def run_quant(args, world, rank):
 def oracle_quant_rate(workload: str, steps: int, warmup: int, values_per_step: int = 1 << 20):
     """Values/s of the oracle's encoder on steps of 2^20 values."""
     import oracle
-    fmt, per, _ = quant_format(workload)
+    fmt = quant_format(workload)[0]
     kind = {0: oracle.KIND_Q80, 1: oracle.KIND_Q2K, 2: oracle.KIND_Q4K}[fmt]
     x = (np.random.default_rng(7).standard_normal(values_per_step) * 0.02).astype(np.float32)
     for _ in range(warmup):
@@ -768,7 +768,7 @@ def main():
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    world, rank, local = dist_setup(args)
+    world, rank, _ = dist_setup(args)
     if args.sweep:
         for line in run_sweep(args, world, rank):
             if rank == 0:

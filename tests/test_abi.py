@@ -59,7 +59,7 @@ def _cfg(moe, **over):
 def test_workspace_size_and_shape_checks(moe):
     p, s = moe.moe_workspace_size(_cfg(moe), 1)
     assert p >= 4 and s > 0
-    p2, s32 = moe.moe_workspace_size(_cfg(moe), 4096)
+    _, s32 = moe.moe_workspace_size(_cfg(moe), 4096)
     assert s32 > s
     for bad, status in ((dict(hidden=4000), moe.MOE_ERR_UNSUPPORTED_SHAPE),
                         (dict(inter=100), moe.MOE_ERR_UNSUPPORTED_SHAPE),

@@ -4,7 +4,6 @@ ABI; the full-shape 32-token case runs on the small-T path."""
 import numpy as np
 import pytest
 
-import oracle
 import synth
 from tests import harness
 

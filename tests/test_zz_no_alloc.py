@@ -4,7 +4,6 @@ program with a fixed device-memory plan).  Its scratch lives in a buffer built
 into the library instead of a caller-provided one.  This file is collected
 last so that a run stopping at the first failure has run every other test.
 """
-import numpy as np
 import pytest
 
 import synth

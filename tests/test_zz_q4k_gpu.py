@@ -27,8 +27,6 @@ def test_q4k_device_fill_is_byte_identical_to_host_fill():
 
 from tests import harness  # noqa: E402
 
-import oracle  # noqa: E402
-
 
 @pytest.fixture(scope="module")
 def moe():
