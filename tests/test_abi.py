@@ -50,6 +50,23 @@ def test_binding_constants_match_the_header(moe):
         assert getattr(moe, name) == v, name
 
 
+def test_the_abi_from_plain_c(moe, tmp_path):
+    """A C program (tests/c_abi_check.c) includes include/moe.h, links the
+    library and runs its host-side checks: the boundary needs no Python."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_check"
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe), "-L", lib_dir, "-lmoe_b200",
+                    f"-Wl,-rpath,{lib_dir}"], check=True)
+    p = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert p.returncode == 0, p.stdout + p.stderr
+    assert "C ABI checks passed" in p.stdout
+
+
 def _cfg(moe, **over):
     base = dict(hidden=4096, inter=2048, n_experts=256, top_k=6, shared_inter=2048, vocab=129280)
     base.update(over)
