@@ -1,6 +1,10 @@
 """GPU checks for the Q4_K routed-expert variant (the q2-q4 build's upgraded
-layers): the device fill of the seeded generator is byte-identical to the
-host fill the oracle reads."""
+layers), through the C ABI against the fp64 oracle: the generator's device
+fill (byte-identical to the host fill the oracle reads); the small-token path
+(tiny layer at T = 1, 3, 8, 32, hash routing with the pre-norm residual,
+V4-Flash shapes at T = 1 and 8); the batched path (tiny layer at T = 33, 64,
+300, hash routing with pre-norm, V4-Flash shapes at T = 512 on sampled rows);
+the tail of the q2-q4 stack; and the missing no-allocation forward."""
 import numpy as np
 import pytest
 
