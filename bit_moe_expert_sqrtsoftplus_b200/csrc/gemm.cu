@@ -304,8 +304,10 @@ __device__ __forceinline__ void fetch(Raw<kFmtQ80> &r, const uint8_t *rowp, int 
 // (e%64)/32): the K step covers the 64-value chunk ks%4 of block ks/4, and
 // item (0, 1) is its sub-block 2*(ks%4) + item, whose 32 codes are the low or
 // the high nibbles of the chunk's 32 code bytes.  The sub-block's step
-// d * scale and offset -dmin * min travel as one f16 pair (their rounding,
-// at most 2^-12 of each, is below that of the f16 / bf16 tile values).
+// d * scale and offset -dmin * min travel as one f16 pair: their rounding (a
+// relative 2^-11 at most while they are normal binary16 values, >= 2^-14) is
+// that of one more f16 rounding, next to the f16 / bf16 rounding of every
+// tile value.
 __device__ __forceinline__ void fetch(Raw<kFmtQ4K> &r, const uint8_t *rowp, int ks, int item) {
   const uint8_t *bp = rowp + (size_t)(ks >> 2) * 144;
   const int c = ks & 3, j = 2 * c + item;
