@@ -51,13 +51,15 @@ def lib():
         L.oracle_row_q80.argtypes = [vp, i32, vp]
         L.oracle_row_q4k.argtypes = [vp, i32, vp]
         L.oracle_matvec.argtypes = [i32, vp, i32, i32, vp, vp, vp]
+        L.oracle_decode_matrix.argtypes = [i32, vp, i32, i32, vp, vp]
         L.oracle_sqrtsoftplus.argtypes = [d]
         L.oracle_sqrtsoftplus.restype = d
         L.oracle_silu.argtypes = [d]
         L.oracle_silu.restype = d
         L.oracle_router_logits.argtypes = [vp, i32, i32, vp, i32, vp]
         L.oracle_select.argtypes = [vp, vp, i32, i32, i32, d, vp, vp, vp]
-        L.oracle_hash_select.argtypes = [vp, i32, vp, i32, i32, d, vp, vp]
+        L.oracle_hash_select.argtypes = [vp, i32, vp, i32, i32, i32, d, vp, vp]
+        L.oracle_hash_select.restype = i32
         L.oracle_swiglu_expert.argtypes = [i32, i32, vp, vp, vp, i32, i32, vp, vp, vp]
         L.oracle_layer.argtypes = [vp, vp, i32, vp, vp, vp]
         L.oracle_layer.restype = i32
@@ -122,8 +124,13 @@ def decode_row(kind: int, row: np.ndarray, cols: int, grid: np.ndarray | None = 
 
 
 def decode_matrix(kind: int, W: np.ndarray, rows: int, cols: int, grid=None) -> np.ndarray:
-    W = np.ascontiguousarray(W, dtype=np.uint8).reshape(rows, -1)
-    return np.stack([decode_row(kind, W[r], cols, grid) for r in range(rows)])
+    """All rows of a packed [rows][cols] matrix decoded to fp64 by the scalar C
+    decoders (one call; the GIL is released while it runs)."""
+    w, pw = _c(np.asarray(W).reshape(rows, -1), np.uint8)
+    g, pg = (None, None) if grid is None else _c(grid, np.uint8)
+    out = np.empty((rows, cols), dtype=np.float64)
+    lib().oracle_decode_matrix(kind, pw, rows, cols, pg, out.ctypes.data)
+    return out
 
 
 def matvec(kind: int, W: np.ndarray, rows: int, cols: int, x: np.ndarray, grid=None) -> np.ndarray:
@@ -172,13 +179,21 @@ def route(x: np.ndarray, Wr: np.ndarray, bias: np.ndarray, k: int, scaling: floa
     return select(router_logits(x, Wr), bias, k, scaling)
 
 
-def hash_route(token_ids: np.ndarray, tid2eid: np.ndarray, k: int, scaling: float = 1.5):
+def hash_route(token_ids: np.ndarray, tid2eid: np.ndarray, k: int, scaling: float = 1.5, n_experts: int = 256):
+    """Hash routing through the table; raises ValueError for a token id outside
+    the table or a used table row that does not hold k distinct ids in
+    [0, n_experts)."""
     t, pt = _c(token_ids, np.int32)
     tab, ptab = _c(tid2eid, np.int32)
     T = t.shape[0]
     idx = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
-    lib().oracle_hash_select(pt, T, ptab, tab.shape[0], k, float(scaling), idx.ctypes.data, w.ctypes.data)
+    rc = lib().oracle_hash_select(pt, T, ptab, tab.shape[0], int(n_experts), k, float(scaling), idx.ctypes.data,
+                                  w.ctypes.data)
+    if rc == -1:
+        raise ValueError("hash routing: token id outside the table")
+    if rc != 0:
+        raise ValueError("hash routing: a table row does not hold distinct expert ids in range")
     return idx, w
 
 
@@ -258,6 +273,57 @@ def layer(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray, t
         rc = lib().oracle_layer(ctypes.byref(lw), px, T, pi, pw, y.ctypes.data)
     if rc != 0:
         raise ValueError("oracle_layer: a selected expert has no weights")
+    return y
+
+
+def layer_dense(weights: dict, shape, x: np.ndarray, idx: np.ndarray, w: np.ndarray, threads: int = 0) -> np.ndarray:
+    """The same layer as :func:`layer`, computed as dequantise-then-multiply:
+    every matrix a call uses is decoded once to fp64 by the scalar C decoders
+    (``decode_matrix``) and the products are numpy fp64 matrix products, the
+    textbook reduction of the fused route.  y = shared(x) + the selected
+    experts' weighted outputs added in ascending expert id, as in ``layer``;
+    results agree with ``layer`` up to the order of the fp64 additions inside
+    each dot product.  Meant for checking many tokens of a full-size call,
+    where the row-by-row route is too slow.  ``threads`` decodes that many
+    experts at once (0: the host's cores)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    H, I, Is, E = shape.hidden, shape.inter, shape.shared_inter, shape.n_experts
+    gk = int(weights.get("gate_kind", KIND_IQ2XXS))
+    dk = int(weights.get("down_kind", KIND_Q2K))
+    grid = weights["grid"]
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    idx = np.asarray(idx)
+    w = np.asarray(w, dtype=np.float64)
+
+    def silu(u):
+        return u / (1.0 + np.exp(-u))
+
+    def expert_of(src, e):
+        a = src.get(e) if isinstance(src, dict) else src[e]
+        if a is None:
+            raise ValueError("layer_dense: a selected expert has no weights")
+        return a
+
+    def run_expert(e):
+        rows_t, slots = np.nonzero(idx == e)
+        Wg = decode_matrix(gk, expert_of(weights["gate"], e), I, H, grid)
+        Wu = decode_matrix(gk, expert_of(weights["up"], e), I, H, grid)
+        Wd = decode_matrix(dk, expert_of(weights["down"], e), H, I, grid)
+        xe = x[rows_t]
+        h = silu(xe @ Wg.T) * (xe @ Wu.T)
+        return rows_t, slots, h @ Wd.T
+
+    Wsg = decode_matrix(KIND_Q80, weights["sh_gate"], Is, H)
+    Wsu = decode_matrix(KIND_Q80, weights["sh_up"], Is, H)
+    Wsd = decode_matrix(KIND_Q80, weights["sh_down"], H, Is)
+    y = (silu(x @ Wsg.T) * (x @ Wsu.T)) @ Wsd.T
+    experts = [int(e) for e in np.unique(idx)]
+    n = threads if threads > 0 else max(1, min(8, os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=n) as pool:
+        # results are added in ascending expert id, whatever order they finish in
+        for rows_t, slots, o in pool.map(run_expert, experts):
+            y[rows_t] += w[rows_t, slots][:, None] * o
     return y
 
 

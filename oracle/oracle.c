@@ -186,6 +186,11 @@ static size_t row_bytes(int kind, int cols) {
                      : (size_t)cols / 32 * 34;
 }
 
+void oracle_decode_matrix(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, double *out) {
+  size_t rb = row_bytes(kind, cols);
+  for (int r = 0; r < rows; ++r) decode_row(kind, W + rb * (size_t)r, cols, grid, out + (size_t)r * cols);
+}
+
 void oracle_matvec(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, const double *x,
                    double *y) {
   double *wrow = (double *)malloc(sizeof(double) * (size_t)cols);
@@ -274,17 +279,38 @@ void oracle_select(const double *z, const float *bias, int T, int E, int k, doub
  * [FLOW] MoE FFN section: layers 0-2 have no router; a static table
  * (tid2eid) maps the token id to expert ids.  Reading: the k table entries
  * each get weight scaling / k (uniform weights summing to the scaling).
+ * A token id outside [0, vocab), or a table row (of a token in the call)
+ * with an id outside [0, n_experts) or an id twice, names no set of k
+ * distinct experts: the call returns -1 (token id) or -2 (table row) and
+ * leaves that token's idx and w unset, as the CUDA layer reports such input
+ * instead of computing with it.
  */
-void oracle_hash_select(const int32_t *token_ids, int T, const int32_t *tid2eid, int vocab, int k,
-                        double scaling, int32_t *idx, double *w) {
+int oracle_hash_select(const int32_t *token_ids, int T, const int32_t *tid2eid, int vocab, int n_experts, int k,
+                       double scaling, int32_t *idx, double *w) {
+  int rc = 0;
   for (int t = 0; t < T; ++t) {
-    int tid = token_ids[t];
-    if (tid < 0 || tid >= vocab) tid = 0;
+    const int tid = token_ids[t];
+    if (tid < 0 || tid >= vocab) {
+      rc = -1;
+      continue;
+    }
+    const int32_t *row = tid2eid + (size_t)tid * k;
+    int ok = 1;
+    for (int i = 0; i < k; ++i) {
+      if (row[i] < 0 || row[i] >= n_experts) ok = 0;
+      for (int j = 0; j < i; ++j)
+        if (row[j] == row[i]) ok = 0;
+    }
+    if (!ok) {
+      if (rc == 0) rc = -2;
+      continue;
+    }
     int32_t *it = idx + (size_t)t * k;
-    for (int i = 0; i < k; ++i) it[i] = tid2eid[(size_t)tid * k + i];
+    for (int i = 0; i < k; ++i) it[i] = row[i];
     qsort(it, (size_t)k, sizeof(int32_t), by_int);
     for (int i = 0; i < k; ++i) w[(size_t)t * k + i] = scaling / (double)k;
   }
+  return rc;
 }
 
 /* --------------------------------------------------------------- SwiGLU */

@@ -52,6 +52,9 @@ void oracle_row_q2k(const uint8_t *row, int cols, double *out);
 void oracle_row_q80(const uint8_t *row, int cols, double *out);
 void oracle_row_q4k(const uint8_t *row, int cols, double *out);
 
+/* Every row of a [rows][cols] matrix decoded into out (row-major fp64). */
+void oracle_decode_matrix(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, double *out);
+
 /* y[r] = sum_c W[r][c] x[c] with W decoded row by row (fused route). */
 void oracle_matvec(int kind, const uint8_t *W, int rows, int cols, const uint8_t *grid, const double *x,
                    double *y);
@@ -61,8 +64,10 @@ double oracle_sqrtsoftplus(double z);
 void oracle_router_logits(const double *x, int T, int H, const uint16_t *Wr, int E, double *z);
 void oracle_select(const double *z, const float *bias, int T, int E, int k, double scaling, int32_t *idx,
                    double *w, double *margin);
-void oracle_hash_select(const int32_t *token_ids, int T, const int32_t *tid2eid, int vocab, int k,
-                        double scaling, int32_t *idx, double *w);
+/* Hash routing; returns 0, -1 (a token id outside [0, vocab)) or -2 (a used
+ * table row with an id outside [0, n_experts) or a repeated id). */
+int oracle_hash_select(const int32_t *token_ids, int T, const int32_t *tid2eid, int vocab, int n_experts, int k,
+                       double scaling, int32_t *idx, double *w);
 
 /* SwiGLU pieces. */
 double oracle_silu(double u);

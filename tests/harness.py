@@ -38,10 +38,33 @@ def oracle_layer(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, toke
         idx, w, margin = oracle.select(z, b, s.top_k, s.routed_scaling)
     else:
         tab = synth.tid2eid(seed, layer, s.vocab, s.n_experts, s.top_k)
-        idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling)
+        idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling, n_experts=s.n_experts)
         margin = np.full(x.shape[0], np.inf)
     W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router, q4k=q4k)
     y = oracle.layer(W, s, xin, idx, w, threads=threads)
+    if prenorm:
+        y = y + x.astype(np.float64)
+    return idx, w, y, margin
+
+
+def oracle_layer_dense(s: synth.LayerShape, seed: int, layer: int, x: np.ndarray, token_ids=None, router=True,
+                       prenorm=False, q4k=False):
+    """As oracle_layer, with the layer computed by oracle.layer_dense (decode
+    each used matrix once, fp64 matrix products): for checking every row of
+    full-size calls."""
+    xin = x.astype(np.float64)
+    if prenorm:
+        xin = oracle.rmsnorm(xin, 1e-6)
+    if router:
+        Wr = synth.router_weight(seed, layer, s.n_experts, s.hidden)
+        b = synth.bias(seed, layer, s.n_experts, s.skew)
+        idx, w, margin = oracle.select(oracle.router_logits(xin, Wr), b, s.top_k, s.routed_scaling)
+    else:
+        tab = synth.tid2eid(seed, layer, s.vocab, s.n_experts, s.top_k)
+        idx, w = oracle.hash_route(token_ids, tab, s.top_k, s.routed_scaling, n_experts=s.n_experts)
+        margin = np.full(x.shape[0], np.inf)
+    W = synth.host_layer(seed, layer, s, experts=np.unique(idx), router=router, q4k=q4k)
+    y = oracle.layer_dense(W, s, xin, idx, w)
     if prenorm:
         y = y + x.astype(np.float64)
     return idx, w, y, margin

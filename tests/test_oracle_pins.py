@@ -294,6 +294,83 @@ def test_hash_route_uniform_weights():
         assert list(idx[t]) == sorted(tab[ids[t]])
 
 
+def test_hash_route_rejects_token_ids_outside_the_table():
+    """A token id outside [0, vocab) names no table row: an error, not row 0."""
+    tab = synth.tid2eid(0, 0, 1000, 256, 6)
+    for bad in (-1, 1000, 1 << 30):
+        ids = np.array([3, bad, 7], dtype=np.int32)
+        with pytest.raises(ValueError, match="token id"):
+            oracle.hash_route(ids, tab, 6)
+
+
+@pytest.mark.parametrize("entry", [-1, 256, 999])
+def test_hash_route_rejects_table_rows_outside_the_experts(entry):
+    tab = synth.tid2eid(0, 0, 100, 256, 6).copy()
+    tab[5, 2] = entry
+    with pytest.raises(ValueError, match="table row"):
+        oracle.hash_route(np.array([5], np.int32), tab, 6)
+    # rows of other tokens are not looked at
+    idx, _ = oracle.hash_route(np.array([4, 6], np.int32), tab, 6)
+    assert list(idx[0]) == sorted(tab[4]) and list(idx[1]) == sorted(tab[6])
+
+
+def test_hash_route_rejects_a_repeated_expert_in_a_row():
+    tab = synth.tid2eid(0, 0, 100, 256, 6).copy()
+    tab[9, 4] = tab[9, 1]
+    with pytest.raises(ValueError, match="table row"):
+        oracle.hash_route(np.array([9], np.int32), tab, 6)
+
+
+@pytest.mark.parametrize("q4k", [False, True])
+def test_threaded_layer_equals_single_thread_bitwise(q4k):
+    """oracle.layer(threads=n) splits the tokens into consecutive slices (7
+    tokens over 3 threads: 3, 2, 2); every token's output must be the
+    single-thread result bit for bit, so a slice offset error in x, idx, w or
+    y shows here.  Both routed formats (q2 build and Q4_K layers)."""
+    s = synth.workload("tiny", tokens=7)
+    x = synth.activations(4, 7, s.hidden).astype(np.float64)
+    Wr = synth.router_weight(4, 0, s.n_experts, s.hidden)
+    b = synth.bias(4, 0, s.n_experts, False)
+    idx, w, _ = oracle.route(x, Wr, b, s.top_k)
+    W = synth.host_layer(4, 0, s, experts=np.unique(idx), q4k=q4k)
+    y1 = oracle.layer(W, s, x, idx, w, threads=1)
+    for n in (2, 3, 7, 16):
+        yn = oracle.layer(W, s, x, idx, w, threads=n)
+        assert np.array_equal(y1.view(np.uint64), yn.view(np.uint64)), n
+    # each token's row is that token's layer alone
+    for t in (0, 3, 6):
+        yt = oracle.layer(W, s, x[t:t + 1], idx[t:t + 1], w[t:t + 1])
+        assert np.array_equal(yt[0].view(np.uint64), y1[t].view(np.uint64))
+
+
+@pytest.mark.parametrize("q4k", [False, True])
+def test_dense_layer_route_equals_the_row_by_row_layer(q4k):
+    """oracle.layer_dense (decode every used matrix, then numpy fp64 matrix
+    products) against oracle.layer (row-by-row fused route): the same layer up
+    to the order of fp64 additions.  Tiny shapes, 23 tokens, router routing."""
+    s = synth.workload("tiny", tokens=23)
+    x = synth.activations(8, 23, s.hidden).astype(np.float64)
+    Wr = synth.router_weight(8, 1, s.n_experts, s.hidden)
+    b = synth.bias(8, 1, s.n_experts, True)
+    idx, w, _ = oracle.route(x, Wr, b, s.top_k)
+    W = synth.host_layer(8, 1, s, experts=np.unique(idx), q4k=q4k)
+    ref = oracle.layer(W, s, x, idx, w)
+    got = oracle.layer_dense(W, s, x, idx, w, threads=3)
+    assert np.max(np.abs(got - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_dense_layer_route_at_full_shape_one_token():
+    s = synth.workload("decode_t1")
+    x = synth.activations(2, 1, s.hidden).astype(np.float64)
+    Wr = synth.router_weight(2, 0, s.n_experts, s.hidden)
+    b = synth.bias(2, 0, s.n_experts, False)
+    idx, w, _ = oracle.route(x, Wr, b, s.top_k)
+    W = synth.host_layer(2, 0, s, experts=np.unique(idx))
+    ref = oracle.layer(W, s, x, idx, w)
+    got = oracle.layer_dense(W, s, x, idx, w)
+    assert np.max(np.abs(got - ref)) <= 1e-11 * np.max(np.abs(ref))
+
+
 # ---------------------------------------------------------------- matvec
 
 @pytest.mark.parametrize("kind,rows,cols", [(0, 12, 512), (1, 12, 512), (2, 12, 256)])
