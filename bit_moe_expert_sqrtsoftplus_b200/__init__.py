@@ -37,7 +37,8 @@ MOE_ROUTED_Q2 = 0
 MOE_ROUTED_Q4K = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
-            "moe_last_error", "moe_set_timing_events", "moe_ffn_forward_noalloc", "moe_quantize", "moe_destroy")
+            "moe_last_error", "moe_set_timing_events", "moe_set_wait_limit", "moe_ffn_forward_noalloc", "moe_quantize",
+            "moe_destroy")
 
 
 class moe_config(ctypes.Structure):
@@ -82,6 +83,8 @@ def lib():
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_set_timing_events.argtypes = [vp, vp, vp]
         L.moe_set_timing_events.restype = i32
+        L.moe_set_wait_limit.argtypes = [vp, ctypes.c_longlong]
+        L.moe_set_wait_limit.restype = i32
         L.moe_quantize.argtypes = [i32, vp, ctypes.c_int64, vp, vp, vp]
         L.moe_quantize.restype = i32
         L.moe_destroy.argtypes = [vp]
@@ -160,6 +163,12 @@ def moe_set_timing_events(handle, ev_begin=None, ev_end=None):
     """ev_begin / ev_end: torch.cuda.Event objects (or None to stop)."""
     _check(lib().moe_set_timing_events(handle, None if ev_begin is None else ev_begin.cuda_event,
                                        None if ev_end is None else ev_end.cuda_event))
+
+
+def moe_set_wait_limit(handle, cycles: int):
+    """Test hook: bound of the device waits on other warps' results, in SM
+    clock cycles (0 restores the default of about 2 s)."""
+    _check(lib().moe_set_wait_limit(handle, int(cycles)))
 
 
 def moe_quantize(fmt, x, out, nonfinite=None, stream=None):

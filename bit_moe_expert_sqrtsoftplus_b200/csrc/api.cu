@@ -93,6 +93,7 @@ moe::LayerDims dims_of(const moe_config &c) {
   d.vocab = c.vocab;
   d.scaling = c.routed_scaling;
   d.eps = c.rms_eps;
+  d.wait_cycles = moe::kDefaultWaitCycles;
   return d;
 }
 
@@ -234,6 +235,22 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   if (e != cudaSuccess) {
     delete h;
     return cuda_fail(e, "init kernels");
+  }
+  if (cfg->mode == MOE_ROUTE_HASH) {
+    // the kernels index the weights with the table's ids and assume a token
+    // selects an expert once: check every row before the handle is used
+    int bad = -1;
+    e = moe::check_tid2eid(h->d, w->tid2eid, h->err + 1, &bad, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->err + 1, 0, sizeof(int), s);
+    if (e != cudaSuccess) {
+      delete h;
+      return cuda_fail(e, "checking tid2eid");
+    }
+    if (bad >= 0) {
+      delete h;
+      return fail(MOE_ERR_INVALID_ARG, "tid2eid row %d does not hold %d distinct expert ids in [0, %d)", bad,
+                  cfg->top_k, cfg->n_experts);
+    }
   }
   *out = h;
   g_last_error.clear();
@@ -439,6 +456,14 @@ moe_status moe_poll_device_error(moe_handle *h, moe_stream_t stream) {
         return fail(MOE_ERR_DEVICE_FAULT, "device error code %d", code);
     }
   }
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_set_wait_limit(moe_handle *h, long long cycles) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (cycles < 0) return fail(MOE_ERR_INVALID_ARG, "cycles=%lld is negative", cycles);
+  h->d.wait_cycles = cycles > 0 ? cycles : moe::kDefaultWaitCycles;
   g_last_error.clear();
   return MOE_OK;
 }

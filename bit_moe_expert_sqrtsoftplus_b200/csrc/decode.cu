@@ -58,7 +58,6 @@ constexpr bool kAheadClaim = MOE_DECODE_AHEAD != 0;
 #define MOE_DECODE_GUNROLL 2
 #endif
 constexpr int kGUnroll = MOE_DECODE_GUNROLL;  // unrolling of the IQ2_XXS group loop
-constexpr long long kSliceWaitCycles = 4000000000ll;  // about 2 s: bound of a wait for an h slice
 constexpr int kThreads2 = kWarps2 * kWarp;
 // k2 threads: 12 warps for four token pairs, whose accumulators need more
 // than the 128 registers a thread has at 16 warps
@@ -515,7 +514,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parit
         : "r"(mb), "r"(parity)
         : "memory");
     if (ok) return true;
-    if (clock64() - t0 > 4000000000ll) {
+    if (clock64() - t0 > kDefaultWaitCycles) {
       set_error(err, kErrTimeout);
       return false;
     }
@@ -1111,14 +1110,14 @@ __device__ void finish_h_tile(const DecodeArgs &a, const float (*hs)[16], int nt
 // Each lane with a flag waits (bounded) until it is set; the warp then reads
 // what the flag's writer published.  A flag that is never set records the
 // timeout error and lets the warp go on.
-__device__ void wait_slice(const int *flag, int *err) {
+__device__ void wait_slice(const int *flag, int *err, long long limit) {
   if (flag) {
     const long long t0 = clock64();
     while (true) {
       int v;
       asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(flag) : "memory");
       if (v) break;
-      if (clock64() - t0 > kSliceWaitCycles) {
+      if (clock64() - t0 > limit) {
         set_error(err, kErrTimeout);
         break;
       }
@@ -1307,7 +1306,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
       const long long t0 = clock64();
       bool ok = true;
       while (*reinterpret_cast<volatile int *>(&S.jobs_ready) == 0) {
-        if (clock64() - t0 > kSliceWaitCycles) {
+        if (clock64() - t0 > d.wait_cycles) {
           set_error(a.err, kErrTimeout);
           ok = false;
           break;
@@ -1543,7 +1542,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     // the routing warps compute units only once the limbs are in place
     const long long t0 = clock64();
     while (*reinterpret_cast<volatile int *>(&S.limbs_ready) == 0) {
-      if (clock64() - t0 > kSliceWaitCycles) {
+      if (clock64() - t0 > d.wait_cycles) {
         set_error(a.err, kErrTimeout);
         break;
       }
@@ -1602,7 +1601,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
         // -------------------------------------------------- down
         if (cc == 0) {
           // the h slices this unit reads: one per token slot
-          wait_slice(lane < cu.ntok ? s.ready + hvec(cu, lane) * s.NSL + cu.kp : nullptr, a.err);
+          wait_slice(lane < cu.ntok ? s.ready + hvec(cu, lane) * s.NSL + cu.kp : nullptr, a.err, d.wait_cycles);
           npairs = (cu.ntok + 1) >> 1;
 #pragma unroll
           for (int p = 0; p < MAXP; ++p) {

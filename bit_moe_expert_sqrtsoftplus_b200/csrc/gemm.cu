@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "layer.cuh"
 #include "launch.cuh"
 
 namespace moe {
@@ -44,7 +45,6 @@ constexpr int kAhead = 3;                          // K steps of packed weights 
 constexpr int BM = 128, BK = 64, BN = 256;
 constexpr int kATile = BM * BK * 2;  // 16 KB
 constexpr int kBTile = BN * BK * 2;  // 32 KB
-constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 
 constexpr int kSB = 4;       // stages of the B (token rows) ring
 constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
@@ -53,6 +53,7 @@ struct alignas(8) GemmCtl {
   uint64_t full[kSB], emptyA[4], emptyB[kSB], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
+  long long wait;  // bound of the role hand-off waits (cycles)
   int n_groups;
   int total_tiles;
   int tile_prefix[257];  // tiles before group g
@@ -80,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, GemmCtl 
   const long long t0 = clock64();
   while (!mbar_try(b, parity)) {
     if (*((volatile int *)&ctl.abort)) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > ctl.wait) {
       *((volatile int *)&ctl.abort) = 1;
       set_error(err, kErrTimeout);
       return false;
@@ -427,6 +428,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     }
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
+    ctl.wait = a.wait_cycles > 0 ? a.wait_cycles : kDefaultWaitCycles;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (tid == 32) {  // group table
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       mma_commit(&ctl.drain);
       const long long t0 = clock64();
       while (!mbar_try(&ctl.drain, 0u)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > kDefaultWaitCycles) {
           set_error(a.err, kErrTimeout);
           break;
         }

@@ -45,6 +45,7 @@ struct GemmArgs {
   const int32_t *perm;
   int k;
   int *err;
+  long long wait_cycles;  // bound of the waits between the kernel's roles (0: the default)
 };
 
 cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms);

@@ -16,7 +16,12 @@ constexpr int kMaxE = 256;
 struct LayerDims {
   int H, I, Is, E, k, mode, flags, vocab;
   float scaling, eps;
+  // bound, in clock cycles, of a device wait on other warps' results (an h
+  // slice, the job table, a tensor-core pipeline hand-off); waits on a
+  // warp's own copies keep the default
+  long long wait_cycles;
 };
+constexpr long long kDefaultWaitCycles = 4000000000ll;  // about 2 s
 
 // Opaque TMA tensor descriptor (the driver's 128-byte, 64-byte aligned
 // CUtensorMap), built on the host and read by the TMA unit from the kernel's

@@ -472,6 +472,41 @@ cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_
   return cudaGetLastError();
 }
 
+namespace {
+// One thread per table row: the row must hold k distinct ids in [0, E);
+// the smallest failing row index is kept in *first_bad.
+__global__ void k_check_tid2eid(const int32_t *tab, int vocab, int k, int E, int *first_bad) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= vocab) return;
+  const int32_t *r = tab + (size_t)row * k;
+  int v[kMaxK];
+  bool ok = true;
+  for (int i = 0; i < k; ++i) {
+    v[i] = r[i];
+    if (v[i] < 0 || v[i] >= E) ok = false;
+    for (int j = 0; j < i; ++j)
+      if (v[j] == v[i]) ok = false;
+  }
+  if (!ok) atomicMin(first_bad, row);
+}
+}  // namespace
+
+cudaError_t check_tid2eid(const LayerDims &d, const int32_t *tab, int *dev_word, int *first_bad, cudaStream_t s) {
+  *first_bad = -1;
+  cudaError_t e = cudaMemsetAsync(dev_word, 0x7F, sizeof(int), s);  // 0x7F7F7F7F > any row index
+  if (e != cudaSuccess) return e;
+  k_check_tid2eid<<<(d.vocab + 255) / 256, 256, 0, s>>>(tab, d.vocab, d.k, d.E, dev_word);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int v = 0;
+  e = cudaMemcpyAsync(&v, dev_word, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  if (v < d.vocab) *first_bad = v;
+  return cudaSuccess;
+}
+
 static double *token_norm_ptr(const PrefillArgs &p) {
   uint8_t *fixp = reinterpret_cast<uint8_t *>(p.s.fix);
   return reinterpret_cast<double *>(fixp + align_up(sizeof(int32_t) * (size_t)(2 * p.T + 1), 256));
@@ -602,6 +637,7 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   g.h_ld = d.I;
   g.h_bf16 = 1;
   g.err = p.err;
+  g.wait_cycles = d.wait_cycles;
   if (p.ev_begin) cudaEventRecord(p.ev_begin, s);
   if ((e = grouped_gemm(g, s, num_sms)) != cudaSuccess) return e;
   if (p.ev_end) cudaEventRecord(p.ev_end, s);
@@ -643,6 +679,7 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   sd.y_ld = d.H;
   sd.res = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr;
   sd.err = p.err;
+  sd.wait_cycles = d.wait_cycles;
   if ((e = grouped_gemm(sd, s, num_sms)) != cudaSuccess) return e;
 
   // routed down: Q2_K x bf16 h, y[token] += w * (W_down h)

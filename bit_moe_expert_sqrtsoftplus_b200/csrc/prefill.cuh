@@ -40,6 +40,10 @@ size_t prefill_scratch_bytes(const LayerDims &d, int T);
 PrefillArgs prefill_args(const LayerDims &d, const LayerWeights &wt, int T, const float *x,
                          const int32_t *token_ids, float *y, void *scratch, const float *row_norms, int *err);
 cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_norms, int *err, cudaStream_t s);
+// Hash mode: checks that every row of the token-id table holds k distinct
+// expert ids in [0, E).  Uses one device int (dev_word) as a temporary, waits
+// for the stream, and sets *first_bad to the first failing row (-1 if none).
+cudaError_t check_tid2eid(const LayerDims &d, const int32_t *tab, int *dev_word, int *first_bad, cudaStream_t s);
 cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStream_t s);
 cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms);
 // Stable grouping of the T*k (token, slot) pairs by expert.

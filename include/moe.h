@@ -121,7 +121,14 @@ moe_status moe_workspace_size(const moe_config *cfg, int max_tokens, size_t *per
  * requires, 16-byte aligned), records them in a host-side handle and
  * enqueues the initialisation of `persist` on `stream` (it checks the
  * codebook range into the device error word).  The weight buffers are read,
- * never written, and must stay valid while the handle is used.
+ * never written, and must stay valid and unchanged while the handle is used.
+ *
+ * Hash mode: every row of tid2eid must hold top_k distinct expert ids in
+ * [0, n_experts) (the kernels index the expert weights with them and count
+ * each selected expert once per token).  moe_init checks the whole table on
+ * `stream` and waits for that check (the one synchronisation of this call);
+ * a row that breaks the rule returns MOE_ERR_INVALID_ARG naming the row, and
+ * no handle is created.
  */
 moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, size_t persist_bytes,
                     moe_stream_t stream, moe_handle **out);
@@ -201,6 +208,21 @@ const char *moe_last_error(void);
  * stop recording.  Recording changes no work the layer does.
  */
 moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end);
+
+/*
+ * Test hook for the device-side error path.  The kernels bound every wait on
+ * work of other warps or blocks (a down-projection unit waiting for the
+ * SwiGLU slice it reads, a warp waiting for its block's routing table, the
+ * hand-offs between the tensor-core kernel's producer, MMA and epilogue
+ * roles) at about 2 s; this sets that bound to `cycles` SM clock cycles for
+ * the later calls on this handle (0 restores the default).  A wait that runs
+ * out records MOE_ERR_TIMEOUT in the device error word and the kernel goes
+ * on or leaves without waiting further on others: it still waits for its
+ * own in-flight copies and tensor-core work (with the default bound), frees
+ * its tensor memory and returns, so the context stays usable.  That call's
+ * output is undefined; the next call starts from clean counters.
+ */
+moe_status moe_set_wait_limit(moe_handle *h, long long cycles);
 
 /*
  * Offline encoder: n fp32 values -> blocks of `format` (MOE_QUANT_Q8_0: n a

@@ -63,6 +63,8 @@ int main(void) {
         "value count not a multiple of 256");
   check(moe_quantize(MOE_QUANT_Q8_0, NULL, 0, NULL, NULL, NULL) == MOE_OK, "no values: a no-op");
 
+  check(moe_set_wait_limit(NULL, 100) == MOE_ERR_INVALID_ARG, "wait limit without a handle");
+
   moe_destroy(NULL);
   if (failures == 0) printf("C ABI checks passed\n");
   return failures == 0 ? 0 : 1;

@@ -62,28 +62,38 @@ def test_tiny_hash_prenorm_large_T(moe):
 
 
 def test_decode32_full_shape(moe):
+    """A second 32-token full-shape call (another seed and layer): it runs on
+    the small-T kernels, so every row is held to the GEMV tolerance."""
     s = synth.workload("decode_t32")
     x, tok, y, _ = _forward(moe, s, 1, 2, 32)
-    rows = np.arange(0, 32, 4)
-    yref = _oracle_rows(s, 1, 2, x, tok, rows)
-    rel, mx = harness.errors(y[rows], yref)
+    _, _, yref, _ = harness.oracle_layer_dense(s, 1, 2, x)
+    rel, mx = harness.errors(y, yref)
     print(f"decode_t32 rel_l2={rel:.3e} max_abs_frac={mx:.3e}")
-    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+    assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
 
 
-def test_prefill_4096_sampled_tokens(moe):
+def test_prefill_4096_every_row(moe):
+    """The full prefill call (4096 tokens, skewed bias): every output row
+    against the oracle (dense route).  The busiest and the quietest expert
+    and an expert whose token count is not a multiple of the 256-column N
+    tile are checked on their own tokens as well."""
     s = synth.workload("prefill_t4096")
     x, tok, y, L = _forward(moe, s, 0, 0, 4096)
-    # sample: spread tokens plus tokens of the most and least loaded experts
-    idx, _ = L.route(torch.from_numpy(x).cuda())
-    idx = idx.cpu().numpy()
+    assert np.all(np.isfinite(y))
+    idx_g, _ = L.route(torch.from_numpy(x).cuda())
+    idx_g = idx_g.cpu().numpy()
+    idx, _, yref, margin = harness.oracle_layer_dense(s, 0, 0, x)
+    assert np.array_equal(idx_g, idx), margin
     counts = np.bincount(idx.ravel(), minlength=s.n_experts)
-    busiest, quietest = int(counts.argmax()), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
-    rows = sorted(set([0, 1, 777, 2048, 4095] + list(np.nonzero((idx == busiest).any(1))[0][:3]) +
-                      list(np.nonzero((idx == quietest).any(1))[0][:2])))
-    yref = _oracle_rows(s, 0, 0, x, tok, np.array(rows))
-    rel, mx = harness.errors(y[rows], yref)
-    print(f"prefill_t4096 rows={rows} rel_l2={rel:.3e} max_abs_frac={mx:.3e} "
+    rel, mx = harness.errors(y, yref)
+    print(f"prefill_t4096 every row: rel_l2={rel:.3e} max_abs_frac={mx:.3e} "
           f"tokens/expert min {counts.min()} max {counts.max()}")
     assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
-    assert np.all(np.isfinite(y))
+    busiest = int(counts.argmax())
+    quietest = int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    ragged = [e for e in np.argsort(-counts) if counts[e] > 256 and counts[e] % 256][:1]
+    assert ragged, counts.max()
+    for e in [busiest, quietest] + ragged:
+        rows = np.nonzero((idx == e).any(1))[0]
+        r, m = harness.errors(y[rows], yref[rows])
+        assert r <= harness.MMA_REL_L2 and m <= harness.MAX_ABS_FRAC, (e, counts[e], r, m)

@@ -26,11 +26,17 @@ def moe():
 
 @pytest.mark.parametrize("name,T", [("tiny", 4), ("decode_t1", 1), ("decode_t1", 8)])
 def test_noalloc_matches_scratch_forward_on_two_calls(moe, name, T):
+    """Two calls in a row through the no-allocation entry point, each against
+    the forward with caller scratch and against the fp64 oracle."""
     s = synth.workload(name, tokens=T)
     W = harness.device_layer(s, 6, 1)
     L = moe.Layer(harness.config_for(s), W, max_tokens=T)
-    x = torch.from_numpy(synth.activations(6, T, s.hidden, stream=1)).cuda()
+    x_np = synth.activations(6, T, s.hidden, stream=1)
+    x = torch.from_numpy(x_np).cuda()
     ref = L.forward(x).cpu().numpy()
+    _, _, yref, _ = harness.oracle_layer_dense(s, 6, 1, x_np)
+    rel, mx = harness.errors(ref, yref)
+    assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
     for _ in range(2):
         y = torch.full_like(x, float("nan"))
         moe.moe_ffn_forward_noalloc(L.handle, x, None, T, y)
@@ -38,6 +44,8 @@ def test_noalloc_matches_scratch_forward_on_two_calls(moe, name, T):
         L.poll()
         got = y.cpu().numpy()
         rel, mx = harness.errors(got, ref)
+        assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+        rel, mx = harness.errors(got, yref)
         assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
 
 
