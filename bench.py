@@ -35,6 +35,7 @@ import subprocess
 import sys
 import threading
 import time
+from dataclasses import replace
 
 import numpy as np
 
@@ -46,21 +47,23 @@ import synth  # noqa: E402
 METRIC = "MoE-layer tokens/s and % HBM roofline (decode) / % bf16 TC roofline (prefill)"
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode_t1",
-                   choices=["decode_t1", "decode_t32", "prefill_t4096", "stack43_t8", "stack43_t8_q2q4",
+                   choices=["decode_t1", "tiny", "decode_t32", "prefill_t4096", "stack43_t8", "stack43_t8_q2q4",
                             "decode_t1_q4k", "quantize_q2k", "quantize_q80", "quantize_q4k"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
     p.add_argument("--sweep", action="store_true",
                    help="time one layer call at T = 1, 2, 4, ..., 256 (skewed bias; one JSON line per T)")
-    return p.parse_args()
+    p.add_argument("--no-extras", action="store_true",
+                   help="decode_t1 only: skip the other workloads and the sweep that the default run adds")
+    return p.parse_args(argv)
 
 
 def load_peaks():
@@ -99,7 +102,8 @@ def load_traffic(workload: str):
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """nvidia-smi samples every 50 ms while the workload runs (warm-up, the
+    timed region and the passes after it)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -112,7 +116,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
@@ -249,11 +253,6 @@ def run_ours(args, world, rank):
     def step(i):
         layers[i % nsets].forward(xs[i % npool], None, ys[i % npool])
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    layers[0].poll()
-
     # distinct experts per call (for the byte count): from the routing of the pool
     nd = []
     for j in range(min(npool, 8)):
@@ -264,6 +263,17 @@ def run_ours(args, world, rank):
     stream = torch.cuda.current_stream()
     clock = ClockSampler(torch.cuda.current_device())
     with clock:
+        # warm-up: W steps, continued (untimed) to at least 0.4 s so that the
+        # clock samples cover the load right before the timed region
+        t_w = time.perf_counter()
+        wu = 0
+        while wu < args.warmup or time.perf_counter() - t_w < 0.4:
+            step(wu)
+            wu += 1
+            if wu % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        layers[0].poll()
         # pass 1: the timed region
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -355,8 +365,10 @@ def run_ours(args, world, rank):
         "config": {"workload": f"{args.workload}: V4-Flash MoE layer, T={T} tokens/call, hidden {s.hidden}, "
                                f"{s.n_experts} experts top-{s.top_k}, inter {s.inter}, shared {s.shared_inter}",
                    "tokens_per_call": T, "weight_sets_rotated": nsets,
-                   "l2": f"{nsets} rotating weight sets of {s.n_experts * s.expert_bytes / 1e9:.2f} GB "
-                         "(inputs far larger than the 126 MB L2)",
+                   "l2": (f"{nsets} rotating weight set(s) of {s.n_experts * s.expert_bytes / 1e9:.2f} GB "
+                          "(inputs far larger than the 126 MB L2)" if s.n_experts * s.expert_bytes > 126e6 else
+                          f"one weight set of {(s.n_experts * s.expert_bytes + s.shared_bytes) / 1e6:.2f} MB, "
+                          "resident in the 126 MB L2 (a latency figure)"),
                    "parallelism": f"replicas x{world}"},
         "roofline": roof if large else
         {"bound": "hbm", "kernel": ("Q4_K expert kernels (input, gate/up with SwiGLU, down with the combine)" if s.q4k
@@ -477,25 +489,32 @@ def run_stack(args, world, rank):
     }
 
 
-def oracle_rate(s: synth.LayerShape, budget_s: float, max_steps: int, seed: int = 0):
-    """Tokens/s of the fp64 oracle on full layer calls of the workload
-    (weight set 0, inputs resident), as many calls as fit in the budget."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_rate(s: synth.LayerShape, budget_s: float, max_steps: int, seed: int = 0, threads: int = 1):
+    """Tokens/s of the fp64 oracle on layer calls of the workload's shapes
+    (weight set 0, inputs resident), as many calls as fit in the budget.
+    A call takes a slice of min(T, max(4, threads)) tokens, split over
+    `threads` threads (the oracle splits a call's tokens)."""
     import oracle
     W = synth.host_layer(seed, 0, s, q4k=s.q4k)
     Wr, b = W["router_w"], W["bias"]
-    T = min(s.tokens, 4)  # large batches: a 4-token slice per oracle call
+    T = min(s.tokens, max(4, threads))
     n = 0
-    t0 = time.perf_counter()
     elapsed = 0.0
     while n < max_steps and (n == 0 or elapsed < budget_s):
         x = synth.activations(7, T, s.hidden, stream=100 + n).astype(np.float64)
         a = time.perf_counter()
         idx, w, _ = oracle.route(x, Wr, b, s.top_k, s.routed_scaling)
-        oracle.layer(W, s, x, idx, w)
+        oracle.layer(W, s, x, idx, w, threads=threads)
         elapsed += time.perf_counter() - a
         n += 1
-    del t0
-    return n * T / elapsed, n, elapsed
+    return n * T / elapsed, n, elapsed, T
 
 
 class OracleSampler:
@@ -745,18 +764,54 @@ def run_sweep(args, world, rank):
     return lines
 
 
-def cpu_baseline(args) -> dict:
-    """The oracle on a bounded sample of the workload, on one host core."""
+def cpu_baseline(args, budget: float = 0.0) -> dict:
+    """The oracle on a bounded sample of the workload, on the host's cores."""
+    budget = budget or args.cpu_seconds
     if args.workload.startswith("quantize_"):
-        steps = max(1, int(args.cpu_seconds / 0.005))  # about 5 ms per 2^20 values
+        steps = max(1, int(budget / 0.005))  # about 5 ms per 2^20 values
         value, elapsed = oracle_quant_rate(args.workload, steps, 3)
         return {"value": value, "unit": "values/s", "cores": 1, "kind": "oracle",
                 "sample": f"{steps} x 2^20 values through the C oracle's encoder, single thread, {elapsed:.1f} s"}
     s = synth.workload(args.workload)
-    value, n, elapsed = oracle_rate(s, args.cpu_seconds, 1000)
-    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} full layer calls (T={s.tokens}) of the fp64 C oracle on weight set 0, "
-                      f"single thread, {elapsed:.1f} s"}
+    stack = s.layers > 1
+    if stack:  # one router layer of the stack, with its pre-norm and skew settings
+        s = replace(s, layers=1, hash_layers=0, q4k_layers=0)
+    threads = min(host_cores(), s.tokens)
+    value, n, elapsed, T = oracle_rate(s, budget, 1000, threads=threads)
+    why = ("; one thread because the oracle splits a call's tokens over threads and this call has one token"
+           if s.tokens == 1 else "")
+    out = {"value": value / (synth.workload(args.workload).layers if stack else 1), "unit": "tokens/s",
+           "cores": threads, "kind": "oracle",
+           "sample": f"{n} layer calls of {T} tokens (the workload's shapes) of the fp64 C oracle on weight set 0, "
+                     f"{threads} thread(s), {elapsed:.1f} s{why}"
+                     + (f"; tokens/s through the {synth.workload(args.workload).layers}-layer stack = one layer's "
+                        f"rate / {synth.workload(args.workload).layers}" if stack else "")}
+    return out
+
+
+EXTRA_WORKLOADS = ("tiny", "decode_t32", "prefill_t4096", "stack43_t8")
+
+
+def run_extras(args, world, rank):
+    """The other configurations of the layer, each measured like the headline
+    (its own timed region, dominant-kernel roofline, end-to-end pass, clocks
+    and oracle baseline), then the batch sweep."""
+    import torch
+    out = {}
+    for name in EXTRA_WORKLOADS:
+        sub = argparse.Namespace(**vars(args))
+        sub.workload = name
+        sub.weight_sets = 0
+        r = run_stack(sub, world, rank) if name.startswith("stack") else run_ours(sub, world, rank)
+        torch.cuda.empty_cache()
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            r["cpu_baseline"] = cpu_baseline(sub, budget=args.cpu_seconds / 2)
+        for k in ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data"):
+            r.pop(k, None)
+        out[name] = r
+    sweep = run_sweep(args, world, rank)
+    torch.cuda.empty_cache()
+    return out, sweep
 
 
 def main():
@@ -785,6 +840,11 @@ def main():
         out = run_ours(args, world, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args)
+    if args.workload == "decode_t1" and not args.no_extras:
+        extras, sweep = run_extras(args, world, rank)
+        out["workloads"] = extras
+        out["sweep"] = sweep
+        out["gpu_launches_all_workloads"] = out["gpu_launches"] + sum(r["gpu_launches"] for r in extras.values())
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -372,8 +372,10 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
 // Scratch for moe_ffn_forward_noalloc: one buffer per device that loads this
 // library, held until the process exits.  Host code must not take the
 // array's address directly (its name stands for a host-side shadow); the
-// device address comes from cudaGetSymbolAddress, looked up once per device
-// with that device current and cached below.
+// device address comes from cudaGetSymbolAddress with the device current.
+// It is looked up again on every call made outside stream capture (after a
+// cudaDeviceReset the module is loaded anew and the array may move) and the
+// last address is kept per device for calls made during a capture.
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
@@ -384,10 +386,13 @@ constexpr int kMaxDevices = 128;
 void *g_static_scratch_addr[kMaxDevices] = {};
 std::mutex g_static_scratch_mutex;
 
-moe_status static_scratch_for(int dev, void **out) {
+moe_status static_scratch_for(int dev, cudaStream_t stream, void **out) {
   if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t ce = cudaStreamIsCapturing(stream, &cap);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaStreamIsCapturing");
   std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-  if (!g_static_scratch_addr[dev]) {
+  if (!g_static_scratch_addr[dev] || cap == cudaStreamCaptureStatusNone) {
     void *p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
@@ -424,7 +429,7 @@ moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t 
   moe_status st = check_device(h);
   if (st != MOE_OK) return st;
   void *scratch = nullptr;
-  st = static_scratch_for(h->device, &scratch);
+  st = static_scratch_for(h->device, reinterpret_cast<cudaStream_t>(stream), &scratch);
   if (st != MOE_OK) return st;
   moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
   const cudaError_t e = moe::decode_forward(a, reinterpret_cast<cudaStream_t>(stream), h->num_sms);

@@ -180,9 +180,11 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
  * in 16 MiB (the V4-Flash shapes need about 6.2 MiB at T = 8); larger requests
  * return MOE_ERR_UNSUPPORTED_SHAPE or MOE_ERR_WORKSPACE_TOO_SMALL with a
  * message.  T = 0 is a no-op.  The current device must be the handle's
- * device.  The first call on a device looks up the buffer's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  Every call on a device shares the one
+ * device.  Each call made outside stream capture looks up the buffer's device
+ * address (cudaGetSymbolAddress, with that device current; the lookup also
+ * follows the buffer after a cudaDeviceReset) and keeps it for calls made
+ * while `stream` is being captured; make the first call on a device before
+ * any stream capture.  Every call on a device shares the one
  * buffer and leaves its contents behind; the kernels clear the counters they
  * need at the start of each call.  Calls whose executions overlap on the GPU
  * (different streams, or different handles on the same device) race on the
