@@ -28,6 +28,8 @@ MOE_ERR_DEVICE_FAULT = -7
 MOE_ROUTE_ROUTER = 0
 MOE_ROUTE_HASH = 1
 MOE_FLAG_PRENORM_RESIDUAL = 1
+MOE_FLAG_EXPERTS_ONLY = 2
+MOE_FLAG_NO_ROUTED = 4
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
 MOE_QUANT_Q8_0 = 0
 MOE_QUANT_Q2_K = 1
@@ -38,7 +40,7 @@ MOE_ROUTED_Q4K = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
             "moe_last_error", "moe_set_timing_events", "moe_set_wait_limit", "moe_ffn_forward_noalloc", "moe_quantize",
-            "moe_destroy")
+            "moe_ep_workspace_size", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_destroy")
 
 
 class moe_config(ctypes.Structure):
@@ -87,6 +89,13 @@ def lib():
         L.moe_set_wait_limit.restype = i32
         L.moe_quantize.argtypes = [i32, vp, ctypes.c_int64, vp, vp, vp]
         L.moe_quantize.restype = i32
+        L.moe_ep_workspace_size.argtypes = [ctypes.POINTER(moe_config), i32, i32, ctypes.POINTER(sz),
+                                            ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.moe_ep_dispatch.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_ep_experts.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+        L.moe_ep_combine.argtypes = [vp, vp, i32, vp, vp, vp, vp, sz, vp]
+        for name in ("moe_ep_workspace_size", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine"):
+            getattr(L, name).restype = i32
         L.moe_destroy.argtypes = [vp]
         L.moe_destroy.restype = None
         for name in ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error"):
@@ -191,6 +200,32 @@ def quantize(fmt, x, stream=None):
     bad = torch.zeros(1, dtype=torch.int32, device=x.device)
     moe_quantize(fmt, x, out, bad, stream)
     return out, bad
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def moe_ep_workspace_size(cfg: moe_config, max_tokens: int, max_recv_rows: int):
+    a, b, c = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib().moe_ep_workspace_size(ctypes.byref(cfg), max_tokens, max_recv_rows, ctypes.byref(a),
+                                       ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def moe_ep_dispatch(handle, x, token_ids, T, offsets, perm, x_send, e_send, w_send, scratch, stream=None):
+    _check(lib().moe_ep_dispatch(handle, _ptr(x), _ptr(token_ids), T, _ptr(offsets), _ptr(perm), _ptr(x_send),
+                                 _ptr(e_send), _ptr(w_send), _ptr(scratch), _nbytes(scratch), _stream(stream)))
+
+
+def moe_ep_experts(handle, x_recv, e_recv, w_recv, N, first_expert, out, scratch, stream=None):
+    _check(lib().moe_ep_experts(handle, _ptr(x_recv), _ptr(e_recv), _ptr(w_recv), N, first_expert, _ptr(out),
+                                _ptr(scratch), _nbytes(scratch), _stream(stream)))
+
+
+def moe_ep_combine(handle, x, T, perm, out_back, y, scratch, stream=None):
+    _check(lib().moe_ep_combine(handle, _ptr(x), T, _ptr(perm), _ptr(out_back), _ptr(y), _ptr(scratch),
+                                _nbytes(scratch), _stream(stream)))
 
 
 def moe_destroy(handle):

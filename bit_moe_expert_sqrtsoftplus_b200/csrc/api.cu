@@ -1,4 +1,5 @@
 // api.cu -- the extern "C" boundary declared in include/moe.h.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
@@ -75,7 +76,10 @@ moe_status check_config(const moe_config *c) {
   if (!isfinite(c->routed_scaling)) return fail(MOE_ERR_INVALID_ARG, "routed_scaling is not finite");
   if ((c->flags & MOE_FLAG_PRENORM_RESIDUAL) && !(c->rms_eps >= 0.f && isfinite(c->rms_eps)))
     return fail(MOE_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
-  if (c->flags & ~MOE_FLAG_PRENORM_RESIDUAL) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
+  if (c->flags & ~(MOE_FLAG_PRENORM_RESIDUAL | MOE_FLAG_EXPERTS_ONLY | MOE_FLAG_NO_ROUTED))
+    return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
+  if ((c->flags & MOE_FLAG_EXPERTS_ONLY) && (c->flags & MOE_FLAG_NO_ROUTED))
+    return fail(MOE_ERR_INVALID_ARG, "MOE_FLAG_EXPERTS_ONLY and MOE_FLAG_NO_ROUTED exclude each other");
   if (c->routed_format != MOE_ROUTED_Q2 && c->routed_format != MOE_ROUTED_Q4K)
     return fail(MOE_ERR_INVALID_ARG, "routed_format=%d is not a MOE_ROUTED_* format", c->routed_format);
   return MOE_OK;
@@ -133,6 +137,13 @@ moe_status check_device(const moe_handle *h) {
   return MOE_OK;
 }
 
+moe_status check_whole_layer(const moe_handle *h) {
+  if (h->d.flags & (MOE_FLAG_EXPERTS_ONLY | MOE_FLAG_NO_ROUTED))
+    return fail(MOE_ERR_INVALID_ARG, "a handle made with MOE_FLAG_EXPERTS_ONLY or MOE_FLAG_NO_ROUTED serves the "
+                                     "moe_ep_* calls only");
+  return MOE_OK;
+}
+
 moe_status check_call(moe_handle *h, const float *x, const int32_t *token_ids, int T, void *scratch,
                       size_t scratch_bytes) {
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
@@ -172,16 +183,23 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
-  const void *need[] = {w->gate_iq2xxs, w->up_iq2xxs, w->down_q2k, w->sh_gate_q80, w->sh_up_q80, w->sh_down_q80,
-                        w->iq2_grid};
-  const char *names[] = {"gate_iq2xxs", "up_iq2xxs", "down_q2k", "sh_gate_q80", "sh_up_q80", "sh_down_q80",
-                         "iq2_grid"};
-  const int n_need = cfg->routed_format == MOE_ROUTED_Q4K ? 6 : 7;  // Q4_K layers read no codebook
-  for (int i = 0; i < n_need; ++i) {
+  const bool experts_only = (cfg->flags & MOE_FLAG_EXPERTS_ONLY) != 0;
+  const bool no_routed = (cfg->flags & MOE_FLAG_NO_ROUTED) != 0;
+  const void *need[] = {w->gate_iq2xxs, w->up_iq2xxs, w->down_q2k, w->iq2_grid, w->sh_gate_q80, w->sh_up_q80,
+                        w->sh_down_q80};
+  const char *names[] = {"gate_iq2xxs", "up_iq2xxs", "down_q2k", "iq2_grid", "sh_gate_q80", "sh_up_q80",
+                         "sh_down_q80"};
+  for (int i = 0; i < 7; ++i) {
+    const bool routed = i < 4;
+    if (routed && no_routed) continue;                                   // router and shared expert only
+    if (!routed && experts_only) continue;                               // routed experts only
+    if (i == 3 && cfg->routed_format == MOE_ROUTED_Q4K) continue;        // Q4_K layers read no codebook
     if (!need[i]) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", names[i]);
     if (!aligned16(need[i])) return fail(MOE_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
   }
-  if (cfg->mode == MOE_ROUTE_ROUTER) {
+  if (experts_only) {
+    // no routing
+  } else if (cfg->mode == MOE_ROUTE_ROUTER) {
     if (!w->router_w_f16 || !w->router_bias) return fail(MOE_ERR_INVALID_ARG, "router mode needs router_w_f16 and router_bias");
     if (!aligned16(w->router_w_f16) || !aligned16(w->router_bias))
       return fail(MOE_ERR_MISALIGNED, "router weights are not 16-byte aligned");
@@ -218,7 +236,7 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   h->wt.sh_down = static_cast<const uint8_t *>(w->sh_down_q80);
   h->wt.grid = w->iq2_grid;
   h->wt.tma = 0;
-  if (cfg->routed_format == MOE_ROUTED_Q2) moe::build_chunk_tensor_maps(h->wt, h->d);
+  if (cfg->routed_format == MOE_ROUTED_Q2 && !no_routed && !experts_only) moe::build_chunk_tensor_maps(h->wt, h->d);
   h->err = static_cast<int *>(persist);
   h->row_norms = reinterpret_cast<float *>(static_cast<uint8_t *>(persist) + kPersistHeader);
   h->num_sms = sms;
@@ -231,12 +249,12 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
     delete h;
     return cuda_fail(e, "cudaMemsetAsync(persist)");
   }
-  e = moe::prefill_init(h->d, h->wt, h->row_norms, h->err, s);
+  if (!experts_only) e = moe::prefill_init(h->d, h->wt, h->row_norms, h->err, s);
   if (e != cudaSuccess) {
     delete h;
     return cuda_fail(e, "init kernels");
   }
-  if (cfg->mode == MOE_ROUTE_HASH) {
+  if (cfg->mode == MOE_ROUTE_HASH && !experts_only) {
     // the kernels index the weights with the table's ids and assume a token
     // selects an expert once: check every row before the handle is used
     int bad = -1;
@@ -315,6 +333,8 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
                      moe_stream_t stream) {
   moe_status st = check_call(h, x, token_ids, T, scratch, scratch_bytes);
   if (st != MOE_OK) return st;
+  if (h->d.flags & MOE_FLAG_EXPERTS_ONLY)
+    return fail(MOE_ERR_INVALID_ARG, "a MOE_FLAG_EXPERTS_ONLY handle has no router");
   if (T == 0) return MOE_OK;
   if (!idx || !w) return fail(MOE_ERR_INVALID_ARG, "idx and w must not be NULL");
   if ((expert_offsets == nullptr) != (perm == nullptr))
@@ -339,8 +359,10 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
 
 moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y, void *scratch,
                            size_t scratch_bytes, moe_stream_t stream) {
-  moe_status st = check_call(h, x, token_ids, T, scratch, scratch_bytes);
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  moe_status st = check_whole_layer(h);
   if (st != MOE_OK) return st;
+  if ((st = check_call(h, x, token_ids, T, scratch, scratch_bytes)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   if (!y) return fail(MOE_ERR_INVALID_ARG, "y is NULL");
   if (!aligned16(y)) return fail(MOE_ERR_MISALIGNED, "y is not 16-byte aligned");
@@ -410,6 +432,8 @@ moe_status moe_ffn_forward_noalloc(moe_handle *h, const float *x, const int32_t 
                                    moe_stream_t stream) {
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  moe_status wl = check_whole_layer(h);
+  if (wl != MOE_OK) return wl;
   if (T == 0) return MOE_OK;
   if (h->cfg.routed_format != MOE_ROUTED_Q2)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_forward_noalloc runs the q2 routed formats only");
@@ -504,6 +528,92 @@ moe_status moe_quantize(int format, const float *x, int64_t n, void *out, int32_
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   e = moe::quantize_blocks(format, x, n / per, out, nonfinite_blocks, reinterpret_cast<cudaStream_t>(stream), sms);
   if (e != cudaSuccess) return cuda_fail(e, "moe_quantize launch");
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ expert parallelism
+
+moe_status moe_ep_workspace_size(const moe_config *cfg, int max_tokens, int max_recv_rows, size_t *dispatch_bytes,
+                                 size_t *experts_bytes, size_t *combine_bytes) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (max_tokens < 0 || max_recv_rows < 0) return fail(MOE_ERR_INVALID_ARG, "negative sizes");
+  const moe::LayerDims d = dims_of(*cfg);
+  if (dispatch_bytes) *dispatch_bytes = max_tokens > 0 ? moe::ep_dispatch_scratch_bytes(d, max_tokens) : 0;
+  if (experts_bytes) *experts_bytes = max_recv_rows > 0 ? moe::ep_experts_scratch_bytes(d, max_recv_rows) : 0;
+  if (combine_bytes) *combine_bytes = max_tokens > 0 ? moe::ep_combine_scratch_bytes(d, max_tokens) : 0;
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_ep_dispatch(moe_handle *h, const float *x, const int32_t *token_ids, int T, int32_t *expert_offsets,
+                           int32_t *perm, void *x_send, int32_t *e_send, float *w_send, void *scratch,
+                           size_t scratch_bytes, moe_stream_t stream) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.flags & MOE_FLAG_EXPERTS_ONLY) return fail(MOE_ERR_INVALID_ARG, "an experts-only handle has no router");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  if (T == 0) return MOE_OK;
+  if (!x || !expert_offsets || !perm || !x_send || !e_send || !w_send || !scratch)
+    return fail(MOE_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(x) || !aligned16(x_send) || !aligned16(scratch))
+    return fail(MOE_ERR_MISALIGNED, "x, x_send and scratch must be 16-byte aligned");
+  if (h->d.mode == MOE_ROUTE_HASH && !token_ids) return fail(MOE_ERR_INVALID_ARG, "hash mode needs token_ids");
+  const size_t need = moe::ep_dispatch_scratch_bytes(h->d, T);
+  if (scratch_bytes < need)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for T=%d", scratch_bytes, need, T);
+  moe_status st = check_device(h);
+  if (st != MOE_OK) return st;
+  moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, nullptr, scratch, h->row_norms, h->err);
+  const cudaError_t e = moe::ep_dispatch(p, expert_offsets, perm, static_cast<__half *>(x_send), e_send, w_send,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "moe_ep_dispatch launch");
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_ep_experts(moe_handle *shard, const void *x_recv, const int32_t *e_recv, const float *w_recv, int N,
+                          int first_expert, float *out, void *scratch, size_t scratch_bytes, moe_stream_t stream) {
+  if (!shard) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (shard->d.flags & MOE_FLAG_NO_ROUTED) return fail(MOE_ERR_INVALID_ARG, "this handle holds no routed experts");
+  if (N < 0 || first_expert < 0) return fail(MOE_ERR_INVALID_ARG, "negative N or first_expert");
+  if (N == 0) return MOE_OK;
+  if (!x_recv || !e_recv || !w_recv || !out || !scratch) return fail(MOE_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(x_recv) || !aligned16(out) || !aligned16(scratch))
+    return fail(MOE_ERR_MISALIGNED, "x_recv, out and scratch must be 16-byte aligned");
+  const size_t need = moe::ep_experts_scratch_bytes(shard->d, N);
+  if (scratch_bytes < need)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for %d rows", scratch_bytes, need, N);
+  moe_status st = check_device(shard);
+  if (st != MOE_OK) return st;
+  const cudaError_t e =
+      moe::ep_experts(shard->d, shard->wt, shard->cfg.routed_format == MOE_ROUTED_Q4K, static_cast<const __half *>(x_recv),
+                      e_recv, w_recv, N, first_expert, out, scratch, shard->err, reinterpret_cast<cudaStream_t>(stream),
+                      shard->num_sms);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_ep_experts launch");
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(moe_handle *h, const float *x, int T, const int32_t *perm, const float *out_back, float *y,
+                          void *scratch, size_t scratch_bytes, moe_stream_t stream) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.flags & MOE_FLAG_EXPERTS_ONLY) return fail(MOE_ERR_INVALID_ARG, "an experts-only handle has no shared expert");
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+  if (T == 0) return MOE_OK;
+  if (!x || !perm || !out_back || !y || !scratch) return fail(MOE_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(x) || !aligned16(out_back) || !aligned16(y) || !aligned16(scratch))
+    return fail(MOE_ERR_MISALIGNED, "x, out_back, y and scratch must be 16-byte aligned");
+  if (y == x && !(h->d.flags & MOE_FLAG_PRENORM_RESIDUAL))
+    return fail(MOE_ERR_INVALID_ARG, "y may alias x only with MOE_FLAG_PRENORM_RESIDUAL");
+  const size_t need = moe::ep_combine_scratch_bytes(h->d, T);
+  if (scratch_bytes < need)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "scratch has %zu bytes, %zu needed for T=%d", scratch_bytes, need, T);
+  moe_status st = check_device(h);
+  if (st != MOE_OK) return st;
+  const cudaError_t e = moe::ep_combine(h->d, h->wt, x, T, perm, out_back, y, scratch, h->err,
+                                        reinterpret_cast<cudaStream_t>(stream), h->num_sms);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_ep_combine launch");
   g_last_error.clear();
   return MOE_OK;
 }

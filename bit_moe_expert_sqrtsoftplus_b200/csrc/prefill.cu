@@ -598,6 +598,124 @@ BigScratch carve_big(const LayerDims &d, int T, void *base) {
 
 size_t prefill_big_bytes(const LayerDims &d, int T) { return carve_big(d, T, nullptr).bytes; }
 
+namespace {
+
+// Routed gate/up GEMM over (token, slot) pairs grouped by expert: column c
+// (offsets[g] <= c < offsets[g+1] for group g) reads activation row
+// perm[c] / b_div of x16; SwiGLU outputs h (bf16) in grouped order.
+GemmArgs routed_gateup_args(const LayerDims &d, const LayerWeights &wt, bool q4k, int n_groups,
+                            const int32_t *offsets, const int32_t *perm, int b_div, const __half *x16,
+                            uint16_t *hperm, int *err) {
+  const size_t rbIQ = (size_t)(d.H / 256) * (q4k ? 144 : 66);
+  GemmArgs g{};
+  g.fmt = q4k ? kFmtQ4K : kFmtIQ2;
+  g.bf16 = 0;
+  g.epi = kEpiSwiGLU;
+  g.M = d.I;
+  g.K = d.H;
+  g.n_groups = n_groups;
+  g.offsets = offsets;
+  g.A0 = wt.gate;
+  g.A1 = wt.up;
+  g.a_group_stride = (size_t)d.I * rbIQ;
+  g.a_row_bytes = rbIQ;
+  g.grid = wt.grid;
+  g.b_base = reinterpret_cast<const uint16_t *>(x16);
+  g.b_ld = d.H;
+  g.b_perm = perm;
+  g.b_div = b_div;
+  g.h_out = hperm;
+  g.h_ld = d.I;
+  g.h_bf16 = 1;
+  g.err = err;
+  g.wait_cycles = d.wait_cycles;
+  return g;
+}
+
+// Routed down GEMM: y[(perm[c] / k) * H + m] += w[perm[c]] * (W_down h)[m].
+GemmArgs routed_down_args(const LayerDims &d, const LayerWeights &wt, bool q4k, int n_groups, const int32_t *offsets,
+                          const int32_t *perm, int k, const uint16_t *hperm, const float *w, float *y, int *err) {
+  const size_t rbQ2 = (size_t)(d.I / 256) * (q4k ? 144 : 84);
+  GemmArgs rd{};
+  rd.fmt = q4k ? kFmtQ4K : kFmtQ2K;
+  rd.bf16 = 1;
+  rd.epi = kEpiScatterAdd;
+  rd.M = d.H;
+  rd.K = d.I;
+  rd.n_groups = n_groups;
+  rd.offsets = offsets;
+  rd.A0 = wt.down;
+  rd.A1 = nullptr;
+  rd.a_group_stride = (size_t)d.H * rbQ2;
+  rd.a_row_bytes = rbQ2;
+  rd.b_base = hperm;
+  rd.b_ld = d.I;
+  rd.b_perm = nullptr;
+  rd.b_div = 1;
+  rd.y = y;
+  rd.y_ld = d.H;
+  rd.w = w;
+  rd.perm = perm;
+  rd.k = k;
+  rd.err = err;
+  rd.wait_cycles = d.wait_cycles;
+  return rd;
+}
+
+// The shared expert over T activation rows: SwiGLU into hs, then the down
+// projection stored into y (plus res, the residual input, when given).
+cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, const __half *x16, uint16_t *hs,
+                         const float *res, float *y, int *err, cudaStream_t s, int num_sms) {
+  GemmArgs sg{};
+  sg.fmt = kFmtQ80;
+  sg.bf16 = 0;
+  sg.epi = kEpiSwiGLU;
+  sg.M = d.Is;
+  sg.K = d.H;
+  sg.n_groups = 1;
+  sg.offsets = nullptr;
+  sg.cols = T;
+  sg.A0 = wt.sh_gate;
+  sg.A1 = wt.sh_up;
+  sg.a_group_stride = 0;
+  sg.a_row_bytes = (size_t)(d.H / 32) * 34;
+  sg.grid = wt.grid;
+  sg.b_base = reinterpret_cast<const uint16_t *>(x16);
+  sg.b_ld = d.H;
+  sg.b_perm = nullptr;
+  sg.b_div = 1;
+  sg.h_out = hs;
+  sg.h_ld = d.Is;
+  sg.h_bf16 = 1;
+  sg.err = err;
+  sg.wait_cycles = d.wait_cycles;
+  cudaError_t e = grouped_gemm(sg, s, num_sms);
+  if (e != cudaSuccess) return e;
+  GemmArgs sd{};
+  sd.fmt = kFmtQ80;
+  sd.bf16 = 1;
+  sd.epi = kEpiStore;
+  sd.M = d.H;
+  sd.K = d.Is;
+  sd.n_groups = 1;
+  sd.offsets = nullptr;
+  sd.cols = T;
+  sd.A0 = wt.sh_down;
+  sd.A1 = nullptr;
+  sd.a_row_bytes = (size_t)(d.Is / 32) * 34;
+  sd.b_base = hs;
+  sd.b_ld = d.Is;
+  sd.b_div = 1;
+  sd.y = y;
+  sd.y_ld = d.H;
+  sd.res = res;
+  sd.err = err;
+  sd.wait_cycles = d.wait_cycles;
+  return grouped_gemm(sd, s, num_sms);
+}
+
+}  // namespace
+
 cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   const LayerDims &d = p.d;
   const int T = p.T;
@@ -609,98 +727,188 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   k_prep_x16<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, b.x16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // routed rows: IQ2_XXS gate/up and Q2_K down, or Q4_K for all three
-  const size_t rbIQ = (size_t)(d.H / 256) * (p.q4k ? 144 : 66);
-  const size_t rbQ2 = (size_t)(d.I / 256) * (p.q4k ? 144 : 84);
-  const size_t rbQ8h = (size_t)(d.H / 32) * 34;
-  const size_t rbQ8s = (size_t)(d.Is / 32) * 34;
-
-  // routed gate/up: IQ2_XXS x f16 activations, SwiGLU -> h (bf16) in permuted order
-  GemmArgs g{};
-  g.fmt = p.q4k ? kFmtQ4K : kFmtIQ2;
-  g.bf16 = 0;
-  g.epi = kEpiSwiGLU;
-  g.M = d.I;
-  g.K = d.H;
-  g.n_groups = d.E;
-  g.offsets = p.s.offsets;
-  g.A0 = p.wt.gate;
-  g.A1 = p.wt.up;
-  g.a_group_stride = (size_t)d.I * rbIQ;
-  g.a_row_bytes = rbIQ;
-  g.grid = p.wt.grid;
-  g.b_base = reinterpret_cast<const uint16_t *>(b.x16);
-  g.b_ld = d.H;
-  g.b_perm = p.s.perm;
-  g.b_div = d.k;
-  g.h_out = b.hperm;
-  g.h_ld = d.I;
-  g.h_bf16 = 1;
-  g.err = p.err;
-  g.wait_cycles = d.wait_cycles;
+  // routed gate/up: IQ2_XXS (or Q4_K) x f16 activations, SwiGLU -> h (bf16) in permuted order
+  const GemmArgs g = routed_gateup_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.x16, b.hperm, p.err);
   if (p.ev_begin) cudaEventRecord(p.ev_begin, s);
   if ((e = grouped_gemm(g, s, num_sms)) != cudaSuccess) return e;
   if (p.ev_end) cudaEventRecord(p.ev_end, s);
+  // shared expert: Q8_0 gate/up over all tokens, down stored into y (plus the residual input when pre-norm)
+  e = shared_gemms(d, p.wt, T, b.x16, b.hs, (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr, p.y, p.err, s,
+                   num_sms);
+  if (e != cudaSuccess) return e;
+  // routed down: Q2_K (or Q4_K) x bf16 h, y[token] += w * (W_down h)
+  return grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, p.s.w, p.y, p.err),
+                      s, num_sms);
+}
 
-  // shared gate/up: Q8_0 x f16 activations over all tokens, SwiGLU -> hs (bf16)
-  GemmArgs sg = g;
-  sg.fmt = kFmtQ80;
-  sg.M = d.Is;
-  sg.n_groups = 1;
-  sg.offsets = nullptr;
-  sg.cols = T;
-  sg.A0 = p.wt.sh_gate;
-  sg.A1 = p.wt.sh_up;
-  sg.a_group_stride = 0;
-  sg.a_row_bytes = rbQ8h;
-  sg.b_perm = nullptr;
-  sg.b_div = 1;
-  sg.h_out = b.hs;
-  sg.h_ld = d.Is;
-  if ((e = grouped_gemm(sg, s, num_sms)) != cudaSuccess) return e;
+// ---------------------------------------------------------------- expert parallelism
 
-  // shared down: Q8_0 x bf16 hs -> y (plus the residual input when pre-norm)
-  GemmArgs sd{};
-  sd.fmt = kFmtQ80;
-  sd.bf16 = 1;
-  sd.epi = kEpiStore;
-  sd.M = d.H;
-  sd.K = d.Is;
-  sd.n_groups = 1;
-  sd.offsets = nullptr;
-  sd.cols = T;
-  sd.A0 = p.wt.sh_down;
-  sd.A1 = nullptr;
-  sd.a_row_bytes = rbQ8s;
-  sd.b_base = b.hs;
-  sd.b_ld = d.Is;
-  sd.b_div = 1;
-  sd.y = p.y;
-  sd.y_ld = d.H;
-  sd.res = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr;
-  sd.err = p.err;
-  sd.wait_cycles = d.wait_cycles;
-  if ((e = grouped_gemm(sd, s, num_sms)) != cudaSuccess) return e;
+namespace {
 
-  // routed down: Q2_K x bf16 h, y[token] += w * (W_down h)
-  GemmArgs rd = sd;
-  rd.fmt = p.q4k ? kFmtQ4K : kFmtQ2K;
-  rd.epi = kEpiScatterAdd;
-  rd.M = d.H;
-  rd.K = d.I;
-  rd.n_groups = d.E;
-  rd.offsets = p.s.offsets;
-  rd.A0 = p.wt.down;
-  rd.a_group_stride = (size_t)d.H * rbQ2;
-  rd.a_row_bytes = rbQ2;
-  rd.b_base = b.hperm;
-  rd.b_ld = d.I;
-  rd.b_perm = nullptr;
-  rd.res = nullptr;
-  rd.w = p.s.w;
-  rd.perm = p.s.perm;
-  rd.k = d.k;
-  return grouped_gemm(rd, s, num_sms);
+// 1 / RMS of each token row in fp64 (1 without the pre-norm flag), as the
+// single-GPU path scales the expert input.
+__global__ void k_ep_inv(const float *x, int T, int H, int flags, float eps, float *inv) {
+  const int t = blockIdx.x;
+  if (!(flags & MOE_FLAG_PRENORM_RESIDUAL)) {
+    if (threadIdx.x == 0) inv[t] = 1.f;
+    return;
+  }
+  double ss = 0.0;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) ss += (double)x[(size_t)t * H + j] * (double)x[(size_t)t * H + j];
+  ss = warp_sum_d(ss);
+  __shared__ double red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    inv[t] = (float)(1.0 / sqrt(tot / (double)H + (double)eps));
+  }
+}
+
+// Dispatch row i (pairs in grouped order): the f16 expert input of token
+// perm[i] / k, its expert id and routing weight.
+__global__ void k_ep_pack(const float *x, const float *inv, int H, int k, const int32_t *idx, const float *w,
+                          const int32_t *perm, __half *x_send, int32_t *e_send, float *w_send) {
+  const int i = blockIdx.x;
+  const int pr = perm[i], t = pr / k;
+  const float sc = inv[t];
+  const float *xt = x + (size_t)t * H;
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4 *>(xt + j);
+    __half2 a = __floats2half2_rn(v.x * sc, v.y * sc);
+    __half2 b = __floats2half2_rn(v.z * sc, v.w * sc);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t *>(&a);
+    o.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(x_send + (size_t)i * H + j) = o;
+  }
+  if (threadIdx.x == 0) {
+    e_send[i] = idx[pr];
+    w_send[i] = w[pr];
+  }
+}
+
+// Received rows: global expert ids -> ids local to the shard; an id outside
+// the shard is reported and its row gets no expert (local id -1).
+__global__ void k_ep_local_ids(const int32_t *e_recv, int N, int e0, int E_local, int32_t *local, int *err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const int e = e_recv[i] - e0;
+  if (e < 0 || e >= E_local) {
+    set_error(err, kErrTokenId);
+    local[i] = -1;
+  } else {
+    local[i] = e;
+  }
+}
+
+// y[t] += sum over the token's k pairs, in ascending slot order, of the
+// returned expert rows; pos[t*k + slot] is the pair's row in the dispatch order.
+__global__ void k_ep_combine(int H, int k, const int32_t *pos, const float *out, float *y) {
+  const int t = blockIdx.x;
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    float4 acc = *reinterpret_cast<const float4 *>(y + (size_t)t * H + j);
+    for (int q = 0; q < k; ++q) {
+      const float4 v = *reinterpret_cast<const float4 *>(out + (size_t)pos[t * k + q] * H + j);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    *reinterpret_cast<float4 *>(y + (size_t)t * H + j) = acc;
+  }
+}
+
+__global__ void k_inverse_perm(const int32_t *perm, int n, int32_t *pos) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) pos[perm[i]] = i;
+}
+
+}  // namespace
+
+size_t ep_dispatch_scratch_bytes(const LayerDims &d, int T) {
+  // the router's scratch (as the batched path carves it), then 1/RMS per token
+  PrefillArgs p = prefill_args(d, LayerWeights{}, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return reinterpret_cast<size_t>(p.s.big) + align_up(sizeof(float) * (size_t)T, 256) + 256;
+}
+
+cudaError_t ep_dispatch(const PrefillArgs &p, int32_t *offsets, int32_t *perm, __half *x_send, int32_t *e_send,
+                        float *w_send, cudaStream_t s) {
+  const LayerDims &d = p.d;
+  const int T = p.T;
+  cudaError_t e = prefill_route(p, p.s.idx, p.s.w, s);
+  if (e != cudaSuccess) return e;
+  e = permute(p.s.idx, T, d.k, d.E, offsets, perm, s);
+  if (e != cudaSuccess) return e;
+  float *inv = reinterpret_cast<float *>(p.s.big);
+  k_ep_inv<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, inv);
+  k_ep_pack<<<T * d.k, 256, 0, s>>>(p.x, inv, d.H, d.k, p.s.idx, p.s.w, perm, x_send, e_send, w_send);
+  return cudaGetLastError();
+}
+
+size_t ep_experts_scratch_bytes(const LayerDims &d, int N) {
+  size_t off = 0;
+  auto take = [&](size_t n) { off = align_up(off, 256) + n; };
+  take(sizeof(int32_t) * (size_t)N);        // local ids
+  take(sizeof(int32_t) * (size_t)(d.E + 1));  // offsets
+  take(sizeof(int32_t) * (size_t)N);        // perm
+  take(2 * (size_t)N * d.I);                // h (bf16), grouped order
+  return off + 256;
+}
+
+cudaError_t ep_experts(const LayerDims &d, const LayerWeights &wt, bool q4k, const __half *x_recv,
+                       const int32_t *e_recv, const float *w_recv, int N, int e0, float *out, void *scratch,
+                       int *err, cudaStream_t s, int num_sms) {
+  uint8_t *base = static_cast<uint8_t *>(scratch);
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    off = align_up(off, 256);
+    uint8_t *q = base + off;
+    off += n;
+    return q;
+  };
+  int32_t *local = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)N));
+  int32_t *offsets = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)(d.E + 1)));
+  int32_t *perm = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)N));
+  uint16_t *h = reinterpret_cast<uint16_t *>(take(2 * (size_t)N * d.I));
+  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N * d.H, s);
+  if (e != cudaSuccess) return e;
+  k_ep_local_ids<<<(N + 255) / 256, 256, 0, s>>>(e_recv, N, e0, d.E, local, err);
+  if ((e = permute(local, N, 1, d.E, offsets, perm, s)) != cudaSuccess) return e;
+  e = grouped_gemm(routed_gateup_args(d, wt, q4k, d.E, offsets, perm, 1, x_recv, h, err), s, num_sms);
+  if (e != cudaSuccess) return e;
+  return grouped_gemm(routed_down_args(d, wt, q4k, d.E, offsets, perm, 1, h, w_recv, out, err), s, num_sms);
+}
+
+size_t ep_combine_scratch_bytes(const LayerDims &d, int T) {
+  return align_up(sizeof(float) * (size_t)T, 256) + align_up(sizeof(int32_t) * (size_t)T * d.k, 256) +
+         align_up(2 * (size_t)T * d.H, 256) + align_up(2 * (size_t)T * d.Is, 256) + 256;
+}
+
+cudaError_t ep_combine(const LayerDims &d, const LayerWeights &wt, const float *x, int T, const int32_t *perm,
+                       const float *out_back, float *y, void *scratch, int *err, cudaStream_t s, int num_sms) {
+  uint8_t *base = static_cast<uint8_t *>(scratch);
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    off = align_up(off, 256);
+    uint8_t *q = base + off;
+    off += n;
+    return q;
+  };
+  (void)take(sizeof(float) * (size_t)T);
+  int32_t *pos = reinterpret_cast<int32_t *>(take(sizeof(int32_t) * (size_t)T * d.k));
+  __half *x16 = reinterpret_cast<__half *>(take(2 * (size_t)T * d.H));
+  uint16_t *hs = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.Is));
+  k_prep_x16<<<T, 256, 0, s>>>(x, T, d.H, d.flags, d.eps, x16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = shared_gemms(d, wt, T, x16, hs, (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? x : nullptr, y, err, s, num_sms);
+  if (e != cudaSuccess) return e;
+  const int n = T * d.k;
+  k_inverse_perm<<<(n + 255) / 256, 256, 0, s>>>(perm, n, pos);
+  k_ep_combine<<<T, 256, 0, s>>>(d.H, d.k, pos, out_back, y);
+  return cudaGetLastError();
 }
 
 cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, cudaStream_t s) {

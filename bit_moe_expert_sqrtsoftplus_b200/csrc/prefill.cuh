@@ -2,6 +2,7 @@
 // token permutation and grouped tensor-core GEMMs.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -46,6 +47,25 @@ cudaError_t prefill_init(const LayerDims &d, const LayerWeights &wt, float *row_
 cudaError_t check_tid2eid(const LayerDims &d, const int32_t *tab, int *dev_word, int *first_bad, cudaStream_t s);
 cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStream_t s);
 cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms);
+// Expert parallelism (experts split over ranks in contiguous blocks).
+//   ep_dispatch: routing, grouping of the T*k pairs by expert (offsets,
+//     perm), and per pair in that order the f16 expert input row, the
+//     expert id and the routing weight.
+//   ep_experts: on a shard of E = d.E experts starting at global id e0, the
+//     rows received for them: out[i] = w[i] * E_{e[i]}(x[i]).
+//   ep_combine: y = shared expert (+ the residual input with the pre-norm
+//     flag) + the returned rows of each token's pairs, in ascending slot order.
+size_t ep_dispatch_scratch_bytes(const LayerDims &d, int T);
+cudaError_t ep_dispatch(const PrefillArgs &p, int32_t *offsets, int32_t *perm, __half *x_send, int32_t *e_send,
+                        float *w_send, cudaStream_t s);
+size_t ep_experts_scratch_bytes(const LayerDims &d, int N);
+cudaError_t ep_experts(const LayerDims &d, const LayerWeights &wt, bool q4k, const __half *x_recv,
+                       const int32_t *e_recv, const float *w_recv, int N, int e0, float *out, void *scratch,
+                       int *err, cudaStream_t s, int num_sms);
+size_t ep_combine_scratch_bytes(const LayerDims &d, int T);
+cudaError_t ep_combine(const LayerDims &d, const LayerWeights &wt, const float *x, int T, const int32_t *perm,
+                       const float *out_back, float *y, void *scratch, int *err, cudaStream_t s, int num_sms);
+
 // Stable grouping of the T*k (token, slot) pairs by expert.
 cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm, cudaStream_t s);
 

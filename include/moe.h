@@ -67,6 +67,10 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 
 /* flags */
 #define MOE_FLAG_PRENORM_RESIDUAL 1 /* forward computes x + MoE(RMSNorm(x)) */
+/* handles for expert parallelism (the moe_ep_* calls below); neither serves
+ * moe_ffn_forward */
+#define MOE_FLAG_EXPERTS_ONLY 2 /* a shard of routed experts: only the routed expert weights are read */
+#define MOE_FLAG_NO_ROUTED 4    /* router (or table) and shared expert only: routed expert pointers may be NULL */
 
 #define MOE_SMALL_T_MAX 32 /* largest T served by the small-token kernels */
 
@@ -244,6 +248,52 @@ moe_status moe_set_wait_limit(moe_handle *h, long long cycles);
  */
 moe_status moe_quantize(int format, const float *x, int64_t n, void *out, int32_t *nonfinite_blocks,
                         moe_stream_t stream);
+
+/*
+ * Expert parallelism: the routed experts of a layer split over G ranks (one
+ * GPU each) in contiguous blocks of E/G experts; rank r owns global ids
+ * [r*E/G, (r+1)*E/G).  The exchange itself (two all-to-alls of rows between
+ * ranks) is the caller's, e.g. NCCL through torch.distributed; these calls do
+ * the work on each side of it.  The pages' counterpart is ds4's mode that
+ * splits one model over two machines ("DeepSeek-V4-Flash one-token
+ * computation flow", section "128GB にどう収めるか"); the split by experts is
+ * this library's choice.  The calls run the batched (tensor-core) kernels
+ * for any T.
+ *
+ *   1. moe_ep_dispatch (every rank, on its own T tokens, with a handle that
+ *      has the router or table and the shared expert; MOE_FLAG_NO_ROUTED lets
+ *      it hold no routed weights): routing, then the T*k (token, slot) pairs
+ *      grouped by expert as moe_route gives them (expert_offsets [E+1], perm
+ *      [T*k]), and for pair perm[i], in row i: x_send [T*k][H] the expert
+ *      input as IEEE f16 (RMSNorm(x) with MOE_FLAG_PRENORM_RESIDUAL, else x),
+ *      e_send [T*k] the global expert id, w_send [T*k] the routing weight.
+ *      The rows for rank r are expert_offsets[r*E/G] .. expert_offsets[(r+1)*E/G].
+ *   2. (exchange: each rank receives the rows for its experts from all ranks)
+ *   3. moe_ep_experts (on the shard handle: MOE_FLAG_EXPERTS_ONLY, n_experts
+ *      = the shard's E/G, routed weight arrays holding only the shard's
+ *      experts, first_expert = the shard's first global id): for the N
+ *      received rows, out[i] = w_recv[i] * E_{e_recv[i]}(x_recv[i]) (fp32
+ *      [N][H]).  A row whose id is outside the shard gets zeros and records
+ *      MOE_ERR_INVALID_ARG in the device error word.
+ *   4. (exchange back: the out rows return to the rank and row they came from)
+ *   5. moe_ep_combine (the dispatching rank): y [T][H] = shared expert (plus x
+ *      with MOE_FLAG_PRENORM_RESIDUAL) + for each token the sum over its k
+ *      pairs, in ascending expert id, of out_back rows (row i for pair
+ *      perm[i]).  y may alias x only with MOE_FLAG_PRENORM_RESIDUAL.
+ *
+ * moe_ep_workspace_size gives each call's scratch for up to max_tokens tokens
+ * and max_recv_rows received rows.  All pointers are device pointers, 16-byte
+ * aligned where they hold rows; every call is asynchronous on `stream`.
+ */
+moe_status moe_ep_workspace_size(const moe_config *cfg, int max_tokens, int max_recv_rows, size_t *dispatch_bytes,
+                                 size_t *experts_bytes, size_t *combine_bytes);
+moe_status moe_ep_dispatch(moe_handle *h, const float *x, const int32_t *token_ids, int T, int32_t *expert_offsets,
+                           int32_t *perm, void *x_send, int32_t *e_send, float *w_send, void *scratch,
+                           size_t scratch_bytes, moe_stream_t stream);
+moe_status moe_ep_experts(moe_handle *shard, const void *x_recv, const int32_t *e_recv, const float *w_recv, int N,
+                          int first_expert, float *out, void *scratch, size_t scratch_bytes, moe_stream_t stream);
+moe_status moe_ep_combine(moe_handle *h, const float *x, int T, const int32_t *perm, const float *out_back, float *y,
+                          void *scratch, size_t scratch_bytes, moe_stream_t stream);
 
 /* Frees the host-side handle (the caller frees `persist`). NULL is a no-op. */
 void moe_destroy(moe_handle *h);

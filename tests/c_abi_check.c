@@ -65,6 +65,25 @@ int main(void) {
 
   check(moe_set_wait_limit(NULL, 100) == MOE_ERR_INVALID_ARG, "wait limit without a handle");
 
+  /* expert parallelism: workspace sizes and argument checks */
+  c.hidden = 4096;
+  c.top_k = 6;
+  c.n_experts = 256;
+  size_t ed = 0, ex = 0, ec = 0;
+  check(moe_ep_workspace_size(&c, 512, 3072, &ed, &ex, &ec) == MOE_OK && ed > 0 && ex > 0 && ec > 0,
+        "expert-parallel workspace sizes");
+  check(moe_ep_workspace_size(NULL, 1, 1, NULL, NULL, NULL) == MOE_ERR_INVALID_ARG, "EP workspace without config");
+  check(moe_ep_workspace_size(&c, -1, 1, NULL, NULL, NULL) == MOE_ERR_INVALID_ARG, "EP negative tokens");
+  c.flags = MOE_FLAG_EXPERTS_ONLY | MOE_FLAG_NO_ROUTED;
+  check(moe_workspace_size(&c, 1, NULL, NULL) == MOE_ERR_INVALID_ARG, "exclusive EP flags");
+  c.flags = 0;
+  check(moe_ep_dispatch(NULL, NULL, NULL, 1, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG,
+        "dispatch without a handle");
+  check(moe_ep_experts(NULL, NULL, NULL, NULL, 1, 0, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG,
+        "experts without a handle");
+  check(moe_ep_combine(NULL, NULL, 1, NULL, NULL, NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG,
+        "combine without a handle");
+
   moe_destroy(NULL);
   if (failures == 0) printf("C ABI checks passed\n");
   return failures == 0 ? 0 : 1;
