@@ -30,6 +30,7 @@ MOE_ROUTE_HASH = 1
 MOE_FLAG_PRENORM_RESIDUAL = 1
 MOE_FLAG_EXPERTS_ONLY = 2
 MOE_FLAG_NO_ROUTED = 4
+MOE_FLAG_DETERMINISTIC = 8
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
 MOE_QUANT_Q8_0 = 0
 MOE_QUANT_Q2_K = 1

@@ -76,7 +76,7 @@ moe_status check_config(const moe_config *c) {
   if (!isfinite(c->routed_scaling)) return fail(MOE_ERR_INVALID_ARG, "routed_scaling is not finite");
   if ((c->flags & MOE_FLAG_PRENORM_RESIDUAL) && !(c->rms_eps >= 0.f && isfinite(c->rms_eps)))
     return fail(MOE_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
-  if (c->flags & ~(MOE_FLAG_PRENORM_RESIDUAL | MOE_FLAG_EXPERTS_ONLY | MOE_FLAG_NO_ROUTED))
+  if (c->flags & ~(MOE_FLAG_PRENORM_RESIDUAL | MOE_FLAG_EXPERTS_ONLY | MOE_FLAG_NO_ROUTED | MOE_FLAG_DETERMINISTIC))
     return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
   if ((c->flags & MOE_FLAG_EXPERTS_ONLY) && (c->flags & MOE_FLAG_NO_ROUTED))
     return fail(MOE_ERR_INVALID_ARG, "MOE_FLAG_EXPERTS_ONLY and MOE_FLAG_NO_ROUTED exclude each other");

@@ -571,10 +571,27 @@ __global__ void k_prep_x16(const float *x, int T, int H, int flags, float eps, _
   }
 }
 
+// y[t] += slots[t*k] + slots[t*k + 1] + ... (ascending slot = ascending expert id)
+__global__ void k_sum_slots(int H, int k, const float *slots, float *y) {
+  const int t = blockIdx.x;
+  for (int j = threadIdx.x * 4; j < H; j += blockDim.x * 4) {
+    float4 acc = *reinterpret_cast<const float4 *>(y + (size_t)t * H + j);
+    for (int q = 0; q < k; ++q) {
+      const float4 v = *reinterpret_cast<const float4 *>(slots + ((size_t)t * k + q) * H + j);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    *reinterpret_cast<float4 *>(y + (size_t)t * H + j) = acc;
+  }
+}
+
 struct BigScratch {
   __half *x16;      // [T][H]
   uint16_t *hperm;  // [T*k][I] bf16, rows in permuted order
   uint16_t *hs;     // [T][Is] bf16
+  float *slots;     // [T*k][H] weighted expert outputs per pair (deterministic combine only)
   size_t bytes;
 };
 
@@ -590,6 +607,8 @@ BigScratch carve_big(const LayerDims &d, int T, void *base) {
   b.x16 = reinterpret_cast<__half *>(take(2 * (size_t)T * d.H));
   b.hperm = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.k * d.I));
   b.hs = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.Is));
+  b.slots = (d.flags & MOE_FLAG_DETERMINISTIC) ? reinterpret_cast<float *>(take(sizeof(float) * (size_t)T * d.k * d.H))
+                                                : nullptr;
   b.bytes = off;
   return b;
 }
@@ -737,8 +756,19 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
                    num_sms);
   if (e != cudaSuccess) return e;
   // routed down: Q2_K (or Q4_K) x bf16 h, y[token] += w * (W_down h)
-  return grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, p.s.w, p.y, p.err),
-                      s, num_sms);
+  if (!(d.flags & MOE_FLAG_DETERMINISTIC))
+    return grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, p.s.w, p.y, p.err),
+                        s, num_sms);
+  // deterministic: each pair's weighted output into its own slot row (one
+  // addition onto zero per element), then every token's slots summed in
+  // ascending slot order
+  const int n = T * d.k;
+  if ((e = cudaMemsetAsync(b.slots, 0, sizeof(float) * (size_t)n * d.H, s)) != cudaSuccess) return e;
+  e = grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, 1, b.hperm, p.s.w, b.slots, p.err), s,
+                   num_sms);
+  if (e != cudaSuccess) return e;
+  k_sum_slots<<<T, 256, 0, s>>>(d.H, d.k, b.slots, p.y);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- expert parallelism

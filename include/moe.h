@@ -67,6 +67,13 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 
 /* flags */
 #define MOE_FLAG_PRENORM_RESIDUAL 1 /* forward computes x + MoE(RMSNorm(x)) */
+/* calls above MOE_SMALL_T_MAX tokens add the routed experts' outputs in a fixed
+ * order (each pair's weighted output in its own row of scratch, then every
+ * token's rows summed in ascending expert id), so repeated calls give the same
+ * bits; without it they are added with atomics in arrival order.  Costs
+ * T*k*H*4 bytes of scratch (403 MB at T = 4096) and their write and read.
+ * The small-token path is deterministic either way. */
+#define MOE_FLAG_DETERMINISTIC 8
 /* handles for expert parallelism (the moe_ep_* calls below); neither serves
  * moe_ffn_forward */
 #define MOE_FLAG_EXPERTS_ONLY 2 /* a shard of routed experts: only the routed expert weights are read */

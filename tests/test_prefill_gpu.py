@@ -97,3 +97,28 @@ def test_prefill_4096_every_row(moe):
         rows = np.nonzero((idx == e).any(1))[0]
         r, m = harness.errors(y[rows], yref[rows])
         assert r <= harness.MMA_REL_L2 and m <= harness.MAX_ABS_FRAC, (e, counts[e], r, m)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 300), ("prefill_t4096", 4096)])
+def test_deterministic_flag_repeats_bitwise(moe, name, T):
+    """MOE_FLAG_DETERMINISTIC: the routed outputs are summed per token in
+    ascending expert id, so two calls give the same bits; the result stays
+    within the tensor-core tolerance of the oracle (tiny) and of the
+    atomic-add combine (full shape)."""
+    s = synth.workload(name, tokens=T)
+    W = harness.device_layer(s, 2, 5)
+    x_np = synth.activations(2, T, s.hidden, stream=5)
+    x = torch.from_numpy(x_np).cuda()
+    Ld = moe.Layer(harness.config_for(s, flags=moe.MOE_FLAG_DETERMINISTIC), W, max_tokens=T)
+    y1 = Ld.forward(x).cpu().numpy()
+    y2 = Ld.forward(x).cpu().numpy()
+    Ld.poll()
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+    if name == "tiny":
+        _, _, yref, _ = harness.oracle_layer(s, 2, 5, x_np)
+    else:
+        La = moe.Layer(harness.config_for(s), W, max_tokens=T)
+        yref = La.forward(x).cpu().numpy()
+        La.poll()
+    rel, mx = harness.errors(y1, yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
