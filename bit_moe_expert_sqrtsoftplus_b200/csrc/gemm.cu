@@ -39,12 +39,21 @@ constexpr int kProdWarps = 16;
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 24
 constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 800
 constexpr int kProd = kProdWarps * 32;             // 512 producer threads
-constexpr int kGridRep = 4;                        // replicas of the f16 codebook table
-constexpr int kSignRep = 4;                        // replicas of the sign-mask table
-constexpr int kAhead = 3;                          // K steps of packed weights fetched ahead
-constexpr int BM = 128, BK = 64, BN = 256;
+// Codebook and sign tables: an entry is read as 16 bytes by 8 lanes per
+// shared-memory wavefront; with 8 replicas, lane l reads replica l % 8, so
+// the 8 lanes of a wavefront hit 8 different 16-byte bank groups whatever
+// the entries.
+constexpr int kGridRep = 8;                        // replicas of the f16 codebook table
+constexpr int kSignRep = 8;                        // replicas of the sign-mask table
+// K steps of packed weights a producer fetches ahead, by format: the ring
+// holds (ahead + 1) items of 3 (IQ2_XXS), 6 (Q2_K) or 9 (Q8_0, Q4_K) words
+__host__ __device__ constexpr int ahead_of(int fmt) { return fmt == 0 ? 6 : fmt == 1 ? 4 : 3; }
+constexpr int BM = 128, BK = 64;
 constexpr int kATile = BM * BK * 2;  // 16 KB
-constexpr int kBTile = BN * BK * 2;  // 32 KB
+// token columns per tile: 128 for a gate/up pair (two accumulators per tile,
+// two tiles in flight fill the 512 TMEM columns), 256 for a single matrix
+__host__ __device__ constexpr int bn_of(bool paired) { return paired ? 128 : 256; }
+__host__ __device__ constexpr int btile_of(bool paired) { return bn_of(paired) * BK * 2; }
 
 constexpr int kSB = 4;       // stages of the B (token rows) ring
 constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
@@ -158,6 +167,7 @@ struct Tile {
   int g, m0, n0, nt, col0;
 };
 
+template <int BN>
 __device__ __forceinline__ Tile tile_at(const GemmCtl &ctl, int t, int m_tiles) {
   int lo = 0, hi = ctl.n_groups - 1;
   while (lo < hi) {  // last group with prefix <= t
@@ -398,18 +408,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
   constexpr int SA = PAIRED ? 2 : 4;
-  // accumulator buffers in tensor memory: a gate/up pair fills all 512
-  // columns; a single matrix uses 256, so two tiles alternate and the
-  // epilogue of one overlaps the main loop of the next
-  constexpr int NACC = PAIRED ? 1 : 2;
+  constexpr int BN = bn_of(PAIRED);
+  constexpr int kBTile = btile_of(PAIRED);
+  // accumulator buffers in tensor memory: two tiles alternate (a pair's two
+  // 128-column accumulators, or one 256-column accumulator, per tile), so the
+  // epilogue of one tile overlaps the main loop of the next
+  constexpr int NACC = 2;
+  constexpr int ACC_COLS = NA * BN;  // columns of one tile's accumulators
   constexpr int ASTAGE = NA * kATile;
+  constexpr bool kTables = FMT == kFmtIQ2;
+  constexpr int kAhead = ahead_of(FMT);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stagesA = smem;
   uint8_t *stagesB = stagesA + SA * ASTAGE;
-  uint8_t *gridh = stagesB + kSB * kBTile;      // 256 x kGridRep x 16 B: codebook as f16
-  uint8_t *signm = gridh + 4096 * kGridRep;     // 128 x kSignRep x 16 B: f16 sign masks
-  GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + 2048 * kSignRep);
+  uint8_t *gridh = stagesB + kSB * kBTile;                // 256 x kGridRep x 16 B: codebook as f16
+  uint8_t *signm = gridh + (kTables ? 4096 * kGridRep : 0);  // 128 x kSignRep x 16 B: f16 sign masks
+  GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + (kTables ? 2048 * kSignRep : 0));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_tiles = a.M / BM;
@@ -476,14 +491,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     const int p = tid - kEpiWarps * 32;
     const uint8_t *gridh_l = gridh + 16 * (lane % kGridRep);
     const uint8_t *signm_l = signm + 16 * (lane % kSignRep);
+    constexpr int kBRows = BN / 64;  // B rows per producer thread and step
     uint32_t it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = tile_at(ctl, t, m_tiles);
+      const Tile tl = tile_at<BN>(ctl, t, m_tiles);
       // B rows this thread copies: rows (p >> 3) + 64 i, chunk p & 7
       const int ch = p & 7;
-      const uint16_t *brow[4];
+      const uint16_t *brow[kBRows];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kBRows; ++i) {
         const int r = (p >> 3) + 64 * i;
         brow[i] = nullptr;
         if (r < tl.nt) {
@@ -513,7 +529,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       auto issue_b = [&](int ks, int sb) {
         uint8_t *Bs = stagesB + sb * kBTile;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kBRows; ++i) {
           if (brow[i]) cp_async16(swz(Bs, (p >> 3) + 64 * i, ch), brow[i] + ks * BK);
         }
         cp_async_commit();
@@ -561,11 +577,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     uint32_t it = 0, tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
-      const Tile tl = tile_at(ctl, t, m_tiles);
+      const Tile tl = tile_at<BN>(ctl, t, m_tiles);
       const int nmma = (tl.nt + 15) & ~15;
       const uint32_t idesc = instr_desc(nmma, a.bf16);
       const uint32_t buf = tc % NACC;
-      const uint32_t dacc = tmem + buf * BN;  // accumulator columns of this tile
+      const uint32_t dacc = tmem + buf * ACC_COLS;  // accumulator columns of this tile
       if (!mbar_wait(&ctl.acc_empty[buf], ((tc / NACC) & 1u) ^ 1u, ctl, a.err)) {
         ok = false;
         break;
@@ -585,7 +601,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             mma_f16(dacc, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
-            if (PAIRED) mma_f16(tmem + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+            if (PAIRED) mma_f16(dacc + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
           }
           mma_commit(&ctl.emptyA[it % SA]);
           mma_commit(&ctl.emptyB[it % kSB]);
@@ -616,15 +632,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
-      const Tile tl = tile_at(ctl, t, m_tiles);
+      const Tile tl = tile_at<BN>(ctl, t, m_tiles);
       const uint32_t buf = tc % NACC;
       if (!mbar_wait(&ctl.acc_full[buf], (tc / NACC) & 1u, ctl, a.err)) break;
       tc_fence_after();
       const int m = tl.m0 + row;
       for (int c0 = 16 * half; c0 < tl.nt; c0 += 32) {
         uint32_t r0[16], r1[16];
-        tmem_ld16(lane_base + buf * BN + c0, r0);
-        if (PAIRED) tmem_ld16(lane_base + BN + c0, r1);
+        tmem_ld16(lane_base + buf * ACC_COLS + c0, r0);
+        if (PAIRED) tmem_ld16(lane_base + buf * ACC_COLS + BN + c0, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -670,16 +686,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 
 }  // namespace
 
-size_t grouped_gemm_smem(int paired) {
+size_t grouped_gemm_smem(int fmt, int paired) {
   const int na = paired ? 2 : 1;
   const int sa = paired ? 2 : 4;
-  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * kBTile + 4096 * kGridRep + 2048 * kSignRep + sizeof(GemmCtl);
+  const size_t tables = fmt == kFmtIQ2 ? 4096 * kGridRep + 2048 * kSignRep : 0;
+  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * btile_of(paired != 0) + tables + sizeof(GemmCtl);
 }
 
 template <int FMT, bool PAIRED>
 static cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   static SmemOptIn opt;
-  const size_t smem = grouped_gemm_smem(PAIRED);
+  const size_t smem = grouped_gemm_smem(FMT, PAIRED);
   cudaError_t e = opt_in_smem(k_grouped_gemm<FMT, PAIRED>, smem, opt);
   if (e != cudaSuccess) return e;
   k_grouped_gemm<FMT, PAIRED><<<num_sms, kGemmThreads, smem, s>>>(a);

@@ -49,6 +49,6 @@ struct GemmArgs {
 };
 
 cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms);
-size_t grouped_gemm_smem(int paired);
+size_t grouped_gemm_smem(int fmt, int paired);
 
 }  // namespace moe
