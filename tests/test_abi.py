@@ -87,7 +87,8 @@ def test_workspace_size_and_shape_checks(moe):
                         (dict(n_experts=4, top_k=6), moe.MOE_ERR_UNSUPPORTED_SHAPE),
                         (dict(mode=7), moe.MOE_ERR_INVALID_ARG),
                         (dict(mode=1, vocab=0), moe.MOE_ERR_INVALID_ARG),
-                        (dict(flags=8), moe.MOE_ERR_INVALID_ARG),
+                        (dict(flags=16), moe.MOE_ERR_INVALID_ARG),
+                        (dict(flags=6), moe.MOE_ERR_INVALID_ARG),
                         (dict(routed_format=5), moe.MOE_ERR_INVALID_ARG)):
         with pytest.raises(moe.MoeError) as ei:
             moe.moe_workspace_size(_cfg(moe, **bad), 1)
