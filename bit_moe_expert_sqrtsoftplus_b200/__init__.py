@@ -40,7 +40,7 @@ MOE_ROUTED_Q2 = 0
 MOE_ROUTED_Q4K = 1
 
 EXPORTED = ("moe_workspace_size", "moe_init", "moe_route", "moe_ffn_forward", "moe_poll_device_error",
-            "moe_last_error", "moe_set_timing_events", "moe_set_wait_limit", "moe_ffn_forward_noalloc", "moe_quantize",
+            "moe_last_error", "moe_set_timing_events", "moe_set_next_layer", "moe_set_wait_limit", "moe_ffn_forward_noalloc", "moe_quantize",
             "moe_ep_workspace_size", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_destroy")
 
 
@@ -86,6 +86,8 @@ def lib():
         L.moe_last_error.restype = ctypes.c_char_p
         L.moe_set_timing_events.argtypes = [vp, vp, vp]
         L.moe_set_timing_events.restype = i32
+        L.moe_set_next_layer.argtypes = [vp, vp]
+        L.moe_set_next_layer.restype = i32
         L.moe_set_wait_limit.argtypes = [vp, ctypes.c_longlong]
         L.moe_set_wait_limit.restype = i32
         L.moe_quantize.argtypes = [i32, vp, ctypes.c_int64, vp, vp, vp]
@@ -175,6 +177,12 @@ def moe_set_timing_events(handle, ev_begin=None, ev_end=None):
                                        None if ev_end is None else ev_end.cuda_event))
 
 
+def moe_set_next_layer(handle, next_handle):
+    """Stacked layers: forwards on `handle` prefetch into L2 the weights the
+    next layer reads first (None clears)."""
+    _check(lib().moe_set_next_layer(handle, next_handle))
+
+
 def moe_set_wait_limit(handle, cycles: int):
     """Test hook: bound of the device waits on other warps' results, in SM
     clock cycles (0 restores the default of about 2 s)."""
@@ -232,6 +240,60 @@ def moe_ep_combine(handle, x, T, perm, out_back, y, scratch, stream=None):
 def moe_destroy(handle):
     if handle:
         lib().moe_destroy(handle)
+
+
+class Stack:
+    """Layers applied in order to the same tokens, each as x <- x +
+    MoE_l(RMSNorm(x)) in place (every layer's config must carry
+    MOE_FLAG_PRENORM_RESIDUAL).  Each layer prefetches the next one's router
+    and shared-expert gate/up weights into L2 (moe_set_next_layer).  With
+    ``graph=True`` the first forward captures the whole pass into a CUDA
+    graph on a side stream and later forwards replay it (the input and
+    token-id buffers are then fixed: forward copies into them)."""
+
+    def __init__(self, layers, graph: bool = False):
+        self.layers = list(layers)
+        for L in self.layers:
+            if not (L.cfg.flags & MOE_FLAG_PRENORM_RESIDUAL):
+                raise MoeError(MOE_ERR_INVALID_ARG, "stacked layers need MOE_FLAG_PRENORM_RESIDUAL")
+        for a, b in zip(self.layers, self.layers[1:]):
+            moe_set_next_layer(a.handle, b.handle)
+        self.graph = graph
+        self._g = None
+
+    def _run(self, x, token_ids):
+        for L in self.layers:
+            L.forward(x, token_ids, y=x)
+
+    def forward(self, x, token_ids=None):
+        """x [T][H] fp32 CUDA tensor, updated in place and returned."""
+        import torch
+        if not self.graph:
+            self._run(x, token_ids)
+            return x
+        if self._g is None:
+            self._x = x.clone()
+            self._tok = None if token_ids is None else token_ids.clone()
+            self._run(self._x, self._tok)  # first pass outside capture (lazy set-up)
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            self._g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(self._g, stream=s):
+                    self._run(self._x, self._tok)
+            torch.cuda.current_stream().wait_stream(s)
+        self._x.copy_(x)
+        if self._tok is not None:
+            self._tok.copy_(token_ids)
+        self._g.replay()
+        x.copy_(self._x)
+        return x
+
+    def close(self):
+        self._g = None
+        for L in self.layers:
+            if L.handle:
+                moe_set_next_layer(L.handle, None)
 
 
 class Layer:

@@ -28,6 +28,7 @@ struct moe_handle {
   int num_sms;
   int device;
   cudaEvent_t ev_begin, ev_end;  // optional timing of the dominant kernel
+  moe::NextLayerPrefetch next;   // the next layer's first-read weights (stack decode)
 };
 
 namespace {
@@ -243,6 +244,7 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   h->device = dev;
   h->ev_begin = nullptr;
   h->ev_end = nullptr;
+  h->next = moe::NextLayerPrefetch{};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   e = cudaMemsetAsync(persist, 0, kPersistHeader, s);
   if (e != cudaSuccess) {
@@ -280,6 +282,7 @@ static moe::DecodeArgs decode_args(moe_handle *h, const float *x, const int32_t 
   moe::DecodeArgs a;
   a.d = h->d;
   a.wt = h->wt;
+  a.pf = h->next;
   a.T = T;
   a.x = x;
   a.token_ids = token_ids;
@@ -493,6 +496,26 @@ moe_status moe_set_wait_limit(moe_handle *h, long long cycles) {
   if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
   if (cycles < 0) return fail(MOE_ERR_INVALID_ARG, "cycles=%lld is negative", cycles);
   h->d.wait_cycles = cycles > 0 ? cycles : moe::kDefaultWaitCycles;
+  g_last_error.clear();
+  return MOE_OK;
+}
+
+moe_status moe_set_next_layer(moe_handle *h, const moe_handle *next) {
+  if (!h) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  h->next = moe::NextLayerPrefetch{};
+  if (next) {
+    if (next->device != h->device) return fail(MOE_ERR_INVALID_ARG, "the next layer's handle is on another device");
+    const moe::LayerDims &d = next->d;
+    if (next->wt.Wr) {
+      h->next.ptr[0] = next->wt.Wr;
+      h->next.bytes[0] = (size_t)d.E * d.H * 2;
+    }
+    if (next->wt.sh_gate && next->wt.sh_up) {
+      h->next.ptr[1] = next->wt.sh_gate;
+      h->next.ptr[2] = next->wt.sh_up;
+      h->next.bytes[1] = h->next.bytes[2] = (size_t)d.Is * (d.H / 32) * 34;
+    }
+  }
   g_last_error.clear();
   return MOE_OK;
 }

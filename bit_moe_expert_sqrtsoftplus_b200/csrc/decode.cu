@@ -690,6 +690,23 @@ __device__ __forceinline__ void run_units(uint8_t *st0, uint8_t *st1, uint64_t *
   }
 }
 
+// This CTA's share of the next layer's prefetch regions, in pieces of at
+// most 64 KB (one thread issues them; they complete on their own).
+__device__ void prefetch_next_layer(const NextLayerPrefetch &pf) {
+  for (int r = 0; r < kPrefetchRegions; ++r) {
+    const size_t n = pf.bytes[r];
+    if (!pf.ptr[r] || n == 0) continue;
+    const size_t per = (n / gridDim.x + 15) & ~(size_t)15;
+    const size_t b0 = per * blockIdx.x;
+    const size_t b1 = min(n, b0 + per);
+    const uint8_t *base = static_cast<const uint8_t *>(pf.ptr[r]);
+    for (size_t o = b0; o < b1; o += 65536) {
+      const uint32_t sz = (uint32_t)min((size_t)65536, b1 - o);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(base + o), "r"(sz) : "memory");
+    }
+  }
+}
+
 // ------------------------------------------------------------------ decoders
 
 // B operand column (the int8 limbs of one vector) in shared or global memory;
@@ -1675,6 +1692,9 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
           }
         }
       });
+  // the CTA's last warp, once out of units, starts this CTA's share of the
+  // next layer's prefetch (set only when the layer runs in a stack)
+  if (warp == nw - 1 && lane == 0) prefetch_next_layer(a.pf);
 }
 
 // ------------------------------------------------------------------ route only

@@ -118,9 +118,20 @@ struct DecodeScratch {
   FastDiv fPH, fTIPH, fTH, fPD;  // divisors PH, (I/16)*PH, H/16, PD of the unit numbering
 };
 
+// Weights of the next layer of a stack that the expert kernel brings into
+// L2 near its end (the router rows and the shared expert's gate/up rows that
+// the next layer reads first); bytes are multiples of 16, pointers 16-byte
+// aligned, unused entries 0.
+constexpr int kPrefetchRegions = 3;
+struct NextLayerPrefetch {
+  const void *ptr[kPrefetchRegions];
+  size_t bytes[kPrefetchRegions];
+};
+
 struct DecodeArgs {
   LayerDims d;
   LayerWeights wt;
+  NextLayerPrefetch pf;
   int T;
   const float *x;
   const int32_t *token_ids;

@@ -223,6 +223,18 @@ const char *moe_last_error(void);
 moe_status moe_set_timing_events(moe_handle *h, void *ev_begin, void *ev_end);
 
 /*
+ * Stacked layers (x <- x + MoE_l(RMSNorm(x)) for l = 0, 1, ...; "DeepSeek-
+ * V4-Flash one-token computation flow", block structure): after
+ * moe_set_next_layer(h, next), every small-token forward on h brings the
+ * weights that `next` reads first -- its router rows and its shared
+ * expert's gate and up rows -- into the L2 cache near the end of h's expert
+ * kernel, so that the next layer's router and shared-expert work start from
+ * L2 rather than HBM.  A prefetch changes no result.  `next` must stay
+ * valid while h is used (NULL clears it).  Records pointers only.
+ */
+moe_status moe_set_next_layer(moe_handle *h, const moe_handle *next);
+
+/*
  * Test hook for the device-side error path.  The kernels bound every wait on
  * work of other warps or blocks (a down-projection unit waiting for the
  * SwiGLU slice it reads, a warp waiting for its block's routing table, the

@@ -51,6 +51,20 @@ def test_stack43_decode_batch8(moe):
     for L in layers:
         L.poll()
 
+    # the stacked forward (each layer prefetching the next one's router and
+    # shared-expert weights into L2), eager and as a replayed CUDA graph, gives
+    # the layer-by-layer result bit for bit
+    stack = moe.Stack(layers)
+    xs = stack.forward(torch.from_numpy(x0).cuda(), tokd).cpu().numpy()
+    assert np.array_equal(xs.view(np.uint32), inputs[-1].view(np.uint32))
+    gstack = moe.Stack(layers, graph=True)
+    for _ in range(2):
+        xg = gstack.forward(torch.from_numpy(x0).cuda(), tokd).cpu().numpy()
+        assert np.array_equal(xg.view(np.uint32), inputs[-1].view(np.uint32))
+    gstack.close()
+    for L in layers:
+        L.poll()
+
     # teacher forced: layer l of the oracle on the GPU's own input to layer l
     worst = 0.0
     for l in range(s.layers):
