@@ -502,17 +502,31 @@ __device__ __forceinline__ int stage_chunk_tma(uint8_t *st, uint64_t *mbar, cons
 }
 
 // Bounded wait for phase `parity` of an mbarrier; false (and the timeout
-// error recorded) if it does not complete.
+// error recorded) if it does not complete.  Each try_wait may suspend the
+// warp for up to kSuspendNs (it resumes as soon as the phase completes), so
+// a waiting warp takes few issue slots from the warps that compute.
+#ifndef MOE_MBAR_SUSPEND_NS
+#define MOE_MBAR_SUSPEND_NS 0
+#endif
+constexpr unsigned kSuspendNs = MOE_MBAR_SUSPEND_NS;
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *mbar, uint32_t parity, int *err) {
   const uint32_t mb = smem_u32(mbar);
   const long long t0 = clock64();
   while (true) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(mb), "r"(parity)
-        : "memory");
+    if (kSuspendNs > 0)
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(ok)
+          : "r"(mb), "r"(parity), "n"(kSuspendNs)
+          : "memory");
+    else
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(ok)
+          : "r"(mb), "r"(parity)
+          : "memory");
     if (ok) return true;
     if (clock64() - t0 > kDefaultWaitCycles) {
       set_error(err, kErrTimeout);
