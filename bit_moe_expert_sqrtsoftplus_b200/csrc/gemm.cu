@@ -84,8 +84,32 @@ __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait; false when this CTA is aborting (timeout here or elsewhere).
+// try_wait may suspend the thread until the phase completes, which can
+// outlast a bound shorter than the default; such bounds poll with the
+// non-blocking test_wait instead.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, GemmCtl &ctl, int *err) {
+  if (ctl.wait < kDefaultWaitCycles) {
+    const long long t0 = clock64();
+    while (!mbar_test(b, parity)) {
+      if (*((volatile int *)&ctl.abort)) return false;
+      if (clock64() - t0 > ctl.wait) {
+        *((volatile int *)&ctl.abort) = 1;
+        set_error(err, kErrTimeout);
+        return false;
+      }
+    }
+    return true;
+  }
   if (mbar_try(b, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(b, parity)) {
