@@ -54,6 +54,12 @@ constexpr int kATile = BM * BK * 2;  // 16 KB
 // two tiles in flight fill the 512 TMEM columns), 256 for a single matrix
 __host__ __device__ constexpr int bn_of(bool paired) { return paired ? 128 : 256; }
 __host__ __device__ constexpr int btile_of(bool paired) { return bn_of(paired) * BK * 2; }
+// stages of the dequantised A ring: how many K steps the producers may run
+// ahead of the MMA (a pair's stage holds both matrices' tiles)
+#ifndef MOE_GEMM_SA_PAIRED
+#define MOE_GEMM_SA_PAIRED 2
+#endif
+__host__ __device__ constexpr int sa_of(bool paired) { return paired ? MOE_GEMM_SA_PAIRED : 4; }
 
 constexpr int kSB = 4;       // stages of the B (token rows) ring
 constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
@@ -75,13 +81,27 @@ __device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count) {
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
 }
+// try_wait may suspend the thread until the phase completes; with a
+// suspend-time hint (ns) the hardware may keep it suspended that long, so a
+// waiting warp spins less and leaves issue slots to the others.
+#ifndef MOE_GEMM_SUSPEND_NS
+#define MOE_GEMM_SUSPEND_NS 0
+#endif
 __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
+  if (MOE_GEMM_SUSPEND_NS > 0)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity), "n"(MOE_GEMM_SUSPEND_NS)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
@@ -431,7 +451,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   // written in the step that hands it to the MMA; step `it` uses A stage
   // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
-  constexpr int SA = PAIRED ? 2 : 4;
+  constexpr int SA = sa_of(PAIRED);
   constexpr int BN = bn_of(PAIRED);
   constexpr int kBTile = btile_of(PAIRED);
   // accumulator buffers in tensor memory: two tiles alternate (a pair's two
@@ -712,7 +732,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 
 size_t grouped_gemm_smem(int fmt, int paired) {
   const int na = paired ? 2 : 1;
-  const int sa = paired ? 2 : 4;
+  const int sa = sa_of(paired != 0);
   const size_t tables = fmt == kFmtIQ2 ? 4096 * kGridRep + 2048 * kSignRep : 0;
   return 1024 + (size_t)sa * na * kATile + (size_t)kSB * btile_of(paired != 0) + tables + sizeof(GemmCtl);
 }
