@@ -1,10 +1,11 @@
-// decode.cu -- the layer for small token counts (T <= 32): two kernels.
+// decode.cu -- the layer for small token counts (T <= 32): three kernels.
 //
 //   k1_prep_router  x -> int8 limbs (optionally RMSNorm first); fp64 router
 //                   logits, scores s = sqrtsoftplus(z) and selection keys
 //                   s + bias, one block per pair of experts.
-//   k2_experts      top-k routing from the keys (comparisons only, per CTA),
-//                   then all the expert work as warp-sized units on one
+//   k_route_jobs    one block: every token's top-k from the keys (comparisons
+//                   only) and the call's job table, for all CTAs of k2.
+//   k2_experts      copies the routing, then all the expert work as warp-sized units on one
 //                   counter: every (16-row tile, 1024-element K part) of the
 //                   shared and the routed gate/up matrices, then every
 //                   (K part, 16-row output tile) of the shared and the routed
@@ -19,9 +20,10 @@
 //                   limbs and flags it, and down units wait for the slices
 //                   they read.  The warp that completes an output tile sums
 //                   its parts in a fixed order (deterministic) into y.
-// k2 is launched as a programmatic dependent of k1: its set-up (tables,
-// shared memory) overlaps k1, and griddepcontrol.wait guards every read of
-// k1's results.
+// k_route_jobs is a programmatic dependent of k1 and k2 of k_route_jobs:
+// k2's set-up (tables, shared memory, the x limbs, the shared expert's first
+// units) overlaps the routing, and griddepcontrol.wait guards every read of
+// the earlier kernels' results.
 //
 // Activations enter the tensor cores as three int8 limbs with one scale per
 // vector (per slice for h): x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254,
@@ -1033,9 +1035,8 @@ __device__ void quantise_vector(const float *src, int n, float vmax, int8_t *dst
 }
 
 // Shared-memory tables of k2: +/- codebook and byte-permute selectors.
-__device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, int *err) {
-  const int tid = threadIdx.x;
-  for (int ix = tid; ix < 256; ix += blockDim.x) {
+__device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, int *err, int tid, int nthreads) {
+  for (int ix = tid; ix < 256; ix += nthreads) {
     const uint2 raw = *reinterpret_cast<const uint2 *>(grid + 8 * ix);
     if ((raw.x | raw.y) & 0x80808080u) set_error(err, kErrGrid);
     // negate each byte: (0x80 - b) ^ 0x80 computed per byte without carries
@@ -1044,7 +1045,7 @@ __device__ void build_tables(const uint8_t *grid, uint8_t *gpm, uint8_t *selt, i
 #pragma unroll
     for (int rep = 0; rep < 8; ++rep) *reinterpret_cast<uint4 *>(gpm + ix * 128 + rep * 16) = e;
   }
-  for (int m7 = tid; m7 < 128; m7 += blockDim.x) {
+  for (int m7 = tid; m7 < 128; m7 += nthreads) {
     const uint32_t m8 = (uint32_t)m7 | ((uint32_t)(__popc(m7) & 1) << 7);
     uint32_t lo = 0, hi = 0;
 #pragma unroll
@@ -1192,17 +1193,24 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&S.mbar[warp][1])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  build_tables(a.wt.grid, gpm, selt, a.err);
-  __syncthreads();  // tables in place for every warp
   const int nw = (int)(blockDim.x >> 5);
+  if (XSMEM) {
+    // the warps that make the x limbs also build the tables (below), on their
+    // own named barrier, and publish both with limbs_ready
+    __syncthreads();  // the mbarriers are initialised
+  } else {
+    build_tables(a.wt.grid, gpm, selt, a.err, tid, (int)blockDim.x);
+    __syncthreads();  // tables in place for every warp
+  }
   constexpr int kUW = 2 * MAXP;  // tokens per unit: 2 per MMA column pair
   if (XSMEM && warp >= T) {
-    // The x limbs of the T tokens are made here from x itself (as k1 makes
-    // them) by the warps that do not route, on a named barrier of their own,
-    // so the shared expert's gate/up units can run while k1 is still
-    // computing the router: nothing before the first counter update below
-    // reads k1's results.
+    // The decoding tables and the x limbs of the T tokens are made here (the
+    // limbs from x itself, as k1 makes them) by the warps that do not copy
+    // the routing, on a named barrier of their own, so the shared expert's
+    // gate/up units can run before the routing is known: nothing before the
+    // first counter update below reads the earlier kernels' results.
     const int ltid = tid - 32 * T, lthreads = (nw - T) * 32;
+    build_tables(a.wt.grid, gpm, selt, a.err, ltid, lthreads);
     const int n4 = d.H / 4;
     for (int t = 0; t < T; ++t) {
       const float4 *xt = reinterpret_cast<const float4 *>(a.x + (size_t)t * d.H);
@@ -1273,21 +1281,20 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   // Warps 0..T-1 route one token each and warp 0 builds the job table; the
   // other warps start on the shared expert's gate/up units, which need no
   // routing, and wait for the table only when they claim a routed unit.
-  const int nr = T < nw ? T : nw;  // routing warps
-  if (warp < nr) {
-    pdl_wait();  // the router's keys
-    for (int t = warp; t < T; t += nr) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * nr) : "memory");
-    if (warp == 0) {
-      warp_build_jobs(S.idx, T, d.k, kUW, S.J);
-      if (blockIdx.x == 0)
-        for (int i = lane; i < T * d.k; i += 32) {
-          s.idx[i] = S.idx[i];
-          s.w[i] = S.w[i];
-        }
-      __threadfence_block();
-      if (lane == 0) *reinterpret_cast<volatile int *>(&S.jobs_ready) = 1;
+  // Warp 0 copies the call's routing (idx, w) and job table, made once by
+  // the routing kernel, into shared memory; warps 1..T-1 (which do not make
+  // limbs) wait for the limbs below like warp 0.
+  if (warp == 0) {
+    pdl_wait();  // the routing kernel's results
+    int *jd = reinterpret_cast<int *>(&S.J);
+    for (int i = lane; i < kJobsInts; i += 32) jd[i] = __ldcg(s.jobs + i);
+    for (int i = lane; i < T * d.k; i += 32) {
+      S.idx[i] = __ldcg(s.idx + i);
+      S.w[i] = __ldcg(s.w + i);
     }
+    __syncwarp();
+    __threadfence_block();
+    if (lane == 0) *reinterpret_cast<volatile int *>(&S.jobs_ready) = 1;
   }
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
@@ -1711,6 +1718,34 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   if (warp == nw - 1 && lane == 0) prefetch_next_layer(a.pf);
 }
 
+// ------------------------------------------------------------------ routing and job table
+
+// One block for the whole call: every token's top-k and weights (one warp
+// per token at a time, as the oracle selects), then the job table of the
+// distinct experts, written to scratch for every CTA of the expert kernel to
+// copy.  Launched as a programmatic dependent of k1 (it waits for the
+// router's keys); the expert kernel is its own programmatic dependent.
+constexpr int kRouteJobsThreads = 256;
+__global__ void __launch_bounds__(kRouteJobsThreads) k_route_jobs(const __grid_constant__ DecodeArgs a) {
+  pdl_launch_dependents();
+  __shared__ int32_t idx[kDecodeMaxT * kMaxK];
+  __shared__ float w[kDecodeMaxT * kMaxK];
+  __shared__ Jobs J;
+  pdl_wait();  // k1's keys and scores (router mode), its counter resets
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int T = a.T, k = a.d.k;
+  for (int t = warp; t < T; t += nw) warp_route_token(a, t, idx + t * k, w + t * k);
+  __syncthreads();
+  if (warp == 0) warp_build_jobs(idx, T, k, a.s.UW, J);
+  __syncthreads();
+  const int *js = reinterpret_cast<const int *>(&J);
+  for (int i = threadIdx.x; i < kJobsInts; i += blockDim.x) a.s.jobs[i] = js[i];
+  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+    a.s.idx[i] = idx[i];
+    a.s.w[i] = w[i];
+  }
+}
+
 // ------------------------------------------------------------------ route only
 
 __global__ void k_route_only(DecodeArgs a, int32_t *idx, float *w) {
@@ -1725,6 +1760,13 @@ size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
   return b;
 }
 constexpr size_t kSmemLimit = kSmemOptInMax;
+
+template <typename K>
+cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a);
+
+cudaError_t launch_route_jobs(const DecodeArgs &a, cudaStream_t stream) {
+  return launch_pdl(k_route_jobs, 1, kRouteJobsThreads, 0, stream, a);
+}
 
 template <typename K>
 cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a) {
@@ -1888,6 +1930,8 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
 
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   cudaError_t e = launch_k1(a, stream);
+  if (e != cudaSuccess) return e;
+  e = launch_route_jobs(a, stream);
   if (e != cudaSuccess) return e;
   // the variant whose unit width the scratch was carved for
   switch (a.s.UW) {

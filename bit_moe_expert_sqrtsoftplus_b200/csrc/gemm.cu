@@ -50,10 +50,14 @@ constexpr int kSignRep = 8;                        // replicas of the sign-mask 
 __host__ __device__ constexpr int ahead_of(int fmt) { return fmt == 0 ? 6 : fmt == 1 ? 4 : 3; }
 constexpr int BM = 128, BK = 64;
 constexpr int kATile = BM * BK * 2;  // 16 KB
-// token columns per tile: 128 for a gate/up pair (two accumulators per tile,
-// two tiles in flight fill the 512 TMEM columns), 256 for a single matrix
-__host__ __device__ constexpr int bn_of(bool paired) { return paired ? 128 : 256; }
-__host__ __device__ constexpr int btile_of(bool paired) { return bn_of(paired) * BK * 2; }
+// token columns per tile: 128 for a routed gate/up pair (two accumulators
+// per tile, two tiles in flight fill the 512 TMEM columns; experts hold few
+// tokens, so narrow tiles waste less), 256 for a single matrix and for the
+// shared expert's pair (all T tokens: wide tiles decode each weight tile
+// fewer times; that pair's one tile fills TMEM alone)
+__host__ __device__ constexpr int bn_of(int fmt, bool paired) { return paired && fmt != 2 ? 128 : 256; }
+__host__ __device__ constexpr int btile_of(int fmt, bool paired) { return bn_of(fmt, paired) * BK * 2; }
+__host__ __device__ constexpr int nacc_of(int fmt, bool paired) { return (paired ? 2 : 1) * bn_of(fmt, paired) <= 256 ? 2 : 1; }
 // stages of the dequantised A ring: how many K steps the producers may run
 // ahead of the MMA (a pair's stage holds both matrices' tiles)
 #ifndef MOE_GEMM_SA_PAIRED
@@ -452,12 +456,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
   constexpr int SA = sa_of(PAIRED);
-  constexpr int BN = bn_of(PAIRED);
-  constexpr int kBTile = btile_of(PAIRED);
+  constexpr int BN = bn_of(FMT, PAIRED);
+  constexpr int kBTile = btile_of(FMT, PAIRED);
   // accumulator buffers in tensor memory: two tiles alternate (a pair's two
   // 128-column accumulators, or one 256-column accumulator, per tile), so the
   // epilogue of one tile overlaps the main loop of the next
-  constexpr int NACC = 2;
+  constexpr int NACC = nacc_of(FMT, PAIRED);
   constexpr int ACC_COLS = NA * BN;  // columns of one tile's accumulators
   constexpr int ASTAGE = NA * kATile;
   constexpr bool kTables = FMT == kFmtIQ2;
@@ -734,7 +738,7 @@ size_t grouped_gemm_smem(int fmt, int paired) {
   const int na = paired ? 2 : 1;
   const int sa = sa_of(paired != 0);
   const size_t tables = fmt == kFmtIQ2 ? 4096 * kGridRep + 2048 * kSignRep : 0;
-  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * btile_of(paired != 0) + tables + sizeof(GemmCtl);
+  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * btile_of(fmt, paired != 0) + tables + sizeof(GemmCtl);
 }
 
 template <int FMT, bool PAIRED>
