@@ -382,10 +382,9 @@ def run_ours(args, world, rank):
          "achieved_gbs": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"], "distinct_experts_per_call": n_distinct},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 4,
                 "d2h_bytes_per_step": T * s.hidden * 4},
-        # batched: router (4), permutation (3), input, 4 GEMMs; small-token: k1, the
-        # routing kernel and k2, or for Q4_K layers k1, the routing kernel and the
-        # 3 expert kernels
-        "gpu_launches": (12 if large else 5 if s.q4k else 3) * args.steps,
+        # batched: router (4), permutation (3), input, 4 GEMMs; small-token: k1 and
+        # k2, or for Q4_K layers k1, the routing kernel and the 3 expert kernels
+        "gpu_launches": (12 if large else 5 if s.q4k else 2) * args.steps,
         "clocks": clocks,
     }
     return out
@@ -483,14 +482,14 @@ def run_stack(args, world, rank):
                    "l2": f"{s.layers} distinct layer weight sets ({s.layers * s.n_experts * s.expert_bytes / 1e9:.1f} "
                          "GB, far larger than the 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": (f"whole stack step ({s.layers - s.q4k_layers} x k1/routing/k2"
+        "roofline": {"bound": "hbm", "kernel": (f"whole stack step ({s.layers - s.q4k_layers} x k1/k2"
                                               + (f", {s.q4k_layers} Q4_K layers x 5 launches)" if s.q4k_layers
                                                  else ")")), "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": peaks["source"], "algorithmic_bytes_per_step": nd_bytes},
         "e2e": {"value": job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * s.hidden * 4, "d2h_bytes_per_step": T * s.hidden * 4},
-        "gpu_launches": (3 * (s.layers - s.q4k_layers) + 5 * s.q4k_layers) * args.steps,
+        "gpu_launches": (2 * (s.layers - s.q4k_layers) + 5 * s.q4k_layers) * args.steps,
         "clocks": clock.summary(),
     }
 

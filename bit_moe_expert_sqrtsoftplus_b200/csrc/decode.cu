@@ -1,11 +1,10 @@
-// decode.cu -- the layer for small token counts (T <= 32): three kernels.
+// decode.cu -- the layer for small token counts (T <= 32): two kernels.
 //
 //   k1_prep_router  x -> int8 limbs (optionally RMSNorm first); fp64 router
 //                   logits, scores s = sqrtsoftplus(z) and selection keys
 //                   s + bias, one block per pair of experts.
-//   k_route_jobs    one block: every token's top-k from the keys (comparisons
-//                   only) and the call's job table, for all CTAs of k2.
-//   k2_experts      copies the routing, then all the expert work as warp-sized units on one
+//   k2_experts      top-k routing from the keys (comparisons only, per CTA),
+//                   then all the expert work as warp-sized units on one
 //                   counter: every (16-row tile, 1024-element K part) of the
 //                   shared and the routed gate/up matrices, then every
 //                   (K part, 16-row output tile) of the shared and the routed
@@ -20,10 +19,9 @@
 //                   limbs and flags it, and down units wait for the slices
 //                   they read.  The warp that completes an output tile sums
 //                   its parts in a fixed order (deterministic) into y.
-// k_route_jobs is a programmatic dependent of k1 and k2 of k_route_jobs:
-// k2's set-up (tables, shared memory, the x limbs, the shared expert's first
-// units) overlaps the routing, and griddepcontrol.wait guards every read of
-// the earlier kernels' results.
+// k2 is launched as a programmatic dependent of k1: its set-up (tables,
+// shared memory, the x limbs, the shared expert's first units) overlaps k1
+// and the routing, and griddepcontrol.wait guards every read of k1's results.
 //
 // Activations enter the tensor cores as three int8 limbs with one scale per
 // vector (per slice for h): x ~= s1*q1 + s2*q2 + s3*q3, s2 = s1/254,
@@ -60,6 +58,10 @@ constexpr bool kAheadClaim = MOE_DECODE_AHEAD != 0;
 #define MOE_DECODE_GUNROLL 2
 #endif
 constexpr int kGUnroll = MOE_DECODE_GUNROLL;  // unrolling of the IQ2_XXS group loop
+#ifndef MOE_DECODE_BUNROLL
+#define MOE_DECODE_BUNROLL 4
+#endif
+constexpr int kBUnroll = MOE_DECODE_BUNROLL;  // unrolling of the IQ2_XXS block loop (code size)
 constexpr int kThreads2 = kWarps2 * kWarp;
 // k2 threads: 12 warps for four token pairs, whose accumulators need more
 // than the 128 registers a thread has at 16 warps
@@ -777,7 +779,7 @@ __device__ __forceinline__ void iq2_chunk(const uint8_t *st, int k0, const uint8
   const int sh7 = 7 * c;
   const uint8_t *row0 = st + r * RS;
   const uint8_t *row1 = row0 + 8 * RS;
-#pragma unroll
+#pragma unroll kBUnroll
   for (int b = 0; b < NB; ++b) {
     const float d0 = half_bits_to_float(lds_u16(row0 + 66 * b)) * 0.125f;
     const float d1 = half_bits_to_float(lds_u16(row1 + 66 * b)) * 0.125f;
@@ -1281,20 +1283,26 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   // Warps 0..T-1 route one token each and warp 0 builds the job table; the
   // other warps start on the shared expert's gate/up units, which need no
   // routing, and wait for the table only when they claim a routed unit.
-  // Warp 0 copies the call's routing (idx, w) and job table, made once by
-  // the routing kernel, into shared memory; warps 1..T-1 (which do not make
-  // limbs) wait for the limbs below like warp 0.
-  if (warp == 0) {
-    pdl_wait();  // the routing kernel's results
-    int *jd = reinterpret_cast<int *>(&S.J);
-    for (int i = lane; i < kJobsInts; i += 32) jd[i] = __ldcg(s.jobs + i);
-    for (int i = lane; i < T * d.k; i += 32) {
-      S.idx[i] = __ldcg(s.idx + i);
-      S.w[i] = __ldcg(s.w + i);
+  // Warps 0..T-1 route one token each and warp 0 builds the job table; the
+  // other warps start on the shared expert's gate/up units, which need no
+  // routing, and wait for the table only when they claim a routed unit.
+  // (Routing in every CTA beats one routing block followed by copies: the
+  // copies would wait for that block's whole kernel to finish.)
+  const int nr = T < nw ? T : nw;  // routing warps
+  if (warp < nr) {
+    pdl_wait();  // the router's keys
+    for (int t = warp; t < T; t += nr) warp_route_token(a, t, S.idx + t * d.k, S.w + t * d.k);
+    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * nr) : "memory");
+    if (warp == 0) {
+      warp_build_jobs(S.idx, T, d.k, kUW, S.J);
+      if (blockIdx.x == 0)
+        for (int i = lane; i < T * d.k; i += 32) {
+          s.idx[i] = S.idx[i];
+          s.w[i] = S.w[i];
+        }
+      __threadfence_block();
+      if (lane == 0) *reinterpret_cast<volatile int *>(&S.jobs_ready) = 1;
     }
-    __syncwarp();
-    __threadfence_block();
-    if (lane == 0) *reinterpret_cast<volatile int *>(&S.jobs_ready) = 1;
   }
 
   const uint8_t *gpm_l = gpm + (lane & 7) * 16;
@@ -1718,34 +1726,6 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   if (warp == nw - 1 && lane == 0) prefetch_next_layer(a.pf);
 }
 
-// ------------------------------------------------------------------ routing and job table
-
-// One block for the whole call: every token's top-k and weights (one warp
-// per token at a time, as the oracle selects), then the job table of the
-// distinct experts, written to scratch for every CTA of the expert kernel to
-// copy.  Launched as a programmatic dependent of k1 (it waits for the
-// router's keys); the expert kernel is its own programmatic dependent.
-constexpr int kRouteJobsThreads = 256;
-__global__ void __launch_bounds__(kRouteJobsThreads) k_route_jobs(const __grid_constant__ DecodeArgs a) {
-  pdl_launch_dependents();
-  __shared__ int32_t idx[kDecodeMaxT * kMaxK];
-  __shared__ float w[kDecodeMaxT * kMaxK];
-  __shared__ Jobs J;
-  pdl_wait();  // k1's keys and scores (router mode), its counter resets
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int T = a.T, k = a.d.k;
-  for (int t = warp; t < T; t += nw) warp_route_token(a, t, idx + t * k, w + t * k);
-  __syncthreads();
-  if (warp == 0) warp_build_jobs(idx, T, k, a.s.UW, J);
-  __syncthreads();
-  const int *js = reinterpret_cast<const int *>(&J);
-  for (int i = threadIdx.x; i < kJobsInts; i += blockDim.x) a.s.jobs[i] = js[i];
-  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-    a.s.idx[i] = idx[i];
-    a.s.w[i] = w[i];
-  }
-}
-
 // ------------------------------------------------------------------ route only
 
 __global__ void k_route_only(DecodeArgs a, int32_t *idx, float *w) {
@@ -1760,13 +1740,6 @@ size_t k2_smem_bytes(const LayerDims &d, int T, bool xsmem) {
   return b;
 }
 constexpr size_t kSmemLimit = kSmemOptInMax;
-
-template <typename K>
-cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a);
-
-cudaError_t launch_route_jobs(const DecodeArgs &a, cudaStream_t stream) {
-  return launch_pdl(k_route_jobs, 1, kRouteJobsThreads, 0, stream, a);
-}
 
 template <typename K>
 cudaError_t launch_pdl(K kernel, int grid, int block, size_t smem, cudaStream_t stream, const DecodeArgs &a) {
@@ -1930,8 +1903,6 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
 
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
   cudaError_t e = launch_k1(a, stream);
-  if (e != cudaSuccess) return e;
-  e = launch_route_jobs(a, stream);
   if (e != cudaSuccess) return e;
   // the variant whose unit width the scratch was carved for
   switch (a.s.UW) {

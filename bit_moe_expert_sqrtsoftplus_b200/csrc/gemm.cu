@@ -65,11 +65,18 @@ __host__ __device__ constexpr int nacc_of(int fmt, bool paired) { return (paired
 #endif
 __host__ __device__ constexpr int sa_of(bool paired) { return paired ? MOE_GEMM_SA_PAIRED : 4; }
 
-constexpr int kSB = 4;       // stages of the B (token rows) ring
-constexpr int kBAhead = 2;   // K steps a B tile is loaded ahead of its use
+// stages of the B (token rows) ring; a B tile is loaded kSB - 2 K steps
+// ahead of its use (the stage it reuses was read by the MMA two steps back)
+#ifndef MOE_GEMM_BSTAGES_NARROW
+#define MOE_GEMM_BSTAGES_NARROW 4
+#endif
+constexpr int kSBMax = 8;
+__host__ __device__ constexpr int sb_of(int fmt, bool paired) {
+  return bn_of(fmt, paired) == 128 ? MOE_GEMM_BSTAGES_NARROW : 4;
+}
 
 struct alignas(8) GemmCtl {
-  uint64_t full[kSB], emptyA[4], emptyB[kSB], acc_full[2], acc_empty[2], drain;
+  uint64_t full[kSBMax], emptyA[4], emptyB[kSBMax], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
   long long wait;  // bound of the role hand-off waits (cycles)
@@ -194,8 +201,33 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t ldg16(const uint8_t *p) { return *reinterpret_cast<const uint16_t *>(p); }
-__device__ __forceinline__ uint32_t ldg32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+// Packed weights are read once per tile; with MOE_GEMM_EVICT_FIRST their
+// loads carry an L2 evict-first policy so the activation rows that every
+// tile of a group re-reads stay in L2.
+#ifndef MOE_GEMM_EVICT_FIRST
+#define MOE_GEMM_EVICT_FIRST 0
+#endif
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint32_t ldg16(const uint8_t *p) {
+  if (MOE_GEMM_EVICT_FIRST) {
+    uint16_t v;
+    asm volatile("ld.global.L2::cache_hint.u16 %0, [%1], %2;\n" : "=h"(v) : "l"(p), "l"(l2_evict_first()));
+    return v;
+  }
+  return *reinterpret_cast<const uint16_t *>(p);
+}
+__device__ __forceinline__ uint32_t ldg32(const uint8_t *p) {
+  if (MOE_GEMM_EVICT_FIRST) {
+    uint32_t v;
+    asm volatile("ld.global.L2::cache_hint.u32 %0, [%1], %2;\n" : "=r"(v) : "l"(p), "l"(l2_evict_first()));
+    return v;
+  }
+  return *reinterpret_cast<const uint32_t *>(p);
+}
 
 __device__ __forceinline__ void sts128(uint8_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
@@ -458,6 +490,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   constexpr int SA = sa_of(PAIRED);
   constexpr int BN = bn_of(FMT, PAIRED);
   constexpr int kBTile = btile_of(FMT, PAIRED);
+  constexpr int kSB = sb_of(FMT, PAIRED);
+  constexpr int kBAhead = kSB - 2;
+  static_assert(kSB <= kSBMax, "B ring");
   // accumulator buffers in tensor memory: two tiles alternate (a pair's two
   // 128-column accumulators, or one 256-column accumulator, per tile), so the
   // epilogue of one tile overlaps the main loop of the next
@@ -738,7 +773,8 @@ size_t grouped_gemm_smem(int fmt, int paired) {
   const int na = paired ? 2 : 1;
   const int sa = sa_of(paired != 0);
   const size_t tables = fmt == kFmtIQ2 ? 4096 * kGridRep + 2048 * kSignRep : 0;
-  return 1024 + (size_t)sa * na * kATile + (size_t)kSB * btile_of(fmt, paired != 0) + tables + sizeof(GemmCtl);
+  return 1024 + (size_t)sa * na * kATile + (size_t)sb_of(fmt, paired != 0) * btile_of(fmt, paired != 0) + tables +
+         sizeof(GemmCtl);
 }
 
 template <int FMT, bool PAIRED>

@@ -163,8 +163,8 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
  * The whole layer.  x: [T][H] fp32 input; y: [T][H] fp32 output
  * (overwritten; may alias x only with MOE_FLAG_PRENORM_RESIDUAL, where
  * y = x + MoE(RMSNorm(x))).  T = 0 is a no-op.  Calls with
- * T <= MOE_SMALL_T_MAX run the small-token path (three kernel launches: input
- * preparation and router, routing, then every expert unit); larger T the batched
+ * T <= MOE_SMALL_T_MAX run the small-token path (two kernel launches: input
+ * preparation and router, then routing and every expert unit); larger T the batched
  * tensor-core path (twelve launches in router mode: router, certificate,
  * fix-up, permutation, four grouped GEMMs).
  */
