@@ -73,55 +73,81 @@ __global__ void k_token_norms(const float *x, int T, int H, int flags, float eps
   }
 }
 
-// z[t][e] for a 64-token x 64-expert tile; 256 threads, each 4 x 4 outputs.
-constexpr int RT = 64, RE = 64, RK = 32;
+// z[t][e] for a 64-token x 128-expert tile; 256 threads, each 4 tokens x 8
+// experts.  Per 32-element K chunk every output is a sum of 32 fp32 FMAs
+// (the chunk the error bound below assumes), added to an fp64 accumulator.
+// Rows are staged with 16-byte loads (x scaled by the token's fp32 inverse
+// RMS, W_r converted from f16), transposed into K-major shared tiles.
+constexpr int RT = 64, RE = 128, RK = 32;
 __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double *inv, const uint16_t *Wr, int T,
                                                     int E, int H, double *z) {
   __shared__ __align__(16) float xs[RK][RT + 4];
   __shared__ __align__(16) float ws[RK][RE + 4];
   const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE;
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads
-  double acc[4][4];
+  const int tx = tid & 15, ty = tid >> 4;  // experts tx*8 .., tokens ty*4 ..
+  // staging roles: x float4 pieces (token i>>3, K quad i&7) and W uint4
+  // pieces (expert i>>2, K octet i&3) for i = tid and tid + 256
+  float invf[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int t = t0 + ((tid + 256 * r) >> 3);
+    invf[r] = t < T ? (float)inv[t] : 0.f;
+  }
+  double acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
   for (int k0 = 0; k0 < H; k0 += RK) {
-    // stage x (scaled by the token's inverse RMS) and W as fp32, K-major
-    for (int i = tid; i < RT * RK; i += 256) {
-      const int tt = i / RK, kk = i % RK;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * r;
+      const int tt = i >> 3, kq = i & 7;
       const int t = t0 + tt;
-      float v = 0.f;
-      if (t < T) v = x[(size_t)t * H + k0 + kk] * (float)inv[t];
-      xs[kk][tt] = v;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < T) v = *reinterpret_cast<const float4 *>(x + (size_t)t * H + k0 + 4 * kq);
+      xs[4 * kq + 0][tt] = v.x * invf[r];
+      xs[4 * kq + 1][tt] = v.y * invf[r];
+      xs[4 * kq + 2][tt] = v.z * invf[r];
+      xs[4 * kq + 3][tt] = v.w * invf[r];
     }
-    for (int i = tid; i < RE * RK; i += 256) {
-      const int ee = i / RK, kk = i % RK;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * r;
+      const int ee = i >> 2, ko = i & 3;
       const int e = e0 + ee;
-      ws[kk][ee] = e < E ? half_bits_to_float(Wr[(size_t)e * H + k0 + kk]) : 0.f;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (e < E) v = *reinterpret_cast<const uint4 *>(Wr + (size_t)e * H + k0 + 8 * ko);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        ws[8 * ko + 2 * q][ee] = half_bits_to_float((uint16_t)(w4[q] & 0xFFFFu));
+        ws[8 * ko + 2 * q + 1][ee] = half_bits_to_float((uint16_t)(w4[q] >> 16));
+      }
     }
     __syncthreads();
-    float part[4][4];
+    float part[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+      for (int j = 0; j < 8; ++j) part[i][j] = 0.f;
 #pragma unroll 8
     for (int kk = 0; kk < RK; ++kk) {
       const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
-      const float4 wv = *reinterpret_cast<const float4 *>(&ws[kk][tx * 4]);
+      const float4 w0 = *reinterpret_cast<const float4 *>(&ws[kk][tx * 8]);
+      const float4 w1 = *reinterpret_cast<const float4 *>(&ws[kk][tx * 8 + 4]);
       const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float wa[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
+        for (int j = 0; j < 8; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
+      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part[i][j];
     __syncthreads();
   }
 #pragma unroll
@@ -129,8 +155,8 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
     const int t = t0 + ty * 4 + i;
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + tx * 8 + j;
       if (e < E) z[(size_t)t * E + e] = acc[i][j];
     }
   }
