@@ -796,7 +796,7 @@ __device__ __forceinline__ void iq2_chunk(const uint8_t *st, int k0, const uint8
       const int kel = k0 + 256 * b + 32 * g;  // the column base includes 8c
 #pragma unroll
       for (int p = 0; p < MAXP; ++p) {
-        if (p < npairs) {
+        if (MAXP == 1 || p < npairs) {
           const uint2 bb = ldb(bcol[p], kel);
           const int zero[4] = {0, 0, 0, 0};
           int cg[4];
@@ -847,7 +847,7 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol 
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
-      for (int p = 0; p < MAXP; ++p) B[kPre ? b : 0][p] = p < npairs ? ldb(bcol[p], k0 + 32 * b) : make_uint2(0u, 0u);
+      for (int p = 0; p < MAXP; ++p) B[kPre ? b : 0][p] = (MAXP == 1 || p < npairs) ? ldb(bcol[p], k0 + 32 * b) : make_uint2(0u, 0u);
   }
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
@@ -859,7 +859,7 @@ __device__ __forceinline__ void q80_chunk(const uint8_t *st, int k0, const BCol 
     q80_vals(row1, o, c, A[1], A[3]);
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
-      if (p < npairs) {
+      if (MAXP == 1 || p < npairs) {
         const uint2 bb = kPre ? B[kPre ? b : 0][p] : ldb(bcol[p], k0 + 32 * b);
         const int zero[4] = {0, 0, 0, 0};
         int cg[4];
@@ -917,9 +917,9 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
 #pragma unroll
           for (int p = 0; p < MAXP; ++p)
             B[kPre ? hf : 0][kPre ? sh : 0][p] =
-                p < npairs ? ldb(bcol[p], k0 + 256 * b + 128 * hf + 32 * sh) : make_uint2(0u, 0u);
+                (MAXP == 1 || p < npairs) ? ldb(bcol[p], k0 + 256 * b + 128 * hf + 32 * sh) : make_uint2(0u, 0u);
 #pragma unroll
-      for (int p = 0; p < MAXP; ++p) BX[p] = p < npairs ? ldx(xcol[p], kb * 16) : 0u;  // base includes 4c
+      for (int p = 0; p < MAXP; ++p) BX[p] = (MAXP == 1 || p < npairs) ? ldx(xcol[p], kb * 16) : 0u;  // base includes 4c
     }
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -941,7 +941,7 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
         A[3] = ((q1.y >> (2 * sh)) & 0x03030303u) * sc1;
 #pragma unroll
         for (int p = 0; p < MAXP; ++p) {
-          if (p < npairs) {
+          if (MAXP == 1 || p < npairs) {
             const uint2 bb = kPre ? B[kPre ? hf : 0][kPre ? sh : 0][p] : ldb(bcol[p], k0 + 256 * b + 128 * hf + 32 * sh);
             mma_s8(Cm[p], A, bb.x, bb.y, Cm[p]);
           }
@@ -956,7 +956,7 @@ __device__ __forceinline__ void q2k_chunk(const uint8_t *st, int k0, const BCol 
     Am[3] = 0u;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
-      if (p < npairs) {
+      if (MAXP == 1 || p < npairs) {
         const uint32_t bx = kPre ? BX[p] : ldx(xcol[p], kb * 16);  // base includes 4c
         const int zero[4] = {0, 0, 0, 0};
         int cn[4];
@@ -1500,7 +1500,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   auto store_part = [&](const Unit &cu, int m) {
 #pragma unroll
     for (int p = 0; p < MAXP; ++p) {
-      if (p < npairs) {
+      if (MAXP == 1 || p < npairs) {
         const int ts = 2 * p + (c >> 1);
         float v0, v1;
         combine_limbs(F[p], ts < cu.ntok ? (XSMEM ? S.xs : s.xs) + 4 * xrow(cu, ts) : nullptr, v0, v1);
@@ -1668,7 +1668,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
           if (cc == cu.nch - 1) {
 #pragma unroll
             for (int p = 0; p < MAXP; ++p) {
-              if (p < npairs) {
+              if (MAXP == 1 || p < npairs) {
                 const int ts = 2 * p + (c >> 1);
                 const bool ok = ts < cu.ntok;
                 const int v = ok ? cu.pairs[ts] : 0;
@@ -1703,7 +1703,7 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
           if (cc == cu.nch - 1) {
 #pragma unroll
             for (int p = 0; p < MAXP; ++p) {
-              if (p < npairs) {
+              if (MAXP == 1 || p < npairs) {
                 const int ts = 2 * p + (c >> 1);
                 const float *sc = ts < cu.ntok ? s.hsc + 4 * ((T * d.k + cu.t0 + ts) * s.NSL + cu.kp) : nullptr;
                 float v0, v1;
