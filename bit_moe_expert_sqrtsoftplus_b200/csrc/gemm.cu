@@ -22,8 +22,6 @@
 // Tiles: M = 128 weight rows, N = up to 256 columns (tokens) of one group, K
 // stepped 64 at a time (four K=16 MMAs per step).  A gate/up pair shares the
 // B tile and uses two accumulators (columns 0-255 and 256-511).
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -41,12 +39,6 @@ constexpr int kProdWarps = 16;
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 24
 constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 800
 constexpr int kProd = kProdWarps * 32;             // 512 producer threads
-// hand-offs counted per warp (lane 0 arrives after __syncwarp) instead of
-// per thread: 16 arrivals per K step on the full barrier instead of 512
-#ifndef MOE_GEMM_WARP_ARRIVE
-#define MOE_GEMM_WARP_ARRIVE 0
-#endif
-constexpr bool kWarpArrive = MOE_GEMM_WARP_ARRIVE != 0;
 // Codebook and sign tables: an entry is read as 16 bytes by 8 lanes per
 // shared-memory wavefront; with 8 replicas, lane l reads replica l % 8, so
 // the 8 lanes of a wavefront hit 8 different 16-byte bank groups whatever
@@ -489,7 +481,7 @@ __device__ __forceinline__ void decode(const Raw<kFmtQ80> &r, uint8_t *tile, int
 // ---------------------------------------------------------------- kernel
 
 template <int FMT, bool PAIRED>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
+__global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   // A (dequantised weights) and B (gathered token rows) have rings of their
   // own: a B tile is loaded kBAhead steps before its use, an A tile is
   // written in the step that hands it to the MMA; step `it` uses A stage
@@ -524,14 +516,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   // ---- set-up
   if (tid == 0) {
     for (int s = 0; s < kSB; ++s) {
-      // producer arrivals, plus the TMA issuer's expect-tx arrival when B comes by TMA
-      mbar_init(&ctl.full[s], (kWarpArrive ? kProdWarps : kProd) + (a.b_tma ? 1 : 0));
+      mbar_init(&ctl.full[s], kProd);
       mbar_init(&ctl.emptyB[s], 1);
     }
     for (int s = 0; s < SA; ++s) mbar_init(&ctl.emptyA[s], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl.acc_full[b], 1);
-      mbar_init(&ctl.acc_empty[b], kWarpArrive ? kEpiWarps : kEpiWarps * 32);
+      mbar_init(&ctl.acc_empty[b], kEpiWarps * 32);
     }
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
@@ -626,31 +617,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         }
         cp_async_commit();
       };
-      // TMA: producer 0 alone waits for the stage, arms the stage's full
-      // barrier with the tile's bytes and issues one 128-byte-swizzled tile
-      // copy of BN rows from the tile's first column (rows past the group
-      // are read too and ignored by the epilogue; rows past the buffer read
-      // as zero); the other producers take no part in B
-      auto issue_b_tma = [&](int ks, int sb) {
-        uint64_t *bar = &ctl.full[sb];
-        const uint32_t mb = smem_u32(bar);
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(mb), "r"((uint32_t)kBTile)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-            "[%4];\n" ::"r"(smem_u32(stagesB + sb * kBTile)),
-            "l"(reinterpret_cast<uint64_t>(&a.tmb)), "r"(ks * BK), "r"(tl.col0), "r"(mb)
-            : "memory");
-      };
       // waits until the B stage of global step g is free, then loads it (or
       // commits an empty group past the tile's last step)
       auto load_b = [&](int ks, uint32_t g) -> bool {
-        if (a.b_tma) {
-          if (ks >= ksteps || p != 0) return true;
-          if (!mbar_wait(&ctl.emptyB[g % kSB], ((g / kSB) & 1u) ^ 1u, ctl, a.err)) return false;
-          issue_b_tma(ks, g % kSB);
-          return true;
-        }
         if (ks >= ksteps) {
           cp_async_commit();
           return true;
@@ -675,15 +644,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           }
           uint8_t *A0s = stagesA + (it % SA) * ASTAGE;
           if (has_a) decode(R[j], A0s + mat * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh_l, signm_l);
-          if (!a.b_tma) cp_async_wait<kBAhead>();  // this step's B tile has landed
+          cp_async_wait<kBAhead>();  // this step's B tile has landed
           fence_proxy_async();
-          if (kWarpArrive) {
-            // one arrival per warp, after every lane's writes are ordered
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl.full[it % kSB]);
-          } else {
-            mbar_arrive(&ctl.full[it % kSB]);
-          }
+          mbar_arrive(&ctl.full[it % kSB]);
           // the next look-ahead fetch goes out after this step is handed over
           if (has_a && ks + kAhead < ksteps) fetch(R[(j + kAhead) % (kAhead + 1)], arow, ks + kAhead, item);
           ++it;
@@ -792,12 +755,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         }
       }
       tc_fence_before();
-      if (kWarpArrive) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl.acc_empty[buf]);
-      } else {
-        mbar_arrive(&ctl.acc_empty[buf]);
-      }
+      mbar_arrive(&ctl.acc_empty[buf]);
     }
   }
 
@@ -829,41 +787,8 @@ static cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   return cudaGetLastError();
 }
 
-// B tensor map for a launch whose B rows are contiguous: [b_rows][K] 16-bit
-// elements, rows b_ld elements apart, box 64 elements (128 bytes) x BN rows,
-// 128-byte swizzle (the layout the MMA descriptors read).  False when the
-// driver entry point is missing or the shape does not allow it.
-static bool encode_b_map(GemmArgs &g, int bn) {
-  static PFN_cuTensorMapEncodeTiled encode = nullptr;
-  static bool looked = false;
-  if (!looked) {
-    looked = true;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&encode), cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      encode = nullptr;
-  }
-  if (!encode || g.b_perm || g.b_rows <= 0 || (reinterpret_cast<uintptr_t>(g.b_base) & 15) || ((size_t)g.b_ld * 2) % 16)
-    return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.b_rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)g.b_ld * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)bn};
-  const cuuint32_t es[2] = {1, 1};
-  return encode(reinterpret_cast<CUtensorMap *>(&g.tmb), CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
-                const_cast<uint16_t *>(g.b_base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-#ifndef MOE_GEMM_TMA_B
-#define MOE_GEMM_TMA_B 0
-#endif
-
-cudaError_t grouped_gemm(const GemmArgs &ain, cudaStream_t s, int num_sms) {
-  GemmArgs a = ain;
+cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   const bool paired = a.A1 != nullptr;
-  a.b_tma = MOE_GEMM_TMA_B && encode_b_map(a, bn_of(a.fmt, paired)) ? 1 : 0;
   if (a.fmt == kFmtIQ2 && paired) return launch_gemm<kFmtIQ2, true>(a, s, num_sms);
   if (a.fmt == kFmtQ80 && paired) return launch_gemm<kFmtQ80, true>(a, s, num_sms);
   if (a.fmt == kFmtQ80 && !paired) return launch_gemm<kFmtQ80, false>(a, s, num_sms);

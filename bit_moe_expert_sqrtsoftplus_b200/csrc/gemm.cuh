@@ -16,17 +16,7 @@ namespace moe {
 enum GemmFmt { kFmtIQ2 = 0, kFmtQ2K = 1, kFmtQ80 = 2, kFmtQ4K = 3 };
 enum GemmEpi { kEpiSwiGLU = 0, kEpiScatterAdd = 1, kEpiStore = 2 };
 
-// B tensor map (the driver's 128-byte CUtensorMap, 64-byte aligned) of a
-// GEMM whose B rows are contiguous: one TMA tile copy per K step replaces
-// the producers' row copies.
-struct alignas(64) GemmTensorMap {
-  uint64_t v[16];
-};
-
 struct GemmArgs {
-  GemmTensorMap tmb;  // valid when b_tma
-  int b_tma;          // 1: B tiles by TMA (b_perm == nullptr, b_rows rows of b_ld elements)
-  int b_rows;         // rows of the B buffer (TMA bounds)
   int fmt;    // GemmFmt of the A operand
   int bf16;   // operand type: 0 = f16, 1 = bf16
   int epi;    // GemmEpi

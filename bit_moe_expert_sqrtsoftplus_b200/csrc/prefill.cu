@@ -679,8 +679,7 @@ GemmArgs routed_gateup_args(const LayerDims &d, const LayerWeights &wt, bool q4k
 
 // Routed down GEMM: y[(perm[c] / k) * H + m] += w[perm[c]] * (W_down h)[m].
 GemmArgs routed_down_args(const LayerDims &d, const LayerWeights &wt, bool q4k, int n_groups, const int32_t *offsets,
-                          const int32_t *perm, int k, const uint16_t *hperm, int rows, const float *w, float *y,
-                          int *err) {
+                          const int32_t *perm, int k, const uint16_t *hperm, const float *w, float *y, int *err) {
   const size_t rbQ2 = (size_t)(d.I / 256) * (q4k ? 144 : 84);
   GemmArgs rd{};
   rd.fmt = q4k ? kFmtQ4K : kFmtQ2K;
@@ -696,7 +695,6 @@ GemmArgs routed_down_args(const LayerDims &d, const LayerWeights &wt, bool q4k, 
   rd.a_row_bytes = rbQ2;
   rd.b_base = hperm;
   rd.b_ld = d.I;
-  rd.b_rows = rows;
   rd.b_perm = nullptr;
   rd.b_div = 1;
   rd.y = y;
@@ -729,7 +727,6 @@ cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, cons
   sg.grid = wt.grid;
   sg.b_base = reinterpret_cast<const uint16_t *>(x16);
   sg.b_ld = d.H;
-  sg.b_rows = T;
   sg.b_perm = nullptr;
   sg.b_div = 1;
   sg.h_out = hs;
@@ -753,7 +750,6 @@ cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, cons
   sd.a_row_bytes = (size_t)(d.Is / 32) * 34;
   sd.b_base = hs;
   sd.b_ld = d.Is;
-  sd.b_rows = T;
   sd.b_div = 1;
   sd.y = y;
   sd.y_ld = d.H;
@@ -787,16 +783,15 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   if (e != cudaSuccess) return e;
   // routed down: Q2_K (or Q4_K) x bf16 h, y[token] += w * (W_down h)
   if (!(d.flags & MOE_FLAG_DETERMINISTIC))
-    return grouped_gemm(
-        routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, T * d.k, p.s.w, p.y, p.err), s,
-        num_sms);
+    return grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, p.s.w, p.y, p.err),
+                        s, num_sms);
   // deterministic: each pair's weighted output into its own slot row (one
   // addition onto zero per element), then every token's slots summed in
   // ascending slot order
   const int n = T * d.k;
   if ((e = cudaMemsetAsync(b.slots, 0, sizeof(float) * (size_t)n * d.H, s)) != cudaSuccess) return e;
-  e = grouped_gemm(
-      routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, 1, b.hperm, n, p.s.w, b.slots, p.err), s, num_sms);
+  e = grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, 1, b.hperm, p.s.w, b.slots, p.err), s,
+                   num_sms);
   if (e != cudaSuccess) return e;
   k_sum_slots<<<T, 256, 0, s>>>(d.H, d.k, b.slots, p.y);
   return cudaGetLastError();
@@ -939,7 +934,7 @@ cudaError_t ep_experts(const LayerDims &d, const LayerWeights &wt, bool q4k, con
   if ((e = permute(local, N, 1, d.E, offsets, perm, s)) != cudaSuccess) return e;
   e = grouped_gemm(routed_gateup_args(d, wt, q4k, d.E, offsets, perm, 1, x_recv, h, err), s, num_sms);
   if (e != cudaSuccess) return e;
-  return grouped_gemm(routed_down_args(d, wt, q4k, d.E, offsets, perm, 1, h, N, w_recv, out, err), s, num_sms);
+  return grouped_gemm(routed_down_args(d, wt, q4k, d.E, offsets, perm, 1, h, w_recv, out, err), s, num_sms);
 }
 
 size_t ep_combine_scratch_bytes(const LayerDims &d, int T) {
