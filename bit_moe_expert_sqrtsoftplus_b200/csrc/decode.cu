@@ -82,14 +82,8 @@ __device__ __forceinline__ double sqrtsoftplus(double z) { return sqrt(fmax(z, 0
 
 constexpr int kRouterThreads = 256;
 
-// Blocks [0, nlimb) make the int8 limbs of x, one token each (nlimb = T when
-// the expert kernel reads them from here, 0 when it makes its own); the
-// other blocks compute the router keys, kRouterEPB experts per block, one
-// warp per expert at a time.  With few blocks the expert kernel's CTAs
-// start on the other SMs while the router runs.
-constexpr int kRouterEPB = 16;
 template <int MAXT>
-__global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a, int nlimb) {
+__global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a) {
   pdl_launch_dependents();
   const LayerDims &d = a.d;
   const int T = a.T;
@@ -118,7 +112,7 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a, i
     }
   }
 
-  if ((int)blockIdx.x < nlimb) {
+  if ((int)blockIdx.x < T) {
     // ---- activation limbs for token t; every thread takes float4 words
     // tid, tid + 256, ... and loads a batch of them before using any
     const int t = blockIdx.x;
@@ -208,50 +202,78 @@ __global__ void __launch_bounds__(kRouterThreads) k1_prep_router(DecodeArgs a, i
   }
 
   if (d.mode != MOE_ROUTE_ROUTER) return;
-  // ---- router logits, scores and keys (fp64): warp w of router block b takes
-  // experts e = kRouterEPB * b + w, + 8, ...; every lane covers elements
-  // 8 * lane + 256 * i of the row, tokens in groups of MAXT
-  const int rb = (int)blockIdx.x - nlimb;
-  for (int e = kRouterEPB * rb + warp; e < min(d.E, kRouterEPB * (rb + 1)); e += NW) {
-    const uint16_t *wr = a.wt.Wr + (size_t)e * d.H;
-    for (int t0 = 0; t0 < T; t0 += MAXT) {
-      const int nt = min(MAXT, T - t0);
-      double acc[MAXT], ssq[MAXT];
+  // ---- router logits, scores and keys for experts e0, e0 + 1 (fp64)
+  const int e0 = 2 * ((int)blockIdx.x - T);
+  if (e0 >= d.E) return;
+  const bool two = e0 + 1 < d.E;
+  const uint16_t *w0 = a.wt.Wr + (size_t)e0 * d.H;
+  const uint16_t *w1 = a.wt.Wr + (size_t)(two ? e0 + 1 : e0) * d.H;
+  // tokens in groups of MAXT (the two weight rows are re-read from L1/L2)
+  for (int t0 = 0; t0 < T; t0 += MAXT) {
+    const int nt = min(MAXT, T - t0);
+    double acc0[MAXT], acc1[MAXT], ssq[MAXT];
 #pragma unroll
-      for (int t = 0; t < MAXT; ++t) acc[t] = ssq[t] = 0.0;
-#pragma unroll 4
-      for (int j = 8 * lane; j < d.H; j += 256) {
-        const uint4 hv = *reinterpret_cast<const uint4 *>(wr + j);
-        const uint16_t *hp = reinterpret_cast<const uint16_t *>(&hv);
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t) {
-          if (t < nt) {
-            const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)(t0 + t) * d.H + j);
-            const float4 x0 = xp[0], x1 = xp[1];
-            const float xe[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const double xd = (double)xe[i];
-              acc[t] = fma((double)half_bits_to_float(hp[i]), xd, acc[t]);
-              ssq[t] = fma(xd, xd, ssq[t]);
-            }
-          }
-        }
-      }
+    for (int t = 0; t < MAXT; ++t) acc0[t] = acc1[t] = ssq[t] = 0.0;
+    // every thread covers 8 consecutive elements per pass; all loads of a pass are independent
+    for (int j = tid * 8; j < d.H; j += kRouterThreads * 8) {
+      const uint4 hv0 = *reinterpret_cast<const uint4 *>(w0 + j);
+      const uint4 hv1 = *reinterpret_cast<const uint4 *>(w1 + j);
+      float4 xv[MAXT][2];
 #pragma unroll
       for (int t = 0; t < MAXT; ++t) {
         if (t < nt) {
-          double z = warp_sum_d(acc[t]);
-          const double s2 = warp_sum_d(ssq[t]);
-          if (lane == 0) {
-            if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) z *= 1.0 / sqrt(s2 / (double)d.H + (double)d.eps);
-            const double sc = sqrtsoftplus(z);
-            a.s.sc[(size_t)(t0 + t) * d.E + e] = sc;
-            a.s.z[(size_t)(t0 + t) * d.E + e] = sc + (double)a.wt.bias[e];
+          const float4 *xp = reinterpret_cast<const float4 *>(a.x + (size_t)(t0 + t) * d.H + j);
+          xv[t][0] = xp[0];
+          xv[t][1] = xp[1];
+        }
+      }
+      const uint16_t *p0 = reinterpret_cast<const uint16_t *>(&hv0);
+      const uint16_t *p1 = reinterpret_cast<const uint16_t *>(&hv1);
+#pragma unroll
+      for (int t = 0; t < MAXT; ++t) {
+        if (t < nt) {
+          const float xe[8] = {xv[t][0].x, xv[t][0].y, xv[t][0].z, xv[t][0].w,
+                               xv[t][1].x, xv[t][1].y, xv[t][1].z, xv[t][1].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const double xd = (double)xe[i];
+            acc0[t] = fma((double)half_bits_to_float(p0[i]), xd, acc0[t]);
+            acc1[t] = fma((double)half_bits_to_float(p1[i]), xd, acc1[t]);
+            ssq[t] = fma(xd, xd, ssq[t]);
           }
         }
       }
     }
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t) {
+      if (t < nt) {
+        const double v0 = warp_sum_d(acc0[t]);
+        const double v1 = warp_sum_d(acc1[t]);
+        const double v2 = warp_sum_d(ssq[t]);
+        if (lane == 0) {
+          red[warp][t] = v0;
+          red[warp][MAXT + t] = v1;
+          red[warp][2 * MAXT + t] = v2;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < 2 * nt) {
+      const int t = tid >> 1, which = tid & 1;
+      if (which == 0 || two) {
+        double z = 0.0, s2 = 0.0;
+        for (int w = 0; w < NW; ++w) {
+          z += red[w][which * MAXT + t];
+          s2 += red[w][2 * MAXT + t];
+        }
+        if (d.flags & MOE_FLAG_PRENORM_RESIDUAL) z *= 1.0 / sqrt(s2 / (double)d.H + (double)d.eps);
+        const int e = e0 + which;
+        const double sc = sqrtsoftplus(z);
+        a.s.sc[(size_t)(t0 + t) * d.E + e] = sc;
+        a.s.z[(size_t)(t0 + t) * d.E + e] = sc + (double)a.wt.bias[e];
+      }
+    }
+    __syncthreads();  // red is reused by the next group
   }
 }
 
@@ -1752,18 +1774,17 @@ cudaError_t launch_k2_tma(const DecodeArgs &a, cudaStream_t stream, int num_sms)
   return a.wt.tma ? launch_k2<MAXP, XSMEM, true>(a, stream, num_sms) : launch_k2<MAXP, XSMEM, false>(a, stream, num_sms);
 }
 
-cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream, bool limbs) {
-  const int nr = a.d.mode == MOE_ROUTE_ROUTER ? (a.d.E + kRouterEPB - 1) / kRouterEPB : 0;
-  const int nlimb = limbs ? a.T : 0;
-  const int grid = nlimb + nr > 0 ? nlimb + nr : 1;  // one block at least, for the counter resets
+cudaError_t launch_k1(const DecodeArgs &a, cudaStream_t stream) {
+  const int nr = a.d.mode == MOE_ROUTE_ROUTER ? (a.d.E + 1) / 2 : 0;
+  const int grid = a.T + nr;
   if (a.T <= 1)
-    k1_prep_router<1><<<grid, kRouterThreads, 0, stream>>>(a, nlimb);
+    k1_prep_router<1><<<grid, kRouterThreads, 0, stream>>>(a);
   else if (a.T <= 2)
-    k1_prep_router<2><<<grid, kRouterThreads, 0, stream>>>(a, nlimb);
+    k1_prep_router<2><<<grid, kRouterThreads, 0, stream>>>(a);
   else if (a.T <= 4)
-    k1_prep_router<4><<<grid, kRouterThreads, 0, stream>>>(a, nlimb);
+    k1_prep_router<4><<<grid, kRouterThreads, 0, stream>>>(a);
   else
-    k1_prep_router<8><<<grid, kRouterThreads, 0, stream>>>(a, nlimb);
+    k1_prep_router<8><<<grid, kRouterThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -1881,15 +1902,12 @@ void decode_carve(DecodeScratch &s, const LayerDims &d, int T, void *base) {
 }
 
 cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms) {
-  // the expert kernel makes the x limbs itself (in shared memory) for up to
-  // two tokens when they fit; otherwise it reads k1's
-  const bool xsmem = a.s.UW == 2 && a.T <= 2 && k2_smem_bytes(a.d, a.T, true) <= kSmemLimit;
-  cudaError_t e = launch_k1(a, stream, !xsmem);
+  cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
   // the variant whose unit width the scratch was carved for
   switch (a.s.UW) {
     case 2:
-      if (xsmem) return launch_k2_tma<1, true>(a, stream, num_sms);
+      if (a.T <= 2 && k2_smem_bytes(a.d, a.T, true) <= kSmemLimit) return launch_k2_tma<1, true>(a, stream, num_sms);
       return launch_k2_tma<1, false>(a, stream, num_sms);
     case 4:
       return launch_k2_tma<2, false>(a, stream, num_sms);
@@ -1901,7 +1919,7 @@ cudaError_t decode_forward(const DecodeArgs &a, cudaStream_t stream, int num_sms
 }
 
 cudaError_t decode_route(const DecodeArgs &a, int32_t *idx, float *w, cudaStream_t stream) {
-  cudaError_t e = launch_k1(a, stream, false);
+  cudaError_t e = launch_k1(a, stream);
   if (e != cudaSuccess) return e;
   k_route_only<<<(a.T + 7) / 8, 256, 0, stream>>>(a, idx, w);
   return cudaGetLastError();
