@@ -400,19 +400,24 @@ def run_stack(args, world, rank):
 
     s = synth.workload(args.workload)
     T = s.tokens
-    layers, scratch = [], None
+    cfgs = []
     for l in range(s.layers):
         router = l >= s.hash_layers
         sl = s.layer_shape(l)
-        W = synth.device_layer(0, l, sl, router=router, q4k=sl.q4k)
-        cfg = moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
-                              routed_scaling=s.routed_scaling, rms_eps=1e-6,
-                              mode=moe.MOE_ROUTE_ROUTER if router else moe.MOE_ROUTE_HASH,
-                              flags=moe.MOE_FLAG_PRENORM_RESIDUAL,
-                              routed_format=moe.MOE_ROUTED_Q4K if sl.q4k else moe.MOE_ROUTED_Q2)
-        L = moe.Layer(cfg, W, max_tokens=T, scratch=scratch)
-        scratch = L.scratch
-        layers.append(L)
+        cfgs.append(moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
+                                    routed_scaling=s.routed_scaling, rms_eps=1e-6,
+                                    mode=moe.MOE_ROUTE_ROUTER if router else moe.MOE_ROUTE_HASH,
+                                    flags=moe.MOE_FLAG_PRENORM_RESIDUAL,
+                                    routed_format=moe.MOE_ROUTED_Q4K if sl.q4k else moe.MOE_ROUTED_Q2))
+    # one scratch buffer serves every layer (they run one after another on
+    # one stream): the largest any layer asks for (Q4_K layers ask for more)
+    sbytes = max(moe.moe_workspace_size(c, T)[1] for c in cfgs)
+    scratch = torch.empty(max(sbytes, 16), dtype=torch.uint8, device="cuda")
+    layers = []
+    for l, cfg in enumerate(cfgs):
+        sl = s.layer_shape(l)
+        W = synth.device_layer(0, l, sl, router=l >= s.hash_layers, q4k=sl.q4k)
+        layers.append(moe.Layer(cfg, W, max_tokens=T, scratch=scratch))
     x0 = torch.from_numpy(synth.activations(7 + rank, T, s.hidden, stream=4242)).cuda()
     tok = torch.from_numpy(synth.token_ids(7 + rank, T, s.vocab, stream=4242)).cuda()
     x = x0.clone()

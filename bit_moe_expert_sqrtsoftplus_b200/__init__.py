@@ -307,7 +307,10 @@ class Layer:
         self.cfg = cfg
         self.weights = weights
         pbytes, sbytes = moe_workspace_size(cfg, max_tokens)
-        self.persist = torch.empty(max(pbytes, 16), dtype=torch.uint8, device=device)
+        self.persist = torch.zeros(max(pbytes, 16), dtype=torch.uint8, device=device)
+        if scratch is not None and _nbytes(scratch) < sbytes:
+            raise MoeError(MOE_ERR_WORKSPACE_TOO_SMALL,
+                           f"shared scratch has {_nbytes(scratch)} bytes, this layer needs {sbytes}")
         self.scratch = scratch if scratch is not None else torch.empty(max(sbytes, 16), dtype=torch.uint8,
                                                                        device=device)
         self.scratch_bytes = sbytes

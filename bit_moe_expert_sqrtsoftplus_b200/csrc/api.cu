@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -11,12 +12,15 @@
 #include <string>
 
 #include "../../include/moe.h"
+#include "gemm.cuh"
 #include "layer.cuh"
 #include "prefill.cuh"
 #include "q4k.cuh"
 #include "quant.cuh"
 
 static_assert(MOE_SMALL_T_MAX == moe::kDecodeMaxT, "header and kernels disagree on the small-T limit");
+
+constexpr int kGemmMaps = 3;  // tensor maps of gate, up and down for the batched path
 
 struct moe_handle {
   moe_config cfg;
@@ -29,6 +33,7 @@ struct moe_handle {
   int device;
   cudaEvent_t ev_begin, ev_end;  // optional timing of the dominant kernel
   moe::NextLayerPrefetch next;   // the next layer's first-read weights (stack decode)
+  moe::TensorMap gemm_tm_host[kGemmMaps];  // host copies of wt.gemm_tm's maps
 };
 
 namespace {
@@ -55,7 +60,17 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 constexpr size_t kPersistHeader = 256;
 
 size_t persist_bytes_for(const moe_config &c) {
-  return kPersistHeader + sizeof(float) * (size_t)(c.n_experts > 0 ? c.n_experts : 0) + 256;
+  // header, row norms, then (64-byte aligned) the batched path's tensor maps
+  return kPersistHeader + sizeof(float) * (size_t)(c.n_experts > 0 ? c.n_experts : 0) + 64 +
+         kGemmMaps * sizeof(moe::TensorMap) + 256;
+}
+
+// MOE_GEMM_TMA=0 in the environment turns the TMA staging of the batched
+// path's packed weight tiles off for handles created afterwards (the
+// producers then load the packed bytes themselves; results are identical).
+bool gemm_tma_wanted() {
+  const char *v = getenv("MOE_GEMM_TMA");
+  return !(v && v[0] == '0' && v[1] == 0);
 }
 
 moe_status check_config(const moe_config *c) {
@@ -240,6 +255,7 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   if (cfg->routed_format == MOE_ROUTED_Q2 && !no_routed && !experts_only) moe::build_chunk_tensor_maps(h->wt, h->d);
   h->err = static_cast<int *>(persist);
   h->row_norms = reinterpret_cast<float *>(static_cast<uint8_t *>(persist) + kPersistHeader);
+  h->wt.gemm_tm = nullptr;
   h->num_sms = sms;
   h->device = dev;
   h->ev_begin = nullptr;
@@ -250,6 +266,23 @@ moe_status moe_init(const moe_config *cfg, const moe_weights *w, void *persist, 
   if (e != cudaSuccess) {
     delete h;
     return cuda_fail(e, "cudaMemsetAsync(persist)");
+  }
+  if (cfg->routed_format == MOE_ROUTED_Q2 && !no_routed && gemm_tma_wanted()) {
+    // tensor maps of the routed matrices, all experts' rows stacked
+    const size_t rbI = (size_t)(cfg->hidden / 256) * 66, rbD = (size_t)(cfg->inter / 256) * 84;
+    const size_t E = (size_t)cfg->n_experts;
+    const uintptr_t at = reinterpret_cast<uintptr_t>(h->row_norms + E);
+    void *maps = reinterpret_cast<void *>((at + 63) & ~uintptr_t(63));
+    if (moe::gemm_tensor_map(&h->gemm_tm_host[0], h->wt.gate, rbI, E * cfg->inter, moe::kFmtIQ2) &&
+        moe::gemm_tensor_map(&h->gemm_tm_host[1], h->wt.up, rbI, E * cfg->inter, moe::kFmtIQ2) &&
+        moe::gemm_tensor_map(&h->gemm_tm_host[2], h->wt.down, rbD, E * cfg->hidden, moe::kFmtQ2K)) {
+      e = cudaMemcpyAsync(maps, h->gemm_tm_host, kGemmMaps * sizeof(moe::TensorMap), cudaMemcpyHostToDevice, s);
+      if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "copying tensor maps");
+      }
+      h->wt.gemm_tm = maps;
+    }
   }
   if (!experts_only) e = moe::prefill_init(h->d, h->wt, h->row_norms, h->err, s);
   if (e != cudaSuccess) {

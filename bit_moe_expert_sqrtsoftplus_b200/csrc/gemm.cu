@@ -1,7 +1,7 @@
 // gemm.cu -- persistent, warp-specialised grouped GEMM on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory).
 //
-// One CTA per SM, 25 warps:
+// One CTA per SM, 25 warps (26 with TMA staging):
 //   warps 0-7   epilogue: tcgen05.ld of the 128-lane accumulator, SwiGLU /
 //               scatter-add / store
 //   warps 8-23  producers: dequantise the 128 x 64 weight tile(s) of a K step
@@ -9,19 +9,26 @@
 //               K-major operand layout, and gather the N x 64 activation tile
 //               with cp.async
 //   warp 24     allocates tensor memory and issues tcgen05.mma (one thread)
+//   warp 25     TMA staging only: issues the tensor copies of the packed
+//               weight tiles (one thread)
 // Shared memory holds a ring of A stages (dequantised weight tiles, written
-// in the step that hands them over) and a ring of B stages (token rows,
-// loaded two K steps ahead); mbarriers carry full/empty hand-offs between
-// producers and the MMA thread and
-// full/empty hand-offs of the accumulator between the MMA thread and the
-// epilogue.  Every wait is bounded: on expiry the CTA records
-// MOE_ERR_TIMEOUT in the device error word, every role leaves its loop, the
-// MMA thread drains its outstanding tensor-core work and tensor memory is
-// freed before the kernel returns.
+// in the step that hands them over), a ring of B stages (token rows,
+// loaded two K steps ahead) and, with TMA staging, a ring of packed stages
+// (one 256-value block of each of the tile's 128 weight rows, i.e. four K
+// steps, brought by one 2-D tensor copy per matrix as soon as the stage is
+// free); without it each producer keeps the packed bytes of its next K steps
+// in a ring of registers.  mbarriers carry the full/empty hand-offs of every
+// ring and of the accumulator between the MMA thread and the epilogue.
+// Every wait is bounded: on expiry the CTA records MOE_ERR_TIMEOUT in the
+// device error word, every role leaves its loop, the MMA thread drains its
+// outstanding tensor-core work, the copy thread waits for its copies in
+// flight, and tensor memory is freed before the kernel returns.
 //
 // Tiles: M = 128 weight rows, N = up to 256 columns (tokens) of one group, K
 // stepped 64 at a time (four K=16 MMAs per step).  A gate/up pair shares the
-// B tile and uses two accumulators (columns 0-255 and 256-511).
+// B tile and uses two accumulators.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -37,7 +44,8 @@ namespace {
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the column groups
 constexpr int kProdWarps = 16;
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;  // 24
-constexpr int kGemmThreads = (kMmaWarp + 1) * 32;  // 800
+constexpr int kTmaWarp = kMmaWarp + 1;             // 25: packed-tile copies (TMA staging only)
+__host__ __device__ constexpr int gemm_threads(bool tma) { return (kMmaWarp + (tma ? 2 : 1)) * 32; }  // 832 / 800
 constexpr int kProd = kProdWarps * 32;             // 512 producer threads
 // Codebook and sign tables: an entry is read as 16 bytes by 8 lanes per
 // shared-memory wavefront; with 8 replicas, lane l reads replica l % 8, so
@@ -63,7 +71,12 @@ __host__ __device__ constexpr int nacc_of(int fmt, bool paired) { return (paired
 #ifndef MOE_GEMM_SA_PAIRED
 #define MOE_GEMM_SA_PAIRED 2
 #endif
-__host__ __device__ constexpr int sa_of(bool paired) { return paired ? MOE_GEMM_SA_PAIRED : 4; }
+#ifndef MOE_GEMM_SA_Q2K
+#define MOE_GEMM_SA_Q2K 4
+#endif
+__host__ __device__ constexpr int sa_of(int fmt, bool paired) {
+  return paired ? MOE_GEMM_SA_PAIRED : fmt == kFmtQ2K ? MOE_GEMM_SA_Q2K : 4;
+}
 
 // stages of the B (token rows) ring; a B tile is loaded kSB - 2 K steps
 // ahead of its use (the stage it reuses was read by the MMA two steps back)
@@ -75,8 +88,36 @@ __host__ __device__ constexpr int sb_of(int fmt, bool paired) {
   return bn_of(fmt, paired) == 128 ? MOE_GEMM_BSTAGES_NARROW : 4;
 }
 
+// TMA staging of packed A tiles: a unit is one 256-value block (four K
+// steps) of each of the tile's 128 rows.  A block starts 2 (IQ2_XXS, 66-byte
+// blocks) or 4 (Q2_K, 84-byte blocks) bytes times its index past a 16-byte
+// boundary; a copy's first byte must sit on one, so the box starts at the
+// boundary below the block and is wide enough for the largest offset
+// (14 + 66 <= 80, 12 + 84 <= 96).
+__host__ __device__ constexpr int blk_bytes_of(int fmt) { return fmt == kFmtIQ2 ? 66 : 84; }
+__host__ __device__ constexpr int pbox_of(int fmt) { return fmt == kFmtIQ2 ? 80 : 96; }
+__host__ __device__ constexpr int pmat_of(int fmt) { return pbox_of(fmt) * BM; }
+__host__ __device__ constexpr int pstage_of(int fmt, bool paired) { return (paired ? 2 : 1) * pmat_of(fmt); }
+// packed stages: with s stages the copy of block b + s - 1 is issued when
+// block b starts (the pair's two 10 KB boxes leave room for two stages only)
+#ifndef MOE_GEMM_SP_Q2K
+#define MOE_GEMM_SP_Q2K 2
+#endif
+constexpr int kSPMax = 4;
+__host__ __device__ constexpr int sp_of(bool paired) { return paired ? 2 : MOE_GEMM_SP_Q2K; }
+// Q2_K (down) tiles by TMA as well (1) or by the producers' own loads (0).
+// Measured on B200 (prefill, 4096 tokens): the IQ2_XXS gate/up GEMM takes
+// 2.47 ms with TMA staging against 2.86 ms without; the Q2_K down GEMM 2.30
+// ms against 2.08 ms (its 16-value items leave little decode to hide the
+// staged reads behind, and the 96-byte staged rows put two of every eight
+// rows of a warp on the same banks), whatever the depth of the rings.
+#ifndef MOE_GEMM_TMA_Q2K
+#define MOE_GEMM_TMA_Q2K 0
+#endif
+
 struct alignas(8) GemmCtl {
   uint64_t full[kSBMax], emptyA[4], emptyB[kSBMax], acc_full[2], acc_empty[2], drain;
+  uint64_t pfull[kSPMax], pempty[kSPMax];
   uint32_t tmem_base;
   int abort;
   long long wait;  // bound of the role hand-off waits (cycles)
@@ -162,6 +203,18 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+// 2-D tensor copy global -> this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // K-major operand tile, 128-byte rows, 128-byte swizzle, 8-row groups 1024 B apart.
@@ -387,6 +440,31 @@ __device__ __forceinline__ void decode(const Raw<kFmtQ2K> &r, uint8_t *tile, int
   sts128(swz(tile, row, chunk + 1), o[4], o[5], o[6], o[7]);
 }
 
+// The same items read from a staged block (TMA path): `bp` is this row's
+// block in the packed stage.  The block's offset in the staged row is that of
+// the global block from a 16-byte boundary, so the alignment tests are the
+// same for every row of a unit.
+__device__ __forceinline__ uint32_t lds16(const uint8_t *p) { return *reinterpret_cast<const uint16_t *>(p); }
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+__device__ __forceinline__ void fetch_staged(Raw<kFmtIQ2> &r, const uint8_t *bp, int ks, int item) {
+  const uint8_t *gp = bp + 2 + 8 * (2 * (ks & 3) + item);
+  r.d16 = lds16(bp);
+  if ((smem_u32(gp) & 3u) == 0) {
+    r.idx4 = lds32(gp);
+    r.S = lds32(gp + 4);
+  } else {
+    r.idx4 = lds16(gp) | (lds16(gp + 2) << 16);
+    r.S = lds16(gp + 4) | (lds16(gp + 6) << 16);
+  }
+}
+__device__ __forceinline__ void fetch_staged(Raw<kFmtQ2K> &r, const uint8_t *bp, int ks, int item) {
+  const int qq = ks & 3, hf = qq >> 1, sh = 2 * (qq & 1) + (item >> 1), sub = item & 1;
+  r.dd = lds32(bp + 80);
+  r.sb = bp[8 * hf + 2 * sh + sub];
+  const uint8_t *qp = bp + 16 + 32 * hf + 16 * sub;  // 4-byte aligned (blocks start 0, 4, 8 or 12 bytes in)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.q[i] = lds32(qp + 4 * i);
+}
 // Q8_0: 32-element block (kel/32) of the row.
 __device__ __forceinline__ void fetch(Raw<kFmtQ80> &r, const uint8_t *rowp, int ks, int item) {
   const int kel = ks * BK + 32 * item;
@@ -497,14 +575,15 @@ __device__ __forceinline__ void decode(const Raw<kFmtQ80> &r, uint8_t *tile, int
 
 // ---------------------------------------------------------------- kernel
 
-template <int FMT, bool PAIRED>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
+template <int FMT, bool PAIRED, bool TMA>
+__global__ void __launch_bounds__(gemm_threads(TMA), 1) k_grouped_gemm(GemmArgs a) {
+  static_assert(!TMA || FMT == kFmtIQ2 || FMT == kFmtQ2K, "TMA staging of IQ2_XXS and Q2_K tiles only");
   // A (dequantised weights) and B (gathered token rows) have rings of their
   // own: a B tile is loaded kBAhead steps before its use, an A tile is
   // written in the step that hands it to the MMA; step `it` uses A stage
   // it % SA and B stage it % kSB, and its full barrier is full[it % kSB]
   constexpr int NA = PAIRED ? 2 : 1;
-  constexpr int SA = sa_of(PAIRED);
+  constexpr int SA = sa_of(FMT, PAIRED);
   constexpr int BN = bn_of(FMT, PAIRED);
   constexpr int kBTile = btile_of(FMT, PAIRED);
   constexpr int kSB = sb_of(FMT, PAIRED);
@@ -520,9 +599,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
   constexpr int kAhead = ahead_of(FMT);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kPMat = pmat_of(FMT), kPStage = TMA ? pstage_of(FMT, PAIRED) : 0;
+  constexpr int kSP = sp_of(PAIRED);
+  static_assert(kSP <= kSPMax, "packed ring");
   uint8_t *stagesA = smem;
   uint8_t *stagesB = stagesA + SA * ASTAGE;
-  uint8_t *gridh = stagesB + kSB * kBTile;                // 256 x kGridRep x 16 B: codebook as f16
+  uint8_t *stagesP = stagesB + kSB * kBTile;              // packed stages (TMA staging)
+  uint8_t *gridh = stagesP + kSP * kPStage;               // 256 x kGridRep x 16 B: codebook as f16
   uint8_t *signm = gridh + (kTables ? 4096 * kGridRep : 0);  // 128 x kSignRep x 16 B: f16 sign masks
   GemmCtl &ctl = *reinterpret_cast<GemmCtl *>(signm + (kTables ? 2048 * kSignRep : 0));
 
@@ -537,6 +620,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       mbar_init(&ctl.emptyB[s], 1);
     }
     for (int s = 0; s < SA; ++s) mbar_init(&ctl.emptyA[s], 1);
+    for (int s = 0; s < kSP; ++s) {
+      mbar_init(&ctl.pfull[s], 1);       // the issuing thread's expect_tx arrival (+ the copies' bytes)
+      mbar_init(&ctl.pempty[s], kProd);  // every producer, after its last read of the unit
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl.acc_full[b], 1);
       mbar_init(&ctl.acc_empty[b], kEpiWarps * 32);
@@ -592,7 +679,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
     const uint8_t *gridh_l = gridh + 16 * (lane % kGridRep);
     const uint8_t *signm_l = signm + 16 * (lane % kSignRep);
     constexpr int kBRows = BN / 64;  // B rows per producer thread and step
-    uint32_t it = 0;
+    uint32_t it = 0, pu = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile tl = tile_at<BN>(ctl, t, m_tiles);
       // B rows this thread copies: rows (p >> 3) + 64 i, chunk p & 7
@@ -614,17 +701,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       const int row = FMT == kFmtQ2K ? (p >> 2) : ((p >> 1) & 127);
       const int item = FMT == kFmtQ2K ? (p & 3) : (p & 1);
       const bool has_a = PAIRED || FMT == kFmtQ2K || p < 256;
-      const uint8_t *arow = (mat ? a.A1 : a.A0) + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
       const int dsel = (FMT == kFmtQ80 || FMT == kFmtQ4K) ? a.bf16 : 0;
-      // packed bytes of K steps ks .. ks + kAhead - 1 are in flight in a ring of
-      // registers; slots are compile-time indices of the unrolled loop below, so
-      // no register copy ever waits on a load
-      Raw<FMT> R[kAhead + 1];
-      if (has_a) {
-#pragma unroll
-        for (int j = 0; j < kAhead; ++j)
-          if (j < ksteps) fetch(R[j], arow, j, item);
-      }
       // B tile of tile-local step ks into B stage `sb` (one cp.async group)
       auto issue_b = [&](int ks, int sb) {
         uint8_t *Bs = stagesB + sb * kBTile;
@@ -649,6 +726,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 #pragma unroll
       for (int q = 0; q < kBAhead; ++q)
         if (ok) ok = load_b(q, it + q);
+      if constexpr (TMA) {
+        // packed unit (block) ks / 4 of this tile is global unit pu; its
+        // stage holds each row's block at the block's offset from a 16-byte
+        // boundary.  The words of step ks + 1 are read from the stage while
+        // step ks is handed over.
+        auto staged = [&](int ks) {
+          const int off = ((ks >> 2) * blk_bytes_of(FMT)) & 15;
+          return stagesP + (pu % kSP) * kPStage + mat * kPMat + row * pbox_of(FMT) + off;
+        };
+        Raw<FMT> rn;
+        if (ok && !mbar_wait(&ctl.pfull[pu % kSP], (pu / kSP) & 1u, ctl, a.err)) ok = false;
+        if (ok) fetch_staged(rn, staged(0), 0, item);
+        for (int ks = 0; ok && ks < ksteps; ++ks) {
+          const Raw<FMT> r = rn;
+          if (!load_b(ks + kBAhead, it + kBAhead) ||
+              !mbar_wait(&ctl.emptyA[it % SA], ((it / SA) & 1u) ^ 1u, ctl, a.err)) {
+            ok = false;
+            break;
+          }
+          decode(r, stagesA + (it % SA) * ASTAGE + mat * kATile, row, item, FMT == kFmtQ2K ? ks : dsel, gridh_l,
+                 signm_l);
+          if ((ks & 3) == 3) {  // every read of this unit is done
+            mbar_arrive(&ctl.pempty[pu % kSP]);
+            ++pu;
+          }
+          if (ks + 1 < ksteps) {
+            if (((ks + 1) & 3) == 0 && !mbar_wait(&ctl.pfull[pu % kSP], (pu / kSP) & 1u, ctl, a.err)) {
+              ok = false;
+              break;
+            }
+            fetch_staged(rn, staged(ks + 1), ks + 1, item);
+          }
+          cp_async_wait<kBAhead>();  // this step's B tile has landed
+          fence_proxy_async();
+          mbar_arrive(&ctl.full[it % kSB]);
+          ++it;
+        }
+        if (!ok) break;
+        continue;
+      }
+      const uint8_t *arow = (mat ? a.A1 : a.A0) + a.a_group_stride * tl.g + a.a_row_bytes * (size_t)(tl.m0 + row);
+      // packed bytes of K steps ks .. ks + kAhead - 1 are in flight in a ring of
+      // registers; slots are compile-time indices of the unrolled loop below, so
+      // no register copy ever waits on a load
+      Raw<FMT> R[kAhead + 1];
+      if (has_a) {
+#pragma unroll
+        for (int j = 0; j < kAhead; ++j)
+          if (j < ksteps) fetch(R[j], arow, j, item);
+      }
       for (int ks0 = 0; ok && ks0 < ksteps; ks0 += kAhead + 1) {
 #pragma unroll
         for (int j = 0; j <= kAhead; ++j) {
@@ -723,6 +850,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
       }
     }
     __syncwarp();
+  } else if (TMA && warp == kTmaWarp) {
+    // =================================================== packed-tile copies
+    // Units in the producers' order (this CTA's tiles, K blocks within a
+    // tile): unit u goes to packed stage u % kSP as soon as every producer
+    // has read unit u - kSP from it.
+    if (lane == 0) {
+      // the maps were written to global memory by a copy from the host
+      // (possibly over older maps at the same address): order that write
+      // before the tensor copies read them
+      asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(a.tmA) : "memory");
+      if (PAIRED)
+        asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(
+                         static_cast<const uint8_t *>(a.tmA) + 128)
+                     : "memory");
+      const int kunits = ksteps / 4;
+      uint32_t pu = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const Tile tn = tile_at<BN>(ctl, t, m_tiles);
+        const int y0 = tn.g * a.M + tn.m0;
+        for (int pk = 0; pk < kunits; ++pk, ++pu) {
+          const uint32_t ps = pu % kSP;
+          if (!mbar_wait(&ctl.pempty[ps], ((pu / kSP) & 1u) ^ 1u, ctl, a.err)) {
+            ok = false;
+            break;
+          }
+          const int x0 = (pk * blk_bytes_of(FMT)) & ~15;  // 16-byte aligned start of the box
+          uint8_t *dst = stagesP + ps * kPStage;
+          mbar_arrive_tx(&ctl.pfull[ps], (uint32_t)kPStage);
+          tma_load_2d(dst, a.tmA, x0, y0, &ctl.pfull[ps]);
+          if (PAIRED) tma_load_2d(dst + kPMat, static_cast<const uint8_t *>(a.tmA) + 128, x0, y0, &ctl.pfull[ps]);
+        }
+      }
+      // every copy issued has landed before the CTA exits
+      for (uint32_t q = pu > kSP ? pu - kSP : 0; q < pu; ++q) {  // the last unit of each stage
+        const long long t1 = clock64();
+        while (!mbar_try(&ctl.pfull[q % kSP], (q / kSP) & 1u)) {
+          if (clock64() - t1 > kDefaultWaitCycles) {
+            set_error(a.err, kErrTimeout);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
   } else {
     // =================================================== epilogue
     // warp w reads TMEM lanes 32 (w % 4) .. + 31 (the quadrant it may access)
@@ -786,33 +958,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(GemmArgs a) {
 
 }  // namespace
 
-size_t grouped_gemm_smem(int fmt, int paired) {
+size_t grouped_gemm_smem(int fmt, int paired, int tma) {
   const int na = paired ? 2 : 1;
-  const int sa = sa_of(paired != 0);
+  const int sa = sa_of(fmt, paired != 0);
   const size_t tables = fmt == kFmtIQ2 ? 4096 * kGridRep + 2048 * kSignRep : 0;
-  return 1024 + (size_t)sa * na * kATile + (size_t)sb_of(fmt, paired != 0) * btile_of(fmt, paired != 0) + tables +
-         sizeof(GemmCtl);
+  const size_t packed = tma ? (size_t)sp_of(paired != 0) * pstage_of(fmt, paired != 0) : 0;
+  return 1024 + (size_t)sa * na * kATile + (size_t)sb_of(fmt, paired != 0) * btile_of(fmt, paired != 0) + packed +
+         tables + sizeof(GemmCtl);
 }
 
-template <int FMT, bool PAIRED>
+template <int FMT, bool PAIRED, bool TMA>
 static cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   static SmemOptIn opt;
-  const size_t smem = grouped_gemm_smem(FMT, PAIRED);
-  cudaError_t e = opt_in_smem(k_grouped_gemm<FMT, PAIRED>, smem, opt);
+  const size_t smem = grouped_gemm_smem(FMT, PAIRED, TMA);
+  cudaError_t e = opt_in_smem(k_grouped_gemm<FMT, PAIRED, TMA>, smem, opt);
   if (e != cudaSuccess) return e;
-  k_grouped_gemm<FMT, PAIRED><<<num_sms, kGemmThreads, smem, s>>>(a);
+  k_grouped_gemm<FMT, PAIRED, TMA><<<num_sms, gemm_threads(TMA), smem, s>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   const bool paired = a.A1 != nullptr;
-  if (a.fmt == kFmtIQ2 && paired) return launch_gemm<kFmtIQ2, true>(a, s, num_sms);
-  if (a.fmt == kFmtQ80 && paired) return launch_gemm<kFmtQ80, true>(a, s, num_sms);
-  if (a.fmt == kFmtQ80 && !paired) return launch_gemm<kFmtQ80, false>(a, s, num_sms);
-  if (a.fmt == kFmtQ2K && !paired) return launch_gemm<kFmtQ2K, false>(a, s, num_sms);
-  if (a.fmt == kFmtQ4K && paired) return launch_gemm<kFmtQ4K, true>(a, s, num_sms);
-  if (a.fmt == kFmtQ4K && !paired) return launch_gemm<kFmtQ4K, false>(a, s, num_sms);
+  // TMA staging needs the groups' matrices back to back (row g * M + m of
+  // the tensor map is row m of group g) and K a whole number of blocks
+  const bool tma = a.tmA != nullptr && a.a_group_stride == (size_t)a.M * a.a_row_bytes && a.K % 256 == 0;
+  if (a.fmt == kFmtIQ2 && paired)
+    return tma ? launch_gemm<kFmtIQ2, true, true>(a, s, num_sms) : launch_gemm<kFmtIQ2, true, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ2K && !paired)
+    return tma && MOE_GEMM_TMA_Q2K ? launch_gemm<kFmtQ2K, false, true>(a, s, num_sms)
+                                   : launch_gemm<kFmtQ2K, false, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ80 && paired) return launch_gemm<kFmtQ80, true, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ80 && !paired) return launch_gemm<kFmtQ80, false, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ4K && paired) return launch_gemm<kFmtQ4K, true, false>(a, s, num_sms);
+  if (a.fmt == kFmtQ4K && !paired) return launch_gemm<kFmtQ4K, false, false>(a, s, num_sms);
   return cudaErrorInvalidValue;
+}
+
+bool gemm_tensor_map(void *map, const void *base, size_t row_bytes, size_t rows, int fmt) {
+  if (fmt != kFmtIQ2 && fmt != kFmtQ2K) return false;
+  const int box = pbox_of(fmt);
+  if (!base || (reinterpret_cast<uintptr_t>(base) & 15u) || row_bytes % 16 || row_bytes < (size_t)box || rows == 0 ||
+      rows > 0xFFFFFFFFull)
+    return false;
+  PFN_cuTensorMapEncodeTiled encode = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&encode), cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !encode)
+    return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t boxd[2] = {(cuuint32_t)box, (cuuint32_t)BM};
+  const cuuint32_t es[2] = {1, 1};
+  return encode(reinterpret_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace moe

@@ -46,9 +46,21 @@ struct GemmArgs {
   int k;
   int *err;
   long long wait_cycles;  // bound of the waits between the kernel's roles (0: the default)
+  // TMA staging of the packed A tiles (IQ2_XXS pairs and Q2_K only): device
+  // address of the tensor maps built by gemm_tensor_map, A0's then (paired)
+  // A1's, 128 bytes each; nullptr: producers load the packed bytes themselves
+  const void *tmA;
 };
 
 cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms);
-size_t grouped_gemm_smem(int fmt, int paired);
+size_t grouped_gemm_smem(int fmt, int paired, int tma);
+
+// Tensor map (128 bytes, written to `map`) of a packed weight array of `rows`
+// rows of `row_bytes` bytes in `fmt` (kFmtIQ2 or kFmtQ2K) for the TMA staging
+// of the grouped GEMM's A tiles: one copy brings one 256-value block of 128
+// consecutive rows.  False when the shape or the driver does not allow it
+// (rows not a multiple of 16 bytes, a misaligned base, no encoder entry
+// point); the GEMM then runs without TMA staging.
+bool gemm_tensor_map(void *map, const void *base, size_t row_bytes, size_t rows, int fmt);
 
 }  // namespace moe

@@ -43,6 +43,10 @@ struct LayerWeights {
   const uint8_t *gate, *up, *down, *sh_gate, *sh_up, *sh_down, *grid;
   int tma;  // 1 when tm[] is valid and every chunk start keeps the decoders' alignment
   TensorMap tm[kNumTm];
+  // device copies of the batched path's tensor maps of gate, up and down
+  // (128 bytes each, 64-byte aligned) for the TMA staging of its packed
+  // weight tiles; nullptr: that path loads the packed bytes without TMA
+  const void *gemm_tm;
 };
 
 // Builds wt.tm[] and sets wt.tma (0 when a shape does not allow TMA chunk

@@ -674,6 +674,7 @@ GemmArgs routed_gateup_args(const LayerDims &d, const LayerWeights &wt, bool q4k
   g.h_bf16 = 1;
   g.err = err;
   g.wait_cycles = d.wait_cycles;
+  g.tmA = q4k ? nullptr : wt.gemm_tm;  // gate's map, then up's
   return g;
 }
 
@@ -704,6 +705,7 @@ GemmArgs routed_down_args(const LayerDims &d, const LayerWeights &wt, bool q4k, 
   rd.k = k;
   rd.err = err;
   rd.wait_cycles = d.wait_cycles;
+  rd.tmA = q4k || !wt.gemm_tm ? nullptr : static_cast<const uint8_t *>(wt.gemm_tm) + 2 * sizeof(TensorMap);
   return rd;
 }
 

@@ -122,3 +122,46 @@ def test_deterministic_flag_repeats_bitwise(moe, name, T):
         La.poll()
     rel, mx = harness.errors(y1, yref)
     assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+def _tma_maps_written(L, s):
+    """Whether the handle holds the batched path's tensor maps: they sit in
+    the persist buffer after the 256-byte header and the E router-row norms,
+    at the next 64-byte boundary (three 128-byte maps)."""
+    base = L.persist.data_ptr()
+    off = ((base + 256 + 4 * s.n_experts + 63) & ~63) - base
+    return bool(L.persist[off:off + 384].any().item())
+
+
+@pytest.mark.parametrize("flags", ["det", "atomic"])
+def test_tma_staged_tiles_match_plain_loads(moe, monkeypatch, flags):
+    """TMA staging of the packed IQ2_XXS / Q2_K tiles (rows of 528 and 336
+    bytes: a 16-byte multiple, so the tensor maps exist) against producers
+    that load the packed bytes themselves (MOE_GEMM_TMA=0 at init): the same
+    decoded tiles and MMA order, so with the deterministic combine the outputs
+    are bitwise equal, and without it equal up to the order of the atomic
+    adds; both agree with the oracle.  16 experts, 300 tokens: several tiles
+    per expert, ragged last tiles, 8 blocks per gate/up row and 4 per down row
+    (every block offset from a 16-byte boundary occurs)."""
+    s = synth.LayerShape(2048, 1024, 512, 16, 2, 300, vocab=1024)
+    T = s.tokens
+    W = harness.device_layer(s, 8, 2)
+    x_np = synth.activations(8, T, s.hidden, stream=2)
+    x = torch.from_numpy(x_np).cuda()
+    fl = moe.MOE_FLAG_DETERMINISTIC if flags == "det" else 0
+    Lt = moe.Layer(harness.config_for(s, flags=fl), W, max_tokens=T)
+    monkeypatch.setenv("MOE_GEMM_TMA", "0")
+    Lp = moe.Layer(harness.config_for(s, flags=fl), W, max_tokens=T)
+    monkeypatch.delenv("MOE_GEMM_TMA")
+    assert _tma_maps_written(Lt, s)
+    yt = Lt.forward(x).cpu().numpy()
+    yp = Lp.forward(x).cpu().numpy()
+    Lt.poll()
+    Lp.poll()
+    if flags == "det":
+        assert np.array_equal(yt.view(np.uint32), yp.view(np.uint32))
+    else:
+        np.testing.assert_allclose(yt, yp, rtol=1e-5, atol=1e-5 * float(np.abs(yp).max()))
+    _, _, yref, _ = harness.oracle_layer_dense(s, 8, 2, x_np)
+    rel, mx = harness.errors(yt, yref)
+    assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
