@@ -294,10 +294,6 @@ __device__ __forceinline__ uint8_t *swz(uint8_t *tile, int row, int chunk) {
 __device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 bits2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-#ifndef MOE_GEMM_IQ2_FOLD
-#define MOE_GEMM_IQ2_FOLD 0
-#endif
-
 // ---------------------------------------------------------------- tile map
 
 struct Tile {
@@ -373,29 +369,17 @@ __device__ __forceinline__ void decode(const Raw<kFmtIQ2> &r, uint8_t *tile, int
                                        const uint8_t *gridh, const uint8_t *signm) {
   const __half2 f2 = __half2half2(__int2half_rn(2 * (int)(r.S >> 28) + 1));
   const __half2 d2 = __half2half2(__hmul(__ushort_as_half((unsigned short)r.d16), __float2half(0.125f)));
-#if MOE_GEMM_IQ2_FOLD
-  // one factor (2s+1) * d/8 per group, rounded to f16 once: one multiply per
-  // value pair instead of two, at one more f16 rounding of each weight
-  const __half2 fd2 = __hmul2(f2, d2);
-#endif
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t ix = (r.idx4 >> (8 * j)) & 255u;
     const uint32_t m7 = (r.S >> (7 * j)) & 127u;
     const uint4 g = *reinterpret_cast<const uint4 *>(gridh + ix * (16u * kGridRep));
     const uint4 sm = *reinterpret_cast<const uint4 *>(signm + m7 * (16u * kSignRep));
-#if MOE_GEMM_IQ2_FOLD
-    const uint32_t o0 = h2bits(__hmul2(bits2h(g.x ^ sm.x), fd2));
-    const uint32_t o1 = h2bits(__hmul2(bits2h(g.y ^ sm.y), fd2));
-    const uint32_t o2 = h2bits(__hmul2(bits2h(g.z ^ sm.z), fd2));
-    const uint32_t o3 = h2bits(__hmul2(bits2h(g.w ^ sm.w), fd2));
-#else
     // grid value times 2s+1 is exact in f16 (at most 43 * 31); one rounding by d/8
     const uint32_t o0 = h2bits(__hmul2(__hmul2(bits2h(g.x ^ sm.x), f2), d2));
     const uint32_t o1 = h2bits(__hmul2(__hmul2(bits2h(g.y ^ sm.y), f2), d2));
     const uint32_t o2 = h2bits(__hmul2(__hmul2(bits2h(g.z ^ sm.z), f2), d2));
     const uint32_t o3 = h2bits(__hmul2(__hmul2(bits2h(g.w ^ sm.w), f2), d2));
-#endif
     sts128(swz(tile, row, 4 * item + j), o0, o1, o2, o3);
   }
 }
