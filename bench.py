@@ -382,9 +382,10 @@ def run_ours(args, world, rank):
          "achieved_gbs": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"], "distinct_experts_per_call": n_distinct},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 4,
                 "d2h_bytes_per_step": T * s.hidden * 4},
-        # batched: router (4), permutation (3), input, 4 GEMMs; small-token: k1 and
-        # k2, or for Q4_K layers k1, the routing kernel and the 3 expert kernels
-        "gpu_launches": (12 if large else 5 if s.q4k else 2) * args.steps,
+        # batched: router (4), permutation (3), input, 4 GEMMs, and from 257
+        # tokens the 3 expansions of the shared expert's rows; small-token: k1
+        # and k2, or for Q4_K layers k1, the routing kernel and the 3 expert kernels
+        "gpu_launches": ((15 if T >= 257 else 12) if large else 5 if s.q4k else 2) * args.steps,
         "clocks": clocks,
     }
     return out

@@ -114,6 +114,10 @@ moe::LayerDims dims_of(const moe_config &c) {
   d.scaling = c.routed_scaling;
   d.eps = c.rms_eps;
   d.wait_cycles = moe::kDefaultWaitCycles;
+  // MOE_SHARED_DENSE=0 in the environment keeps the batched path's shared
+  // expert on per-tile Q8_0 decoding (results are identical)
+  const char *sd = getenv("MOE_SHARED_DENSE");
+  d.shared_dense = (sd && sd[0] == '0' && sd[1] == 0) ? 0 : 1;
   return d;
 }
 

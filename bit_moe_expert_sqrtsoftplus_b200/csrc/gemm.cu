@@ -169,7 +169,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
 // try_wait may suspend the thread until the phase completes, which can
 // outlast a bound shorter than the default; such bounds poll with the
 // non-blocking test_wait instead.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, GemmCtl &ctl, int *err) {
+template <typename Ctl>
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, Ctl &ctl, int *err) {
   if (ctl.wait < kDefaultWaitCycles) {
     const long long t0 = clock64();
     while (!mbar_test(b, parity)) {
@@ -293,6 +294,31 @@ __device__ __forceinline__ uint8_t *swz(uint8_t *tile, int row, int chunk) {
 
 __device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 bits2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// One accumulator element (row m of the tile's weights, global column c):
+// dv = D of the first matrix, u = D of the pair's second (SwiGLU only).
+__device__ __forceinline__ void epilogue_one(const GemmArgs &a, float dv, float u, int c, int m) {
+  if (a.epi == kEpiSwiGLU) {
+    // SiLU with the fast exponential and reciprocal (rcp(inf) = 0 for large -dv)
+    const float h = dv * __frcp_rn(1.f + __expf(-dv)) * u;
+    uint16_t hb;
+    if (a.h_bf16) {
+      __nv_bfloat16 v = __float2bfloat16_rn(h);
+      hb = *reinterpret_cast<uint16_t *>(&v);
+    } else {
+      __half v = __float2half_rn(h);
+      hb = *reinterpret_cast<uint16_t *>(&v);
+    }
+    a.h_out[(size_t)c * a.h_ld + m] = hb;
+  } else if (a.epi == kEpiScatterAdd) {
+    const int pr = a.perm[c];
+    atomicAdd(a.y + (size_t)(pr / a.k) * a.y_ld + m, a.w[pr] * dv);
+  } else {
+    float v = dv;
+    if (a.res) v += a.res[(size_t)c * a.y_ld + m];
+    a.y[(size_t)c * a.y_ld + m] = v;
+  }
+}
 
 // ---------------------------------------------------------------- tile map
 
@@ -902,29 +928,7 @@ __global__ void __launch_bounds__(gemm_threads(TMA), 1) k_grouped_gemm(GemmArgs 
         for (int j = 0; j < 16; ++j) {
           const int n = c0 + j;
           if (n >= tl.nt) break;
-          const int c = tl.col0 + n;
-          const float dv = __uint_as_float(r0[j]);
-          if (a.epi == kEpiSwiGLU) {
-            const float u = __uint_as_float(PAIRED ? r1[j] : 0u);
-            // SiLU with the fast exponential and reciprocal (rcp(inf) = 0 for large -dv)
-            const float h = dv * __frcp_rn(1.f + __expf(-dv)) * u;
-            uint16_t hb;
-            if (a.h_bf16) {
-              __nv_bfloat16 v = __float2bfloat16_rn(h);
-              hb = *reinterpret_cast<uint16_t *>(&v);
-            } else {
-              __half v = __float2half_rn(h);
-              hb = *reinterpret_cast<uint16_t *>(&v);
-            }
-            a.h_out[(size_t)c * a.h_ld + m] = hb;
-          } else if (a.epi == kEpiScatterAdd) {
-            const int pr = a.perm[c];
-            atomicAdd(a.y + (size_t)(pr / a.k) * a.y_ld + m, a.w[pr] * dv);
-          } else {
-            float v = dv;
-            if (a.res) v += a.res[(size_t)c * a.y_ld + m];
-            a.y[(size_t)c * a.y_ld + m] = v;
-          }
+          epilogue_one(a, __uint_as_float(r0[j]), __uint_as_float(PAIRED ? r1[j] : 0u), tl.col0 + n, m);
         }
       }
       tc_fence_before();
@@ -938,6 +942,212 @@ __global__ void __launch_bounds__(gemm_threads(TMA), 1) k_grouped_gemm(GemmArgs 
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512));
   }
+}
+
+// ---------------------------------------------------------------- dense GEMM
+//
+// D = A B^T with A [M][K] and B [N][K] both plain 16-bit rows in global
+// memory (the shared expert at large T: its Q8_0 rows expanded once per call
+// by k_expand_q80, the tokens' activation rows as they are).  Both operands
+// arrive by TMA as 128-byte-swizzled K-major tiles, so there are no producer
+// warps: warps 0-7 epilogue (as above), warp 8 tensor memory and
+// tcgen05.mma, warp 9 the tensor copies.  Tiles, MMA order and epilogue are
+// those of the grouped kernel for the same matrix, so the results are the
+// same bits.
+
+constexpr int kDenseMmaWarp = kEpiWarps;       // 8
+constexpr int kDenseCopyWarp = kEpiWarps + 1;  // 9
+constexpr int kDenseThreads = (kEpiWarps + 2) * 32;
+constexpr int kDenseBN = 256;
+__host__ __device__ constexpr int dense_stages(bool paired) { return paired ? 3 : 4; }
+__host__ __device__ constexpr int dense_stage_bytes(bool paired) { return (paired ? 2 : 1) * kATile + kDenseBN * BK * 2; }
+
+struct alignas(8) DenseCtl {
+  uint64_t full[4], empty[4], acc_full[2], acc_empty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  long long wait;
+};
+
+template <bool PAIRED>
+__global__ void __launch_bounds__(kDenseThreads, 1)
+    k_dense_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                 const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+  constexpr int NA = PAIRED ? 2 : 1;
+  constexpr int BN = kDenseBN;
+  constexpr int NACC = nacc_of(kFmtQ80, PAIRED);  // a pair's 2 x 256 columns fill TMEM: one buffer
+  constexpr int ACC_COLS = NA * BN;
+  constexpr int KS = dense_stages(PAIRED);
+  constexpr int STAGE = dense_stage_bytes(PAIRED);
+  static_assert(bn_of(kFmtQ80, PAIRED) == BN, "same tiles as the grouped kernel");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  DenseCtl &ctl = *reinterpret_cast<DenseCtl *>(smem + KS * STAGE);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m_tiles = a.M / BM, n_tiles = (a.cols + BN - 1) / BN, total = m_tiles * n_tiles;
+  const int ksteps = a.K / BK;
+
+  if (tid == 0) {
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&ctl.full[s], 1);   // the copy thread's expect_tx arrival (+ the copies' bytes)
+      mbar_init(&ctl.empty[s], 1);  // the MMA thread's commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl.acc_full[b], 1);
+      mbar_init(&ctl.acc_empty[b], kEpiWarps * 32);
+    }
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    ctl.wait = a.wait_cycles > 0 ? a.wait_cycles : kDefaultWaitCycles;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == kDenseMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&ctl.tmem_base)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == kDenseCopyWarp) {
+    // =================================================== tensor copies
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const uint32_t s = it % KS;
+          if (!mbar_wait(&ctl.empty[s], ((it / KS) & 1u) ^ 1u, ctl, a.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t *st = smem + s * STAGE;
+          mbar_arrive_tx(&ctl.full[s], (uint32_t)STAGE);
+          tma_load_2d(st, &tmA0, ks * BK, m0, &ctl.full[s]);
+          if (PAIRED) tma_load_2d(st + kATile, &tmA1, ks * BK, m0, &ctl.full[s]);
+          tma_load_2d(st + NA * kATile, &tmB, ks * BK, n0, &ctl.full[s]);  // rows past N read as zeros
+        }
+      }
+      // every copy issued has landed before the CTA exits
+      for (uint32_t q = it > KS ? it - KS : 0; q < it; ++q) {
+        const long long t1 = clock64();
+        while (!mbar_try(&ctl.full[q % KS], (q / KS) & 1u)) {
+          if (clock64() - t1 > kDefaultWaitCycles) {
+            set_error(a.err, kErrTimeout);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kDenseMmaWarp) {
+    // =================================================== MMA issue
+    uint32_t it = 0, tc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
+      const int n0 = (t % n_tiles) * BN;
+      const int nt = min(BN, a.cols - n0);
+      const uint32_t idesc = instr_desc((nt + 15) & ~15, a.bf16);
+      const uint32_t buf = tc % NACC;
+      const uint32_t dacc = tmem + buf * ACC_COLS;
+      if (!mbar_wait(&ctl.acc_empty[buf], ((tc / NACC) & 1u) ^ 1u, ctl, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        const uint32_t s = it % KS;
+        if (!mbar_wait(&ctl.full[s], (it / KS) & 1u, ctl, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(smem + s * STAGE), b0 = a0 + NA * kATile;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            mma_f16(dacc, smem_desc(a0 + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+            if (PAIRED) mma_f16(dacc + BN, smem_desc(a0 + kATile + 32 * kk), smem_desc(b0 + 32 * kk), idesc, acc);
+          }
+          mma_commit(&ctl.empty[s]);
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) mma_commit(&ctl.acc_full[buf]);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      mma_commit(&ctl.drain);
+      const long long t0 = clock64();
+      while (!mbar_try(&ctl.drain, 0u)) {
+        if (clock64() - t0 > kDefaultWaitCycles) {
+          set_error(a.err, kErrTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // =================================================== epilogue (warps 0-7)
+    const int row = (warp & 3) * 32 + lane;
+    const int half = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    uint32_t tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const int m0 = (t / n_tiles) * BM, n0 = (t % n_tiles) * BN;
+      const int nt = min(BN, a.cols - n0);
+      const uint32_t buf = tc % NACC;
+      if (!mbar_wait(&ctl.acc_full[buf], (tc / NACC) & 1u, ctl, a.err)) break;
+      tc_fence_after();
+      for (int c0 = 16 * half; c0 < nt; c0 += 32) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(lane_base + buf * ACC_COLS + c0, r0);
+        if (PAIRED) tmem_ld16(lane_base + buf * ACC_COLS + BN + c0, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + j;
+          if (n >= nt) break;
+          epilogue_one(a, __uint_as_float(r0[j]), __uint_as_float(PAIRED ? r1[j] : 0u), n0 + n, m0 + row);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl.acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kDenseMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512));
+  }
+}
+
+// out[r][k] = the Q8_0 value d * q of W's row r, rounded once to f16 (bf16 =
+// 0) or bf16 (bf16 = 1): the operand the grouped kernel's Q8_0 producers make.
+// One thread per 8 values.
+__global__ void k_expand_q80(const uint8_t *__restrict__ W, int rows, int K, int bf16, uint16_t *__restrict__ out) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_row = K / 8;
+  if (i >= (size_t)rows * per_row) return;
+  const size_t r = i / per_row;
+  const int c8 = (int)(i - r * per_row);
+  const uint8_t *bp = W + r * (size_t)(K / 32) * 34 + (size_t)(c8 >> 2) * 34;
+  const float d = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(bp)));
+  const uint8_t *qp = bp + 2 + 8 * (c8 & 3);  // 2-byte aligned
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t qq = *reinterpret_cast<const uint16_t *>(qp + 2 * j);
+    const float v0 = (float)(int8_t)(qq & 255u) * d, v1 = (float)(int8_t)(qq >> 8) * d;  // exact products
+    o[j] = bf16 ? bf16pair(v0, v1) : h2bits(__floats2half2_rn(v0, v1));
+  }
+  *reinterpret_cast<uint4 *>(out + r * (size_t)K + 8 * (size_t)c8) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace
@@ -978,18 +1188,73 @@ cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms) {
   return cudaErrorInvalidValue;
 }
 
+static PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
+  PFN_cuTensorMapEncodeTiled encode = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&encode), cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return encode;
+}
+
+// [rows][K] 16-bit rows, box 64 values x box_rows rows, 128-byte swizzle.
+static bool rows16_map(CUtensorMap *m, const void *base, int bf16, size_t rows, size_t K, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled encode = tensor_map_encoder();
+  if (!encode || !base || (reinterpret_cast<uintptr_t>(base) & 15u) || (K * 2) % 16 || K % BK) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t dense_gemm_smem(int paired) {
+  return 1024 + (size_t)dense_stages(paired != 0) * dense_stage_bytes(paired != 0) + sizeof(DenseCtl);
+}
+
+template <bool PAIRED>
+static cudaError_t launch_dense(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b, const GemmArgs &a,
+                                cudaStream_t s, int num_sms) {
+  static SmemOptIn opt;
+  const size_t smem = dense_gemm_smem(PAIRED);
+  cudaError_t e = opt_in_smem(k_dense_gemm<PAIRED>, smem, opt);
+  if (e != cudaSuccess) return e;
+  k_dense_gemm<PAIRED><<<num_sms, kDenseThreads, smem, s>>>(a0, a1, b, a);
+  return cudaGetLastError();
+}
+
+cudaError_t dense_gemm(const GemmArgs &a, const uint16_t *A0, const uint16_t *A1, const uint16_t *B, cudaStream_t s,
+                       int num_sms) {
+  if (a.M % BM || a.K % BK || a.cols <= 0 || a.epi == kEpiScatterAdd || (a.epi == kEpiSwiGLU) != (A1 != nullptr))
+    return cudaErrorInvalidValue;
+  CUtensorMap m0, m1, mb;
+  if (!rows16_map(&m0, A0, a.bf16, (size_t)a.M, (size_t)a.K, BM) ||
+      (A1 && !rows16_map(&m1, A1, a.bf16, (size_t)a.M, (size_t)a.K, BM)) ||
+      !rows16_map(&mb, B, a.bf16, (size_t)a.cols, (size_t)a.K, kDenseBN))
+    return cudaErrorInvalidValue;
+  if (!A1) m1 = m0;
+  return A1 ? launch_dense<true>(m0, m1, mb, a, s, num_sms) : launch_dense<false>(m0, m1, mb, a, s, num_sms);
+}
+
+cudaError_t expand_q80(const uint8_t *W, int rows, int K, int bf16, uint16_t *out, cudaStream_t s) {
+  const size_t n = (size_t)rows * (K / 8);
+  if (n == 0) return cudaSuccess;
+  k_expand_q80<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(W, rows, K, bf16, out);
+  return cudaGetLastError();
+}
+
 bool gemm_tensor_map(void *map, const void *base, size_t row_bytes, size_t rows, int fmt) {
   if (fmt != kFmtIQ2 && fmt != kFmtQ2K) return false;
   const int box = pbox_of(fmt);
   if (!base || (reinterpret_cast<uintptr_t>(base) & 15u) || row_bytes % 16 || row_bytes < (size_t)box || rows == 0 ||
       rows > 0xFFFFFFFFull)
     return false;
-  PFN_cuTensorMapEncodeTiled encode = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&encode), cudaEnableDefault, &q) !=
-          cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || !encode)
-    return false;
+  PFN_cuTensorMapEncodeTiled encode = tensor_map_encoder();
+  if (!encode) return false;
   const cuuint64_t dims[2] = {row_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t boxd[2] = {(cuuint32_t)box, (cuuint32_t)BM};

@@ -55,6 +55,20 @@ struct GemmArgs {
 cudaError_t grouped_gemm(const GemmArgs &a, cudaStream_t s, int num_sms);
 size_t grouped_gemm_smem(int fmt, int paired, int tma);
 
+// D = A B^T for plain 16-bit operand rows (A0 [M][K], B [cols][K], both with
+// row stride K, f16 or bf16 as a.bf16 says): the same tiles, MMA order and
+// epilogues (SwiGLU with A1 = the pair's up rows, or store) as grouped_gemm on
+// one group, fed by TMA instead of producer warps.  Reads a.bf16, epi, M, K,
+// cols, the epilogue fields, err and wait_cycles.
+cudaError_t dense_gemm(const GemmArgs &a, const uint16_t *A0, const uint16_t *A1, const uint16_t *B, cudaStream_t s,
+                       int num_sms);
+size_t dense_gemm_smem(int paired);
+
+// out [rows][K] = the values of Q8_0 rows W (K a multiple of 32), each d * q
+// rounded once to f16 (bf16 = 0) or bf16: the operands grouped_gemm's Q8_0
+// producers make, for dense_gemm.
+cudaError_t expand_q80(const uint8_t *W, int rows, int K, int bf16, uint16_t *out, cudaStream_t s);
+
 // Tensor map (128 bytes, written to `map`) of a packed weight array of `rows`
 // rows of `row_bytes` bytes in `fmt` (kFmtIQ2 or kFmtQ2K) for the TMA staging
 // of the grouped GEMM's A tiles: one copy brings one 256-value block of 128

@@ -20,8 +20,16 @@ struct LayerDims {
   // slice, the job table, a tensor-core pipeline hand-off); waits on a
   // warp's own copies keep the default
   long long wait_cycles;
+  // batched path: 1 = the shared expert's weights are expanded to 16-bit
+  // rows once per call and multiplied by a TMA-fed GEMM when the call has at
+  // least kSharedDenseMinT tokens; 0 = its producers decode Q8_0 per tile
+  int shared_dense;
 };
 constexpr long long kDefaultWaitCycles = 4000000000ll;  // about 2 s
+#ifndef MOE_SHARED_DENSE_MIN_T
+#define MOE_SHARED_DENSE_MIN_T 257
+#endif
+constexpr int kSharedDenseMinT = MOE_SHARED_DENSE_MIN_T;
 
 // Opaque TMA tensor descriptor (the driver's 128-byte, 64-byte aligned
 // CUtensorMap), built on the host and read by the TMA unit from the kernel's

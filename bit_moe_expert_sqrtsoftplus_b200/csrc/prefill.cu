@@ -73,32 +73,34 @@ __global__ void k_token_norms(const float *x, int T, int H, int flags, float eps
   }
 }
 
-// z[t][e] for a 64-token x 128-expert tile; 256 threads, each 4 tokens x 8
-// experts.  Per 32-element K chunk every output is a sum of 32 fp32 FMAs
-// (the chunk the error bound below assumes), added to an fp64 accumulator.
-// Rows are staged with 16-byte loads (x scaled by the token's fp32 inverse
-// RMS, W_r converted from f16), transposed into K-major shared tiles.
-constexpr int RT = 64, RE = 128, RK = 32;
+// z[t][e] for a 64-token x 64-expert tile (T = 4096 and E = 256 give 256
+// blocks, so every SM has work); 256 threads, each 4 tokens x 4 experts.  Per
+// 32-element K chunk every output is a sum of 32 fp32 FMAs (the chunk the
+// error bound below assumes), added to an fp64 accumulator; the tile shape
+// does not change any output's arithmetic.  Rows are staged with 16-byte
+// loads (x scaled by the token's fp32 inverse RMS, W_r converted from f16),
+// transposed into K-major shared tiles.
+constexpr int RT = 64, RE = 64, RK = 32;
 __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double *inv, const uint16_t *Wr, int T,
                                                     int E, int H, double *z) {
   __shared__ __align__(16) float xs[RK][RT + 4];
   __shared__ __align__(16) float ws[RK][RE + 4];
   const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE;
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;  // experts tx*8 .., tokens ty*4 ..
-  // staging roles: x float4 pieces (token i>>3, K quad i&7) and W uint4
-  // pieces (expert i>>2, K octet i&3) for i = tid and tid + 256
+  const int tx = tid & 15, ty = tid >> 4;  // experts tx*4 .., tokens ty*4 ..
+  // staging roles: x float4 pieces (token i>>3, K quad i&7) for i = tid and
+  // tid + 256, and one W uint4 piece (expert tid>>2, K octet tid&3)
   float invf[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int t = t0 + ((tid + 256 * r) >> 3);
     invf[r] = t < T ? (float)inv[t] : 0.f;
   }
-  double acc[4][8];
+  double acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
   for (int k0 = 0; k0 < H; k0 += RK) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -112,10 +114,8 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
       xs[4 * kq + 2][tt] = v.z * invf[r];
       xs[4 * kq + 3][tt] = v.w * invf[r];
     }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = tid + 256 * r;
-      const int ee = i >> 2, ko = i & 3;
+    {
+      const int ee = tid >> 2, ko = tid & 3;
       const int e = e0 + ee;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (e < E) v = *reinterpret_cast<const uint4 *>(Wr + (size_t)e * H + k0 + 8 * ko);
@@ -127,27 +127,26 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
       }
     }
     __syncthreads();
-    float part[4][8];
+    float part[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) part[i][j] = 0.f;
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
 #pragma unroll 8
     for (int kk = 0; kk < RK; ++kk) {
       const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
-      const float4 w0 = *reinterpret_cast<const float4 *>(&ws[kk][tx * 8]);
-      const float4 w1 = *reinterpret_cast<const float4 *>(&ws[kk][tx * 8 + 4]);
+      const float4 wv = *reinterpret_cast<const float4 *>(&ws[kk][tx * 4]);
       const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wa[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part[i][j];
+      for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
     __syncthreads();
   }
 #pragma unroll
@@ -155,8 +154,8 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
     const int t = t0 + ty * 4 + i;
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = e0 + tx * 8 + j;
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
       if (e < E) z[(size_t)t * E + e] = acc[i][j];
     }
   }
@@ -618,6 +617,7 @@ struct BigScratch {
   uint16_t *hperm;  // [T*k][I] bf16, rows in permuted order
   uint16_t *hs;     // [T][Is] bf16
   float *slots;     // [T*k][H] weighted expert outputs per pair (deterministic combine only)
+  uint16_t *sh16;   // shared expert rows expanded to 16 bits (T >= kSharedDenseMinT only): gate, up [Is][H], down [H][Is]
   size_t bytes;
 };
 
@@ -635,6 +635,7 @@ BigScratch carve_big(const LayerDims &d, int T, void *base) {
   b.hs = reinterpret_cast<uint16_t *>(take(2 * (size_t)T * d.Is));
   b.slots = (d.flags & MOE_FLAG_DETERMINISTIC) ? reinterpret_cast<float *>(take(sizeof(float) * (size_t)T * d.k * d.H))
                                                 : nullptr;
+  b.sh16 = T >= kSharedDenseMinT ? reinterpret_cast<uint16_t *>(take(2 * 3 * (size_t)d.Is * d.H)) : nullptr;
   b.bytes = off;
   return b;
 }
@@ -711,8 +712,8 @@ GemmArgs routed_down_args(const LayerDims &d, const LayerWeights &wt, bool q4k, 
 
 // The shared expert over T activation rows: SwiGLU into hs, then the down
 // projection stored into y (plus res, the residual input, when given).
-cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, const __half *x16, uint16_t *hs,
-                         const float *res, float *y, int *err, cudaStream_t s, int num_sms) {
+GemmArgs shared_gateup_args(const LayerDims &d, const LayerWeights &wt, int T, const __half *x16, uint16_t *hs,
+                            int *err) {
   GemmArgs sg{};
   sg.fmt = kFmtQ80;
   sg.bf16 = 0;
@@ -736,8 +737,11 @@ cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, cons
   sg.h_bf16 = 1;
   sg.err = err;
   sg.wait_cycles = d.wait_cycles;
-  cudaError_t e = grouped_gemm(sg, s, num_sms);
-  if (e != cudaSuccess) return e;
+  return sg;
+}
+
+GemmArgs shared_down_args(const LayerDims &d, const LayerWeights &wt, int T, const uint16_t *hs, const float *res,
+                          float *y, int *err) {
   GemmArgs sd{};
   sd.fmt = kFmtQ80;
   sd.bf16 = 1;
@@ -758,7 +762,30 @@ cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, cons
   sd.res = res;
   sd.err = err;
   sd.wait_cycles = d.wait_cycles;
-  return grouped_gemm(sd, s, num_sms);
+  return sd;
+}
+
+cudaError_t shared_gemms(const LayerDims &d, const LayerWeights &wt, int T, const __half *x16, uint16_t *hs,
+                         const float *res, float *y, int *err, cudaStream_t s, int num_sms) {
+  cudaError_t e = grouped_gemm(shared_gateup_args(d, wt, T, x16, hs, err), s, num_sms);
+  if (e != cudaSuccess) return e;
+  return grouped_gemm(shared_down_args(d, wt, T, hs, res, y, err), s, num_sms);
+}
+
+// The same with the shared expert's rows expanded to 16 bits first (sh16:
+// gate and up [Is][H] f16, then down [H][Is] bf16) and TMA-fed GEMMs: at
+// large T every weight tile would otherwise be decoded once per 256 tokens.
+cudaError_t shared_gemms_dense(const LayerDims &d, const LayerWeights &wt, int T, const __half *x16, uint16_t *hs,
+                               uint16_t *sh16, const float *res, float *y, int *err, cudaStream_t s, int num_sms) {
+  uint16_t *g16 = sh16, *u16 = g16 + (size_t)d.Is * d.H, *dn16 = u16 + (size_t)d.Is * d.H;
+  cudaError_t e = expand_q80(wt.sh_gate, d.Is, d.H, 0, g16, s);
+  if (e == cudaSuccess) e = expand_q80(wt.sh_up, d.Is, d.H, 0, u16, s);
+  if (e == cudaSuccess) e = expand_q80(wt.sh_down, d.H, d.Is, 1, dn16, s);
+  if (e != cudaSuccess) return e;
+  e = dense_gemm(shared_gateup_args(d, wt, T, x16, hs, err), g16, u16, reinterpret_cast<const uint16_t *>(x16), s,
+                 num_sms);
+  if (e != cudaSuccess) return e;
+  return dense_gemm(shared_down_args(d, wt, T, hs, res, y, err), dn16, nullptr, hs, s, num_sms);
 }
 
 }  // namespace
@@ -780,8 +807,9 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   if ((e = grouped_gemm(g, s, num_sms)) != cudaSuccess) return e;
   if (p.ev_end) cudaEventRecord(p.ev_end, s);
   // shared expert: Q8_0 gate/up over all tokens, down stored into y (plus the residual input when pre-norm)
-  e = shared_gemms(d, p.wt, T, b.x16, b.hs, (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr, p.y, p.err, s,
-                   num_sms);
+  const float *res = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? p.x : nullptr;
+  e = b.sh16 && d.shared_dense ? shared_gemms_dense(d, p.wt, T, b.x16, b.hs, b.sh16, res, p.y, p.err, s, num_sms)
+                               : shared_gemms(d, p.wt, T, b.x16, b.hs, res, p.y, p.err, s, num_sms);
   if (e != cudaSuccess) return e;
   // routed down: Q2_K (or Q4_K) x bf16 h, y[token] += w * (W_down h)
   if (!(d.flags & MOE_FLAG_DETERMINISTIC))

@@ -7,8 +7,9 @@
 //   y[t] = shared(x̂[t]) + sum_i w[t][i] * E_idx[t][i](x̂[t])   (+ x[t] with the
 //   pre-norm residual), E(v) = W_down (SiLU(W_gate v) * (W_up v))
 // with fp32 dot products over blocks decoded in registers: one warp per
-// output row.  It is the plain first form of this path (three launches, no
-// tensor cores); its arithmetic is exact decoding and fp32 accumulation.
+// output row (gate and up rows of a pair together; all k routed down rows of
+// a token together), three launches, no tensor cores; its arithmetic is exact
+// decoding and fp32 accumulation.
 //
 // Q4_K block (144 bytes, 256 values; "2bit 量子化はなぜ「冗談ではない」のか",
 // section 3 type table; layout read as the public GGUF block): f16 d at 0,
@@ -39,59 +40,70 @@ __device__ __forceinline__ float f16_at(const uint8_t *p) {
   return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(p)));
 }
 
-// sum_k W[row][k] v[k] over K values of Q4_K blocks (K a multiple of 256);
-// every lane returns the sum.
-__device__ float dot_q4k(const uint8_t *row, const float *v, int K, int lane) {
-  const float4 *v4 = reinterpret_cast<const float4 *>(v);
-  const int j = lane >> 2, jj = j & 3;
-  const int code_off = 16 + 32 * (lane >> 3) + 8 * (lane & 3);
-  const int shift = 4 * ((lane & 7) >> 2);
-  float part = 0.0f;
-#pragma unroll 4
-  for (int b = 0; b < K / 256; ++b) {  // unrolled so several blocks' loads are in flight
-    const uint8_t *blk = row + (size_t)b * 144;
-    const uint4 hd = *reinterpret_cast<const uint4 *>(blk);  // d, dmin, scale bytes 0..11
-    const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
-    const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
-    const uint32_t b03 = hd.y, b47 = hd.z, b811 = hd.w;  // scale bytes 0-3, 4-7, 8-11
-    int sc, mn;
-    if (j < 4) {
-      sc = (int)((b03 >> (8 * jj)) & 63u);
-      mn = (int)((b47 >> (8 * jj)) & 63u);
-    } else {
-      const uint32_t lowb = (b811 >> (8 * jj)) & 255u;
-      sc = (int)((lowb & 15u) | (((b03 >> (8 * jj + 6)) & 3u) << 4));
-      mn = (int)((lowb >> 4) | (((b47 >> (8 * jj + 6)) & 3u) << 4));
-    }
-    const uint2 cw = *reinterpret_cast<const uint2 *>(blk + code_off);
-    const float4 x0 = v4[64 * b + 2 * lane], x1 = v4[64 * b + 2 * lane + 1];
-    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    float sqx = 0.0f, sx = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 255u;
-      const float q = (float)((byte >> shift) & 15u);
-      sqx = fmaf(q, xs[k], sqx);
-      sx += xs[k];
-    }
-    part += d * (float)sc * sqx - dmin * (float)mn * sx;
+// Lane l's share of a Q4_K block: values 8l .. 8l+7, i.e. sub-block l/4,
+// code bytes 32*(l/8) + 8*(l%4) .. +7, nibble (l%8)/4.
+struct Q4kLane {
+  int j, jj, code_off, shift;
+  __device__ explicit Q4kLane(int lane)
+      : j(lane >> 2), jj((lane >> 2) & 3), code_off(16 + 32 * (lane >> 3) + 8 * (lane & 3)),
+        shift(4 * ((lane & 7) >> 2)) {}
+};
+
+// Lane l's part of one block's dot product with its 8 values xs of v:
+// d*scale*sum(q*x) - dmin*min*sum(x), sx = sum(x) given.
+__device__ __forceinline__ float q4k_part(const uint4 hd, const uint2 cw, const Q4kLane &L, const float (&xs)[8],
+                                          float sx) {
+  const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
+  const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
+  const uint32_t b03 = hd.y, b47 = hd.z, b811 = hd.w;  // scale bytes 0-3, 4-7, 8-11
+  int sc, mn;
+  if (L.j < 4) {
+    sc = (int)((b03 >> (8 * L.jj)) & 63u);
+    mn = (int)((b47 >> (8 * L.jj)) & 63u);
+  } else {
+    const uint32_t lowb = (b811 >> (8 * L.jj)) & 255u;
+    sc = (int)((lowb & 15u) | (((b03 >> (8 * L.jj + 6)) & 3u) << 4));
+    mn = (int)((lowb >> 4) | (((b47 >> (8 * L.jj + 6)) & 3u) << 4));
   }
+  float sqx = 0.0f;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  return part;
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 255u;
+    sqx = fmaf((float)((byte >> L.shift) & 15u), xs[k], sqx);
+  }
+  return d * (float)sc * sqx - dmin * (float)mn * sx;
 }
 
-// The same over Q8_0 blocks (K a multiple of 32): lane l takes value l of
-// every block.
-__device__ float dot_q80(const uint8_t *row, const float *v, int K, int lane) {
-  float part = 0.0f;
-#pragma unroll 8
-  for (int b = 0; b < K / 32; ++b) {
-    const uint8_t *blk = row + (size_t)b * 34;
-    part = fmaf(f16_at(blk) * (float)(int8_t)blk[2 + lane], v[32 * b + lane], part);
-  }
+__device__ __forceinline__ void load8(const float *v, float (&xs)[8], float &sx) {
+  const float4 a = reinterpret_cast<const float4 *>(v)[0], b = reinterpret_cast<const float4 *>(v)[1];
+  xs[0] = a.x, xs[1] = a.y, xs[2] = a.z, xs[3] = a.w, xs[4] = b.x, xs[5] = b.y, xs[6] = b.z, xs[7] = b.w;
+  sx = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-  for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Lane l's part of sum_k W[row][k] v[k] over Q8_0 blocks (K a multiple of
+// 128): per iteration the warp takes four blocks, lane l the values
+// 4*(l%8) .. +3 of block l/8 of them (two 16-bit loads: blocks are 34 bytes,
+// so their quants are 2-byte aligned).
+__device__ __forceinline__ float q80_part(const uint8_t *row, const float *v, int K, int lane) {
+  const int sub = lane >> 3, q4 = 4 * (lane & 7);
+  float part = 0.0f;
+#pragma unroll 4
+  for (int b = sub; b < K / 32; b += 4) {
+    const uint8_t *blk = row + (size_t)b * 34;
+    const float d = f16_at(blk);
+    const uint32_t lo = *reinterpret_cast<const uint16_t *>(blk + 2 + q4);
+    const uint32_t hi = *reinterpret_cast<const uint16_t *>(blk + 4 + q4);
+    const float4 x = *reinterpret_cast<const float4 *>(v + 32 * b + q4);
+    const float s = (float)(int8_t)(lo & 255u) * x.x + (float)(int8_t)(lo >> 8) * x.y +
+                    (float)(int8_t)(hi & 255u) * x.z + (float)(int8_t)(hi >> 8) * x.w;
+    part = fmaf(d, s, part);
+  }
   return part;
 }
 
@@ -131,12 +143,25 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
     const int t = p / d.k, e = a.idx[p];
     float hv = 0.0f;
     if (e >= 0 && e < d.E) {
+      // gate and up rows of the pair together: both rows' loads of a block
+      // are in flight at once, and the x values and their sum serve both
       const size_t rb = (size_t)(d.H / 256) * 144;
-      const size_t off = ((size_t)e * d.I + row) * rb;
+      const uint8_t *gr = a.gate + ((size_t)e * d.I + row) * rb, *ur = a.up + ((size_t)e * d.I + row) * rb;
       const float *xt = a.xn + (size_t)t * d.H;
-      const float g = dot_q4k(a.gate + off, xt, d.H, lane);
-      const float u = dot_q4k(a.up + off, xt, d.H, lane);
-      hv = silu(g) * u;
+      const Q4kLane L(lane);
+      float pg = 0.0f, pu = 0.0f;
+#pragma unroll 4
+      for (int b = 0; b < d.H / 256; ++b) {
+        const uint4 hg = *reinterpret_cast<const uint4 *>(gr + (size_t)b * 144);
+        const uint4 hu = *reinterpret_cast<const uint4 *>(ur + (size_t)b * 144);
+        const uint2 cg = *reinterpret_cast<const uint2 *>(gr + (size_t)b * 144 + L.code_off);
+        const uint2 cu = *reinterpret_cast<const uint2 *>(ur + (size_t)b * 144 + L.code_off);
+        float xs[8], sx;
+        load8(xt + 256 * b + 8 * lane, xs, sx);
+        pg += q4k_part(hg, cg, L, xs, sx);
+        pu += q4k_part(hu, cu, L, xs, sx);
+      }
+      hv = silu(warp_sum(pg)) * warp_sum(pu);
     }
     if (lane == 0) a.h[(size_t)p * d.I + row] = hv;
   } else {
@@ -144,26 +169,50 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
     const int t = p - npairs;
     const size_t rb = (size_t)(d.H / 32) * 34;
     const float *xt = a.xn + (size_t)t * d.H;
-    const float g = dot_q80(a.sh_gate + (size_t)row * rb, xt, d.H, lane);
-    const float u = dot_q80(a.sh_up + (size_t)row * rb, xt, d.H, lane);
+    const float g = warp_sum(q80_part(a.sh_gate + (size_t)row * rb, xt, d.H, lane));
+    const float u = warp_sum(q80_part(a.sh_up + (size_t)row * rb, xt, d.H, lane));
     if (lane == 0) a.hs[(size_t)t * d.Is + row] = silu(g) * u;
   }
 }
 
-// y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i],
-// the routed terms in the routing's ascending expert order.
+// y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i]:
+// one warp per output row; the routed rows of the token's k pairs are read
+// block by block together (k rows' loads of a block in flight at once), each
+// lane weighting its parts by w in the routing's ascending expert order
+// before one reduction over the warp.
 __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31, r = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5), t = blockIdx.y;
   if (r >= d.H) return;
   const size_t rbs = (size_t)(d.Is / 32) * 34, rbd = (size_t)(d.I / 256) * 144;
-  float acc = dot_q80(a.sh_down + (size_t)r * rbs, a.hs + (size_t)t * d.Is, d.Is, lane);
-  for (int i = 0; i < d.k; ++i) {
-    const int p = t * d.k + i, e = a.idx[p];
-    if (e < 0 || e >= d.E) continue;
-    const float o = dot_q4k(a.down + ((size_t)e * d.H + r) * rbd, a.h + (size_t)p * d.I, d.I, lane);
-    acc = fmaf(a.w[p], o, acc);
+  const uint8_t *row[kMaxK];
+  float wt[kMaxK];
+#pragma unroll
+  for (int i = 0; i < kMaxK; ++i) {
+    const int e = i < d.k ? a.idx[t * d.k + i] : -1;
+    const bool ok = e >= 0 && e < d.E;
+    row[i] = ok ? a.down + ((size_t)e * d.H + r) * rbd : nullptr;
+    wt[i] = ok ? a.w[t * d.k + i] : 0.0f;
   }
+  const Q4kLane L(lane);
+  float part[kMaxK];
+#pragma unroll
+  for (int i = 0; i < kMaxK; ++i) part[i] = 0.0f;
+  for (int b = 0; b < d.I / 256; ++b) {
+#pragma unroll
+    for (int i = 0; i < kMaxK; ++i) {
+      if (!row[i]) continue;
+      const uint4 hd = *reinterpret_cast<const uint4 *>(row[i] + (size_t)b * 144);
+      const uint2 cw = *reinterpret_cast<const uint2 *>(row[i] + (size_t)b * 144 + L.code_off);
+      float xs[8], sx;
+      load8(a.h + (size_t)(t * d.k + i) * d.I + 256 * b + 8 * lane, xs, sx);
+      part[i] += q4k_part(hd, cw, L, xs, sx);
+    }
+  }
+  float acc = q80_part(a.sh_down + (size_t)r * rbs, a.hs + (size_t)t * d.Is, d.Is, lane);
+#pragma unroll
+  for (int i = 0; i < kMaxK; ++i) acc = fmaf(wt[i], part[i], acc);
+  acc = warp_sum(acc);
   if (lane == 0) {
     const size_t at = (size_t)t * d.H + r;
     a.y[at] = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[at] + acc : acc;

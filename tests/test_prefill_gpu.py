@@ -165,3 +165,30 @@ def test_tma_staged_tiles_match_plain_loads(moe, monkeypatch, flags):
     _, _, yref, _ = harness.oracle_layer_dense(s, 8, 2, x_np)
     rel, mx = harness.errors(yt, yref)
     assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 300), ("prefill_t4096", 4096)])
+def test_dense_shared_expert_matches_per_tile_decoding(moe, monkeypatch, name, T):
+    """From 257 tokens the shared expert's Q8_0 rows are expanded to 16 bits
+    once per call and multiplied by TMA-fed GEMMs; its operands, tiles and
+    MMA order are those of the per-tile decoding path (MOE_SHARED_DENSE=0 at
+    init), so with the deterministic combine the outputs are the same bits.
+    The tiny case is also checked against the oracle."""
+    s = synth.workload(name, tokens=T)
+    W = harness.device_layer(s, 9, 4)
+    x_np = synth.activations(9, T, s.hidden, stream=4)
+    x = torch.from_numpy(x_np).cuda()
+    fl = moe.MOE_FLAG_DETERMINISTIC | moe.MOE_FLAG_PRENORM_RESIDUAL
+    Ld = moe.Layer(harness.config_for(s, flags=fl), W, max_tokens=T)
+    monkeypatch.setenv("MOE_SHARED_DENSE", "0")
+    Lp = moe.Layer(harness.config_for(s, flags=fl), W, max_tokens=T)
+    monkeypatch.delenv("MOE_SHARED_DENSE")
+    yd = Ld.forward(x).cpu().numpy()
+    yp = Lp.forward(x).cpu().numpy()
+    Ld.poll()
+    Lp.poll()
+    assert np.array_equal(yd.view(np.uint32), yp.view(np.uint32))
+    if name == "tiny":
+        _, _, yref, _ = harness.oracle_layer(s, 9, 4, x_np, prenorm=True)
+        rel, mx = harness.errors(yd, yref)
+        assert rel <= harness.MMA_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
