@@ -58,6 +58,8 @@ def parse(argv=None):
                             "decode_t1_q4k", "quantize_q2k", "quantize_q80", "quantize_q4k"])
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--deterministic", action="store_true",
+                   help="layers made with MOE_FLAG_DETERMINISTIC (fixed-order combine above 32 tokens)")
     p.add_argument("--weight-sets", type=int, default=0, help="override the number of rotating weight sets")
     p.add_argument("--sweep", action="store_true",
                    help="time one layer call at T = 1, 2, 4, ..., 256 (skewed bias; one JSON line per T)")
@@ -240,6 +242,7 @@ def run_ours(args, world, rank):
         W = synth.device_layer(0, i, s, q4k=s.q4k)
         cfg = moe.make_config(s.hidden, s.inter, s.n_experts, s.top_k, s.shared_inter, vocab=s.vocab,
                               routed_scaling=s.routed_scaling,
+                              flags=moe.MOE_FLAG_DETERMINISTIC if args.deterministic else 0,
                               routed_format=moe.MOE_ROUTED_Q4K if s.q4k else moe.MOE_ROUTED_Q2)
         L = moe.Layer(cfg, W, max_tokens=T, scratch=scratch)
         scratch = L.scratch
@@ -365,6 +368,7 @@ def run_ours(args, world, rank):
         "config": {"workload": f"{args.workload}: V4-Flash MoE layer, T={T} tokens/call, hidden {s.hidden}, "
                                f"{s.n_experts} experts top-{s.top_k}, inter {s.inter}, shared {s.shared_inter}",
                    "tokens_per_call": T, "weight_sets_rotated": nsets,
+                   **({"combine": "deterministic (slot rows summed in expert order)"} if args.deterministic else {}),
                    "l2": (f"{nsets} rotating weight set(s) of {s.n_experts * s.expert_bytes / 1e9:.2f} GB "
                           "(inputs far larger than the 126 MB L2)" if s.n_experts * s.expert_bytes > 126e6 else
                           f"one weight set of {(s.n_experts * s.expert_bytes + s.shared_bytes) / 1e6:.2f} MB, "
@@ -382,10 +386,12 @@ def run_ours(args, world, rank):
          "achieved_gbs": layer_gbs, "frac": layer_gbs / peaks["hbm_gbs"], "distinct_experts_per_call": n_distinct},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 4,
                 "d2h_bytes_per_step": T * s.hidden * 4},
-        # batched: router (4), permutation (3), input, 4 GEMMs, and from 257
-        # tokens the 3 expansions of the shared expert's rows; small-token: k1
-        # and k2, or for Q4_K layers k1, the routing kernel and the 3 expert kernels
-        "gpu_launches": ((15 if T >= 257 else 12) if large else 5 if s.q4k else 2) * args.steps,
+        # batched: router (4), permutation (3), input, 4 GEMMs, from 257 tokens
+        # the 3 expansions of the shared expert's rows, and with the
+        # deterministic flag the slot sum; small-token: k1 and k2, or for Q4_K
+        # layers k1, the routing kernel and the 3 expert kernels
+        "gpu_launches": ((15 if T >= 257 else 12) + (1 if args.deterministic else 0) if large else
+                         5 if s.q4k else 2) * args.steps,
         "clocks": clocks,
     }
     return out

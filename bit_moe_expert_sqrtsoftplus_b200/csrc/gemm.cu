@@ -313,6 +313,9 @@ __device__ __forceinline__ void epilogue_one(const GemmArgs &a, float dv, float 
   } else if (a.epi == kEpiScatterAdd) {
     const int pr = a.perm[c];
     atomicAdd(a.y + (size_t)(pr / a.k) * a.y_ld + m, a.w[pr] * dv);
+  } else if (a.epi == kEpiSlotStore) {
+    const int pr = a.perm[c];
+    a.y[(size_t)pr * a.y_ld + m] = a.w[pr] * dv;
   } else {
     float v = dv;
     if (a.res) v += a.res[(size_t)c * a.y_ld + m];
@@ -1229,7 +1232,8 @@ static cudaError_t launch_dense(const CUtensorMap &a0, const CUtensorMap &a1, co
 
 cudaError_t dense_gemm(const GemmArgs &a, const uint16_t *A0, const uint16_t *A1, const uint16_t *B, cudaStream_t s,
                        int num_sms) {
-  if (a.M % BM || a.K % BK || a.cols <= 0 || a.epi == kEpiScatterAdd || (a.epi == kEpiSwiGLU) != (A1 != nullptr))
+  if (a.M % BM || a.K % BK || a.cols <= 0 || a.epi == kEpiScatterAdd || a.epi == kEpiSlotStore ||
+      (a.epi == kEpiSwiGLU) != (A1 != nullptr))
     return cudaErrorInvalidValue;
   CUtensorMap m0, m1, mb;
   if (!rows16_map(&m0, A0, a.bf16, (size_t)a.M, (size_t)a.K, BM) ||

@@ -14,7 +14,7 @@
 namespace moe {
 
 enum GemmFmt { kFmtIQ2 = 0, kFmtQ2K = 1, kFmtQ80 = 2, kFmtQ4K = 3 };
-enum GemmEpi { kEpiSwiGLU = 0, kEpiScatterAdd = 1, kEpiStore = 2 };
+enum GemmEpi { kEpiSwiGLU = 0, kEpiScatterAdd = 1, kEpiStore = 2, kEpiSlotStore = 3 };
 
 struct GemmArgs {
   int fmt;    // GemmFmt of the A operand
@@ -40,6 +40,7 @@ struct GemmArgs {
   int h_bf16;
   float *y;          // ScatterAdd: y[(perm[c]/k) * y_ld + m] += w[perm[c]] * D
   int y_ld;          // Store: y[c * y_ld + m] = D (+ res[c * y_ld + m])
+                     // SlotStore: y[perm[c] * y_ld + m] = w[perm[c]] * D (one row per pair)
   const float *res;
   const float *w;
   const int32_t *perm;

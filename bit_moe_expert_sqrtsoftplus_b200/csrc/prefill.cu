@@ -396,10 +396,31 @@ __global__ void k_hash_route(const int32_t *token_ids, const int32_t *tid2eid, i
 // ---------------------------------------------------------------- permutation
 
 // counts[e] = number of pairs routed to e (one block per expert).
-__global__ void k_perm_count(const int32_t *idx, int n, int32_t *counts) {
+// The 8 expert ids of pairs i .. i+7 (-1 past n): two 16-byte loads when
+// all 8 exist and idx is 16-byte aligned (i is a multiple of 8; a caller's
+// idx from moe_route may be only 4-byte aligned).
+__device__ __forceinline__ void load8_ids(const int32_t *idx, int n, int i, int (&v)[8]) {
+  if (i + 8 <= n && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0) {
+    const int4 a = *reinterpret_cast<const int4 *>(idx + i), b = *reinterpret_cast<const int4 *>(idx + i + 4);
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = i + j < n ? idx[i + j] : -1;
+  }
+}
+
+// counts[e] = pairs with expert e; one block per expert, 8 pairs per thread
+// per pass.
+__global__ void __launch_bounds__(256) k_perm_count(const int32_t *idx, int n, int32_t *counts) {
   const int e = blockIdx.x;
   int c = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) c += idx[i] == e;
+#pragma unroll 2
+  for (int i = 8 * threadIdx.x; i < n; i += 8 * blockDim.x) {
+    int v[8];
+    load8_ids(idx, n, i, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c += v[j] == e;
+  }
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   __shared__ int red[32];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
@@ -411,36 +432,64 @@ __global__ void k_perm_count(const int32_t *idx, int n, int32_t *counts) {
   }
 }
 
-__global__ void k_perm_scan(const int32_t *counts, int E, int32_t *offsets) {
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = counts[e];  // counts may alias offsets: read before writing
-      offsets[e] = run;
-      run += c;
-    }
-    offsets[E] = run;
+// Exclusive prefix sum of E <= kMaxE counts (one block of kMaxE threads):
+// every count is read before any offset is written (counts may alias
+// offsets), then a scan of warp sums.
+__global__ void __launch_bounds__(kMaxE) k_perm_scan(const int32_t *counts, int E, int32_t *offsets) {
+  __shared__ int wsum[kMaxE / 32];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int c = e < E ? counts[e] : 0;
+  int incl = c;  // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();  // every count has been read
+  int before = 0;
+  for (int q = 0; q < warp; ++q) before += wsum[q];
+  if (e < E) offsets[e] = before + incl - c;
+  if (e == kMaxE - 1) {
+    int total = 0;
+    for (int q = 0; q < kMaxE / 32; ++q) total += wsum[q];
+    offsets[E] = total;
   }
 }
 
 // perm[offsets[e] + rank] = pair id, ranks in ascending pair order (stable).
-__global__ void k_perm_scatter(const int32_t *idx, int n, const int32_t *offsets, int32_t *perm) {
+// One block per expert; per pass each thread takes 8 consecutive pairs, so
+// the block's hits of a pass are ranked by a scan over threads (thread order
+// is pair order).
+__global__ void __launch_bounds__(256) k_perm_scatter(const int32_t *idx, int n, const int32_t *offsets, int32_t *perm) {
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   __shared__ int wcount[32];
   int base = offsets[e];
-  for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const bool hit = i < n && idx[i] == e;
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) wcount[warp] = __popc(m);
+  for (int i0 = 0; i0 < n; i0 += 8 * blockDim.x) {
+    const int i = i0 + 8 * threadIdx.x;
+    int v[8];
+    load8_ids(idx, n, i, v);
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mine += v[j] == e;
+    int incl = mine;  // inclusive scan of the hit counts over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) wcount[warp] = incl;
     __syncthreads();
     int before = 0, total = 0;
     for (int q = 0; q < nw; ++q) {
       if (q < warp) before += wcount[q];
       total += wcount[q];
     }
-    if (hit) perm[base + before + __popc(m & ((1u << lane) - 1u))] = i;
+    int at = base + before + incl - mine;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (v[j] == e) perm[at++] = i + j;
     base += total;
     __syncthreads();
   }
@@ -815,14 +864,13 @@ cudaError_t prefill_forward(const PrefillArgs &p, cudaStream_t s, int num_sms) {
   if (!(d.flags & MOE_FLAG_DETERMINISTIC))
     return grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, d.k, b.hperm, p.s.w, p.y, p.err),
                         s, num_sms);
-  // deterministic: each pair's weighted output into its own slot row (one
-  // addition onto zero per element), then every token's slots summed in
-  // ascending slot order
-  const int n = T * d.k;
-  if ((e = cudaMemsetAsync(b.slots, 0, sizeof(float) * (size_t)n * d.H, s)) != cudaSuccess) return e;
-  e = grouped_gemm(routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, 1, b.hperm, p.s.w, b.slots, p.err), s,
-                   num_sms);
-  if (e != cudaSuccess) return e;
+  // deterministic: each pair's weighted output stored into its own slot row
+  // (every pair is in exactly one expert's columns and every row of H is in
+  // one tile, so each slot element is written once), then every token's
+  // slots summed in ascending slot order
+  GemmArgs rd = routed_down_args(d, p.wt, p.q4k, d.E, p.s.offsets, p.s.perm, 1, b.hperm, p.s.w, b.slots, p.err);
+  rd.epi = kEpiSlotStore;
+  if ((e = grouped_gemm(rd, s, num_sms)) != cudaSuccess) return e;
   k_sum_slots<<<T, 256, 0, s>>>(d.H, d.k, b.slots, p.y);
   return cudaGetLastError();
 }
@@ -964,7 +1012,11 @@ cudaError_t ep_experts(const LayerDims &d, const LayerWeights &wt, bool q4k, con
   if ((e = permute(local, N, 1, d.E, offsets, perm, s)) != cudaSuccess) return e;
   e = grouped_gemm(routed_gateup_args(d, wt, q4k, d.E, offsets, perm, 1, x_recv, h, err), s, num_sms);
   if (e != cudaSuccess) return e;
-  return grouped_gemm(routed_down_args(d, wt, q4k, d.E, offsets, perm, 1, h, w_recv, out, err), s, num_sms);
+  // each received row is in one expert's columns at most: a plain store of
+  // w * E(x) into its row (rows outside the shard stay zero)
+  GemmArgs rd = routed_down_args(d, wt, q4k, d.E, offsets, perm, 1, h, w_recv, out, err);
+  rd.epi = kEpiSlotStore;
+  return grouped_gemm(rd, s, num_sms);
 }
 
 size_t ep_combine_scratch_bytes(const LayerDims &d, int T) {
@@ -1001,7 +1053,7 @@ cudaError_t permute(const int32_t *idx, int T, int k, int E, int32_t *offsets, i
   // the counts are written into offsets[0..E) and scanned in place
   const int n = T * k;
   k_perm_count<<<E, 256, 0, s>>>(idx, n, offsets);
-  k_perm_scan<<<1, 32, 0, s>>>(offsets, E, offsets);
+  k_perm_scan<<<1, kMaxE, 0, s>>>(offsets, E, offsets);
   k_perm_scatter<<<E, 256, 0, s>>>(idx, n, offsets, perm);
   return cudaGetLastError();
 }

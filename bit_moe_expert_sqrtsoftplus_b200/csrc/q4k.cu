@@ -7,9 +7,8 @@
 //   y[t] = shared(x̂[t]) + sum_i w[t][i] * E_idx[t][i](x̂[t])   (+ x[t] with the
 //   pre-norm residual), E(v) = W_down (SiLU(W_gate v) * (W_up v))
 // with fp32 dot products over blocks decoded in registers: one warp per
-// output row (gate and up rows of a pair together; all k routed down rows of
-// a token together), three launches, no tensor cores; its arithmetic is exact
-// decoding and fp32 accumulation.
+// output row (gate and up rows of a pair read together), three launches, no
+// tensor cores; its arithmetic is exact decoding and fp32 accumulation.
 //
 // Q4_K block (144 bytes, 256 values; "2bit 量子化はなぜ「冗談ではない」のか",
 // section 3 type table; layout read as the public GGUF block): f16 d at 0,
@@ -175,44 +174,39 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
   }
 }
 
-// y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i]:
-// one warp per output row; the routed rows of the token's k pairs are read
-// block by block together (k rows' loads of a block in flight at once), each
-// lane weighting its parts by w in the routing's ascending expert order
-// before one reduction over the warp.
+// Lane l's part of sum_k W[row][k] v[k] over Q4_K blocks (K a multiple of
+// 256), several blocks' loads in flight.
+__device__ __forceinline__ float q4k_row_part(const uint8_t *row, const float *v, int K, const Q4kLane &L, int lane) {
+  float part = 0.0f;
+#pragma unroll 4
+  for (int b = 0; b < K / 256; ++b) {
+    const uint4 hd = *reinterpret_cast<const uint4 *>(row + (size_t)b * 144);
+    const uint2 cw = *reinterpret_cast<const uint2 *>(row + (size_t)b * 144 + L.code_off);
+    float xs[8], sx;
+    load8(v + 256 * b + 8 * lane, xs, sx);
+    part += q4k_part(hd, cw, L, xs, sx);
+  }
+  return part;
+}
+
+// y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i],
+// the routed terms in the routing's ascending expert order; one warp per
+// output row, one dot product after the other.  (Reading the k routed rows
+// block by block together measured slower: 68 against 44 us per launch at
+// one token.)
 __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31, r = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5), t = blockIdx.y;
   if (r >= d.H) return;
   const size_t rbs = (size_t)(d.Is / 32) * 34, rbd = (size_t)(d.I / 256) * 144;
-  const uint8_t *row[kMaxK];
-  float wt[kMaxK];
-#pragma unroll
-  for (int i = 0; i < kMaxK; ++i) {
-    const int e = i < d.k ? a.idx[t * d.k + i] : -1;
-    const bool ok = e >= 0 && e < d.E;
-    row[i] = ok ? a.down + ((size_t)e * d.H + r) * rbd : nullptr;
-    wt[i] = ok ? a.w[t * d.k + i] : 0.0f;
-  }
   const Q4kLane L(lane);
-  float part[kMaxK];
-#pragma unroll
-  for (int i = 0; i < kMaxK; ++i) part[i] = 0.0f;
-  for (int b = 0; b < d.I / 256; ++b) {
-#pragma unroll
-    for (int i = 0; i < kMaxK; ++i) {
-      if (!row[i]) continue;
-      const uint4 hd = *reinterpret_cast<const uint4 *>(row[i] + (size_t)b * 144);
-      const uint2 cw = *reinterpret_cast<const uint2 *>(row[i] + (size_t)b * 144 + L.code_off);
-      float xs[8], sx;
-      load8(a.h + (size_t)(t * d.k + i) * d.I + 256 * b + 8 * lane, xs, sx);
-      part[i] += q4k_part(hd, cw, L, xs, sx);
-    }
+  float acc = warp_sum(q80_part(a.sh_down + (size_t)r * rbs, a.hs + (size_t)t * d.Is, d.Is, lane));
+  for (int i = 0; i < d.k; ++i) {
+    const int p = t * d.k + i, e = a.idx[p];
+    if (e < 0 || e >= d.E) continue;
+    const float o = warp_sum(q4k_row_part(a.down + ((size_t)e * d.H + r) * rbd, a.h + (size_t)p * d.I, d.I, L, lane));
+    acc = fmaf(a.w[p], o, acc);
   }
-  float acc = q80_part(a.sh_down + (size_t)r * rbs, a.hs + (size_t)t * d.Is, d.Is, lane);
-#pragma unroll
-  for (int i = 0; i < kMaxK; ++i) acc = fmaf(wt[i], part[i], acc);
-  acc = warp_sum(acc);
   if (lane == 0) {
     const size_t at = (size_t)t * d.H + r;
     a.y[at] = (d.flags & MOE_FLAG_PRENORM_RESIDUAL) ? a.x[at] + acc : acc;
