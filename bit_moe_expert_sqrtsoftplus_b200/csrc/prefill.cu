@@ -56,9 +56,13 @@ __global__ void k_row_norms(const uint16_t *Wr, int E, int H, float *out) {
 __global__ void k_token_norms(const float *x, int T, int H, int flags, float eps, double *inv, double *nrm) {
   const int t = blockIdx.x;
   double ss = 0.0;
-  for (int j = threadIdx.x; j < H; j += blockDim.x) {
-    double v = x[(size_t)t * H + j];
-    ss += v * v;
+  // 16-byte loads (H is a multiple of 256 and rows are 16-byte aligned), four in flight per thread
+  const float4 *x4 = reinterpret_cast<const float4 *>(x + (size_t)t * H);
+#pragma unroll 4
+  for (int j = threadIdx.x; j < H / 4; j += blockDim.x) {
+    const float4 v = x4[j];
+    ss += (double)v.x * (double)v.x + (double)v.y * (double)v.y + (double)v.z * (double)v.z +
+          (double)v.w * (double)v.w;
   }
   ss = warp_sum_d(ss);
   __shared__ double red[32];
@@ -79,7 +83,8 @@ __global__ void k_token_norms(const float *x, int T, int H, int flags, float eps
 // error bound below assumes), added to an fp64 accumulator; the tile shape
 // does not change any output's arithmetic.  Rows are staged with 16-byte
 // loads (x scaled by the token's fp32 inverse RMS, W_r converted from f16),
-// transposed into K-major shared tiles.
+// transposed into K-major shared tiles; the next chunk's loads are in flight
+// while the current one is multiplied.
 constexpr int RT = 64, RE = 64, RK = 32;
 __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double *inv, const uint16_t *Wr, int T,
                                                     int E, int H, double *z) {
@@ -89,26 +94,40 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;  // experts tx*4 .., tokens ty*4 ..
   // staging roles: x float4 pieces (token i>>3, K quad i&7) for i = tid and
-  // tid + 256, and one W uint4 piece (expert tid>>2, K octet tid&3)
+  // tid + 256, and one W uint4 piece (expert tid>>2, K octet tid&3); the
+  // pieces of chunk k0 + RK are loaded into registers while chunk k0 is
+  // multiplied
   float invf[2];
+  const float *xrow[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int t = t0 + ((tid + 256 * r) >> 3);
+    const int i = tid + 256 * r;
+    const int t = t0 + (i >> 3);
     invf[r] = t < T ? (float)inv[t] : 0.f;
+    xrow[r] = t < T ? x + (size_t)t * H + 4 * (i & 7) : nullptr;
   }
+  const int we = e0 + (tid >> 2);
+  const uint16_t *wrow = we < E ? Wr + (size_t)we * H + 8 * (tid & 3) : nullptr;
+  float4 xv_next[2];
+  uint4 wv_next;
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+      xv_next[r] = xrow[r] ? *reinterpret_cast<const float4 *>(xrow[r] + k0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv_next = wrow ? *reinterpret_cast<const uint4 *>(wrow + k0) : make_uint4(0u, 0u, 0u, 0u);
+  };
   double acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  fetch(0);
   for (int k0 = 0; k0 < H; k0 += RK) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int i = tid + 256 * r;
       const int tt = i >> 3, kq = i & 7;
-      const int t = t0 + tt;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < T) v = *reinterpret_cast<const float4 *>(x + (size_t)t * H + k0 + 4 * kq);
+      const float4 v = xv_next[r];
       xs[4 * kq + 0][tt] = v.x * invf[r];
       xs[4 * kq + 1][tt] = v.y * invf[r];
       xs[4 * kq + 2][tt] = v.z * invf[r];
@@ -116,10 +135,7 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
     }
     {
       const int ee = tid >> 2, ko = tid & 3;
-      const int e = e0 + ee;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (e < E) v = *reinterpret_cast<const uint4 *>(Wr + (size_t)e * H + k0 + 8 * ko);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      const uint32_t w4[4] = {wv_next.x, wv_next.y, wv_next.z, wv_next.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         ws[8 * ko + 2 * q][ee] = half_bits_to_float((uint16_t)(w4[q] & 0xFFFFu));
@@ -127,6 +143,7 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
       }
     }
     __syncthreads();
+    if (k0 + RK < H) fetch(k0 + RK);
     float part[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -179,18 +196,16 @@ __global__ void k_topk_cert(const double *z, const float *bias, const float *wn,
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   const double *zt = z + (size_t)t * E;
-  double key[8], lo[8], hi[8];
+  double key[8], dzs[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      const double b = (double)bias[e];
-      const double dz = logit_bound(wn[e], xn[t]);
-      key[i] = sqrtsoftplus(zt[e]) + b;
-      lo[i] = sqrtsoftplus(zt[e] - dz) + b - 1e-12;
-      hi[i] = sqrtsoftplus(zt[e] + dz) + b + 1e-12;
+      dzs[i] = logit_bound(wn[e], xn[t]);
+      key[i] = sqrtsoftplus(zt[e]) + (double)bias[e];
     } else {
-      key[i] = lo[i] = hi[i] = -DBL_MAX;
+      key[i] = -DBL_MAX;
+      dzs[i] = 0.0;
     }
   }
   unsigned taken = 0;
@@ -222,21 +237,48 @@ __global__ void k_topk_cert(const double *z, const float *bias, const float *wn,
       sel[r] = be;
     }
   }
-  // certificate: min lower end of the selected vs max upper end of the rest
+  // certificate: min lower end of the selected vs max upper end of the rest.
+  // sqrt(softplus) has slope below 0.71 everywhere, so key -/+ dz (plus the
+  // fp64 slack) bound an expert's interval; the exact ends
+  // sqrtsoftplus(z -/+ dz) are evaluated only for experts whose coarse
+  // bound does not settle the comparison, which certifies the same tokens.
   double sel_lo = DBL_MAX, rest_hi = -DBL_MAX;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
     if (e >= E) continue;
     if ((taken >> i) & 1u)
-      sel_lo = fmin(sel_lo, lo[i]);
+      sel_lo = fmin(sel_lo, key[i] - dzs[i] - 2e-12);
     else
-      rest_hi = fmax(rest_hi, hi[i]);
+      rest_hi = fmax(rest_hi, key[i] + dzs[i] + 2e-12);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     sel_lo = fmin(sel_lo, __shfl_xor_sync(0xffffffffu, sel_lo, o));
     rest_hi = fmax(rest_hi, __shfl_xor_sync(0xffffffffu, rest_hi, o));
+  }
+  if (!(sel_lo > rest_hi)) {
+    const double coarse_lo = sel_lo, coarse_hi = rest_hi;
+    sel_lo = DBL_MAX;
+    rest_hi = -DBL_MAX;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e >= E) continue;
+      const double b = (double)bias[e];
+      if ((taken >> i) & 1u) {
+        const double c = key[i] - dzs[i] - 2e-12;
+        sel_lo = fmin(sel_lo, c > coarse_hi ? c : sqrtsoftplus(zt[e] - dzs[i]) + b - 1e-12);
+      } else {
+        const double c = key[i] + dzs[i] + 2e-12;
+        rest_hi = fmax(rest_hi, c < coarse_lo ? c : sqrtsoftplus(zt[e] + dzs[i]) + b + 1e-12);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sel_lo = fmin(sel_lo, __shfl_xor_sync(0xffffffffu, sel_lo, o));
+      rest_hi = fmax(rest_hi, __shfl_xor_sync(0xffffffffu, rest_hi, o));
+    }
   }
   const bool certified = (k == E) || sel_lo > rest_hi;
   if (lane != 0) return;
