@@ -357,11 +357,13 @@ static cudaError_t q4k_forward(moe_handle *h, const float *x, const int32_t *tok
   q.y = y;
   q.idx = idx;
   q.w = w;
-  q.xn = reinterpret_cast<float *>(base + off);
-  off += align256(sizeof(float) * (size_t)T * h->d.H);
   q.h = reinterpret_cast<float *>(base + off);
   off += align256(sizeof(float) * (size_t)T * h->d.k * h->d.I);
   q.hs = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * (size_t)T * h->d.Is);
+  q.xsum = reinterpret_cast<float *>(base + off);
+  q.xq = a.s.xq;
+  q.xs = a.s.xs;
   if (h->ev_begin) cudaEventRecord(h->ev_begin, s);
   e = moe::q4k_experts(q, s);
   if (h->ev_end) cudaEventRecord(h->ev_end, s);

@@ -6,9 +6,13 @@
 // (idx, w) and computes
 //   y[t] = shared(x̂[t]) + sum_i w[t][i] * E_idx[t][i](x̂[t])   (+ x[t] with the
 //   pre-norm residual), E(v) = W_down (SiLU(W_gate v) * (W_up v))
-// with fp32 dot products over blocks decoded in registers: one warp per
-// output row (gate and up rows of a pair read together), three launches, no
-// tensor cores; its arithmetic is exact decoding and fp32 accumulation.
+// with one warp per output row (gate and up rows of a pair read together),
+// three launches, no tensor cores.  Gate/up take the expert input as the three
+// int8 limbs the small-token router kernel makes (within 6e-8 of max|x|):
+// sum q * x per sub-block is exact in int32 (dp4a), the min term uses the
+// fp32 sum of x over the sub-block.  Down takes h in fp32 (codes converted
+// exactly, fp32 FMAs, lane l on values 8l .. 8l+7 of every block).  Both
+// decode exactly and accumulate in fp32.
 //
 // Q4_K block (144 bytes, 256 values; "2bit 量子化はなぜ「冗談ではない」のか",
 // section 3 type table; layout read as the public GGUF block): f16 d at 0,
@@ -18,9 +22,7 @@
 // scale byte j+4 plus the top two bits of scale byte j-4 as bits 4-5, min =
 // high nibble of scale byte j+4 plus the top two bits of scale byte j.  The
 // code of value e is nibble (e%64)/32 of code byte 32*(e/64) + e%32.  Value =
-// d*scale*q - dmin*min.  Lane l of a warp takes values 8l .. 8l+7 of each
-// block: sub-block l/4, eight consecutive code bytes at 32*(l/8) + 8*(l%4),
-// nibble (l%8)/4.
+// d*scale*q - dmin*min.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -106,9 +108,119 @@ __device__ __forceinline__ float q80_part(const uint8_t *row, const float *v, in
   return part;
 }
 
-// xn[t] = x[t], or x[t] / sqrt(mean(x[t]^2) + eps) with the pre-norm residual.
+// Scale step d*scale and offset dmin*min of sub-block j (0..7) of a Q4_K
+// block whose first 16 bytes are hd.
+__device__ __forceinline__ void q4k_sc_mn(const uint4 hd, int j, float &dsc, float &dmn) {
+  const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
+  const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
+  const int jj = j & 3;
+  int sc, mn;
+  if (j < 4) {
+    sc = (int)((hd.y >> (8 * jj)) & 63u);
+    mn = (int)((hd.z >> (8 * jj)) & 63u);
+  } else {
+    const uint32_t lowb = (hd.w >> (8 * jj)) & 255u;
+    sc = (int)((lowb & 15u) | (((hd.y >> (8 * jj + 6)) & 3u) << 4));
+    mn = (int)((lowb >> 4) | (((hd.z >> (8 * jj + 6)) & 3u) << 4));
+  }
+  dsc = d * (float)sc;
+  dmn = dmin * (float)mn;
+}
+
+// Sub-block j of a Q4_K block holds values 32j .. 32j+31: the low (j even) or
+// high (j odd) nibbles of the 32 code bytes at 16 + 32 * (j/2).  In the
+// routines below lane l takes sub-block l%8 of the blocks l/8, l/8 + 4, ...
+// of a row.
+__device__ __forceinline__ void q4k_codes(const uint8_t *blk, int j, uint32_t (&qn)[8]) {
+  const uint4 c0 = *reinterpret_cast<const uint4 *>(blk + 16 + 32 * (j >> 1));
+  const uint4 c1 = *reinterpret_cast<const uint4 *>(blk + 32 + 32 * (j >> 1));
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const int shift = 4 * (j & 1);
+#pragma unroll
+  for (int w = 0; w < 8; ++w) qn[w] = (cw[w] >> shift) & 0x0F0F0F0Fu;  // four codes 0..15 as bytes
+}
+
+// The expert input as three int8 limbs (x = s1 q1 + s2 q2 + s3 q3 per value,
+// the small-token path's representation, within 6e-8 of max|x|): lane l's
+// part of the gate and up rows' dot products, sum q * x exact in int32 by
+// dp4a per limb, the min term from the fp32 sum S of x over the sub-block.
+__device__ __forceinline__ void q4k_pair_part_limbs(const uint8_t *gr, const uint8_t *ur, const int8_t *xq, int H,
+                                                    const float (&s)[3], const float *S, int lane, float &pg,
+                                                    float &pu) {
+  const int j = lane & 7;
+  for (int b = lane >> 3; b < H / 256; b += 4) {
+    const int sb = 8 * b + j;  // sub-block of the row
+    uint32_t x[3][8];
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      const uint4 *xl = reinterpret_cast<const uint4 *>(xq + (size_t)l * H + 32 * sb);
+      const uint4 a = xl[0], c = xl[1];
+      x[l][0] = a.x, x[l][1] = a.y, x[l][2] = a.z, x[l][3] = a.w;
+      x[l][4] = c.x, x[l][5] = c.y, x[l][6] = c.z, x[l][7] = c.w;
+    }
+    const float sx = S[sb];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint8_t *blk = (m ? ur : gr) + (size_t)b * 144;
+      const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+      uint32_t qn[8];
+      q4k_codes(blk, j, qn);
+      int acc[3] = {0, 0, 0};
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+#pragma unroll
+        for (int l = 0; l < 3; ++l) acc[l] = __dp4a((int)qn[w], (int)x[l][w], acc[l]);
+      float dsc, dmn;
+      q4k_sc_mn(hd, j, dsc, dmn);
+      const float f = fmaf(s[0], (float)acc[0], fmaf(s[1], (float)acc[1], s[2] * (float)acc[2]));
+      float &pp = m ? pu : pg;
+      pp = fmaf(dsc, f, fmaf(-dmn, sx, pp));
+    }
+  }
+}
+
+// Lane l's part of a Q8_0 row's dot product with the expert input's int8
+// limbs: lane l takes the 32-value blocks l, l + 32, ...; sum q * x per block
+// exact in int32 (dp4a per limb).  A block's codes start 2 bytes into it, so
+// they are 4-byte aligned when its index is odd and otherwise read as the
+// aligned words around them (the last as 16 bits, to stay in the block).
+__device__ __forceinline__ float q80_row_part_limbs(const uint8_t *row, const int8_t *xq, int H,
+                                                    const float (&s)[3], int lane) {
+  float part = 0.0f;
+  for (int b = lane; b < H / 32; b += 32) {
+    const uint8_t *blk = row + (size_t)b * 34;
+    const float d = f16_at(blk);
+    uint32_t q[8];
+    if ((reinterpret_cast<uintptr_t>(blk + 2) & 3u) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = *reinterpret_cast<const uint32_t *>(blk + 2 + 4 * i);
+    } else {
+      uint32_t u[9];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[i] = *reinterpret_cast<const uint32_t *>(blk + 4 * i);
+      u[8] = *reinterpret_cast<const uint16_t *>(blk + 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = __byte_perm(u[i], u[i + 1], 0x5432);
+    }
+    int acc[3] = {0, 0, 0};
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      const uint4 *xl = reinterpret_cast<const uint4 *>(xq + (size_t)l * H + 32 * b);
+      const uint4 a = xl[0], c = xl[1];
+      const uint32_t xw[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int w = 0; w < 8; ++w) acc[l] = __dp4a((int)q[w], (int)xw[w], acc[l]);
+    }
+    part = fmaf(d, fmaf(s[0], (float)acc[0], fmaf(s[1], (float)acc[1], s[2] * (float)acc[2])), part);
+  }
+  return part;
+}
+
+// Per token: the sums of the expert input xhat = x (or x / sqrt(mean(x^2) + eps)
+// with the pre-norm residual) over each 32-value sub-block, for the min
+// terms of the Q4_K gate/up rows.
 __global__ void __launch_bounds__(256) k_q4k_input(const float *__restrict__ x, int H, int flags, float eps,
-                                                   float *__restrict__ xn) {
+                                                   float *__restrict__ xsum) {
   __shared__ double red[8];
   __shared__ float inv_s;
   const int t = blockIdx.x, tid = threadIdx.x;
@@ -128,7 +240,21 @@ __global__ void __launch_bounds__(256) k_q4k_input(const float *__restrict__ x, 
     __syncthreads();
     inv = inv_s;
   }
-  for (int c = tid; c < H; c += 256) xn[(size_t)t * H + c] = xt[c] * inv;
+  // two threads per sub-block, 16 values each
+  for (int base = 0; base < H / 16; base += 256) {  // the same trip count in every thread
+    const int h2 = base + tid;
+    float acc = 0.0f;
+    if (h2 < H / 16) {
+      const float4 *x4 = reinterpret_cast<const float4 *>(xt + 16 * h2);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = x4[i];
+        acc += ((v.x * inv + v.y * inv) + (v.z * inv + v.w * inv));
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (h2 < H / 16 && (h2 & 1) == 0) xsum[(size_t)t * (H / 32) + (h2 >> 1)] = acc;
+  }
 }
 
 // Blocks (row tile, p): p < T*k is the routed pair p (Q4_K gate/up rows of
@@ -142,24 +268,13 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
     const int t = p / d.k, e = a.idx[p];
     float hv = 0.0f;
     if (e >= 0 && e < d.E) {
-      // gate and up rows of the pair together: both rows' loads of a block
-      // are in flight at once, and the x values and their sum serve both
+      // gate and up rows of the pair together, on the input's int8 limbs
       const size_t rb = (size_t)(d.H / 256) * 144;
       const uint8_t *gr = a.gate + ((size_t)e * d.I + row) * rb, *ur = a.up + ((size_t)e * d.I + row) * rb;
-      const float *xt = a.xn + (size_t)t * d.H;
-      const Q4kLane L(lane);
+      const float sc[3] = {a.xs[4 * t], a.xs[4 * t + 1], a.xs[4 * t + 2]};
       float pg = 0.0f, pu = 0.0f;
-#pragma unroll 4
-      for (int b = 0; b < d.H / 256; ++b) {
-        const uint4 hg = *reinterpret_cast<const uint4 *>(gr + (size_t)b * 144);
-        const uint4 hu = *reinterpret_cast<const uint4 *>(ur + (size_t)b * 144);
-        const uint2 cg = *reinterpret_cast<const uint2 *>(gr + (size_t)b * 144 + L.code_off);
-        const uint2 cu = *reinterpret_cast<const uint2 *>(ur + (size_t)b * 144 + L.code_off);
-        float xs[8], sx;
-        load8(xt + 256 * b + 8 * lane, xs, sx);
-        pg += q4k_part(hg, cg, L, xs, sx);
-        pu += q4k_part(hu, cu, L, xs, sx);
-      }
+      q4k_pair_part_limbs(gr, ur, a.xq + (size_t)t * 3 * d.H, d.H, sc, a.xsum + (size_t)t * (d.H / 32), lane, pg,
+                          pu);
       hv = silu(warp_sum(pg)) * warp_sum(pu);
     }
     if (lane == 0) a.h[(size_t)p * d.I + row] = hv;
@@ -167,9 +282,10 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
     if (row >= d.Is) return;
     const int t = p - npairs;
     const size_t rb = (size_t)(d.H / 32) * 34;
-    const float *xt = a.xn + (size_t)t * d.H;
-    const float g = warp_sum(q80_part(a.sh_gate + (size_t)row * rb, xt, d.H, lane));
-    const float u = warp_sum(q80_part(a.sh_up + (size_t)row * rb, xt, d.H, lane));
+    const int8_t *xq = a.xq + (size_t)t * 3 * d.H;
+    const float sc[3] = {a.xs[4 * t], a.xs[4 * t + 1], a.xs[4 * t + 2]};
+    const float g = warp_sum(q80_row_part_limbs(a.sh_gate + (size_t)row * rb, xq, d.H, sc, lane));
+    const float u = warp_sum(q80_row_part_limbs(a.sh_up + (size_t)row * rb, xq, d.H, sc, lane));
     if (lane == 0) a.hs[(size_t)t * d.Is + row] = silu(g) * u;
   }
 }
@@ -191,9 +307,9 @@ __device__ __forceinline__ float q4k_row_part(const uint8_t *row, const float *v
 
 // y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i],
 // the routed terms in the routing's ascending expert order; one warp per
-// output row, one dot product after the other.  (Reading the k routed rows
-// block by block together measured slower: 68 against 44 us per launch at
-// one token.)
+// output row, one dot product after the other.  (Measured slower at one
+// token: reading the k routed rows block by block together, 68 against 43 us
+// per launch; one block per output row with a warp per dot product, 48 us.)
 __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31, r = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5), t = blockIdx.y;
@@ -217,14 +333,14 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) 
 
 size_t q4k_expert_bytes(const LayerDims &d, int T) {
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
-  return al(sizeof(float) * (size_t)T * d.H) + al(sizeof(float) * (size_t)T * d.k * d.I) +
-         al(sizeof(float) * (size_t)T * d.Is);
+  return al(sizeof(float) * (size_t)T * d.k * d.I) + al(sizeof(float) * (size_t)T * d.Is) +
+         al(sizeof(float) * (size_t)T * (d.H / 32));
 }
 
 cudaError_t q4k_experts(const Q4kArgs &a, cudaStream_t stream) {
   const LayerDims &d = a.d;
   if (a.T <= 0) return cudaSuccess;
-  k_q4k_input<<<a.T, 256, 0, stream>>>(a.x, d.H, d.flags, d.eps, a.xn);
+  k_q4k_input<<<a.T, 256, 0, stream>>>(a.x, d.H, d.flags, d.eps, a.xsum);
   const int rmax = d.I > d.Is ? d.I : d.Is;
   k_q4k_gate_up<<<dim3((rmax + kRowsPerCta - 1) / kRowsPerCta, a.T * d.k + a.T), kRowsPerCta * 32, 0, stream>>>(a);
   k_q4k_down<<<dim3((d.H + kRowsPerCta - 1) / kRowsPerCta, a.T), kRowsPerCta * 32, 0, stream>>>(a);

@@ -19,12 +19,14 @@ struct Q4kArgs {
   float *y;        // [T][H]; may alias x with MOE_FLAG_PRENORM_RESIDUAL
   const int32_t *idx;  // [T][k] ascending expert ids
   const float *w;      // [T][k]
-  float *xn;           // [T][H] scratch: the expert input (x, or RMSNorm(x))
   float *h;            // [T*k][I] scratch: routed SwiGLU outputs
   float *hs;           // [T][Is] scratch: shared SwiGLU outputs
+  float *xsum;         // [T][H/32] scratch: sums of the expert input over each 32-value sub-block
+  const int8_t *xq;    // [T][3][H] int8 limbs of the expert input (the small-token router kernel's)
+  const float *xs;     // [T][4] limb scales
 };
 
-// Scratch the expert kernels take beside the routing scratch (xn, h, hs).
+// Scratch the expert kernels take beside the routing scratch (h, hs, xsum).
 size_t q4k_expert_bytes(const LayerDims &d, int T);
 
 // The expert work of one call, after the routing (idx, w) is in place:
