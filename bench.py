@@ -429,9 +429,9 @@ def run_ours(args, world, rank):
         # batched: router (4), permutation (3), input, 4 GEMMs, from 257 tokens
         # the 3 expansions of the shared expert's rows, and with the
         # deterministic flag the slot sum; small-token: k1 and k2, or for Q4_K
-        # layers k1, the routing kernel and the 3 expert kernels
+        # layers k1, the routing kernel and the 4 expert kernels
         "gpu_launches": ((15 if T >= 257 else 12) + (1 if args.deterministic else 0) if large else
-                         5 if s.q4k else 2) * args.steps,
+                         6 if s.q4k else 2) * args.steps,
         "clocks": clocks,
     }
     return out
@@ -541,7 +541,7 @@ def run_stack(args, world, rank):
                      "peak_source": peaks["source"], "algorithmic_bytes_per_step": nd_bytes},
         "e2e": {"value": job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * s.hidden * 4, "d2h_bytes_per_step": T * s.hidden * 4},
-        "gpu_launches": (2 * (s.layers - s.q4k_layers) + 5 * s.q4k_layers) * args.steps,
+        "gpu_launches": (2 * (s.layers - s.q4k_layers) + 6 * s.q4k_layers) * args.steps,
         "clocks": clock.summary(),
     }
 

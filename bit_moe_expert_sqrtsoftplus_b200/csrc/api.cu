@@ -362,6 +362,13 @@ static cudaError_t q4k_forward(moe_handle *h, const float *x, const int32_t *tok
   q.hs = reinterpret_cast<float *>(base + off);
   off += align256(sizeof(float) * (size_t)T * h->d.Is);
   q.xsum = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * (size_t)T * (h->d.H / 32));
+  const size_t nh = (size_t)T * h->d.k * h->d.I + (size_t)T * h->d.Is;
+  q.hq = reinterpret_cast<int8_t *>(base + off);
+  off += align256(3 * nh);
+  q.hqs = reinterpret_cast<float *>(base + off);
+  off += align256(sizeof(float) * 4 * ((size_t)T * h->d.k + T));
+  q.hsum = reinterpret_cast<float *>(base + off);
   q.xq = a.s.xq;
   q.xs = a.s.xs;
   if (h->ev_begin) cudaEventRecord(h->ev_begin, s);

@@ -7,12 +7,12 @@
 //   y[t] = shared(x̂[t]) + sum_i w[t][i] * E_idx[t][i](x̂[t])   (+ x[t] with the
 //   pre-norm residual), E(v) = W_down (SiLU(W_gate v) * (W_up v))
 // with one warp per output row (gate and up rows of a pair read together),
-// three launches, no tensor cores.  Gate/up take the expert input as the three
-// int8 limbs the small-token router kernel makes (within 6e-8 of max|x|):
-// sum q * x per sub-block is exact in int32 (dp4a), the min term uses the
-// fp32 sum of x over the sub-block.  Down takes h in fp32 (codes converted
-// exactly, fp32 FMAs, lane l on values 8l .. 8l+7 of every block).  Both
-// decode exactly and accumulate in fp32.
+// four launches, no tensor cores.  Every product takes its input vector as
+// three int8 limbs (within 6e-8 of its max |value|: the expert input's from
+// the small-token router kernel, h's and hs's from a kernel of their own):
+// sum q * v per 32-value block is exact in int32 (dp4a), and the Q4_K min
+// term uses the fp32 sum of v over the sub-block.  Decoding is exact and the
+// sums over blocks are fp32.
 //
 // Q4_K block (144 bytes, 256 values; "2bit 量子化はなぜ「冗談ではない」のか",
 // section 3 type table; layout read as the public GGUF block): f16 d at 0,
@@ -41,71 +41,10 @@ __device__ __forceinline__ float f16_at(const uint8_t *p) {
   return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(p)));
 }
 
-// Lane l's share of a Q4_K block: values 8l .. 8l+7, i.e. sub-block l/4,
-// code bytes 32*(l/8) + 8*(l%4) .. +7, nibble (l%8)/4.
-struct Q4kLane {
-  int j, jj, code_off, shift;
-  __device__ explicit Q4kLane(int lane)
-      : j(lane >> 2), jj((lane >> 2) & 3), code_off(16 + 32 * (lane >> 3) + 8 * (lane & 3)),
-        shift(4 * ((lane & 7) >> 2)) {}
-};
-
-// Lane l's part of one block's dot product with its 8 values xs of v:
-// d*scale*sum(q*x) - dmin*min*sum(x), sx = sum(x) given.
-__device__ __forceinline__ float q4k_part(const uint4 hd, const uint2 cw, const Q4kLane &L, const float (&xs)[8],
-                                          float sx) {
-  const float d = __half2float(__ushort_as_half((uint16_t)(hd.x & 0xffffu)));
-  const float dmin = __half2float(__ushort_as_half((uint16_t)(hd.x >> 16)));
-  const uint32_t b03 = hd.y, b47 = hd.z, b811 = hd.w;  // scale bytes 0-3, 4-7, 8-11
-  int sc, mn;
-  if (L.j < 4) {
-    sc = (int)((b03 >> (8 * L.jj)) & 63u);
-    mn = (int)((b47 >> (8 * L.jj)) & 63u);
-  } else {
-    const uint32_t lowb = (b811 >> (8 * L.jj)) & 255u;
-    sc = (int)((lowb & 15u) | (((b03 >> (8 * L.jj + 6)) & 3u) << 4));
-    mn = (int)((lowb >> 4) | (((b47 >> (8 * L.jj + 6)) & 3u) << 4));
-  }
-  float sqx = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 255u;
-    sqx = fmaf((float)((byte >> L.shift) & 15u), xs[k], sqx);
-  }
-  return d * (float)sc * sqx - dmin * (float)mn * sx;
-}
-
-__device__ __forceinline__ void load8(const float *v, float (&xs)[8], float &sx) {
-  const float4 a = reinterpret_cast<const float4 *>(v)[0], b = reinterpret_cast<const float4 *>(v)[1];
-  xs[0] = a.x, xs[1] = a.y, xs[2] = a.z, xs[3] = a.w, xs[4] = b.x, xs[5] = b.y, xs[6] = b.z, xs[7] = b.w;
-  sx = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-// Lane l's part of sum_k W[row][k] v[k] over Q8_0 blocks (K a multiple of
-// 128): per iteration the warp takes four blocks, lane l the values
-// 4*(l%8) .. +3 of block l/8 of them (two 16-bit loads: blocks are 34 bytes,
-// so their quants are 2-byte aligned).
-__device__ __forceinline__ float q80_part(const uint8_t *row, const float *v, int K, int lane) {
-  const int sub = lane >> 3, q4 = 4 * (lane & 7);
-  float part = 0.0f;
-#pragma unroll 4
-  for (int b = sub; b < K / 32; b += 4) {
-    const uint8_t *blk = row + (size_t)b * 34;
-    const float d = f16_at(blk);
-    const uint32_t lo = *reinterpret_cast<const uint16_t *>(blk + 2 + q4);
-    const uint32_t hi = *reinterpret_cast<const uint16_t *>(blk + 4 + q4);
-    const float4 x = *reinterpret_cast<const float4 *>(v + 32 * b + q4);
-    const float s = (float)(int8_t)(lo & 255u) * x.x + (float)(int8_t)(lo >> 8) * x.y +
-                    (float)(int8_t)(hi & 255u) * x.z + (float)(int8_t)(hi >> 8) * x.w;
-    part = fmaf(d, s, part);
-  }
-  return part;
 }
 
 // Scale step d*scale and offset dmin*min of sub-block j (0..7) of a Q4_K
@@ -140,28 +79,28 @@ __device__ __forceinline__ void q4k_codes(const uint8_t *blk, int j, uint32_t (&
   for (int w = 0; w < 8; ++w) qn[w] = (cw[w] >> shift) & 0x0F0F0F0Fu;  // four codes 0..15 as bytes
 }
 
-// The expert input as three int8 limbs (x = s1 q1 + s2 q2 + s3 q3 per value,
-// the small-token path's representation, within 6e-8 of max|x|): lane l's
-// part of the gate and up rows' dot products, sum q * x exact in int32 by
-// dp4a per limb, the min term from the fp32 sum S of x over the sub-block.
-__device__ __forceinline__ void q4k_pair_part_limbs(const uint8_t *gr, const uint8_t *ur, const int8_t *xq, int H,
-                                                    const float (&s)[3], const float *S, int lane, float &pg,
-                                                    float &pu) {
+// A vector v as three int8 limbs (v = s1 q1 + s2 q2 + s3 q3 per value, the
+// small-token path's representation, within 6e-8 of max|v|): lane l's part of
+// the dot products of NR Q4_K rows with v, sum q * v exact in int32 by dp4a
+// per limb, the min term from the fp32 sum S of v over the sub-block.
+template <int NR>
+__device__ __forceinline__ void q4k_rows_part_limbs(const uint8_t *const (&rows)[NR], const int8_t *vq, int K,
+                                                    const float (&s)[3], const float *S, int lane, float (&part)[NR]) {
   const int j = lane & 7;
-  for (int b = lane >> 3; b < H / 256; b += 4) {
+  for (int b = lane >> 3; b < K / 256; b += 4) {
     const int sb = 8 * b + j;  // sub-block of the row
     uint32_t x[3][8];
 #pragma unroll
     for (int l = 0; l < 3; ++l) {
-      const uint4 *xl = reinterpret_cast<const uint4 *>(xq + (size_t)l * H + 32 * sb);
+      const uint4 *xl = reinterpret_cast<const uint4 *>(vq + (size_t)l * K + 32 * sb);
       const uint4 a = xl[0], c = xl[1];
       x[l][0] = a.x, x[l][1] = a.y, x[l][2] = a.z, x[l][3] = a.w;
       x[l][4] = c.x, x[l][5] = c.y, x[l][6] = c.z, x[l][7] = c.w;
     }
     const float sx = S[sb];
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const uint8_t *blk = (m ? ur : gr) + (size_t)b * 144;
+    for (int m = 0; m < NR; ++m) {
+      const uint8_t *blk = rows[m] + (size_t)b * 144;
       const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
       uint32_t qn[8];
       q4k_codes(blk, j, qn);
@@ -173,8 +112,7 @@ __device__ __forceinline__ void q4k_pair_part_limbs(const uint8_t *gr, const uin
       float dsc, dmn;
       q4k_sc_mn(hd, j, dsc, dmn);
       const float f = fmaf(s[0], (float)acc[0], fmaf(s[1], (float)acc[1], s[2] * (float)acc[2]));
-      float &pp = m ? pu : pg;
-      pp = fmaf(dsc, f, fmaf(-dmn, sx, pp));
+      part[m] = fmaf(dsc, f, fmaf(-dmn, sx, part[m]));
     }
   }
 }
@@ -272,10 +210,10 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
       const size_t rb = (size_t)(d.H / 256) * 144;
       const uint8_t *gr = a.gate + ((size_t)e * d.I + row) * rb, *ur = a.up + ((size_t)e * d.I + row) * rb;
       const float sc[3] = {a.xs[4 * t], a.xs[4 * t + 1], a.xs[4 * t + 2]};
-      float pg = 0.0f, pu = 0.0f;
-      q4k_pair_part_limbs(gr, ur, a.xq + (size_t)t * 3 * d.H, d.H, sc, a.xsum + (size_t)t * (d.H / 32), lane, pg,
-                          pu);
-      hv = silu(warp_sum(pg)) * warp_sum(pu);
+      const uint8_t *const rows[2] = {gr, ur};
+      float pp[2] = {0.0f, 0.0f};
+      q4k_rows_part_limbs<2>(rows, a.xq + (size_t)t * 3 * d.H, d.H, sc, a.xsum + (size_t)t * (d.H / 32), lane, pp);
+      hv = silu(warp_sum(pp[0])) * warp_sum(pp[1]);
     }
     if (lane == 0) a.h[(size_t)p * d.I + row] = hv;
   } else {
@@ -290,38 +228,94 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_gate_up(const Q4kArgs 
   }
 }
 
-// Lane l's part of sum_k W[row][k] v[k] over Q4_K blocks (K a multiple of
-// 256), several blocks' loads in flight.
-__device__ __forceinline__ float q4k_row_part(const uint8_t *row, const float *v, int K, const Q4kLane &L, int lane) {
-  float part = 0.0f;
-#pragma unroll 4
-  for (int b = 0; b < K / 256; ++b) {
-    const uint4 hd = *reinterpret_cast<const uint4 *>(row + (size_t)b * 144);
-    const uint2 cw = *reinterpret_cast<const uint2 *>(row + (size_t)b * 144 + L.code_off);
-    float xs[8], sx;
-    load8(v + 256 * b + 8 * lane, xs, sx);
-    part += q4k_part(hd, cw, L, xs, sx);
+// The down projection's inputs as int8 limbs: block v < T*k takes the routed
+// SwiGLU output h[v] (I values), block T*k + t the shared one hs[t] (Is
+// values): the vector's max |value| sets the limb scales (as for the expert
+// input), each value becomes three int8 limbs, and the fp32 sums over each
+// 32-value sub-block serve the min terms.
+__global__ void __launch_bounds__(256) k_q4k_hlimbs(const Q4kArgs a) {
+  const LayerDims &d = a.d;
+  const int v = blockIdx.x, npairs = a.T * d.k, tid = threadIdx.x;
+  const bool routed = v < npairs;
+  const int len = routed ? d.I : d.Is;
+  const float *src = routed ? a.h + (size_t)v * d.I : a.hs + (size_t)(v - npairs) * d.Is;
+  int8_t *q = a.hq + (routed ? (size_t)v * 3 * d.I : (size_t)npairs * 3 * d.I + (size_t)(v - npairs) * 3 * d.Is);
+  float *sum = a.hsum + (routed ? (size_t)v * (d.I / 32) : (size_t)npairs * (d.I / 32) + (size_t)(v - npairs) * (d.Is / 32));
+  __shared__ float red[8];
+  float amax = 0.0f;
+  for (int i = tid; i < len; i += 256) amax = fmaxf(amax, fabsf(src[i]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+  __syncthreads();
+  amax = 0.0f;
+  for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float s1 = amax > 0.f ? amax / 127.f : 1.f;
+  const float s2 = s1 / 254.f, s3 = s2 / 254.f;
+  const float r1 = 1.f / s1, r2 = 1.f / s2, r3 = 1.f / s3;
+  uint32_t *q32 = reinterpret_cast<uint32_t *>(q);
+  const int n4 = len / 4;
+  for (int j = tid; j < n4; j += 256) {
+    const float4 x4 = reinterpret_cast<const float4 *>(src)[j];
+    const float e[4] = {x4.x, x4.y, x4.z, x4.w};
+    uint32_t w1 = 0u, w2 = 0u, w3 = 0u;
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const float x = e[k4];
+      const float q1 = fminf(fmaxf(rintf(x * r1), -127.f), 127.f);
+      const float e1 = fmaf(-q1, s1, x);
+      const float q2 = fminf(fmaxf(rintf(e1 * r2), -127.f), 127.f);
+      const float e2 = fmaf(-q2, s2, e1);
+      const float q3 = fminf(fmaxf(rintf(e2 * r3), -127.f), 127.f);
+      w1 |= ((uint32_t)(int)q1 & 255u) << (8 * k4);
+      w2 |= ((uint32_t)(int)q2 & 255u) << (8 * k4);
+      w3 |= ((uint32_t)(int)q3 & 255u) << (8 * k4);
+    }
+    q32[j] = w1;
+    q32[n4 + j] = w2;
+    q32[2 * n4 + j] = w3;
   }
-  return part;
+  for (int g = tid; g < len / 32; g += 256) {
+    const float4 *x4 = reinterpret_cast<const float4 *>(src + 32 * g);
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 x = x4[i];
+      acc += (x.x + x.y) + (x.z + x.w);
+    }
+    sum[g] = acc;
+  }
+  if (tid == 0) {
+    a.hqs[4 * v] = s1;
+    a.hqs[4 * v + 1] = s2;
+    a.hqs[4 * v + 2] = s3;
+    a.hqs[4 * v + 3] = 0.f;
+  }
 }
 
 // y[t][r] = (x[t][r]) + shared_down[r] . hs[t] + sum_i w[t][i] down_e[r] . h[t,i],
 // the routed terms in the routing's ascending expert order; one warp per
-// output row, one dot product after the other.  (Measured slower at one
-// token: reading the k routed rows block by block together, 68 against 43 us
-// per launch; one block per output row with a warp per dot product, 48 us.)
+// output row, one dot product after the other, on the int8 limbs of h and hs
+// by dp4a.  (Measured slower at one token with fp32 h: reading the k routed
+// rows block by block together, 68 against 43 us per launch; one block per
+// output row with a warp per dot product, 48 us.)
 __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) {
   const LayerDims &d = a.d;
   const int lane = threadIdx.x & 31, r = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5), t = blockIdx.y;
   if (r >= d.H) return;
+  const int npairs = a.T * d.k, vs = npairs + t;
   const size_t rbs = (size_t)(d.Is / 32) * 34, rbd = (size_t)(d.I / 256) * 144;
-  const Q4kLane L(lane);
-  float acc = warp_sum(q80_part(a.sh_down + (size_t)r * rbs, a.hs + (size_t)t * d.Is, d.Is, lane));
+  const float ss[3] = {a.hqs[4 * vs], a.hqs[4 * vs + 1], a.hqs[4 * vs + 2]};
+  float acc = warp_sum(q80_row_part_limbs(a.sh_down + (size_t)r * rbs,
+                                          a.hq + (size_t)npairs * 3 * d.I + (size_t)t * 3 * d.Is, d.Is, ss, lane));
   for (int i = 0; i < d.k; ++i) {
     const int p = t * d.k + i, e = a.idx[p];
     if (e < 0 || e >= d.E) continue;
-    const float o = warp_sum(q4k_row_part(a.down + ((size_t)e * d.H + r) * rbd, a.h + (size_t)p * d.I, d.I, L, lane));
-    acc = fmaf(a.w[p], o, acc);
+    const uint8_t *const rows[1] = {a.down + ((size_t)e * d.H + r) * rbd};
+    const float sp[3] = {a.hqs[4 * p], a.hqs[4 * p + 1], a.hqs[4 * p + 2]};
+    float o[1] = {0.0f};
+    q4k_rows_part_limbs<1>(rows, a.hq + (size_t)p * 3 * d.I, d.I, sp, a.hsum + (size_t)p * (d.I / 32), lane, o);
+    acc = fmaf(a.w[p], warp_sum(o[0]), acc);
   }
   if (lane == 0) {
     const size_t at = (size_t)t * d.H + r;
@@ -333,8 +327,10 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_q4k_down(const Q4kArgs a) 
 
 size_t q4k_expert_bytes(const LayerDims &d, int T) {
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  const size_t nh = (size_t)T * d.k * d.I + (size_t)T * d.Is;  // down inputs: routed h, then shared hs
   return al(sizeof(float) * (size_t)T * d.k * d.I) + al(sizeof(float) * (size_t)T * d.Is) +
-         al(sizeof(float) * (size_t)T * (d.H / 32));
+         al(sizeof(float) * (size_t)T * (d.H / 32)) + al(3 * nh) + al(sizeof(float) * 4 * ((size_t)T * d.k + T)) +
+         al(sizeof(float) * (nh / 32));
 }
 
 cudaError_t q4k_experts(const Q4kArgs &a, cudaStream_t stream) {
@@ -343,6 +339,7 @@ cudaError_t q4k_experts(const Q4kArgs &a, cudaStream_t stream) {
   k_q4k_input<<<a.T, 256, 0, stream>>>(a.x, d.H, d.flags, d.eps, a.xsum);
   const int rmax = d.I > d.Is ? d.I : d.Is;
   k_q4k_gate_up<<<dim3((rmax + kRowsPerCta - 1) / kRowsPerCta, a.T * d.k + a.T), kRowsPerCta * 32, 0, stream>>>(a);
+  k_q4k_hlimbs<<<a.T * d.k + a.T, 256, 0, stream>>>(a);
   k_q4k_down<<<dim3((d.H + kRowsPerCta - 1) / kRowsPerCta, a.T), kRowsPerCta * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -24,14 +24,18 @@ struct Q4kArgs {
   float *xsum;         // [T][H/32] scratch: sums of the expert input over each 32-value sub-block
   const int8_t *xq;    // [T][3][H] int8 limbs of the expert input (the small-token router kernel's)
   const float *xs;     // [T][4] limb scales
+  int8_t *hq;          // scratch: int8 limbs of the down inputs, [T*k][3][I] (h) then [T][3][Is] (hs)
+  float *hqs;          // [T*k + T][4] their limb scales
+  float *hsum;         // their sums over each 32-value sub-block, [T*k][I/32] then [T][Is/32]
 };
 
-// Scratch the expert kernels take beside the routing scratch (h, hs, xsum).
+// Scratch the expert kernels take beside the routing scratch (h, hs, xsum and
+// the down inputs' limbs, scales and sums).
 size_t q4k_expert_bytes(const LayerDims &d, int T);
 
-// The expert work of one call, after the routing (idx, w) is in place:
-// three launches on `stream` (input, gate/up with SwiGLU, down with the
-// weighted combine).
+// The expert work of one call, after the routing (idx, w) is in place: four
+// launches on `stream` (input sums, gate/up with SwiGLU, the down inputs'
+// limbs, down with the weighted combine).
 cudaError_t q4k_experts(const Q4kArgs &a, cudaStream_t stream);
 
 }  // namespace moe

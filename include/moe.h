@@ -131,8 +131,17 @@ moe_status moe_workspace_size(const moe_config *cfg, int max_tokens, size_t *per
  * Validates the configuration and the weight pointers (non-null as the mode
  * requires, 16-byte aligned), records them in a host-side handle and
  * enqueues the initialisation of `persist` on `stream` (it checks the
- * codebook range into the device error word).  The weight buffers are read,
- * never written, and must stay valid and unchanged while the handle is used.
+ * codebook range into the device error word, computes the router rows'
+ * norms, and copies the tensor maps through which the batched path's
+ * tensor-memory-access unit reads the routed weight tiles).  The weight
+ * buffers are read, never written, and must stay valid and unchanged while
+ * the handle is used.
+ *
+ * Two environment variables, read here, select equivalent forms of the
+ * batched path (same results, for comparison and testing): MOE_GEMM_TMA set
+ * to "0" has its producer warps load the packed weight tiles themselves
+ * instead of through tensor copies; MOE_SHARED_DENSE set to "0" keeps the
+ * shared expert on per-tile Q8_0 decoding at every token count.
  *
  * Hash mode: every row of tid2eid must hold top_k distinct expert ids in
  * [0, n_experts) (the kernels index the expert weights with them and count
