@@ -63,7 +63,12 @@ constexpr int kATile = BM * BK * 2;  // 16 KB
 // tokens, so narrow tiles waste less), 256 for a single matrix and for the
 // shared expert's pair (all T tokens: wide tiles decode each weight tile
 // fewer times; that pair's one tile fills TMEM alone)
-__host__ __device__ constexpr int bn_of(int fmt, bool paired) { return paired && fmt != 2 ? 128 : 256; }
+#ifndef MOE_GEMM_BN_Q2K
+#define MOE_GEMM_BN_Q2K 256
+#endif
+__host__ __device__ constexpr int bn_of(int fmt, bool paired) {
+  return paired && fmt != 2 ? 128 : (!paired && fmt == 1 ? MOE_GEMM_BN_Q2K : 256);
+}
 __host__ __device__ constexpr int btile_of(int fmt, bool paired) { return bn_of(fmt, paired) * BK * 2; }
 __host__ __device__ constexpr int nacc_of(int fmt, bool paired) { return (paired ? 2 : 1) * bn_of(fmt, paired) <= 256 ? 2 : 1; }
 // stages of the dequantised A ring: how many K steps the producers may run
