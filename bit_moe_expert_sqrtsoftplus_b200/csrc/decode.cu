@@ -1283,9 +1283,6 @@ __global__ void __launch_bounds__(k2_threads(MAXP), 1) k2_experts(const __grid_c
   // Warps 0..T-1 route one token each and warp 0 builds the job table; the
   // other warps start on the shared expert's gate/up units, which need no
   // routing, and wait for the table only when they claim a routed unit.
-  // Warps 0..T-1 route one token each and warp 0 builds the job table; the
-  // other warps start on the shared expert's gate/up units, which need no
-  // routing, and wait for the table only when they claim a routed unit.
   // (Routing in every CTA beats one routing block followed by copies: the
   // copies would wait for that block's whole kernel to finish.)
   const int nr = T < nw ? T : nw;  // routing warps
