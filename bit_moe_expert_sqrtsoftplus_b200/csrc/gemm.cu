@@ -60,11 +60,13 @@ constexpr int BM = 128, BK = 64;
 constexpr int kATile = BM * BK * 2;  // 16 KB
 // token columns per tile: 128 for a routed gate/up pair (two accumulators
 // per tile, two tiles in flight fill the 512 TMEM columns; experts hold few
-// tokens, so narrow tiles waste less), 256 for a single matrix and for the
-// shared expert's pair (all T tokens: wide tiles decode each weight tile
-// fewer times; that pair's one tile fills TMEM alone)
+// tokens, so narrow tiles waste less) and for the routed Q2_K down matrix
+// (measured on B200 at 4096 tokens: the layer 5.08 ms against 5.28 ms with
+// 256-column tiles, whose producers each copy twice the token rows per K
+// step), 256 for the shared expert (all T tokens: wide tiles decode each
+// weight tile fewer times; its pair's one tile fills TMEM alone)
 #ifndef MOE_GEMM_BN_Q2K
-#define MOE_GEMM_BN_Q2K 256
+#define MOE_GEMM_BN_Q2K 128
 #endif
 __host__ __device__ constexpr int bn_of(int fmt, bool paired) {
   return paired && fmt != 2 ? 128 : (!paired && fmt == 1 ? MOE_GEMM_BN_Q2K : 256);
