@@ -780,8 +780,8 @@ SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 128, 256)
 def run_sweep(args, world, rank):
     """Latency and bandwidth of one layer call against the union of the
     experts its tokens select: V4-Flash shapes with the skewed bias, one
-    weight set, T = 1 ... 256 (the small-token path up to 32, the batched path
-    above).  Bytes per call = distinct experts x 7,077,888 + the shared expert
+    weight set, T = 1 ... 256 (the small-token path up to 32, twice up to 64,
+    the batched path above).  Bytes per call = distinct experts x 7,077,888 + the shared expert
     + the router, the least a call must read."""
     import torch
 
@@ -812,7 +812,8 @@ def run_sweep(args, world, rank):
         ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
         nbytes = nd * base.expert_bytes + base.shared_bytes + base.n_experts * base.hidden * 2
         gbs = nbytes / (ms / 1e3) / 1e9
-        lines.append({"sweep_T": T, "path": "small-token" if T <= moe.MOE_SMALL_T_MAX else "batched",
+        lines.append({"sweep_T": T, "path": "small-token" if T <= moe.MOE_SMALL_T_MAX else
+                      "small-token, two chunks" if T <= moe.MOE_CHUNKED_T_MAX else "batched",
                       "ms_per_call": ms, "tokens_per_s": job_throughput(world, 1, T, ms),
                       "distinct_experts": nd, "bytes_per_call": nbytes, "achieved_gbs": gbs,
                       "hbm_frac": gbs / peaks["hbm_gbs"], "floor_ms": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,

@@ -32,6 +32,7 @@ MOE_FLAG_EXPERTS_ONLY = 2
 MOE_FLAG_NO_ROUTED = 4
 MOE_FLAG_DETERMINISTIC = 8
 MOE_SMALL_T_MAX = 32  # calls with T <= this run the small-token kernels
+MOE_CHUNKED_T_MAX = 64  # q2 layers up to this T: the small-token kernels on 32 tokens, then the rest
 MOE_QUANT_Q8_0 = 0
 MOE_QUANT_Q2_K = 1
 MOE_QUANT_Q4_K = 2

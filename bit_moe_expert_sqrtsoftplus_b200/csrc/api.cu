@@ -19,6 +19,9 @@
 #include "quant.cuh"
 
 static_assert(MOE_SMALL_T_MAX == moe::kDecodeMaxT, "header and kernels disagree on the small-T limit");
+// q2 layers with up to this many tokens run the small-token kernels twice
+constexpr int kChunkedMaxT = MOE_CHUNKED_T_MAX;
+static_assert(kChunkedMaxT == 2 * moe::kDecodeMaxT, "two small-token chunks");
 
 constexpr int kGemmMaps = 3;  // tensor maps of gate, up and down for the batched path
 
@@ -424,6 +427,20 @@ moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_i
   } else if (T <= moe::kDecodeMaxT) {
     moe::DecodeArgs a = decode_args(h, x, token_ids, T, y, scratch);
     e = moe::decode_forward(a, s, h->num_sms);
+  } else if (T <= kChunkedMaxT && h->cfg.routed_format == MOE_ROUTED_Q2) {
+    // two small-token calls, the first 32 tokens and the rest, one after the
+    // other on the stream (a token's result depends on its own row only, so
+    // the split changes no bit of it): each chunk reads the union of its own
+    // tokens' experts, which up to 64 tokens costs less than the batched
+    // path's fixed work (measured on B200 at 64 tokens: 1.54 against 1.88 ms)
+    moe::DecodeArgs a0 = decode_args(h, x, token_ids, moe::kDecodeMaxT, y, scratch);
+    e = moe::decode_forward(a0, s, h->num_sms);
+    if (e == cudaSuccess) {
+      const size_t off = (size_t)moe::kDecodeMaxT * h->d.H;
+      moe::DecodeArgs a1 = decode_args(h, x + off, token_ids ? token_ids + moe::kDecodeMaxT : nullptr,
+                                       T - moe::kDecodeMaxT, y + off, scratch);
+      e = moe::decode_forward(a1, s, h->num_sms);
+    }
   } else {
     moe::PrefillArgs p = moe::prefill_args(h->d, h->wt, T, x, token_ids, y, scratch, h->row_norms, h->err);
     p.ev_begin = h->ev_begin;

@@ -80,6 +80,7 @@ typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_HASH = 1 } moe_route_mode;
 #define MOE_FLAG_NO_ROUTED 4    /* router (or table) and shared expert only: routed expert pointers may be NULL */
 
 #define MOE_SMALL_T_MAX 32 /* largest T served by the small-token kernels */
+#define MOE_CHUNKED_T_MAX 64 /* q2 layers: up to this T, the small-token kernels run on 32 tokens, then the rest */
 
 /* formats of the routed experts (moe_config.routed_format) */
 #define MOE_ROUTED_Q2 0  /* the q2 build: gate/up IQ2_XXS, down Q2_K */
@@ -173,9 +174,11 @@ moe_status moe_route(moe_handle *h, const float *x, const int32_t *token_ids, in
  * (overwritten; may alias x only with MOE_FLAG_PRENORM_RESIDUAL, where
  * y = x + MoE(RMSNorm(x))).  T = 0 is a no-op.  Calls with
  * T <= MOE_SMALL_T_MAX run the small-token path (two kernel launches: input
- * preparation and router, then routing and every expert unit); larger T the batched
- * tensor-core path (twelve launches in router mode: router, certificate,
- * fix-up, permutation, four grouped GEMMs).
+ * preparation and router, then routing and every expert unit); q2 layers with
+ * T <= MOE_CHUNKED_T_MAX run it twice, on the first MOE_SMALL_T_MAX tokens and
+ * then on the rest (the same results per token); larger T the batched
+ * tensor-core path (router, certificate, fix-up, permutation, the grouped
+ * GEMMs, and from 257 tokens the shared expert's expansion and dense GEMMs).
  */
 moe_status moe_ffn_forward(moe_handle *h, const float *x, const int32_t *token_ids, int T, float *y,
                            void *scratch, size_t scratch_bytes, moe_stream_t stream);

@@ -255,3 +255,27 @@ def test_route_and_permutation_bit_exact(moe, name, T):
     assert np.array_equal(off.cpu().numpy(), roff)
     assert np.array_equal(perm.cpu().numpy(), rperm)
     print(f"{name}: min margin {margin.min():.3e}, counts min/max {np.diff(roff).min()}/{np.diff(roff).max()}")
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 40), ("decode_t32", 64)])
+def test_chunked_small_token_calls(moe, name, T):
+    """From 33 to 64 tokens a q2 layer runs the small-token kernels on the
+    first 32 tokens and then on the rest: the output equals, bit for bit, the
+    two calls made separately, and matches the oracle at the small-token
+    tolerance (every row)."""
+    s = synth.workload(name, tokens=T)
+    W = harness.device_layer(s, 4, 3)
+    L = moe.Layer(harness.config_for(s), W, max_tokens=T)
+    x_np = synth.activations(4, T, s.hidden, stream=3)
+    x = torch.from_numpy(x_np).cuda()
+    y = L.forward(x).cpu().numpy()
+    y0 = L.forward(x[:32].contiguous()).cpu().numpy()
+    y1 = L.forward(x[32:].contiguous()).cpu().numpy()
+    L.poll()
+    assert np.array_equal(y.view(np.uint32), np.concatenate([y0, y1]).view(np.uint32))
+    _, _, yref, _ = harness.oracle_layer_dense(s, 4, 3, x_np)
+    rel, mx = harness.errors(y, yref)
+    assert rel <= harness.GEMV_REL_L2 and mx <= harness.MAX_ABS_FRAC, (rel, mx)
+    for t in range(T):
+        r, _ = harness.errors(y[t], yref[t])
+        assert r <= harness.GEMV_REL_L2, (t, r)
