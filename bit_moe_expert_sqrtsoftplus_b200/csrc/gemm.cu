@@ -117,7 +117,8 @@ __host__ __device__ constexpr int sp_of(bool paired) { return paired ? 2 : MOE_G
 // 2.47 ms with TMA staging against 2.86 ms without; the Q2_K down GEMM 2.30
 // ms against 2.08 ms (its 16-value items leave little decode to hide the
 // staged reads behind, and the 96-byte staged rows put two of every eight
-// rows of a warp on the same banks), whatever the depth of the rings.
+// rows of a warp on the same banks), whatever the depth of the rings; with
+// 128-column down tiles the layer took 5.18 ms with staging against 5.09.
 #ifndef MOE_GEMM_TMA_Q2K
 #define MOE_GEMM_TMA_Q2K 0
 #endif
