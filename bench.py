@@ -329,29 +329,34 @@ def run_ours(args, world, rank):
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def pipelined(n):
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+            for i in range(n):
+                j, b2 = i % npool, i % 2
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_done[b2])  # step i-2 has read dxs[b2]
+                    dxs[b2].copy_(hx[j], non_blocking=True)
+                    ev_in[b2].record(s_in)
+                stream.wait_event(ev_in[b2])
+                if i >= 2:
+                    stream.wait_event(ev_out[b2])  # step i-2's output has left dys[b2]
+                layers[i % nsets].forward(dxs[b2], None, dys[b2])
+                ev_done[b2].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[b2])
+                    hy[j].copy_(dys[b2], non_blocking=True)
+                    ev_out[b2].record(s_out)
+            stream.wait_stream(s_out)
+
+        pipelined(max(3, args.warmup))  # untimed: the copy streams' first use
         torch.cuda.synchronize()
         barrier(world)
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         g0.record(stream)
-        s_in.wait_stream(stream)
-        s_out.wait_stream(stream)
-        for i in range(args.steps):
-            j, b2 = i % npool, i % 2
-            with torch.cuda.stream(s_in):
-                if i >= 2:
-                    s_in.wait_event(ev_done[b2])  # step i-2 has read dxs[b2]
-                dxs[b2].copy_(hx[j], non_blocking=True)
-                ev_in[b2].record(s_in)
-            stream.wait_event(ev_in[b2])
-            if i >= 2:
-                stream.wait_event(ev_out[b2])  # step i-2's output has left dys[b2]
-            layers[i % nsets].forward(dxs[b2], None, dys[b2])
-            ev_done[b2].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_done[b2])
-                hy[j].copy_(dys[b2], non_blocking=True)
-                ev_out[b2].record(s_out)
-        stream.wait_stream(s_out)
+        pipelined(args.steps)
         g1.record(stream)
         barrier(world)
         e2e_ms = g0.elapsed_time(g1)
