@@ -85,22 +85,32 @@ __global__ void k_token_norms(const float *x, int T, int H, int flags, float eps
 // loads (x scaled by the token's fp32 inverse RMS, W_r converted from f16),
 // transposed into K-major shared tiles; the next chunk's loads are in flight
 // while the current one is multiplied.
-constexpr int RT = 64, RE = 64, RK = 32;
+constexpr int RE = 64, RK = 32;
+// Router GEMM tiles: 128 tokens per block (8 per thread: 32 accumulators, one
+// block per SM) once there are enough tokens to give every SM a block at E =
+// 256, 64 below.
+#ifndef MOE_ROUTER_WIDE_MIN_T
+#define MOE_ROUTER_WIDE_MIN_T 2048
+#endif
+template <int RTT>
 __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double *inv, const uint16_t *Wr, int T,
                                                     int E, int H, double *z) {
-  __shared__ __align__(16) float xs[RK][RT + 4];
+  // RTT tokens x RE experts per block; thread (tx, ty) owns tokens ty*TPT ..
+  // and experts tx*4 ..
+  constexpr int TPT = RTT / 16, XP = RTT / 32;
+  __shared__ __align__(16) float xs[RK][RTT + 4];
   __shared__ __align__(16) float ws[RK][RE + 4];
-  const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE;
+  const int t0 = blockIdx.x * RTT, e0 = blockIdx.y * RE;
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;  // experts tx*4 .., tokens ty*4 ..
-  // staging roles: x float4 pieces (token i>>3, K quad i&7) for i = tid and
-  // tid + 256, and one W uint4 piece (expert tid>>2, K octet tid&3); the
-  // pieces of chunk k0 + RK are loaded into registers while chunk k0 is
+  const int tx = tid & 15, ty = tid >> 4;
+  // staging roles: x float4 pieces (token i>>3, K quad i&7) for i = tid,
+  // tid + 256, ..., and one W uint4 piece (expert tid>>2, K octet tid&3);
+  // the pieces of chunk k0 + RK are loaded into registers while chunk k0 is
   // multiplied
-  float invf[2];
-  const float *xrow[2];
+  float invf[XP];
+  const float *xrow[XP];
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int r = 0; r < XP; ++r) {
     const int i = tid + 256 * r;
     const int t = t0 + (i >> 3);
     invf[r] = t < T ? (float)inv[t] : 0.f;
@@ -108,23 +118,23 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
   }
   const int we = e0 + (tid >> 2);
   const uint16_t *wrow = we < E ? Wr + (size_t)we * H + 8 * (tid & 3) : nullptr;
-  float4 xv_next[2];
+  float4 xv_next[XP];
   uint4 wv_next;
   auto fetch = [&](int k0) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < XP; ++r)
       xv_next[r] = xrow[r] ? *reinterpret_cast<const float4 *>(xrow[r] + k0) : make_float4(0.f, 0.f, 0.f, 0.f);
     wv_next = wrow ? *reinterpret_cast<const uint4 *>(wrow + k0) : make_uint4(0u, 0u, 0u, 0u);
   };
-  double acc[4][4];
+  double acc[TPT][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < TPT; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
   fetch(0);
   for (int k0 = 0; k0 < H; k0 += RK) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < XP; ++r) {
       const int i = tid + 256 * r;
       const int tt = i >> 3, kq = i & 7;
       const float4 v = xv_next[r];
@@ -144,31 +154,40 @@ __global__ void __launch_bounds__(256) k_router_f32(const float *x, const double
     }
     __syncthreads();
     if (k0 + RK < H) fetch(k0 + RK);
-    float part[4][4];
+    // each logit: a 32-term fp32 FMA chain from zero in K order, then added
+    // into its fp64 accumulator (the same arithmetic whatever the tile)
+    float part[TPT][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < TPT; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
 #pragma unroll 8
     for (int kk = 0; kk < RK; ++kk) {
-      const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
+      float xa[TPT];
+#pragma unroll
+      for (int q = 0; q < TPT / 4; ++q) {
+        const float4 xv = *reinterpret_cast<const float4 *>(&xs[kk][ty * TPT + 4 * q]);
+        xa[4 * q] = xv.x;
+        xa[4 * q + 1] = xv.y;
+        xa[4 * q + 2] = xv.z;
+        xa[4 * q + 3] = xv.w;
+      }
       const float4 wv = *reinterpret_cast<const float4 *>(&ws[kk][tx * 4]);
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
       const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < TPT; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < TPT; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] += (double)part[i][j];
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
+  for (int i = 0; i < TPT; ++i) {
+    const int t = t0 + ty * TPT + i;
     if (t >= T) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -642,8 +661,13 @@ cudaError_t prefill_route(const PrefillArgs &p, int32_t *idx, float *w, cudaStre
   cudaError_t e = cudaMemsetAsync(p.s.fix, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return e;
   k_token_norms<<<T, 256, 0, s>>>(p.x, T, d.H, d.flags, d.eps, inv, xn);
-  dim3 g((T + RT - 1) / RT, (d.E + RE - 1) / RE);
-  k_router_f32<<<g, 256, 0, s>>>(p.x, inv, p.wt.Wr, T, d.E, d.H, z);
+  if (T >= MOE_ROUTER_WIDE_MIN_T) {
+    const dim3 g((T + 127) / 128, (d.E + RE - 1) / RE);
+    k_router_f32<128><<<g, 256, 0, s>>>(p.x, inv, p.wt.Wr, T, d.E, d.H, z);
+  } else {
+    const dim3 g((T + 63) / 64, (d.E + RE - 1) / RE);
+    k_router_f32<64><<<g, 256, 0, s>>>(p.x, inv, p.wt.Wr, T, d.E, d.H, z);
+  }
   k_topk_cert<<<(T + 7) / 8, 256, 0, s>>>(z, p.wt.bias, p.row_norms, xn, T, d.E, d.k, d.scaling, idx, w, p.s.fix);
   // enough blocks for the usual handful of queued tokens; more stride
   const int nfix_items = T * ((d.E + kFixGroup - 1) / kFixGroup);

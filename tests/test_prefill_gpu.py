@@ -44,7 +44,8 @@ def _oracle_rows(s, seed, layer, x_np, tok_np, rows, router=True, prenorm=False)
     return yref
 
 
-@pytest.mark.parametrize("T", [9, 64, 300])
+# 2100 tokens: the router GEMM's 128-token tiles with a ragged last tile
+@pytest.mark.parametrize("T", [9, 64, 300, 2100])
 def test_tiny_shapes_large_T(moe, T):
     s = synth.workload("tiny", tokens=T)
     x, tok, y, _ = _forward(moe, s, 0, 0, T)
