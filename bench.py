@@ -78,6 +78,71 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e, nominal
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, nominal
+
+
+def box_peaks() -> dict:
+    """This box's own achievable peaks, measured after the workloads: a
+    device-to-device copy of 2 GiB (bytes read + written per second, best of
+    10 timed copies after 3 warm-up copies) and a cuBLAS bf16 GEMM of
+    8192 x 8192 x 8192 (best of 10 after 3).  Reported beside the roofline,
+    whose peak stays the pool's figure."""
+    import torch
+
+    out = {"copy": "torch copy_ of 2 GiB on the device, best of 10",
+           "gemm": "torch.matmul bf16 8192^3 (cuBLAS), best of 10"}
+    try:
+        torch.cuda.empty_cache()
+        a = torch.empty(1 << 31, dtype=torch.uint8, device="cuda")
+        b = torch.empty_like(a)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        best = float("inf")
+        for i in range(13):
+            ev[0].record()
+            b.copy_(a)
+            ev[1].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                best = min(best, ev[0].elapsed_time(ev[1]))
+        out["copy_gbs"] = 2 * a.numel() / (best / 1e3) / 1e9
+        del a, b
+        n = 8192
+        x = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+        y = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+        best = float("inf")
+        for i in range(13):
+            ev[0].record()
+            torch.matmul(x, y)
+            ev[1].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                best = min(best, ev[0].elapsed_time(ev[1]))
+        out["bf16_tflops"] = 2 * n ** 3 / (best / 1e3) / 1e12
+        del x, y
+        torch.cuda.empty_cache()
+    except Exception as ex:  # a failed measurement leaves the line as it is
+        out["error"] = str(ex)[:200]
+    return out
+
+
+def add_box_fracs(line: dict, bp: dict) -> None:
+    """The roofline's achieved figure also as fractions of this box's
+    measured peak and of the nominal one."""
+    r = line.get("roofline")
+    if not r or "achieved" not in r:
+        return
+    if r.get("unit") == "GB/s":
+        box, nominal = bp.get("copy_gbs"), NOMINAL_HBM_GBS
+    elif r.get("unit") == "TFLOP/s":
+        box, nominal = bp.get("bf16_tflops"), NOMINAL_BF16_TFLOPS
+    else:
+        return
+    if box:
+        r["frac_of_box_peak"] = r["achieved"] / box
+    r["frac_of_nominal"] = r["achieved"] / nominal
+
+
 def load_traffic(workload: str):
     """DRAM bytes per launch of the workload's dominant kernel from the ncu
     capture recorded in profiles/traffic.txt, or None when the kernel's
@@ -908,6 +973,11 @@ def main():
         out["workloads"] = extras
         out["sweep"] = sweep
         out["gpu_launches_all_workloads"] = out["gpu_launches"] + sum(r["gpu_launches"] for r in extras.values())
+    bp = box_peaks()
+    out["box_peaks"] = bp
+    add_box_fracs(out, bp)
+    for r in out.get("workloads", {}).values():
+        add_box_fracs(r, bp)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

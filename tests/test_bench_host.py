@@ -42,3 +42,18 @@ def test_decode_bytes_follow_the_routed_format():
     assert b["k2_experts"] == 69_206_016  # six q2 experts and the shared expert (page figures)
     s4 = synth.workload("decode_t1_q4k")
     assert bench.decode_bytes(s4, 6.0)["experts"] == 6 * 3 * 4096 * 2048 * 144 // 256 + 26_738_688
+
+
+def test_box_fractions():
+    """The box-measured and nominal fractions divide the roofline's achieved
+    figure by the peak of its own unit, and leave the pool's frac alone."""
+    line = {"roofline": {"achieved": 1600.0, "unit": "GB/s", "frac": 0.24}}
+    bench.add_box_fracs(line, {"copy_gbs": 6400.0, "bf16_tflops": 1500.0})
+    r = line["roofline"]
+    assert r["frac_of_box_peak"] == pytest.approx(0.25)
+    assert r["frac_of_nominal"] == pytest.approx(0.2)
+    assert r["frac"] == 0.24
+    line = {"roofline": {"achieved": 450.0, "unit": "TFLOP/s"}}
+    bench.add_box_fracs(line, {"error": "no GPU"})
+    assert "frac_of_box_peak" not in line["roofline"]
+    assert line["roofline"]["frac_of_nominal"] == pytest.approx(0.2)
